@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Throughput of the fused edge-conditioned tensor-product convolution on B200.
+
+One step = one pass of the hot path over the NequIP-like workload (1,536 atoms, 46,080
+directed edges, 32x(0e,1o,2e) -> 32x(0e,1e,1o,2e,2o), SH lmax 2, uvu, all 15 paths):
+forward (tp_conv_fwd), the stable sender transpose (tp_csr_transpose) and backward with
+gradients for node features and edge weights (tp_conv_bwd), all through the C ABI.
+Inputs are resident in HBM; R seeded copies rotate so that one step's inputs are never
+left in L2 by the previous steps (R x input bytes > 2 x L2).
+
+Prints one JSON line (rank 0).  `--impl reference` times the float64 CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes as C
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "edges/sec for fused TP conv fwd/fwd+bwd on 1 B200; % of HBM/FLOP roofline"
+WORKLOADS = {
+    "c2": "NequIP-like: 1,536 atoms, 46,080 directed edges, 32x0e+32x1o+32x2e -> "
+          "32x0e+32x1e+32x1o+32x2e+32x2o, SH lmax 2, uvu, 15 paths; step = fwd + transpose + bwd(gx, gw)",
+    "c3": "SevenNet/MACE-like l=3: 4,096 atoms, ~163k edges, 64x(0e,1o,2e,3o), SH lmax 3, uvu, 34 paths; "
+          "step = fwd + transpose + bwd(gx, gw)",
+    "c5": "skewed degree 3-120: 8,192 atoms, ~295k edges, 32x(0e,1o,2e,3o), SH lmax 3, uvu, 34 paths; "
+          "step = fwd + transpose + bwd(gx, gw, gvec)",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="c2", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ------------------------------------------------------------------------------------------
+# Algorithmic counts (bytes a perfect kernel must move; stated in the design notes)
+# ------------------------------------------------------------------------------------------
+
+def fwd_bytes(N, E, in_dim, out_dim, nw):
+    return E * (4 + 12 + 4 * nw) + 4 * N * (in_dim + out_dim) + 4 * (N + 1)
+
+
+def bwd_bytes(N, E, in_dim, out_dim, nw, gvec):
+    # perm + vec + w read + gw write (+ gvec write); x read, gy read, gx write; colptr + rowptr
+    return E * (4 + 12 + 8 * nw + (12 if gvec else 0)) + 4 * N * (2 * in_dim + out_dim) + 8 * (N + 1)
+
+
+# ------------------------------------------------------------------------------------------
+# Clocks (NVML reads only; nothing is changed)
+# ------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    def __init__(self, index: int, period=0.05):
+        self.samples, self.reasons = [], set()
+        self.period = period
+        self.ok = False
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = nv.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as exc:  # noqa: BLE001
+            self.err = str(exc)
+        self._stop = threading.Event()
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:  # noqa: BLE001
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        names = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+                 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+        for bit, n in names.items():
+            if r & bit:
+                self.reasons.add(n)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------
+# CPU side: the float64 oracle on a bounded sample
+# ------------------------------------------------------------------------------------------
+
+def oracle_sample(d, n_rows, seed):
+    """fwd on the edges into n_rows receivers, bwd on the edges leaving n_rows senders."""
+    from oracle import OraclePlan, backward, forward
+    spec = d["spec"]
+    op = OraclePlan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, spec.mode)
+    N = len(d["rowptr"]) - 1
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(N, size=min(n_rows, N), replace=False))
+    rp = np.asarray(d["rowptr"], dtype=np.int64)
+    eids = np.concatenate([np.arange(rp[i], rp[i + 1]) for i in rows])
+    rpf = np.concatenate([[0], np.cumsum(rp[rows + 1] - rp[rows])])
+    mask = np.isin(d["src"], rows)
+    eb = np.nonzero(mask)[0]
+    rpb = np.concatenate([[0], np.cumsum(np.bincount(d["dst"][eb], minlength=N))])
+    t0 = time.perf_counter()
+    forward(op, rpf, d["src"][eids], d["x"], d["vec"][eids], w=d["w"][eids])
+    t1 = time.perf_counter()
+    backward(op, rpb, d["src"][eb], d["x"], d["vec"][eb], d["gy"], w=d["w"][eb])
+    t2 = time.perf_counter()
+    return len(eids), t1 - t0, len(eb), t2 - t1
+
+
+def cpu_edges_per_s(ef, tf, eb, tb):
+    return 1.0 / (tf / ef + tb / eb)
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    import synth
+    from oracle.conv import set_threads
+    cores = set_threads()
+    d = synth.make_inputs(args.workload)
+    oracle_sample(d, 4, seed=0)                      # CG tables cached outside the timing
+    ef, tf, eb, tb = oracle_sample(d, 16, seed=1)
+    per_row = (tf + tb) / 16
+    # size each step so the whole run stays near a minute of host time
+    rows_per_step = int(max(2, min(256, 60.0 / max(1, args.steps + args.warmup) / per_row)))
+    for k in range(args.warmup):
+        oracle_sample(d, rows_per_step, seed=k)
+    tot_e, tot_t = 0.0, 0.0
+    per = []
+    for k in range(args.steps):
+        ef, tf, eb, tb = oracle_sample(d, rows_per_step, seed=1000 + k)
+        per.append(cpu_edges_per_s(ef, tf, eb, tb))
+        tot_t += tf + tb
+        tot_e += 1.0 / (tf / ef + tb / eb) * (tf + tb)
+    value = tot_e / tot_t
+    sample = (f"{rows_per_step} random receivers (fwd on their incoming edges) and {rows_per_step} random "
+              f"senders (bwd on their outgoing edges) per step, float64")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload], "name": args.workload},
+            "cpu_baseline": {"value": value, "unit": "edges/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------
+# GPU side
+# ------------------------------------------------------------------------------------------
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("tp_kernels.cuh", "tp_common.h", "csr.cu", "codegen.py"):
+        with open(os.path.join(ROOT, "equivariant_tensor_product_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if the kernels are unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        rec = json.load(open(path))
+        e = rec.get(workload, {}).get(kernel)
+        if e and e.get("source_hash") == kernel_source_hash():
+            return e["dram_bytes_per_launch"]
+    except Exception:  # noqa: BLE001
+        return None
+    return None
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return p.get("hbm_gbs", 6650.0), p.get("bf16_tflops", 1590.0), "of measured"
+    return 6650.0, 1590.0, "of fallback"
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from equivariant_tensor_product_b200 import build as tpbuild
+    tpbuild.build()
+    import equivariant_tensor_product_b200 as tp
+    import synth
+    lib = tp.load()
+
+    spec = synth.CONFIGS[args.workload]
+    d = synth.make_inputs(args.workload, seed=spec.seed + 7919 * rank)
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, spec.mode)
+    N, E = len(d["rowptr"]) - 1, len(d["src"])
+    in_dim, out_dim, nw = plan.in_dim, plan.out_dim, plan.n_edge_weights
+    want_gvec = "dbwd" in spec.passes or args.workload == "c5"
+
+    keys = ["rowptr", "src", "x", "vec", "w", "gy"]
+    copy_bytes = sum(d[k].nbytes for k in keys)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(2, math.ceil(2.5 * l2 / copy_bytes))
+    copies = []
+    for r in range(R):
+        if r == 0:
+            src_d = d
+        else:
+            rng = np.random.default_rng(spec.seed + 31 * r + 7919 * rank)
+            src_d = dict(d)
+            src_d["x"] = rng.standard_normal(d["x"].shape, dtype=np.float32)
+            src_d["gy"] = rng.standard_normal(d["gy"].shape, dtype=np.float32)
+            src_d["w"] = (d["w"] * rng.uniform(0.5, 1.5, size=(1, d["w"].shape[1]))).astype(np.float32)
+        copies.append({k: torch.as_tensor(np.ascontiguousarray(src_d[k])).to(dev) for k in keys})
+    y = torch.empty(N, out_dim, device=dev)
+    gx = torch.empty(N, in_dim, device=dev)
+    gw = torch.empty(E, nw, device=dev)
+    gvec = torch.empty(E, 3, device=dev) if want_gvec else None
+    colptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(E, dtype=torch.int32, device=dev)
+    ws_bytes = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    h = plan.handle
+    P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None
+
+    argsets = []
+    for cp in copies:
+        argsets.append((
+            (h, N, E, P(cp["rowptr"]), P(cp["src"]), P(cp["x"]), P(cp["vec"]), P(cp["w"]), None, P(y), None, 0, sh),
+            (N, E, P(cp["rowptr"]), P(cp["src"]), P(colptr), P(perm), P(ws), ws_bytes, sh),
+            (h, N, E, P(cp["rowptr"]), P(cp["src"]), P(colptr), P(perm), P(cp["x"]), P(cp["vec"]), P(cp["w"]),
+             None, P(cp["gy"]), P(gx), P(gw), P(gvec), None, P(ws), ws_bytes, sh),
+        ))
+    fwd_f, tr_f, bwd_f = lib.tp_conv_fwd, lib.tp_csr_transpose, lib.tp_conv_bwd
+
+    def step(k, ev=None):
+        a_f, a_t, a_b = argsets[k % R]
+        if ev is not None:
+            ev[0].record(stream)
+        st = fwd_f(*a_f)
+        if ev is not None:
+            ev[1].record(stream)
+        st |= tr_f(*a_t)
+        if ev is not None:
+            ev[2].record(stream)
+        st |= bwd_f(*a_b)
+        if ev is not None:
+            ev[3].record(stream)
+        if st:
+            raise RuntimeError(lib.tp_last_error_message().decode())
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    n0 = lib.tp_launch_count()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            step(k, evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    launches = lib.tp_launch_count() - n0
+    if world > 1:
+        dist.barrier()
+    elapsed = start.elapsed_time(stop) / 1e3
+    t = torch.tensor([elapsed], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_max = float(t.item())
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    tr_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    # end to end through the same calls, inputs from pinned host memory, outputs back to host
+    host_in = {k: torch.as_tensor(np.ascontiguousarray(d[k])).pin_memory() for k in keys}
+    dev_in = {k: torch.empty_like(host_in[k], device=dev) for k in keys}
+    host_out = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in (y, gx, gw)]
+    e2e_args = (
+        (h, N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(dev_in["x"]), P(dev_in["vec"]), P(dev_in["w"]), None,
+         P(y), None, 0, sh),
+        (N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(ws), ws_bytes, sh),
+        (h, N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(dev_in["x"]), P(dev_in["vec"]),
+         P(dev_in["w"]), None, P(dev_in["gy"]), P(gx), P(gw), P(gvec), None, P(ws), ws_bytes, sh))
+
+    def e2e_step():
+        for k in keys:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        st = fwd_f(*e2e_args[0]) | tr_f(*e2e_args[1]) | bwd_f(*e2e_args[2])
+        if st:
+            raise RuntimeError(lib.tp_last_error_message().decode())
+        for ho, dv in zip(host_out, (y, gx, gw)):
+            ho.copy_(dv, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = e0.elapsed_time(e1) / 1e3
+    te = torch.tensor([e2e_s], device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * args.e2e_steps * E / float(te.item())
+    h2d = sum(host_in[k].numel() * host_in[k].element_size() for k in keys)
+    d2h = sum(t_.numel() * t_.element_size() for t_ in host_out)
+
+    if rank == 0:
+        hbm, _, peak_note = measured_peaks()
+        fb = fwd_bytes(N, E, in_dim, out_dim, nw)
+        bb = bwd_bytes(N, E, in_dim, out_dim, nw, want_gvec)
+        if bwd_ms >= fwd_ms:
+            kname, kbytes, kms = "k_bwd_uvu", bb, bwd_ms
+        else:
+            kname, kbytes, kms = "k_fwd_uvu", fb, fwd_ms
+        achieved = kbytes / (kms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "peak_note": peak_note,
+                "traffic": traffic_from_profile(kname, args.workload),
+                "algorithmic_bytes_per_launch": kbytes,
+                "kernel_ms": {"fwd": fwd_ms, "transpose": tr_ms, "bwd": bwd_ms},
+                "step_roofline_frac": ((fb + bb) / (hbm * 1e9)) / (elapsed / args.steps)}
+        cpu = None
+        if not args.no_cpu_baseline and world >= 1:
+            from oracle.conv import set_threads
+            cores = set_threads()
+            oracle_sample(d, 4, seed=0)              # CG tables cached outside the timing
+            n_rows = min(N, 1536)
+            ef, tf, eb, tb = oracle_sample(d, n_rows, seed=3)
+            cpu = {"value": cpu_edges_per_s(ef, tf, eb, tb), "unit": "edges/s", "cores": cores, "kind": "oracle",
+                   "sample": f"fwd on the {ef} edges into {n_rows} receivers + bwd on the {eb} edges leaving "
+                             f"{n_rows} senders of the same workload (rank 0's copy), float64 torch CPU, "
+                             f"{tf + tb:.1f} s"}
+        value = world * args.steps * E / elapsed_max
+        line = {
+            "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * elapsed_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload], "name": args.workload, "N": N, "E": E,
+                       "l2": f"{R} rotating input copies of {copy_bytes / 1e6:.1f} MB (> 2x L2 of "
+                             f"{l2 / 1e6:.0f} MB)", "parallelism": "replicas" if world > 1 else "single"},
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "edges/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": args.e2e_steps},
+            "gpu_launches": int(launches), "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    return run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

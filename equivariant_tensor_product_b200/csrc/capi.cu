@@ -1,0 +1,508 @@
+// C ABI of the tensor-product convolution: plans, argument checks, workspace layout and
+// dispatch to the compiled specialisations.  See include/tp.h for the contract.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/tp.h"
+#include "tp_common.h"
+
+using namespace tp;
+
+struct IrrepBlock {
+  int mul, l, parity;
+};
+
+struct tp_plan_s {
+  const SpecOps* ops;
+  int mode;
+  int mul_in, mul_out;
+  int64_t in_dim, out_dim, nw, n_shared;
+  int n_paths;
+  int has_coeff;
+  float coeff[kMaxPaths];
+  uint32_t flags;
+};
+
+#include <atomic>
+namespace tp {
+static std::atomic<long long> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace tp
+
+namespace {
+
+thread_local std::string g_msg;
+
+tp_status_t fail(tp_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_msg = buf;
+  return st;
+}
+
+tp_status_t cuda_fail(cudaError_t e, const char* where) {
+  return fail(TP_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool parse_irreps(const char* s, std::vector<IrrepBlock>& out, std::string& why) {
+  out.clear();
+  if (!s) {
+    why = "null irreps string";
+    return false;
+  }
+  std::string str;
+  for (const char* p = s; *p; ++p)
+    if (*p != ' ') str.push_back(*p);
+  if (str.empty()) {
+    why = "empty irreps string";
+    return false;
+  }
+  size_t pos = 0;
+  while (pos <= str.size()) {
+    size_t end = str.find('+', pos);
+    if (end == std::string::npos) end = str.size();
+    std::string term = str.substr(pos, end - pos);
+    size_t x = term.find('x');
+    if (x == std::string::npos || x == 0 || x + 2 > term.size()) {
+      why = "bad irreps term '" + term + "'";
+      return false;
+    }
+    const std::string mul_s = term.substr(0, x), l_s = term.substr(x + 1, term.size() - x - 2);
+    const char par = term.back();
+    if (l_s.empty() || (par != 'e' && par != 'o') || mul_s.size() > 7 || l_s.size() > 3) {
+      why = "bad irreps term '" + term + "'";
+      return false;
+    }
+    for (char ch : mul_s + l_s)
+      if (ch < '0' || ch > '9') {
+        why = "bad irreps term '" + term + "'";
+        return false;
+      }
+    IrrepBlock b{std::atoi(mul_s.c_str()), std::atoi(l_s.c_str()), par == 'e' ? 1 : -1};
+    if (b.mul <= 0) {
+      why = "multiplicity must be positive";
+      return false;
+    }
+    out.push_back(b);
+    if (end == str.size()) break;
+    pos = end + 1;
+    if (pos == str.size()) {
+      why = "trailing '+'";
+      return false;
+    }
+  }
+  return true;
+}
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t header, colptr, counts, perm, tmp, total;
+};
+
+// header (error word) | colptr[N+1] | counts[N] | perm[E] | tmp[E]
+WsLayout ws_layout(int64_t N, int64_t E) {
+  WsLayout L{};
+  size_t off = 0;
+  L.header = off;
+  off += 256;
+  L.colptr = off;
+  off += align256(sizeof(int32_t) * (size_t)(N + 1));
+  L.counts = off;
+  off += align256(sizeof(int32_t) * (size_t)(N > 0 ? N : 1));
+  L.perm = off;
+  off += align256(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+  L.tmp = off;
+  off += align256(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+  L.total = off;
+  return L;
+}
+
+int pick_split(int64_t N, int64_t E) {
+  if (N <= 0) return 1;
+  const double avg = (double)E / (double)N;
+  if (avg >= 24.0) return 4;
+  if (avg >= 8.0) return 2;
+  return 1;
+}
+
+tp_status_t check_sizes(tp_plan_t plan, int64_t N, int64_t E) {
+  if (!plan) return fail(TP_ERR_INVALID_ARG, "plan is NULL");
+  if (N < 0 || E < 0) return fail(TP_ERR_INVALID_ARG, "N and E must be non-negative");
+  if (N >= (int64_t)1 << 31 || E >= (int64_t)1 << 31)
+    return fail(TP_ERR_UNSUPPORTED, "N and E must be below 2^31 (int32 indices)");
+  const int64_t slices = (plan->mul_in + 31) / 32;
+  if (N * slices >= (int64_t)1 << 31) return fail(TP_ERR_UNSUPPORTED, "N * channel slices must be below 2^31");
+  return TP_OK;
+}
+
+LaunchArgs base_args(tp_plan_t plan, int64_t N, int64_t E) {
+  LaunchArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.N = (int)N;
+  a.E = (int)E;
+  a.mul = plan->mul_in;
+  a.mul_out = plan->mul_out;
+  a.in_dim = (int)plan->in_dim;
+  a.out_dim = (int)plan->out_dim;
+  a.nw = (int)plan->nw;
+  a.split = pick_split(N, E);
+  a.n_slices = (plan->mul_in + 31) / 32;
+  a.has_coeff = plan->has_coeff;
+  a.check = (plan->flags & TP_FLAG_CHECK_INDICES) ? 1 : 0;
+  std::memcpy(a.coeff, plan->coeff, sizeof(a.coeff));
+  return a;
+}
+
+// Validates the CSR on the device (debug flag only) and resets the error word.
+tp_status_t debug_prologue(tp_plan_t plan, int64_t N, int64_t E, const int32_t* rowptr,
+                           const int32_t* src, void* ws, cudaStream_t s, int** err) {
+  *err = nullptr;
+  if (!(plan->flags & TP_FLAG_CHECK_INDICES)) return TP_OK;
+  if (!ws) return fail(TP_ERR_WORKSPACE, "TP_FLAG_CHECK_INDICES needs a workspace for the error word");
+  int* e = reinterpret_cast<int*>(ws);
+  cudaError_t st = cudaMemsetAsync(e, 0, sizeof(int), s);
+  if (st != cudaSuccess) return cuda_fail(st, "cudaMemsetAsync(error word)");
+  st = launch_csr_validate((int)N, (int)E, rowptr, src, e, s);
+  if (st != cudaSuccess) return cuda_fail(st, "csr_validate");
+  *err = e;
+  return TP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tp_version(void) { return "tp-b200 0.1 (sm_100a)"; }
+
+int64_t tp_launch_count(void) { return tp::g_launches.load(std::memory_order_relaxed); }
+
+const char* tp_status_string(tp_status_t s) {
+  switch (s) {
+    case TP_OK: return "ok";
+    case TP_ERR_INVALID_ARG: return "invalid argument";
+    case TP_ERR_UNSUPPORTED: return "unsupported";
+    case TP_ERR_BAD_GRAPH: return "bad graph";
+    case TP_ERR_WORKSPACE: return "workspace too small";
+    case TP_ERR_CUDA: return "CUDA error";
+    case TP_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* tp_last_error_message(void) { return g_msg.c_str(); }
+
+tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* irreps_sh,
+                           const char* irreps_out, const int32_t* paths, int32_t n_paths, int32_t mode,
+                           const double* path_coeff, uint32_t flags) {
+  if (!plan) return fail(TP_ERR_INVALID_ARG, "plan out-pointer is NULL");
+  *plan = nullptr;
+  std::vector<IrrepBlock> bi, bs, bo;
+  std::string why;
+  if (!parse_irreps(irreps_in, bi, why)) return fail(TP_ERR_INVALID_ARG, "irreps_in: %s", why.c_str());
+  if (!parse_irreps(irreps_sh, bs, why)) return fail(TP_ERR_INVALID_ARG, "irreps_sh: %s", why.c_str());
+  if (!parse_irreps(irreps_out, bo, why)) return fail(TP_ERR_INVALID_ARG, "irreps_out: %s", why.c_str());
+  if (mode != TP_MODE_UVU && mode != TP_MODE_UVW) return fail(TP_ERR_INVALID_ARG, "mode must be TP_MODE_UVU or TP_MODE_UVW");
+  if (!paths || n_paths <= 0) return fail(TP_ERR_INVALID_ARG, "empty path list");
+  if (n_paths > kMaxPaths) return fail(TP_ERR_UNSUPPORTED, "at most %d paths", kMaxPaths);
+  if ((int)bi.size() > kMaxBlocks || (int)bs.size() > kMaxBlocks || (int)bo.size() > kMaxBlocks)
+    return fail(TP_ERR_UNSUPPORTED, "at most %d irreps blocks", kMaxBlocks);
+  for (auto* v : {&bi, &bs, &bo})
+    for (auto& b : *v)
+      if (b.l > 3) return fail(TP_ERR_UNSUPPORTED, "l = %d > 3", b.l);
+  for (auto& b : bs)
+    if (b.mul != 1 || b.parity != ((b.l & 1) ? -1 : 1))
+      return fail(TP_ERR_INVALID_ARG, "spherical-harmonic irreps must be 1x<l> with parity (-1)^l");
+  for (int p = 0; p < n_paths; ++p) {
+    const int a = paths[3 * p], b = paths[3 * p + 1], o = paths[3 * p + 2];
+    if (a < 0 || a >= (int)bi.size() || b < 0 || b >= (int)bs.size() || o < 0 || o >= (int)bo.size())
+      return fail(TP_ERR_INVALID_ARG, "path %d: block index out of range", p);
+    const int l1 = bi[a].l, l2 = bs[b].l, l3 = bo[o].l;
+    if (l3 < std::abs(l1 - l2) || l3 > l1 + l2)
+      return fail(TP_ERR_INVALID_ARG, "path %d (%d,%d,%d): triangle rule violated", p, l1, l2, l3);
+    if (bo[o].parity != bi[a].parity * bs[b].parity)
+      return fail(TP_ERR_INVALID_ARG, "path %d: parity rule violated", p);
+    if (mode == TP_MODE_UVU && bi[a].mul != bo[o].mul)
+      return fail(TP_ERR_INVALID_ARG, "path %d: uvu needs equal input and output multiplicity", p);
+  }
+  const int mul_in = bi[0].mul, mul_out = bo[0].mul;
+  for (auto& b : bi)
+    if (b.mul != mul_in) return fail(TP_ERR_UNSUPPORTED, "input blocks must share one multiplicity");
+  for (auto& b : bo)
+    if (b.mul != mul_out) return fail(TP_ERR_UNSUPPORTED, "output blocks must share one multiplicity");
+  // find the compiled specialisation
+  const SpecOps* found = nullptr;
+  for (int r = 0; r < kRegistrySize && !found; ++r) {
+    const SpecOps* s = kRegistry[r];
+    if (s->n_in != (int)bi.size() || s->n_sh != (int)bs.size() || s->n_out != (int)bo.size() ||
+        s->n_paths != n_paths)
+      continue;
+    bool ok = true;
+    for (int k = 0; k < s->n_in && ok; ++k) ok = s->in_ls[k] == bi[k].l;
+    for (int k = 0; k < s->n_sh && ok; ++k) ok = s->sh_ls[k] == bs[k].l;
+    for (int k = 0; k < s->n_out && ok; ++k) ok = s->out_ls[k] == bo[k].l;
+    for (int p = 0; p < n_paths && ok; ++p)
+      ok = s->paths[p][0] == paths[3 * p] && s->paths[p][1] == paths[3 * p + 1] &&
+           s->paths[p][2] == paths[3 * p + 2];
+    if (ok) found = s;
+  }
+  if (!found)
+    return fail(TP_ERR_UNSUPPORTED,
+                "no compiled specialisation for this irreps/path list (shipped: all-paths lmax 1/2/3 "
+                "and the 4-path lmax-1 list)");
+  if (mode == TP_MODE_UVW && (!found->uvw_edge || !found->uvw_bwd))
+    return fail(TP_ERR_UNSUPPORTED, "spec '%s' has no uvw kernels", found->name);
+  tp_plan_s* pl = new (std::nothrow) tp_plan_s;
+  if (!pl) return fail(TP_ERR_INVALID_ARG, "out of host memory");
+  std::memset(pl, 0, sizeof(*pl));
+  pl->ops = found;
+  pl->mode = mode;
+  pl->mul_in = mul_in;
+  pl->mul_out = mul_out;
+  int64_t in_dim = 0, out_dim = 0;
+  for (auto& b : bi) in_dim += (int64_t)b.mul * (2 * b.l + 1);
+  for (auto& b : bo) out_dim += (int64_t)b.mul * (2 * b.l + 1);
+  pl->in_dim = in_dim;
+  pl->out_dim = out_dim;
+  pl->n_paths = n_paths;
+  pl->nw = mode == TP_MODE_UVU ? (int64_t)n_paths * mul_in : n_paths;
+  pl->n_shared = mode == TP_MODE_UVW ? (int64_t)n_paths * mul_in * mul_out : 0;
+  pl->has_coeff = 0;
+  for (int p = 0; p < kMaxPaths; ++p) pl->coeff[p] = 1.0f;
+  if (path_coeff) {
+    for (int p = 0; p < n_paths; ++p) {
+      if (!std::isfinite(path_coeff[p])) {
+        delete pl;
+        return fail(TP_ERR_INVALID_ARG, "path_coeff[%d] is not finite", p);
+      }
+      pl->coeff[p] = (float)path_coeff[p];
+      if (path_coeff[p] != 1.0) pl->has_coeff = 1;
+    }
+  }
+  pl->flags = flags;
+  *plan = pl;
+  return TP_OK;
+}
+
+tp_status_t tp_plan_destroy(tp_plan_t plan) {
+  delete plan;
+  return TP_OK;
+}
+
+tp_status_t tp_plan_query(tp_plan_t plan, int64_t* in_dim, int64_t* out_dim, int64_t* n_edge_weights,
+                          int64_t* n_shared_weights) {
+  if (!plan) return fail(TP_ERR_INVALID_ARG, "plan is NULL");
+  if (in_dim) *in_dim = plan->in_dim;
+  if (out_dim) *out_dim = plan->out_dim;
+  if (n_edge_weights) *n_edge_weights = plan->nw;
+  if (n_shared_weights) *n_shared_weights = plan->n_shared;
+  return TP_OK;
+}
+
+tp_status_t tp_workspace_size(tp_plan_t plan, int64_t N, int64_t E, int32_t op, size_t* bytes) {
+  tp_status_t st = check_sizes(plan, N, E);
+  if (st != TP_OK) return st;
+  if (!bytes) return fail(TP_ERR_INVALID_ARG, "bytes is NULL");
+  if (op != TP_OP_FWD && op != TP_OP_BWD && op != TP_OP_DBWD) return fail(TP_ERR_INVALID_ARG, "bad op");
+  size_t need = 0;
+  if (op == TP_OP_FWD) need = (plan->flags & TP_FLAG_CHECK_INDICES) ? 256 : 0;
+  else need = ws_layout(N, E).total;   // enough to build the transpose in place
+  *bytes = need;
+  return TP_OK;
+}
+
+tp_status_t tp_csr_transpose(int64_t N, int64_t E, const int32_t* rowptr, const int32_t* src,
+                             int32_t* colptr, int32_t* perm, void* ws, size_t ws_bytes,
+                             tp_stream_t stream) {
+  (void)rowptr;
+  if (N < 0 || E < 0 || N >= (int64_t)1 << 31 || E >= (int64_t)1 << 31)
+    return fail(TP_ERR_INVALID_ARG, "N and E must be in [0, 2^31)");
+  if (!colptr || (E > 0 && (!src || !perm))) return fail(TP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned4(src) || !aligned4(colptr) || !aligned4(perm)) return fail(TP_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  const WsLayout L = ws_layout(N, E);
+  const size_t need = L.tmp + align256(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+  if (!ws || ws_bytes < need) return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  char* w = static_cast<char*>(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_csr_transpose((int)N, (int)E, src, colptr, perm,
+                                       reinterpret_cast<int32_t*>(w + L.counts),
+                                       reinterpret_cast<int32_t*>(w + L.tmp), s);
+  if (e != cudaSuccess) return cuda_fail(e, "csr_transpose");
+  return TP_OK;
+}
+
+tp_status_t tp_conv_fwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* rowptr, const int32_t* src,
+                        const float* x, const float* vec, const float* w, const float* W, float* y,
+                        void* ws, size_t ws_bytes, tp_stream_t stream) {
+  tp_status_t st = check_sizes(plan, N, E);
+  if (st != TP_OK) return st;
+  if (N == 0) return TP_OK;
+  if (!rowptr || !y) return fail(TP_ERR_INVALID_ARG, "rowptr and y must not be NULL");
+  if (E > 0 && (!src || !x || !vec || !w)) return fail(TP_ERR_INVALID_ARG, "src, x, vec and w must not be NULL");
+  if (plan->mode == TP_MODE_UVW && !W) return fail(TP_ERR_INVALID_ARG, "uvw mode needs W");
+  for (const void* p : {(const void*)rowptr, (const void*)src, (const void*)x, (const void*)vec,
+                        (const void*)w, (const void*)W, (const void*)y})
+    if (!aligned4(p)) return fail(TP_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  size_t need = 0;
+  tp_workspace_size(plan, N, E, TP_OP_FWD, &need);
+  if (need > 0 && (!ws || ws_bytes < need)) return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  LaunchArgs a = base_args(plan, N, E);
+  st = debug_prologue(plan, N, E, rowptr, src, ws, s, &a.err);
+  if (st != TP_OK) return st;
+  a.rowptr = rowptr;
+  a.src = src;
+  a.x = x;
+  a.vec = vec;
+  a.w = w;
+  a.y = y;
+  if (plan->mode != TP_MODE_UVU) return fail(TP_ERR_UNSUPPORTED, "uvw forward not available");
+  cudaError_t e = plan->ops->fwd_uvu(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tp_conv_fwd launch");
+  return TP_OK;
+}
+
+namespace {
+
+// Puts colptr / perm in place, building the transpose in the workspace when not supplied.
+tp_status_t sender_order(int64_t N, int64_t E, const int32_t* src, const int32_t*& colptr,
+                         const int32_t*& perm, void* ws, size_t ws_bytes, cudaStream_t s) {
+  if ((colptr == nullptr) != (perm == nullptr))
+    return fail(TP_ERR_INVALID_ARG, "colptr and perm must both be given or both be NULL");
+  if (colptr) return TP_OK;
+  const WsLayout L = ws_layout(N, E);
+  if (!ws || ws_bytes < L.total) return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes", L.total);
+  char* w = static_cast<char*>(ws);
+  int32_t* cp = reinterpret_cast<int32_t*>(w + L.colptr);
+  int32_t* pm = reinterpret_cast<int32_t*>(w + L.perm);
+  cudaError_t e = launch_csr_transpose((int)N, (int)E, src, cp, pm, reinterpret_cast<int32_t*>(w + L.counts),
+                                       reinterpret_cast<int32_t*>(w + L.tmp), s);
+  if (e != cudaSuccess) return cuda_fail(e, "csr_transpose");
+  colptr = cp;
+  perm = pm;
+  return TP_OK;
+}
+
+}  // namespace
+
+tp_status_t tp_conv_bwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* rowptr, const int32_t* src,
+                        const int32_t* colptr, const int32_t* perm, const float* x, const float* vec,
+                        const float* w, const float* W, const float* gy, float* gx, float* gw, float* gvec,
+                        float* gW, void* ws, size_t ws_bytes, tp_stream_t stream) {
+  tp_status_t st = check_sizes(plan, N, E);
+  if (st != TP_OK) return st;
+  if (N == 0) return TP_OK;
+  if (!rowptr || !gy || !x) return fail(TP_ERR_INVALID_ARG, "rowptr, x and gy must not be NULL");
+  if (E > 0 && (!src || !vec || !w)) return fail(TP_ERR_INVALID_ARG, "src, vec and w must not be NULL");
+  if (plan->mode == TP_MODE_UVW && !W) return fail(TP_ERR_INVALID_ARG, "uvw mode needs W");
+  for (const void* p : {(const void*)rowptr, (const void*)src, (const void*)colptr, (const void*)perm,
+                        (const void*)x, (const void*)vec, (const void*)w, (const void*)W, (const void*)gy,
+                        (const void*)gx, (const void*)gw, (const void*)gvec, (const void*)gW})
+    if (!aligned4(p)) return fail(TP_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  if (plan->mode != TP_MODE_UVU) return fail(TP_ERR_UNSUPPORTED, "uvw backward not available");
+  (void)gW;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  LaunchArgs a = base_args(plan, N, E);
+  st = debug_prologue(plan, N, E, rowptr, src, ws, s, &a.err);
+  if (st != TP_OK) return st;
+  if (!gx && !gw && !gvec) return TP_OK;
+  st = sender_order(N, E, src, colptr, perm, ws, ws_bytes, s);
+  if (st != TP_OK) return st;
+  a.rowptr = rowptr;
+  a.src = src;
+  a.colptr = colptr;
+  a.perm = perm;
+  a.x = x;
+  a.vec = vec;
+  a.w = w;
+  a.gy = gy;
+  a.gx = gx;
+  a.gw = gw;
+  a.gvec = gvec;
+  if (gvec) {
+    const int nsl = a.n_slices <= 1 ? 1 : (a.n_slices == 2 ? 2 : 4);
+    while (a.split * nsl > 4) a.split >>= 1;
+  }
+  cudaError_t e = plan->ops->bwd_uvu(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tp_conv_bwd launch");
+  return TP_OK;
+}
+
+tp_status_t tp_conv_dbwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* rowptr, const int32_t* src,
+                         const int32_t* colptr, const int32_t* perm, const float* x, const float* vec,
+                         const float* w, const float* W, const float* gy, const float* ggx, const float* ggw,
+                         const float* ggvec, float* g_gy, float* g_x, float* g_w, float* g_vec, void* ws,
+                         size_t ws_bytes, tp_stream_t stream) {
+  tp_status_t st = check_sizes(plan, N, E);
+  if (st != TP_OK) return st;
+  if (N == 0) return TP_OK;
+  (void)W;
+  if (plan->mode != TP_MODE_UVU) return fail(TP_ERR_UNSUPPORTED, "double backward is implemented for uvu");
+  if (!rowptr || !gy || !x) return fail(TP_ERR_INVALID_ARG, "rowptr, x and gy must not be NULL");
+  if (E > 0 && (!src || !vec || !w)) return fail(TP_ERR_INVALID_ARG, "src, vec and w must not be NULL");
+  for (const void* p : {(const void*)rowptr, (const void*)src, (const void*)colptr, (const void*)perm,
+                        (const void*)x, (const void*)vec, (const void*)w, (const void*)gy, (const void*)ggx,
+                        (const void*)ggw, (const void*)ggvec, (const void*)g_gy, (const void*)g_x,
+                        (const void*)g_w, (const void*)g_vec})
+    if (!aligned4(p)) return fail(TP_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  LaunchArgs a = base_args(plan, N, E);
+  st = debug_prologue(plan, N, E, rowptr, src, ws, s, &a.err);
+  if (st != TP_OK) return st;
+  a.rowptr = rowptr;
+  a.src = src;
+  a.x = x;
+  a.vec = vec;
+  a.w = w;
+  a.gy = gy;
+  a.ggx = ggx;
+  a.ggw = ggw;
+  a.ggvec = ggvec;
+  if (g_gy) {
+    a.y = g_gy;
+    cudaError_t e = plan->ops->dbwd_recv(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tp_conv_dbwd receiver pass");
+  }
+  if (!g_x && !g_w && !g_vec) return TP_OK;
+  st = sender_order(N, E, src, colptr, perm, ws, ws_bytes, s);
+  if (st != TP_OK) return st;
+  a.colptr = colptr;
+  a.perm = perm;
+  a.gx = g_x;
+  a.gw = g_w;
+  a.gvec = g_vec;
+  if (g_vec) {
+    const int nsl = a.n_slices <= 1 ? 1 : (a.n_slices == 2 ? 2 : 4);
+    while (a.split * nsl > 4) a.split >>= 1;
+  }
+  cudaError_t e = plan->ops->dbwd_send(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tp_conv_dbwd sender pass");
+  return TP_OK;
+}
+
+tp_status_t tp_get_device_error(tp_plan_t plan, void* ws, tp_stream_t stream, int32_t* code) {
+  if (!plan || !code) return fail(TP_ERR_INVALID_ARG, "plan and code must not be NULL");
+  *code = 0;
+  if (!(plan->flags & TP_FLAG_CHECK_INDICES)) return TP_OK;
+  if (!ws) return fail(TP_ERR_WORKSPACE, "workspace is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "tp_get_device_error");
+  *code = v;
+  return TP_OK;
+}
+
+}  // extern "C"

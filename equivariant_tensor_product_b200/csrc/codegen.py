@@ -1,0 +1,755 @@
+"""Generator for the compile-time tables and unrolled per-path bodies of the CUDA kernels.
+
+Product code (build step).  It computes, on its own route:
+  * complex Clebsch-Gordan coefficients by the Racah closed form (exact rationals under
+    one square root), turned into the real basis of the spherical harmonics below, then
+    normalised (||C||_F^2 = 2 l3 + 1 by construction) and signed so that the first
+    non-zero entry in row-major (m1, m2, m3) order is positive;
+  * real spherical harmonics as Cartesian polynomials P_lm(r_hat) for l <= 3 (component
+    normalisation, no Condon-Shortley phase, m = -l..l), with exact gradients and
+    Hessians taken symbolically, for the backward and double-backward passes.
+
+These are the ingredients named by "The GPU Workload That Rewrites Molecular Physics"
+(section "Equivariant feature transforms": spherical harmonics and Clebsch-Gordan tensor
+products) and "FlashTP" (abstract: sparse computation -- only non-zero CG entries are
+emitted).  For every supported path list ("spec") the generator writes one header with
+straight-line device functions: loads and stores of a channel's slice of a feature row,
+the SH evaluation, and the contraction bodies of forward, backward, double backward and
+the uvw edge pass, each a chain of FFMAs over the non-zero CG entries only.
+
+Usage: python codegen.py OUTDIR
+"""
+from __future__ import annotations
+
+import math
+import os
+import sys
+from fractions import Fraction
+from itertools import product
+from typing import Dict, List, Tuple
+
+# ---------------------------------------------------------------------------
+# Clebsch-Gordan by the Racah formula
+# ---------------------------------------------------------------------------
+
+
+def _f(n: int) -> int:
+    return math.factorial(n)
+
+
+def cg_complex(j1: int, m1: int, j2: int, m2: int, J: int, M: int) -> float:
+    """<j1 m1 j2 m2 | J M> (Condon-Shortley convention), Racah's closed form."""
+    if m1 + m2 != M or not (abs(j1 - j2) <= J <= j1 + j2):
+        return 0.0
+    if abs(m1) > j1 or abs(m2) > j2 or abs(M) > J:
+        return 0.0
+    pre = Fraction((2 * J + 1) * _f(J + j1 - j2) * _f(J - j1 + j2) * _f(j1 + j2 - J), _f(j1 + j2 + J + 1))
+    pre *= _f(J + M) * _f(J - M) * _f(j1 - m1) * _f(j1 + m1) * _f(j2 - m2) * _f(j2 + m2)
+    s = Fraction(0)
+    for k in range(0, j1 + j2 + J + 1):
+        args = [k, j1 + j2 - J - k, j1 - m1 - k, j2 + m2 - k, J - j2 + m1 + k, J - j1 - m2 + k]
+        if min(args) < 0:
+            continue
+        den = 1
+        for a in args:
+            den *= _f(a)
+        s += Fraction((-1) ** k, den)
+    return float(s) * math.sqrt(float(pre))
+
+
+def _real_basis(l: int):
+    """Rows: real index m; columns: complex index mu.  Real SH (no Condon-Shortley phase)
+    in terms of complex SH (with it): m>0 -> ((-1)^m Y^m + Y^-m)/sqrt2,
+    m<0 (k=|m|) -> ((-1)^k Y^k - Y^-k)/(i sqrt2), m=0 -> Y^0."""
+    d = 2 * l + 1
+    U = [[0j] * d for _ in range(d)]
+    r2 = math.sqrt(2.0)
+    for m in range(-l, l + 1):
+        if m > 0:
+            U[m + l][m + l] = (-1) ** m / r2
+            U[m + l][-m + l] = 1 / r2
+        elif m < 0:
+            k = -m
+            U[m + l][k + l] = (-1) ** k / (1j * r2)
+            U[m + l][-k + l] = -1 / (1j * r2)
+        else:
+            U[l][l] = 1.0
+    return U
+
+
+_CG_CACHE: Dict[Tuple[int, int, int], List[List[List[float]]]] = {}
+
+
+def cg_real(l1: int, l2: int, l3: int):
+    """Real CG tensor as nested lists [m1][m2][m3] (indices 0..2l)."""
+    key = (l1, l2, l3)
+    if key in _CG_CACHE:
+        return _CG_CACHE[key]
+    d1, d2, d3 = 2 * l1 + 1, 2 * l2 + 1, 2 * l3 + 1
+    U1, U2, U3 = _real_basis(l1), _real_basis(l2), _real_basis(l3)
+    Cc = {}
+    for a in range(d1):
+        for b in range(d2):
+            c = (a - l1) + (b - l2) + l3
+            if 0 <= c < d3:
+                v = cg_complex(l1, a - l1, l2, b - l2, l3, c - l3)
+                if v != 0.0:
+                    Cc[(a, b, c)] = v
+    R = [[[0j] * d3 for _ in range(d2)] for _ in range(d1)]
+    for i in range(d1):
+        for j in range(d2):
+            for k in range(d3):
+                acc = 0j
+                for (a, b, c), v in Cc.items():
+                    acc += U3[k][c] * v * U1[i][a].conjugate() * U2[j][b].conjugate()
+                R[i][j][k] = acc
+    mre = max(abs(R[i][j][k].real) for i in range(d1) for j in range(d2) for k in range(d3))
+    mim = max(abs(R[i][j][k].imag) for i in range(d1) for j in range(d2) for k in range(d3))
+    take_im = mim > mre
+    out = [[[0.0] * d3 for _ in range(d2)] for _ in range(d1)]
+    for i in range(d1):
+        for j in range(d2):
+            for k in range(d3):
+                z = R[i][j][k]
+                main, other = (z.imag, z.real) if take_im else (z.real, z.imag)
+                if abs(other) > 1e-12:
+                    raise ArithmeticError("real change of basis left a mixed phase")
+                out[i][j][k] = main if abs(main) > 1e-12 else 0.0
+    first = next(v for i in range(d1) for j in range(d2) for k in range(d3)
+                 for v in [out[i][j][k]] if v != 0.0)
+    if first < 0:
+        out = [[[-v + 0.0 for v in row] for row in pl] for pl in out]
+    _CG_CACHE[key] = out
+    return out
+
+
+def cg_nonzeros(l1, l2, l3):
+    C = cg_real(l1, l2, l3)
+    return [(i, j, k, C[i][j][k]) for i in range(2 * l1 + 1) for j in range(2 * l2 + 1)
+            for k in range(2 * l3 + 1) if C[i][j][k] != 0.0]
+
+
+# ---------------------------------------------------------------------------
+# Spherical-harmonic polynomials with symbolic derivatives
+# ---------------------------------------------------------------------------
+
+Poly = Dict[Tuple[int, int, int], float]      # monomial (i,j,k) of (x,y,z) -> coefficient
+
+
+def _p(*terms) -> Poly:
+    out: Poly = {}
+    for c, mono in terms:
+        out[mono] = out.get(mono, 0.0) + c
+    return out
+
+
+def sh_polys() -> Dict[int, List[Poly]]:
+    s = math.sqrt
+    X, Y, Z = (1, 0, 0), (0, 1, 0), (0, 0, 1)
+    return {
+        0: [_p((1.0, (0, 0, 0)))],
+        1: [_p((s(3), Y)), _p((s(3), Z)), _p((s(3), X))],
+        2: [_p((s(15), (1, 1, 0))), _p((s(15), (0, 1, 1))),
+            _p((s(5), (0, 0, 2)), (-s(5) / 2, (2, 0, 0)), (-s(5) / 2, (0, 2, 0))),
+            _p((s(15), (1, 0, 1))), _p((s(15) / 2, (2, 0, 0)), (-s(15) / 2, (0, 2, 0)))],
+        3: [_p((3 * s(70) / 4, (2, 1, 0)), (-s(70) / 4, (0, 3, 0))),
+            _p((s(105), (1, 1, 1))),
+            _p((s(42), (0, 1, 2)), (-s(42) / 4, (2, 1, 0)), (-s(42) / 4, (0, 3, 0))),
+            _p((s(7), (0, 0, 3)), (-3 * s(7) / 2, (2, 0, 1)), (-3 * s(7) / 2, (0, 2, 1))),
+            _p((s(42), (1, 0, 2)), (-s(42) / 4, (3, 0, 0)), (-s(42) / 4, (1, 2, 0))),
+            _p((s(105) / 2, (2, 0, 1)), (-s(105) / 2, (0, 2, 1))),
+            _p((s(70) / 4, (3, 0, 0)), (-3 * s(70) / 4, (1, 2, 0)))],
+    }
+
+
+def dpoly(p: Poly, axis: int) -> Poly:
+    out: Poly = {}
+    for mono, c in p.items():
+        if mono[axis] == 0:
+            continue
+        m = list(mono)
+        k = m[axis]
+        m[axis] -= 1
+        out[tuple(m)] = out.get(tuple(m), 0.0) + c * k
+    return {k: v for k, v in out.items() if v != 0.0}
+
+
+def _flt(v: float) -> str:
+    if v == 0.0:
+        return "0.0f"
+    return f"{v:.9e}f"
+
+
+MONO_NAMES = {(0, 0, 0): "1.0f"}
+
+
+def _mono_expr(mono) -> str:
+    i, j, k = mono
+    if mono == (0, 0, 0):
+        return "1.0f"
+    return "m_" + "x" * i + "y" * j + "z" * k
+
+
+def _poly_expr(p: Poly) -> str:
+    terms = [(c, mono) for mono, c in sorted(p.items()) if c != 0.0]
+    if not terms:
+        return "0.0f"
+    out = ""
+    for c, mono in terms:
+        me = _mono_expr(mono)
+        term = _flt(c) if me == "1.0f" else f"{_flt(c)} * {me}"
+        out = term if not out else f"{out} + {term}"
+    return out
+
+
+def _monomials_code(maxdeg: int, indent="    ") -> List[str]:
+    """Declares every monomial of (x,y,z) up to maxdeg as m_xxy... from rx, ry, rz."""
+    lines = []
+    names = {}
+    for deg in range(1, maxdeg + 1):
+        for i in range(deg + 1):
+            for j in range(deg + 1 - i):
+                k = deg - i - j
+                mono = (i, j, k)
+                name = _mono_expr(mono)
+                if deg == 1:
+                    src = {(1, 0, 0): "rx", (0, 1, 0): "ry", (0, 0, 1): "rz"}[mono]
+                else:
+                    # build from a lower monomial times one variable
+                    if i > 0:
+                        lower, var = (i - 1, j, k), "rx"
+                    elif j > 0:
+                        lower, var = (i, j - 1, k), "ry"
+                    else:
+                        lower, var = (i, j, k - 1), "rz"
+                    src = f"{_mono_expr(lower)} * {var}"
+                lines.append(f"{indent}const float {name} = {src};")
+                names[mono] = name
+    return lines
+
+
+# ---------------------------------------------------------------------------
+# Specs
+# ---------------------------------------------------------------------------
+
+
+class Spec:
+    def __init__(self, name, in_ls, sh_ls, out_ls, paths):
+        self.name = name
+        self.in_ls, self.sh_ls, self.out_ls = list(in_ls), list(sh_ls), list(out_ls)
+        self.paths = [tuple(p) for p in paths]
+        self.in_d = [2 * l + 1 for l in self.in_ls]
+        self.sh_d = [2 * l + 1 for l in self.sh_ls]
+        self.out_d = [2 * l + 1 for l in self.out_ls]
+        self.in_cum = [sum(self.in_d[:i]) for i in range(len(self.in_d))]
+        self.sh_cum = [sum(self.sh_d[:i]) for i in range(len(self.sh_d))]
+        self.out_cum = [sum(self.out_d[:i]) for i in range(len(self.out_d))]
+        self.IN_PC, self.NSH, self.OUT_PC = sum(self.in_d), sum(self.sh_d), sum(self.out_d)
+        self.P = len(self.paths)
+        self.triples = [(self.in_ls[a], self.sh_ls[b], self.out_ls[o]) for a, b, o in self.paths]
+        for (a, b, o), (l1, l2, l3) in zip(self.paths, self.triples):
+            if not abs(l1 - l2) <= l3 <= l1 + l2:
+                raise ValueError(f"{name}: path {(a, b, o)} breaks the triangle rule")
+        # uvw: per-path accumulator blocks (d3 per path)
+        self.a_d = [2 * t[2] + 1 for t in self.triples]
+        self.a_cum = [sum(self.a_d[:p]) for p in range(self.P)]
+        self.A_PC = sum(self.a_d)
+        self.LMAX_SH = max(self.sh_ls)
+
+    def nnz_total(self):
+        return sum(len(cg_nonzeros(*t)) for t in self.triples)
+
+
+def _lines_load(name, n_blocks, d, cum, arr, const=True):
+    """Straight-line load of one channel's slice of a [u][m] row."""
+    out = [f"  __device__ __forceinline__ static void {name}(const float* __restrict__ row, int mul, int c, float (&{arr})[{sum(d)}]) {{"]
+    for a in range(n_blocks):
+        out.append(f"    {{ const float* p = row + mul * {cum[a]} + c * {d[a]};")
+        for m in range(d[a]):
+            out.append(f"      {arr}[{cum[a] + m}] = __ldg(p + {m});")
+        out.append("    }")
+    out.append("  }")
+    return out
+
+
+def _lines_store(name, n_blocks, d, cum, arr):
+    out = [f"  __device__ __forceinline__ static void {name}(float* __restrict__ row, int mul, int c, const float (&{arr})[{sum(d)}]) {{"]
+    for a in range(n_blocks):
+        out.append(f"    {{ float* p = row + mul * {cum[a]} + c * {d[a]};")
+        for m in range(d[a]):
+            out.append(f"      p[{m}] = {arr}[{cum[a] + m}];")
+        out.append("    }")
+    out.append("  }")
+    return out
+
+
+def _gen_sh(spec: Spec) -> List[str]:
+    polys = sh_polys()
+    L = []
+    maxdeg = spec.LMAX_SH
+    # Y
+    L.append(f"  __device__ __forceinline__ static void sh(float rx, float ry, float rz, float (&Y)[{spec.NSH}]) {{")
+    L += _monomials_code(maxdeg)
+    for b, l in enumerate(spec.sh_ls):
+        for m in range(2 * l + 1):
+            L.append(f"    Y[{spec.sh_cum[b] + m}] = {_poly_expr(polys[l][m])};")
+    L.append("  }")
+    # gradient of P at r_hat: G[k][3]
+    L.append(f"  __device__ __forceinline__ static void sh_grad(float rx, float ry, float rz, float (&G)[{spec.NSH}][3]) {{")
+    L += _monomials_code(max(maxdeg - 1, 1))
+    for b, l in enumerate(spec.sh_ls):
+        for m in range(2 * l + 1):
+            for ax in range(3):
+                L.append(f"    G[{spec.sh_cum[b] + m}][{ax}] = {_poly_expr(dpoly(polys[l][m], ax))};")
+    L.append("  }")
+    # Hessian of P at r_hat times d: HD[k][3]
+    L.append(f"  __device__ __forceinline__ static void sh_hess_dot(float rx, float ry, float rz, float dx, float dy, float dz, float (&HD)[{spec.NSH}][3]) {{")
+    L += _monomials_code(max(maxdeg - 2, 1))
+    L.append("    (void)rx; (void)ry; (void)rz;")
+    dn = ["dx", "dy", "dz"]
+    for b, l in enumerate(spec.sh_ls):
+        for m in range(2 * l + 1):
+            for ax in range(3):
+                terms = []
+                g = dpoly(polys[l][m], ax)
+                for ax2 in range(3):
+                    h = dpoly(g, ax2)
+                    if h:
+                        terms.append(f"({_poly_expr(h)}) * {dn[ax2]}")
+                expr = " + ".join(terms) if terms else "0.0f"
+                L.append(f"    HD[{spec.sh_cum[b] + m}][{ax}] = {expr};")
+    L.append("  }")
+    # degree of each SH component (for the homogeneous derivative formulas)
+    degs = []
+    for l in spec.sh_ls:
+        degs += [l] * (2 * l + 1)
+    L.append(f"  __device__ __forceinline__ static float sh_degree(int k) {{ constexpr float d[{spec.NSH}] = {{{', '.join(f'{v}.0f' for v in degs)}}}; return d[k]; }}")
+    return L
+
+
+def _group(spec: Spec, key):
+    groups: Dict[Tuple[int, int], List[int]] = {}
+    for p, path in enumerate(spec.paths):
+        groups.setdefault(key(path), []).append(p)
+    return groups
+
+
+def _chain(terms, tgt, decl=True):
+    """Emit tgt = sum_i c_i * q_i as an FMUL followed by FFMAs."""
+    out = []
+    first = True
+    for c, q in terms:
+        if first:
+            out.append(f"      {'float ' if decl else ''}{tgt} = {_flt(c)} * {q};")
+            first = False
+        else:
+            out.append(f"      {tgt} = fmaf({_flt(c)}, {q}, {tgt});")
+    if first:
+        out.append(f"      {'float ' if decl else ''}{tgt} = 0.0f;")
+    return out
+
+
+def _gen_fwd(spec: Spec, name="fwd", weighted_out="acc", per_path_out=False) -> List[str]:
+    """acc[out(p), m3] += w[p] * sum C x[in(p), m1] Y[sh(p), m2]  (per_path_out: A blocks)."""
+    OUT = spec.A_PC if per_path_out else spec.OUT_PC
+    L = [f"  __device__ __forceinline__ static void {name}(const float (&x)[{spec.IN_PC}], const float (&Y)[{spec.NSH}], const float (&w)[{spec.P}], float (&{weighted_out})[{OUT}]) {{"]
+    groups = _group(spec, lambda p: (p[0], p[1]))
+    for (a, b), plist in groups.items():
+        la, lb = spec.in_ls[a], spec.sh_ls[b]
+        L.append(f"    {{ // in block {a} (l={la}) x SH block {b} (l={lb})")
+        used = set()
+        for p in plist:
+            for (i, j, k, c) in cg_nonzeros(*spec.triples[p]):
+                used.add((i, j))
+        for (i, j) in sorted(used):
+            xs, ys = f"x[{spec.in_cum[a] + i}]", f"Y[{spec.sh_cum[b] + j}]"
+            if lb == 0:
+                L.append(f"      const float q{i}_{j} = {xs};")
+            else:
+                L.append(f"      const float q{i}_{j} = {xs} * {ys};")
+        for p in plist:
+            o = spec.paths[p][2]
+            nz = cg_nonzeros(*spec.triples[p])
+            d3 = 2 * spec.triples[p][2] + 1
+            base = spec.a_cum[p] if per_path_out else spec.out_cum[o]
+            for k in range(d3):
+                terms = [(c, f"q{i}_{j}") for (i, j, kk, c) in nz if kk == k]
+                if not terms:
+                    continue
+                L += _chain(terms, f"t{p}_{k}")
+                L.append(f"      {weighted_out}[{base + k}] = fmaf(w[{p}], t{p}_{k}, {weighted_out}[{base + k}]);")
+        L.append("    }")
+    L.append("  }")
+    return L
+
+
+def _gen_bwd(spec: Spec) -> List[str]:
+    """Sender-side backward for one edge and one channel:
+       gw[p]        = sum C x[m1] Y[m2] gy[m3]
+       gx[in(p)]   += w[p] * sum_{m2,m3} C Y[m2] gy[m3]
+       gY[sh(p)]   += w[p] * sum_{m1,m3} C x[m1] gy[m3]      (WITH_GY)"""
+    L = ["  template <bool WITH_GY>",
+         f"  __device__ __forceinline__ static void bwd(const float (&x)[{spec.IN_PC}], const float (&Y)[{spec.NSH}], const float (&w)[{spec.P}], const float (&gy)[{spec.OUT_PC}], float (&gx)[{spec.IN_PC}], float (&gw)[{spec.P}], float (&gY)[{spec.NSH}]) {{"]
+    # Z_p[m1] = sum C Y[m2] gy[m3]  with products r = Y[m2] gy[m3] grouped by (b, o)
+    groups = _group(spec, lambda p: (p[1], p[2]))
+    for (b, o), plist in groups.items():
+        lb = spec.sh_ls[b]
+        L.append(f"    {{ // SH block {b} x out block {o}")
+        used = set()
+        for p in plist:
+            for (i, j, k, c) in cg_nonzeros(*spec.triples[p]):
+                used.add((j, k))
+        for (j, k) in sorted(used):
+            gs, ys = f"gy[{spec.out_cum[o] + k}]", f"Y[{spec.sh_cum[b] + j}]"
+            L.append(f"      const float r{j}_{k} = {gs};" if lb == 0 else f"      const float r{j}_{k} = {ys} * {gs};")
+        for p in plist:
+            a = spec.paths[p][0]
+            nz = cg_nonzeros(*spec.triples[p])
+            d1 = 2 * spec.triples[p][0] + 1
+            gwterms = []
+            for i in range(d1):
+                terms = [(c, f"r{j}_{k}") for (ii, j, k, c) in nz if ii == i]
+                if not terms:
+                    continue
+                L += _chain(terms, f"z{p}_{i}")
+                L.append(f"      gx[{spec.in_cum[a] + i}] = fmaf(w[{p}], z{p}_{i}, gx[{spec.in_cum[a] + i}]);")
+                gwterms.append(i)
+            if gwterms:
+                i0 = gwterms[0]
+                L.append(f"      float gwp{p} = x[{spec.in_cum[a] + i0}] * z{p}_{i0};")
+                for i in gwterms[1:]:
+                    L.append(f"      gwp{p} = fmaf(x[{spec.in_cum[a] + i}], z{p}_{i}, gwp{p});")
+                L.append(f"      gw[{p}] = gwp{p};")
+            else:
+                L.append(f"      gw[{p}] = 0.0f;")
+        L.append("    }")
+    # gY: products s = x[m1] gy[m3] grouped by (a, o)
+    L.append("    if constexpr (WITH_GY) {")
+    groups = _group(spec, lambda p: (p[0], p[2]))
+    for (a, o), plist in groups.items():
+        L.append(f"    {{ // in block {a} x out block {o}")
+        used = set()
+        for p in plist:
+            if spec.sh_ls[spec.paths[p][1]] == 0:
+                continue            # Y_0 is constant: no contribution to the direction gradient
+            for (i, j, k, c) in cg_nonzeros(*spec.triples[p]):
+                used.add((i, k))
+        for (i, k) in sorted(used):
+            L.append(f"      const float s{i}_{k} = x[{spec.in_cum[a] + i}] * gy[{spec.out_cum[o] + k}];")
+        for p in plist:
+            b = spec.paths[p][1]
+            if spec.sh_ls[b] == 0:
+                continue
+            nz = cg_nonzeros(*spec.triples[p])
+            d2 = 2 * spec.triples[p][1] + 1
+            for j in range(d2):
+                terms = [(c, f"s{i}_{k}") for (i, jj, k, c) in nz if jj == j]
+                if not terms:
+                    continue
+                L += _chain(terms, f"qq{p}_{j}")
+                L.append(f"      gY[{spec.sh_cum[b] + j}] = fmaf(w[{p}], qq{p}_{j}, gY[{spec.sh_cum[b] + j}]);")
+        L.append("    }")
+    L.append("    }")
+    L.append("  }")
+    return L
+
+
+def _gen_dbwd_recv(spec: Spec) -> List[str]:
+    """Receiver-side double backward for one edge and one channel:
+       acc[out(p)] += ggw[p] * C(x, Y) + w[p] * (C(ggx, Y) + C(x, Yp))"""
+    L = [f"  __device__ __forceinline__ static void dbwd_recv(const float (&x)[{spec.IN_PC}], const float (&ggx)[{spec.IN_PC}], const float (&Y)[{spec.NSH}], const float (&Yp)[{spec.NSH}], const float (&w)[{spec.P}], const float (&ggw)[{spec.P}], float (&acc)[{spec.OUT_PC}]) {{"]
+    groups = _group(spec, lambda p: (p[0], p[1]))
+    for (a, b), plist in groups.items():
+        lb = spec.sh_ls[b]
+        L.append(f"    {{ // in block {a} x SH block {b}")
+        used = set()
+        for p in plist:
+            for (i, j, k, c) in cg_nonzeros(*spec.triples[p]):
+                used.add((i, j))
+        for (i, j) in sorted(used):
+            xs, gs = f"x[{spec.in_cum[a] + i}]", f"ggx[{spec.in_cum[a] + i}]"
+            ys, yps = f"Y[{spec.sh_cum[b] + j}]", f"Yp[{spec.sh_cum[b] + j}]"
+            if lb == 0:
+                L.append(f"      const float q{i}_{j} = {xs};")
+                L.append(f"      const float h{i}_{j} = {gs};")
+            else:
+                L.append(f"      const float q{i}_{j} = {xs} * {ys};")
+                L.append(f"      const float h{i}_{j} = fmaf({gs}, {ys}, {xs} * {yps});")
+        for p in plist:
+            o = spec.paths[p][2]
+            nz = cg_nonzeros(*spec.triples[p])
+            d3 = 2 * spec.triples[p][2] + 1
+            for k in range(d3):
+                t1 = [(c, f"q{i}_{j}") for (i, j, kk, c) in nz if kk == k]
+                t2 = [(c, f"h{i}_{j}") for (i, j, kk, c) in nz if kk == k]
+                if not t1:
+                    continue
+                L += _chain(t1, f"t{p}_{k}")
+                L += _chain(t2, f"u{p}_{k}")
+                L.append(f"      acc[{spec.out_cum[o] + k}] = fmaf(ggw[{p}], t{p}_{k}, fmaf(w[{p}], u{p}_{k}, acc[{spec.out_cum[o] + k}]));")
+        L.append("    }")
+    L.append("  }")
+    return L
+
+
+def _gen_dbwd_send(spec: Spec) -> List[str]:
+    """Sender-side double backward for one edge and one channel:
+       gx[in(p)]  += sum_{m2,m3} C (ggw[p] Y[m2] + w[p] Yp[m2]) gy[m3]
+       gw[p]       = sum C (ggx[m1] Y[m2] + x[m1] Yp[m2]) gy[m3]
+       G1[sh(p)]  += ggw[p] Q(x, gy) + w[p] Q(ggx, gy);  G2[sh(p)] += w[p] Q(x, gy)
+       with Q(a, g)[m2] = sum_{m1,m3} C a[m1] g[m3]."""
+    L = [f"  __device__ __forceinline__ static void dbwd_send(const float (&x)[{spec.IN_PC}], const float (&ggx)[{spec.IN_PC}], const float (&Y)[{spec.NSH}], const float (&Yp)[{spec.NSH}], const float (&w)[{spec.P}], const float (&ggw)[{spec.P}], const float (&gy)[{spec.OUT_PC}], float (&gx)[{spec.IN_PC}], float (&gw)[{spec.P}], float (&G1)[{spec.NSH}], float (&G2)[{spec.NSH}]) {{"]
+    groups = _group(spec, lambda p: (p[1], p[2]))
+    for (b, o), plist in groups.items():
+        lb = spec.sh_ls[b]
+        L.append(f"    {{ // SH block {b} x out block {o}")
+        used = set()
+        for p in plist:
+            for (i, j, k, c) in cg_nonzeros(*spec.triples[p]):
+                used.add((j, k))
+        for (j, k) in sorted(used):
+            gs = f"gy[{spec.out_cum[o] + k}]"
+            ys, yps = f"Y[{spec.sh_cum[b] + j}]", f"Yp[{spec.sh_cum[b] + j}]"
+            if lb == 0:
+                L.append(f"      const float r{j}_{k} = {gs};")
+            else:
+                L.append(f"      const float r{j}_{k} = {ys} * {gs};")
+                L.append(f"      const float rp{j}_{k} = {yps} * {gs};")
+        for p in plist:
+            a = spec.paths[p][0]
+            nz = cg_nonzeros(*spec.triples[p])
+            d1 = 2 * spec.triples[p][0] + 1
+            gw_terms = []
+            for i in range(d1):
+                t1 = [(c, f"r{j}_{k}") for (ii, j, k, c) in nz if ii == i]
+                if not t1:
+                    continue
+                L += _chain(t1, f"z{p}_{i}")
+                if lb == 0:
+                    L.append(f"      const float zp{p}_{i} = 0.0f;")
+                else:
+                    L += _chain([(c, f"rp{j}_{k}") for (ii, j, k, c) in nz if ii == i], f"zp{p}_{i}")
+                ia = spec.in_cum[a] + i
+                L.append(f"      gx[{ia}] = fmaf(ggw[{p}], z{p}_{i}, fmaf(w[{p}], zp{p}_{i}, gx[{ia}]));")
+                gw_terms.append(i)
+            if gw_terms:
+                L.append(f"      float gwp{p} = 0.0f;")
+                for i in gw_terms:
+                    ia = spec.in_cum[a] + i
+                    L.append(f"      gwp{p} = fmaf(ggx[{ia}], z{p}_{i}, fmaf(x[{ia}], zp{p}_{i}, gwp{p}));")
+                L.append(f"      gw[{p}] = gwp{p};")
+            else:
+                L.append(f"      gw[{p}] = 0.0f;")
+        L.append("    }")
+    groups = _group(spec, lambda p: (p[0], p[2]))
+    for (a, o), plist in groups.items():
+        plist = [p for p in plist if spec.sh_ls[spec.paths[p][1]] != 0]
+        if not plist:
+            continue
+        L.append(f"    {{ // in block {a} x out block {o}")
+        used = set()
+        for p in plist:
+            for (i, j, k, c) in cg_nonzeros(*spec.triples[p]):
+                used.add((i, k))
+        for (i, k) in sorted(used):
+            L.append(f"      const float s{i}_{k} = x[{spec.in_cum[a] + i}] * gy[{spec.out_cum[o] + k}];")
+            L.append(f"      const float sg{i}_{k} = ggx[{spec.in_cum[a] + i}] * gy[{spec.out_cum[o] + k}];")
+        for p in plist:
+            b = spec.paths[p][1]
+            nz = cg_nonzeros(*spec.triples[p])
+            d2 = 2 * spec.triples[p][1] + 1
+            for j in range(d2):
+                t1 = [(c, f"s{i}_{k}") for (i, jj, k, c) in nz if jj == j]
+                if not t1:
+                    continue
+                L += _chain(t1, f"qa{p}_{j}")
+                L += _chain([(c, f"sg{i}_{k}") for (i, jj, k, c) in nz if jj == j], f"qb{p}_{j}")
+                kb = spec.sh_cum[b] + j
+                L.append(f"      G1[{kb}] = fmaf(ggw[{p}], qa{p}_{j}, fmaf(w[{p}], qb{p}_{j}, G1[{kb}]));")
+                L.append(f"      G2[{kb}] = fmaf(w[{p}], qa{p}_{j}, G2[{kb}]);")
+        L.append("    }")
+    L.append("  }")
+    return L
+
+
+def _gen_uvw_bwd(spec: Spec) -> List[str]:
+    """uvw sender pass for one edge and one channel u, given G[p, u, m3] (gradient of the
+    per-path aggregated state, gathered from the receiver):
+       gx[in(p)] += s[p] * sum_{m2,m3} C Y[m2] G[p, m3]
+       gs[p]     += sum C x[m1] Y[m2] G[p, m3]     (partial over this channel)
+       gY[sh(p)] += s[p] * sum_{m1,m3} C x[m1] G[p, m3]   (WITH_GY)"""
+    L = ["  template <bool WITH_GY>",
+         f"  __device__ __forceinline__ static void uvw_bwd(const float (&x)[{spec.IN_PC}], const float (&Y)[{spec.NSH}], const float (&s)[{spec.P}], const float (&G)[{spec.A_PC}], float (&gx)[{spec.IN_PC}], float (&gs)[{spec.P}], float (&gY)[{spec.NSH}]) {{"]
+    for p, (a, b, o) in enumerate(spec.paths):
+        lb = spec.sh_ls[b]
+        nz = cg_nonzeros(*spec.triples[p])
+        d1, d2 = 2 * spec.triples[p][0] + 1, 2 * spec.triples[p][1] + 1
+        L.append(f"    {{ // path {p}")
+        used = sorted({(j, k) for (i, j, k, c) in nz})
+        for (j, k) in used:
+            gs_ = f"G[{spec.a_cum[p] + k}]"
+            L.append(f"      const float r{j}_{k} = {gs_};" if lb == 0 else f"      const float r{j}_{k} = Y[{spec.sh_cum[b] + j}] * {gs_};")
+        gterms = []
+        for i in range(d1):
+            t = [(c, f"r{j}_{k}") for (ii, j, k, c) in nz if ii == i]
+            if not t:
+                continue
+            L += _chain(t, f"z{i}")
+            L.append(f"      gx[{spec.in_cum[a] + i}] = fmaf(s[{p}], z{i}, gx[{spec.in_cum[a] + i}]);")
+            gterms.append(i)
+        for i in gterms:
+            L.append(f"      gs[{p}] = fmaf(x[{spec.in_cum[a] + i}], z{i}, gs[{p}]);")
+        if lb != 0:
+            L.append("      if constexpr (WITH_GY) {")
+            used2 = sorted({(i, k) for (i, j, k, c) in nz})
+            for (i, k) in used2:
+                L.append(f"      const float s{i}_{k} = x[{spec.in_cum[a] + i}] * G[{spec.a_cum[p] + k}];")
+            for j in range(d2):
+                t = [(c, f"s{i}_{k}") for (i, jj, k, c) in nz if jj == j]
+                if not t:
+                    continue
+                L += _chain(t, f"qq{j}")
+                L.append(f"      gY[{spec.sh_cum[b] + j}] = fmaf(s[{p}], qq{j}, gY[{spec.sh_cum[b] + j}]);")
+            L.append("      }")
+        L.append("    }")
+    L.append("  }")
+    return L
+
+
+def gen_spec_header(spec: Spec) -> str:
+    L = [f"// Generated by codegen.py for spec '{spec.name}'.  Do not edit.",
+         f"// inputs l={spec.in_ls}  SH l={spec.sh_ls}  outputs l={spec.out_ls}",
+         f"// paths (in, sh, out) = {spec.paths}",
+         f"// non-zero CG entries: {spec.nnz_total()}",
+         "#pragma once",
+         f"struct Spec_{spec.name} {{",
+         f"  static constexpr int IN_PC = {spec.IN_PC};",
+         f"  static constexpr int OUT_PC = {spec.OUT_PC};",
+         f"  static constexpr int NSH = {spec.NSH};",
+         f"  static constexpr int P = {spec.P};",
+         f"  static constexpr int A_PC = {spec.A_PC};",
+         f"  static constexpr int LMAX_SH = {spec.LMAX_SH};",
+         f"  static constexpr int NNZ = {spec.nnz_total()};"]
+    L += _lines_load("load_in", len(spec.in_ls), spec.in_d, spec.in_cum, "x")
+    L += _lines_store("store_in", len(spec.in_ls), spec.in_d, spec.in_cum, "x")
+    L += _lines_load("load_out", len(spec.out_ls), spec.out_d, spec.out_cum, "y")
+    L += _lines_store("store_out", len(spec.out_ls), spec.out_d, spec.out_cum, "y")
+    # uvw per-path state rows [p][u][m3]
+    L += _lines_load("load_a", spec.P, spec.a_d, spec.a_cum, "a")
+    L += _lines_store("store_a", spec.P, spec.a_d, spec.a_cum, "a")
+    L += _gen_sh(spec)
+    L += _gen_fwd(spec)
+    L += _gen_fwd(spec, name="uvw_edge", weighted_out="A", per_path_out=True)
+    L += _gen_bwd(spec)
+    L += _gen_dbwd_recv(spec)
+    L += _gen_dbwd_send(spec)
+    L += _gen_uvw_bwd(spec)
+    L.append("};")
+    return "\n".join(L) + "\n"
+
+
+# ---------------------------------------------------------------------------
+# The compiled specialisations
+# ---------------------------------------------------------------------------
+
+def _all_paths(in_ls, in_par, sh_ls, out_irreps):
+    """(in, sh, out) index triples in (l1, l2, l3) lexicographic order over the given irreps."""
+    out = []
+    for a, (l1, p1) in enumerate(zip(in_ls, in_par)):
+        for b, l2 in enumerate(sh_ls):
+            for o, (l3, p3) in enumerate(out_irreps):
+                if abs(l1 - l2) <= l3 <= l1 + l2 and p3 == p1 * (-1) ** l2:
+                    out.append((a, b, o))
+    return out
+
+
+def builtin_specs() -> List[Spec]:
+    specs = []
+    # lmax 1: c1-style (4 paths into 0e + 1o)
+    specs.append(Spec("l1_c1", [0, 1], [0, 1], [0, 1], [(0, 0, 0), (0, 1, 1), (1, 0, 1), (1, 1, 0)]))
+    for L in (1, 2, 3):
+        ins = list(range(L + 1))
+        par = [(-1) ** l for l in ins]
+        outs = []
+        for l in range(L + 1):
+            for p in (1, -1):
+                if l == 0 and p == -1:
+                    continue
+                outs.append((l, p))
+        paths = _all_paths(ins, par, ins, outs)
+        # keep only reachable outputs
+        reach = sorted({o for _, _, o in paths})
+        remap = {o: k for k, o in enumerate(reach)}
+        paths = [(a, b, remap[o]) for a, b, o in paths]
+        specs.append(Spec(f"full_l{L}", ins, ins, [outs[o][0] for o in reach], paths))
+    return specs
+
+
+def _ops_initializer(s: Spec, fns) -> str:
+    def arr(v, n):
+        v = list(v) + [0] * (n - len(v))
+        return "{" + ", ".join(map(str, v)) + "}"
+    paths = "{" + ", ".join("{%d, %d, %d}" % p for p in s.paths) + "}"
+    return (f"  \"{s.name}\", {len(s.in_ls)}, {arr(s.in_ls, 16)}, {len(s.sh_ls)}, {arr(s.sh_ls, 16)}, "
+            f"{len(s.out_ls)}, {arr(s.out_ls, 16)}, {s.P}, {paths},\n"
+            f"  {s.IN_PC}, {s.OUT_PC}, {s.NSH}, {s.P}, {s.A_PC},\n  " + ", ".join(fns))
+
+
+# kernels of each spec, split into translation units that compile in parallel
+PARTS = {
+    "fwd": [("fwd_uvu", "launch_fwd_uvu")],
+    "bwd": [("bwd_uvu", "launch_bwd_uvu")],
+    "dbwd": [("dbwd_recv", "launch_dbwd_recv"), ("dbwd_send", "launch_dbwd_send")],
+}
+SLOTS = ["fwd_uvu", "bwd_uvu", "dbwd_recv", "dbwd_send", "uvw_edge", "uvw_bwd"]
+
+
+def main(outdir: str):
+    os.makedirs(outdir, exist_ok=True)
+    specs = builtin_specs()
+    written = []
+
+    def write(name, text):
+        path = os.path.join(outdir, name)
+        old = open(path).read() if os.path.exists(path) else None
+        if old != text:                      # keep mtimes stable for incremental builds
+            with open(path, "w") as f:
+                f.write(text)
+        written.append(name)
+
+    for s in specs:
+        write(f"spec_{s.name}.h", gen_spec_header(s))
+        for part, fns in PARTS.items():
+            body = [f"// Generated by codegen.py: {part} kernels of spec '{s.name}'.",
+                    '#include "tp_kernels.cuh"', f'#include "spec_{s.name}.h"', "namespace tp {"]
+            for slot, tmpl in fns:
+                body.append(f"cudaError_t {s.name}_{slot}(const LaunchArgs& a, cudaStream_t st) "
+                            f"{{ return {tmpl}<Spec_{s.name}>(a, st); }}")
+            body.append("}  // namespace tp")
+            write(f"k_{s.name}_{part}.cu", "\n".join(body) + "\n")
+    reg = ["// Generated by codegen.py: registry of compiled specialisations.",
+           '#include "tp_common.h"', "namespace tp {"]
+    have = {slot for fns in PARTS.values() for slot, _ in fns}
+    for s in specs:
+        for slot in SLOTS:
+            if slot in have:
+                reg.append(f"cudaError_t {s.name}_{slot}(const LaunchArgs&, cudaStream_t);")
+    for s in specs:
+        fns = [f"&{s.name}_{slot}" if slot in have else "nullptr" for slot in SLOTS]
+        reg.append(f"static const SpecOps ops_{s.name} = {{\n{_ops_initializer(s, fns)}}};")
+    reg.append("const SpecOps* const kRegistry[] = {" + ", ".join(f"&ops_{s.name}" for s in specs) + "};")
+    reg.append(f"const int kRegistrySize = {len(specs)};")
+    reg.append("}  // namespace tp")
+    write("registry.cu", "\n".join(reg) + "\n")
+    # CG table dump (text) for the host-side table tests
+    lines = []
+    for l1, l2, l3 in product(range(4), repeat=3):
+        if abs(l1 - l2) <= l3 <= l1 + l2:
+            for (i, j, k, c) in cg_nonzeros(l1, l2, l3):
+                lines.append(f"{l1} {l2} {l3} {i} {j} {k} {c:.17e}")
+    write("cg_tables.txt", "\n".join(lines) + "\n")
+    return specs, written
+
+
+if __name__ == "__main__":
+    main(sys.argv[1] if len(sys.argv) > 1 else os.path.join(os.path.dirname(__file__), "gen"))

@@ -1,0 +1,81 @@
+// Shared host/device declarations of the tensor-product convolution library (internal).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace tp {
+
+constexpr int kMaxPaths = 64;
+constexpr int kMaxBlocks = 16;
+constexpr int kMaxThreads = 128;   // launch bound of every edge kernel
+
+// Device error codes written to the workspace error word (debug index checks).
+enum DeviceError : int {
+  kDevOk = 0,
+  kDevBadRowptr = 1,
+  kDevBadSrc = 2,
+  kDevBadPerm = 3,
+};
+
+// Everything an edge kernel needs, passed by value as a kernel parameter.
+struct LaunchArgs {
+  int N;               // nodes
+  int E;               // edges
+  int mul;             // channels per irrep block (uniform), uvu: in == out
+  int mul_out;         // uvw: output channels
+  int in_dim, out_dim, nw, a_dim;
+  int split;           // warps per node row that split its edges (1..4)
+  int n_slices;        // 32-channel slices per row = ceil(mul / 32)
+  int has_coeff;       // path coefficients differ from 1
+  int check;           // bounds-check indices and report through *err
+  const int32_t* rowptr;
+  const int32_t* src;
+  const int32_t* colptr;
+  const int32_t* perm;
+  const float* x;
+  const float* vec;
+  const float* w;       // uvu w[E, P, mul]; uvw s[E, P]
+  const float* gy;
+  const float* ggx;
+  const float* ggw;
+  const float* ggvec;
+  const float* G;       // uvw: gradient of the per-path node state A
+  float* y;             // fwd output / dbwd g_gy / uvw A
+  float* gx;
+  float* gw;
+  float* gvec;
+  int* err;
+  float coeff[kMaxPaths];
+};
+
+// Number of kernels the library has launched in this process (diagnostics).
+void count_launches(int n);
+
+// Host-side launchers of one compiled specialisation.
+typedef cudaError_t (*LaunchFn)(const LaunchArgs&, cudaStream_t);
+
+struct SpecOps {
+  const char* name;
+  int n_in, in_ls[kMaxBlocks];
+  int n_sh, sh_ls[kMaxBlocks];
+  int n_out, out_ls[kMaxBlocks];
+  int n_paths, paths[kMaxPaths][3];
+  int IN_PC, OUT_PC, NSH, P, A_PC;
+  LaunchFn fwd_uvu;         // y = conv(x)
+  LaunchFn bwd_uvu;         // gx, gw (gvec when args.gvec != nullptr), sender order
+  LaunchFn dbwd_recv;       // g_gy, receiver order
+  LaunchFn dbwd_send;       // g_x, g_w, g_vec, sender order
+  LaunchFn uvw_edge;        // A[i, p, u, m3] aggregated per path (uvw forward edge pass)
+  LaunchFn uvw_bwd;         // gx, gs (gvec) from G = dA, sender order
+};
+
+extern const SpecOps* const kRegistry[];
+extern const int kRegistrySize;
+
+// CSR helpers (csr.cu)
+cudaError_t launch_csr_validate(int N, int E, const int32_t* rowptr, const int32_t* src, int* err,
+                                cudaStream_t s);
+cudaError_t launch_csr_transpose(int N, int E, const int32_t* src, int32_t* colptr, int32_t* perm,
+                                 int32_t* counts, int32_t* tmp, cudaStream_t s);
+
+}  // namespace tp

@@ -1,0 +1,624 @@
+// Edge kernels of the tensor-product convolution, templated on a generated spec S.
+//
+// Operation ("Sobek: Streaming Equivariant Tensor Product Convolutions", abstract;
+// "FlashTP", abstract): for each receiver i and each incoming edge e = (j -> i)
+//   y[i, out(p), u, m3] += w[e, p, u] * sum_{m1,m2} C_p[m1, m2, m3] x[j, in(p), u, m1] Y_l2(r_e)[m2]
+// with the real spherical harmonics Y of the edge direction evaluated in registers and
+// only the non-zero C_p entries unrolled (S::fwd, generated).
+//
+// Schedule (B200): a CTA owns one node row and one 32-channel slice of it; lane = channel,
+// so the per-channel work of an edge is identical on every lane and variable degree costs
+// no divergence.  Up to four warps of a CTA ("phases") take interleaved edges of the same
+// row and their register accumulators are summed in a fixed order through shared memory:
+// the result is deterministic and no float atomics touch the output.  Rows are scheduled
+// dynamically by the hardware block scheduler, which balances the degree spread.  Edge
+// geometry (sender index, edge vector) is loaded 32 edges at a time, one per lane
+// (coalesced), and broadcast with warp shuffles.  No edge-sized message, weight or adjoint
+// is written anywhere: each edge's products are consumed straight into receiver (forward,
+// double-backward receiver pass) or sender (backward, double-backward sender pass) state.
+#pragma once
+#include "tp_common.h"
+
+namespace tp {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ void edge_geometry(float vx, float vy, float vz, float& rx, float& ry,
+                                              float& rz, float& inv_r) {
+  const float r2 = fmaf(vx, vx, fmaf(vy, vy, vz * vz));
+  inv_r = r2 > 0.f ? rsqrtf(r2) : 0.f;
+  rx = vx * inv_r;
+  ry = vy * inv_r;
+  rz = vz * inv_r;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Receiver of edge e: the last row i with rowptr[i] <= e (empty rows share their start).
+__device__ __forceinline__ int find_row(const int32_t* __restrict__ rowptr, int N, int e) {
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(rowptr + mid) <= e) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void report(const LaunchArgs& a, int code) {
+  if (a.err) atomicCAS(a.err, 0, code);
+}
+
+template <int P>
+__device__ __forceinline__ void load_path_weights(const LaunchArgs& a, int e, int c, float (&w)[P]) {
+  const float* row = a.w + (int64_t)e * a.nw + c;
+#pragma unroll
+  for (int p = 0; p < P; ++p) w[p] = __ldg(row + (int64_t)p * a.mul);
+  if (a.has_coeff) {
+#pragma unroll
+    for (int p = 0; p < P; ++p) w[p] *= a.coeff[p];
+  }
+}
+
+template <int P>
+__device__ __forceinline__ void load_path_weights_from(const LaunchArgs& a, const float* base, int e,
+                                                       int c, float (&w)[P]) {
+  if (base == nullptr) {
+#pragma unroll
+    for (int p = 0; p < P; ++p) w[p] = 0.f;
+    return;
+  }
+  const float* row = base + (int64_t)e * a.nw + c;
+#pragma unroll
+  for (int p = 0; p < P; ++p) w[p] = __ldg(row + (int64_t)p * a.mul);
+  if (a.has_coeff) {
+#pragma unroll
+    for (int p = 0; p < P; ++p) w[p] *= a.coeff[p];
+  }
+}
+
+// Sums per-phase register arrays into phase 0 through shared memory, in phase order.
+template <int N>
+__device__ __forceinline__ void reduce_phases(float (&acc)[N], float* smem, int phase, int split,
+                                              int lane, int group, int ngroups) {
+  if (split <= 1) return;
+  // layout: [(phase-1)][group][N][32]
+  if (phase > 0) {
+    float* dst = smem + (((size_t)(phase - 1) * ngroups + group) * N) * 32 + lane;
+#pragma unroll
+    for (int k = 0; k < N; ++k) dst[k * 32] = acc[k];
+  }
+  __syncthreads();
+  if (phase == 0) {
+    for (int ph = 1; ph < split; ++ph) {
+      const float* s = smem + (((size_t)(ph - 1) * ngroups + group) * N) * 32 + lane;
+#pragma unroll
+      for (int k = 0; k < N; ++k) acc[k] += s[k * 32];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Forward, uvu, receiver order.  grid = N * n_slices, block = 32 * split.
+// ---------------------------------------------------------------------------------------
+template <class S>
+__global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__ LaunchArgs a) {
+  extern __shared__ float smem[];
+  const int lane = threadIdx.x & 31;
+  const int phase = threadIdx.x >> 5;
+  const int row = blockIdx.x / a.n_slices;
+  const int sl = blockIdx.x - row * a.n_slices;
+  const int c = sl * 32 + lane;
+  const bool act = c < a.mul;
+  int e0 = __ldg(a.rowptr + row), e1 = __ldg(a.rowptr + row + 1);
+  if (a.check) {  // never read outside [0, E) whatever rowptr holds
+    e0 = max(0, min(e0, a.E));
+    e1 = max(e0, min(e1, a.E));
+  }
+  const int st = a.split;
+  float acc[S::OUT_PC];
+#pragma unroll
+  for (int k = 0; k < S::OUT_PC; ++k) acc[k] = 0.f;
+
+  for (int base = e0 + phase; base < e1; base += 32 * st) {
+    const int my_e = base + lane * st;
+    int my_j = 0;
+    float vx = 0.f, vy = 0.f, vz = 0.f;
+    if (my_e < e1) {
+      my_j = __ldg(a.src + my_e);
+      vx = __ldg(a.vec + 3 * (int64_t)my_e);
+      vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
+      vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
+      if (a.check && (unsigned)my_j >= (unsigned)a.N) {
+        report(a, kDevBadSrc);
+        vx = vy = vz = 0.f;
+        my_j = -1;
+      }
+    }
+    const int ne = min(32, (e1 - base + st - 1) / st);
+    for (int k = 0; k < ne; ++k) {
+      const int e = base + k * st;
+      const int j = __shfl_sync(kFull, my_j, k);
+      const float ux = __shfl_sync(kFull, vx, k);
+      const float uy = __shfl_sync(kFull, vy, k);
+      const float uz = __shfl_sync(kFull, vz, k);
+      if (j < 0) continue;
+      float rx, ry, rz, ir;
+      edge_geometry(ux, uy, uz, rx, ry, rz, ir);
+      float Y[S::NSH];
+      S::sh(rx, ry, rz, Y);
+      if (act) {
+        float x[S::IN_PC];
+        S::load_in(a.x + (int64_t)j * a.in_dim, a.mul, c, x);
+        float w[S::P];
+        load_path_weights(a, e, c, w);
+        S::fwd(x, Y, w, acc);
+      }
+    }
+  }
+  reduce_phases(acc, smem, phase, st, lane, 0, 1);
+  if (phase == 0 && act) S::store_out(a.y + (int64_t)row * a.out_dim, a.mul, c, acc);
+}
+
+// ---------------------------------------------------------------------------------------
+// Backward, uvu, sender order (through the stable transpose perm; each edge's receiver is
+// found by a binary search of rowptr, one lane per edge).
+//   gx[j]  = sum over edges leaving j (segmented, in registers)
+//   gw[e]  = per edge, written at its own position
+//   gvec[e]= per edge, channel sum: warp reduction, then across slice warps via smem.
+// GVEC=false: grid = N * n_slices, block = 32*split (slices independent).
+// GVEC=true : grid = N, block = 32*split*NSL (all slices of a row in one CTA).
+// ---------------------------------------------------------------------------------------
+template <class S, bool GVEC, int NSL>
+__global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__ LaunchArgs a) {
+  extern __shared__ float smem[];
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  const int st = a.split;
+  const int phase = wid % st;
+  int node, sl;
+  if (GVEC) {
+    node = blockIdx.x;
+    sl = wid / st;
+  } else {
+    node = blockIdx.x / a.n_slices;
+    sl = blockIdx.x - node * a.n_slices;
+  }
+  const int c = sl * 32 + lane;
+  const bool act = c < a.mul;
+  int q0 = __ldg(a.colptr + node), q1 = __ldg(a.colptr + node + 1);
+  if (a.check) {
+    q0 = max(0, min(q0, a.E));
+    q1 = max(q0, min(q1, a.E));
+  }
+
+  float x[S::IN_PC];
+  float gx[S::IN_PC];
+#pragma unroll
+  for (int k = 0; k < S::IN_PC; ++k) gx[k] = 0.f;
+  if (act) S::load_in(a.x + (int64_t)node * a.in_dim, a.mul, c, x);
+  else {
+#pragma unroll
+    for (int k = 0; k < S::IN_PC; ++k) x[k] = 0.f;
+  }
+  // gvec partial slots: [phase][edge-in-batch][slice][4]
+  float* gslot = smem + (size_t)(st > 1 ? (st - 1) * NSL * S::IN_PC * 32 : 0);
+
+  for (int base = q0 + phase; base < q1; base += 32 * st) {
+    const int my_q = base + lane * st;
+    int my_e = -1, my_i = 0;
+    float vx = 0.f, vy = 0.f, vz = 0.f;
+    if (my_q < q1) {
+      my_e = __ldg(a.perm + my_q);
+      if (a.check && (unsigned)my_e >= (unsigned)a.E) {
+        report(a, kDevBadPerm);
+        my_e = -1;
+      } else {
+        my_i = find_row(a.rowptr, a.N, my_e);
+        vx = __ldg(a.vec + 3 * (int64_t)my_e);
+        vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
+        vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
+      }
+    }
+    const int ne = min(32, (q1 - base + st - 1) / st);
+    for (int k = 0; k < ne; ++k) {
+      const int e = __shfl_sync(kFull, my_e, k);
+      const int i = __shfl_sync(kFull, my_i, k);
+      const float ux = __shfl_sync(kFull, vx, k);
+      const float uy = __shfl_sync(kFull, vy, k);
+      const float uz = __shfl_sync(kFull, vz, k);
+      float rx, ry, rz, ir;
+      edge_geometry(ux, uy, uz, rx, ry, rz, ir);
+      float Y[S::NSH];
+      S::sh(rx, ry, rz, Y);
+      float gY[S::NSH];
+#pragma unroll
+      for (int m = 0; m < S::NSH; ++m) gY[m] = 0.f;
+      if (act && e >= 0) {
+        float gyv[S::OUT_PC];
+        S::load_out(a.gy + (int64_t)i * a.out_dim, a.mul, c, gyv);
+        float w[S::P];
+        load_path_weights(a, e, c, w);
+        float gw[S::P];
+        S::template bwd<GVEC>(x, Y, w, gyv, gx, gw, gY);
+        if (a.gw) {
+          float* row = a.gw + (int64_t)e * a.nw + c;
+#pragma unroll
+          for (int p = 0; p < S::P; ++p) row[(int64_t)p * a.mul] = a.has_coeff ? gw[p] * a.coeff[p] : gw[p];
+        }
+      }
+      if constexpr (GVEC) {
+        // d Y_m / d v = (grad P_m(r) - l_m Y_m r) / |v|
+        float G[S::NSH][3];
+        S::sh_grad(rx, ry, rz, G);
+        float h0 = 0.f, h1 = 0.f, h2 = 0.f, sdeg = 0.f;
+#pragma unroll
+        for (int m = 0; m < S::NSH; ++m) {
+          h0 = fmaf(gY[m], G[m][0], h0);
+          h1 = fmaf(gY[m], G[m][1], h1);
+          h2 = fmaf(gY[m], G[m][2], h2);
+          sdeg = fmaf(S::sh_degree(m) * gY[m], Y[m], sdeg);
+        }
+        h0 = warp_sum(h0);
+        h1 = warp_sum(h1);
+        h2 = warp_sum(h2);
+        sdeg = warp_sum(sdeg);
+        if (NSL == 1) {
+          if (lane == 0 && e >= 0) {
+            float* g = a.gvec + 3 * (int64_t)e;
+            g[0] = ir * (h0 - rx * sdeg);
+            g[1] = ir * (h1 - ry * sdeg);
+            g[2] = ir * (h2 - rz * sdeg);
+          }
+        } else if (lane == 0) {
+          float* s = gslot + (((size_t)phase * 32 + k) * NSL + sl) * 4;
+          s[0] = h0;
+          s[1] = h1;
+          s[2] = h2;
+          s[3] = sdeg;
+        }
+      }
+    }
+    if constexpr (GVEC && NSL > 1) {
+      named_barrier(1 + phase, 32 * NSL);
+      if (sl == 0 && lane < ne && my_e >= 0) {
+        float h0 = 0.f, h1 = 0.f, h2 = 0.f, sdeg = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < NSL; ++s2) {
+          const float* s = gslot + (((size_t)phase * 32 + lane) * NSL + s2) * 4;
+          h0 += s[0];
+          h1 += s[1];
+          h2 += s[2];
+          sdeg += s[3];
+        }
+        float rx, ry, rz, ir;
+        edge_geometry(vx, vy, vz, rx, ry, rz, ir);
+        float* g = a.gvec + 3 * (int64_t)my_e;
+        g[0] = ir * (h0 - rx * sdeg);
+        g[1] = ir * (h1 - ry * sdeg);
+        g[2] = ir * (h2 - rz * sdeg);
+      }
+      named_barrier(1 + phase, 32 * NSL);
+    }
+  }
+  reduce_phases(gx, smem, phase, st, lane, GVEC ? sl : 0, GVEC ? NSL : 1);
+  if (phase == 0 && act && a.gx) S::store_in(a.gx + (int64_t)node * a.in_dim, a.mul, c, gx);
+}
+
+// ---------------------------------------------------------------------------------------
+// Double backward, receiver pass: g_gy[i] = sum_e TP(ggx; Y, w) + TP(x; Y, ggw) + TP(x; dY[ggvec], w)
+// ---------------------------------------------------------------------------------------
+template <class S>
+__global__ void __launch_bounds__(kMaxThreads) k_dbwd_recv(const __grid_constant__ LaunchArgs a) {
+  extern __shared__ float smem[];
+  const int lane = threadIdx.x & 31;
+  const int phase = threadIdx.x >> 5;
+  const int row = blockIdx.x / a.n_slices;
+  const int sl = blockIdx.x - row * a.n_slices;
+  const int c = sl * 32 + lane;
+  const bool act = c < a.mul;
+  int e0 = __ldg(a.rowptr + row), e1 = __ldg(a.rowptr + row + 1);
+  if (a.check) {  // never read outside [0, E) whatever rowptr holds
+    e0 = max(0, min(e0, a.E));
+    e1 = max(e0, min(e1, a.E));
+  }
+  const int st = a.split;
+  float acc[S::OUT_PC];
+#pragma unroll
+  for (int k = 0; k < S::OUT_PC; ++k) acc[k] = 0.f;
+
+  for (int base = e0 + phase; base < e1; base += 32 * st) {
+    const int my_e = base + lane * st;
+    int my_j = 0;
+    float vx = 0.f, vy = 0.f, vz = 0.f, dx = 0.f, dy = 0.f, dz = 0.f;
+    if (my_e < e1) {
+      my_j = __ldg(a.src + my_e);
+      vx = __ldg(a.vec + 3 * (int64_t)my_e);
+      vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
+      vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
+      if (a.ggvec) {
+        dx = __ldg(a.ggvec + 3 * (int64_t)my_e);
+        dy = __ldg(a.ggvec + 3 * (int64_t)my_e + 1);
+        dz = __ldg(a.ggvec + 3 * (int64_t)my_e + 2);
+      }
+      if (a.check && (unsigned)my_j >= (unsigned)a.N) {
+        report(a, kDevBadSrc);
+        my_j = -1;
+      }
+    }
+    const int ne = min(32, (e1 - base + st - 1) / st);
+    for (int k = 0; k < ne; ++k) {
+      const int e = base + k * st;
+      const int j = __shfl_sync(kFull, my_j, k);
+      const float ux = __shfl_sync(kFull, vx, k);
+      const float uy = __shfl_sync(kFull, vy, k);
+      const float uz = __shfl_sync(kFull, vz, k);
+      const float ddx = __shfl_sync(kFull, dx, k);
+      const float ddy = __shfl_sync(kFull, dy, k);
+      const float ddz = __shfl_sync(kFull, dz, k);
+      if (j < 0) continue;
+      float rx, ry, rz, ir;
+      edge_geometry(ux, uy, uz, rx, ry, rz, ir);
+      float Y[S::NSH], Yp[S::NSH];
+      S::sh(rx, ry, rz, Y);
+      {
+        float G[S::NSH][3];
+        S::sh_grad(rx, ry, rz, G);
+        const float rd = fmaf(rx, ddx, fmaf(ry, ddy, rz * ddz));
+#pragma unroll
+        for (int m = 0; m < S::NSH; ++m) {
+          const float gd = fmaf(G[m][0], ddx, fmaf(G[m][1], ddy, G[m][2] * ddz));
+          Yp[m] = ir * (gd - S::sh_degree(m) * Y[m] * rd);
+        }
+      }
+      if (act) {
+        float x[S::IN_PC], ggx[S::IN_PC];
+        S::load_in(a.x + (int64_t)j * a.in_dim, a.mul, c, x);
+        if (a.ggx) S::load_in(a.ggx + (int64_t)j * a.in_dim, a.mul, c, ggx);
+        else {
+#pragma unroll
+          for (int m = 0; m < S::IN_PC; ++m) ggx[m] = 0.f;
+        }
+        float w[S::P], ggw[S::P];
+        load_path_weights(a, e, c, w);
+        load_path_weights_from(a, a.ggw, e, c, ggw);
+        S::dbwd_recv(x, ggx, Y, Yp, w, ggw, acc);
+      }
+    }
+  }
+  reduce_phases(acc, smem, phase, st, lane, 0, 1);
+  if (phase == 0 && act) S::store_out(a.y + (int64_t)row * a.out_dim, a.mul, c, acc);
+}
+
+// ---------------------------------------------------------------------------------------
+// Double backward, sender pass: g_x[j] (segmented), g_w[e], g_vec[e].
+// ---------------------------------------------------------------------------------------
+template <class S, bool GVEC, int NSL>
+__global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant__ LaunchArgs a) {
+  extern __shared__ float smem[];
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  const int st = a.split;
+  const int phase = wid % st;
+  int node, sl;
+  if (GVEC) {
+    node = blockIdx.x;
+    sl = wid / st;
+  } else {
+    node = blockIdx.x / a.n_slices;
+    sl = blockIdx.x - node * a.n_slices;
+  }
+  const int c = sl * 32 + lane;
+  const bool act = c < a.mul;
+  int q0 = __ldg(a.colptr + node), q1 = __ldg(a.colptr + node + 1);
+  if (a.check) {
+    q0 = max(0, min(q0, a.E));
+    q1 = max(q0, min(q1, a.E));
+  }
+
+  float x[S::IN_PC], ggx[S::IN_PC], gx[S::IN_PC];
+#pragma unroll
+  for (int k = 0; k < S::IN_PC; ++k) {
+    gx[k] = 0.f;
+    x[k] = 0.f;
+    ggx[k] = 0.f;
+  }
+  if (act) {
+    S::load_in(a.x + (int64_t)node * a.in_dim, a.mul, c, x);
+    if (a.ggx) S::load_in(a.ggx + (int64_t)node * a.in_dim, a.mul, c, ggx);
+  }
+  float* gslot = smem + (size_t)(st > 1 ? (st - 1) * NSL * S::IN_PC * 32 : 0);
+
+  for (int base = q0 + phase; base < q1; base += 32 * st) {
+    const int my_q = base + lane * st;
+    int my_e = -1, my_i = 0;
+    float vx = 0.f, vy = 0.f, vz = 0.f, dx = 0.f, dy = 0.f, dz = 0.f;
+    if (my_q < q1) {
+      my_e = __ldg(a.perm + my_q);
+      if (a.check && (unsigned)my_e >= (unsigned)a.E) {
+        report(a, kDevBadPerm);
+        my_e = -1;
+      } else {
+        my_i = find_row(a.rowptr, a.N, my_e);
+        vx = __ldg(a.vec + 3 * (int64_t)my_e);
+        vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
+        vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
+        if (a.ggvec) {
+          dx = __ldg(a.ggvec + 3 * (int64_t)my_e);
+          dy = __ldg(a.ggvec + 3 * (int64_t)my_e + 1);
+          dz = __ldg(a.ggvec + 3 * (int64_t)my_e + 2);
+        }
+      }
+    }
+    const int ne = min(32, (q1 - base + st - 1) / st);
+    for (int k = 0; k < ne; ++k) {
+      const int e = __shfl_sync(kFull, my_e, k);
+      const int i = __shfl_sync(kFull, my_i, k);
+      const float ux = __shfl_sync(kFull, vx, k);
+      const float uy = __shfl_sync(kFull, vy, k);
+      const float uz = __shfl_sync(kFull, vz, k);
+      const float ddx = __shfl_sync(kFull, dx, k);
+      const float ddy = __shfl_sync(kFull, dy, k);
+      const float ddz = __shfl_sync(kFull, dz, k);
+      float rx, ry, rz, ir;
+      edge_geometry(ux, uy, uz, rx, ry, rz, ir);
+      const float rd = fmaf(rx, ddx, fmaf(ry, ddy, rz * ddz));
+      float Y[S::NSH], Yp[S::NSH], G[S::NSH][3];
+      S::sh(rx, ry, rz, Y);
+      S::sh_grad(rx, ry, rz, G);
+#pragma unroll
+      for (int m = 0; m < S::NSH; ++m) {
+        const float gd = fmaf(G[m][0], ddx, fmaf(G[m][1], ddy, G[m][2] * ddz));
+        Yp[m] = ir * (gd - S::sh_degree(m) * Y[m] * rd);
+      }
+      float G1[S::NSH], G2[S::NSH];
+#pragma unroll
+      for (int m = 0; m < S::NSH; ++m) G1[m] = G2[m] = 0.f;
+      if (act && e >= 0) {
+        float gyv[S::OUT_PC];
+        S::load_out(a.gy + (int64_t)i * a.out_dim, a.mul, c, gyv);
+        float w[S::P], ggw[S::P];
+        load_path_weights(a, e, c, w);
+        load_path_weights_from(a, a.ggw, e, c, ggw);
+        float gw[S::P];
+        S::dbwd_send(x, ggx, Y, Yp, w, ggw, gyv, gx, gw, G1, G2);
+        if (a.gw) {
+          float* row = a.gw + (int64_t)e * a.nw + c;
+#pragma unroll
+          for (int p = 0; p < S::P; ++p) row[(int64_t)p * a.mul] = a.has_coeff ? gw[p] * a.coeff[p] : gw[p];
+        }
+      }
+      if constexpr (GVEC) {
+        // g = sum_m G1_m dY_m/dv + G2_m (d^2 Y_m/dv^2) ggvec
+        float HD[S::NSH][3];
+        S::sh_hess_dot(rx, ry, rz, ddx, ddy, ddz, HD);
+        float g0 = 0.f, g1 = 0.f, g2 = 0.f;
+        const float ir2 = ir * ir;
+#pragma unroll
+        for (int m = 0; m < S::NSH; ++m) {
+          const float l = S::sh_degree(m);
+          const float gdm = fmaf(G[m][0], ddx, fmaf(G[m][1], ddy, G[m][2] * ddz));
+          const float cJ = G1[m] * ir;                   // J_mk = ir (G_mk - l Y_m r_k)
+          const float cK = G2[m] * ir2;                  // K_mk = ir^2 [ ... ]
+          const float lY = l * Y[m];
+          const float rcoef = -cJ * lY + cK * (-l * gdm + l * (l + 2.f) * Y[m] * rd);
+          const float gcoef = cJ - cK * l * rd;
+          const float dcoef = -cK * lY;
+          g0 += gcoef * G[m][0] + cK * HD[m][0] + rcoef * rx + dcoef * ddx;
+          g1 += gcoef * G[m][1] + cK * HD[m][1] + rcoef * ry + dcoef * ddy;
+          g2 += gcoef * G[m][2] + cK * HD[m][2] + rcoef * rz + dcoef * ddz;
+        }
+        g0 = warp_sum(g0);
+        g1 = warp_sum(g1);
+        g2 = warp_sum(g2);
+        if (NSL == 1) {
+          if (lane == 0 && e >= 0) {
+            float* g = a.gvec + 3 * (int64_t)e;
+            g[0] = g0;
+            g[1] = g1;
+            g[2] = g2;
+          }
+        } else if (lane == 0) {
+          float* s = gslot + (((size_t)phase * 32 + k) * NSL + sl) * 4;
+          s[0] = g0;
+          s[1] = g1;
+          s[2] = g2;
+        }
+      }
+    }
+    if constexpr (GVEC && NSL > 1) {
+      named_barrier(1 + phase, 32 * NSL);
+      if (sl == 0 && lane < ne && my_e >= 0) {
+        float g0 = 0.f, g1 = 0.f, g2 = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < NSL; ++s2) {
+          const float* s = gslot + (((size_t)phase * 32 + lane) * NSL + s2) * 4;
+          g0 += s[0];
+          g1 += s[1];
+          g2 += s[2];
+        }
+        float* g = a.gvec + 3 * (int64_t)my_e;
+        g[0] = g0;
+        g[1] = g1;
+        g[2] = g2;
+      }
+      named_barrier(1 + phase, 32 * NSL);
+    }
+  }
+  reduce_phases(gx, smem, phase, st, lane, GVEC ? sl : 0, GVEC ? NSL : 1);
+  if (phase == 0 && act && a.gx) S::store_in(a.gx + (int64_t)node * a.in_dim, a.mul, c, gx);
+}
+
+// ---------------------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------------------
+template <class S>
+cudaError_t launch_fwd_uvu(const LaunchArgs& a, cudaStream_t s) {
+  if (a.N == 0) return cudaSuccess;
+  const size_t sm = (size_t)(a.split - 1) * S::OUT_PC * 32 * sizeof(float);
+  k_fwd_uvu<S><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <class S>
+cudaError_t launch_dbwd_recv(const LaunchArgs& a, cudaStream_t s) {
+  if (a.N == 0) return cudaSuccess;
+  const size_t sm = (size_t)(a.split - 1) * S::OUT_PC * 32 * sizeof(float);
+  k_dbwd_recv<S><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <class S, bool GVEC, int NSL>
+cudaError_t launch_sender_bwd(const LaunchArgs& a, cudaStream_t s) {
+  const int st = a.split;
+  const int groups = GVEC ? NSL : 1;
+  const size_t sm = (size_t)(st > 1 ? (st - 1) * groups * S::IN_PC * 32 : 0) * sizeof(float) +
+                    (GVEC && NSL > 1 ? (size_t)st * 32 * NSL * 4 * sizeof(float) : 0);
+  const unsigned grid = GVEC ? (unsigned)a.N : (unsigned)a.N * a.n_slices;
+  k_bwd_uvu<S, GVEC, NSL><<<grid, 32 * st * groups, sm, s>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <class S, bool GVEC, int NSL>
+cudaError_t launch_sender_dbwd(const LaunchArgs& a, cudaStream_t s) {
+  const int st = a.split;
+  const int groups = GVEC ? NSL : 1;
+  const size_t sm = (size_t)(st > 1 ? (st - 1) * groups * S::IN_PC * 32 : 0) * sizeof(float) +
+                    (GVEC && NSL > 1 ? (size_t)st * 32 * NSL * 4 * sizeof(float) : 0);
+  const unsigned grid = GVEC ? (unsigned)a.N : (unsigned)a.N * a.n_slices;
+  k_dbwd_send<S, GVEC, NSL><<<grid, 32 * st * groups, sm, s>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// The host chooses split so that split * NSL <= 4 whenever gvec is requested.
+template <class S>
+cudaError_t launch_bwd_uvu(const LaunchArgs& a, cudaStream_t s) {
+  if (a.N == 0) return cudaSuccess;
+  if (a.gvec == nullptr) return launch_sender_bwd<S, false, 1>(a, s);
+  if (a.n_slices <= 1) return launch_sender_bwd<S, true, 1>(a, s);
+  if (a.n_slices == 2) return launch_sender_bwd<S, true, 2>(a, s);
+  return launch_sender_bwd<S, true, 4>(a, s);
+}
+
+template <class S>
+cudaError_t launch_dbwd_send(const LaunchArgs& a, cudaStream_t s) {
+  if (a.N == 0) return cudaSuccess;
+  if (a.gvec == nullptr) return launch_sender_dbwd<S, false, 1>(a, s);
+  if (a.n_slices <= 1) return launch_sender_dbwd<S, true, 1>(a, s);
+  if (a.n_slices == 2) return launch_sender_dbwd<S, true, 2>(a, s);
+  return launch_sender_dbwd<S, true, 4>(a, s);
+}
+
+}  // namespace tp

@@ -1,0 +1,149 @@
+/*
+ * tp.h -- C ABI of the B200 edge-conditioned E(3)-equivariant tensor-product convolution.
+ *
+ * The operation ("Sobek: Streaming Equivariant Tensor Product Convolutions", abstract;
+ * "FlashTP: Fused, Sparsity-Aware Tensor Product for Machine Learning Interatomic
+ * Potentials", abstract; "The GPU Workload That Rewrites Molecular Physics", section
+ * "Equivariant feature transforms"): for every directed edge e = (j -> i) of a graph,
+ * couple the sender features x[j] with the real spherical harmonics Y(v_e / |v_e|) of the
+ * edge vector through the real Clebsch-Gordan tensor C_p of each path p = (in, sh, out),
+ * scale by the edge's radial weights and sum into the receiver:
+ *
+ *   y[i, out(p), w, m3] = sum_{e into i} sum_p sum_{m1,m2} C_p[m1,m2,m3] Y_sh(p)(v_e)[m2] X_pe[w,m1]
+ *     uvu mode: X_pe[u, m1] = c_p * w[e, p, u] * x[j, in(p), u, m1]
+ *     uvw mode: X_pe[w, m1] = c_p * s[e, p] * sum_u W[p, u, w] * x[j, in(p), u, m1]
+ *
+ * tp_conv_bwd returns the vector-Jacobian product against gy; tp_conv_dbwd the VJP of the
+ * backward map (x, vec, w, gy) -> (gx, gw, gvec) against (ggx, ggw, ggvec) ("Sobek",
+ * abstract: forward, backward and double backward).
+ *
+ * Conventions.  Real spherical harmonics, m = -l..l, component normalisation
+ * (sum_m Y_lm^2 = 2l+1, Y_0 = 1), no Condon-Shortley phase; l = 1 is sqrt(3)(y, z, x).  A
+ * zero edge vector has Y_0 = 1, Y_{l>0} = 0 and zero derivatives.  Real CG tensors have
+ * ||C||_F^2 = 2 l3 + 1 and a positive first non-zero entry in row-major (m1, m2, m3)
+ * order.  l <= 3 everywhere.
+ *
+ * Layouts (all row-major, fp32 unless noted, device memory):
+ *   x     [N, in_dim]   blocks in irreps order, inside a block [u][m] (m fastest)
+ *   y     [N, out_dim]  same rule on the output irreps
+ *   vec   [E, 3]        edge vector of edge e (any convention; the bench uses sender - receiver)
+ *   w     [E, P, mul]   uvu radial weights, paths outer, channel inner
+ *   s     [E, P]        uvw per-edge path scalars (passed as `w`)
+ *   W     [P, mul_in, mul_out]  uvw shared mixing matrices (NULL in uvu)
+ *   rowptr[N+1], src[E] int32: receiver-sorted CSR, edges of receiver i are
+ *                       rowptr[i] .. rowptr[i+1]-1 and src[e] is their sender
+ *   colptr[N+1], perm[E] int32: sender-sorted transpose, perm = stable argsort(src)
+ *
+ * Ownership.  The caller owns every buffer, including the workspace (size it with
+ * tp_workspace_size).  The library owns only the plan (host memory).  Inputs are read
+ * only; outputs are fully overwritten, never accumulated.
+ *
+ * Streams.  Every call only enqueues work on `stream` and returns; nothing synchronises
+ * except tp_get_device_error.
+ *
+ * Errors.  Host-side checks (null pointers, sizes, 4-byte alignment, irreps and path
+ * rules) return a status before any work is enqueued.  No C++ exception crosses the ABI.
+ * CUDA launch failures return TP_ERR_CUDA.  Kernels never trap: with TP_FLAG_CHECK_INDICES
+ * they bounds-check rowptr/src/perm, skip bad entries and record the first problem in the
+ * workspace error word, readable with tp_get_device_error; outputs are then unspecified.
+ * tp_last_error_message returns this thread's detail text of the last failing call.
+ */
+#ifndef TP_H_
+#define TP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* tp_stream_t; /* identical to cudaStream_t; NULL = legacy default stream */
+typedef struct tp_plan_s* tp_plan_t;
+
+typedef enum {
+  TP_OK = 0,
+  TP_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misalignment, bad irreps string */
+  TP_ERR_UNSUPPORTED = 2,  /* valid request this build has no kernel for (l > 3, ...) */
+  TP_ERR_BAD_GRAPH = 3,    /* inconsistent CSR found on the host (sizes) */
+  TP_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than tp_workspace_size */
+  TP_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
+  TP_ERR_TIMEOUT = 6       /* reserved: a bounded device wait gave up */
+} tp_status_t;
+
+enum { TP_MODE_UVU = 0, TP_MODE_UVW = 1 };
+enum { TP_FLAG_CHECK_INDICES = 1 };
+enum { TP_OP_FWD = 0, TP_OP_BWD = 1, TP_OP_DBWD = 2 };
+
+/* Builds a plan from irreps strings and a path list.
+ *   irreps_in/out: "32x0e+32x1o+32x2e" (mul x l parity); irreps_sh: "1x0e+1x1o+1x2e"
+ *   (multiplicity 1, parity (-1)^l).  paths: [n_paths][3] = (i_in, i_sh, i_out) block
+ *   indices; their order fixes the weight layout.  Rules: triangle |l1-l2| <= l3 <= l1+l2,
+ *   parity p3 = p1 * p2, uvu needs mul_in == mul_out.  path_coeff: NULL = all 1.0.
+ *   All blocks of irreps_in share one multiplicity, and of irreps_out too.
+ * Errors: TP_ERR_INVALID_ARG (syntax, rule violations), TP_ERR_UNSUPPORTED (no compiled
+ * specialisation for this path list: the build ships lmax 1/2/3 "all paths" lists and the
+ * 4-path lmax-1 list; or l > 3; or uvw on a list without a uvw kernel). */
+tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* irreps_sh,
+                           const char* irreps_out, const int32_t* paths, int32_t n_paths,
+                           int32_t mode, const double* path_coeff, uint32_t flags);
+tp_status_t tp_plan_destroy(tp_plan_t plan);
+
+/* Sizes of the plan: feature widths, per-edge weights per edge, shared uvw weights. */
+tp_status_t tp_plan_query(tp_plan_t plan, int64_t* in_dim, int64_t* out_dim,
+                          int64_t* n_edge_weights, int64_t* n_shared_weights);
+
+/* Bytes of device workspace a call of kind op (TP_OP_*) needs for N nodes and E edges:
+ * forward 0 (256 with TP_FLAG_CHECK_INDICES, for the error word); backward and double
+ * backward 256 + int32 colptr[N+1], counts[N], perm[E], tmp[E] (room to build the
+ * transpose in place; only the 256-byte header is used when colptr/perm are given).
+ * The workspace never holds an edge x feature float tensor. */
+tp_status_t tp_workspace_size(tp_plan_t plan, int64_t N, int64_t E, int32_t op, size_t* bytes);
+
+/* Stable receiver->sender transpose: colptr[N+1] = exclusive scan of bincount(src),
+ * perm[E] = stable argsort of src (bit exact).  rowptr may be NULL.  Workspace: at least
+ * tp_workspace_size(., N, E, TP_OP_BWD) bytes or 4*(N+E)+256. */
+tp_status_t tp_csr_transpose(int64_t N, int64_t E, const int32_t* rowptr, const int32_t* src,
+                             int32_t* colptr, int32_t* perm, void* ws, size_t ws_bytes,
+                             tp_stream_t stream);
+
+/* Forward: y[N, out_dim].  W is NULL in uvu mode. */
+tp_status_t tp_conv_fwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* rowptr,
+                        const int32_t* src, const float* x, const float* vec, const float* w,
+                        const float* W, float* y, void* ws, size_t ws_bytes, tp_stream_t stream);
+
+/* Backward against gy[N, out_dim].  colptr/perm: a transpose from tp_csr_transpose, or both
+ * NULL to have it built in the workspace.  Outputs gx[N, in_dim], gw[E, nw] (uvu w or uvw
+ * s), gvec[E, 3], gW[P, mul_in, mul_out] (uvw); each NULL output is skipped. */
+tp_status_t tp_conv_bwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* rowptr,
+                        const int32_t* src, const int32_t* colptr, const int32_t* perm,
+                        const float* x, const float* vec, const float* w, const float* W,
+                        const float* gy, float* gx, float* gw, float* gvec, float* gW, void* ws,
+                        size_t ws_bytes, tp_stream_t stream);
+
+/* Double backward (uvu): inputs ggx[N, in_dim], ggw[E, nw], ggvec[E, 3], each NULL = zero;
+ * outputs g_gy[N, out_dim], g_x[N, in_dim], g_w[E, nw], g_vec[E, 3], each NULL = skipped. */
+tp_status_t tp_conv_dbwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* rowptr,
+                         const int32_t* src, const int32_t* colptr, const int32_t* perm,
+                         const float* x, const float* vec, const float* w, const float* W,
+                         const float* gy, const float* ggx, const float* ggw, const float* ggvec,
+                         float* g_gy, float* g_x, float* g_w, float* g_vec, void* ws,
+                         size_t ws_bytes, tp_stream_t stream);
+
+/* Reads (and clears) the device error word of a workspace after the work on `stream`
+ * finished; synchronises the stream.  *code: 0 = none, 1 = bad rowptr, 2 = bad src,
+ * 3 = bad perm / transpose entry. */
+tp_status_t tp_get_device_error(tp_plan_t plan, void* ws, tp_stream_t stream, int32_t* code);
+
+/* Number of kernels this library has launched in the calling process (diagnostics: lets a
+ * benchmark count its own launches in a timed region). */
+int64_t tp_launch_count(void);
+
+const char* tp_status_string(tp_status_t status);
+const char* tp_last_error_message(void);
+const char* tp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TP_H_ */

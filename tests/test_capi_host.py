@@ -1,0 +1,148 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol
+include/tp.h declares, and rejects bad plans and bad calls with the documented status
+before touching the device."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from equivariant_tensor_product_b200 import build
+    build.build()
+    from equivariant_tensor_product_b200 import _lib
+    return _lib.load()
+
+
+@pytest.fixture(scope="module")
+def tp(lib):
+    import equivariant_tensor_product_b200 as tp
+    return tp
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "tp.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tp_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    out = os.popen(f"nm -D --defined-only {os.path.join(ROOT, 'equivariant_tensor_product_b200', 'libtp.so')}").read()
+    for n in names:
+        assert re.search(rf"\bT {n}\b", out), f"{n} not exported as a text symbol"
+
+
+def test_version_and_status_strings(lib):
+    assert b"sm_100a" in lib.tp_version()
+    assert lib.tp_status_string(0) == b"ok"
+    assert lib.tp_status_string(4) == b"workspace too small"
+
+
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", pytest.param("c4", marks=pytest.mark.xfail(
+    reason="uvw kernels not built yet", strict=False)), "c5"])
+def test_plan_matches_config_sizes(tp, name):
+    spec = synth.CONFIGS[name]
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, spec.mode)
+    assert plan.in_dim == synth.irreps_dim(spec.irreps_in)
+    assert plan.out_dim == synth.irreps_dim(spec.irreps_out)
+    assert plan.n_edge_weights == synth.n_edge_weights(spec)
+    if spec.mode == "uvw":
+        P, U, V = synth.shared_weight_shape(spec)
+        assert plan.n_shared_weights == P * U * V
+
+
+@pytest.mark.parametrize("args,status", [
+    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 0, 0), (0, 1, 1), (1, 0, 1), (1, 1, 0)]), 0),
+    (("4x0e+4x1q", "1x0e+1x1o", "4x0e+4x1o", [(0, 0, 0)]), 1),          # bad parity letter
+    (("4x0e+", "1x0e", "4x0e", [(0, 0, 0)]), 1),                           # trailing +
+    (("0x0e", "1x0e", "4x0e", [(0, 0, 0)]), 1),                            # zero multiplicity
+    (("4x4e", "1x0e", "4x4e", [(0, 0, 0)]), 2),                            # l > 3
+    (("4x0e+4x1o", "1x0e+1x1e", "4x0e+4x1o", [(0, 0, 0)]), 1),          # SH parity
+    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 1, 0)]), 1),          # triangle
+    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(1, 1, 1)]), 1),          # parity 1o x 1o -> 1o
+    (("4x0e+4x1o", "1x0e+1x1o", "8x0e+8x1o", [(0, 0, 0)]), 1),          # uvu multiplicity
+    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 0, 0)]), 2),          # valid, not compiled
+    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 0, 2)]), 1),          # index out of range
+])
+def test_plan_validation(tp, args, status):
+    if status == 0:
+        tp.Plan(*args)
+        return
+    with pytest.raises(tp.TPError) as ei:
+        tp.Plan(*args)
+    assert ei.value.status == status, str(ei.value)
+
+
+def test_path_coeff_rejects_nan(tp):
+    spec = synth.CONFIGS["c1"]
+    with pytest.raises(tp.TPError):
+        tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvu",
+                path_coeff=[1.0, float("nan"), 1.0, 1.0])
+
+
+def test_workspace_contract(tp):
+    spec = synth.CONFIGS["c2"]
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths)
+    N, E = 1536, 46080
+    assert tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD) == 0
+    for op in (tp.TP_OP_BWD, tp.TP_OP_DBWD):
+        b = tp.tp_workspace_size(plan, N, E, op)
+        # int32 graph indices only: at most 8 bytes per edge + O(N) + alignment
+        assert 8 * E <= b <= 8 * E + 8 * (N + 1) + 6 * 256
+
+
+def test_calls_reject_bad_arguments_before_the_device(lib, tp):
+    spec = synth.CONFIGS["c1"]
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths)
+    h = plan.handle
+    fake = C.c_void_p(0x10000)     # never dereferenced: every call below fails host checks
+    odd = C.c_void_p(0x10002)
+    # null plan
+    assert lib.tp_conv_fwd(None, 4, 8, fake, fake, fake, fake, fake, None, fake, None, 0, None) == 1
+    # negative sizes
+    assert lib.tp_conv_fwd(h, -1, 8, fake, fake, fake, fake, fake, None, fake, None, 0, None) == 1
+    # null output
+    assert lib.tp_conv_fwd(h, 4, 8, fake, fake, fake, fake, fake, None, None, None, 0, None) == 1
+    # null edge inputs with E > 0
+    assert lib.tp_conv_fwd(h, 4, 8, fake, None, fake, fake, fake, None, fake, None, 0, None) == 1
+    # misaligned pointer
+    assert lib.tp_conv_fwd(h, 4, 8, fake, fake, odd, fake, fake, None, fake, None, 0, None) == 1
+    # N = 0 is a no-op
+    assert lib.tp_conv_fwd(h, 0, 0, None, None, None, None, None, None, None, None, 0, None) == 0
+    # backward: workspace too small
+    st = lib.tp_conv_bwd(h, 4, 8, fake, fake, None, None, fake, fake, fake, None, fake, fake, fake, None, None,
+                         fake, 16, None)
+    assert st == 4
+    # colptr without perm
+    st = lib.tp_conv_bwd(h, 4, 8, fake, fake, fake, None, fake, fake, fake, None, fake, fake, fake, None, None,
+                         fake, 1 << 20, None)
+    assert st == 1
+    # transpose: null outputs
+    assert lib.tp_csr_transpose(4, 8, None, fake, None, fake, fake, 1 << 20, None) == 1
+    msg = lib.tp_last_error_message()
+    assert msg and b"null" in msg.lower()
+    # over int32 range
+    assert lib.tp_conv_fwd(h, 1 << 31, 8, fake, fake, fake, fake, fake, None, fake, None, 0, None) == 2
+
+
+def test_no_cpu_fallback_without_device(lib, tp):
+    """A call that passes host checks goes to CUDA; with no device it fails loudly."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("device present")
+    spec = synth.CONFIGS["c1"]
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, flags=tp.TP_FLAG_CHECK_INDICES)
+    fake = C.c_void_p(0x10000)
+    st = lib.tp_conv_fwd(plan.handle, 4, 8, fake, fake, fake, fake, fake, None, fake, fake, 256, None)
+    assert st == 5
+    assert b"cuda" in lib.tp_last_error_message().lower() or lib.tp_last_error_message()
