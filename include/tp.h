@@ -107,6 +107,23 @@ tp_status_t tp_csr_transpose(int64_t N, int64_t E, const int32_t* rowptr, const 
                              int32_t* colptr, int32_t* perm, void* ws, size_t ws_bytes,
                              tp_stream_t stream);
 
+/* Same result as tp_csr_transpose (bit for bit), for callers that cannot allocate device
+ * memory -- e.g. an MD engine whose device memory is owned by a pool it does not control,
+ * a framework that has reserved nearly all of the GPU up front, or a loop that must avoid
+ * cudaMalloc/cudaFree because they synchronise the device.  It takes no workspace: its
+ * scratch (per-sender counters and the scatter buffer) is a fixed int32 array inside the
+ * library (about 4.5 MB, held on every GPU that loads the library until exit).  The source
+ * pages have no counterpart; this is an interface convenience.
+ *   Limits: N <= 131072 and E <= 1048576, else TP_ERR_UNSUPPORTED with nothing enqueued.
+ *   Calls share the array: calls whose work overlaps on the GPU race; order them on one
+ *   stream.  Counters are cleared at the start of every call.  The first call on a device
+ *   looks up the array's device address with that device current: make it before any
+ *   stream capture.  Other errors: TP_ERR_INVALID_ARG (null, misaligned, negative sizes),
+ *   TP_ERR_CUDA.  No message is set for tp_last_error_message. */
+tp_status_t tp_csr_transpose_noalloc(int64_t N, int64_t E, const int32_t* rowptr,
+                                     const int32_t* src, int32_t* colptr, int32_t* perm,
+                                     tp_stream_t stream);
+
 /* Forward: y[N, out_dim].  W is NULL in uvu mode. */
 tp_status_t tp_conv_fwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* rowptr,
                         const int32_t* src, const float* x, const float* vec, const float* w,
