@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <string>
@@ -128,6 +129,38 @@ WsLayout ws_layout(int64_t N, int64_t E) {
   return L;
 }
 
+// Tuning override read once from the environment: TP_TUNE_PREFETCH=0/1 forces the register
+// double buffering of edge gathers off/on (default: per-spec heuristic).
+int tune_prefetch() {
+  static const int v = [] {
+    const char* e = std::getenv("TP_TUNE_PREFETCH");
+    return (e && (e[0] == '0' || e[0] == '1')) ? e[0] - '0' : -1;
+  }();
+  return v;
+}
+
+// uvw regions after the transpose region: A | G | Wt | part (floats, 256-byte aligned)
+constexpr int kUvwSplits = 64;
+struct UvwLayout {
+  size_t A, G, Wt, part, total;
+};
+UvwLayout uvw_layout(tp_plan_t plan, int64_t N, int64_t E, bool bwd) {
+  UvwLayout U{};
+  size_t off = bwd ? ws_layout(N, E).total : 256;
+  const size_t a_bytes = sizeof(float) * (size_t)N * plan->ops->A_PC * plan->mul_in;
+  const size_t w_bytes = sizeof(float) * (size_t)plan->n_shared;
+  U.A = off;
+  off += align256(a_bytes > 0 ? a_bytes : 1);
+  U.G = off;
+  if (bwd) off += align256(a_bytes > 0 ? a_bytes : 1);
+  U.Wt = off;
+  off += align256(w_bytes);
+  U.part = off;
+  if (bwd) off += align256(w_bytes * kUvwSplits);
+  U.total = off;
+  return U;
+}
+
 int pick_split(int64_t N, int64_t E) {
   if (N <= 0) return 1;
   const double avg = (double)E / (double)N;
@@ -160,6 +193,7 @@ LaunchArgs base_args(tp_plan_t plan, int64_t N, int64_t E) {
   a.n_slices = (plan->mul_in + 31) / 32;
   a.has_coeff = plan->has_coeff;
   a.check = (plan->flags & TP_FLAG_CHECK_INDICES) ? 1 : 0;
+  a.prefetch = tune_prefetch();
   std::memcpy(a.coeff, plan->coeff, sizeof(a.coeff));
   return a;
 }
@@ -260,7 +294,7 @@ tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* i
     return fail(TP_ERR_UNSUPPORTED,
                 "no compiled specialisation for this irreps/path list (shipped: all-paths lmax 1/2/3 "
                 "and the 4-path lmax-1 list)");
-  if (mode == TP_MODE_UVW && (!found->uvw_edge || !found->uvw_bwd))
+  if (mode == TP_MODE_UVW && (!found->uvw_fwd || !found->uvw_bwd))
     return fail(TP_ERR_UNSUPPORTED, "spec '%s' has no uvw kernels", found->name);
   tp_plan_s* pl = new (std::nothrow) tp_plan_s;
   if (!pl) return fail(TP_ERR_INVALID_ARG, "out of host memory");
@@ -315,8 +349,14 @@ tp_status_t tp_workspace_size(tp_plan_t plan, int64_t N, int64_t E, int32_t op, 
   if (!bytes) return fail(TP_ERR_INVALID_ARG, "bytes is NULL");
   if (op != TP_OP_FWD && op != TP_OP_BWD && op != TP_OP_DBWD) return fail(TP_ERR_INVALID_ARG, "bad op");
   size_t need = 0;
-  if (op == TP_OP_FWD) need = (plan->flags & TP_FLAG_CHECK_INDICES) ? 256 : 0;
-  else need = ws_layout(N, E).total;   // enough to build the transpose in place
+  if (plan->mode == TP_MODE_UVW) {
+    if (op == TP_OP_DBWD) return fail(TP_ERR_UNSUPPORTED, "double backward is implemented for uvu");
+    need = uvw_layout(plan, N, E, op == TP_OP_BWD).total;
+  } else if (op == TP_OP_FWD) {
+    need = (plan->flags & TP_FLAG_CHECK_INDICES) ? 256 : 0;
+  } else {
+    need = ws_layout(N, E).total;   // enough to build the transpose in place
+  }
   *bytes = need;
   return TP_OK;
 }
@@ -366,8 +406,18 @@ tp_status_t tp_conv_fwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* row
   a.vec = vec;
   a.w = w;
   a.y = y;
-  if (plan->mode != TP_MODE_UVU) return fail(TP_ERR_UNSUPPORTED, "uvw forward not available");
-  cudaError_t e = plan->ops->fwd_uvu(a, s);
+  cudaError_t e;
+  if (plan->mode == TP_MODE_UVW) {
+    const UvwLayout U = uvw_layout(plan, N, E, false);
+    char* wsb = static_cast<char*>(ws);
+    a.W = W;
+    a.A = reinterpret_cast<float*>(wsb + U.A);
+    a.Wt = reinterpret_cast<float*>(wsb + U.Wt);
+    a.nw = plan->n_paths;
+    e = plan->ops->uvw_fwd(a, s);
+  } else {
+    e = plan->ops->fwd_uvu(a, s);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "tp_conv_fwd launch");
   return TP_OK;
 }
@@ -409,13 +459,16 @@ tp_status_t tp_conv_bwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* row
                         (const void*)x, (const void*)vec, (const void*)w, (const void*)W, (const void*)gy,
                         (const void*)gx, (const void*)gw, (const void*)gvec, (const void*)gW})
     if (!aligned4(p)) return fail(TP_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
-  if (plan->mode != TP_MODE_UVU) return fail(TP_ERR_UNSUPPORTED, "uvw backward not available");
-  (void)gW;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   LaunchArgs a = base_args(plan, N, E);
   st = debug_prologue(plan, N, E, rowptr, src, ws, s, &a.err);
   if (st != TP_OK) return st;
-  if (!gx && !gw && !gvec) return TP_OK;
+  if (!gx && !gw && !gvec && !gW) return TP_OK;
+  if (plan->mode == TP_MODE_UVW) {
+    size_t need = 0;
+    tp_workspace_size(plan, N, E, TP_OP_BWD, &need);
+    if (!ws || ws_bytes < need) return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  }
   st = sender_order(N, E, src, colptr, perm, ws, ws_bytes, s);
   if (st != TP_OK) return st;
   a.rowptr = rowptr;
@@ -429,6 +482,21 @@ tp_status_t tp_conv_bwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* row
   a.gx = gx;
   a.gw = gw;
   a.gvec = gvec;
+  if (plan->mode == TP_MODE_UVW) {
+    const UvwLayout U = uvw_layout(plan, N, E, true);
+    char* wsb = static_cast<char*>(ws);
+    a.W = W;
+    a.A = reinterpret_cast<float*>(wsb + U.A);
+    a.G = reinterpret_cast<float*>(wsb + U.G);
+    a.Wt = reinterpret_cast<float*>(wsb + U.Wt);
+    a.part = reinterpret_cast<float*>(wsb + U.part);
+    a.splits = kUvwSplits;
+    a.gW = gW;
+    a.nw = plan->n_paths;
+    cudaError_t e = plan->ops->uvw_bwd(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tp_conv_bwd (uvw) launch");
+    return TP_OK;
+  }
   if (gvec) {
     const int nsl = a.n_slices <= 1 ? 1 : (a.n_slices == 2 ? 2 : 4);
     while (a.split * nsl > 4) a.split >>= 1;

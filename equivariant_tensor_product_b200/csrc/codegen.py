@@ -616,6 +616,53 @@ def _gen_uvw_bwd(spec: Spec) -> List[str]:
     return L
 
 
+def _uvw_tables(spec: Spec):
+    """Per output irrep o: paths into o (in path order), d3, count, and the per-(node, channel)
+    offset of its region in the uvw node state A (regions in output order)."""
+    outs = []
+    cum = 0
+    for o, l3 in enumerate(spec.out_ls):
+        plist = [p for p, path in enumerate(spec.paths) if path[2] == o]
+        d3 = 2 * l3 + 1
+        outs.append(dict(o=o, d3=d3, paths=plist, cnt=len(plist), cumA=cum))
+        cum += d3 * len(plist)
+    assert cum == spec.A_PC
+    return outs
+
+
+def _gen_uvw_layout(spec: Spec) -> List[str]:
+    outs = _uvw_tables(spec)
+    n = len(outs)
+    maxc = max(1, max(t["cnt"] for t in outs))
+    L = [f"  static constexpr int N_OUT = {n};",
+         f"  static constexpr int MAX_CNT = {maxc};"]
+    for name, vals in (("out_d3_at", [t["d3"] for t in outs]), ("out_cnt_at", [t["cnt"] for t in outs]),
+                       ("out_cumA_at", [t["cumA"] for t in outs]), ("out_cumY_at", list(spec.out_cum))):
+        L.append(f"  __host__ __device__ static int {name}(int o) {{ constexpr int v[{n}] = "
+                 f"{{{', '.join(map(str, vals))}}}; return v[o]; }}")
+    flat = []
+    for t in outs:
+        flat += t["paths"] + [-1] * (maxc - t["cnt"])
+    L.append(f"  __host__ __device__ static int path_of_at(int o, int pl) {{ constexpr int v[{n * maxc}] = "
+             f"{{{', '.join(map(str, flat))}}}; return v[o * {maxc} + pl]; }}")
+    # store / load of one channel's per-path state, [N*mul*cumA_o] + ((i*d3+m3)*cnt + pl)*mul + c
+    for name, const, arr in (("store_uvw", False, "a"), ("load_uvw", True, "a")):
+        sig = (f"  __device__ __forceinline__ static void {name}({'const ' if const else ''}float* __restrict__ base, "
+               f"int64_t N, int mul, int64_t i, int c, {'float' if const else 'const float'} (&{arr})[{spec.A_PC}]) {{")
+        L.append(sig)
+        for t in outs:
+            for pl, p in enumerate(t["paths"]):
+                for m3 in range(t["d3"]):
+                    idx = (f"N * mul * {t['cumA']} + ((i * {t['d3']} + {m3}) * {t['cnt']} + {pl}) * (int64_t)mul + c")
+                    k = spec.a_cum[p] + m3
+                    if const:
+                        L.append(f"    {arr}[{k}] = __ldg(base + {idx});")
+                    else:
+                        L.append(f"    base[{idx}] = {arr}[{k}];")
+        L.append("  }")
+    return L
+
+
 def gen_spec_header(spec: Spec) -> str:
     L = [f"// Generated by codegen.py for spec '{spec.name}'.  Do not edit.",
          f"// inputs l={spec.in_ls}  SH l={spec.sh_ls}  outputs l={spec.out_ls}",
@@ -644,6 +691,7 @@ def gen_spec_header(spec: Spec) -> str:
     L += _gen_dbwd_recv(spec)
     L += _gen_dbwd_send(spec)
     L += _gen_uvw_bwd(spec)
+    L += _gen_uvw_layout(spec)
     L.append("};")
     return "\n".join(L) + "\n"
 
@@ -700,8 +748,9 @@ PARTS = {
     "fwd": [("fwd_uvu", "launch_fwd_uvu")],
     "bwd": [("bwd_uvu", "launch_bwd_uvu")],
     "dbwd": [("dbwd_recv", "launch_dbwd_recv"), ("dbwd_send", "launch_dbwd_send")],
+    "uvw": [("uvw_fwd", "launch_uvw_fwd"), ("uvw_bwd", "launch_uvw_bwd")],
 }
-SLOTS = ["fwd_uvu", "bwd_uvu", "dbwd_recv", "dbwd_send", "uvw_edge", "uvw_bwd"]
+SLOTS = ["fwd_uvu", "bwd_uvu", "dbwd_recv", "dbwd_send", "uvw_fwd", "uvw_bwd"]
 
 
 def main(outdir: str):
@@ -720,8 +769,9 @@ def main(outdir: str):
     for s in specs:
         write(f"spec_{s.name}.h", gen_spec_header(s))
         for part, fns in PARTS.items():
+            inc = "tp_uvw.cuh" if part == "uvw" else "tp_kernels.cuh"
             body = [f"// Generated by codegen.py: {part} kernels of spec '{s.name}'.",
-                    '#include "tp_kernels.cuh"', f'#include "spec_{s.name}.h"', "namespace tp {"]
+                    f'#include "{inc}"', f'#include "spec_{s.name}.h"', "namespace tp {"]
             for slot, tmpl in fns:
                 body.append(f"cudaError_t {s.name}_{slot}(const LaunchArgs& a, cudaStream_t st) "
                             f"{{ return {tmpl}<Spec_{s.name}>(a, st); }}")

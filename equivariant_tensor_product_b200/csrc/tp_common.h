@@ -28,6 +28,7 @@ struct LaunchArgs {
   int n_slices;        // 32-channel slices per row = ceil(mul / 32)
   int has_coeff;       // path coefficients differ from 1
   int check;           // bounds-check indices and report through *err
+  int prefetch;        // -1: heuristic; 0/1: force register double-buffering of edge gathers
   const int32_t* rowptr;
   const int32_t* src;
   const int32_t* colptr;
@@ -39,8 +40,14 @@ struct LaunchArgs {
   const float* ggx;
   const float* ggw;
   const float* ggvec;
-  const float* G;       // uvw: gradient of the per-path node state A
-  float* y;             // fwd output / dbwd g_gy / uvw A
+  const float* W;       // uvw: shared mixing matrices [P][mul][mul_out]
+  float* A;             // uvw: per-path node state (workspace), layout of S::store_uvw
+  float* G;             // uvw: gradient of A (workspace), same layout
+  float* Wt;            // uvw: W regrouped per output irrep, [o][w][pl*mul + u] (workspace)
+  float* gW;            // uvw: gradient of W (output)
+  float* part;          // uvw: split-K partials of gW (workspace)
+  int splits;           // uvw: number of split-K partials
+  float* y;             // fwd output / dbwd g_gy
   float* gx;
   float* gw;
   float* gvec;
@@ -65,8 +72,8 @@ struct SpecOps {
   LaunchFn bwd_uvu;         // gx, gw (gvec when args.gvec != nullptr), sender order
   LaunchFn dbwd_recv;       // g_gy, receiver order
   LaunchFn dbwd_send;       // g_x, g_w, g_vec, sender order
-  LaunchFn uvw_edge;        // A[i, p, u, m3] aggregated per path (uvw forward edge pass)
-  LaunchFn uvw_bwd;         // gx, gs (gvec) from G = dA, sender order
+  LaunchFn uvw_fwd;         // edge pass into A, then y = mix(A, W)
+  LaunchFn uvw_bwd;         // A again, G = W gy, gW = A^T gy, then the sender pass for gx, gs, gvec
 };
 
 extern const SpecOps* const kRegistry[];

@@ -109,7 +109,7 @@ __device__ __forceinline__ void reduce_phases(float (&acc)[N], float* smem, int 
 // ---------------------------------------------------------------------------------------
 // Forward, uvu, receiver order.  grid = N * n_slices, block = 32 * split.
 // ---------------------------------------------------------------------------------------
-template <class S>
+template <class S, bool PF>
 __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__ LaunchArgs a) {
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
@@ -144,23 +144,43 @@ __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__
       }
     }
     const int ne = min(32, (e1 - base + st - 1) / st);
-    for (int k = 0; k < ne; ++k) {
-      const int e = base + k * st;
+    // gathers of edge k: sender slice x[j] and the edge's weight row
+    auto fetch = [&](int k, float (&xx)[S::IN_PC], float (&ww)[S::P]) {
+      const int j = __shfl_sync(kFull, my_j, k);
+      if (act && j >= 0) {
+        S::load_in(a.x + (int64_t)j * a.in_dim, a.mul, c, xx);
+        load_path_weights(a, base + k * st, c, ww);
+      }
+    };
+    auto compute = [&](int k, const float (&xx)[S::IN_PC], const float (&ww)[S::P]) {
       const int j = __shfl_sync(kFull, my_j, k);
       const float ux = __shfl_sync(kFull, vx, k);
       const float uy = __shfl_sync(kFull, vy, k);
       const float uz = __shfl_sync(kFull, vz, k);
-      if (j < 0) continue;
+      if (j < 0) return;
       float rx, ry, rz, ir;
       edge_geometry(ux, uy, uz, rx, ry, rz, ir);
       float Y[S::NSH];
       S::sh(rx, ry, rz, Y);
-      if (act) {
-        float x[S::IN_PC];
-        S::load_in(a.x + (int64_t)j * a.in_dim, a.mul, c, x);
-        float w[S::P];
-        load_path_weights(a, e, c, w);
-        S::fwd(x, Y, w, acc);
+      if (act) S::fwd(xx, Y, ww, acc);
+    };
+    float xa[S::IN_PC], wa[S::P];
+    if constexpr (PF) {
+      // two register buffers: the gathers of edge k+1 are in flight while edge k computes
+      float xb[S::IN_PC], wb[S::P];
+      fetch(0, xa, wa);
+      for (int k = 0; k < ne; k += 2) {
+        if (k + 1 < ne) fetch(k + 1, xb, wb);
+        compute(k, xa, wa);
+        if (k + 1 >= ne) break;
+        if (k + 2 < ne) fetch(k + 2, xa, wa);
+        compute(k + 1, xb, wb);
+      }
+    } else {
+#pragma unroll 1
+      for (int k = 0; k < ne; ++k) {
+        fetch(k, xa, wa);
+        compute(k, xa, wa);
       }
     }
   }
@@ -177,7 +197,7 @@ __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__
 // GVEC=false: grid = N * n_slices, block = 32*split (slices independent).
 // GVEC=true : grid = N, block = 32*split*NSL (all slices of a row in one CTA).
 // ---------------------------------------------------------------------------------------
-template <class S, bool GVEC, int NSL>
+template <class S, bool GVEC, int NSL, bool PF>
 __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__ LaunchArgs a) {
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
@@ -229,9 +249,17 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
       }
     }
     const int ne = min(32, (q1 - base + st - 1) / st);
-    for (int k = 0; k < ne; ++k) {
+    // gathers of edge k: receiver slice gy[i] and the edge's weight row
+    auto fetch = [&](int k, float (&gg)[S::OUT_PC], float (&ww)[S::P]) {
       const int e = __shfl_sync(kFull, my_e, k);
       const int i = __shfl_sync(kFull, my_i, k);
+      if (act && e >= 0) {
+        S::load_out(a.gy + (int64_t)i * a.out_dim, a.mul, c, gg);
+        load_path_weights(a, e, c, ww);
+      }
+    };
+    auto compute = [&](int k, const float (&gyv)[S::OUT_PC], const float (&w)[S::P]) {
+      const int e = __shfl_sync(kFull, my_e, k);
       const float ux = __shfl_sync(kFull, vx, k);
       const float uy = __shfl_sync(kFull, vy, k);
       const float uz = __shfl_sync(kFull, vz, k);
@@ -243,10 +271,6 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
 #pragma unroll
       for (int m = 0; m < S::NSH; ++m) gY[m] = 0.f;
       if (act && e >= 0) {
-        float gyv[S::OUT_PC];
-        S::load_out(a.gy + (int64_t)i * a.out_dim, a.mul, c, gyv);
-        float w[S::P];
-        load_path_weights(a, e, c, w);
         float gw[S::P];
         S::template bwd<GVEC>(x, Y, w, gyv, gx, gw, gY);
         if (a.gw) {
@@ -285,6 +309,24 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
           s[2] = h2;
           s[3] = sdeg;
         }
+      }
+    };
+    float ga[S::OUT_PC], wa[S::P];
+    if constexpr (PF) {
+      float gb[S::OUT_PC], wb[S::P];
+      fetch(0, ga, wa);
+      for (int k = 0; k < ne; k += 2) {
+        if (k + 1 < ne) fetch(k + 1, gb, wb);
+        compute(k, ga, wa);
+        if (k + 1 >= ne) break;
+        if (k + 2 < ne) fetch(k + 2, ga, wa);
+        compute(k + 1, gb, wb);
+      }
+    } else {
+#pragma unroll 1
+      for (int k = 0; k < ne; ++k) {
+        fetch(k, ga, wa);
+        compute(k, ga, wa);
       }
     }
     if constexpr (GVEC && NSL > 1) {
@@ -560,11 +602,23 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant
 // ---------------------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------------------
+// Register double buffering of the per-edge gathers pays when the buffers are small (lmax
+// <= 2); for lmax 3 the extra registers cost more occupancy than the overlap gains.
+// a.prefetch: -1 = this heuristic, 0/1 = forced (tuning override).
+template <class S>
+inline bool use_prefetch(const LaunchArgs& a) {
+  if (a.prefetch >= 0) return a.prefetch != 0;
+  return S::IN_PC + S::P + S::OUT_PC <= 48;
+}
+
 template <class S>
 cudaError_t launch_fwd_uvu(const LaunchArgs& a, cudaStream_t s) {
   if (a.N == 0) return cudaSuccess;
   const size_t sm = (size_t)(a.split - 1) * S::OUT_PC * 32 * sizeof(float);
-  k_fwd_uvu<S><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
+  if (use_prefetch<S>(a))
+    k_fwd_uvu<S, true><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
+  else
+    k_fwd_uvu<S, false><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -585,7 +639,10 @@ cudaError_t launch_sender_bwd(const LaunchArgs& a, cudaStream_t s) {
   const size_t sm = (size_t)(st > 1 ? (st - 1) * groups * S::IN_PC * 32 : 0) * sizeof(float) +
                     (GVEC && NSL > 1 ? (size_t)st * 32 * NSL * 4 * sizeof(float) : 0);
   const unsigned grid = GVEC ? (unsigned)a.N : (unsigned)a.N * a.n_slices;
-  k_bwd_uvu<S, GVEC, NSL><<<grid, 32 * st * groups, sm, s>>>(a);
+  if (use_prefetch<S>(a))
+    k_bwd_uvu<S, GVEC, NSL, true><<<grid, 32 * st * groups, sm, s>>>(a);
+  else
+    k_bwd_uvu<S, GVEC, NSL, false><<<grid, 32 * st * groups, sm, s>>>(a);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -48,8 +48,7 @@ def test_version_and_status_strings(lib):
     assert lib.tp_status_string(4) == b"workspace too small"
 
 
-@pytest.mark.parametrize("name", ["c1", "c2", "c3", pytest.param("c4", marks=pytest.mark.xfail(
-    reason="uvw kernels not built yet", strict=False)), "c5"])
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5"])
 def test_plan_matches_config_sizes(tp, name):
     spec = synth.CONFIGS[name]
     plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, spec.mode)
@@ -99,6 +98,20 @@ def test_workspace_contract(tp):
         b = tp.tp_workspace_size(plan, N, E, op)
         # int32 graph indices only: at most 8 bytes per edge + O(N) + alignment
         assert 8 * E <= b <= 8 * E + 8 * (N + 1) + 6 * 256
+
+
+def test_uvw_workspace_is_node_sized(tp):
+    spec = synth.CONFIGS["c4"]
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvw")
+    N, E = 100_000, 3_001_138
+    a_bytes = 4 * N * 51 * 128                   # per-path node state A (and its gradient G)
+    f = tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD)
+    b = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD)
+    assert a_bytes <= f <= a_bytes + plan.n_shared_weights * 4 + 4096
+    # bwd: transpose ints (8 bytes/edge + O(N)), A, G, W regrouped, 64 split-K partials of gW
+    assert b <= 8 * E + 12 * (N + 1) + 2 * a_bytes + 65 * 4 * plan.n_shared_weights + 16 * 256
+    with pytest.raises(tp.TPError):
+        tp.tp_workspace_size(plan, N, E, tp.TP_OP_DBWD)
 
 
 def test_calls_reject_bad_arguments_before_the_device(lib, tp):
