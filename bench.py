@@ -37,6 +37,8 @@ WORKLOADS = {
           "step = fwd + transpose + bwd(gx, gw)",
     "c5": "skewed degree 3-120: 8,192 atoms, ~295k edges, 32x(0e,1o,2e,3o), SH lmax 3, uvu, 34 paths; "
           "step = fwd + transpose + bwd(gx, gw, gvec)",
+    "c4": "large streaming uvw: 100,000 atoms, ~3.0M edges, 128x(0e,1o,2e) -> 128x(0e,1e,1o,2e,2o), SH lmax 2, "
+          "per-path 128x128 mixing, 15 paths; step = fwd + transpose + bwd(gx, gs, gW)",
 }
 
 
@@ -251,7 +253,9 @@ def run_ours(args, rank, world, local):
     in_dim, out_dim, nw = plan.in_dim, plan.out_dim, plan.n_edge_weights
     want_gvec = "dbwd" in spec.passes or args.workload == "c5"
 
-    keys = ["rowptr", "src", "x", "vec", "w", "gy"]
+    uvw = spec.mode == "uvw"
+    wkey = "s" if uvw else "w"
+    keys = ["rowptr", "src", "x", "vec", wkey, "gy"] + (["W"] if uvw else [])
     copy_bytes = sum(d[k].nbytes for k in keys)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     R = max(2, math.ceil(2.5 * l2 / copy_bytes))
@@ -264,51 +268,73 @@ def run_ours(args, rank, world, local):
             src_d = dict(d)
             src_d["x"] = rng.standard_normal(d["x"].shape, dtype=np.float32)
             src_d["gy"] = rng.standard_normal(d["gy"].shape, dtype=np.float32)
-            src_d["w"] = (d["w"] * rng.uniform(0.5, 1.5, size=(1, d["w"].shape[1]))).astype(np.float32)
+            src_d[wkey] = (d[wkey] * rng.uniform(0.5, 1.5, size=(1, d[wkey].shape[1]))).astype(np.float32)
         copies.append({k: torch.as_tensor(np.ascontiguousarray(src_d[k])).to(dev) for k in keys})
     y = torch.empty(N, out_dim, device=dev)
     gx = torch.empty(N, in_dim, device=dev)
     gw = torch.empty(E, nw, device=dev)
     gvec = torch.empty(E, 3, device=dev) if want_gvec else None
-    colptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
-    perm = torch.empty(E, dtype=torch.int32, device=dev)
-    ws_bytes = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD)
+    # one transpose per input copy: the transpose of step k runs on a side stream while the
+    # forward of step k runs on the main stream (they are independent); the backward waits
+    colptrs = [torch.empty(N + 1, dtype=torch.int32, device=dev) for _ in range(R)]
+    perms = [torch.empty(E, dtype=torch.int32, device=dev) for _ in range(R)]
+    colptr, perm = colptrs[0], perms[0]
+    gW = torch.empty(plan.n_shared_weights, device=dev) if uvw else None
+    ws_bytes = max(tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD), tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_t_bytes = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD) if not uvw else 256 + 8 * (N + E) + 4096
+    ws_t = torch.empty(ws_t_bytes, dtype=torch.uint8, device=dev)      # side-stream transpose scratch
     stream = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(dev)
     sh = stream.cuda_stream
+    sh_side = side.cuda_stream
     h = plan.handle
     P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None
 
     argsets = []
-    for cp in copies:
+    for r, cp in enumerate(copies):
+        Wp = P(cp["W"]) if uvw else None
         argsets.append((
-            (h, N, E, P(cp["rowptr"]), P(cp["src"]), P(cp["x"]), P(cp["vec"]), P(cp["w"]), None, P(y), None, 0, sh),
-            (N, E, P(cp["rowptr"]), P(cp["src"]), P(colptr), P(perm), P(ws), ws_bytes, sh),
-            (h, N, E, P(cp["rowptr"]), P(cp["src"]), P(colptr), P(perm), P(cp["x"]), P(cp["vec"]), P(cp["w"]),
-             None, P(cp["gy"]), P(gx), P(gw), P(gvec), None, P(ws), ws_bytes, sh),
+            (h, N, E, P(cp["rowptr"]), P(cp["src"]), P(cp["x"]), P(cp["vec"]), P(cp[wkey]), Wp, P(y), P(ws), ws_bytes,
+             sh),
+            (N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(ws_t), ws_t_bytes, sh_side),
+            (h, N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(cp["x"]), P(cp["vec"]),
+             P(cp[wkey]), Wp, P(cp["gy"]), P(gx), P(gw), P(gvec), P(gW), P(ws), ws_bytes, sh),
         ))
+    tr_done = [torch.cuda.Event() for _ in range(R)]
+    bwd_done = [torch.cuda.Event() for _ in range(R)]
     fwd_f, tr_f, bwd_f = lib.tp_conv_fwd, lib.tp_csr_transpose, lib.tp_conv_bwd
 
     def step(k, ev=None):
-        a_f, a_t, a_b = argsets[k % R]
+        r = k % R
+        a_f, a_t, a_b = argsets[r]
+        # side stream: this step's transpose, once the backward that last read this copy is done
+        side.wait_event(bwd_done[r])
+        if ev is not None:
+            ev[4].record(side)
+        st = tr_f(*a_t)
+        if ev is not None:
+            ev[5].record(side)
+        tr_done[r].record(side)
         if ev is not None:
             ev[0].record(stream)
-        st = fwd_f(*a_f)
+        st |= fwd_f(*a_f)
         if ev is not None:
             ev[1].record(stream)
-        st |= tr_f(*a_t)
+        stream.wait_event(tr_done[r])
         if ev is not None:
             ev[2].record(stream)
         st |= bwd_f(*a_b)
         if ev is not None:
             ev[3].record(stream)
+        bwd_done[r].record(stream)
         if st:
             raise RuntimeError(lib.tp_last_error_message().decode())
 
     for k in range(args.warmup):
         step(k)
     torch.cuda.synchronize(dev)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -329,19 +355,21 @@ def run_ours(args, rank, world, local):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     elapsed_max = float(t.item())
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    tr_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    tr_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in evs)
     bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
 
     # end to end through the same calls, inputs from pinned host memory, outputs back to host
     host_in = {k: torch.as_tensor(np.ascontiguousarray(d[k])).pin_memory() for k in keys}
     dev_in = {k: torch.empty_like(host_in[k], device=dev) for k in keys}
-    host_out = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in (y, gx, gw)]
+    outs = (y, gx, gw) + ((gW,) if uvw else ())
+    host_out = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in outs]
+    Wd = P(dev_in["W"]) if uvw else None
     e2e_args = (
-        (h, N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(dev_in["x"]), P(dev_in["vec"]), P(dev_in["w"]), None,
-         P(y), None, 0, sh),
-        (N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(ws), ws_bytes, sh),
+        (h, N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(dev_in["x"]), P(dev_in["vec"]), P(dev_in[wkey]), Wd,
+         P(y), P(ws), ws_bytes, sh),
+        (N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(ws_t), ws_t_bytes, sh),
         (h, N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(dev_in["x"]), P(dev_in["vec"]),
-         P(dev_in["w"]), None, P(dev_in["gy"]), P(gx), P(gw), P(gvec), None, P(ws), ws_bytes, sh))
+         P(dev_in[wkey]), Wd, P(dev_in["gy"]), P(gx), P(gw), P(gvec), P(gW), P(ws), ws_bytes, sh))
 
     def e2e_step():
         for k in keys:
@@ -349,7 +377,7 @@ def run_ours(args, rank, world, local):
         st = fwd_f(*e2e_args[0]) | tr_f(*e2e_args[1]) | bwd_f(*e2e_args[2])
         if st:
             raise RuntimeError(lib.tp_last_error_message().decode())
-        for ho, dv in zip(host_out, (y, gx, gw)):
+        for ho, dv in zip(host_out, outs):
             ho.copy_(dv, non_blocking=True)
 
     for _ in range(3):
@@ -385,7 +413,7 @@ def run_ours(args, rank, world, local):
                 "kernel_ms": {"fwd": fwd_ms, "transpose": tr_ms, "bwd": bwd_ms},
                 "step_roofline_frac": ((fb + bb) / (hbm * 1e9)) / (elapsed / args.steps)}
         cpu = None
-        if not args.no_cpu_baseline and world >= 1:
+        if not args.no_cpu_baseline and not uvw:
             from oracle.conv import set_threads
             cores = set_threads()
             oracle_sample(d, 4, seed=0)              # CG tables cached outside the timing

@@ -1,5 +1,6 @@
 // C ABI of the tensor-product convolution: plans, argument checks, workspace layout and
 // dispatch to the compiled specialisations.  See include/tp.h for the contract.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -161,6 +162,15 @@ UvwLayout uvw_layout(tp_plan_t plan, int64_t N, int64_t E, bool bwd) {
   return U;
 }
 
+// TP_TUNE_GEMM=simt runs the uvw mixing GEMMs on the fp32 SIMT kernel instead of tcgen05.
+int tune_use_tc() {
+  static const int v = [] {
+    const char* e = std::getenv("TP_TUNE_GEMM");
+    return (e && std::strcmp(e, "simt") == 0) ? 0 : 1;
+  }();
+  return v;
+}
+
 int pick_split(int64_t N, int64_t E) {
   if (N <= 0) return 1;
   const double avg = (double)E / (double)N;
@@ -194,6 +204,8 @@ LaunchArgs base_args(tp_plan_t plan, int64_t N, int64_t E) {
   a.has_coeff = plan->has_coeff;
   a.check = (plan->flags & TP_FLAG_CHECK_INDICES) ? 1 : 0;
   a.prefetch = tune_prefetch();
+  a.use_tc = tune_use_tc();
+
   std::memcpy(a.coeff, plan->coeff, sizeof(a.coeff));
   return a;
 }

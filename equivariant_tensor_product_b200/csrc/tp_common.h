@@ -29,6 +29,7 @@ struct LaunchArgs {
   int has_coeff;       // path coefficients differ from 1
   int check;           // bounds-check indices and report through *err
   int prefetch;        // -1: heuristic; 0/1: force register double-buffering of edge gathers
+  int use_tc;          // uvw mixing GEMMs on tcgen05 (1) or the fp32 SIMT kernel (0)
   const int32_t* rowptr;
   const int32_t* src;
   const int32_t* colptr;

@@ -17,6 +17,8 @@
 // is written anywhere: each edge's products are consumed straight into receiver (forward,
 // double-backward receiver pass) or sender (backward, double-backward sender pass) state.
 #pragma once
+#include <algorithm>
+
 #include "tp_common.h"
 
 namespace tp {
@@ -177,16 +179,30 @@ __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__
         compute(k + 1, xb, wb);
       }
     } else {
-#pragma unroll 1
+      // one edge at a time, gathers issued after the SH evaluation (fewer live registers)
       for (int k = 0; k < ne; ++k) {
-        fetch(k, xa, wa);
-        compute(k, xa, wa);
+        const int e = base + k * st;
+        const int j = __shfl_sync(kFull, my_j, k);
+        const float ux = __shfl_sync(kFull, vx, k);
+        const float uy = __shfl_sync(kFull, vy, k);
+        const float uz = __shfl_sync(kFull, vz, k);
+        if (j < 0) continue;
+        float rx, ry, rz, ir;
+        edge_geometry(ux, uy, uz, rx, ry, rz, ir);
+        float Y[S::NSH];
+        S::sh(rx, ry, rz, Y);
+        if (act) {
+          S::load_in(a.x + (int64_t)j * a.in_dim, a.mul, c, xa);
+          load_path_weights(a, e, c, wa);
+          S::fwd(xa, Y, wa, acc);
+        }
       }
     }
   }
   reduce_phases(acc, smem, phase, st, lane, 0, 1);
   if (phase == 0 && act) S::store_out(a.y + (int64_t)row * a.out_dim, a.mul, c, acc);
 }
+
 
 // ---------------------------------------------------------------------------------------
 // Backward, uvu, sender order (through the stable transpose perm; each edge's receiver is
@@ -249,6 +265,39 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
       }
     }
     const int ne = min(32, (q1 - base + st - 1) / st);
+    // gvec[e] = sum_m gY_m dY_m/dv with dY_m/dv = (grad P_m(r) - l_m Y_m r) / |v|; the
+    // channel sum is a warp reduction, then (NSL > 1) a sum over the slice warps
+    auto gvec_edge = [&](int k, int e, float rx, float ry, float rz, float ir, const float (&Y)[S::NSH],
+                         const float (&gY)[S::NSH]) {
+      float G[S::NSH][3];
+      S::sh_grad(rx, ry, rz, G);
+      float h0 = 0.f, h1 = 0.f, h2 = 0.f, sdeg = 0.f;
+#pragma unroll
+      for (int m = 0; m < S::NSH; ++m) {
+        h0 = fmaf(gY[m], G[m][0], h0);
+        h1 = fmaf(gY[m], G[m][1], h1);
+        h2 = fmaf(gY[m], G[m][2], h2);
+        sdeg = fmaf(S::sh_degree(m) * gY[m], Y[m], sdeg);
+      }
+      h0 = warp_sum(h0);
+      h1 = warp_sum(h1);
+      h2 = warp_sum(h2);
+      sdeg = warp_sum(sdeg);
+      if (NSL == 1) {
+        if (lane == 0 && e >= 0) {
+          float* g = a.gvec + 3 * (int64_t)e;
+          g[0] = ir * (h0 - rx * sdeg);
+          g[1] = ir * (h1 - ry * sdeg);
+          g[2] = ir * (h2 - rz * sdeg);
+        }
+      } else if (lane == 0) {
+        float* s = gslot + (((size_t)phase * 32 + k) * NSL + sl) * 4;
+        s[0] = h0;
+        s[1] = h1;
+        s[2] = h2;
+        s[3] = sdeg;
+      }
+    };
     // gathers of edge k: receiver slice gy[i] and the edge's weight row
     auto fetch = [&](int k, float (&gg)[S::OUT_PC], float (&ww)[S::P]) {
       const int e = __shfl_sync(kFull, my_e, k);
@@ -279,37 +328,7 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
           for (int p = 0; p < S::P; ++p) row[(int64_t)p * a.mul] = a.has_coeff ? gw[p] * a.coeff[p] : gw[p];
         }
       }
-      if constexpr (GVEC) {
-        // d Y_m / d v = (grad P_m(r) - l_m Y_m r) / |v|
-        float G[S::NSH][3];
-        S::sh_grad(rx, ry, rz, G);
-        float h0 = 0.f, h1 = 0.f, h2 = 0.f, sdeg = 0.f;
-#pragma unroll
-        for (int m = 0; m < S::NSH; ++m) {
-          h0 = fmaf(gY[m], G[m][0], h0);
-          h1 = fmaf(gY[m], G[m][1], h1);
-          h2 = fmaf(gY[m], G[m][2], h2);
-          sdeg = fmaf(S::sh_degree(m) * gY[m], Y[m], sdeg);
-        }
-        h0 = warp_sum(h0);
-        h1 = warp_sum(h1);
-        h2 = warp_sum(h2);
-        sdeg = warp_sum(sdeg);
-        if (NSL == 1) {
-          if (lane == 0 && e >= 0) {
-            float* g = a.gvec + 3 * (int64_t)e;
-            g[0] = ir * (h0 - rx * sdeg);
-            g[1] = ir * (h1 - ry * sdeg);
-            g[2] = ir * (h2 - rz * sdeg);
-          }
-        } else if (lane == 0) {
-          float* s = gslot + (((size_t)phase * 32 + k) * NSL + sl) * 4;
-          s[0] = h0;
-          s[1] = h1;
-          s[2] = h2;
-          s[3] = sdeg;
-        }
-      }
+      if constexpr (GVEC) gvec_edge(k, e, rx, ry, rz, ir, Y, gY);
     };
     float ga[S::OUT_PC], wa[S::P];
     if constexpr (PF) {
@@ -323,10 +342,33 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
         compute(k + 1, gb, wb);
       }
     } else {
-#pragma unroll 1
+      // one edge at a time; the gathers are issued after the SH evaluation so that fewer
+      // values are live at once (the lmax-3 bodies are register bound)
       for (int k = 0; k < ne; ++k) {
-        fetch(k, ga, wa);
-        compute(k, ga, wa);
+        const int e = __shfl_sync(kFull, my_e, k);
+        const int i = __shfl_sync(kFull, my_i, k);
+        const float ux = __shfl_sync(kFull, vx, k);
+        const float uy = __shfl_sync(kFull, vy, k);
+        const float uz = __shfl_sync(kFull, vz, k);
+        float rx, ry, rz, ir;
+        edge_geometry(ux, uy, uz, rx, ry, rz, ir);
+        float Y[S::NSH];
+        S::sh(rx, ry, rz, Y);
+        float gY[S::NSH];
+#pragma unroll
+        for (int m = 0; m < S::NSH; ++m) gY[m] = 0.f;
+        if (act && e >= 0) {
+          S::load_out(a.gy + (int64_t)i * a.out_dim, a.mul, c, ga);
+          load_path_weights(a, e, c, wa);
+          float gw[S::P];
+          S::template bwd<GVEC>(x, Y, wa, ga, gx, gw, gY);
+          if (a.gw) {
+            float* row = a.gw + (int64_t)e * a.nw + c;
+#pragma unroll
+            for (int p = 0; p < S::P; ++p) row[(int64_t)p * a.mul] = a.has_coeff ? gw[p] * a.coeff[p] : gw[p];
+          }
+        }
+        if constexpr (GVEC) gvec_edge(k, e, rx, ry, rz, ir, Y, gY);
       }
     }
     if constexpr (GVEC && NSL > 1) {

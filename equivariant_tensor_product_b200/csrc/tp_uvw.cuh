@@ -14,6 +14,7 @@
 #include <algorithm>
 
 #include "tp_kernels.cuh"
+#include "tp_mma.cuh"
 
 namespace tp {
 
@@ -236,6 +237,134 @@ struct GradWOp {
   }
 };
 
+
+// ---------------------------------------------------------------------------------------
+// The same three contractions for the tcgen05 GEMM (tp_mma.cuh): element accessors, vector
+// accessors for k-contiguous operands, and coalesced tile stores.
+// ---------------------------------------------------------------------------------------
+template <class S>
+struct TcMixFwdOp {           // y_o[(i, m3), w] = sum_k A_o[(i, m3), k] Wt_o[w, k]
+  int o;
+  static constexpr bool A_KCONTIG = true, B_KCONTIG = true;
+  __device__ int64_t M(const LaunchArgs& a) const { return (int64_t)a.N * S::out_d3_at(o); }
+  __device__ int Nn(const LaunchArgs& a) const { return a.mul_out; }
+  __device__ int K(const LaunchArgs& a) const { return S::out_cnt_at(o) * a.mul; }
+  __device__ void k_range(const LaunchArgs& a, int, int64_t& b, int64_t& e) const { b = 0; e = K(a); }
+  __device__ const float* Abase(const LaunchArgs& a) const { return a.A + (int64_t)a.N * a.mul * S::out_cumA_at(o); }
+  __device__ const float* Bbase(const LaunchArgs& a) const {
+    int64_t off = 0;
+    for (int q = 0; q < o; ++q) off += (int64_t)S::out_cnt_at(q) * a.mul * a.mul_out;
+    return a.Wt + off;
+  }
+  __device__ float A(const LaunchArgs& a, int64_t m, int64_t k) const { return Abase(a)[m * K(a) + k]; }
+  __device__ float B(const LaunchArgs& a, int n, int64_t k) const { return Bbase(a)[(int64_t)n * K(a) + k]; }
+  __device__ float4 A4(const LaunchArgs& a, int64_t m, int64_t k) const {
+    return *reinterpret_cast<const float4*>(Abase(a) + m * K(a) + k);
+  }
+  __device__ float4 B4(const LaunchArgs& a, int n, int64_t k) const {
+    return *reinterpret_cast<const float4*>(Bbase(a) + (int64_t)n * K(a) + k);
+  }
+  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0) const {
+    const int d3 = S::out_d3_at(o);
+    const int64_t Mx = M(a);
+    const int64_t i0 = m0 / d3, i1 = (min(Mx, m0 + TC_BM) - 1) / d3;
+    const int cols = min(TC_BN, a.mul_out - n0);
+    const int per_i = cols * d3;
+    const int64_t total = (i1 - i0 + 1) * per_i;
+    for (int64_t t = threadIdx.x; t < total; t += blockDim.x) {
+      const int64_t i = i0 + t / per_i;
+      const int q = (int)(t % per_i);
+      const int w = q / d3, m3 = q - (q / d3) * d3;
+      const int64_t row = i * d3 + m3 - m0;
+      if (row < 0 || row >= TC_BM || i * d3 + m3 >= Mx) continue;
+      a.y[i * a.out_dim + (int64_t)a.mul_out * S::out_cumY_at(o) + (int64_t)(n0 + w) * d3 + m3] = T[row * ld + w];
+    }
+  }
+};
+
+template <class S>
+struct TcGradStateOp {        // G_o[(i, m3), (pl, u)] = sum_w gy_o[(i, m3), w] W_p[u, w]
+  int o;
+  static constexpr bool A_KCONTIG = false, B_KCONTIG = true;
+  __device__ int64_t M(const LaunchArgs& a) const { return (int64_t)a.N * S::out_d3_at(o); }
+  __device__ int Nn(const LaunchArgs& a) const { return S::out_cnt_at(o) * a.mul; }
+  __device__ void k_range(const LaunchArgs& a, int, int64_t& b, int64_t& e) const { b = 0; e = a.mul_out; }
+  __device__ float A(const LaunchArgs& a, int64_t m, int64_t k) const {
+    const int d3 = S::out_d3_at(o);
+    const int64_t i = m / d3;
+    const int m3 = (int)(m - i * d3);
+    return a.gy[i * a.out_dim + (int64_t)a.mul_out * S::out_cumY_at(o) + k * d3 + m3];
+  }
+  __device__ float4 A4(const LaunchArgs& a, int64_t m, int64_t k) const {
+    return make_float4(A(a, m, k), A(a, m, k + 1), A(a, m, k + 2), A(a, m, k + 3));
+  }
+  __device__ const float* Brow(const LaunchArgs& a, int n) const {
+    const int pl = n / a.mul, u = n - pl * a.mul;
+    return a.W + ((int64_t)S::path_of_at(o, pl) * a.mul + u) * a.mul_out;
+  }
+  __device__ float B(const LaunchArgs& a, int n, int64_t k) const { return Brow(a, n)[k]; }
+  __device__ float4 B4(const LaunchArgs& a, int n, int64_t k) const {
+    return *reinterpret_cast<const float4*>(Brow(a, n) + k);
+  }
+  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0) const {
+    const int64_t Mx = M(a);
+    const int Kn = Nn(a);
+    const int cols = min(TC_BN, Kn - n0);
+    float* G = a.G + (int64_t)a.N * a.mul * S::out_cumA_at(o);
+    for (int t = threadIdx.x; t < TC_BM * cols; t += blockDim.x) {
+      const int r = t / cols, c = t - r * cols;
+      if (m0 + r < Mx) G[(m0 + r) * Kn + n0 + c] = T[r * ld + c];
+    }
+  }
+};
+
+template <class S>
+struct TcGradWOp {            // part[z][p][u][w] = sum_{(i, m3) in split z} A_o[(i, m3), (pl, u)] gy_o[(i, m3), w]
+  int o;
+  static constexpr bool A_KCONTIG = false, B_KCONTIG = false;
+  __device__ int64_t M(const LaunchArgs& a) const { return (int64_t)S::out_cnt_at(o) * a.mul; }
+  __device__ int Nn(const LaunchArgs& a) const { return a.mul_out; }
+  __device__ void k_range(const LaunchArgs& a, int z, int64_t& b, int64_t& e) const {
+    const int64_t rows = (int64_t)a.N * S::out_d3_at(o);
+    const int64_t chunk = ((rows + a.splits - 1) / a.splits + TC_BK - 1) / TC_BK * TC_BK;
+    b = min(rows, (int64_t)z * chunk);
+    e = min(rows, b + chunk);
+  }
+  __device__ float A(const LaunchArgs& a, int64_t m, int64_t k) const {
+    return a.A[(int64_t)a.N * a.mul * S::out_cumA_at(o) + k * M(a) + m];
+  }
+  __device__ float4 A4(const LaunchArgs& a, int64_t m, int64_t k) const {
+    return make_float4(A(a, m, k), A(a, m, k + 1), A(a, m, k + 2), A(a, m, k + 3));
+  }
+  __device__ float B(const LaunchArgs& a, int n, int64_t k) const {
+    const int d3 = S::out_d3_at(o);
+    const int64_t i = k / d3;
+    const int m3 = (int)(k - i * d3);
+    return a.gy[i * a.out_dim + (int64_t)a.mul_out * S::out_cumY_at(o) + (int64_t)n * d3 + m3];
+  }
+  __device__ float4 B4(const LaunchArgs& a, int n, int64_t k) const {
+    return make_float4(B(a, n, k), B(a, n, k + 1), B(a, n, k + 2), B(a, n, k + 3));
+  }
+  __device__ void store_tile(const LaunchArgs& a, int z, const float* T, int ld, int64_t m0, int n0) const {
+    const int64_t Mx = M(a);
+    const int cols = min(TC_BN, a.mul_out - n0);
+    for (int t = threadIdx.x; t < TC_BM * cols; t += blockDim.x) {
+      const int r = t / cols, c = t - r * cols;
+      const int64_t m = m0 + r;
+      if (m >= Mx) continue;
+      const int pl = (int)(m / a.mul), u = (int)(m - (int64_t)pl * a.mul);
+      const int p = S::path_of_at(o, pl);
+      a.part[((int64_t)z * S::P + p) * a.mul * a.mul_out + (int64_t)u * a.mul_out + n0 + c] = T[r * ld + c];
+    }
+  }
+};
+
+// The tensor-core path reads k-contiguous operand rows (A, G, Wt in the workspace and the
+// caller's W) as float4: it needs multiplicities divisible by 4 and a 16-byte aligned W.
+inline bool tc_usable(const LaunchArgs& a) {
+  return a.use_tc && a.mul % 4 == 0 && a.mul_out % 4 == 0 && (reinterpret_cast<uintptr_t>(a.W) & 15u) == 0;
+}
+
 // gW[idx] = sum_z part[z][idx] in split order (deterministic)
 static __global__ void k_reduce_splits(const float* __restrict__ part, int splits, int64_t n, float* gW) {
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < n; t += (int64_t)gridDim.x * blockDim.x) {
@@ -402,8 +531,10 @@ cudaError_t launch_uvw_fwd(const LaunchArgs& a, cudaStream_t s) {
   k_uvw_prep_wt<S><<<64, 256, 0, s>>>(a);
   count_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const bool tc = tc_usable(a);
   for (int o = 0; o < S::N_OUT; ++o) {
-    e = launch_gemm(a, MixFwdOp<S>{o}, (int64_t)a.N * S::out_d3_at(o), a.mul_out, 1, s);
+    const int64_t M = (int64_t)a.N * S::out_d3_at(o);
+    e = tc ? launch_gemm_tc(a, TcMixFwdOp<S>{o}, M, a.mul_out, 1, s) : launch_gemm(a, MixFwdOp<S>{o}, M, a.mul_out, 1, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -414,11 +545,15 @@ cudaError_t launch_uvw_bwd(const LaunchArgs& a, cudaStream_t s) {
   if (a.N == 0) return cudaSuccess;
   cudaError_t e = launch_uvw_edge<S>(a, s);
   if (e != cudaSuccess) return e;
+  const bool tc = tc_usable(a);
   for (int o = 0; o < S::N_OUT; ++o) {
-    e = launch_gemm(a, GradStateOp<S>{o}, (int64_t)a.N * S::out_d3_at(o), S::out_cnt_at(o) * a.mul, 1, s);
+    const int64_t M = (int64_t)a.N * S::out_d3_at(o);
+    const int K = S::out_cnt_at(o) * a.mul;
+    e = tc ? launch_gemm_tc(a, TcGradStateOp<S>{o}, M, K, 1, s) : launch_gemm(a, GradStateOp<S>{o}, M, K, 1, s);
     if (e != cudaSuccess) return e;
     if (a.gW) {
-      e = launch_gemm(a, GradWOp<S>{o}, (int64_t)S::out_cnt_at(o) * a.mul, a.mul_out, a.splits, s);
+      e = tc ? launch_gemm_tc(a, TcGradWOp<S>{o}, K, a.mul_out, a.splits, s)
+             : launch_gemm(a, GradWOp<S>{o}, K, a.mul_out, a.splits, s);
       if (e != cudaSuccess) return e;
     }
   }
