@@ -51,7 +51,25 @@ def parse():
     ap.add_argument("--workload", default="c2", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--n-atoms", type=int, default=None,
+                    help="same-density replica with fewer atoms (profiling small cases)")
     return ap.parse_args()
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (device time is taken as the slowest rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(edges_per_replica: int, steps: int, world: int, elapsed_max_s: float) -> float:
+    """Whole-job edges/s: every rank processes its own replica of the workload (weak scaling)."""
+    return world * steps * edges_per_replica / elapsed_max_s
 
 
 def dist_env():
@@ -247,7 +265,7 @@ def run_ours(args, rank, world, local):
     lib = tp.load()
 
     spec = synth.CONFIGS[args.workload]
-    d = synth.make_inputs(args.workload, seed=spec.seed + 7919 * rank)
+    d = synth.make_inputs(args.workload, args.n_atoms, seed=spec.seed + 7919 * rank)
     plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, spec.mode)
     N, E = len(d["rowptr"]) - 1, len(d["src"])
     in_dim, out_dim, nw = plan.in_dim, plan.out_dim, plan.n_edge_weights
@@ -350,10 +368,7 @@ def run_ours(args, rank, world, local):
     if world > 1:
         dist.barrier()
     elapsed = start.elapsed_time(stop) / 1e3
-    t = torch.tensor([elapsed], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_max = float(t.item())
+    elapsed_max = max_over_ranks(elapsed, world, dev)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     tr_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in evs)
     bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -390,10 +405,7 @@ def run_ours(args, rank, world, local):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_s = e0.elapsed_time(e1) / 1e3
-    te = torch.tensor([e2e_s], device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * args.e2e_steps * E / float(te.item())
+    e2e_value = replica_throughput(E, args.e2e_steps, world, max_over_ranks(e2e_s, world, dev))
     h2d = sum(host_in[k].numel() * host_in[k].element_size() for k in keys)
     d2h = sum(t_.numel() * t_.element_size() for t_ in host_out)
 
@@ -423,7 +435,7 @@ def run_ours(args, rank, world, local):
                    "sample": f"fwd on the {ef} edges into {n_rows} receivers + bwd on the {eb} edges leaving "
                              f"{n_rows} senders of the same workload (rank 0's copy), float64 torch CPU, "
                              f"{tf + tb:.1f} s"}
-        value = world * args.steps * E / elapsed_max
+        value = replica_throughput(E, args.steps, world, elapsed_max)
         line = {
             "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * elapsed_max / args.steps, "higher_is_better": True,
