@@ -148,7 +148,9 @@ struct UvwLayout {
 UvwLayout uvw_layout(tp_plan_t plan, int64_t N, int64_t E, bool bwd) {
   UvwLayout U{};
   size_t off = bwd ? ws_layout(N, E).total : 256;
-  const size_t a_bytes = sizeof(float) * (size_t)N * plan->ops->A_PC * plan->mul_in;
+  // forward: receiver state A (A_PC x mul per node); backward: x W and B (XT_PC x mul_out)
+  const size_t a_bytes = bwd ? sizeof(float) * (size_t)N * plan->ops->XT_PC * plan->mul_out
+                             : sizeof(float) * (size_t)N * plan->ops->A_PC * plan->mul_in;
   const size_t w_bytes = sizeof(float) * (size_t)plan->n_shared;
   U.A = off;
   off += align256(a_bytes > 0 ? a_bytes : 1);
@@ -160,15 +162,6 @@ UvwLayout uvw_layout(tp_plan_t plan, int64_t N, int64_t E, bool bwd) {
   if (bwd) off += align256(w_bytes * kUvwSplits);
   U.total = off;
   return U;
-}
-
-// TP_TUNE_GEMM=simt runs the uvw mixing GEMMs on the fp32 SIMT kernel instead of tcgen05.
-int tune_use_tc() {
-  static const int v = [] {
-    const char* e = std::getenv("TP_TUNE_GEMM");
-    return (e && std::strcmp(e, "simt") == 0) ? 0 : 1;
-  }();
-  return v;
 }
 
 int pick_split(int64_t N, int64_t E) {
@@ -204,7 +197,7 @@ LaunchArgs base_args(tp_plan_t plan, int64_t N, int64_t E) {
   a.has_coeff = plan->has_coeff;
   a.check = (plan->flags & TP_FLAG_CHECK_INDICES) ? 1 : 0;
   a.prefetch = tune_prefetch();
-  a.use_tc = tune_use_tc();
+
 
   std::memcpy(a.coeff, plan->coeff, sizeof(a.coeff));
   return a;

@@ -572,50 +572,6 @@ def _gen_dbwd_send(spec: Spec) -> List[str]:
     return L
 
 
-def _gen_uvw_bwd(spec: Spec) -> List[str]:
-    """uvw sender pass for one edge and one channel u, given G[p, u, m3] (gradient of the
-    per-path aggregated state, gathered from the receiver):
-       gx[in(p)] += s[p] * sum_{m2,m3} C Y[m2] G[p, m3]
-       gs[p]     += sum C x[m1] Y[m2] G[p, m3]     (partial over this channel)
-       gY[sh(p)] += s[p] * sum_{m1,m3} C x[m1] G[p, m3]   (WITH_GY)"""
-    L = ["  template <bool WITH_GY>",
-         f"  __device__ __forceinline__ static void uvw_bwd(const float (&x)[{spec.IN_PC}], const float (&Y)[{spec.NSH}], const float (&s)[{spec.P}], const float (&G)[{spec.A_PC}], float (&gx)[{spec.IN_PC}], float (&gs)[{spec.P}], float (&gY)[{spec.NSH}]) {{"]
-    for p, (a, b, o) in enumerate(spec.paths):
-        lb = spec.sh_ls[b]
-        nz = cg_nonzeros(*spec.triples[p])
-        d1, d2 = 2 * spec.triples[p][0] + 1, 2 * spec.triples[p][1] + 1
-        L.append(f"    {{ // path {p}")
-        used = sorted({(j, k) for (i, j, k, c) in nz})
-        for (j, k) in used:
-            gs_ = f"G[{spec.a_cum[p] + k}]"
-            L.append(f"      const float r{j}_{k} = {gs_};" if lb == 0 else f"      const float r{j}_{k} = Y[{spec.sh_cum[b] + j}] * {gs_};")
-        gterms = []
-        for i in range(d1):
-            t = [(c, f"r{j}_{k}") for (ii, j, k, c) in nz if ii == i]
-            if not t:
-                continue
-            L += _chain(t, f"z{i}")
-            L.append(f"      gx[{spec.in_cum[a] + i}] = fmaf(s[{p}], z{i}, gx[{spec.in_cum[a] + i}]);")
-            gterms.append(i)
-        for i in gterms:
-            L.append(f"      gs[{p}] = fmaf(x[{spec.in_cum[a] + i}], z{i}, gs[{p}]);")
-        if lb != 0:
-            L.append("      if constexpr (WITH_GY) {")
-            used2 = sorted({(i, k) for (i, j, k, c) in nz})
-            for (i, k) in used2:
-                L.append(f"      const float s{i}_{k} = x[{spec.in_cum[a] + i}] * G[{spec.a_cum[p] + k}];")
-            for j in range(d2):
-                t = [(c, f"s{i}_{k}") for (i, jj, k, c) in nz if jj == j]
-                if not t:
-                    continue
-                L += _chain(t, f"qq{j}")
-                L.append(f"      gY[{spec.sh_cum[b] + j}] = fmaf(s[{p}], qq{j}, gY[{spec.sh_cum[b] + j}]);")
-            L.append("      }")
-        L.append("    }")
-    L.append("  }")
-    return L
-
-
 def _uvw_tables(spec: Spec):
     """Per output irrep o: paths into o (in path order), d3, count, and the per-(node, channel)
     offset of its region in the uvw node state A (regions in output order)."""
@@ -663,6 +619,109 @@ def _gen_uvw_layout(spec: Spec) -> List[str]:
     return L
 
 
+def _uvw_in_tables(spec: Spec):
+    """Per input irrep a: paths reading a (in path order), d1, count, and the per-(node, channel)
+    offset of its region in the sender-side state (x W and its gradient partner B)."""
+    ins = []
+    cum = 0
+    for a, l1 in enumerate(spec.in_ls):
+        plist = [p for p, path in enumerate(spec.paths) if path[0] == a]
+        d1 = 2 * l1 + 1
+        ins.append(dict(a=a, d1=d1, paths=plist, cnt=len(plist), cumX=cum))
+        cum += d1 * len(plist)
+    return ins, cum
+
+
+def _gen_uvw_send_layout(spec: Spec) -> List[str]:
+    ins, xt_pc = _uvw_in_tables(spec)
+    n = len(ins)
+    maxc = max(1, max(t["cnt"] for t in ins))
+    # per path: block offset inside one channel's xt row (path order)
+    xt_cum = [0] * spec.P
+    c = 0
+    for p in range(spec.P):
+        xt_cum[p] = c
+        c += 2 * spec.triples[p][0] + 1
+    L = [f"  static constexpr int XT_PC = {xt_pc};",
+         f"  static constexpr int N_IN = {n};",
+         f"  static constexpr int MAX_CNT_IN = {maxc};"]
+    for name, vals in (("in_d1_at", [t["d1"] for t in ins]), ("in_cnt_at", [t["cnt"] for t in ins]),
+                       ("in_cumX_at", [t["cumX"] for t in ins]), ("in_cum_at", list(spec.in_cum))):
+        L.append(f"  __host__ __device__ static int {name}(int a) {{ constexpr int v[{n}] = "
+                 f"{{{', '.join(map(str, vals))}}}; return v[a]; }}")
+    flat = []
+    for t in ins:
+        flat += t["paths"] + [-1] * (maxc - t["cnt"])
+    L.append(f"  __host__ __device__ static int path_in_at(int a, int pl) {{ constexpr int v[{n * maxc}] = "
+             f"{{{', '.join(map(str, flat))}}}; return v[a * {maxc} + pl]; }}")
+    # region a of the sender state: N*mul*cumX_a + ((j*d1 + m1)*cnt_a + pl)*mul + c ; register xt[xt_cum[p] + m1]
+    for name, const in (("load_xt", True), ("store_xt", False)):
+        L.append(f"  __device__ __forceinline__ static void {name}({'const ' if const else ''}float* __restrict__ base, "
+                 f"int64_t N, int mul, int64_t j, int c, {'float' if const else 'const float'} (&v)[{xt_pc}]) {{")
+        for t in ins:
+            for pl, p in enumerate(t["paths"]):
+                for m1 in range(t["d1"]):
+                    idx = f"N * mul * {t['cumX']} + ((j * {t['d1']} + {m1}) * {t['cnt']} + {pl}) * (int64_t)mul + c"
+                    k = xt_cum[p] + m1
+                    L.append(f"    v[{k}] = __ldg(base + {idx});" if const else f"    base[{idx}] = v[{k}];")
+        L.append("  }")
+    return L, xt_cum, xt_pc
+
+
+def _gen_uvw_send(spec: Spec, xt_cum, xt_pc) -> List[str]:
+    """uvw sender pass for one edge and one output channel w, with xt = (x W)[sender] per path:
+       Z_p[m1]  = sum_{m2,m3} C Y[m2] gy[out(p), m3]
+       bt[p]   += s[p] Z_p            (sender state; gx = bt W^T, gW = x^T bt)
+       gs[p]   += sum_m1 xt_p[m1] Z_p[m1]      (partial over this channel)
+       gY[sh(p)] += s[p] sum_{m1,m3} C xt_p[m1] gy[m3]   (WITH_GY)"""
+    L = ["  template <bool WITH_GY>",
+         f"  __device__ __forceinline__ static void uvw_send(const float (&xt)[{xt_pc}], const float (&Y)[{spec.NSH}], const float (&s)[{spec.P}], const float (&gy)[{spec.OUT_PC}], float (&bt)[{xt_pc}], float (&gs)[{spec.P}], float (&gY)[{spec.NSH}]) {{"]
+    groups = _group(spec, lambda p: (p[1], p[2]))
+    for (b, o), plist in groups.items():
+        lb = spec.sh_ls[b]
+        L.append(f"    {{ // SH block {b} x out block {o}")
+        used = set()
+        for p in plist:
+            for (i, j, k, c) in cg_nonzeros(*spec.triples[p]):
+                used.add((j, k))
+        for (j, k) in sorted(used):
+            gs_ = f"gy[{spec.out_cum[o] + k}]"
+            L.append(f"      const float r{j}_{k} = {gs_};" if lb == 0 else f"      const float r{j}_{k} = Y[{spec.sh_cum[b] + j}] * {gs_};")
+        for p in plist:
+            nz = cg_nonzeros(*spec.triples[p])
+            d1 = 2 * spec.triples[p][0] + 1
+            zs = []
+            for i in range(d1):
+                terms = [(c, f"r{j}_{k}") for (ii, j, k, c) in nz if ii == i]
+                if not terms:
+                    continue
+                L += _chain(terms, f"z{p}_{i}")
+                L.append(f"      bt[{xt_cum[p] + i}] = fmaf(s[{p}], z{p}_{i}, bt[{xt_cum[p] + i}]);")
+                zs.append(i)
+            for i in zs:
+                L.append(f"      gs[{p}] = fmaf(xt[{xt_cum[p] + i}], z{p}_{i}, gs[{p}]);")
+        L.append("    }")
+    L.append("    if constexpr (WITH_GY) {")
+    for p, (a, b, o) in enumerate(spec.paths):
+        if spec.sh_ls[b] == 0:
+            continue
+        nz = cg_nonzeros(*spec.triples[p])
+        d2 = 2 * spec.triples[p][1] + 1
+        L.append(f"    {{ // path {p}")
+        for (i, k) in sorted({(i, k) for (i, j, k, c) in nz}):
+            L.append(f"      const float t{i}_{k} = xt[{xt_cum[p] + i}] * gy[{spec.out_cum[o] + k}];")
+        for j in range(d2):
+            terms = [(c, f"t{i}_{k}") for (i, jj, k, c) in nz if jj == j]
+            if not terms:
+                continue
+            L += _chain(terms, f"q{j}")
+            L.append(f"      gY[{spec.sh_cum[b] + j}] = fmaf(s[{p}], q{j}, gY[{spec.sh_cum[b] + j}]);")
+        L.append("    }")
+    L.append("    }")
+    L.append("  }")
+    return L
+
+
 def gen_spec_header(spec: Spec) -> str:
     L = [f"// Generated by codegen.py for spec '{spec.name}'.  Do not edit.",
          f"// inputs l={spec.in_ls}  SH l={spec.sh_ls}  outputs l={spec.out_ls}",
@@ -690,8 +749,10 @@ def gen_spec_header(spec: Spec) -> str:
     L += _gen_bwd(spec)
     L += _gen_dbwd_recv(spec)
     L += _gen_dbwd_send(spec)
-    L += _gen_uvw_bwd(spec)
     L += _gen_uvw_layout(spec)
+    lay, xt_cum, xt_pc = _gen_uvw_send_layout(spec)
+    L += lay
+    L += _gen_uvw_send(spec, xt_cum, xt_pc)
     L.append("};")
     return "\n".join(L) + "\n"
 
@@ -738,9 +799,10 @@ def _ops_initializer(s: Spec, fns) -> str:
         v = list(v) + [0] * (n - len(v))
         return "{" + ", ".join(map(str, v)) + "}"
     paths = "{" + ", ".join("{%d, %d, %d}" % p for p in s.paths) + "}"
+    xt_pc = _uvw_in_tables(s)[1]
     return (f"  \"{s.name}\", {len(s.in_ls)}, {arr(s.in_ls, 16)}, {len(s.sh_ls)}, {arr(s.sh_ls, 16)}, "
             f"{len(s.out_ls)}, {arr(s.out_ls, 16)}, {s.P}, {paths},\n"
-            f"  {s.IN_PC}, {s.OUT_PC}, {s.NSH}, {s.P}, {s.A_PC},\n  " + ", ".join(fns))
+            f"  {s.IN_PC}, {s.OUT_PC}, {s.NSH}, {s.P}, {s.A_PC}, {xt_pc},\n  " + ", ".join(fns))
 
 
 # kernels of each spec, split into translation units that compile in parallel

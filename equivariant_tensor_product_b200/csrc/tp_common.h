@@ -29,7 +29,6 @@ struct LaunchArgs {
   int has_coeff;       // path coefficients differ from 1
   int check;           // bounds-check indices and report through *err
   int prefetch;        // -1: heuristic; 0/1: force register double-buffering of edge gathers
-  int use_tc;          // uvw mixing GEMMs on tcgen05 (1) or the fp32 SIMT kernel (0)
   const int32_t* rowptr;
   const int32_t* src;
   const int32_t* colptr;
@@ -42,9 +41,10 @@ struct LaunchArgs {
   const float* ggw;
   const float* ggvec;
   const float* W;       // uvw: shared mixing matrices [P][mul][mul_out]
-  float* A;             // uvw: per-path node state (workspace), layout of S::store_uvw
-  float* G;             // uvw: gradient of A (workspace), same layout
-  float* Wt;            // uvw: W regrouped per output irrep, [o][w][pl*mul + u] (workspace)
+  float* A;             // uvw forward: per-path receiver state (workspace), S::store_uvw layout;
+                        // uvw backward: x W per path and sender, S::load_xt layout
+  float* G;             // uvw backward: sender state B (workspace), S::store_xt layout
+  float* Wt;            // uvw: W regrouped for the GEMM B operands (workspace)
   float* gW;            // uvw: gradient of W (output)
   float* part;          // uvw: split-K partials of gW (workspace)
   int splits;           // uvw: number of split-K partials
@@ -68,13 +68,13 @@ struct SpecOps {
   int n_sh, sh_ls[kMaxBlocks];
   int n_out, out_ls[kMaxBlocks];
   int n_paths, paths[kMaxPaths][3];
-  int IN_PC, OUT_PC, NSH, P, A_PC;
+  int IN_PC, OUT_PC, NSH, P, A_PC, XT_PC;
   LaunchFn fwd_uvu;         // y = conv(x)
   LaunchFn bwd_uvu;         // gx, gw (gvec when args.gvec != nullptr), sender order
   LaunchFn dbwd_recv;       // g_gy, receiver order
   LaunchFn dbwd_send;       // g_x, g_w, g_vec, sender order
   LaunchFn uvw_fwd;         // edge pass into A, then y = mix(A, W)
-  LaunchFn uvw_bwd;         // A again, G = W gy, gW = A^T gy, then the sender pass for gx, gs, gvec
+  LaunchFn uvw_bwd;         // x W, the sender pass for B, gs, gvec, then gx = B W^T, gW = x^T B
 };
 
 extern const SpecOps* const kRegistry[];

@@ -117,47 +117,79 @@ __device__ __forceinline__ void stage4(char* hi_blk, char* lo_blk, int row, int 
   *reinterpret_cast<float4*>(lo_blk + off) = l;
 }
 
+// Operand addressing.  Element (r, k) of an operand lives at
+//   base[row(r) + kpart(k)],  kpart(k) = (k / kd) * ks1 + (k % kd) * ks2   (kd = 0: k * ks1)
+// row(r) is any per-row offset (computed once per row and K block); the k part is affine or
+// splits k into (outer, inner) with a small inner extent, which covers every uvw layout.
+struct TcOperand {
+  const float* base;
+  int kd;              // 0: plain stride ks1; else k = (k / kd, k % kd)
+  int64_t ks1, ks2;
+  bool vec4;           // rows are k-contiguous and 16-byte aligned: load 4 k at once
+  __device__ __forceinline__ int64_t kpart(int64_t k) const {
+    if (kd == 0) return k * ks1;
+    const int64_t q = k / kd;
+    return q * ks1 + (k - q * kd) * ks2;
+  }
+};
+
 // Op interface:
-//   int64_t M(a); int Nn(a); void k_range(a, z, &k0, &k1);
-//   static constexpr bool A_KCONTIG, B_KCONTIG   (operand contiguous along k in memory)
-//   float A(a, m, k), B(a, n, k)                 (scalar element, caller checks bounds)
-//   float4 A4(a, m, k), B4(a, n, k)              (4 consecutive k, K-contiguous operands only)
-//   void store_tile(a, z, const float* T, ld, m0, n0)   (T[row][col], row < 128, col < 128)
-// The whole CTA (128 threads) stages one operand block.
+//   int64_t M, Nn; void k_range(a, z, &k0, &k1)
+//   TcOperand A, B (set on the host);  static constexpr bool A_KCONTIG, B_KCONTIG (thread mapping)
+//   __device__ int64_t a_row(a, m), b_row(a, n)   (offset of row m of A / row n of B)
+//   __device__ void store_tile(a, z, const float* T, int ld, int64_t m0, int n0)
+// A thread of the CTA stages a fixed (row, chunk) set of a 128 x 32 block: with k-contiguous
+// operands consecutive threads walk along k, otherwise along rows (coalesced either way).
 template <class Op, bool IS_A>
-__device__ __forceinline__ void stage_block(const LaunchArgs& a, const Op& op, char* hi, char* lo, int64_t r0,
-                                            int64_t rows, int64_t k0, int64_t k1) {
-  const int t = threadIdx.x;
-  constexpr bool KC = IS_A ? Op::A_KCONTIG : Op::B_KCONTIG;
-#pragma unroll
-  for (int it = 0; it < (TC_BM * TC_BK / 4) / 128; ++it) {
-    const int q = t + 128 * it;
-    int row, chunk;
-    if (KC) {               // consecutive threads walk along k (coalesced on k)
+struct TcStager {
+  static constexpr bool KC = IS_A ? Op::A_KCONTIG : Op::B_KCONTIG;
+  static constexpr int NIT = (TC_BM * TC_BK / 4) / 128;   // 8 chunks of 4 per thread
+  float4 v[NIT];
+  __device__ __forceinline__ static void slot(int it, int& row, int& chunk) {
+    const int q = threadIdx.x + 128 * it;
+    if (KC) {
       row = q >> 3;
       chunk = q & 7;
-    } else {                // consecutive threads walk along rows (coalesced on rows)
+    } else {
       row = q & 127;
       chunk = q >> 7;
     }
-    const int64_t r = r0 + row, k = k0 + 4 * chunk;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < rows) {
-      if (KC && k + 3 < k1) {
-        v = IS_A ? op.A4(a, r, k) : op.B4(a, (int)r, k);
-      } else {
-        float e[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) e[j] = (k + j < k1) ? (IS_A ? op.A(a, r, k + j) : op.B(a, (int)r, k + j)) : 0.f;
-        v = make_float4(e[0], e[1], e[2], e[3]);
-      }
-    }
-    stage4(hi, lo, row, chunk, v);
   }
-}
+  __device__ __forceinline__ void load(const LaunchArgs& a, const Op& op, int64_t r0, int64_t rows, int64_t k0,
+                                       int64_t k1) {
+    const TcOperand& od = IS_A ? op.A : op.B;
+#pragma unroll
+    for (int it = 0; it < NIT; ++it) {
+      int row, chunk;
+      slot(it, row, chunk);
+      const int64_t r = r0 + row, k = k0 + 4 * chunk;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < rows && k < k1) {
+        const float* p = od.base + (IS_A ? op.a_row(a, r) : op.b_row(a, r));
+        if (od.vec4 && k + 3 < k1) {
+          x = *reinterpret_cast<const float4*>(p + k);
+        } else {
+          float e[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) e[j] = (k + j < k1) ? __ldg(p + od.kpart(k + j)) : 0.f;
+          x = make_float4(e[0], e[1], e[2], e[3]);
+        }
+      }
+      v[it] = x;
+    }
+  }
+  __device__ __forceinline__ void store(char* hi, char* lo) const {
+#pragma unroll
+    for (int it = 0; it < NIT; ++it) {
+      int row, chunk;
+      slot(it, row, chunk);
+      stage4(hi, lo, row, chunk, v[it]);
+    }
+  }
+};
 
 template <class Op>
-__global__ void __launch_bounds__(128, 1) k_gemm_tc(const __grid_constant__ LaunchArgs a, const Op op) {
+__global__ void __launch_bounds__(128, 1) k_gemm_tc(const __grid_constant__ LaunchArgs a, const __grid_constant__ Op op) {
   extern __shared__ __align__(1024) char tc_smem_raw[];
   __shared__ uint64_t mbar[TC_STAGES];
   __shared__ uint32_t tmem_holder;
@@ -166,8 +198,6 @@ __global__ void __launch_bounds__(128, 1) k_gemm_tc(const __grid_constant__ Laun
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t m0 = (int64_t)blockIdx.x * TC_BM;
   const int n0 = blockIdx.y * TC_BN;
-  const int64_t M = op.M(a);
-  const int Nn = op.Nn(a);
   int64_t k_begin, k_end;
   op.k_range(a, blockIdx.z, k_begin, k_end);
 
@@ -187,7 +217,12 @@ __global__ void __launch_bounds__(128, 1) k_gemm_tc(const __grid_constant__ Laun
   const uint32_t tmem = tmem_holder;
 
   const int nkb = (int)((k_end - k_begin + TC_BK - 1) / TC_BK);
-  uint32_t issued = 0;   // MMA groups committed per stage, for the parity of the next wait
+  TcStager<Op, true> sa;
+  TcStager<Op, false> sb;
+  if (nkb > 0) {
+    sa.load(a, op, m0, op.M, k_begin, k_end);
+    sb.load(a, op, n0, op.Nn, k_begin, k_end);
+  }
   for (int kb = 0; kb < nkb; ++kb) {
     const int s = kb % TC_STAGES;
     char* st = smem + s * TC_STAGE_BYTES;
@@ -197,9 +232,8 @@ __global__ void __launch_bounds__(128, 1) k_gemm_tc(const __grid_constant__ Laun
     }
     __syncthreads();
     if (abort_flag) break;
-    const int64_t k0 = k_begin + (int64_t)kb * TC_BK;
-    stage_block<Op, true>(a, op, st, st + TC_TILE_BYTES, m0, M, k0, k_end);
-    stage_block<Op, false>(a, op, st + 2 * TC_TILE_BYTES, st + 3 * TC_TILE_BYTES, n0, Nn, k0, k_end);
+    sa.store(st, st + TC_TILE_BYTES);
+    sb.store(st + 2 * TC_TILE_BYTES, st + 3 * TC_TILE_BYTES);
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
@@ -216,16 +250,21 @@ __global__ void __launch_bounds__(128, 1) k_gemm_tc(const __grid_constant__ Laun
       }
       mma_commit(smem_u32(&mbar[s]));
     }
-    ++issued;
+    // global loads of the next block are in flight while the tensor cores work on this one
+    if (kb + 1 < nkb) {
+      const int64_t k0 = k_begin + (int64_t)(kb + 1) * TC_BK;
+      sa.load(a, op, m0, op.M, k0, k_end);
+      sb.load(a, op, n0, op.Nn, k0, k_end);
+    }
   }
-  // wait for the last committed group of every stage still in flight
+  // wait for the last committed group of each stage
   if (!abort_flag && nkb > 0) {
     const int last = nkb - 1;
-    const int s = last % TC_STAGES;
-    if (!mbar_wait(smem_u32(&mbar[s]), (uint32_t)((last / TC_STAGES) & 1))) atomicExch(&abort_flag, 1);
+    if (!mbar_wait(smem_u32(&mbar[last % TC_STAGES]), (uint32_t)((last / TC_STAGES) & 1))) atomicExch(&abort_flag, 1);
     if (nkb > 1) {
-      const int prev = nkb - 2, s2 = prev % TC_STAGES;
-      if (!mbar_wait(smem_u32(&mbar[s2]), (uint32_t)((prev / TC_STAGES) & 1))) atomicExch(&abort_flag, 1);
+      const int prev = nkb - 2;
+      if (!mbar_wait(smem_u32(&mbar[prev % TC_STAGES]), (uint32_t)((prev / TC_STAGES) & 1)))
+        atomicExch(&abort_flag, 1);
     }
   }
   tc_fence_before();
@@ -258,7 +297,9 @@ __global__ void __launch_bounds__(128, 1) k_gemm_tc(const __grid_constant__ Laun
 }
 
 template <class Op>
-cudaError_t launch_gemm_tc(const LaunchArgs& a, const Op& op, int64_t M, int Nn, int splits, cudaStream_t s) {
+cudaError_t launch_gemm_tc(const LaunchArgs& a, const Op& op, int splits, cudaStream_t s) {
+  const int64_t M = op.M;
+  const int Nn = (int)op.Nn;
   if (M <= 0 || Nn <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<Op>, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_BYTES);
   if (e != cudaSuccess) return e;

@@ -6,10 +6,17 @@
 //   y[i, o, w, m3] = sum_{p into o} sum_u W_p[u, w] A_p[i, u, m3]
 //   A_p[i, u, m3]  = sum_{e into i} c_p s[e, p] sum_{m1,m2} C_p[m1,m2,m3] x[j, in(p), u, m1] Y(v_e)[m2]
 //
-// A is node-sized state (N x sum_p mul x (2 l3 + 1) floats), aggregated by the receiver-order
-// edge pass below and consumed by the mixing GEMM.  Backward: gW_p = sum_i A_p[i]^T gy_o[i]
-// (split-K GEMM with a fixed-order reduction), G_p[i] = W_p gy_o[i] (GEMM), then one
-// sender-order pass that gives gx (segmented in registers), gs[e, p] and gvec[e].
+// Forward: A is node-sized state (N x sum_p mul (2 l3 + 1) floats), aggregated by the
+// receiver-order edge pass below (which gathers the narrow x rows) and mixed by a tcgen05
+// GEMM per output irrep.  Backward, re-associated on the sender side so that the per-edge
+// gather is the gy row (sum_o mul_out (2 l3 + 1) floats) rather than a per-path gradient
+// state:
+//   xt_p[j, w, m1] = sum_u x[j, in(p), u, m1] W_p[u, w]                       (GEMM)
+//   B_p[j, w, m1]  = sum_{e from j} c_p s[e,p] sum_{m2,m3} C Y[m2] gy[i, o(p), w, m3]   (sender pass)
+//   gs[e, p]       = c_p sum_{w,m1,m2,m3} C xt_p[j,w,m1] Y[m2] gy[i,o(p),w,m3]        (sender pass)
+//   gx[j, a, u, m1] = sum_{p: in(p)=a} sum_w B_p[j, w, m1] W_p[u, w]          (GEMM)
+//   gW_p[u, w]     = sum_j sum_m1 x[j, in(p), u, m1] B_p[j, w, m1]           (split-K GEMM)
+// All sums run in a fixed order: the results are deterministic.
 #pragma once
 #include <algorithm>
 
@@ -101,269 +108,140 @@ __global__ void k_uvw_prep_wt(const __grid_constant__ LaunchArgs a) {
   }
 }
 
-// ---------------------------------------------------------------------------------------
-// SIMT fp32 GEMM  C[m, n] = sum_k A(m, k) B(n, k), tile 64 x 128 x 16, 256 threads, each
-// thread 4 x 8 outputs.  The operand accessors define the three uvw contractions.
-// ---------------------------------------------------------------------------------------
-constexpr int GBM = 64, GBN = 128, GBK = 16;
-
-template <class Op>
-__global__ void __launch_bounds__(256) k_gemm_simt(const __grid_constant__ LaunchArgs a, const Op op) {
-  __shared__ float As[GBK][GBM + 4];
-  __shared__ float Bs[GBK][GBN + 4];
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int64_t m0 = (int64_t)blockIdx.x * GBM;
-  const int n0 = blockIdx.y * GBN;
-  int64_t k_begin, k_end;
-  op.k_range(a, blockIdx.z, k_begin, k_end);
-  float acc[4][8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  for (int64_t k0 = k_begin; k0 < k_end; k0 += GBK) {
-#pragma unroll
-    for (int r = 0; r < (GBM * GBK) / 256; ++r) {
-      const int q = tid + 256 * r;
-      const int mm = q / GBK, kk = q % GBK;
-      const int64_t m = m0 + mm, k = k0 + kk;
-      As[kk][mm] = (m < op.M(a) && k < k_end) ? op.A(a, m, k) : 0.f;
+// Wt[o][w][pl * mul + u] = W[path_of(o, pl)][u][w]  (forward mixing, B operand)
+// is k_uvw_prep_wt above; Wg[a][u][pl * mul_out + w] = W[path_in(a, pl)][u][w] (gx, B operand).
+template <class S>
+__global__ void k_uvw_prep_wg(const __grid_constant__ LaunchArgs a) {
+  const int64_t per_path = (int64_t)a.mul * a.mul_out;
+  const int64_t total = per_path * S::P;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+    int64_t rem = t, base = 0;
+    int ai = 0;
+    for (; ai < S::N_IN; ++ai) {
+      const int64_t sz = (int64_t)S::in_cnt_at(ai) * per_path;
+      if (rem < sz) break;
+      rem -= sz;
+      base += sz;
     }
-#pragma unroll
-    for (int r = 0; r < (GBN * GBK) / 256; ++r) {
-      const int q = tid + 256 * r;
-      const int nn = q / GBK, kk = q % GBK;
-      const int n = n0 + nn;
-      const int64_t k = k0 + kk;
-      Bs[kk][nn] = (n < op.Nn(a) && k < k_end) ? op.B(a, n, k) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < GBK; ++kk) {
-      float av[4], bv[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) bv[j] = Bs[kk][tx + 16 * j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
+    const int K = S::in_cnt_at(ai) * a.mul_out;
+    const int u = (int)(rem / K), kk = (int)(rem % K);
+    const int pl = kk / a.mul_out, w = kk % a.mul_out;
+    const int p = S::path_in_at(ai, pl);
+    a.Wt[base + rem] = a.W[(int64_t)p * per_path + (int64_t)u * a.mul_out + w];
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int64_t m = m0 + ty + 16 * i;
-      const int n = n0 + tx + 16 * j;
-      if (m < op.M(a) && n < op.Nn(a)) op.C(a, blockIdx.z, m, n, acc[i][j]);
-    }
 }
 
-// y_o[(i, m3), w] = sum_{(pl, u)} A_o[(i, m3), (pl, u)] Wt_o[w, (pl, u)]
-template <class S>
-struct MixFwdOp {
-  int o;
-  __device__ int64_t M(const LaunchArgs& a) const { return (int64_t)a.N * S::out_d3_at(o); }
-  __device__ int Nn(const LaunchArgs& a) const { return a.mul_out; }
-  __device__ int K(const LaunchArgs& a) const { return S::out_cnt_at(o) * a.mul; }
-  __device__ void k_range(const LaunchArgs& a, int, int64_t& b, int64_t& e) const { b = 0; e = K(a); }
-  __device__ float A(const LaunchArgs& a, int64_t m, int64_t k) const {
-    return a.A[(int64_t)a.N * a.mul * S::out_cumA_at(o) + m * K(a) + k];
+// Stores a 128 x cols accumulator tile whose rows are (node, m) pairs, m < D, into a feature
+// row layout [node][base + col * D + m]: one contiguous run of cols * D floats per node.
+template <int D>
+__device__ __forceinline__ void store_node_rows(float* out, int64_t row_stride, int64_t base, const float* T,
+                                                int ld, int64_t m0, int64_t M, int n0, int cols) {
+  const int64_t mlast = min(M, m0 + TC_BM) - 1;
+  const int64_t i0 = m0 / D, i1 = mlast / D;
+  const int per_i = cols * D;
+  const int total = (int)(i1 - i0 + 1) * per_i;
+  for (int t = threadIdx.x; t < total; t += blockDim.x) {
+    const int il = t / per_i;
+    const int q = t - il * per_i;
+    const int w = q / D, m = q - w * D;
+    const int64_t i = i0 + il;
+    const int64_t row = i * D + m;
+    if (row < m0 || row > mlast) continue;
+    out[i * row_stride + base + (int64_t)(n0 + w) * D + m] = T[(int)(row - m0) * ld + w];
   }
-  __device__ float B(const LaunchArgs& a, int n, int64_t k) const {
-    int64_t off = 0;
-    for (int q = 0; q < o; ++q) off += (int64_t)S::out_cnt_at(q) * a.mul * a.mul_out;
-    return a.Wt[off + (int64_t)n * K(a) + k];
-  }
-  __device__ void C(const LaunchArgs& a, int, int64_t m, int n, float v) const {
-    const int d3 = S::out_d3_at(o);
-    const int64_t i = m / d3;
-    const int m3 = (int)(m - i * d3);
-    a.y[i * a.out_dim + (int64_t)a.mul_out * S::out_cumY_at(o) + (int64_t)n * d3 + m3] = v;
-  }
-};
+}
 
-// G_o[(i, m3), (pl, u)] = sum_w gy_o[(i, m3), w] W_{p(pl)}[u, w]
-template <class S>
-struct GradStateOp {
-  int o;
-  __device__ int64_t M(const LaunchArgs& a) const { return (int64_t)a.N * S::out_d3_at(o); }
-  __device__ int Nn(const LaunchArgs& a) const { return S::out_cnt_at(o) * a.mul; }
-  __device__ void k_range(const LaunchArgs& a, int, int64_t& b, int64_t& e) const { b = 0; e = a.mul_out; }
-  __device__ float A(const LaunchArgs& a, int64_t m, int64_t k) const {
-    const int d3 = S::out_d3_at(o);
-    const int64_t i = m / d3;
-    const int m3 = (int)(m - i * d3);
-    return a.gy[i * a.out_dim + (int64_t)a.mul_out * S::out_cumY_at(o) + k * d3 + m3];
-  }
-  __device__ float B(const LaunchArgs& a, int n, int64_t k) const {
-    const int pl = n / a.mul, u = n - pl * a.mul;
-    const int p = S::path_of_at(o, pl);
-    return a.W[((int64_t)p * a.mul + u) * a.mul_out + k];
-  }
-  __device__ void C(const LaunchArgs& a, int, int64_t m, int n, float v) const {
-    a.G[(int64_t)a.N * a.mul * S::out_cumA_at(o) + m * Nn(a) + n] = v;
-  }
-};
-
-// part[z][p][u][w] = sum_{(i, m3) in split z} A_o[(i, m3), (pl, u)] gy_o[(i, m3), w]
-template <class S>
-struct GradWOp {
-  int o;
-  __device__ int64_t M(const LaunchArgs& a) const { return (int64_t)S::out_cnt_at(o) * a.mul; }
-  __device__ int Nn(const LaunchArgs& a) const { return a.mul_out; }
-  __device__ void k_range(const LaunchArgs& a, int z, int64_t& b, int64_t& e) const {
-    const int64_t rows = (int64_t)a.N * S::out_d3_at(o);
-    const int64_t chunk = ((rows + a.splits - 1) / a.splits + GBK - 1) / GBK * GBK;
-    b = min(rows, (int64_t)z * chunk);
-    e = min(rows, b + chunk);
-  }
-  __device__ float A(const LaunchArgs& a, int64_t m, int64_t k) const {
-    return a.A[(int64_t)a.N * a.mul * S::out_cumA_at(o) + k * M(a) + m];
-  }
-  __device__ float B(const LaunchArgs& a, int n, int64_t k) const {
-    const int d3 = S::out_d3_at(o);
-    const int64_t i = k / d3;
-    const int m3 = (int)(k - i * d3);
-    return a.gy[i * a.out_dim + (int64_t)a.mul_out * S::out_cumY_at(o) + (int64_t)n * d3 + m3];
-  }
-  __device__ void C(const LaunchArgs& a, int z, int64_t m, int n, float v) const {
-    const int pl = (int)(m / a.mul), u = (int)(m - (int64_t)pl * a.mul);
-    const int p = S::path_of_at(o, pl);
-    a.part[((int64_t)z * S::P + p) * a.mul * a.mul_out + (int64_t)u * a.mul_out + n] = v;
-  }
-};
-
-
-// ---------------------------------------------------------------------------------------
-// The same three contractions for the tcgen05 GEMM (tp_mma.cuh): element accessors, vector
-// accessors for k-contiguous operands, and coalesced tile stores.
-// ---------------------------------------------------------------------------------------
-template <class S>
-struct TcMixFwdOp {           // y_o[(i, m3), w] = sum_k A_o[(i, m3), k] Wt_o[w, k]
-  int o;
+// y_o[(i, m3), w] = sum_k A_o[(i, m3), k] Wt_o[w, k],  k = (pl, u)
+template <int D3>
+struct MixFwdTc {
+  int64_t M, Nn;
+  int K;
+  int64_t ybase;
+  TcOperand A, B;
   static constexpr bool A_KCONTIG = true, B_KCONTIG = true;
-  __device__ int64_t M(const LaunchArgs& a) const { return (int64_t)a.N * S::out_d3_at(o); }
-  __device__ int Nn(const LaunchArgs& a) const { return a.mul_out; }
-  __device__ int K(const LaunchArgs& a) const { return S::out_cnt_at(o) * a.mul; }
-  __device__ void k_range(const LaunchArgs& a, int, int64_t& b, int64_t& e) const { b = 0; e = K(a); }
-  __device__ const float* Abase(const LaunchArgs& a) const { return a.A + (int64_t)a.N * a.mul * S::out_cumA_at(o); }
-  __device__ const float* Bbase(const LaunchArgs& a) const {
-    int64_t off = 0;
-    for (int q = 0; q < o; ++q) off += (int64_t)S::out_cnt_at(q) * a.mul * a.mul_out;
-    return a.Wt + off;
-  }
-  __device__ float A(const LaunchArgs& a, int64_t m, int64_t k) const { return Abase(a)[m * K(a) + k]; }
-  __device__ float B(const LaunchArgs& a, int n, int64_t k) const { return Bbase(a)[(int64_t)n * K(a) + k]; }
-  __device__ float4 A4(const LaunchArgs& a, int64_t m, int64_t k) const {
-    return *reinterpret_cast<const float4*>(Abase(a) + m * K(a) + k);
-  }
-  __device__ float4 B4(const LaunchArgs& a, int n, int64_t k) const {
-    return *reinterpret_cast<const float4*>(Bbase(a) + (int64_t)n * K(a) + k);
-  }
+  __device__ void k_range(const LaunchArgs&, int, int64_t& b, int64_t& e) const { b = 0; e = K; }
+  __device__ int64_t a_row(const LaunchArgs&, int64_t m) const { return m * K; }
+  __device__ int64_t b_row(const LaunchArgs&, int64_t n) const { return n * K; }
   __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0) const {
-    const int d3 = S::out_d3_at(o);
-    const int64_t Mx = M(a);
-    const int64_t i0 = m0 / d3, i1 = (min(Mx, m0 + TC_BM) - 1) / d3;
-    const int cols = min(TC_BN, a.mul_out - n0);
-    const int per_i = cols * d3;
-    const int64_t total = (i1 - i0 + 1) * per_i;
-    for (int64_t t = threadIdx.x; t < total; t += blockDim.x) {
-      const int64_t i = i0 + t / per_i;
-      const int q = (int)(t % per_i);
-      const int w = q / d3, m3 = q - (q / d3) * d3;
-      const int64_t row = i * d3 + m3 - m0;
-      if (row < 0 || row >= TC_BM || i * d3 + m3 >= Mx) continue;
-      a.y[i * a.out_dim + (int64_t)a.mul_out * S::out_cumY_at(o) + (int64_t)(n0 + w) * d3 + m3] = T[row * ld + w];
-    }
+    store_node_rows<D3>(a.y, a.out_dim, ybase, T, ld, m0, M, n0, (int)min((int64_t)TC_BN, Nn - n0));
   }
 };
 
-template <class S>
-struct TcGradStateOp {        // G_o[(i, m3), (pl, u)] = sum_w gy_o[(i, m3), w] W_p[u, w]
-  int o;
-  static constexpr bool A_KCONTIG = false, B_KCONTIG = true;
-  __device__ int64_t M(const LaunchArgs& a) const { return (int64_t)a.N * S::out_d3_at(o); }
-  __device__ int Nn(const LaunchArgs& a) const { return S::out_cnt_at(o) * a.mul; }
-  __device__ void k_range(const LaunchArgs& a, int, int64_t& b, int64_t& e) const { b = 0; e = a.mul_out; }
-  __device__ float A(const LaunchArgs& a, int64_t m, int64_t k) const {
-    const int d3 = S::out_d3_at(o);
-    const int64_t i = m / d3;
-    const int m3 = (int)(m - i * d3);
-    return a.gy[i * a.out_dim + (int64_t)a.mul_out * S::out_cumY_at(o) + k * d3 + m3];
+// xt_a[(j, m1), (pl, w)] = sum_u x[j, a, u, m1] W_{p(a, pl)}[u, w]
+template <int D1>
+struct XtTc {
+  int64_t M, Nn;
+  int K;                 // mul
+  int64_t xbase;         // mul * in_cum[a]
+  int in_dim, mul_out;
+  int64_t wstride;       // mul * mul_out
+  int paths[kMaxPaths];
+  float* out;            // region a of the xt buffer, row-major [M][Nn]
+  TcOperand A, B;
+  static constexpr bool A_KCONTIG = (D1 == 1), B_KCONTIG = false;
+  __device__ void k_range(const LaunchArgs&, int, int64_t& b, int64_t& e) const { b = 0; e = K; }
+  __device__ int64_t a_row(const LaunchArgs&, int64_t m) const {
+    const int64_t j = m / D1;
+    return j * in_dim + xbase + (m - j * D1);
   }
-  __device__ float4 A4(const LaunchArgs& a, int64_t m, int64_t k) const {
-    return make_float4(A(a, m, k), A(a, m, k + 1), A(a, m, k + 2), A(a, m, k + 3));
+  __device__ int64_t b_row(const LaunchArgs&, int64_t n) const {
+    const int pl = (int)(n / mul_out);
+    return paths[pl] * wstride + (n - (int64_t)pl * mul_out);
   }
-  __device__ const float* Brow(const LaunchArgs& a, int n) const {
-    const int pl = n / a.mul, u = n - pl * a.mul;
-    return a.W + ((int64_t)S::path_of_at(o, pl) * a.mul + u) * a.mul_out;
-  }
-  __device__ float B(const LaunchArgs& a, int n, int64_t k) const { return Brow(a, n)[k]; }
-  __device__ float4 B4(const LaunchArgs& a, int n, int64_t k) const {
-    return *reinterpret_cast<const float4*>(Brow(a, n) + k);
-  }
-  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0) const {
-    const int64_t Mx = M(a);
-    const int Kn = Nn(a);
-    const int cols = min(TC_BN, Kn - n0);
-    float* G = a.G + (int64_t)a.N * a.mul * S::out_cumA_at(o);
+  __device__ void store_tile(const LaunchArgs&, int, const float* T, int ld, int64_t m0, int n0) const {
+    const int cols = (int)min((int64_t)TC_BN, Nn - n0);
     for (int t = threadIdx.x; t < TC_BM * cols; t += blockDim.x) {
       const int r = t / cols, c = t - r * cols;
-      if (m0 + r < Mx) G[(m0 + r) * Kn + n0 + c] = T[r * ld + c];
+      if (m0 + r < M) out[(m0 + r) * Nn + n0 + c] = T[r * ld + c];
     }
   }
 };
 
-template <class S>
-struct TcGradWOp {            // part[z][p][u][w] = sum_{(i, m3) in split z} A_o[(i, m3), (pl, u)] gy_o[(i, m3), w]
-  int o;
+// gx[j, a, u, m1] = sum_k B_a[(j, m1), k] Wg_a[u, k],  k = (pl, w)
+template <int D1>
+struct GxTc {
+  int64_t M, Nn;
+  int K;
+  int64_t xbase;
+  TcOperand A, B;
+  static constexpr bool A_KCONTIG = true, B_KCONTIG = true;
+  __device__ void k_range(const LaunchArgs&, int, int64_t& b, int64_t& e) const { b = 0; e = K; }
+  __device__ int64_t a_row(const LaunchArgs&, int64_t m) const { return m * K; }
+  __device__ int64_t b_row(const LaunchArgs&, int64_t n) const { return n * K; }
+  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0) const {
+    store_node_rows<D1>(a.gx, a.in_dim, xbase, T, ld, m0, M, n0, (int)min((int64_t)TC_BN, Nn - n0));
+  }
+};
+
+// part[z][p][u][w] = sum_{(j, m1) in split z} x[j, a, u, m1] B_a[(j, m1), (pl, w)]
+template <int D1>
+struct GwTc {
+  int64_t M, Nn;         // mul, cnt_a * mul_out
+  int64_t rows;          // N * d1
+  int splits, mul_out, P;
+  int64_t wstride;
+  int paths[kMaxPaths];
+  TcOperand A, B;
   static constexpr bool A_KCONTIG = false, B_KCONTIG = false;
-  __device__ int64_t M(const LaunchArgs& a) const { return (int64_t)S::out_cnt_at(o) * a.mul; }
-  __device__ int Nn(const LaunchArgs& a) const { return a.mul_out; }
-  __device__ void k_range(const LaunchArgs& a, int z, int64_t& b, int64_t& e) const {
-    const int64_t rows = (int64_t)a.N * S::out_d3_at(o);
-    const int64_t chunk = ((rows + a.splits - 1) / a.splits + TC_BK - 1) / TC_BK * TC_BK;
+  __device__ void k_range(const LaunchArgs&, int z, int64_t& b, int64_t& e) const {
+    const int64_t chunk = ((rows + splits - 1) / splits + TC_BK - 1) / TC_BK * TC_BK;
     b = min(rows, (int64_t)z * chunk);
     e = min(rows, b + chunk);
   }
-  __device__ float A(const LaunchArgs& a, int64_t m, int64_t k) const {
-    return a.A[(int64_t)a.N * a.mul * S::out_cumA_at(o) + k * M(a) + m];
-  }
-  __device__ float4 A4(const LaunchArgs& a, int64_t m, int64_t k) const {
-    return make_float4(A(a, m, k), A(a, m, k + 1), A(a, m, k + 2), A(a, m, k + 3));
-  }
-  __device__ float B(const LaunchArgs& a, int n, int64_t k) const {
-    const int d3 = S::out_d3_at(o);
-    const int64_t i = k / d3;
-    const int m3 = (int)(k - i * d3);
-    return a.gy[i * a.out_dim + (int64_t)a.mul_out * S::out_cumY_at(o) + (int64_t)n * d3 + m3];
-  }
-  __device__ float4 B4(const LaunchArgs& a, int n, int64_t k) const {
-    return make_float4(B(a, n, k), B(a, n, k + 1), B(a, n, k + 2), B(a, n, k + 3));
-  }
+  __device__ int64_t a_row(const LaunchArgs&, int64_t m) const { return m * D1; }
+  __device__ int64_t b_row(const LaunchArgs&, int64_t n) const { return n; }
   __device__ void store_tile(const LaunchArgs& a, int z, const float* T, int ld, int64_t m0, int n0) const {
-    const int64_t Mx = M(a);
-    const int cols = min(TC_BN, a.mul_out - n0);
+    const int cols = (int)min((int64_t)TC_BN, Nn - n0);
     for (int t = threadIdx.x; t < TC_BM * cols; t += blockDim.x) {
       const int r = t / cols, c = t - r * cols;
-      const int64_t m = m0 + r;
-      if (m >= Mx) continue;
-      const int pl = (int)(m / a.mul), u = (int)(m - (int64_t)pl * a.mul);
-      const int p = S::path_of_at(o, pl);
-      a.part[((int64_t)z * S::P + p) * a.mul * a.mul_out + (int64_t)u * a.mul_out + n0 + c] = T[r * ld + c];
+      const int64_t u = m0 + r;
+      if (u >= M) continue;
+      const int n = n0 + c;
+      const int pl = n / mul_out, w = n - pl * mul_out;
+      a.part[((int64_t)z * P + paths[pl]) * wstride + u * mul_out + w] = T[r * ld + c];
     }
   }
 };
-
-// The tensor-core path reads k-contiguous operand rows (A, G, Wt in the workspace and the
-// caller's W) as float4: it needs multiplicities divisible by 4 and a 16-byte aligned W.
-inline bool tc_usable(const LaunchArgs& a) {
-  return a.use_tc && a.mul % 4 == 0 && a.mul_out % 4 == 0 && (reinterpret_cast<uintptr_t>(a.W) & 15u) == 0;
-}
 
 // gW[idx] = sum_z part[z][idx] in split order (deterministic)
 static __global__ void k_reduce_splits(const float* __restrict__ part, int splits, int64_t n, float* gW) {
@@ -375,30 +253,31 @@ static __global__ void k_reduce_splits(const float* __restrict__ part, int split
 }
 
 // ---------------------------------------------------------------------------------------
-// Sender pass: gx[j] (segmented), gs[e, p] and gvec[e] (channel sums across all slices of a
-// row, which share one CTA).  grid = N, block = 32 * NSL (one edge phase).
+// Sender pass: B (per sender, per path), gs[e, p] and gvec[e]; lane = output channel w.
+// gs and gvec are channel sums across all slices of the sender, which share one CTA.
+// grid = N, block = 32 * NSL.
 // ---------------------------------------------------------------------------------------
 template <class S, bool GVEC, int NSL>
 __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant__ LaunchArgs a) {
   extern __shared__ float smem[];
-  constexpr int NV = S::P + 4;   // per edge and slice: P gs partials, 3 gvec partials (+ degree sum)
+  constexpr int NV = S::P + 4;   // per edge and slice: P gs partials, 3 gvec partials, degree sum
   const int lane = threadIdx.x & 31;
   const int sl = threadIdx.x >> 5;
   const int node = blockIdx.x;
   const int c = sl * 32 + lane;
-  const bool act = c < a.mul;
+  const bool act = c < a.mul_out;
   int q0 = __ldg(a.colptr + node), q1 = __ldg(a.colptr + node + 1);
   if (a.check) {
     q0 = max(0, min(q0, a.E));
     q1 = max(q0, min(q1, a.E));
   }
-  float x[S::IN_PC], gx[S::IN_PC];
+  float xt[S::XT_PC], bt[S::XT_PC];
 #pragma unroll
-  for (int k = 0; k < S::IN_PC; ++k) {
-    gx[k] = 0.f;
-    x[k] = 0.f;
+  for (int k = 0; k < S::XT_PC; ++k) {
+    bt[k] = 0.f;
+    xt[k] = 0.f;
   }
-  if (act) S::load_in(a.x + (int64_t)node * a.in_dim, a.mul, c, x);
+  if (act) S::load_xt(a.A, a.N, a.mul_out, node, c, xt);
   float* slot = smem;   // [32 edges][NSL][NV]
 
   for (int base = q0; base < q1; base += 32) {
@@ -440,9 +319,9 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
 #pragma unroll
         for (int p = 0; p < S::P; ++p) s[p] = __ldg(srow + p) * (a.has_coeff ? a.coeff[p] : 1.f);
         if (act) {
-          float g[S::A_PC];
-          S::load_uvw(a.G, a.N, a.mul, i, c, g);
-          S::template uvw_bwd<GVEC>(x, Y, s, g, gx, gs, gY);
+          float gyv[S::OUT_PC];
+          S::load_out(a.gy + (int64_t)i * a.out_dim, a.mul_out, c, gyv);
+          S::template uvw_send<GVEC>(xt, Y, s, gyv, bt, gs, gY);
         }
       }
       float h0 = 0.f, h1 = 0.f, h2 = 0.f, sdeg = 0.f;
@@ -500,19 +379,30 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
     }
     __syncthreads();
   }
-  if (act && a.gx) S::store_in(a.gx + (int64_t)node * a.in_dim, a.mul, c, gx);
+  if (act) S::store_xt(a.G, a.N, a.mul_out, node, c, bt);
 }
 
 // ---------------------------------------------------------------------------------------
 // Host sequences
 // ---------------------------------------------------------------------------------------
-template <class Op>
-static cudaError_t launch_gemm(const LaunchArgs& a, const Op& op, int64_t M, int Nn, int splits, cudaStream_t s) {
-  if (M <= 0 || Nn <= 0) return cudaSuccess;
-  dim3 grid((unsigned)((M + GBM - 1) / GBM), (unsigned)((Nn + GBN - 1) / GBN), (unsigned)splits);
-  k_gemm_simt<Op><<<grid, 256, 0, s>>>(a, op);
-  count_launches(1);
-  return cudaGetLastError();
+inline TcOperand tc_operand(const float* base, int kd, int64_t ks1, int64_t ks2, bool vec4) {
+  TcOperand o;
+  o.base = base;
+  o.kd = kd;
+  o.ks1 = ks1;
+  o.ks2 = ks2;
+  o.vec4 = vec4 && ((reinterpret_cast<uintptr_t>(base) & 15u) == 0);
+  return o;
+}
+
+template <template <int> class Op, class F>
+cudaError_t with_d(int d, F&& f) {
+  switch (d) {
+    case 1: return f(Op<1>{});
+    case 3: return f(Op<3>{});
+    case 5: return f(Op<5>{});
+    default: return f(Op<7>{});
+  }
 }
 
 template <class S>
@@ -531,11 +421,21 @@ cudaError_t launch_uvw_fwd(const LaunchArgs& a, cudaStream_t s) {
   k_uvw_prep_wt<S><<<64, 256, 0, s>>>(a);
   count_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const bool tc = tc_usable(a);
+  int64_t wt_off = 0;
   for (int o = 0; o < S::N_OUT; ++o) {
-    const int64_t M = (int64_t)a.N * S::out_d3_at(o);
-    e = tc ? launch_gemm_tc(a, TcMixFwdOp<S>{o}, M, a.mul_out, 1, s) : launch_gemm(a, MixFwdOp<S>{o}, M, a.mul_out, 1, s);
+    const int d3 = S::out_d3_at(o), cnt = S::out_cnt_at(o);
+    const int K = cnt * a.mul;
+    e = with_d<MixFwdTc>(d3, [&](auto op) {
+      op.M = (int64_t)a.N * d3;
+      op.Nn = a.mul_out;
+      op.K = K;
+      op.ybase = (int64_t)a.mul_out * S::out_cumY_at(o);
+      op.A = tc_operand(a.A + (int64_t)a.N * a.mul * S::out_cumA_at(o), 0, 1, 0, K % 4 == 0);
+      op.B = tc_operand(a.Wt + wt_off, 0, 1, 0, K % 4 == 0);
+      return launch_gemm_tc(a, op, 1, s);
+    });
     if (e != cudaSuccess) return e;
+    wt_off += (int64_t)K * a.mul_out;
   }
   return cudaSuccess;
 }
@@ -543,28 +443,33 @@ cudaError_t launch_uvw_fwd(const LaunchArgs& a, cudaStream_t s) {
 template <class S>
 cudaError_t launch_uvw_bwd(const LaunchArgs& a, cudaStream_t s) {
   if (a.N == 0) return cudaSuccess;
-  cudaError_t e = launch_uvw_edge<S>(a, s);
-  if (e != cudaSuccess) return e;
-  const bool tc = tc_usable(a);
-  for (int o = 0; o < S::N_OUT; ++o) {
-    const int64_t M = (int64_t)a.N * S::out_d3_at(o);
-    const int K = S::out_cnt_at(o) * a.mul;
-    e = tc ? launch_gemm_tc(a, TcGradStateOp<S>{o}, M, K, 1, s) : launch_gemm(a, GradStateOp<S>{o}, M, K, 1, s);
+  cudaError_t e;
+  k_uvw_prep_wg<S><<<64, 256, 0, s>>>(a);
+  count_launches(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t wstride = (int64_t)a.mul * a.mul_out;
+  // xt = x W per input irrep
+  for (int ai = 0; ai < S::N_IN; ++ai) {
+    const int d1 = S::in_d1_at(ai), cnt = S::in_cnt_at(ai);
+    if (cnt == 0) continue;
+    e = with_d<XtTc>(d1, [&](auto op) {
+      op.M = (int64_t)a.N * d1;
+      op.Nn = (int64_t)cnt * a.mul_out;
+      op.K = a.mul;
+      op.xbase = (int64_t)a.mul * S::in_cum_at(ai);
+      op.in_dim = a.in_dim;
+      op.mul_out = a.mul_out;
+      op.wstride = wstride;
+      for (int pl = 0; pl < cnt; ++pl) op.paths[pl] = S::path_in_at(ai, pl);
+      op.out = a.A + (int64_t)a.N * a.mul_out * S::in_cumX_at(ai);
+      op.A = tc_operand(a.x, 0, d1, 0, d1 == 1 && a.in_dim % 4 == 0 && op.xbase % 4 == 0);
+      op.B = tc_operand(a.W, 0, a.mul_out, 0, false);
+      return launch_gemm_tc(a, op, 1, s);
+    });
     if (e != cudaSuccess) return e;
-    if (a.gW) {
-      e = tc ? launch_gemm_tc(a, TcGradWOp<S>{o}, K, a.mul_out, a.splits, s)
-             : launch_gemm(a, GradWOp<S>{o}, K, a.mul_out, a.splits, s);
-      if (e != cudaSuccess) return e;
-    }
   }
-  if (a.gW) {
-    const int64_t n = (int64_t)S::P * a.mul * a.mul_out;
-    k_reduce_splits<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, s>>>(a.part, a.splits, n, a.gW);
-    count_launches(1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  if (!a.gx && !a.gw && !a.gvec) return cudaSuccess;
-  const int nsl = a.n_slices <= 1 ? 1 : (a.n_slices == 2 ? 2 : 4);
+  // sender pass: B, gs, gvec
+  const int nsl = (a.mul_out + 31) / 32 <= 1 ? 1 : ((a.mul_out + 31) / 32 == 2 ? 2 : 4);
   const size_t sm = (size_t)32 * nsl * (S::P + 4) * sizeof(float);
   const bool gv = a.gvec != nullptr;
 #define TP_UVW_SEND(G, NS) k_uvw_send<S, G, NS><<<(unsigned)a.N, 32 * NS, sm, s>>>(a)
@@ -573,7 +478,50 @@ cudaError_t launch_uvw_bwd(const LaunchArgs& a, cudaStream_t s) {
   else { if (gv) TP_UVW_SEND(true, 4); else TP_UVW_SEND(false, 4); }
 #undef TP_UVW_SEND
   count_launches(1);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  int64_t wg_off = 0;
+  for (int ai = 0; ai < S::N_IN; ++ai) {
+    const int d1 = S::in_d1_at(ai), cnt = S::in_cnt_at(ai);
+    if (cnt == 0) continue;
+    const int K = cnt * a.mul_out;
+    const float* Bbuf = a.G + (int64_t)a.N * a.mul_out * S::in_cumX_at(ai);
+    if (a.gx) {
+      e = with_d<GxTc>(d1, [&](auto op) {
+        op.M = (int64_t)a.N * d1;
+        op.Nn = a.mul;
+        op.K = K;
+        op.xbase = (int64_t)a.mul * S::in_cum_at(ai);
+        op.A = tc_operand(Bbuf, 0, 1, 0, K % 4 == 0);
+        op.B = tc_operand(a.Wt + wg_off, 0, 1, 0, K % 4 == 0);
+        return launch_gemm_tc(a, op, 1, s);
+      });
+      if (e != cudaSuccess) return e;
+    }
+    if (a.gW) {
+      e = with_d<GwTc>(d1, [&](auto op) {
+        op.M = a.mul;
+        op.Nn = (int64_t)cnt * a.mul_out;
+        op.rows = (int64_t)a.N * d1;
+        op.splits = a.splits;
+        op.mul_out = a.mul_out;
+        op.P = S::P;
+        op.wstride = wstride;
+        for (int pl = 0; pl < cnt; ++pl) op.paths[pl] = S::path_in_at(ai, pl);
+        op.A = tc_operand(a.x + (int64_t)a.mul * S::in_cum_at(ai), d1, a.in_dim, 1, false);
+        op.B = tc_operand(Bbuf, 0, (int64_t)cnt * a.mul_out, 0, false);
+        return launch_gemm_tc(a, op, a.splits, s);
+      });
+      if (e != cudaSuccess) return e;
+    }
+    wg_off += (int64_t)a.mul * K;
+  }
+  if (a.gW) {
+    const int64_t n = (int64_t)S::P * wstride;
+    k_reduce_splits<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, s>>>(a.part, a.splits, n, a.gW);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace tp
