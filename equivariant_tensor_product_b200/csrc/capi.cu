@@ -130,16 +130,6 @@ WsLayout ws_layout(int64_t N, int64_t E) {
   return L;
 }
 
-// Tuning override read once from the environment: TP_TUNE_PREFETCH=0/1 forces the register
-// double buffering of edge gathers off/on (default: per-spec heuristic).
-int tune_prefetch() {
-  static const int v = [] {
-    const char* e = std::getenv("TP_TUNE_PREFETCH");
-    return (e && (e[0] == '0' || e[0] == '1')) ? e[0] - '0' : -1;
-  }();
-  return v;
-}
-
 // uvw regions after the transpose region: A | G | Wt | part (floats, 256-byte aligned)
 constexpr int kUvwSplits = 64;
 struct UvwLayout {
@@ -196,7 +186,6 @@ LaunchArgs base_args(tp_plan_t plan, int64_t N, int64_t E) {
   a.n_slices = (plan->mul_in + 31) / 32;
   a.has_coeff = plan->has_coeff;
   a.check = (plan->flags & TP_FLAG_CHECK_INDICES) ? 1 : 0;
-  a.prefetch = tune_prefetch();
 
 
   std::memcpy(a.coeff, plan->coeff, sizeof(a.coeff));

@@ -234,8 +234,9 @@ def _monomials_code(maxdeg: int, indent="    ") -> List[str]:
 
 
 class Spec:
-    def __init__(self, name, in_ls, sh_ls, out_ls, paths):
+    def __init__(self, name, in_ls, sh_ls, out_ls, paths, fast_muls=()):
         self.name = name
+        self.fast_muls = list(fast_muls) + [0] * (2 - len(fast_muls))
         self.in_ls, self.sh_ls, self.out_ls = list(in_ls), list(sh_ls), list(out_ls)
         self.paths = [tuple(p) for p in paths]
         self.in_d = [2 * l + 1 for l in self.in_ls]
@@ -735,7 +736,9 @@ def gen_spec_header(spec: Spec) -> str:
          f"  static constexpr int P = {spec.P};",
          f"  static constexpr int A_PC = {spec.A_PC};",
          f"  static constexpr int LMAX_SH = {spec.LMAX_SH};",
-         f"  static constexpr int NNZ = {spec.nnz_total()};"]
+         f"  static constexpr int NNZ = {spec.nnz_total()};",
+         f"  static constexpr int FAST_MUL0 = {spec.fast_muls[0]};",
+         f"  static constexpr int FAST_MUL1 = {spec.fast_muls[1]};"]
     L += _lines_load("load_in", len(spec.in_ls), spec.in_d, spec.in_cum, "x")
     L += _lines_store("store_in", len(spec.in_ls), spec.in_d, spec.in_cum, "x")
     L += _lines_load("load_out", len(spec.out_ls), spec.out_d, spec.out_cum, "y")
@@ -790,7 +793,9 @@ def builtin_specs() -> List[Spec]:
         reach = sorted({o for _, _, o in paths})
         remap = {o: k for k, o in enumerate(reach)}
         paths = [(a, b, remap[o]) for a, b, o in paths]
-        specs.append(Spec(f"full_l{L}", ins, ins, [outs[o][0] for o in reach], paths))
+        # channel counts compiled as constants: 32 and 128 for lmax 2, 32 and 64 for lmax 3
+        fast = {1: (), 2: (32, 128), 3: (32, 64)}[L]
+        specs.append(Spec(f"full_l{L}", ins, ins, [outs[o][0] for o in reach], paths, fast))
     return specs
 
 

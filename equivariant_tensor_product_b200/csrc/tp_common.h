@@ -28,7 +28,6 @@ struct LaunchArgs {
   int n_slices;        // 32-channel slices per row = ceil(mul / 32)
   int has_coeff;       // path coefficients differ from 1
   int check;           // bounds-check indices and report through *err
-  int prefetch;        // -1: heuristic; 0/1: force register double-buffering of edge gathers
   const int32_t* rowptr;
   const int32_t* src;
   const int32_t* colptr;

@@ -60,28 +60,17 @@ __device__ __forceinline__ void report(const LaunchArgs& a, int code) {
 }
 
 template <int P>
-__device__ __forceinline__ void load_path_weights(const LaunchArgs& a, int e, int c, float (&w)[P]) {
-  const float* row = a.w + (int64_t)e * a.nw + c;
-#pragma unroll
-  for (int p = 0; p < P; ++p) w[p] = __ldg(row + (int64_t)p * a.mul);
-  if (a.has_coeff) {
-#pragma unroll
-    for (int p = 0; p < P; ++p) w[p] *= a.coeff[p];
-  }
-}
-
-template <int P>
-__device__ __forceinline__ void load_path_weights_from(const LaunchArgs& a, const float* base, int e,
-                                                       int c, float (&w)[P]) {
+__device__ __forceinline__ void load_path_weights(const LaunchArgs& a, const float* base, int nw, int mul,
+                                                  bool has_coeff, int e, int c, float (&w)[P]) {
   if (base == nullptr) {
 #pragma unroll
     for (int p = 0; p < P; ++p) w[p] = 0.f;
     return;
   }
-  const float* row = base + (int64_t)e * a.nw + c;
+  const float* row = base + (int64_t)e * nw + c;
 #pragma unroll
-  for (int p = 0; p < P; ++p) w[p] = __ldg(row + (int64_t)p * a.mul);
-  if (a.has_coeff) {
+  for (int p = 0; p < P; ++p) w[p] = __ldg(row + p * mul);
+  if (has_coeff) {
 #pragma unroll
     for (int p = 0; p < P; ++p) w[p] *= a.coeff[p];
   }
@@ -111,17 +100,25 @@ __device__ __forceinline__ void reduce_phases(float (&acc)[N], float* smem, int 
 // ---------------------------------------------------------------------------------------
 // Forward, uvu, receiver order.  grid = N * n_slices, block = 32 * split.
 // ---------------------------------------------------------------------------------------
-template <class S, bool PF>
+template <class S, bool PF, int MUL, bool FAST>
 __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__ LaunchArgs a) {
+  constexpr bool kFast = FAST;
+  const int mul = MUL ? MUL : a.mul;
+  const int nw = MUL ? S::P * MUL : a.nw;
+  const int in_dim = MUL ? S::IN_PC * MUL : a.in_dim;
+  const int out_dim = MUL ? S::OUT_PC * MUL : a.out_dim;
+  const bool check = !kFast && a.check;
+  const bool has_coeff = !kFast && a.has_coeff;
+  (void)nw; (void)in_dim; (void)out_dim; (void)has_coeff;
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
   const int phase = threadIdx.x >> 5;
   const int row = blockIdx.x / a.n_slices;
   const int sl = blockIdx.x - row * a.n_slices;
   const int c = sl * 32 + lane;
-  const bool act = c < a.mul;
+  const bool act = c < mul;
   int e0 = __ldg(a.rowptr + row), e1 = __ldg(a.rowptr + row + 1);
-  if (a.check) {  // never read outside [0, E) whatever rowptr holds
+  if (check) {  // never read outside [0, E) whatever rowptr holds
     e0 = max(0, min(e0, a.E));
     e1 = max(e0, min(e1, a.E));
   }
@@ -139,7 +136,7 @@ __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__
       vx = __ldg(a.vec + 3 * (int64_t)my_e);
       vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
       vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
-      if (a.check && (unsigned)my_j >= (unsigned)a.N) {
+      if (check && (unsigned)my_j >= (unsigned)a.N) {
         report(a, kDevBadSrc);
         vx = vy = vz = 0.f;
         my_j = -1;
@@ -150,8 +147,8 @@ __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__
     auto fetch = [&](int k, float (&xx)[S::IN_PC], float (&ww)[S::P]) {
       const int j = __shfl_sync(kFull, my_j, k);
       if (act && j >= 0) {
-        S::load_in(a.x + (int64_t)j * a.in_dim, a.mul, c, xx);
-        load_path_weights(a, base + k * st, c, ww);
+        S::load_in(a.x + (int64_t)j * in_dim, mul, c, xx);
+        load_path_weights(a, a.w, nw, mul, has_coeff, base + k * st, c, ww);
       }
     };
     auto compute = [&](int k, const float (&xx)[S::IN_PC], const float (&ww)[S::P]) {
@@ -192,15 +189,15 @@ __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__
         float Y[S::NSH];
         S::sh(rx, ry, rz, Y);
         if (act) {
-          S::load_in(a.x + (int64_t)j * a.in_dim, a.mul, c, xa);
-          load_path_weights(a, e, c, wa);
+          S::load_in(a.x + (int64_t)j * in_dim, mul, c, xa);
+          load_path_weights(a, a.w, nw, mul, has_coeff, e, c, wa);
           S::fwd(xa, Y, wa, acc);
         }
       }
     }
   }
   reduce_phases(acc, smem, phase, st, lane, 0, 1);
-  if (phase == 0 && act) S::store_out(a.y + (int64_t)row * a.out_dim, a.mul, c, acc);
+  if (phase == 0 && act) S::store_out(a.y + (int64_t)row * out_dim, mul, c, acc);
 }
 
 
@@ -213,8 +210,16 @@ __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__
 // GVEC=false: grid = N * n_slices, block = 32*split (slices independent).
 // GVEC=true : grid = N, block = 32*split*NSL (all slices of a row in one CTA).
 // ---------------------------------------------------------------------------------------
-template <class S, bool GVEC, int NSL, bool PF>
+template <class S, bool GVEC, int NSL, bool PF, int MUL, bool FAST>
 __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__ LaunchArgs a) {
+  constexpr bool kFast = FAST;
+  const int mul = MUL ? MUL : a.mul;
+  const int nw = MUL ? S::P * MUL : a.nw;
+  const int in_dim = MUL ? S::IN_PC * MUL : a.in_dim;
+  const int out_dim = MUL ? S::OUT_PC * MUL : a.out_dim;
+  const bool check = !kFast && a.check;
+  const bool has_coeff = !kFast && a.has_coeff;
+  (void)nw; (void)in_dim; (void)out_dim; (void)has_coeff;
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
@@ -229,9 +234,9 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
     sl = blockIdx.x - node * a.n_slices;
   }
   const int c = sl * 32 + lane;
-  const bool act = c < a.mul;
+  const bool act = c < mul;
   int q0 = __ldg(a.colptr + node), q1 = __ldg(a.colptr + node + 1);
-  if (a.check) {
+  if (check) {
     q0 = max(0, min(q0, a.E));
     q1 = max(q0, min(q1, a.E));
   }
@@ -240,7 +245,7 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
   float gx[S::IN_PC];
 #pragma unroll
   for (int k = 0; k < S::IN_PC; ++k) gx[k] = 0.f;
-  if (act) S::load_in(a.x + (int64_t)node * a.in_dim, a.mul, c, x);
+  if (act) S::load_in(a.x + (int64_t)node * in_dim, mul, c, x);
   else {
 #pragma unroll
     for (int k = 0; k < S::IN_PC; ++k) x[k] = 0.f;
@@ -254,7 +259,7 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
     float vx = 0.f, vy = 0.f, vz = 0.f;
     if (my_q < q1) {
       my_e = __ldg(a.perm + my_q);
-      if (a.check && (unsigned)my_e >= (unsigned)a.E) {
+      if (check && (unsigned)my_e >= (unsigned)a.E) {
         report(a, kDevBadPerm);
         my_e = -1;
       } else {
@@ -303,8 +308,8 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
       const int e = __shfl_sync(kFull, my_e, k);
       const int i = __shfl_sync(kFull, my_i, k);
       if (act && e >= 0) {
-        S::load_out(a.gy + (int64_t)i * a.out_dim, a.mul, c, gg);
-        load_path_weights(a, e, c, ww);
+        S::load_out(a.gy + (int64_t)i * out_dim, mul, c, gg);
+        load_path_weights(a, a.w, nw, mul, has_coeff, e, c, ww);
       }
     };
     auto compute = [&](int k, const float (&gyv)[S::OUT_PC], const float (&w)[S::P]) {
@@ -323,9 +328,9 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
         float gw[S::P];
         S::template bwd<GVEC>(x, Y, w, gyv, gx, gw, gY);
         if (a.gw) {
-          float* row = a.gw + (int64_t)e * a.nw + c;
+          float* row = a.gw + (int64_t)e * nw + c;
 #pragma unroll
-          for (int p = 0; p < S::P; ++p) row[(int64_t)p * a.mul] = a.has_coeff ? gw[p] * a.coeff[p] : gw[p];
+          for (int p = 0; p < S::P; ++p) row[(int64_t)p * mul] = has_coeff ? gw[p] * a.coeff[p] : gw[p];
         }
       }
       if constexpr (GVEC) gvec_edge(k, e, rx, ry, rz, ir, Y, gY);
@@ -358,14 +363,14 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
 #pragma unroll
         for (int m = 0; m < S::NSH; ++m) gY[m] = 0.f;
         if (act && e >= 0) {
-          S::load_out(a.gy + (int64_t)i * a.out_dim, a.mul, c, ga);
-          load_path_weights(a, e, c, wa);
+          S::load_out(a.gy + (int64_t)i * out_dim, mul, c, ga);
+          load_path_weights(a, a.w, nw, mul, has_coeff, e, c, wa);
           float gw[S::P];
           S::template bwd<GVEC>(x, Y, wa, ga, gx, gw, gY);
           if (a.gw) {
-            float* row = a.gw + (int64_t)e * a.nw + c;
+            float* row = a.gw + (int64_t)e * nw + c;
 #pragma unroll
-            for (int p = 0; p < S::P; ++p) row[(int64_t)p * a.mul] = a.has_coeff ? gw[p] * a.coeff[p] : gw[p];
+            for (int p = 0; p < S::P; ++p) row[(int64_t)p * mul] = has_coeff ? gw[p] * a.coeff[p] : gw[p];
           }
         }
         if constexpr (GVEC) gvec_edge(k, e, rx, ry, rz, ir, Y, gY);
@@ -394,23 +399,31 @@ __global__ void __launch_bounds__(kMaxThreads) k_bwd_uvu(const __grid_constant__
     }
   }
   reduce_phases(gx, smem, phase, st, lane, GVEC ? sl : 0, GVEC ? NSL : 1);
-  if (phase == 0 && act && a.gx) S::store_in(a.gx + (int64_t)node * a.in_dim, a.mul, c, gx);
+  if (phase == 0 && act && a.gx) S::store_in(a.gx + (int64_t)node * in_dim, mul, c, gx);
 }
 
 // ---------------------------------------------------------------------------------------
 // Double backward, receiver pass: g_gy[i] = sum_e TP(ggx; Y, w) + TP(x; Y, ggw) + TP(x; dY[ggvec], w)
 // ---------------------------------------------------------------------------------------
-template <class S>
+template <class S, int MUL, bool FAST>
 __global__ void __launch_bounds__(kMaxThreads) k_dbwd_recv(const __grid_constant__ LaunchArgs a) {
+  constexpr bool kFast = FAST;
+  const int mul = MUL ? MUL : a.mul;
+  const int nw = MUL ? S::P * MUL : a.nw;
+  const int in_dim = MUL ? S::IN_PC * MUL : a.in_dim;
+  const int out_dim = MUL ? S::OUT_PC * MUL : a.out_dim;
+  const bool check = !kFast && a.check;
+  const bool has_coeff = !kFast && a.has_coeff;
+  (void)nw; (void)in_dim; (void)out_dim; (void)has_coeff;
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
   const int phase = threadIdx.x >> 5;
   const int row = blockIdx.x / a.n_slices;
   const int sl = blockIdx.x - row * a.n_slices;
   const int c = sl * 32 + lane;
-  const bool act = c < a.mul;
+  const bool act = c < mul;
   int e0 = __ldg(a.rowptr + row), e1 = __ldg(a.rowptr + row + 1);
-  if (a.check) {  // never read outside [0, E) whatever rowptr holds
+  if (check) {  // never read outside [0, E) whatever rowptr holds
     e0 = max(0, min(e0, a.E));
     e1 = max(e0, min(e1, a.E));
   }
@@ -433,7 +446,7 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_recv(const __grid_constant
         dy = __ldg(a.ggvec + 3 * (int64_t)my_e + 1);
         dz = __ldg(a.ggvec + 3 * (int64_t)my_e + 2);
       }
-      if (a.check && (unsigned)my_j >= (unsigned)a.N) {
+      if (check && (unsigned)my_j >= (unsigned)a.N) {
         report(a, kDevBadSrc);
         my_j = -1;
       }
@@ -465,28 +478,36 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_recv(const __grid_constant
       }
       if (act) {
         float x[S::IN_PC], ggx[S::IN_PC];
-        S::load_in(a.x + (int64_t)j * a.in_dim, a.mul, c, x);
-        if (a.ggx) S::load_in(a.ggx + (int64_t)j * a.in_dim, a.mul, c, ggx);
+        S::load_in(a.x + (int64_t)j * in_dim, mul, c, x);
+        if (a.ggx) S::load_in(a.ggx + (int64_t)j * in_dim, mul, c, ggx);
         else {
 #pragma unroll
           for (int m = 0; m < S::IN_PC; ++m) ggx[m] = 0.f;
         }
         float w[S::P], ggw[S::P];
-        load_path_weights(a, e, c, w);
-        load_path_weights_from(a, a.ggw, e, c, ggw);
+        load_path_weights(a, a.w, nw, mul, has_coeff, e, c, w);
+        load_path_weights(a, a.ggw, nw, mul, has_coeff, e, c, ggw);
         S::dbwd_recv(x, ggx, Y, Yp, w, ggw, acc);
       }
     }
   }
   reduce_phases(acc, smem, phase, st, lane, 0, 1);
-  if (phase == 0 && act) S::store_out(a.y + (int64_t)row * a.out_dim, a.mul, c, acc);
+  if (phase == 0 && act) S::store_out(a.y + (int64_t)row * out_dim, mul, c, acc);
 }
 
 // ---------------------------------------------------------------------------------------
 // Double backward, sender pass: g_x[j] (segmented), g_w[e], g_vec[e].
 // ---------------------------------------------------------------------------------------
-template <class S, bool GVEC, int NSL>
+template <class S, bool GVEC, int NSL, int MUL, bool FAST>
 __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant__ LaunchArgs a) {
+  constexpr bool kFast = FAST;
+  const int mul = MUL ? MUL : a.mul;
+  const int nw = MUL ? S::P * MUL : a.nw;
+  const int in_dim = MUL ? S::IN_PC * MUL : a.in_dim;
+  const int out_dim = MUL ? S::OUT_PC * MUL : a.out_dim;
+  const bool check = !kFast && a.check;
+  const bool has_coeff = !kFast && a.has_coeff;
+  (void)nw; (void)in_dim; (void)out_dim; (void)has_coeff;
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
@@ -501,9 +522,9 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant
     sl = blockIdx.x - node * a.n_slices;
   }
   const int c = sl * 32 + lane;
-  const bool act = c < a.mul;
+  const bool act = c < mul;
   int q0 = __ldg(a.colptr + node), q1 = __ldg(a.colptr + node + 1);
-  if (a.check) {
+  if (check) {
     q0 = max(0, min(q0, a.E));
     q1 = max(q0, min(q1, a.E));
   }
@@ -516,8 +537,8 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant
     ggx[k] = 0.f;
   }
   if (act) {
-    S::load_in(a.x + (int64_t)node * a.in_dim, a.mul, c, x);
-    if (a.ggx) S::load_in(a.ggx + (int64_t)node * a.in_dim, a.mul, c, ggx);
+    S::load_in(a.x + (int64_t)node * in_dim, mul, c, x);
+    if (a.ggx) S::load_in(a.ggx + (int64_t)node * in_dim, mul, c, ggx);
   }
   float* gslot = smem + (size_t)(st > 1 ? (st - 1) * NSL * S::IN_PC * 32 : 0);
 
@@ -527,7 +548,7 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant
     float vx = 0.f, vy = 0.f, vz = 0.f, dx = 0.f, dy = 0.f, dz = 0.f;
     if (my_q < q1) {
       my_e = __ldg(a.perm + my_q);
-      if (a.check && (unsigned)my_e >= (unsigned)a.E) {
+      if (check && (unsigned)my_e >= (unsigned)a.E) {
         report(a, kDevBadPerm);
         my_e = -1;
       } else {
@@ -568,16 +589,16 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant
       for (int m = 0; m < S::NSH; ++m) G1[m] = G2[m] = 0.f;
       if (act && e >= 0) {
         float gyv[S::OUT_PC];
-        S::load_out(a.gy + (int64_t)i * a.out_dim, a.mul, c, gyv);
+        S::load_out(a.gy + (int64_t)i * out_dim, mul, c, gyv);
         float w[S::P], ggw[S::P];
-        load_path_weights(a, e, c, w);
-        load_path_weights_from(a, a.ggw, e, c, ggw);
+        load_path_weights(a, a.w, nw, mul, has_coeff, e, c, w);
+        load_path_weights(a, a.ggw, nw, mul, has_coeff, e, c, ggw);
         float gw[S::P];
         S::dbwd_send(x, ggx, Y, Yp, w, ggw, gyv, gx, gw, G1, G2);
         if (a.gw) {
-          float* row = a.gw + (int64_t)e * a.nw + c;
+          float* row = a.gw + (int64_t)e * nw + c;
 #pragma unroll
-          for (int p = 0; p < S::P; ++p) row[(int64_t)p * a.mul] = a.has_coeff ? gw[p] * a.coeff[p] : gw[p];
+          for (int p = 0; p < S::P; ++p) row[(int64_t)p * mul] = has_coeff ? gw[p] * a.coeff[p] : gw[p];
         }
       }
       if constexpr (GVEC) {
@@ -638,7 +659,7 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant
     }
   }
   reduce_phases(gx, smem, phase, st, lane, GVEC ? sl : 0, GVEC ? NSL : 1);
-  if (phase == 0 && act && a.gx) S::store_in(a.gx + (int64_t)node * a.in_dim, a.mul, c, gx);
+  if (phase == 0 && act && a.gx) S::store_in(a.gx + (int64_t)node * in_dim, mul, c, gx);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -646,78 +667,95 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant
 // ---------------------------------------------------------------------------------------
 // Register double buffering of the per-edge gathers pays when the buffers are small (lmax
 // <= 2); for lmax 3 the extra registers cost more occupancy than the overlap gains.
-// a.prefetch: -1 = this heuristic, 0/1 = forced (tuning override).
 template <class S>
-inline bool use_prefetch(const LaunchArgs& a) {
-  if (a.prefetch >= 0) return a.prefetch != 0;
-  return S::IN_PC + S::P + S::OUT_PC <= 48;
+constexpr bool kPrefetch = S::IN_PC + S::P + S::OUT_PC <= 48;
+
+// Calls f.template run<MUL, FAST>(): a specialisation with the channel count fixed at
+// compile time (constant load offsets, no index checks, no path coefficients) when the spec
+// ships one for a.mul and the call needs neither; otherwise the general kernel.
+template <class S, class F>
+cudaError_t dispatch_mul(const LaunchArgs& a, int mul, F&& f) {
+  if (!a.check && !a.has_coeff) {
+    if constexpr (S::FAST_MUL0 > 0)
+      if (mul == S::FAST_MUL0) return f.template run<S::FAST_MUL0, true>();
+    if constexpr (S::FAST_MUL1 > 0)
+      if (mul == S::FAST_MUL1) return f.template run<S::FAST_MUL1, true>();
+  }
+  return f.template run<0, false>();
 }
+
+template <class S>
+struct FwdLaunch {
+  const LaunchArgs& a;
+  cudaStream_t s;
+  template <int MUL, bool FAST>
+  cudaError_t run() const {
+    const size_t sm = (size_t)(a.split - 1) * S::OUT_PC * 32 * sizeof(float);
+    k_fwd_uvu<S, kPrefetch<S>, MUL, FAST><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+  }
+};
 
 template <class S>
 cudaError_t launch_fwd_uvu(const LaunchArgs& a, cudaStream_t s) {
   if (a.N == 0) return cudaSuccess;
-  const size_t sm = (size_t)(a.split - 1) * S::OUT_PC * 32 * sizeof(float);
-  if (use_prefetch<S>(a))
-    k_fwd_uvu<S, true><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
-  else
-    k_fwd_uvu<S, false><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
-  count_launches(1);
-  return cudaGetLastError();
+  return dispatch_mul<S>(a, a.mul, FwdLaunch<S>{a, s});
 }
+
+template <class S>
+struct DbwdRecvLaunch {
+  const LaunchArgs& a;
+  cudaStream_t s;
+  template <int MUL, bool FAST>
+  cudaError_t run() const {
+    const size_t sm = (size_t)(a.split - 1) * S::OUT_PC * 32 * sizeof(float);
+    k_dbwd_recv<S, MUL, FAST><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+  }
+};
 
 template <class S>
 cudaError_t launch_dbwd_recv(const LaunchArgs& a, cudaStream_t s) {
   if (a.N == 0) return cudaSuccess;
-  const size_t sm = (size_t)(a.split - 1) * S::OUT_PC * 32 * sizeof(float);
-  k_dbwd_recv<S><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
-  count_launches(1);
-  return cudaGetLastError();
+  return dispatch_mul<S>(a, a.mul, DbwdRecvLaunch<S>{a, s});
 }
 
-template <class S, bool GVEC, int NSL>
-cudaError_t launch_sender_bwd(const LaunchArgs& a, cudaStream_t s) {
-  const int st = a.split;
-  const int groups = GVEC ? NSL : 1;
-  const size_t sm = (size_t)(st > 1 ? (st - 1) * groups * S::IN_PC * 32 : 0) * sizeof(float) +
-                    (GVEC && NSL > 1 ? (size_t)st * 32 * NSL * 4 * sizeof(float) : 0);
-  const unsigned grid = GVEC ? (unsigned)a.N : (unsigned)a.N * a.n_slices;
-  if (use_prefetch<S>(a))
-    k_bwd_uvu<S, GVEC, NSL, true><<<grid, 32 * st * groups, sm, s>>>(a);
-  else
-    k_bwd_uvu<S, GVEC, NSL, false><<<grid, 32 * st * groups, sm, s>>>(a);
-  count_launches(1);
-  return cudaGetLastError();
-}
-
-template <class S, bool GVEC, int NSL>
-cudaError_t launch_sender_dbwd(const LaunchArgs& a, cudaStream_t s) {
-  const int st = a.split;
-  const int groups = GVEC ? NSL : 1;
-  const size_t sm = (size_t)(st > 1 ? (st - 1) * groups * S::IN_PC * 32 : 0) * sizeof(float) +
-                    (GVEC && NSL > 1 ? (size_t)st * 32 * NSL * 4 * sizeof(float) : 0);
-  const unsigned grid = GVEC ? (unsigned)a.N : (unsigned)a.N * a.n_slices;
-  k_dbwd_send<S, GVEC, NSL><<<grid, 32 * st * groups, sm, s>>>(a);
-  count_launches(1);
-  return cudaGetLastError();
-}
+template <class S, bool GVEC, int NSL, bool DBWD>
+struct SenderLaunch {
+  const LaunchArgs& a;
+  cudaStream_t s;
+  template <int MUL, bool FAST>
+  cudaError_t run() const {
+    const int st = a.split;
+    const int groups = GVEC ? NSL : 1;
+    const size_t sm = (size_t)(st > 1 ? (st - 1) * groups * S::IN_PC * 32 : 0) * sizeof(float) +
+                      (GVEC && NSL > 1 ? (size_t)st * 32 * NSL * 4 * sizeof(float) : 0);
+    const unsigned grid = GVEC ? (unsigned)a.N : (unsigned)a.N * a.n_slices;
+    if constexpr (DBWD)
+      k_dbwd_send<S, GVEC, NSL, MUL, FAST><<<grid, 32 * st * groups, sm, s>>>(a);
+    else
+      k_bwd_uvu<S, GVEC, NSL, kPrefetch<S>, MUL, FAST><<<grid, 32 * st * groups, sm, s>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+  }
+};
 
 // The host chooses split so that split * NSL <= 4 whenever gvec is requested.
-template <class S>
-cudaError_t launch_bwd_uvu(const LaunchArgs& a, cudaStream_t s) {
+template <class S, bool DBWD>
+cudaError_t launch_sender(const LaunchArgs& a, cudaStream_t s) {
   if (a.N == 0) return cudaSuccess;
-  if (a.gvec == nullptr) return launch_sender_bwd<S, false, 1>(a, s);
-  if (a.n_slices <= 1) return launch_sender_bwd<S, true, 1>(a, s);
-  if (a.n_slices == 2) return launch_sender_bwd<S, true, 2>(a, s);
-  return launch_sender_bwd<S, true, 4>(a, s);
+  if (a.gvec == nullptr) return dispatch_mul<S>(a, a.mul, SenderLaunch<S, false, 1, DBWD>{a, s});
+  if (a.n_slices <= 1) return dispatch_mul<S>(a, a.mul, SenderLaunch<S, true, 1, DBWD>{a, s});
+  if (a.n_slices == 2) return dispatch_mul<S>(a, a.mul, SenderLaunch<S, true, 2, DBWD>{a, s});
+  return dispatch_mul<S>(a, a.mul, SenderLaunch<S, true, 4, DBWD>{a, s});
 }
 
 template <class S>
-cudaError_t launch_dbwd_send(const LaunchArgs& a, cudaStream_t s) {
-  if (a.N == 0) return cudaSuccess;
-  if (a.gvec == nullptr) return launch_sender_dbwd<S, false, 1>(a, s);
-  if (a.n_slices <= 1) return launch_sender_dbwd<S, true, 1>(a, s);
-  if (a.n_slices == 2) return launch_sender_dbwd<S, true, 2>(a, s);
-  return launch_sender_dbwd<S, true, 4>(a, s);
-}
+cudaError_t launch_bwd_uvu(const LaunchArgs& a, cudaStream_t s) { return launch_sender<S, false>(a, s); }
+
+template <class S>
+cudaError_t launch_dbwd_send(const LaunchArgs& a, cudaStream_t s) { return launch_sender<S, true>(a, s); }
 
 }  // namespace tp
