@@ -723,6 +723,59 @@ def _gen_uvw_send(spec: Spec, xt_cum, xt_pc) -> List[str]:
     return L
 
 
+# ---------------------------------------------------------------------------
+# Edge-pair variants: every value is a float2 holding the same quantity for two edges of
+# one row, so each CG FMA is one packed __ffma2_rn (two FMAs per lane and instruction).
+# ---------------------------------------------------------------------------
+
+def _c2(c):
+    return f"make_float2({_flt(c)}, {_flt(c)})"
+
+
+def _chain2(terms, tgt):
+    out = []
+    first = True
+    for c, q in terms:
+        if first:
+            out.append(f"      float2 {tgt} = {q};" if c == 1.0 else f"      float2 {tgt} = __fmul2_rn({_c2(c)}, {q});")
+            first = False
+        else:
+            out.append(f"      {tgt} = __fadd2_rn({q}, {tgt});" if c == 1.0 else f"      {tgt} = __ffma2_rn({_c2(c)}, {q}, {tgt});")
+    if first:
+        out.append(f"      float2 {tgt} = make_float2(0.0f, 0.0f);")
+    return out
+
+
+def _gen_fwd2(spec: Spec) -> List[str]:
+    """Edge-pair forward: acc[out(p), m3] += w[p] * sum C x[in(p), m1] Y[sh(p), m2] (float2)."""
+    L = [f"  __device__ __forceinline__ static void fwd2(const float2 (&x)[{spec.IN_PC}], const float2 (&Y)[{spec.NSH}], const float2 (&w)[{spec.P}], float2 (&acc)[{spec.OUT_PC}]) {{"]
+    groups = _group(spec, lambda p: (p[0], p[1]))
+    for (a, b), plist in groups.items():
+        lb = spec.sh_ls[b]
+        L.append(f"    {{ // in block {a} x SH block {b}")
+        used = set()
+        for p in plist:
+            for (i, j, k, c) in cg_nonzeros(*spec.triples[p]):
+                used.add((i, j))
+        for (i, j) in sorted(used):
+            xs, ys = f"x[{spec.in_cum[a] + i}]", f"Y[{spec.sh_cum[b] + j}]"
+            L.append(f"      const float2 q{i}_{j} = {xs};" if lb == 0 else f"      const float2 q{i}_{j} = __fmul2_rn({xs}, {ys});")
+        for p in plist:
+            o = spec.paths[p][2]
+            nz = cg_nonzeros(*spec.triples[p])
+            d3 = 2 * spec.triples[p][2] + 1
+            for k in range(d3):
+                terms = [(c, f"q{i}_{j}") for (i, j, kk, c) in nz if kk == k]
+                if not terms:
+                    continue
+                L += _chain2(terms, f"t{p}_{k}")
+                idx = spec.out_cum[o] + k
+                L.append(f"      acc[{idx}] = __ffma2_rn(w[{p}], t{p}_{k}, acc[{idx}]);")
+        L.append("    }")
+    L.append("  }")
+    return L
+
+
 def gen_spec_header(spec: Spec) -> str:
     L = [f"// Generated by codegen.py for spec '{spec.name}'.  Do not edit.",
          f"// inputs l={spec.in_ls}  SH l={spec.sh_ls}  outputs l={spec.out_ls}",
@@ -750,6 +803,7 @@ def gen_spec_header(spec: Spec) -> str:
     L += _gen_fwd(spec)
     L += _gen_fwd(spec, name="uvw_edge", weighted_out="A", per_path_out=True)
     L += _gen_bwd(spec)
+    L += _gen_fwd2(spec)
     L += _gen_dbwd_recv(spec)
     L += _gen_dbwd_send(spec)
     L += _gen_uvw_layout(spec)

@@ -124,8 +124,11 @@ __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__
   }
   const int st = a.split;
   float acc[S::OUT_PC];
+  float2 acc2[PF ? S::OUT_PC : 1];
 #pragma unroll
   for (int k = 0; k < S::OUT_PC; ++k) acc[k] = 0.f;
+#pragma unroll
+  for (int k = 0; k < (PF ? S::OUT_PC : 1); ++k) acc2[k] = make_float2(0.f, 0.f);
 
   for (int base = e0 + phase; base < e1; base += 32 * st) {
     const int my_e = base + lane * st;
@@ -143,37 +146,42 @@ __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__
       }
     }
     const int ne = min(32, (e1 - base + st - 1) / st);
-    // gathers of edge k: sender slice x[j] and the edge's weight row
-    auto fetch = [&](int k, float (&xx)[S::IN_PC], float (&ww)[S::P]) {
-      const int j = __shfl_sync(kFull, my_j, k);
-      if (act && j >= 0) {
-        S::load_in(a.x + (int64_t)j * in_dim, mul, c, xx);
-        load_path_weights(a, a.w, nw, mul, has_coeff, base + k * st, c, ww);
-      }
-    };
-    auto compute = [&](int k, const float (&xx)[S::IN_PC], const float (&ww)[S::P]) {
-      const int j = __shfl_sync(kFull, my_j, k);
-      const float ux = __shfl_sync(kFull, vx, k);
-      const float uy = __shfl_sync(kFull, vy, k);
-      const float uz = __shfl_sync(kFull, vz, k);
-      if (j < 0) return;
-      float rx, ry, rz, ir;
-      edge_geometry(ux, uy, uz, rx, ry, rz, ir);
-      float Y[S::NSH];
-      S::sh(rx, ry, rz, Y);
-      if (act) S::fwd(xx, Y, ww, acc);
-    };
     float xa[S::IN_PC], wa[S::P];
     if constexpr (PF) {
-      // two register buffers: the gathers of edge k+1 are in flight while edge k computes
-      float xb[S::IN_PC], wb[S::P];
-      fetch(0, xa, wa);
+      // edge pairs: both edges' gathers are in flight together and every CG FMA is a packed
+      // __ffma2_rn over (edge k, edge k+1); an odd tail pairs with a zero-weight copy
       for (int k = 0; k < ne; k += 2) {
-        if (k + 1 < ne) fetch(k + 1, xb, wb);
-        compute(k, xa, wa);
-        if (k + 1 >= ne) break;
-        if (k + 2 < ne) fetch(k + 2, xa, wa);
-        compute(k + 1, xb, wb);
+        const bool two = k + 1 < ne;
+        const int kb = two ? k + 1 : k;
+        int ja = __shfl_sync(kFull, my_j, k), jb = __shfl_sync(kFull, my_j, kb);
+        const float ax = __shfl_sync(kFull, vx, k), ay = __shfl_sync(kFull, vy, k), az = __shfl_sync(kFull, vz, k);
+        const float bx = __shfl_sync(kFull, vx, kb), by = __shfl_sync(kFull, vy, kb), bz = __shfl_sync(kFull, vz, kb);
+        const bool oka = ja >= 0, okb = two && jb >= 0;
+        if (!oka && !okb) continue;
+        if (!oka) ja = jb;
+        if (!okb) jb = ja;
+        float2 x2[S::IN_PC], w2[S::P], Y2[S::NSH];
+        if (act) {
+          float xb[S::IN_PC], wb[S::P];
+          S::load_in(a.x + (int64_t)ja * in_dim, mul, c, xa);
+          S::load_in(a.x + (int64_t)jb * in_dim, mul, c, xb);
+          load_path_weights(a, a.w, nw, mul, has_coeff, base + k * st, c, wa);
+          load_path_weights(a, a.w, nw, mul, has_coeff, base + kb * st, c, wb);
+#pragma unroll
+          for (int q = 0; q < S::IN_PC; ++q) x2[q] = make_float2(xa[q], xb[q]);
+#pragma unroll
+          for (int q = 0; q < S::P; ++q) w2[q] = make_float2(oka ? wa[q] : 0.f, okb ? wb[q] : 0.f);
+        }
+        {
+          float rx, ry, rz, ir, Ya[S::NSH], Yb[S::NSH];
+          edge_geometry(ax, ay, az, rx, ry, rz, ir);
+          S::sh(rx, ry, rz, Ya);
+          edge_geometry(bx, by, bz, rx, ry, rz, ir);
+          S::sh(rx, ry, rz, Yb);
+#pragma unroll
+          for (int q = 0; q < S::NSH; ++q) Y2[q] = make_float2(Ya[q], Yb[q]);
+        }
+        if (act) S::fwd2(x2, Y2, w2, acc2);
       }
     } else {
       // one edge at a time, gathers issued after the SH evaluation (fewer live registers)
@@ -195,6 +203,10 @@ __global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__
         }
       }
     }
+  }
+  if constexpr (PF) {
+#pragma unroll
+    for (int k = 0; k < S::OUT_PC; ++k) acc[k] = acc2[k].x + acc2[k].y;
   }
   reduce_phases(acc, smem, phase, st, lane, 0, 1);
   if (phase == 0 && act) S::store_out(a.y + (int64_t)row * out_dim, mul, c, acc);
