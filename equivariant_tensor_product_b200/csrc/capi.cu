@@ -130,10 +130,11 @@ WsLayout ws_layout(int64_t N, int64_t E) {
   return L;
 }
 
-// uvw regions after the transpose region: A | G | Wt | part (floats, 256-byte aligned)
+// uvw regions (floats, 256-byte aligned).  Forward: A | Wt (hi, lo).  Backward, after the
+// transpose region: A (x W) | G (B) | xT | Wt (Wg hi, lo, Wx hi, lo) | part.
 constexpr int kUvwSplits = 64;
 struct UvwLayout {
-  size_t A, G, Wt, part, total;
+  size_t A, G, xT, Wt, part, total;
 };
 UvwLayout uvw_layout(tp_plan_t plan, int64_t N, int64_t E, bool bwd) {
   UvwLayout U{};
@@ -146,8 +147,10 @@ UvwLayout uvw_layout(tp_plan_t plan, int64_t N, int64_t E, bool bwd) {
   off += align256(a_bytes > 0 ? a_bytes : 1);
   U.G = off;
   if (bwd) off += align256(a_bytes > 0 ? a_bytes : 1);
+  U.xT = off;
+  if (bwd) off += align256(sizeof(float) * (size_t)(N > 0 ? N : 1) * plan->in_dim);
   U.Wt = off;
-  off += align256(w_bytes);
+  off += align256(w_bytes * (bwd ? 4 : 2));
   U.part = off;
   if (bwd) off += align256(w_bytes * kUvwSplits);
   U.total = off;
@@ -290,6 +293,10 @@ tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* i
                 "and the 4-path lmax-1 list)");
   if (mode == TP_MODE_UVW && (!found->uvw_fwd || !found->uvw_bwd))
     return fail(TP_ERR_UNSUPPORTED, "spec '%s' has no uvw kernels", found->name);
+  // the uvw GEMMs load their operands by TMA, whose row pitches are multiples of 16 bytes
+  if (mode == TP_MODE_UVW && (mul_in % 4 != 0 || mul_out % 4 != 0))
+    return fail(TP_ERR_UNSUPPORTED, "uvw needs multiplicities that are multiples of 4 (got %d, %d)", mul_in,
+                mul_out);
   tp_plan_s* pl = new (std::nothrow) tp_plan_s;
   if (!pl) return fail(TP_ERR_INVALID_ARG, "out of host memory");
   std::memset(pl, 0, sizeof(*pl));
@@ -483,6 +490,7 @@ tp_status_t tp_conv_bwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* row
     a.A = reinterpret_cast<float*>(wsb + U.A);
     a.G = reinterpret_cast<float*>(wsb + U.G);
     a.Wt = reinterpret_cast<float*>(wsb + U.Wt);
+    a.xT = reinterpret_cast<float*>(wsb + U.xT);
     a.part = reinterpret_cast<float*>(wsb + U.part);
     a.splits = kUvwSplits;
     a.gW = gW;

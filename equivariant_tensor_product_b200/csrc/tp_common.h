@@ -43,7 +43,8 @@ struct LaunchArgs {
   float* A;             // uvw forward: per-path receiver state (workspace), S::store_uvw layout;
                         // uvw backward: x W per path and sender, S::load_xt layout
   float* G;             // uvw backward: sender state B (workspace), S::store_xt layout
-  float* Wt;            // uvw: W regrouped for the GEMM B operands (workspace)
+  float* Wt;            // uvw: W regrouped for the GEMM B operands, TF32 hi and lo (workspace)
+  float* xT;            // uvw backward: x per input irrep as [node][m1][u] rows (workspace)
   float* gW;            // uvw: gradient of W (output)
   float* part;          // uvw: split-K partials of gW (workspace)
   int splits;           // uvw: number of split-K partials

@@ -6,15 +6,34 @@
 // (e.g. Ootomo & Yokota, 2022).
 //
 // CTA tile: M = 128 rows, N = 128 columns, K in blocks of 32 fp32 (one 128-byte swizzle
-// row).  All 128 threads stage operand blocks (global -> registers -> hi/lo split -> shared
-// memory in the canonical K-major 128B-swizzled layout); one elected thread issues the
-// tcgen05.mma instructions (kind::tf32, M128 N128 K8) and commits them to an mbarrier; two
-// stages let the staging of block k+1 overlap the MMAs of block k.  The epilogue moves the
-// accumulator TMEM -> registers (tcgen05.ld 32x32b) -> shared memory, and the operation
-// functor writes it out with coalesced stores.  Every wait is bounded: on timeout the CTA
-// records TP device error 6, stops issuing work and releases its TMEM.
+// row).  Warp-specialised, 192 threads, one CTA per SM:
+//   warp 0     one lane issues the TMA loads of each K block into a ring of stages;
+//   warp 1     owns the TMEM accumulator; one lane issues tcgen05.mma (kind::tf32,
+//              M128 N128 K8, three per K step for the split) and commits each stage back to
+//              the producer;
+//   warps 2-5  split the raw fp32 operand tiles into TF32 hi/lo tiles in the canonical
+//              K-major 128B-swizzled layout (transposing tiles that arrive M/N-major), then
+//              run the epilogue (tcgen05.ld 32x32b -> shared memory -> the op's stores).
+// Operands come in one of three forms (per op, at compile time):
+//   FMT_K      [rows][K] fp32, K contiguous: TMA with the 128B swizzle lands the tile in the
+//              MMA layout; the split rewrites it in place (hi) and writes lo beside it;
+//   FMT_MN     [K][rows] fp32, rows contiguous: TMA lands a plain 32 x 128 tile, the split
+//              transposes it;
+//   FMT_SPLIT  two K-major arrays already split into hi and lo (the shared weights, split
+//              once per call): TMA straight into the MMA tiles, no conversion.
+// The tensor-core accumulator does not round to nearest, so its error grows with the number
+// of MMAs summed into it.  Ops with a deep K (the split-K gW GEMM) set PROMOTE = R: every R K
+// blocks the epilogue warps add the TMEM accumulator into fp32 registers (round to nearest)
+// and the MMAs restart from zero, which bounds that growth at R blocks.
+// Every wait is bounded: on timeout the CTA records TP device error 6, the other roles see
+// the abort flag and stop, loads and MMAs already issued are waited for (again bounded) and
+// the TMEM is released.
 #pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cstdint>
+#include <mutex>
 
 #include "tp_common.h"
 
@@ -22,12 +41,30 @@ namespace tp {
 
 constexpr int TC_BM = 128, TC_BN = 128, TC_BK = 32;
 constexpr int TC_TILE_BYTES = TC_BM * TC_BK * 4;           // 16 KB: one 128 x 32 fp32 operand block
-constexpr int TC_STAGE_BYTES = 4 * TC_TILE_BYTES;          // A_hi, A_lo, B_hi, B_lo
-constexpr int TC_STAGES = 2;
+constexpr int TC_SMEM_BUDGET = 196608;                     // ring of stages (192 KB)
 constexpr int TC_EPI_LD = TC_BN + 1;                       // padded row of the staged accumulator
-constexpr int TC_SMEM_BYTES = TC_STAGES * TC_STAGE_BYTES + 1024;   // + alignment slack
+constexpr int TC_THREADS = 192;
 constexpr int kDevTimeout = 6;
-constexpr long long kWaitPolls = 1ll << 26;
+constexpr unsigned long long kWaitNs = 4000000000ull;   // a wait gives up after 4 s
+
+enum TcFmt { FMT_K = 0, FMT_MN = 1, FMT_SPLIT = 2 };
+
+__host__ __device__ constexpr int tc_operand_bytes(int fmt) {
+  return fmt == FMT_MN ? 3 * TC_TILE_BYTES : 2 * TC_TILE_BYTES;   // (raw +) hi + lo
+}
+__host__ __device__ constexpr int tc_load_bytes(int fmt) {
+  return fmt == FMT_SPLIT ? 2 * TC_TILE_BYTES : TC_TILE_BYTES;
+}
+template <class Op>
+struct TcShape {
+  static constexpr int A_BYTES = tc_operand_bytes(Op::A_FMT);
+  static constexpr int STAGE_BYTES = A_BYTES + tc_operand_bytes(Op::B_FMT);
+  static constexpr int STAGES = TC_SMEM_BUDGET / STAGE_BYTES > 4 ? 4 : TC_SMEM_BUDGET / STAGE_BYTES;
+  static constexpr uint32_t TX_BYTES = tc_load_bytes(Op::A_FMT) + tc_load_bytes(Op::B_FMT);
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;   // + alignment slack
+  static_assert(STAGES >= 2, "ring needs two stages");
+  static_assert(TC_BM * TC_EPI_LD * 4 <= STAGES * STAGE_BYTES, "epilogue tile reuses the ring");
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -63,6 +100,14 @@ __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -74,16 +119,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait; false after kWaitPolls unsuccessful polls.
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
-  for (long long it = 0; it < kWaitPolls; ++it)
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait bounded in time (a try_wait may suspend the thread for a while, so the bound is on
+// the clock, not on the number of polls) that also gives up when another role has aborted.
+// On its own timeout it raises the abort flag.  Returns false when the caller must stop.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volatile int* abort_flag) {
+  const unsigned long long t0 = global_ns();
+  for (;;) {
     if (mbar_try_wait(mbar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > kWaitNs) break;
+  }
+  *abort_flag = 1;
   return false;
+}
+
+// Time-bounded wait that ignores the abort flag: used to drain work already issued.
+__device__ __forceinline__ void mbar_drain(uint32_t mbar, uint32_t parity) {
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(mbar, parity))
+    if (global_ns() - t0 > kWaitNs) return;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t mbar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(mbar)
+      : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void epi_barrier() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -108,106 +182,98 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// Stages four consecutive k of one row (hi and lo parts) into a block pair.
-__device__ __forceinline__ void stage4(char* hi_blk, char* lo_blk, int row, int chunk, float4 v) {
-  float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
-  float4 l = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
-  const uint32_t off = sw128_off(row, chunk);
-  *reinterpret_cast<float4*>(hi_blk + off) = h;
-  *reinterpret_cast<float4*>(lo_blk + off) = l;
+// Split of one operand tile of a stage by converter thread ct (of 128).
+template <int FMT>
+__device__ __forceinline__ void tc_split(char* op_base, int ct) {
+  if constexpr (FMT == FMT_K) {
+    // the raw tile is already in the swizzled layout at op_base (it becomes hi); lo follows
+    char* lo = op_base + TC_TILE_BYTES;
+#pragma unroll
+    for (int i = 0; i < TC_TILE_BYTES / 16 / 128; ++i) {
+      const uint32_t off = (uint32_t)(ct + 128 * i) * 16u;
+      const float4 v = *reinterpret_cast<const float4*>(op_base + off);
+      const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+      *reinterpret_cast<float4*>(op_base + off) = h;
+      *reinterpret_cast<float4*>(lo + off) = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+    }
+  } else if constexpr (FMT == FMT_MN) {
+    // raw [32 k][128 rows] at op_base; the hi and lo K-major swizzled tiles follow it
+    const float* raw = reinterpret_cast<const float*>(op_base);
+    char* hi = op_base + TC_TILE_BYTES;
+    char* lo = op_base + 2 * TC_TILE_BYTES;
+    const int r = ct;
+#pragma unroll
+    for (int c = 0; c < TC_BK / 4; ++c) {
+      const float4 v = make_float4(raw[(4 * c + 0) * TC_BM + r], raw[(4 * c + 1) * TC_BM + r],
+                                   raw[(4 * c + 2) * TC_BM + r], raw[(4 * c + 3) * TC_BM + r]);
+      const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+      const uint32_t off = sw128_off(r, c);
+      *reinterpret_cast<float4*>(hi + off) = h;
+      *reinterpret_cast<float4*>(lo + off) = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+    }
+  }
 }
 
-// Operand addressing.  Element (r, k) of an operand lives at
-//   base[row(r) + kpart(k)],  kpart(k) = (k / kd) * ks1 + (k % kd) * ks2   (kd = 0: k * ks1)
-// row(r) is any per-row offset (computed once per row and K block); the k part is affine or
-// splits k into (outer, inner) with a small inner extent, which covers every uvw layout.
-struct TcOperand {
-  const float* base;
-  int kd;              // 0: plain stride ks1; else k = (k / kd, k % kd)
-  int64_t ks1, ks2;
-  bool vec4;           // rows are k-contiguous and 16-byte aligned: load 4 k at once
-  __device__ __forceinline__ int64_t kpart(int64_t k) const {
-    if (kd == 0) return k * ks1;
-    const int64_t q = k / kd;
-    return q * ks1 + (k - q * kd) * ks2;
+// Shared-memory address of the hi MMA tile of an operand in a stage (lo follows it).
+template <int FMT>
+__device__ __forceinline__ uint32_t tc_hi(uint32_t op_base) {
+  return FMT == FMT_MN ? op_base + TC_TILE_BYTES : op_base;
+}
+
+// Issues the TMA load(s) of one K block of an operand.  FMT_K / FMT_SPLIT maps are
+// (K inner, rows) with box (32, 128); FMT_MN maps are (rows inner, K) with box (128, 32).
+template <int FMT>
+__device__ __forceinline__ void tc_load(uint32_t op_base, const CUtensorMap* m0, const CUtensorMap* m1,
+                                        uint32_t mbar, int k0, int r0) {
+  if constexpr (FMT == FMT_K) {
+    tma_load_2d(op_base, m0, mbar, k0, r0);
+  } else if constexpr (FMT == FMT_MN) {
+    tma_load_2d(op_base, m0, mbar, r0, k0);
+  } else {
+    tma_load_2d(op_base, m0, mbar, k0, r0);
+    tma_load_2d(op_base + TC_TILE_BYTES, m1, mbar, k0, r0);
   }
-};
+}
 
 // Op interface:
-//   int64_t M, Nn; void k_range(a, z, &k0, &k1)
-//   TcOperand A, B (set on the host);  static constexpr bool A_KCONTIG, B_KCONTIG (thread mapping)
-//   __device__ int64_t a_row(a, m), b_row(a, n)   (offset of row m of A / row n of B)
-//   __device__ void store_tile(a, z, const float* T, int ld, int64_t m0, int n0)
-// A thread of the CTA stages a fixed (row, chunk) set of a 128 x 32 block: with k-contiguous
-// operands consecutive threads walk along k, otherwise along rows (coalesced either way).
-template <class Op, bool IS_A>
-struct TcStager {
-  static constexpr bool KC = IS_A ? Op::A_KCONTIG : Op::B_KCONTIG;
-  static constexpr int NIT = (TC_BM * TC_BK / 4) / 128;   // 8 chunks of 4 per thread
-  float4 v[NIT];
-  __device__ __forceinline__ static void slot(int it, int& row, int& chunk) {
-    const int q = threadIdx.x + 128 * it;
-    if (KC) {
-      row = q >> 3;
-      chunk = q & 7;
-    } else {
-      row = q & 127;
-      chunk = q >> 7;
-    }
-  }
-  __device__ __forceinline__ void load(const LaunchArgs& a, const Op& op, int64_t r0, int64_t rows, int64_t k0,
-                                       int64_t k1) {
-    const TcOperand& od = IS_A ? op.A : op.B;
-#pragma unroll
-    for (int it = 0; it < NIT; ++it) {
-      int row, chunk;
-      slot(it, row, chunk);
-      const int64_t r = r0 + row, k = k0 + 4 * chunk;
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < rows && k < k1) {
-        const float* p = od.base + (IS_A ? op.a_row(a, r) : op.b_row(a, r));
-        if (od.vec4 && k + 3 < k1) {
-          x = *reinterpret_cast<const float4*>(p + k);
-        } else {
-          float e[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) e[j] = (k + j < k1) ? __ldg(p + od.kpart(k + j)) : 0.f;
-          x = make_float4(e[0], e[1], e[2], e[3]);
-        }
-      }
-      v[it] = x;
-    }
-  }
-  __device__ __forceinline__ void store(char* hi, char* lo) const {
-#pragma unroll
-    for (int it = 0; it < NIT; ++it) {
-      int row, chunk;
-      slot(it, row, chunk);
-      stage4(hi, lo, row, chunk, v[it]);
-    }
-  }
-};
-
+//   int64_t M, Nn;  static constexpr int A_FMT, B_FMT, PROMOTE (0: off, else chunk of K blocks);
+//   CUtensorMap tA, tA2, tB, tB2   (tA2 / tB2 used only by FMT_SPLIT: the lo array)
+//   __device__ void k_range(a, z, &k0, &k1)   (k0 a multiple of 32)
+//   __device__ void store_tile(a, z, const float* T, int ld, int64_t m0, int n0, int t, int nt)
 template <class Op>
-__global__ void __launch_bounds__(128, 1) k_gemm_tc(const __grid_constant__ LaunchArgs a, const __grid_constant__ Op op) {
+__global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant__ LaunchArgs a,
+                                                           const __grid_constant__ Op op) {
+  using SH = TcShape<Op>;
+  constexpr int ST = SH::STAGES;
+  constexpr int R = Op::PROMOTE;
   extern __shared__ __align__(1024) char tc_smem_raw[];
-  __shared__ uint64_t mbar[TC_STAGES];
+  __shared__ __align__(8) uint64_t full_bar[ST];
+  __shared__ __align__(8) uint64_t conv_bar[ST];
+  __shared__ __align__(8) uint64_t empty_bar[ST];
+  __shared__ __align__(8) uint64_t acc_bar;
   __shared__ uint32_t tmem_holder;
-  __shared__ int abort_flag;
+  __shared__ volatile int abort_flag;
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t smem_s = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t m0 = (int64_t)blockIdx.x * TC_BM;
   const int n0 = blockIdx.y * TC_BN;
   int64_t k_begin, k_end;
   op.k_range(a, blockIdx.z, k_begin, k_end);
+  const int nkb = k_end > k_begin ? (int)((k_end - k_begin + TC_BK - 1) / TC_BK) : 0;
 
-  if (warp == 0) {
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_holder)),
                  "r"(TC_BN));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-    for (int s = 0; s < TC_STAGES; ++s) mbar_init(smem_u32(&mbar[s]), 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&conv_bar[s]), 128);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    mbar_init(smem_u32(&acc_bar), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     abort_flag = 0;
   }
@@ -216,84 +282,177 @@ __global__ void __launch_bounds__(128, 1) k_gemm_tc(const __grid_constant__ Laun
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
 
-  const int nkb = (int)((k_end - k_begin + TC_BK - 1) / TC_BK);
-  TcStager<Op, true> sa;
-  TcStager<Op, false> sb;
-  if (nkb > 0) {
-    sa.load(a, op, m0, op.M, k_begin, k_end);
-    sb.load(a, op, n0, op.Nn, k_begin, k_end);
-  }
-  for (int kb = 0; kb < nkb; ++kb) {
-    const int s = kb % TC_STAGES;
-    char* st = smem + s * TC_STAGE_BYTES;
-    if (kb >= TC_STAGES) {   // the MMAs that read this stage (block kb - TC_STAGES) must be done
-      const uint32_t parity = (uint32_t)((kb / TC_STAGES - 1) & 1);
-      if (!mbar_wait(smem_u32(&mbar[s]), parity)) atomicExch(&abort_flag, 1);
-    }
-    __syncthreads();
-    if (abort_flag) break;
-    sa.store(st, st + TC_TILE_BYTES);
-    sb.store(st + 2 * TC_TILE_BYTES, st + 3 * TC_TILE_BYTES);
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t ah = smem_u32(st), al = ah + TC_TILE_BYTES;
-      const uint32_t bh = ah + 2 * TC_TILE_BYTES, bl = ah + 3 * TC_TILE_BYTES;
-#pragma unroll
-      for (int ks = 0; ks < TC_BK / 8; ++ks) {      // K = 8 tf32 (32 bytes) per MMA
-        const uint32_t kofs = ks * 32;
-        const uint32_t acc0 = (kb > 0 || ks > 0) ? 1u : 0u;
-        mma_tf32(tmem, kmajor_sw128_desc(ah + kofs), kmajor_sw128_desc(bh + kofs), acc0);
-        mma_tf32(tmem, kmajor_sw128_desc(ah + kofs), kmajor_sw128_desc(bl + kofs), 1u);
-        mma_tf32(tmem, kmajor_sw128_desc(al + kofs), kmajor_sw128_desc(bh + kofs), 1u);
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % ST;
+        if (kb >= ST && !mbar_wait(smem_u32(&empty_bar[s]), (uint32_t)((kb / ST - 1) & 1), &abort_flag)) break;
+        const uint32_t st = smem_s + (uint32_t)(s * SH::STAGE_BYTES);
+        const uint32_t fb = smem_u32(&full_bar[s]);
+        mbar_expect_tx(fb, SH::TX_BYTES);
+        const int k0 = (int)(k_begin + (int64_t)kb * TC_BK);
+        tc_load<Op::A_FMT>(st, &op.tA, &op.tA2, fb, k0, (int)m0);
+        tc_load<Op::B_FMT>(st + SH::A_BYTES, &op.tB, &op.tB2, fb, k0, n0);
+        issued = kb + 1;
       }
-      mma_commit(smem_u32(&mbar[s]));
+      if (abort_flag) {   // let the loads already issued land before the CTA exits
+        for (int kb = issued > ST ? issued - ST : 0; kb < issued; ++kb)
+          mbar_drain(smem_u32(&full_bar[kb % ST]), (uint32_t)((kb / ST) & 1));
+      }
     }
-    // global loads of the next block are in flight while the tensor cores work on this one
-    if (kb + 1 < nkb) {
-      const int64_t k0 = k_begin + (int64_t)(kb + 1) * TC_BK;
-      sa.load(a, op, m0, op.M, k0, k_end);
-      sb.load(a, op, n0, op.Nn, k0, k_end);
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % ST;
+        if (!mbar_wait(smem_u32(&conv_bar[s]), (uint32_t)((kb / ST) & 1), &abort_flag)) break;
+        tc_fence_after();
+        const uint32_t st = smem_s + (uint32_t)(s * SH::STAGE_BYTES);
+        const uint32_t ah = tc_hi<Op::A_FMT>(st), al = ah + TC_TILE_BYTES;
+        const uint32_t bh = tc_hi<Op::B_FMT>(st + SH::A_BYTES), bl = bh + TC_TILE_BYTES;
+        const int kc = R > 0 ? kb % R : kb;   // position inside the current accumulation chunk
+        for (int ks = 0; ks < TC_BK / 8; ++ks) {   // K = 8 tf32 (32 bytes) per MMA
+          const uint32_t kofs = ks * 32;
+          const uint32_t acc0 = (kc > 0 || ks > 0) ? 1u : 0u;
+          mma_tf32(tmem, kmajor_sw128_desc(ah + kofs), kmajor_sw128_desc(bh + kofs), acc0);
+          mma_tf32(tmem, kmajor_sw128_desc(ah + kofs), kmajor_sw128_desc(bl + kofs), 1u);
+          mma_tf32(tmem, kmajor_sw128_desc(al + kofs), kmajor_sw128_desc(bh + kofs), 1u);
+        }
+        mma_commit(smem_u32(&empty_bar[s]));
+        issued = kb + 1;
+        // end of an accumulation chunk: arrives once its MMAs have completed
+        if (R > 0 && kc == R - 1 && kb + 1 < nkb) mma_commit(smem_u32(&acc_bar));
+      }
+      if (issued > 0) {
+        mma_commit(smem_u32(&acc_bar));   // arrives once every MMA issued above has completed
+        if (abort_flag) mbar_drain(smem_u32(&acc_bar), (uint32_t)((R > 0 ? (issued - 1) / R : 0) & 1));
+      }
     }
-  }
-  // wait for the last committed group of each stage
-  if (!abort_flag && nkb > 0) {
-    const int last = nkb - 1;
-    if (!mbar_wait(smem_u32(&mbar[last % TC_STAGES]), (uint32_t)((last / TC_STAGES) & 1))) atomicExch(&abort_flag, 1);
-    if (nkb > 1) {
-      const int prev = nkb - 2;
-      if (!mbar_wait(smem_u32(&mbar[prev % TC_STAGES]), (uint32_t)((prev / TC_STAGES) & 1)))
-        atomicExch(&abort_flag, 1);
+  } else {
+    // ---------------- split, then epilogue (warps 2-5) ----------------
+    const int ct = tid - 64;
+    const int q = warp & 3;   // a warp reads the TMEM lane quarter given by its id % 4
+    const int row = q * 32 + lane;
+    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+    float acc[R > 0 ? TC_BN : 1];
+    if constexpr (R > 0) {
+#pragma unroll
+      for (int i = 0; i < TC_BN; ++i) acc[i] = 0.f;
+    }
+    // adds the accumulator of a completed chunk into the fp32 registers
+    auto promote = [&]() {
+#pragma unroll
+      for (int c0 = 0; c0 < TC_BN; c0 += 32) {
+        float v[32];
+        tmem_ld32(tq + (uint32_t)c0, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[c0 + i] += v[i];
+      }
+      tc_fence_before();
+    };
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % ST;
+      if constexpr (R > 0) {
+        if (kb > 0 && kb % R == 0) {   // the previous chunk must be drained before its MMAs restart
+          if (!mbar_wait(smem_u32(&acc_bar), (uint32_t)((kb / R - 1) & 1), &abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          promote();
+        }
+      }
+      if (!mbar_wait(smem_u32(&full_bar[s]), (uint32_t)((kb / ST) & 1), &abort_flag)) {
+        ok = false;
+        break;
+      }
+      char* st = smem + s * SH::STAGE_BYTES;
+      tc_split<Op::A_FMT>(st, ct);
+      tc_split<Op::B_FMT>(st + SH::A_BYTES, ct);
+      fence_async_smem();
+      mbar_arrive(smem_u32(&conv_bar[s]));
+    }
+    ok = ok && !abort_flag;
+    if (ok && nkb > 0)
+      ok = mbar_wait(smem_u32(&acc_bar), (uint32_t)((R > 0 ? (nkb - 1) / R : 0) & 1), &abort_flag);
+    tc_fence_after();
+    epi_barrier();
+    if (ok && !abort_flag) {
+      float* T = reinterpret_cast<float*>(smem);
+      if constexpr (R > 0) {
+        if (nkb > 0) promote();
+#pragma unroll
+        for (int i = 0; i < TC_BN; ++i) T[row * TC_EPI_LD + i] = acc[i];
+      } else {
+#pragma unroll 1
+        for (int c0 = 0; c0 < TC_BN; c0 += 32) {
+          float v[32];
+          if (nkb > 0) {
+            tmem_ld32(tq + (uint32_t)c0, v);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) T[row * TC_EPI_LD + c0 + i] = v[i];
+        }
+        tc_fence_before();
+      }
+      epi_barrier();
+      op.store_tile(a, blockIdx.z, T, TC_EPI_LD, m0, n0, ct, 128);
     }
   }
   tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  if (abort_flag) {
-    if (tid == 0 && a.err) atomicCAS(a.err, 0, kDevTimeout);
-  } else {
-    // TMEM -> registers -> shared staging tile (fp32, padded rows), then the op's stores
-    float* T = reinterpret_cast<float*>(smem);
-    const int row = warp * 32 + lane;
-#pragma unroll 1
-    for (int c0 = 0; c0 < TC_BN; c0 += 32) {
-      float v[32];
-      if (nkb > 0) {
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) T[row * TC_EPI_LD + c0 + i] = v[i];
-    }
-    tc_fence_before();
-    __syncthreads();
-    op.store_tile(a, blockIdx.z, T, TC_EPI_LD, m0, n0);
+  if (tid == 0 && abort_flag && a.err) atomicCAS(a.err, 0, kDevTimeout);
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_BN));
   }
-  __syncthreads();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_BN));
+}
+
+// ---------------------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------------------
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D fp32 tensor map over `rows` rows of `inner` elements (row pitch `pitch` floats).
+// FMT_K / FMT_SPLIT: box 32 (inner) x 128 rows with the 128-byte swizzle;
+// FMT_MN:            box 128 (inner) x 32 rows, no swizzle.
+// Box elements outside the tensor read as zero.  Needs a 16-byte aligned base and pitch.
+inline cudaError_t make_tmap(CUtensorMap* m, const float* base, int64_t inner, int64_t rows, int64_t pitch,
+                             int fmt) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) || (pitch * 4) % 16 != 0 || inner <= 0 || rows <= 0 ||
+      pitch < inner)
+    return cudaErrorInvalidValue;
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)pitch * 4};
+  const cuuint32_t box_k[2] = {TC_BK, TC_BM};
+  const cuuint32_t box_mn[2] = {TC_BM, TC_BK};
+  const cuuint32_t estr[2] = {1, 1};
+  const bool mn = fmt == FMT_MN;
+  const CUresult r =
+      enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, mn ? box_mn : box_k, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, mn ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <class Op>
@@ -301,10 +460,11 @@ cudaError_t launch_gemm_tc(const LaunchArgs& a, const Op& op, int splits, cudaSt
   const int64_t M = op.M;
   const int Nn = (int)op.Nn;
   if (M <= 0 || Nn <= 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<Op>, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_BYTES);
+  constexpr int smem = TcShape<Op>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<Op>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((M + TC_BM - 1) / TC_BM), (unsigned)((Nn + TC_BN - 1) / TC_BN), (unsigned)splits);
-  k_gemm_tc<Op><<<grid, 128, TC_SMEM_BYTES, s>>>(a, op);
+  k_gemm_tc<Op><<<grid, TC_THREADS, smem, s>>>(a, op);
   count_launches(1);
   return cudaGetLastError();
 }

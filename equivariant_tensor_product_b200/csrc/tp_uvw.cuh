@@ -85,7 +85,15 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_edge(const __grid_constant_
   if (phase == 0 && act) S::store_uvw(a.A, a.N, a.mul, row, c, acc);
 }
 
-// Wt[o][w][pl * mul + u] = W[path_of[o][pl]][u][w]  (B operand of the forward mixing GEMM)
+// Split of one shared weight into its TF32 hi part (at dst) and lo part (at dst + n).
+__device__ __forceinline__ void put_split(float* dst, int64_t n, float v) {
+  const float h = tf32_hi(v);
+  dst[0] = h;
+  dst[n] = v - h;
+}
+
+// Wt[o][w][pl * mul + u] = W[path_of(o, pl)][u][w]: B operand of the forward mixing GEMM
+// (hi at Wt, lo at Wt + P * mul * mul_out).
 template <class S>
 __global__ void k_uvw_prep_wt(const __grid_constant__ LaunchArgs a) {
   const int64_t per_path = (int64_t)a.mul * a.mul_out;
@@ -104,12 +112,13 @@ __global__ void k_uvw_prep_wt(const __grid_constant__ LaunchArgs a) {
     const int w = (int)(rem / K), kk = (int)(rem % K);
     const int pl = kk / a.mul, u = kk % a.mul;
     const int p = S::path_of_at(o, pl);
-    a.Wt[base + rem] = a.W[(int64_t)p * per_path + (int64_t)u * a.mul_out + w];
+    put_split(a.Wt + base + rem, total, a.W[(int64_t)p * per_path + (int64_t)u * a.mul_out + w]);
   }
 }
 
-// Wt[o][w][pl * mul + u] = W[path_of(o, pl)][u][w]  (forward mixing, B operand)
-// is k_uvw_prep_wt above; Wg[a][u][pl * mul_out + w] = W[path_in(a, pl)][u][w] (gx, B operand).
+// Backward B operands, per input irrep a (paths pl of that irrep), hi and lo each:
+//   Wg[a][u][pl * mul_out + w]  = W[path_in(a, pl)][u][w]   (gx GEMM)       at Wt, Wt + n
+//   Wx[a][pl * mul_out + w][u]  = W[path_in(a, pl)][u][w]   (x W GEMM)      at Wt + 2n, Wt + 3n
 template <class S>
 __global__ void k_uvw_prep_wg(const __grid_constant__ LaunchArgs a) {
   const int64_t per_path = (int64_t)a.mul * a.mul_out;
@@ -127,7 +136,27 @@ __global__ void k_uvw_prep_wg(const __grid_constant__ LaunchArgs a) {
     const int u = (int)(rem / K), kk = (int)(rem % K);
     const int pl = kk / a.mul_out, w = kk % a.mul_out;
     const int p = S::path_in_at(ai, pl);
-    a.Wt[base + rem] = a.W[(int64_t)p * per_path + (int64_t)u * a.mul_out + w];
+    const float v = a.W[(int64_t)p * per_path + (int64_t)u * a.mul_out + w];
+    put_split(a.Wt + base + rem, total, v);
+    put_split(a.Wt + 2 * total + base + (int64_t)kk * a.mul + u, total, v);
+  }
+}
+
+// xT[a][(j, m1)][u] = x[j, a, u, m1]: the input irreps as K-contiguous rows for the x W
+// GEMM (and, read M-major, for the gW GEMM).  grid = N, one node row per CTA.
+template <class S>
+__global__ void k_uvw_xt(const __grid_constant__ LaunchArgs a) {
+  const int j = blockIdx.x;
+  const float* xr = a.x + (int64_t)j * a.in_dim;
+  for (int ai = 0; ai < S::N_IN; ++ai) {
+    const int d1 = S::in_d1_at(ai);
+    const int n = d1 * a.mul;
+    const int64_t xbase = (int64_t)a.mul * S::in_cum_at(ai);
+    float* dst = a.xT + (int64_t)a.N * xbase + (int64_t)j * n;
+    for (int t = threadIdx.x; t < n; t += blockDim.x) {
+      const int m1 = t / a.mul, u = t - m1 * a.mul;
+      dst[t] = __ldg(xr + xbase + (int64_t)u * d1 + m1);
+    }
   }
 }
 
@@ -135,12 +164,13 @@ __global__ void k_uvw_prep_wg(const __grid_constant__ LaunchArgs a) {
 // row layout [node][base + col * D + m]: one contiguous run of cols * D floats per node.
 template <int D>
 __device__ __forceinline__ void store_node_rows(float* out, int64_t row_stride, int64_t base, const float* T,
-                                                int ld, int64_t m0, int64_t M, int n0, int cols) {
+                                                int ld, int64_t m0, int64_t M, int n0, int cols, int t0,
+                                                int nt) {
   const int64_t mlast = min(M, m0 + TC_BM) - 1;
   const int64_t i0 = m0 / D, i1 = mlast / D;
   const int per_i = cols * D;
   const int total = (int)(i1 - i0 + 1) * per_i;
-  for (int t = threadIdx.x; t < total; t += blockDim.x) {
+  for (int t = t0; t < total; t += nt) {
     const int il = t / per_i;
     const int q = t - il * per_i;
     const int w = q / D, m = q - w * D;
@@ -151,46 +181,36 @@ __device__ __forceinline__ void store_node_rows(float* out, int64_t row_stride, 
   }
 }
 
+struct TcMaps {
+  CUtensorMap tA, tA2, tB, tB2;
+};
+
 // y_o[(i, m3), w] = sum_k A_o[(i, m3), k] Wt_o[w, k],  k = (pl, u)
 template <int D3>
-struct MixFwdTc {
+struct MixFwdTc : TcMaps {
   int64_t M, Nn;
-  int K;
   int64_t ybase;
-  TcOperand A, B;
-  static constexpr bool A_KCONTIG = true, B_KCONTIG = true;
+  int K;
+  static constexpr int A_FMT = FMT_K, B_FMT = FMT_SPLIT, PROMOTE = 0;
   __device__ void k_range(const LaunchArgs&, int, int64_t& b, int64_t& e) const { b = 0; e = K; }
-  __device__ int64_t a_row(const LaunchArgs&, int64_t m) const { return m * K; }
-  __device__ int64_t b_row(const LaunchArgs&, int64_t n) const { return n * K; }
-  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0) const {
-    store_node_rows<D3>(a.y, a.out_dim, ybase, T, ld, m0, M, n0, (int)min((int64_t)TC_BN, Nn - n0));
+  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0, int t,
+                             int nt) const {
+    store_node_rows<D3>(a.y, a.out_dim, ybase, T, ld, m0, M, n0, (int)min((int64_t)TC_BN, Nn - n0), t, nt);
   }
 };
 
-// xt_a[(j, m1), (pl, w)] = sum_u x[j, a, u, m1] W_{p(a, pl)}[u, w]
+// xt_a[(j, m1), (pl, w)] = sum_u xT_a[(j, m1), u] Wx_a[(pl, w), u]
 template <int D1>
-struct XtTc {
+struct XtTc : TcMaps {
   int64_t M, Nn;
   int K;                 // mul
-  int64_t xbase;         // mul * in_cum[a]
-  int in_dim, mul_out;
-  int64_t wstride;       // mul * mul_out
-  int paths[kMaxPaths];
   float* out;            // region a of the xt buffer, row-major [M][Nn]
-  TcOperand A, B;
-  static constexpr bool A_KCONTIG = (D1 == 1), B_KCONTIG = false;
+  static constexpr int A_FMT = FMT_K, B_FMT = FMT_SPLIT, PROMOTE = 0;
   __device__ void k_range(const LaunchArgs&, int, int64_t& b, int64_t& e) const { b = 0; e = K; }
-  __device__ int64_t a_row(const LaunchArgs&, int64_t m) const {
-    const int64_t j = m / D1;
-    return j * in_dim + xbase + (m - j * D1);
-  }
-  __device__ int64_t b_row(const LaunchArgs&, int64_t n) const {
-    const int pl = (int)(n / mul_out);
-    return paths[pl] * wstride + (n - (int64_t)pl * mul_out);
-  }
-  __device__ void store_tile(const LaunchArgs&, int, const float* T, int ld, int64_t m0, int n0) const {
+  __device__ void store_tile(const LaunchArgs&, int, const float* T, int ld, int64_t m0, int n0, int t0,
+                             int nt) const {
     const int cols = (int)min((int64_t)TC_BN, Nn - n0);
-    for (int t = threadIdx.x; t < TC_BM * cols; t += blockDim.x) {
+    for (int t = t0; t < TC_BM * cols; t += nt) {
       const int r = t / cols, c = t - r * cols;
       if (m0 + r < M) out[(m0 + r) * Nn + n0 + c] = T[r * ld + c];
     }
@@ -199,40 +219,36 @@ struct XtTc {
 
 // gx[j, a, u, m1] = sum_k B_a[(j, m1), k] Wg_a[u, k],  k = (pl, w)
 template <int D1>
-struct GxTc {
+struct GxTc : TcMaps {
   int64_t M, Nn;
-  int K;
   int64_t xbase;
-  TcOperand A, B;
-  static constexpr bool A_KCONTIG = true, B_KCONTIG = true;
+  int K;
+  static constexpr int A_FMT = FMT_K, B_FMT = FMT_SPLIT, PROMOTE = 0;
   __device__ void k_range(const LaunchArgs&, int, int64_t& b, int64_t& e) const { b = 0; e = K; }
-  __device__ int64_t a_row(const LaunchArgs&, int64_t m) const { return m * K; }
-  __device__ int64_t b_row(const LaunchArgs&, int64_t n) const { return n * K; }
-  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0) const {
-    store_node_rows<D1>(a.gx, a.in_dim, xbase, T, ld, m0, M, n0, (int)min((int64_t)TC_BN, Nn - n0));
+  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0, int t,
+                             int nt) const {
+    store_node_rows<D1>(a.gx, a.in_dim, xbase, T, ld, m0, M, n0, (int)min((int64_t)TC_BN, Nn - n0), t, nt);
   }
 };
 
-// part[z][p][u][w] = sum_{(j, m1) in split z} x[j, a, u, m1] B_a[(j, m1), (pl, w)]
+// part[z][p][u][w] = sum_{(j, m1) in split z} xT_a[(j, m1), u] B_a[(j, m1), (pl, w)]
 template <int D1>
-struct GwTc {
+struct GwTc : TcMaps {
   int64_t M, Nn;         // mul, cnt_a * mul_out
-  int64_t rows;          // N * d1
-  int splits, mul_out, P;
+  int64_t rows;          // N * d1 (the reduction)
   int64_t wstride;
+  int splits, mul_out, P;
   int paths[kMaxPaths];
-  TcOperand A, B;
-  static constexpr bool A_KCONTIG = false, B_KCONTIG = false;
+  static constexpr int A_FMT = FMT_MN, B_FMT = FMT_MN, PROMOTE = 16;   // K = N * d1 / splits rows
   __device__ void k_range(const LaunchArgs&, int z, int64_t& b, int64_t& e) const {
     const int64_t chunk = ((rows + splits - 1) / splits + TC_BK - 1) / TC_BK * TC_BK;
     b = min(rows, (int64_t)z * chunk);
     e = min(rows, b + chunk);
   }
-  __device__ int64_t a_row(const LaunchArgs&, int64_t m) const { return m * D1; }
-  __device__ int64_t b_row(const LaunchArgs&, int64_t n) const { return n; }
-  __device__ void store_tile(const LaunchArgs& a, int z, const float* T, int ld, int64_t m0, int n0) const {
+  __device__ void store_tile(const LaunchArgs& a, int z, const float* T, int ld, int64_t m0, int n0, int t0,
+                             int nt) const {
     const int cols = (int)min((int64_t)TC_BN, Nn - n0);
-    for (int t = threadIdx.x; t < TC_BM * cols; t += blockDim.x) {
+    for (int t = t0; t < TC_BM * cols; t += nt) {
       const int r = t / cols, c = t - r * cols;
       const int64_t u = m0 + r;
       if (u >= M) continue;
@@ -385,16 +401,6 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
 // ---------------------------------------------------------------------------------------
 // Host sequences
 // ---------------------------------------------------------------------------------------
-inline TcOperand tc_operand(const float* base, int kd, int64_t ks1, int64_t ks2, bool vec4) {
-  TcOperand o;
-  o.base = base;
-  o.kd = kd;
-  o.ks1 = ks1;
-  o.ks2 = ks2;
-  o.vec4 = vec4 && ((reinterpret_cast<uintptr_t>(base) & 15u) == 0);
-  return o;
-}
-
 template <template <int> class Op, class F>
 cudaError_t with_d(int d, F&& f) {
   switch (d) {
@@ -421,6 +427,7 @@ cudaError_t launch_uvw_fwd(const LaunchArgs& a, cudaStream_t s) {
   k_uvw_prep_wt<S><<<64, 256, 0, s>>>(a);
   count_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t n_shared = (int64_t)S::P * a.mul * a.mul_out;
   int64_t wt_off = 0;
   for (int o = 0; o < S::N_OUT; ++o) {
     const int d3 = S::out_d3_at(o), cnt = S::out_cnt_at(o);
@@ -430,8 +437,10 @@ cudaError_t launch_uvw_fwd(const LaunchArgs& a, cudaStream_t s) {
       op.Nn = a.mul_out;
       op.K = K;
       op.ybase = (int64_t)a.mul_out * S::out_cumY_at(o);
-      op.A = tc_operand(a.A + (int64_t)a.N * a.mul * S::out_cumA_at(o), 0, 1, 0, K % 4 == 0);
-      op.B = tc_operand(a.Wt + wt_off, 0, 1, 0, K % 4 == 0);
+      cudaError_t r = make_tmap(&op.tA, a.A + (int64_t)a.N * a.mul * S::out_cumA_at(o), K, op.M, K, FMT_K);
+      if (r == cudaSuccess) r = make_tmap(&op.tB, a.Wt + wt_off, K, a.mul_out, K, FMT_SPLIT);
+      if (r == cudaSuccess) r = make_tmap(&op.tB2, a.Wt + n_shared + wt_off, K, a.mul_out, K, FMT_SPLIT);
+      if (r != cudaSuccess) return r;
       return launch_gemm_tc(a, op, 1, s);
     });
     if (e != cudaSuccess) return e;
@@ -447,8 +456,13 @@ cudaError_t launch_uvw_bwd(const LaunchArgs& a, cudaStream_t s) {
   k_uvw_prep_wg<S><<<64, 256, 0, s>>>(a);
   count_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  k_uvw_xt<S><<<(unsigned)a.N, 128, 0, s>>>(a);
+  count_launches(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int64_t wstride = (int64_t)a.mul * a.mul_out;
+  const int64_t n_shared = wstride * S::P;
   // xt = x W per input irrep
+  int64_t wg_off = 0;
   for (int ai = 0; ai < S::N_IN; ++ai) {
     const int d1 = S::in_d1_at(ai), cnt = S::in_cnt_at(ai);
     if (cnt == 0) continue;
@@ -456,17 +470,16 @@ cudaError_t launch_uvw_bwd(const LaunchArgs& a, cudaStream_t s) {
       op.M = (int64_t)a.N * d1;
       op.Nn = (int64_t)cnt * a.mul_out;
       op.K = a.mul;
-      op.xbase = (int64_t)a.mul * S::in_cum_at(ai);
-      op.in_dim = a.in_dim;
-      op.mul_out = a.mul_out;
-      op.wstride = wstride;
-      for (int pl = 0; pl < cnt; ++pl) op.paths[pl] = S::path_in_at(ai, pl);
       op.out = a.A + (int64_t)a.N * a.mul_out * S::in_cumX_at(ai);
-      op.A = tc_operand(a.x, 0, d1, 0, d1 == 1 && a.in_dim % 4 == 0 && op.xbase % 4 == 0);
-      op.B = tc_operand(a.W, 0, a.mul_out, 0, false);
+      const float* xT = a.xT + (int64_t)a.N * a.mul * S::in_cum_at(ai);
+      cudaError_t r = make_tmap(&op.tA, xT, a.mul, op.M, a.mul, FMT_K);
+      if (r == cudaSuccess) r = make_tmap(&op.tB, a.Wt + 2 * n_shared + wg_off, a.mul, op.Nn, a.mul, FMT_SPLIT);
+      if (r == cudaSuccess) r = make_tmap(&op.tB2, a.Wt + 3 * n_shared + wg_off, a.mul, op.Nn, a.mul, FMT_SPLIT);
+      if (r != cudaSuccess) return r;
       return launch_gemm_tc(a, op, 1, s);
     });
     if (e != cudaSuccess) return e;
+    wg_off += (int64_t)cnt * wstride;
   }
   // sender pass: B, gs, gvec
   const int nsl = (a.mul_out + 31) / 32 <= 1 ? 1 : ((a.mul_out + 31) / 32 == 2 ? 2 : 4);
@@ -479,20 +492,23 @@ cudaError_t launch_uvw_bwd(const LaunchArgs& a, cudaStream_t s) {
 #undef TP_UVW_SEND
   count_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  int64_t wg_off = 0;
+  wg_off = 0;
   for (int ai = 0; ai < S::N_IN; ++ai) {
     const int d1 = S::in_d1_at(ai), cnt = S::in_cnt_at(ai);
     if (cnt == 0) continue;
     const int K = cnt * a.mul_out;
+    const int64_t rows = (int64_t)a.N * d1;
     const float* Bbuf = a.G + (int64_t)a.N * a.mul_out * S::in_cumX_at(ai);
     if (a.gx) {
       e = with_d<GxTc>(d1, [&](auto op) {
-        op.M = (int64_t)a.N * d1;
+        op.M = rows;
         op.Nn = a.mul;
         op.K = K;
         op.xbase = (int64_t)a.mul * S::in_cum_at(ai);
-        op.A = tc_operand(Bbuf, 0, 1, 0, K % 4 == 0);
-        op.B = tc_operand(a.Wt + wg_off, 0, 1, 0, K % 4 == 0);
+        cudaError_t r = make_tmap(&op.tA, Bbuf, K, rows, K, FMT_K);
+        if (r == cudaSuccess) r = make_tmap(&op.tB, a.Wt + wg_off, K, a.mul, K, FMT_SPLIT);
+        if (r == cudaSuccess) r = make_tmap(&op.tB2, a.Wt + n_shared + wg_off, K, a.mul, K, FMT_SPLIT);
+        if (r != cudaSuccess) return r;
         return launch_gemm_tc(a, op, 1, s);
       });
       if (e != cudaSuccess) return e;
@@ -500,20 +516,22 @@ cudaError_t launch_uvw_bwd(const LaunchArgs& a, cudaStream_t s) {
     if (a.gW) {
       e = with_d<GwTc>(d1, [&](auto op) {
         op.M = a.mul;
-        op.Nn = (int64_t)cnt * a.mul_out;
-        op.rows = (int64_t)a.N * d1;
+        op.Nn = K;
+        op.rows = rows;
         op.splits = a.splits;
         op.mul_out = a.mul_out;
         op.P = S::P;
         op.wstride = wstride;
         for (int pl = 0; pl < cnt; ++pl) op.paths[pl] = S::path_in_at(ai, pl);
-        op.A = tc_operand(a.x + (int64_t)a.mul * S::in_cum_at(ai), d1, a.in_dim, 1, false);
-        op.B = tc_operand(Bbuf, 0, (int64_t)cnt * a.mul_out, 0, false);
+        const float* xT = a.xT + (int64_t)a.N * a.mul * S::in_cum_at(ai);
+        cudaError_t r = make_tmap(&op.tA, xT, a.mul, rows, a.mul, FMT_MN);
+        if (r == cudaSuccess) r = make_tmap(&op.tB, Bbuf, K, rows, K, FMT_MN);
+        if (r != cudaSuccess) return r;
         return launch_gemm_tc(a, op, a.splits, s);
       });
       if (e != cudaSuccess) return e;
     }
-    wg_off += (int64_t)a.mul * K;
+    wg_off += (int64_t)cnt * wstride;
   }
   if (a.gW) {
     const int64_t n = (int64_t)S::P * wstride;

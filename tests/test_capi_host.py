@@ -107,9 +107,12 @@ def test_uvw_workspace_is_node_sized(tp):
     a_bytes = 4 * N * 51 * 128                   # per-path node state A (and its gradient G)
     f = tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD)
     b = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD)
-    assert a_bytes <= f <= a_bytes + plan.n_shared_weights * 4 + 4096
-    # bwd: transpose ints (8 bytes/edge + O(N)), A, G, W regrouped, 64 split-K partials of gW
-    assert b <= 8 * E + 12 * (N + 1) + 2 * a_bytes + 65 * 4 * plan.n_shared_weights + 16 * 256
+    # fwd: A and W regrouped for the GEMM (TF32 hi and lo)
+    assert a_bytes <= f <= a_bytes + 2 * 4 * plan.n_shared_weights + 4096
+    # bwd: transpose ints (8 bytes/edge + O(N)), A, G, x as K-contiguous rows, W regrouped
+    # twice (hi and lo each), 64 split-K partials of gW
+    x_bytes = 4 * N * plan.in_dim
+    assert b <= 8 * E + 12 * (N + 1) + 2 * a_bytes + x_bytes + 68 * 4 * plan.n_shared_weights + 16 * 256
     with pytest.raises(tp.TPError):
         tp.tp_workspace_size(plan, N, E, tp.TP_OP_DBWD)
 

@@ -62,7 +62,7 @@ def test_c4_full_size_sampled_and_adjoint(tp):
     assert_close(gx[torch.as_tensor(senders).cuda()], r["gx"][senders], "c4 gx[sampled]")
     assert_close(gs[torch.as_tensor(e2).cuda()], r["gs"], "c4 gs[sampled]")
     # gW at full size: y is linear in W, so <gW, dW> = <gy, y(dW)>
-    dW = torch.randn_like(g["W"])
+    dW = torch.randn(g["W"].shape, device="cuda", generator=torch.Generator(device="cuda").manual_seed(3))
     lhs = float((gW.double() * dW.view(-1).double()).sum())
     rhs = float((g["gy"].double() * _fwd(tp, plan, g, W=dW).double()).sum())
     assert abs(lhs - rhs) <= 1e-4 * max(abs(lhs), abs(rhs)), (lhs, rhs)
