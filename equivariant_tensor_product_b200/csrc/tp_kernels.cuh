@@ -101,7 +101,7 @@ __device__ __forceinline__ void reduce_phases(float (&acc)[N], float* smem, int 
 // Forward, uvu, receiver order.  grid = N * n_slices, block = 32 * split.
 // ---------------------------------------------------------------------------------------
 template <class S, bool PF, int MUL, bool FAST>
-__global__ void __launch_bounds__(kMaxThreads) k_fwd_uvu(const __grid_constant__ LaunchArgs a) {
+__global__ void __launch_bounds__(kMaxThreads, PF ? 4 : 1) k_fwd_uvu(const __grid_constant__ LaunchArgs a) {
   constexpr bool kFast = FAST;
   const int mul = MUL ? MUL : a.mul;
   const int nw = MUL ? S::P * MUL : a.nw;

@@ -273,6 +273,23 @@ static __global__ void k_reduce_splits(const float* __restrict__ part, int split
 // gs and gvec are channel sums across all slices of the sender, which share one CTA.
 // grid = N, block = 32 * NSL.
 // ---------------------------------------------------------------------------------------
+// Sums 16 values over the 32 lanes of a warp with 16 exchanges (against 80 for 16 separate
+// butterflies): at each halving step a lane keeps half of its values and trades the other
+// half with its partner.  Returns, in lanes 2v and 2v + 1, the warp sum of value v.
+__device__ __forceinline__ float warp_reduce_scatter16(float* v, int lane) {
+#pragma unroll
+  for (int h = 8; h >= 1; h >>= 1) {
+    const bool up = lane & (2 * h);
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = up ? v[i] : v[i + h];
+      const float keep = up ? v[i + h] : v[i];
+      v[i] = keep + __shfl_xor_sync(kFull, send, 2 * h);
+    }
+  }
+  return v[0] + __shfl_xor_sync(kFull, v[0], 1);
+}
+
 template <class S, bool GVEC, int NSL>
 __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant__ LaunchArgs a) {
   extern __shared__ float smem[];
@@ -351,21 +368,27 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
           h2 = fmaf(gY[m], G[m][2], h2);
           sdeg = fmaf(S::sh_degree(m) * gY[m], Y[m], sdeg);
         }
-        h0 = warp_sum(h0);
-        h1 = warp_sum(h1);
-        h2 = warp_sum(h2);
-        sdeg = warp_sum(sdeg);
       }
+      // channel sums of the NR per-edge values: 16 at a time, each lane pair ends up
+      // holding one of them (reduce-scatter), which one lane writes to the slice slot
+      constexpr int NR = GVEC ? S::P + 4 : S::P;
+      float r[(NR + 15) / 16 * 16];
 #pragma unroll
-      for (int p = 0; p < S::P; ++p) gs[p] = warp_sum(gs[p]);
-      if (lane == 0) {
-        float* sp = slot + ((size_t)k * NSL + sl) * NV;
+      for (int v = 0; v < (NR + 15) / 16 * 16; ++v) r[v] = 0.f;
 #pragma unroll
-        for (int p = 0; p < S::P; ++p) sp[p] = gs[p];
-        sp[S::P] = h0;
-        sp[S::P + 1] = h1;
-        sp[S::P + 2] = h2;
-        sp[S::P + 3] = sdeg;
+      for (int p = 0; p < S::P; ++p) r[p] = gs[p];
+      if constexpr (GVEC) {
+        r[S::P] = h0;
+        r[S::P + 1] = h1;
+        r[S::P + 2] = h2;
+        r[S::P + 3] = sdeg;
+      }
+      float* sp = slot + ((size_t)k * NSL + sl) * NV;
+#pragma unroll
+      for (int g = 0; g < (NR + 15) / 16; ++g) {
+        const float tot = warp_reduce_scatter16(&r[16 * g], lane);
+        const int v = 16 * g + ((lane >> 1) & 15);
+        if (!(lane & 1) && v < NR) sp[v] = tot;
       }
     }
     __syncthreads();
