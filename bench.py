@@ -36,7 +36,7 @@ WORKLOADS = {
     "c3": "SevenNet/MACE-like l=3: 4,096 atoms, ~163k edges, 64x(0e,1o,2e,3o), SH lmax 3, uvu, 34 paths; "
           "step = fwd + transpose + bwd(gx, gw)",
     "c5": "skewed degree 3-120: 8,192 atoms, ~295k edges, 32x(0e,1o,2e,3o), SH lmax 3, uvu, 34 paths; "
-          "step = fwd + transpose + bwd(gx, gw, gvec)",
+          "step = fwd + transpose + bwd(gx, gw, gvec) + dbwd(g_gy, g_x, g_w, g_vec)",
     "c4": "large streaming uvw: 100,000 atoms, ~3.0M edges, 128x(0e,1o,2e) -> 128x(0e,1e,1o,2e,2o), SH lmax 2, "
           "per-path 128x128 mixing, 15 paths; step = fwd + transpose + bwd(gx, gs, gW)",
 }
@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--n-atoms", type=int, default=None,
                     help="same-density replica with fewer atoms (profiling small cases)")
+    ap.add_argument("--order", default="random", choices=["random", "cell"],
+                    help="atom labels in generation order (random) or relabelled by spatial cell")
     return ap.parse_args()
 
 
@@ -85,6 +87,31 @@ def dist_env():
 
 def fwd_bytes(N, E, in_dim, out_dim, nw):
     return E * (4 + 12 + 4 * nw) + 4 * N * (in_dim + out_dim) + 4 * (N + 1)
+
+
+def dbwd_bytes(N, E, in_dim, out_dim, nw):
+    # src/perm/colptr + vec, ggvec read, g_vec write; w, ggw read, g_w write; x, ggx, gy read,
+    # g_x, g_gy write
+    return E * (48 + 12 * nw) + 4 * N * (3 * in_dim + 2 * out_dim)
+
+
+def uvw_bwd_flops(spec, E):
+    """Useful fp32 flops of the uvw sender pass per call: per edge and output channel, the
+    coupling Z_p = C (Y x gy) (2 nnz_p + 2 d2 d3 for the outer products, shared per (l2, l3)),
+    the state update B_p += s_p Z_p and the scalar gradient gs_p += <xt_p, Z_p> (2 d1 each)."""
+    from equivariant_tensor_product_b200.csrc.codegen import cg_nonzeros
+    mul = int(spec.irreps_out.split("x")[0])
+    ls_in = [int(b.split("x")[1][0]) for b in spec.irreps_in.split("+")]
+    ls_sh = [int(b.split("x")[1][0]) for b in spec.irreps_sh.split("+")]
+    ls_out = [int(b.split("x")[1][0]) for b in spec.irreps_out.split("+")]
+    per = 0
+    pairs = set()
+    for (a, b, o) in spec.paths:
+        l1, l2, l3 = ls_in[a], ls_sh[b], ls_out[o]
+        per += 2 * len(cg_nonzeros(l1, l2, l3)) + 4 * (2 * l1 + 1)
+        pairs.add((b, o))
+    per += sum(2 * (2 * ls_sh[b] + 1) * (2 * ls_out[o] + 1) for (b, o) in pairs)
+    return E * mul * per
 
 
 def bwd_bytes(N, E, in_dim, out_dim, nw, gvec):
@@ -142,6 +169,9 @@ class ClockSampler:
             self._stop.set()
             self.t.join()
             self._sample()
+
+    def max_mhz_or(self, default: float) -> float:
+        return float(self.max_mhz) if self.ok else default
 
     def summary(self):
         if not self.ok:
@@ -265,7 +295,10 @@ def run_ours(args, rank, world, local):
     lib = tp.load()
 
     spec = synth.CONFIGS[args.workload]
-    d = synth.make_inputs(args.workload, args.n_atoms, seed=spec.seed + 7919 * rank)
+    with_dbwd = "dbwd" in spec.passes
+    d = synth.make_inputs(args.workload, args.n_atoms, with_gg=with_dbwd, seed=spec.seed + 7919 * rank)
+    if args.order == "cell":
+        d = synth.cell_sorted(d)
     plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, spec.mode)
     N, E = len(d["rowptr"]) - 1, len(d["src"])
     in_dim, out_dim, nw = plan.in_dim, plan.out_dim, plan.n_edge_weights
@@ -298,7 +331,8 @@ def run_ours(args, rank, world, local):
     perms = [torch.empty(E, dtype=torch.int32, device=dev) for _ in range(R)]
     colptr, perm = colptrs[0], perms[0]
     gW = torch.empty(plan.n_shared_weights, device=dev) if uvw else None
-    ws_bytes = max(tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD), tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD))
+    ws_bytes = max(tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD), tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD),
+                   tp.tp_workspace_size(plan, N, E, tp.TP_OP_DBWD) if with_dbwd else 0)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     ws_t_bytes = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD) if not uvw else 256 + 8 * (N + E) + 4096
     ws_t = torch.empty(ws_t_bytes, dtype=torch.uint8, device=dev)      # side-stream transpose scratch
@@ -319,6 +353,16 @@ def run_ours(args, rank, world, local):
             (h, N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(cp["x"]), P(cp["vec"]),
              P(cp[wkey]), Wp, P(cp["gy"]), P(gx), P(gw), P(gvec), P(gW), P(ws), ws_bytes, sh),
         ))
+    if with_dbwd:   # second-order upstream gradients, one set shared by the copies (each > L2)
+        gg = {k: torch.as_tensor(np.ascontiguousarray(d[k])).to(dev) for k in ("ggx", "ggw", "ggvec")}
+        g_gy = torch.empty(N, out_dim, device=dev)
+        g_x = torch.empty(N, in_dim, device=dev)
+        g_w = torch.empty(E, nw, device=dev)
+        g_vec = torch.empty(E, 3, device=dev)
+        dargs = [(h, N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(cp["x"]), P(cp["vec"]),
+                  P(cp[wkey]), None, P(cp["gy"]), P(gg["ggx"]), P(gg["ggw"]), P(gg["ggvec"]), P(g_gy), P(g_x),
+                  P(g_w), P(g_vec), P(ws), ws_bytes, sh) for r, cp in enumerate(copies)]
+    dbwd_f = lib.tp_conv_dbwd
     tr_done = [torch.cuda.Event() for _ in range(R)]
     bwd_done = [torch.cuda.Event() for _ in range(R)]
     fwd_f, tr_f, bwd_f = lib.tp_conv_fwd, lib.tp_csr_transpose, lib.tp_conv_bwd
@@ -345,6 +389,10 @@ def run_ours(args, rank, world, local):
         st |= bwd_f(*a_b)
         if ev is not None:
             ev[3].record(stream)
+        if with_dbwd:
+            st |= dbwd_f(*dargs[r])
+            if ev is not None:
+                ev[6].record(stream)
         bwd_done[r].record(stream)
         if st:
             raise RuntimeError(lib.tp_last_error_message().decode())
@@ -352,7 +400,7 @@ def run_ours(args, rank, world, local):
     for k in range(args.warmup):
         step(k)
     torch.cuda.synchronize(dev)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -372,11 +420,14 @@ def run_ours(args, rank, world, local):
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     tr_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in evs)
     bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    dbwd_ms = statistics.mean(e[3].elapsed_time(e[6]) for e in evs) if with_dbwd else None
 
     # end to end through the same calls, inputs from pinned host memory, outputs back to host
-    host_in = {k: torch.as_tensor(np.ascontiguousarray(d[k])).pin_memory() for k in keys}
-    dev_in = {k: torch.empty_like(host_in[k], device=dev) for k in keys}
-    outs = (y, gx, gw) + ((gW,) if uvw else ())
+    e2e_keys = keys + (["ggx", "ggw", "ggvec"] if with_dbwd else [])
+    host_in = {k: torch.as_tensor(np.ascontiguousarray(d[k])).pin_memory() for k in e2e_keys}
+    dev_in = {k: torch.empty_like(host_in[k], device=dev) for k in e2e_keys}
+    outs = (y, gx, gw) + ((gvec,) if want_gvec else ()) + ((gW,) if uvw else ()) + \
+        ((g_gy, g_x, g_w, g_vec) if with_dbwd else ())
     host_out = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in outs]
     Wd = P(dev_in["W"]) if uvw else None
     e2e_args = (
@@ -385,11 +436,17 @@ def run_ours(args, rank, world, local):
         (N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(ws_t), ws_t_bytes, sh),
         (h, N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(dev_in["x"]), P(dev_in["vec"]),
          P(dev_in[wkey]), Wd, P(dev_in["gy"]), P(gx), P(gw), P(gvec), P(gW), P(ws), ws_bytes, sh))
+    if with_dbwd:
+        e2e_dargs = (h, N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(dev_in["x"]),
+                     P(dev_in["vec"]), P(dev_in[wkey]), None, P(dev_in["gy"]), P(dev_in["ggx"]), P(dev_in["ggw"]),
+                     P(dev_in["ggvec"]), P(g_gy), P(g_x), P(g_w), P(g_vec), P(ws), ws_bytes, sh)
 
     def e2e_step():
-        for k in keys:
+        for k in e2e_keys:
             dev_in[k].copy_(host_in[k], non_blocking=True)
         st = fwd_f(*e2e_args[0]) | tr_f(*e2e_args[1]) | bwd_f(*e2e_args[2])
+        if with_dbwd:
+            st |= dbwd_f(*e2e_dargs)
         if st:
             raise RuntimeError(lib.tp_last_error_message().decode())
         for ho, dv in zip(host_out, outs):
@@ -406,24 +463,39 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize(dev)
     e2e_s = e0.elapsed_time(e1) / 1e3
     e2e_value = replica_throughput(E, args.e2e_steps, world, max_over_ranks(e2e_s, world, dev))
-    h2d = sum(host_in[k].numel() * host_in[k].element_size() for k in keys)
+    h2d = sum(host_in[k].numel() * host_in[k].element_size() for k in e2e_keys)
     d2h = sum(t_.numel() * t_.element_size() for t_ in host_out)
 
     if rank == 0:
         hbm, _, peak_note = measured_peaks()
         fb = fwd_bytes(N, E, in_dim, out_dim, nw)
         bb = bwd_bytes(N, E, in_dim, out_dim, nw, want_gvec)
-        if bwd_ms >= fwd_ms:
-            kname, kbytes, kms = "k_bwd_uvu", bb, bwd_ms
+        db = dbwd_bytes(N, E, in_dim, out_dim, nw) if with_dbwd else 0
+        kernel_ms = {"fwd": fwd_ms, "transpose": tr_ms, "bwd": bwd_ms}
+        if with_dbwd:
+            kernel_ms["dbwd"] = dbwd_ms
+        if uvw:
+            # CUDA-core bound: the per-edge CG work of the backward call (sender pass) against
+            # 2 flop x 128 fp32 lanes x SMs x max SM clock; the mixing GEMMs are not counted
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            peak = 2 * 128 * sms * clk.max_mhz_or(1965.0) * 1e6 / 1e12
+            flops = uvw_bwd_flops(spec, E)
+            achieved = flops / (bwd_ms * 1e-3) / 1e12
+            roof = {"bound": "alu", "kernel": "tp_conv_bwd (uvw: k_uvw_send, x W / B W^T / x^T B GEMMs)",
+                    "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                    "peak_note": "fp32 FMA peak from the unit counts and max clock", "traffic": None,
+                    "algorithmic_flops_per_call": flops, "kernel_ms": kernel_ms}
         else:
-            kname, kbytes, kms = "k_fwd_uvu", fb, fwd_ms
-        achieved = kbytes / (kms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "peak_note": peak_note,
-                "traffic": traffic_from_profile(kname, args.workload),
-                "algorithmic_bytes_per_launch": kbytes,
-                "kernel_ms": {"fwd": fwd_ms, "transpose": tr_ms, "bwd": bwd_ms},
-                "step_roofline_frac": ((fb + bb) / (hbm * 1e9)) / (elapsed / args.steps)}
+            cands = [("k_fwd_uvu", fb, fwd_ms), ("k_bwd_uvu", bb, bwd_ms)]
+            if with_dbwd:
+                cands.append(("k_dbwd_recv + k_dbwd_send", db, dbwd_ms))
+            kname, kbytes, kms = max(cands, key=lambda t: t[2])
+            achieved = kbytes / (kms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "peak_note": peak_note,
+                    "traffic": traffic_from_profile(kname, args.workload),
+                    "algorithmic_bytes_per_launch": kbytes, "kernel_ms": kernel_ms,
+                    "step_roofline_frac": ((fb + bb + db) / (hbm * 1e9)) / (elapsed / args.steps)}
         cpu = None
         if not args.no_cpu_baseline and not uvw:
             from oracle.conv import set_threads
@@ -441,6 +513,7 @@ def run_ours(args, rank, world, local):
             "warmup": args.warmup, "ms_per_step": 1e3 * elapsed_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOADS[args.workload], "name": args.workload, "N": N, "E": E,
+                       "order": "cell-sorted" if args.order == "cell" else "generation order (random)",
                        "l2": f"{R} rotating input copies of {copy_bytes / 1e6:.1f} MB (> 2x L2 of "
                              f"{l2 / 1e6:.0f} MB)", "parallelism": "replicas" if world > 1 else "single"},
             "roofline": roof, "cpu_baseline": cpu,
