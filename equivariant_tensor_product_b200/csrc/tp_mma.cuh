@@ -6,14 +6,18 @@
 // (e.g. Ootomo & Yokota, 2022).
 //
 // CTA tile: M = 128 rows, N = 128 columns, K in blocks of 32 fp32 (one 128-byte swizzle
-// row).  Warp-specialised, 192 threads, one CTA per SM:
-//   warp 0     one lane issues the TMA loads of each K block into a ring of stages;
-//   warp 1     owns the TMEM accumulator; one lane issues tcgen05.mma (kind::tf32,
-//              M128 N128 K8, three per K step for the split) and commits each stage back to
-//              the producer;
+// row).  Persistent and warp-specialised: one CTA per SM walks a static list of tiles with
+// 320 threads:
+//   warp 0     one lane issues the TMA loads of every K block of every tile into a ring of
+//              stages;
+//   warp 1     owns two TMEM accumulators (256 columns); one lane issues tcgen05.mma
+//              (kind::tf32, M128 N128 K8, three per K step for the split) into them in turn
+//              and commits each stage back to the producer and each finished accumulator
+//              to the epilogue;
 //   warps 2-5  split the raw fp32 operand tiles into TF32 hi/lo tiles in the canonical
-//              K-major 128B-swizzled layout (transposing tiles that arrive M/N-major), then
-//              run the epilogue (tcgen05.ld 32x32b -> shared memory -> the op's stores).
+//              K-major 128B-swizzled layout (transposing tiles that arrive M/N-major);
+//   warps 6-9  epilogue: tcgen05.ld 32x32b -> registers -> a 128 x 32 shared tile -> the
+//              op's stores, while the MMAs of the next tile run on the other accumulator.
 // Operands come in one of three forms (per op, at compile time):
 //   FMT_K      [rows][K] fp32, K contiguous: TMA with the 128B swizzle lands the tile in the
 //              MMA layout; the split rewrites it in place (hi) and writes lo beside it;
@@ -32,6 +36,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <mutex>
 
@@ -42,8 +47,10 @@ namespace tp {
 constexpr int TC_BM = 128, TC_BN = 128, TC_BK = 32;
 constexpr int TC_TILE_BYTES = TC_BM * TC_BK * 4;           // 16 KB: one 128 x 32 fp32 operand block
 constexpr int TC_SMEM_BUDGET = 196608;                     // ring of stages (192 KB)
-constexpr int TC_EPI_LD = TC_BN + 1;                       // padded row of the staged accumulator
-constexpr int TC_THREADS = 192;
+constexpr int TC_EPI_COLS = 32;                            // epilogue sub-tile: 128 rows x 32 columns
+constexpr int TC_EPI_LD = TC_EPI_COLS + 1;                 // padded row of the staged sub-tile
+constexpr int TC_EPI_BYTES = (TC_BM * TC_EPI_LD * 4 + 1023) / 1024 * 1024;
+constexpr int TC_THREADS = 320;
 constexpr int kDevTimeout = 6;
 constexpr unsigned long long kWaitNs = 4000000000ull;   // a wait gives up after 4 s
 
@@ -61,9 +68,8 @@ struct TcShape {
   static constexpr int STAGE_BYTES = A_BYTES + tc_operand_bytes(Op::B_FMT);
   static constexpr int STAGES = TC_SMEM_BUDGET / STAGE_BYTES > 4 ? 4 : TC_SMEM_BUDGET / STAGE_BYTES;
   static constexpr uint32_t TX_BYTES = tc_load_bytes(Op::A_FMT) + tc_load_bytes(Op::B_FMT);
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;   // + alignment slack
+  static constexpr int SMEM = STAGES * STAGE_BYTES + TC_EPI_BYTES + 1024;   // + alignment slack
   static_assert(STAGES >= 2, "ring needs two stages");
-  static_assert(TC_BM * TC_EPI_LD * 4 <= STAGES * STAGE_BYTES, "epilogue tile reuses the ring");
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -157,7 +163,22 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void epi_barrier() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Tile t of the static schedule -> (m block, n block, split); n runs fastest so that the
+// CTAs working at the same time share their A tile through L2.
+struct TcTile {
+  int64_t m0;
+  int n0, z;
+};
+__device__ __forceinline__ TcTile tc_tile(int64_t t, int64_t mtiles, int ntiles) {
+  const int64_t per_z = mtiles * ntiles;
+  TcTile r;
+  r.z = (int)(t / per_z);
+  const int64_t rem = t - (int64_t)r.z * per_z;
+  r.m0 = (rem / ntiles) * TC_BM;
+  r.n0 = (int)(rem % ntiles) * TC_BN;
+  return r;
+}
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -239,10 +260,12 @@ __device__ __forceinline__ void tc_load(uint32_t op_base, const CUtensorMap* m0,
 //   int64_t M, Nn;  static constexpr int A_FMT, B_FMT, PROMOTE (0: off, else chunk of K blocks);
 //   CUtensorMap tA, tA2, tB, tB2   (tA2 / tB2 used only by FMT_SPLIT: the lo array)
 //   __device__ void k_range(a, z, &k0, &k1)   (k0 a multiple of 32)
-//   __device__ void store_tile(a, z, const float* T, int ld, int64_t m0, int n0, int t, int nt)
+//   __device__ void store_tile(a, z, const float* T, int ld, int64_t r0, int rows, int n0, int cols, int lane)
+//     stores, with the 32 lanes of one warp, the rows x cols block T (row stride ld) whose
+//     first element is at global row r0 and global column n0.
 template <class Op>
 __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant__ LaunchArgs a,
-                                                           const __grid_constant__ Op op) {
+                                                           const __grid_constant__ Op op, int splits) {
   using SH = TcShape<Op>;
   constexpr int ST = SH::STAGES;
   constexpr int R = Op::PROMOTE;
@@ -250,21 +273,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
   __shared__ __align__(8) uint64_t full_bar[ST];
   __shared__ __align__(8) uint64_t conv_bar[ST];
   __shared__ __align__(8) uint64_t empty_bar[ST];
-  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ __align__(8) uint64_t accf_bar[2];
+  __shared__ __align__(8) uint64_t acce_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ volatile int abort_flag;
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+  float* T = reinterpret_cast<float*>(smem + ST * SH::STAGE_BYTES);
   const uint32_t smem_s = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t m0 = (int64_t)blockIdx.x * TC_BM;
-  const int n0 = blockIdx.y * TC_BN;
-  int64_t k_begin, k_end;
-  op.k_range(a, blockIdx.z, k_begin, k_end);
-  const int nkb = k_end > k_begin ? (int)((k_end - k_begin + TC_BK - 1) / TC_BK) : 0;
+  const int64_t mtiles = (op.M + TC_BM - 1) / TC_BM;
+  const int ntiles = (int)((op.Nn + TC_BN - 1) / TC_BN);
+  const int64_t tiles = mtiles * ntiles * splits;
+  // K blocks of the tile and its accumulation segments (R K blocks each when promoting)
+  auto tile_kb = [&](const TcTile& tt, int64_t& kb0) {
+    int64_t k0, k1;
+    op.k_range(a, tt.z, k0, k1);
+    kb0 = k0;
+    return k1 > k0 ? (int)((k1 - k0 + TC_BK - 1) / TC_BK) : 0;
+  };
 
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_holder)),
-                 "r"(TC_BN));
+                 "r"(2 * TC_BN));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
@@ -273,7 +304,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
       mbar_init(smem_u32(&conv_bar[s]), 128);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
-    mbar_init(smem_u32(&acc_bar), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&accf_bar[b]), 1);
+      mbar_init(smem_u32(&acce_bar[b]), 128);
+    }
+    mbar_init(smem_u32(&drain_bar), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     abort_flag = 0;
   }
@@ -285,125 +320,171 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
   if (warp == 0) {
     // ---------------- producer ----------------
     if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % ST;
-        if (kb >= ST && !mbar_wait(smem_u32(&empty_bar[s]), (uint32_t)((kb / ST - 1) & 1), &abort_flag)) break;
-        const uint32_t st = smem_s + (uint32_t)(s * SH::STAGE_BYTES);
-        const uint32_t fb = smem_u32(&full_bar[s]);
-        mbar_expect_tx(fb, SH::TX_BYTES);
-        const int k0 = (int)(k_begin + (int64_t)kb * TC_BK);
-        tc_load<Op::A_FMT>(st, &op.tA, &op.tA2, fb, k0, (int)m0);
-        tc_load<Op::B_FMT>(st + SH::A_BYTES, &op.tB, &op.tB2, fb, k0, n0);
-        issued = kb + 1;
+      int64_t q = 0;   // position in the ring over all tiles
+      for (int64_t t = blockIdx.x; t < tiles && !abort_flag; t += gridDim.x) {
+        const TcTile tt = tc_tile(t, mtiles, ntiles);
+        int64_t kb0;
+        const int nkb = tile_kb(tt, kb0);
+        for (int kb = 0; kb < nkb; ++kb, ++q) {
+          const int s = (int)(q % ST);
+          if (q >= ST && !mbar_wait(smem_u32(&empty_bar[s]), (uint32_t)((q / ST - 1) & 1), &abort_flag)) break;
+          const uint32_t st = smem_s + (uint32_t)(s * SH::STAGE_BYTES);
+          const uint32_t fb = smem_u32(&full_bar[s]);
+          mbar_expect_tx(fb, SH::TX_BYTES);
+          const int k0 = (int)(kb0 + (int64_t)kb * TC_BK);
+          tc_load<Op::A_FMT>(st, &op.tA, &op.tA2, fb, k0, (int)tt.m0);
+          tc_load<Op::B_FMT>(st + SH::A_BYTES, &op.tB, &op.tB2, fb, k0, tt.n0);
+        }
       }
       if (abort_flag) {   // let the loads already issued land before the CTA exits
-        for (int kb = issued > ST ? issued - ST : 0; kb < issued; ++kb)
-          mbar_drain(smem_u32(&full_bar[kb % ST]), (uint32_t)((kb / ST) & 1));
+        for (int64_t u = q > ST ? q - ST : 0; u < q; ++u)
+          mbar_drain(smem_u32(&full_bar[u % ST]), (uint32_t)((u / ST) & 1));
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % ST;
-        if (!mbar_wait(smem_u32(&conv_bar[s]), (uint32_t)((kb / ST) & 1), &abort_flag)) break;
-        tc_fence_after();
-        const uint32_t st = smem_s + (uint32_t)(s * SH::STAGE_BYTES);
-        const uint32_t ah = tc_hi<Op::A_FMT>(st), al = ah + TC_TILE_BYTES;
-        const uint32_t bh = tc_hi<Op::B_FMT>(st + SH::A_BYTES), bl = bh + TC_TILE_BYTES;
-        const int kc = R > 0 ? kb % R : kb;   // position inside the current accumulation chunk
-        for (int ks = 0; ks < TC_BK / 8; ++ks) {   // K = 8 tf32 (32 bytes) per MMA
-          const uint32_t kofs = ks * 32;
-          const uint32_t acc0 = (kc > 0 || ks > 0) ? 1u : 0u;
-          mma_tf32(tmem, kmajor_sw128_desc(ah + kofs), kmajor_sw128_desc(bh + kofs), acc0);
-          mma_tf32(tmem, kmajor_sw128_desc(ah + kofs), kmajor_sw128_desc(bl + kofs), 1u);
-          mma_tf32(tmem, kmajor_sw128_desc(al + kofs), kmajor_sw128_desc(bh + kofs), 1u);
+      int64_t q = 0, g = 0;   // ring position, accumulation segment
+      bool issued = false;
+      for (int64_t t = blockIdx.x; t < tiles && !abort_flag; t += gridDim.x) {
+        const TcTile tt = tc_tile(t, mtiles, ntiles);
+        int64_t kb0;
+        const int nkb = tile_kb(tt, kb0);
+        for (int kb = 0; kb < nkb; ++kb, ++q) {
+          const int kc = R > 0 ? kb % R : kb;   // position inside the segment
+          const int b = (int)(g & 1);
+          if (kc == 0 && g >= 2 &&
+              !mbar_wait(smem_u32(&acce_bar[b]), (uint32_t)(((g >> 1) - 1) & 1), &abort_flag))
+            break;
+          const int s = (int)(q % ST);
+          if (!mbar_wait(smem_u32(&conv_bar[s]), (uint32_t)((q / ST) & 1), &abort_flag)) break;
+          tc_fence_after();
+          const uint32_t st = smem_s + (uint32_t)(s * SH::STAGE_BYTES);
+          const uint32_t ah = tc_hi<Op::A_FMT>(st), al = ah + TC_TILE_BYTES;
+          const uint32_t bh = tc_hi<Op::B_FMT>(st + SH::A_BYTES), bl = bh + TC_TILE_BYTES;
+          const uint32_t acc = tmem + (uint32_t)(b * TC_BN);
+          for (int ks = 0; ks < TC_BK / 8; ++ks) {   // K = 8 tf32 (32 bytes) per MMA
+            const uint32_t kofs = ks * 32;
+            const uint32_t acc0 = (kc > 0 || ks > 0) ? 1u : 0u;
+            mma_tf32(acc, kmajor_sw128_desc(ah + kofs), kmajor_sw128_desc(bh + kofs), acc0);
+            mma_tf32(acc, kmajor_sw128_desc(ah + kofs), kmajor_sw128_desc(bl + kofs), 1u);
+            mma_tf32(acc, kmajor_sw128_desc(al + kofs), kmajor_sw128_desc(bh + kofs), 1u);
+          }
+          issued = true;
+          mma_commit(smem_u32(&empty_bar[s]));
+          if ((R > 0 && kc == R - 1) || kb == nkb - 1) {   // end of a segment
+            mma_commit(smem_u32(&accf_bar[b]));
+            ++g;
+          }
         }
-        mma_commit(smem_u32(&empty_bar[s]));
-        issued = kb + 1;
-        // end of an accumulation chunk: arrives once its MMAs have completed
-        if (R > 0 && kc == R - 1 && kb + 1 < nkb) mma_commit(smem_u32(&acc_bar));
       }
-      if (issued > 0) {
-        mma_commit(smem_u32(&acc_bar));   // arrives once every MMA issued above has completed
-        if (abort_flag) mbar_drain(smem_u32(&acc_bar), (uint32_t)((R > 0 ? (issued - 1) / R : 0) & 1));
+      if (abort_flag && issued) {   // every MMA issued above must finish before TMEM is freed
+        mma_commit(smem_u32(&drain_bar));
+        mbar_drain(smem_u32(&drain_bar), 0u);
       }
+    }
+  } else if (warp < 6) {
+    // ---------------- split (warps 2-5) ----------------
+    const int ct = tid - 64;
+    int64_t q = 0;
+    for (int64_t t = blockIdx.x; t < tiles && !abort_flag; t += gridDim.x) {
+      const TcTile tt = tc_tile(t, mtiles, ntiles);
+      int64_t kb0;
+      const int nkb = tile_kb(tt, kb0);
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb, ++q) {
+        const int s = (int)(q % ST);
+        if (!mbar_wait(smem_u32(&full_bar[s]), (uint32_t)((q / ST) & 1), &abort_flag)) {
+          ok = false;
+          break;
+        }
+        char* st = smem + s * SH::STAGE_BYTES;
+        tc_split<Op::A_FMT>(st, ct);
+        tc_split<Op::B_FMT>(st + SH::A_BYTES, ct);
+        fence_async_smem();
+        mbar_arrive(smem_u32(&conv_bar[s]));
+      }
+      if (!ok) break;
     }
   } else {
-    // ---------------- split, then epilogue (warps 2-5) ----------------
-    const int ct = tid - 64;
-    const int q = warp & 3;   // a warp reads the TMEM lane quarter given by its id % 4
-    const int row = q * 32 + lane;
-    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
-    float acc[R > 0 ? TC_BN : 1];
-    if constexpr (R > 0) {
-#pragma unroll
-      for (int i = 0; i < TC_BN; ++i) acc[i] = 0.f;
-    }
-    // adds the accumulator of a completed chunk into the fp32 registers
-    auto promote = [&]() {
-#pragma unroll
-      for (int c0 = 0; c0 < TC_BN; c0 += 32) {
-        float v[32];
-        tmem_ld32(tq + (uint32_t)c0, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[c0 + i] += v[i];
-      }
-      tc_fence_before();
-    };
-    bool ok = true;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % ST;
+    // ---------------- epilogue (warps 6-9) ----------------
+    // Each warp owns the 32 accumulator rows of its TMEM lane quarter (warp id % 4) and
+    // stages and stores them on its own: no barrier spans warps, and every wait result is
+    // made warp-uniform before the warp-collective TMEM loads.
+    const int qd = warp & 3;
+    float* Tw = T + qd * 32 * TC_EPI_LD;
+    int64_t g = 0;
+    for (int64_t t = blockIdx.x; t < tiles && !abort_flag; t += gridDim.x) {
+      const TcTile tt = tc_tile(t, mtiles, ntiles);
+      int64_t kb0;
+      const int nkb = tile_kb(tt, kb0);
+      const int nseg = nkb == 0 ? 0 : (R > 0 ? (nkb + R - 1) / R : 1);
+      const int cols_all = (int)min((int64_t)TC_BN, op.Nn - tt.n0);
+      const int64_t r0 = tt.m0 + qd * 32;
+      bool ok = true;
       if constexpr (R > 0) {
-        if (kb > 0 && kb % R == 0) {   // the previous chunk must be drained before its MMAs restart
-          if (!mbar_wait(smem_u32(&acc_bar), (uint32_t)((kb / R - 1) & 1), &abort_flag)) {
-            ok = false;
-            break;
-          }
+        // segments add into fp32 registers (round to nearest)
+        float acc[TC_BN];
+#pragma unroll
+        for (int i = 0; i < TC_BN; ++i) acc[i] = 0.f;
+        for (int sg = 0; sg < nseg; ++sg, ++g) {
+          const int b = (int)(g & 1);
+          ok = __all_sync(kFull, mbar_wait(smem_u32(&accf_bar[b]), (uint32_t)((g >> 1) & 1), &abort_flag));
+          if (!ok) break;
           tc_fence_after();
-          promote();
-        }
-      }
-      if (!mbar_wait(smem_u32(&full_bar[s]), (uint32_t)((kb / ST) & 1), &abort_flag)) {
-        ok = false;
-        break;
-      }
-      char* st = smem + s * SH::STAGE_BYTES;
-      tc_split<Op::A_FMT>(st, ct);
-      tc_split<Op::B_FMT>(st + SH::A_BYTES, ct);
-      fence_async_smem();
-      mbar_arrive(smem_u32(&conv_bar[s]));
-    }
-    ok = ok && !abort_flag;
-    if (ok && nkb > 0)
-      ok = mbar_wait(smem_u32(&acc_bar), (uint32_t)((R > 0 ? (nkb - 1) / R : 0) & 1), &abort_flag);
-    tc_fence_after();
-    epi_barrier();
-    if (ok && !abort_flag) {
-      float* T = reinterpret_cast<float*>(smem);
-      if constexpr (R > 0) {
-        if (nkb > 0) promote();
+          const uint32_t tq = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(b * TC_BN);
 #pragma unroll
-        for (int i = 0; i < TC_BN; ++i) T[row * TC_EPI_LD + i] = acc[i];
+          for (int c0 = 0; c0 < TC_BN; c0 += 32) {
+            float v[32];
+            tmem_ld32(tq + (uint32_t)c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[c0 + i] += v[i];
+          }
+          tc_fence_before();
+          mbar_arrive(smem_u32(&acce_bar[b]));
+        }
+        if (!ok) break;
+#pragma unroll
+        for (int c0 = 0; c0 < TC_BN; c0 += TC_EPI_COLS) {
+          if (c0 < cols_all) {
+#pragma unroll
+            for (int i = 0; i < TC_EPI_COLS; ++i) Tw[lane * TC_EPI_LD + i] = acc[c0 + i];
+            __syncwarp();
+            op.store_tile(a, tt.z, Tw, TC_EPI_LD, r0, 32, tt.n0 + c0, min(TC_EPI_COLS, cols_all - c0), lane);
+            __syncwarp();
+          }
+        }
       } else {
+        const int b = (int)(g & 1);
+        if (nseg > 0) {
+          ok = __all_sync(kFull, mbar_wait(smem_u32(&accf_bar[b]), (uint32_t)((g >> 1) & 1), &abort_flag));
+          if (!ok) break;
+        }
+        tc_fence_after();
+        const uint32_t tq = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(b * TC_BN);
 #pragma unroll 1
-        for (int c0 = 0; c0 < TC_BN; c0 += 32) {
+        for (int c0 = 0; c0 < TC_BN; c0 += TC_EPI_COLS) {
           float v[32];
-          if (nkb > 0) {
+          if (nseg > 0) {
             tmem_ld32(tq + (uint32_t)c0, v);
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.f;
           }
+          if (nseg > 0 && c0 + TC_EPI_COLS == TC_BN) {   // accumulator fully read: hand it back
+            tc_fence_before();
+            mbar_arrive(smem_u32(&acce_bar[b]));
+          }
+          if (c0 < cols_all) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) T[row * TC_EPI_LD + c0 + i] = v[i];
+            for (int i = 0; i < TC_EPI_COLS; ++i) Tw[lane * TC_EPI_LD + i] = v[i];
+            __syncwarp();
+            op.store_tile(a, tt.z, Tw, TC_EPI_LD, r0, 32, tt.n0 + c0, min(TC_EPI_COLS, cols_all - c0), lane);
+            __syncwarp();
+          }
         }
-        tc_fence_before();
+        g += nseg;
       }
-      epi_barrier();
-      op.store_tile(a, blockIdx.z, T, TC_EPI_LD, m0, n0, ct, 128);
     }
   }
   tc_fence_before();
@@ -411,7 +492,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
   if (tid == 0 && abort_flag && a.err) atomicCAS(a.err, 0, kDevTimeout);
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_BN));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * TC_BN));
   }
 }
 
@@ -455,16 +536,29 @@ inline cudaError_t make_tmap(CUtensorMap* m, const float* base, int64_t inner, i
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+inline int sm_count() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  });
+  return n;
+}
+
 template <class Op>
 cudaError_t launch_gemm_tc(const LaunchArgs& a, const Op& op, int splits, cudaStream_t s) {
   const int64_t M = op.M;
-  const int Nn = (int)op.Nn;
-  if (M <= 0 || Nn <= 0) return cudaSuccess;
+  const int64_t Nn = op.Nn;
+  if (M <= 0 || Nn <= 0 || splits <= 0) return cudaSuccess;
   constexpr int smem = TcShape<Op>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<Op>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((M + TC_BM - 1) / TC_BM), (unsigned)((Nn + TC_BN - 1) / TC_BN), (unsigned)splits);
-  k_gemm_tc<Op><<<grid, TC_THREADS, smem, s>>>(a, op);
+  const int64_t tiles = ((M + TC_BM - 1) / TC_BM) * ((Nn + TC_BN - 1) / TC_BN) * splits;
+  const unsigned grid = (unsigned)std::min<int64_t>(tiles, sm_count());   // persistent: one CTA per SM
+  k_gemm_tc<Op><<<grid, TC_THREADS, smem, s>>>(a, op, splits);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -160,25 +160,36 @@ __global__ void k_uvw_xt(const __grid_constant__ LaunchArgs a) {
   }
 }
 
-// Stores a 128 x cols accumulator tile whose rows are (node, m) pairs, m < D, into a feature
-// row layout [node][base + col * D + m]: one contiguous run of cols * D floats per node.
+// Warp-level epilogue stores.  T holds a rows x cols block (row stride ld) of the
+// accumulator whose first element sits at global row r0, global column n0; the 32 lanes of
+// one warp store it with one contiguous 128-byte run per instruction.
+
+// Rows are (node, m) pairs, m < D; the output layout is [node][base + col * D + m], so the
+// block of node i is one contiguous run of cols * D floats.
 template <int D>
 __device__ __forceinline__ void store_node_rows(float* out, int64_t row_stride, int64_t base, const float* T,
-                                                int ld, int64_t m0, int64_t M, int n0, int cols, int t0,
-                                                int nt) {
-  const int64_t mlast = min(M, m0 + TC_BM) - 1;
-  const int64_t i0 = m0 / D, i1 = mlast / D;
-  const int per_i = cols * D;
-  const int total = (int)(i1 - i0 + 1) * per_i;
-  for (int t = t0; t < total; t += nt) {
-    const int il = t / per_i;
-    const int q = t - il * per_i;
-    const int w = q / D, m = q - w * D;
-    const int64_t i = i0 + il;
-    const int64_t row = i * D + m;
-    if (row < m0 || row > mlast) continue;
-    out[i * row_stride + base + (int64_t)(n0 + w) * D + m] = T[(int)(row - m0) * ld + w];
+                                                int ld, int64_t r0, int rows, int64_t M, int n0, int cols,
+                                                int lane) {
+  const int64_t rlast = min(M, r0 + rows) - 1;
+  if (rlast < r0) return;
+  const int64_t i0 = r0 / D, i1 = rlast / D;
+  for (int64_t i = i0; i <= i1; ++i) {
+    float* dst = out + i * row_stride + base + (int64_t)n0 * D;
+    for (int q = lane; q < cols * D; q += 32) {
+      const int w = q / D, m = q - w * D;
+      const int64_t row = i * D + m;
+      if (row >= r0 && row <= rlast) dst[q] = T[(int)(row - r0) * ld + w];
+    }
   }
+}
+
+// Row-major [M][Nn] output: lane = column, one row per instruction.
+__device__ __forceinline__ void store_rows(float* out, int64_t Nn, const float* T, int ld, int64_t r0, int rows,
+                                           int64_t M, int n0, int cols, int lane) {
+  if (lane >= cols) return;
+  const int nr = (int)min((int64_t)rows, M - r0);
+  float* dst = out + r0 * Nn + n0 + lane;
+  for (int r = 0; r < nr; ++r) dst[(int64_t)r * Nn] = T[r * ld + lane];
 }
 
 struct TcMaps {
@@ -193,9 +204,9 @@ struct MixFwdTc : TcMaps {
   int K;
   static constexpr int A_FMT = FMT_K, B_FMT = FMT_SPLIT, PROMOTE = 0;
   __device__ void k_range(const LaunchArgs&, int, int64_t& b, int64_t& e) const { b = 0; e = K; }
-  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0, int t,
-                             int nt) const {
-    store_node_rows<D3>(a.y, a.out_dim, ybase, T, ld, m0, M, n0, (int)min((int64_t)TC_BN, Nn - n0), t, nt);
+  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t r0, int rows, int n0,
+                             int cols, int lane) const {
+    store_node_rows<D3>(a.y, a.out_dim, ybase, T, ld, r0, rows, M, n0, cols, lane);
   }
 };
 
@@ -207,13 +218,9 @@ struct XtTc : TcMaps {
   float* out;            // region a of the xt buffer, row-major [M][Nn]
   static constexpr int A_FMT = FMT_K, B_FMT = FMT_SPLIT, PROMOTE = 0;
   __device__ void k_range(const LaunchArgs&, int, int64_t& b, int64_t& e) const { b = 0; e = K; }
-  __device__ void store_tile(const LaunchArgs&, int, const float* T, int ld, int64_t m0, int n0, int t0,
-                             int nt) const {
-    const int cols = (int)min((int64_t)TC_BN, Nn - n0);
-    for (int t = t0; t < TC_BM * cols; t += nt) {
-      const int r = t / cols, c = t - r * cols;
-      if (m0 + r < M) out[(m0 + r) * Nn + n0 + c] = T[r * ld + c];
-    }
+  __device__ void store_tile(const LaunchArgs&, int, const float* T, int ld, int64_t r0, int rows, int n0,
+                             int cols, int lane) const {
+    store_rows(out, Nn, T, ld, r0, rows, M, n0, cols, lane);
   }
 };
 
@@ -225,9 +232,9 @@ struct GxTc : TcMaps {
   int K;
   static constexpr int A_FMT = FMT_K, B_FMT = FMT_SPLIT, PROMOTE = 0;
   __device__ void k_range(const LaunchArgs&, int, int64_t& b, int64_t& e) const { b = 0; e = K; }
-  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t m0, int n0, int t,
-                             int nt) const {
-    store_node_rows<D1>(a.gx, a.in_dim, xbase, T, ld, m0, M, n0, (int)min((int64_t)TC_BN, Nn - n0), t, nt);
+  __device__ void store_tile(const LaunchArgs& a, int, const float* T, int ld, int64_t r0, int rows, int n0,
+                             int cols, int lane) const {
+    store_node_rows<D1>(a.gx, a.in_dim, xbase, T, ld, r0, rows, M, n0, cols, lane);
   }
 };
 
@@ -245,17 +252,14 @@ struct GwTc : TcMaps {
     b = min(rows, (int64_t)z * chunk);
     e = min(rows, b + chunk);
   }
-  __device__ void store_tile(const LaunchArgs& a, int z, const float* T, int ld, int64_t m0, int n0, int t0,
-                             int nt) const {
-    const int cols = (int)min((int64_t)TC_BN, Nn - n0);
-    for (int t = t0; t < TC_BM * cols; t += nt) {
-      const int r = t / cols, c = t - r * cols;
-      const int64_t u = m0 + r;
-      if (u >= M) continue;
-      const int n = n0 + c;
-      const int pl = n / mul_out, w = n - pl * mul_out;
-      a.part[((int64_t)z * P + paths[pl]) * wstride + u * mul_out + w] = T[r * ld + c];
-    }
+  __device__ void store_tile(const LaunchArgs& a, int z, const float* T, int ld, int64_t r0, int rows, int n0,
+                             int cols, int lane) const {
+    if (lane >= cols) return;
+    const int n = n0 + lane;
+    const int pl = n / mul_out, w = n - pl * mul_out;
+    float* dst = a.part + ((int64_t)z * P + paths[pl]) * wstride + w;
+    const int nr = (int)min((int64_t)rows, M - r0);
+    for (int r = 0; r < nr; ++r) dst[(r0 + r) * mul_out] = T[r * ld + lane];
   }
 };
 
