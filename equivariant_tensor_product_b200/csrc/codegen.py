@@ -261,13 +261,14 @@ class Spec:
         return sum(len(cg_nonzeros(*t)) for t in self.triples)
 
 
-def _lines_load(name, n_blocks, d, cum, arr, const=True):
-    """Straight-line load of one channel's slice of a [u][m] row."""
+def _lines_load(name, n_blocks, d, cum, arr, const=True, shared=False):
+    """Straight-line load of one channel's slice of a [u][m] row (read-only global path, or
+    plain loads for a row staged in shared memory)."""
     out = [f"  __device__ __forceinline__ static void {name}(const float* __restrict__ row, int mul, int c, float (&{arr})[{sum(d)}]) {{"]
     for a in range(n_blocks):
         out.append(f"    {{ const float* p = row + mul * {cum[a]} + c * {d[a]};")
         for m in range(d[a]):
-            out.append(f"      {arr}[{cum[a] + m}] = __ldg(p + {m});")
+            out.append(f"      {arr}[{cum[a] + m}] = p[{m}];" if shared else f"      {arr}[{cum[a] + m}] = __ldg(p + {m});")
         out.append("    }")
     out.append("  }")
     return out
@@ -793,8 +794,10 @@ def gen_spec_header(spec: Spec) -> str:
          f"  static constexpr int FAST_MUL0 = {spec.fast_muls[0]};",
          f"  static constexpr int FAST_MUL1 = {spec.fast_muls[1]};"]
     L += _lines_load("load_in", len(spec.in_ls), spec.in_d, spec.in_cum, "x")
+    L += _lines_load("load_in_shared", len(spec.in_ls), spec.in_d, spec.in_cum, "x", shared=True)
     L += _lines_store("store_in", len(spec.in_ls), spec.in_d, spec.in_cum, "x")
     L += _lines_load("load_out", len(spec.out_ls), spec.out_d, spec.out_cum, "y")
+    L += _lines_load("load_out_shared", len(spec.out_ls), spec.out_d, spec.out_cum, "y", shared=True)
     L += _lines_store("store_out", len(spec.out_ls), spec.out_d, spec.out_cum, "y")
     # uvw per-path state rows [p][u][m3]
     L += _lines_load("load_a", spec.P, spec.a_d, spec.a_cum, "a")

@@ -55,6 +55,41 @@ __device__ __forceinline__ int find_row(const int32_t* __restrict__ rowptr, int 
   return lo;
 }
 
+// Receiver search with a coarse copy of rowptr in shared memory: tab[k] = rowptr[k * stride]
+// for k < ntab (ntab <= kRowTab).  The coarse bracket is found in shared memory, the last
+// log2(stride) steps read rowptr itself.
+constexpr int kRowTab = 1024;
+
+struct RowTab {
+  int stride, ntab;
+};
+
+// Fills the table (all threads of the CTA take part; the caller synchronises afterwards).
+__device__ __forceinline__ RowTab load_row_tab(const int32_t* __restrict__ rowptr, int N, int32_t* tab) {
+  RowTab rt;
+  rt.stride = max(1, (N + kRowTab - 2) / (kRowTab - 1));
+  rt.ntab = N / rt.stride + 1;
+  for (int k = threadIdx.x; k < rt.ntab; k += blockDim.x) tab[k] = __ldg(rowptr + (int64_t)k * rt.stride);
+  return rt;
+}
+
+__device__ __forceinline__ int find_row_tab(const int32_t* __restrict__ rowptr, int N, const int32_t* tab,
+                                            RowTab rt, int e) {
+  int lo = 0, hi = rt.ntab - 1;   // last k with tab[k] <= e
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tab[mid] <= e) lo = mid;
+    else hi = mid - 1;
+  }
+  int rlo = lo * rt.stride, rhi = min(N - 1, rlo + rt.stride - 1);
+  while (rlo < rhi) {
+    const int mid = (rlo + rhi + 1) >> 1;
+    if (__ldg(rowptr + mid) <= e) rlo = mid;
+    else rhi = mid - 1;
+  }
+  return rlo;
+}
+
 __device__ __forceinline__ void report(const LaunchArgs& a, int code) {
   if (a.err) atomicCAS(a.err, 0, code);
 }
@@ -212,6 +247,188 @@ __global__ void __launch_bounds__(kMaxThreads, PF ? 4 : 1) k_fwd_uvu(const __gri
   if (phase == 0 && act) S::store_out(a.y + (int64_t)row * out_dim, mul, c, acc);
 }
 
+
+// ---------------------------------------------------------------------------------------
+// Forward with the per-edge rows staged by the copy engine (lmax <= 2 specs, 32 channels,
+// fast instance).  Same schedule and arithmetic as k_fwd_uvu's edge-pair path, but the two
+// rows an edge needs -- the sender's x row (IN_PC * 32 floats, contiguous) and the edge's
+// weight row (P * 32 floats, contiguous) -- are fetched by cp.async.bulk into a private ring
+// of kGatherSlots shared-memory slots per warp, kGatherSlots - 2 edges ahead of the pair
+// being computed, with an mbarrier per slot counting the bytes.  The gathers' latency then
+// overlaps the CG arithmetic instead of stalling it.  Waits are bounded by the global
+// timer; on a timeout the CTA records TP device error 6, lets the copies it issued land
+// (again bounded) and stops.
+// ---------------------------------------------------------------------------------------
+constexpr int kGatherSlots = 4;
+constexpr unsigned long long kGatherWaitNs = 4000000000ull;
+constexpr int kDevGatherTimeout = 6;
+
+__device__ __forceinline__ uint32_t sm_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(mbar)
+               : "memory");
+}
+
+__device__ __forceinline__ bool slot_ready(uint32_t mbar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(mbar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Time-bounded wait on a slot; false on timeout.
+__device__ __forceinline__ bool slot_wait(uint32_t mbar, uint32_t parity) {
+  if (slot_ready(mbar, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  while (!slot_ready(mbar, parity))
+    if (now_ns() - t0 > kGatherWaitNs) return false;
+  return true;
+}
+
+template <class S>
+struct GatherFwd {
+  static constexpr int XB = S::IN_PC * 32 * 4;   // bytes of one x row
+  static constexpr int WB = S::P * 32 * 4;       // bytes of one weight row
+  static constexpr int SLOT = XB + WB;
+  static constexpr size_t smem_bytes(int split) {
+    return (size_t)split * kGatherSlots * SLOT + (size_t)(split - 1) * S::OUT_PC * 32 * sizeof(float);
+  }
+};
+
+template <class S>
+__global__ void __launch_bounds__(kMaxThreads, 4) k_fwd_uvu_gather(const __grid_constant__ LaunchArgs a) {
+  using G = GatherFwd<S>;
+  constexpr int MUL = 32;
+  constexpr int in_dim = S::IN_PC * MUL, nw = S::P * MUL;
+  extern __shared__ __align__(128) unsigned char gsm[];
+  __shared__ __align__(8) uint64_t bars[kMaxThreads / 32][kGatherSlots];
+  const int lane = threadIdx.x & 31;
+  const int phase = threadIdx.x >> 5;
+  const int st = a.split;
+  const int row = blockIdx.x;
+  const int e0 = __ldg(a.rowptr + row), e1 = __ldg(a.rowptr + row + 1);
+  unsigned char* ring = gsm + (size_t)phase * kGatherSlots * G::SLOT;
+  float* red = reinterpret_cast<float*>(gsm + (size_t)st * kGatherSlots * G::SLOT);
+  if (lane == 0) {
+    for (int s2 = 0; s2 < kGatherSlots; ++s2)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sm_addr(&bars[phase][s2])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  uint32_t parity = 0;   // bit s: phase of slot s's next completion
+  int issued = 0;        // fills issued on this warp's ring (slot = fill % kGatherSlots)
+  int consumed = 0;      // fills waited for, in fill order
+  bool failed = false;
+
+  float2 acc2[S::OUT_PC];
+#pragma unroll
+  for (int k = 0; k < S::OUT_PC; ++k) acc2[k] = make_float2(0.f, 0.f);
+
+  for (int base = e0 + phase; base < e1 && !failed; base += 32 * st) {
+    const int my_e = base + lane * st;
+    int my_j = 0;
+    float vx = 0.f, vy = 0.f, vz = 0.f;
+    if (my_e < e1) {
+      my_j = __ldg(a.src + my_e);
+      vx = __ldg(a.vec + 3 * (int64_t)my_e);
+      vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
+      vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
+    }
+    const int ne = min(32, (e1 - base + st - 1) / st);
+    // copy edge k of this batch into the next ring slot (lane 0 issues; every lane learns j)
+    auto fill = [&](int k) {
+      const int j = __shfl_sync(kFull, my_j, k);
+      if (lane == 0) {
+        const int s2 = issued % kGatherSlots;
+        unsigned char* slot = ring + (size_t)s2 * G::SLOT;
+        const uint32_t mb = sm_addr(&bars[phase][s2]);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(G::SLOT) : "memory");
+        bulk_g2s(sm_addr(slot), a.x + (int64_t)j * in_dim, G::XB, mb);
+        bulk_g2s(sm_addr(slot + G::XB), a.w + (int64_t)(base + k * st) * nw, G::WB, mb);
+      }
+      ++issued;
+    };
+    const int first = issued;   // fill index of edge 0 of this batch
+    for (int k = 0; k < min(ne, kGatherSlots); ++k) fill(k);
+    for (int k = 0; k < ne; k += 2) {
+      const bool two = k + 1 < ne;
+      const int kb = two ? k + 1 : k;
+      const int sa = (first + k) % kGatherSlots, sb = (first + kb) % kGatherSlots;
+      bool ok = slot_wait(sm_addr(&bars[phase][sa]), (parity >> sa) & 1u);
+      if (two) ok = ok && slot_wait(sm_addr(&bars[phase][sb]), (parity >> sb) & 1u);
+      if (!__all_sync(kFull, ok)) {
+        failed = true;
+        break;
+      }
+      parity ^= 1u << sa;
+      if (two) parity ^= 1u << sb;
+      consumed += two ? 2 : 1;
+      const float* xa = reinterpret_cast<const float*>(ring + (size_t)sa * G::SLOT);
+      const float* xb = reinterpret_cast<const float*>(ring + (size_t)sb * G::SLOT);
+      float2 x2[S::IN_PC], w2[S::P], Y2[S::NSH];
+      {
+        float ta[S::IN_PC], tb[S::IN_PC];
+        S::load_in_shared(xa, MUL, lane, ta);
+        S::load_in_shared(xb, MUL, lane, tb);
+#pragma unroll
+        for (int q = 0; q < S::IN_PC; ++q) x2[q] = make_float2(ta[q], two ? tb[q] : ta[q]);
+        const float* wa = xa + G::XB / 4 + lane;
+        const float* wb = xb + G::XB / 4 + lane;
+#pragma unroll
+        for (int p = 0; p < S::P; ++p) w2[p] = make_float2(wa[p * MUL], two ? wb[p * MUL] : 0.f);
+      }
+      // both slots are read: refill them with the edges kGatherSlots ahead
+      __syncwarp();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      if (k + kGatherSlots < ne) fill(k + kGatherSlots);
+      if (two && kb + kGatherSlots < ne) fill(kb + kGatherSlots);
+      {
+        const float ax = __shfl_sync(kFull, vx, k), ay = __shfl_sync(kFull, vy, k), az = __shfl_sync(kFull, vz, k);
+        const float bx = __shfl_sync(kFull, vx, kb), by = __shfl_sync(kFull, vy, kb), bz = __shfl_sync(kFull, vz, kb);
+        float rx, ry, rz, ir, Ya[S::NSH], Yb[S::NSH];
+        edge_geometry(ax, ay, az, rx, ry, rz, ir);
+        S::sh(rx, ry, rz, Ya);
+        edge_geometry(bx, by, bz, rx, ry, rz, ir);
+        S::sh(rx, ry, rz, Yb);
+#pragma unroll
+        for (int q = 0; q < S::NSH; ++q) Y2[q] = make_float2(Ya[q], Yb[q]);
+      }
+      S::fwd2(x2, Y2, w2, acc2);
+    }
+  }
+  if (failed) {
+    // let every copy this warp issued land before the CTA exits, then report
+    if (lane == 0) {
+      for (int f = consumed; f < issued; ++f) {
+        const int s2 = f % kGatherSlots;
+        const unsigned long long t0 = now_ns();
+        while (!slot_ready(sm_addr(&bars[phase][s2]), (parity >> s2) & 1u) && now_ns() - t0 < kGatherWaitNs) {
+        }
+        parity ^= 1u << s2;
+      }
+      report(a, kDevGatherTimeout);
+    }
+  }
+  float acc[S::OUT_PC];
+#pragma unroll
+  for (int k = 0; k < S::OUT_PC; ++k) acc[k] = acc2[k].x + acc2[k].y;
+  reduce_phases(acc, red, phase, st, lane, 0, 1);
+  if (phase == 0) S::store_out(a.y + (int64_t)row * (S::OUT_PC * MUL), MUL, lane, acc);
+}
 
 // ---------------------------------------------------------------------------------------
 // Backward, uvu, sender order (through the stable transpose perm; each edge's receiver is
@@ -702,6 +919,17 @@ struct FwdLaunch {
   cudaStream_t s;
   template <int MUL, bool FAST>
   cudaError_t run() const {
+    if constexpr (kPrefetch<S> && MUL == 32 && FAST) {
+      // rows start on 16-byte boundaries: stage them with the copy engine
+      if (((reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.w)) & 15u) == 0) {
+        const size_t sm = GatherFwd<S>::smem_bytes(a.split);
+        cudaError_t e = cudaFuncSetAttribute(k_fwd_uvu_gather<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        k_fwd_uvu_gather<S><<<(unsigned)a.N, 32 * a.split, sm, s>>>(a);
+        count_launches(1);
+        return cudaGetLastError();
+      }
+    }
     const size_t sm = (size_t)(a.split - 1) * S::OUT_PC * 32 * sizeof(float);
     k_fwd_uvu<S, kPrefetch<S>, MUL, FAST><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
     count_launches(1);

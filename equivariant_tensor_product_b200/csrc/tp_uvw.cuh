@@ -19,6 +19,7 @@
 // All sums run in a fixed order: the results are deterministic.
 #pragma once
 #include <algorithm>
+#include <type_traits>
 
 #include "tp_kernels.cuh"
 #include "tp_mma.cuh"
@@ -90,6 +91,122 @@ __device__ __forceinline__ void put_split(float* dst, int64_t n, float v) {
   const float h = tf32_hi(v);
   dst[0] = h;
   dst[n] = v - h;
+}
+
+// Receiver pass with the senders' x rows staged whole by cp.async.bulk into a ring of
+// kEdgeSlots shared-memory slots read by all NSL slice warps of the CTA (one CTA per
+// receiver, warp = 32-channel slice, every warp walks all edges of the row); the last warp
+// to finish with a slot refills it with the row kEdgeSlots edges ahead.  Same arithmetic
+// as k_uvw_edge.  Needs no index checks, a CTA that covers every input channel and 16-byte
+// aligned rows (the launcher checks).
+constexpr int kEdgeSlots = 4;
+
+template <class S, int NSL>
+__global__ void __launch_bounds__(kMaxThreads) k_uvw_edge_staged(const __grid_constant__ LaunchArgs a) {
+  extern __shared__ __align__(128) unsigned char esm[];
+  __shared__ __align__(8) uint64_t full_bar[kEdgeSlots];
+  __shared__ uint32_t read_cnt[kEdgeSlots];
+  __shared__ int last_fill[kEdgeSlots];
+  __shared__ volatile int gather_failed;
+  const int lane = threadIdx.x & 31;
+  const int sl = threadIdx.x >> 5;
+  const int row = blockIdx.x;
+  const int c = sl * 32 + lane;
+  const bool act = c < a.mul;
+  const int e0 = __ldg(a.rowptr + row), e1 = __ldg(a.rowptr + row + 1);
+  const uint32_t row_bytes = (uint32_t)a.in_dim * 4u;
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < kEdgeSlots; ++s2) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sm_addr(&full_bar[s2])) : "memory");
+      read_cnt[s2] = 0;
+      last_fill[s2] = -1;
+    }
+    gather_failed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  auto fill = [&](int f, int j) {
+    const int s2 = f % kEdgeSlots;
+    const uint32_t mb = sm_addr(&full_bar[s2]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(row_bytes) : "memory");
+    bulk_g2s(sm_addr(esm + (size_t)s2 * row_bytes), a.x + (int64_t)j * a.in_dim, row_bytes, mb);
+    last_fill[s2] = f;
+  };
+  float acc[S::A_PC];
+#pragma unroll
+  for (int k = 0; k < S::A_PC; ++k) acc[k] = 0.f;
+  int first = 0;
+  for (int base = e0; base < e1; base += 32) {
+    const int my_e = base + lane;
+    int my_j = 0;
+    float vx = 0.f, vy = 0.f, vz = 0.f;
+    if (my_e < e1) {
+      my_j = __ldg(a.src + my_e);
+      vx = __ldg(a.vec + 3 * (int64_t)my_e);
+      vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
+      vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
+    }
+    const int ne = min(32, e1 - base);
+    if (sl == 0) {
+      for (int k = 0; k < min(ne, kEdgeSlots); ++k) {
+        const int j = __shfl_sync(kFull, my_j, k);
+        if (lane == 0) fill(first + k, j);
+      }
+    }
+#pragma unroll 1
+    for (int k = 0; k < ne; ++k) {
+      const int f = first + k, s2 = f % kEdgeSlots;
+      bool ok = !gather_failed;
+      if (ok) ok = slot_wait(sm_addr(&full_bar[s2]), (uint32_t)((f / kEdgeSlots) & 1));
+      ok = __all_sync(kFull, ok);
+      if (!ok) gather_failed = 1;
+      const float* xrow = reinterpret_cast<const float*>(esm + (size_t)s2 * row_bytes);
+      float x[S::IN_PC];
+      if (ok && act) S::load_in_shared(xrow, a.mul, c, x);
+      // this warp is done with the slot; the last of the NSL warps refills it
+      __syncwarp();
+      int last = 0;
+      if (lane == 0 && ok) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        uint32_t old;
+        asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(old) : "r"(sm_addr(&read_cnt[s2])) : "memory");
+        last = old == NSL - 1;
+      }
+      last = __shfl_sync(kFull, last, 0);
+      const int jnext = __shfl_sync(kFull, my_j, min(k + kEdgeSlots, 31));
+      if (last && lane == 0) {
+        read_cnt[s2] = 0;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (k + kEdgeSlots < ne) fill(f + kEdgeSlots, jnext);
+      }
+      if (!ok) continue;
+      const int e = base + k;
+      float sp[S::P];
+      const float* srow = a.w + (int64_t)e * S::P;
+#pragma unroll
+      for (int p = 0; p < S::P; ++p) sp[p] = __ldg(srow + p) * (a.has_coeff ? a.coeff[p] : 1.f);
+      const float ux = __shfl_sync(kFull, vx, k), uy = __shfl_sync(kFull, vy, k), uz = __shfl_sync(kFull, vz, k);
+      float rx, ry, rz, ir;
+      edge_geometry(ux, uy, uz, rx, ry, rz, ir);
+      float Y[S::NSH];
+      S::sh(rx, ry, rz, Y);
+      if (act) S::uvw_edge(x, Y, sp, acc);
+    }
+    __syncthreads();   // every warp is done with this batch's slots
+    first += ne;
+  }
+  if (gather_failed && threadIdx.x == 0) {   // let the issued copies land, then report
+    for (int s2 = 0; s2 < kEdgeSlots; ++s2) {
+      const int f = last_fill[s2];
+      if (f < 0) continue;
+      const uint32_t mb = sm_addr(&full_bar[s2]);
+      const unsigned long long t0 = now_ns();
+      while (!slot_ready(mb, (uint32_t)((f / kEdgeSlots) & 1)) && now_ns() - t0 < kGatherWaitNs) {
+      }
+    }
+    report(a, kDevGatherTimeout);
+  }
+  if (act) S::store_uvw(a.A, a.N, a.mul, row, c, acc);
 }
 
 // Wt[o][w][pl * mul + u] = W[path_of(o, pl)][u][w]: B operand of the forward mixing GEMM
@@ -294,10 +411,29 @@ __device__ __forceinline__ float warp_reduce_scatter16(float* v, int lane) {
   return v[0] + __shfl_xor_sync(kFull, v[0], 1);
 }
 
+// STAGED: the receivers' gy rows are fetched whole by cp.async.bulk into a ring of
+// kSendSlots shared-memory slots that all NSL slice warps of the CTA read; the last warp to
+// finish with a slot refills it with the row kSendSlots edges ahead.  Needs no index checks,
+// a CTA that covers every output channel and 16-byte aligned rows (the launcher checks).
+constexpr int kSendSlots = 3;
+
 template <class S, bool GVEC, int NSL>
+struct SendShape {
+  static constexpr int NV = S::P + 4;
+  static size_t smem_bytes(bool staged, int out_dim) {
+    return (size_t)32 * NSL * NV * sizeof(float) + (staged ? (size_t)kSendSlots * out_dim * sizeof(float) : 0);
+  }
+};
+
+template <class S, bool GVEC, int NSL, bool STAGED>
 __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant__ LaunchArgs a) {
   extern __shared__ float smem[];
   constexpr int NV = S::P + 4;   // per edge and slice: P gs partials, 3 gvec partials, degree sum
+  __shared__ __align__(8) uint64_t full_bar[kSendSlots];
+  __shared__ uint32_t read_cnt[kSendSlots];
+  __shared__ int last_fill[kSendSlots];
+  __shared__ volatile int gather_failed;
+  __shared__ int32_t rtab[kRowTab];
   const int lane = threadIdx.x & 31;
   const int sl = threadIdx.x >> 5;
   const int node = blockIdx.x;
@@ -308,6 +444,30 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
     q0 = max(0, min(q0, a.E));
     q1 = max(q0, min(q1, a.E));
   }
+  unsigned char* ring = reinterpret_cast<unsigned char*>(smem + 32 * NSL * NV);
+  const uint32_t row_bytes = (uint32_t)a.out_dim * 4u;
+  if constexpr (STAGED) {
+    if (threadIdx.x == 0) {
+      for (int s2 = 0; s2 < kSendSlots; ++s2) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sm_addr(&full_bar[s2])) : "memory");
+        read_cnt[s2] = 0;
+        last_fill[s2] = -1;
+      }
+      gather_failed = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+  }
+  const RowTab rt = load_row_tab(a.rowptr, a.N, rtab);
+  __syncthreads();
+  // fill f (a running index over this CTA's edges) -> slot f % kSendSlots
+  auto fill = [&](int f, int i) {
+    const int s2 = f % kSendSlots;
+    const uint32_t mb = sm_addr(&full_bar[s2]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(row_bytes) : "memory");
+    bulk_g2s(sm_addr(ring + (size_t)s2 * row_bytes), a.gy + (int64_t)i * a.out_dim, row_bytes, mb);
+    last_fill[s2] = f;
+  };
+  int first = 0;   // fill index of edge 0 of the current batch
   float xt[S::XT_PC], bt[S::XT_PC];
 #pragma unroll
   for (int k = 0; k < S::XT_PC; ++k) {
@@ -327,17 +487,36 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
         report(a, kDevBadPerm);
         my_e = -1;
       } else {
-        my_i = find_row(a.rowptr, a.N, my_e);
+        my_i = find_row_tab(a.rowptr, a.N, rtab, rt, my_e);
         vx = __ldg(a.vec + 3 * (int64_t)my_e);
         vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
         vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
       }
     }
     const int ne = min(32, q1 - base);
+    if constexpr (STAGED) {
+      if (sl == 0) {
+        for (int k = 0; k < min(ne, kSendSlots); ++k) {
+          const int i = __shfl_sync(kFull, my_i, k);
+          if (lane == 0) fill(first + k, i);
+        }
+      }
+    }
 #pragma unroll 1
     for (int k = 0; k < ne; ++k) {
       const int e = __shfl_sync(kFull, my_e, k);
       const int i = __shfl_sync(kFull, my_i, k);
+      const float* grow = nullptr;   // this edge's gy row (staged slot or global)
+      if constexpr (STAGED) {
+        const int f = first + k, s2 = f % kSendSlots;
+        bool ok = !gather_failed;
+        if (ok) ok = slot_wait(sm_addr(&full_bar[s2]), (uint32_t)((f / kSendSlots) & 1));
+        ok = __all_sync(kFull, ok);
+        if (!ok) gather_failed = 1;
+        grow = ok ? reinterpret_cast<const float*>(ring + (size_t)s2 * row_bytes) : nullptr;
+      } else {
+        grow = a.gy + (int64_t)i * a.out_dim;
+      }
       const float ux = __shfl_sync(kFull, vx, k);
       const float uy = __shfl_sync(kFull, vy, k);
       const float uz = __shfl_sync(kFull, vz, k);
@@ -355,10 +534,37 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
         const float* srow = a.w + (int64_t)e * S::P;
 #pragma unroll
         for (int p = 0; p < S::P; ++p) s[p] = __ldg(srow + p) * (a.has_coeff ? a.coeff[p] : 1.f);
-        if (act) {
+        if (act && grow) {
           float gyv[S::OUT_PC];
-          S::load_out(a.gy + (int64_t)i * a.out_dim, a.mul_out, c, gyv);
+          if constexpr (STAGED) {
+            S::load_out_shared(grow, a.mul_out, c, gyv);
+          } else {
+            S::load_out(grow, a.mul_out, c, gyv);
+          }
           S::template uvw_send<GVEC>(xt, Y, s, gyv, bt, gs, gY);
+        }
+      }
+      if constexpr (STAGED) {
+        // this warp is done with the slot; the last of the NSL warps refills it
+        __syncwarp();
+        int last = 0;
+        if (lane == 0 && grow) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          uint32_t old;
+          asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                       : "=r"(old)
+                       : "r"(sm_addr(&read_cnt[(first + k) % kSendSlots]))
+                       : "memory");
+          last = old == NSL - 1;
+        }
+        last = __shfl_sync(kFull, last, 0);
+        const int inext = __shfl_sync(kFull, my_i, min(k + kSendSlots, 31));
+        if (last) {
+          if (lane == 0) {
+            read_cnt[(first + k) % kSendSlots] = 0;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            if (k + kSendSlots < ne) fill(first + k + kSendSlots, inext);
+          }
         }
       }
       float h0 = 0.f, h1 = 0.f, h2 = 0.f, sdeg = 0.f;
@@ -421,6 +627,20 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
       }
     }
     __syncthreads();
+    first += ne;
+  }
+  if constexpr (STAGED) {
+    if (gather_failed && threadIdx.x == 0) {   // let the issued copies land, then report
+      for (int s2 = 0; s2 < kSendSlots; ++s2) {
+        const int f = last_fill[s2];
+        if (f < 0) continue;
+        const uint32_t mb = sm_addr(&full_bar[s2]);
+        const unsigned long long t0 = now_ns();
+        while (!slot_ready(mb, (uint32_t)((f / kSendSlots) & 1)) && now_ns() - t0 < kGatherWaitNs) {
+        }
+      }
+      report(a, kDevGatherTimeout);
+    }
   }
   if (act) S::store_xt(a.G, a.N, a.mul_out, node, c, bt);
 }
@@ -440,6 +660,16 @@ cudaError_t with_d(int d, F&& f) {
 
 template <class S>
 cudaError_t launch_uvw_edge(const LaunchArgs& a, cudaStream_t s) {
+  const int nsl = (a.mul + 31) / 32;
+  if (!a.check && nsl == 4 && a.in_dim % 4 == 0 && (reinterpret_cast<uintptr_t>(a.x) & 15u) == 0) {
+    // every slice of a receiver in one CTA, the x rows staged by the copy engine
+    const size_t sm = (size_t)kEdgeSlots * a.in_dim * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(k_uvw_edge_staged<S, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    k_uvw_edge_staged<S, 4><<<(unsigned)a.N, 128, sm, s>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+  }
   const size_t sm = (size_t)(a.split - 1) * S::A_PC * 32 * sizeof(float);
   k_uvw_edge<S><<<(unsigned)a.N * a.n_slices, 32 * a.split, sm, s>>>(a);
   count_launches(1);
@@ -510,13 +740,30 @@ cudaError_t launch_uvw_bwd(const LaunchArgs& a, cudaStream_t s) {
   }
   // sender pass: B, gs, gvec
   const int nsl = (a.mul_out + 31) / 32 <= 1 ? 1 : ((a.mul_out + 31) / 32 == 2 ? 2 : 4);
-  const size_t sm = (size_t)32 * nsl * (S::P + 4) * sizeof(float);
   const bool gv = a.gvec != nullptr;
-#define TP_UVW_SEND(G, NS) k_uvw_send<S, G, NS><<<(unsigned)a.N, 32 * NS, sm, s>>>(a)
-  if (nsl == 1) { if (gv) TP_UVW_SEND(true, 1); else TP_UVW_SEND(false, 1); }
-  else if (nsl == 2) { if (gv) TP_UVW_SEND(true, 2); else TP_UVW_SEND(false, 2); }
-  else { if (gv) TP_UVW_SEND(true, 4); else TP_UVW_SEND(false, 4); }
-#undef TP_UVW_SEND
+  // stage the gy rows when the CTA covers every channel and the rows are 16-byte aligned
+  const bool staged = !a.check && 32 * nsl >= a.mul_out && a.out_dim % 4 == 0 &&
+                      (reinterpret_cast<uintptr_t>(a.gy) & 15u) == 0;
+  auto send = [&](auto gvec_tag, auto nsl_tag) -> cudaError_t {
+    constexpr bool G = decltype(gvec_tag)::value;
+    constexpr int NS = decltype(nsl_tag)::value;
+    const size_t sm = SendShape<S, G, NS>::smem_bytes(staged, a.out_dim);
+    if (staged) {
+      cudaError_t r = cudaFuncSetAttribute(k_uvw_send<S, G, NS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      if (r != cudaSuccess) return r;
+      k_uvw_send<S, G, NS, true><<<(unsigned)a.N, 32 * NS, sm, s>>>(a);
+    } else {
+      k_uvw_send<S, G, NS, false><<<(unsigned)a.N, 32 * NS, sm, s>>>(a);
+    }
+    return cudaSuccess;
+  };
+  using T1 = std::integral_constant<int, 1>;
+  using T2 = std::integral_constant<int, 2>;
+  using T4 = std::integral_constant<int, 4>;
+  if (nsl == 1) e = gv ? send(std::true_type{}, T1{}) : send(std::false_type{}, T1{});
+  else if (nsl == 2) e = gv ? send(std::true_type{}, T2{}) : send(std::false_type{}, T2{});
+  else e = gv ? send(std::true_type{}, T4{}) : send(std::false_type{}, T4{});
+  if (e != cudaSuccess) return e;
   count_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   wg_off = 0;
