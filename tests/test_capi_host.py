@@ -100,6 +100,17 @@ def test_workspace_contract(tp):
         assert 8 * E <= b <= 8 * E + 8 * (N + 1) + 6 * 256
 
 
+def test_uvw_rejects_multiplicities_off_the_tma_pitch(tp):
+    # the mixing GEMMs load rows by TMA, whose row pitch must be a multiple of 16 bytes
+    spec = synth.CONFIGS["c4"]
+    bad_in = "+".join(f"30x{b.split('x')[1]}" for b in spec.irreps_in.split("+"))
+    with pytest.raises(tp.TPError) as e:
+        tp.Plan(bad_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvw")
+    assert e.value.status == 2
+    ok_in = "+".join(f"36x{b.split('x')[1]}" for b in spec.irreps_in.split("+"))
+    tp.Plan(ok_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvw")
+
+
 def test_uvw_workspace_is_node_sized(tp):
     spec = synth.CONFIGS["c4"]
     plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvw")
