@@ -499,8 +499,24 @@ def _gen_dbwd_send(spec: Spec) -> List[str]:
        gx[in(p)]  += sum_{m2,m3} C (ggw[p] Y[m2] + w[p] Yp[m2]) gy[m3]
        gw[p]       = sum C (ggx[m1] Y[m2] + x[m1] Yp[m2]) gy[m3]
        G1[sh(p)]  += ggw[p] Q(x, gy) + w[p] Q(ggx, gy);  G2[sh(p)] += w[p] Q(x, gy)
-       with Q(a, g)[m2] = sum_{m1,m3} C a[m1] g[m3]."""
-    L = [f"  __device__ __forceinline__ static void dbwd_send(const float (&x)[{spec.IN_PC}], const float (&ggx)[{spec.IN_PC}], const float (&Y)[{spec.NSH}], const float (&Yp)[{spec.NSH}], const float (&w)[{spec.P}], const float (&ggw)[{spec.P}], const float (&gy)[{spec.OUT_PC}], float (&gx)[{spec.IN_PC}], float (&gw)[{spec.P}], float (&G1)[{spec.NSH}], float (&G2)[{spec.NSH}]) {{"]
+       with Q(a, g)[m2] = sum_{m1,m3} C a[m1] g[m3].
+    Emitted three ways: dbwd_send (all of it), dbwd_send_gx (gx and gw only) and
+    dbwd_send_gv (G1 and G2 only), so that a large spec can run the two halves as two
+    kernels with half the straight-line code each."""
+    sig = "(const float (&x)[{i}], const float (&ggx)[{i}], const float (&Y)[{n}], const float (&Yp)[{n}], const float (&w)[{p}], const float (&ggw)[{p}], const float (&gy)[{o}], float (&gx)[{i}], float (&gw)[{p}], float (&G1)[{n}], float (&G2)[{n}])".format(
+        i=spec.IN_PC, n=spec.NSH, p=spec.P, o=spec.OUT_PC)
+    s1 = _dbwd_send_gx_lines(spec)
+    s2 = _dbwd_send_gv_lines(spec)
+    L = []
+    for name, parts in (("dbwd_send", s1 + s2), ("dbwd_send_gx", s1), ("dbwd_send_gv", s2)):
+        L.append(f"  __device__ __forceinline__ static void {name}{sig} {{")
+        L += parts
+        L.append("  }")
+    return L
+
+
+def _dbwd_send_gx_lines(spec: Spec) -> List[str]:
+    L = []
     groups = _group(spec, lambda p: (p[1], p[2]))
     for (b, o), plist in groups.items():
         lb = spec.sh_ls[b]
@@ -543,6 +559,11 @@ def _gen_dbwd_send(spec: Spec) -> List[str]:
             else:
                 L.append(f"      gw[{p}] = 0.0f;")
         L.append("    }")
+    return L
+
+
+def _dbwd_send_gv_lines(spec: Spec) -> List[str]:
+    L = []
     groups = _group(spec, lambda p: (p[0], p[2]))
     for (a, o), plist in groups.items():
         plist = [p for p in plist if spec.sh_ls[spec.paths[p][1]] != 0]
@@ -570,7 +591,6 @@ def _gen_dbwd_send(spec: Spec) -> List[str]:
                 L.append(f"      G1[{kb}] = fmaf(ggw[{p}], qa{p}_{j}, fmaf(w[{p}], qb{p}_{j}, G1[{kb}]));")
                 L.append(f"      G2[{kb}] = fmaf(w[{p}], qa{p}_{j}, G2[{kb}]);")
         L.append("    }")
-    L.append("  }")
     return L
 
 

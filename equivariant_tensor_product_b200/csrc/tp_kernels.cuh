@@ -726,8 +726,14 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_recv(const __grid_constant
 
 // ---------------------------------------------------------------------------------------
 // Double backward, sender pass: g_x[j] (segmented), g_w[e], g_vec[e].
+// PART 0 computes all three; large specs run PART 1 (g_x, g_w) and PART 2 (g_vec) as two
+// launches, each with half of the generated straight-line body, so that the instruction
+// working set of a kernel stays closer to what the instruction caches hold.
 // ---------------------------------------------------------------------------------------
-template <class S, bool GVEC, int NSL, int MUL, bool FAST>
+template <class S>
+constexpr bool kSplitDbwd = S::P > 15;
+
+template <class S, bool GVEC, int NSL, int MUL, bool FAST, int PART = 0>
 __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant__ LaunchArgs a) {
   constexpr bool kFast = FAST;
   const int mul = MUL ? MUL : a.mul;
@@ -823,8 +829,10 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant
         load_path_weights(a, a.w, nw, mul, has_coeff, e, c, w);
         load_path_weights(a, a.ggw, nw, mul, has_coeff, e, c, ggw);
         float gw[S::P];
-        S::dbwd_send(x, ggx, Y, Yp, w, ggw, gyv, gx, gw, G1, G2);
-        if (a.gw) {
+        if constexpr (PART == 0) S::dbwd_send(x, ggx, Y, Yp, w, ggw, gyv, gx, gw, G1, G2);
+        if constexpr (PART == 1) S::dbwd_send_gx(x, ggx, Y, Yp, w, ggw, gyv, gx, gw, G1, G2);
+        if constexpr (PART == 2) S::dbwd_send_gv(x, ggx, Y, Yp, w, ggw, gyv, gx, gw, G1, G2);
+        if (PART != 2 && a.gw) {
           float* row = a.gw + (int64_t)e * nw + c;
 #pragma unroll
           for (int p = 0; p < S::P; ++p) row[(int64_t)p * mul] = has_coeff ? gw[p] * a.coeff[p] : gw[p];
@@ -887,8 +895,10 @@ __global__ void __launch_bounds__(kMaxThreads) k_dbwd_send(const __grid_constant
       named_barrier(1 + phase, 32 * NSL);
     }
   }
-  reduce_phases(gx, smem, phase, st, lane, GVEC ? sl : 0, GVEC ? NSL : 1);
-  if (phase == 0 && act && a.gx) S::store_in(a.gx + (int64_t)node * in_dim, mul, c, gx);
+  if constexpr (PART != 2) {
+    reduce_phases(gx, smem, phase, st, lane, GVEC ? sl : 0, GVEC ? NSL : 1);
+    if (phase == 0 && act && a.gx) S::store_in(a.gx + (int64_t)node * in_dim, mul, c, gx);
+  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -973,7 +983,15 @@ struct SenderLaunch {
     const size_t sm = (size_t)(st > 1 ? (st - 1) * groups * S::IN_PC * 32 : 0) * sizeof(float) +
                       (GVEC && NSL > 1 ? (size_t)st * 32 * NSL * 4 * sizeof(float) : 0);
     const unsigned grid = GVEC ? (unsigned)a.N : (unsigned)a.N * a.n_slices;
-    if constexpr (DBWD)
+    if constexpr (DBWD && GVEC && kSplitDbwd<S>) {
+      // g_x and g_w first (no g_vec work, slices independent), then g_vec
+      const size_t sm1 = (size_t)(st > 1 ? (st - 1) * S::IN_PC * 32 : 0) * sizeof(float);
+      k_dbwd_send<S, false, 1, MUL, FAST, 1><<<(unsigned)a.N * a.n_slices, 32 * st, sm1, s>>>(a);
+      count_launches(1);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      k_dbwd_send<S, GVEC, NSL, MUL, FAST, 2><<<grid, 32 * st * groups, sm, s>>>(a);
+    } else if constexpr (DBWD)
       k_dbwd_send<S, GVEC, NSL, MUL, FAST><<<grid, 32 * st * groups, sm, s>>>(a);
     else
       k_bwd_uvu<S, GVEC, NSL, kPrefetch<S>, MUL, FAST><<<grid, 32 * st * groups, sm, s>>>(a);
