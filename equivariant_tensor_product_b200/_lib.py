@@ -35,6 +35,7 @@ SIGNATURES = {
     "tp_last_error_message": (C.c_char_p, []),
     "tp_version": (C.c_char_p, []),
     "tp_launch_count": (C.c_int64, []),
+    "tp_check_bounded_waits": (C.c_int, [_i64, _p, C.POINTER(_i32)]),
 }
 
 _LIB = None

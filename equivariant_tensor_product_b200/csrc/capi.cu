@@ -31,6 +31,7 @@ struct tp_plan_s {
 };
 
 #include <atomic>
+#include <mutex>
 namespace tp {
 static std::atomic<long long> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
@@ -196,10 +197,31 @@ LaunchArgs base_args(tp_plan_t plan, int64_t N, int64_t E) {
 }
 
 // Validates the CSR on the device (debug flag only) and resets the error word.
+// Sticky per-device error word for plans without TP_FLAG_CHECK_INDICES: the pipelined
+// kernels record a wait that gave up (code 6) here; tp_get_device_error reads and clears it.
+__device__ int g_device_error;
+
+int* device_error_word() {
+  static std::mutex mu;
+  static int* ptr[64] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    ptr[dev] = static_cast<int*>(p);
+  }
+  return ptr[dev];
+}
+
 tp_status_t debug_prologue(tp_plan_t plan, int64_t N, int64_t E, const int32_t* rowptr,
                            const int32_t* src, void* ws, cudaStream_t s, int** err) {
   *err = nullptr;
-  if (!(plan->flags & TP_FLAG_CHECK_INDICES)) return TP_OK;
+  if (!(plan->flags & TP_FLAG_CHECK_INDICES)) {
+    *err = device_error_word();
+    return TP_OK;
+  }
   if (!ws) return fail(TP_ERR_WORKSPACE, "TP_FLAG_CHECK_INDICES needs a workspace for the error word");
   int* e = reinterpret_cast<int*>(ws);
   cudaError_t st = cudaMemsetAsync(e, 0, sizeof(int), s);
@@ -563,9 +585,19 @@ tp_status_t tp_conv_dbwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* ro
 tp_status_t tp_get_device_error(tp_plan_t plan, void* ws, tp_stream_t stream, int32_t* code) {
   if (!plan || !code) return fail(TP_ERR_INVALID_ARG, "plan and code must not be NULL");
   *code = 0;
-  if (!(plan->flags & TP_FLAG_CHECK_INDICES)) return TP_OK;
-  if (!ws) return fail(TP_ERR_WORKSPACE, "workspace is NULL");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!(plan->flags & TP_FLAG_CHECK_INDICES)) {
+    int* word = device_error_word();
+    if (!word) return fail(TP_ERR_CUDA, "device error word unavailable");
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, word, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e, "tp_get_device_error");
+    *code = v;
+    return TP_OK;
+  }
+  if (!ws) return fail(TP_ERR_WORKSPACE, "workspace is NULL");
   int32_t v = 0;
   cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);

@@ -291,11 +291,12 @@ __device__ __forceinline__ unsigned long long now_ns() {
 }
 
 // Time-bounded wait on a slot; false on timeout.
-__device__ __forceinline__ bool slot_wait(uint32_t mbar, uint32_t parity) {
+__device__ __forceinline__ bool slot_wait(uint32_t mbar, uint32_t parity,
+                                          unsigned long long limit_ns = kGatherWaitNs) {
   if (slot_ready(mbar, parity)) return true;
   const unsigned long long t0 = now_ns();
   while (!slot_ready(mbar, parity))
-    if (now_ns() - t0 > kGatherWaitNs) return false;
+    if (now_ns() - t0 > limit_ns) return false;
   return true;
 }
 

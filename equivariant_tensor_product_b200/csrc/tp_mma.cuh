@@ -134,12 +134,13 @@ __device__ __forceinline__ unsigned long long global_ns() {
 // Wait bounded in time (a try_wait may suspend the thread for a while, so the bound is on
 // the clock, not on the number of polls) that also gives up when another role has aborted.
 // On its own timeout it raises the abort flag.  Returns false when the caller must stop.
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns = kWaitNs) {
   const unsigned long long t0 = global_ns();
   for (;;) {
     if (mbar_try_wait(mbar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_ns() - t0 > kWaitNs) break;
+    if (global_ns() - t0 > limit_ns) break;
   }
   *abort_flag = 1;
   return false;

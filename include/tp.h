@@ -46,6 +46,14 @@
  * CUDA launch failures return TP_ERR_CUDA.  Kernels never trap: with TP_FLAG_CHECK_INDICES
  * they bounds-check rowptr/src/perm, skip bad entries and record the first problem in the
  * workspace error word, readable with tp_get_device_error; outputs are then unspecified.
+ * Every device-side wait (the copy-engine rings of the staged edge passes, the tensor-core
+ * pipeline of the uvw GEMMs) is bounded by the GPU clock (4 s); a wait that gives up records
+ * code 6 (= TP_ERR_TIMEOUT) -- in the workspace word in check mode, otherwise in a per-device
+ * word -- and the kernel drains its copies and returns; tp_get_device_error reports it.
+ *
+ * Alignment.  4 bytes is required.  Rows that start on 16-byte boundaries (any torch
+ * allocation) let the 32-channel lmax-2 forward and the uvw edge passes stage them with the
+ * copy engine; otherwise the same results come from the unstaged kernels.
  * tp_last_error_message returns this thread's detail text of the last failing call.
  */
 #ifndef TP_H_
@@ -68,7 +76,7 @@ typedef enum {
   TP_ERR_BAD_GRAPH = 3,    /* inconsistent CSR found on the host (sizes) */
   TP_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than tp_workspace_size */
   TP_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
-  TP_ERR_TIMEOUT = 6       /* reserved: a bounded device wait gave up */
+  TP_ERR_TIMEOUT = 6       /* a bounded device wait gave up (device error code 6) */
 } tp_status_t;
 
 enum { TP_MODE_UVU = 0, TP_MODE_UVW = 1 };
@@ -80,7 +88,9 @@ enum { TP_OP_FWD = 0, TP_OP_BWD = 1, TP_OP_DBWD = 2 };
  *   (multiplicity 1, parity (-1)^l).  paths: [n_paths][3] = (i_in, i_sh, i_out) block
  *   indices; their order fixes the weight layout.  Rules: triangle |l1-l2| <= l3 <= l1+l2,
  *   parity p3 = p1 * p2, uvu needs mul_in == mul_out.  path_coeff: NULL = all 1.0.
- *   All blocks of irreps_in share one multiplicity, and of irreps_out too.
+ *   All blocks of irreps_in share one multiplicity, and of irreps_out too.  uvw needs
+ *   multiplicities that are multiples of 4 (its GEMM operands are loaded by TMA, whose row
+ *   pitch must be a multiple of 16 bytes); others return TP_ERR_UNSUPPORTED.
  * Errors: TP_ERR_INVALID_ARG (syntax, rule violations), TP_ERR_UNSUPPORTED (no compiled
  * specialisation for this path list: the build ships lmax 1/2/3 "all paths" lists and the
  * 4-path lmax-1 list; or l > 3; or uvw on a list without a uvw kernel). */
@@ -147,10 +157,19 @@ tp_status_t tp_conv_dbwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* ro
                          float* g_gy, float* g_x, float* g_w, float* g_vec, void* ws,
                          size_t ws_bytes, tp_stream_t stream);
 
-/* Reads (and clears) the device error word of a workspace after the work on `stream`
- * finished; synchronises the stream.  *code: 0 = none, 1 = bad rowptr, 2 = bad src,
- * 3 = bad perm / transpose entry. */
+/* Reads (and clears) the device error word after the work on `stream` finished;
+ * synchronises the stream.  Check-mode plans read the word of workspace `ws`; other plans
+ * read the per-device word (ws unused).  *code: 0 = none, 1 = bad rowptr, 2 = bad src,
+ * 3 = bad perm / transpose entry, 6 = a bounded device wait gave up. */
 tp_status_t tp_get_device_error(tp_plan_t plan, void* ws, tp_stream_t stream, int32_t* code);
+
+/* Self-check of the bounded waits (no counterpart on the pages; failure detection).  Runs the
+ * two wait primitives the pipelined kernels use -- the copy-engine slot wait and the
+ * tensor-core pipeline wait with its abort flag -- on a barrier that is never signalled,
+ * with limit_ns (1 ns .. 1 s), and synchronises `stream`.  *gave_up: bit 0 = slot wait gave
+ * up, bit 1 = pipeline wait gave up, bit 2 = it raised the abort flag; 7 is the designed
+ * outcome.  TP_ERR_INVALID_ARG for a NULL result or a limit outside (0, 1 s]. */
+tp_status_t tp_check_bounded_waits(int64_t limit_ns, tp_stream_t stream, int32_t* gave_up);
 
 /* Number of kernels this library has launched in the calling process (diagnostics: lets a
  * benchmark count its own launches in a timed region). */

@@ -173,3 +173,10 @@ def test_no_cpu_fallback_without_device(lib, tp):
     st = lib.tp_conv_fwd(plan.handle, 4, 8, fake, fake, fake, fake, fake, None, fake, fake, 256, None)
     assert st == 5
     assert b"cuda" in lib.tp_last_error_message().lower() or lib.tp_last_error_message()
+
+
+def test_bounded_wait_check_rejects_bad_arguments_before_the_device(lib):
+    res = C.c_int32(-1)
+    assert lib.tp_check_bounded_waits(0, None, C.byref(res)) == 1
+    assert lib.tp_check_bounded_waits(2_000_000_000, None, C.byref(res)) == 1
+    assert lib.tp_check_bounded_waits(1000, None, None) == 1
