@@ -422,43 +422,79 @@ def run_ours(args, rank, world, local):
     bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     dbwd_ms = statistics.mean(e[3].elapsed_time(e[6]) for e in evs) if with_dbwd else None
 
-    # end to end through the same calls, inputs from pinned host memory, outputs back to host
+    # End to end through the same calls: every step copies its inputs from pinned host memory
+    # and its results back.  Two device buffer sets let the copies overlap: the inputs of step
+    # k+1 go up and the results of step k-1 come down (each on its own copy stream) while step
+    # k computes; nothing is skipped or cached between steps.
     e2e_keys = keys + (["ggx", "ggw", "ggvec"] if with_dbwd else [])
     host_in = {k: torch.as_tensor(np.ascontiguousarray(d[k])).pin_memory() for k in e2e_keys}
-    dev_in = {k: torch.empty_like(host_in[k], device=dev) for k in e2e_keys}
     outs = (y, gx, gw) + ((gvec,) if want_gvec else ()) + ((gW,) if uvw else ()) + \
         ((g_gy, g_x, g_w, g_vec) if with_dbwd else ())
     host_out = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in outs]
-    Wd = P(dev_in["W"]) if uvw else None
-    e2e_args = (
-        (h, N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(dev_in["x"]), P(dev_in["vec"]), P(dev_in[wkey]), Wd,
-         P(y), P(ws), ws_bytes, sh),
-        (N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(ws_t), ws_t_bytes, sh),
-        (h, N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(dev_in["x"]), P(dev_in["vec"]),
-         P(dev_in[wkey]), Wd, P(dev_in["gy"]), P(gx), P(gw), P(gvec), P(gW), P(ws), ws_bytes, sh))
-    if with_dbwd:
-        e2e_dargs = (h, N, E, P(dev_in["rowptr"]), P(dev_in["src"]), P(colptr), P(perm), P(dev_in["x"]),
-                     P(dev_in["vec"]), P(dev_in[wkey]), None, P(dev_in["gy"]), P(dev_in["ggx"]), P(dev_in["ggw"]),
-                     P(dev_in["ggvec"]), P(g_gy), P(g_x), P(g_w), P(g_vec), P(ws), ws_bytes, sh)
-
-    def e2e_step():
-        for k in e2e_keys:
-            dev_in[k].copy_(host_in[k], non_blocking=True)
-        st = fwd_f(*e2e_args[0]) | tr_f(*e2e_args[1]) | bwd_f(*e2e_args[2])
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    sets = []
+    for b in range(2):
+        dv = {k: torch.empty_like(host_in[k], device=dev) for k in e2e_keys}
+        ob = [torch.empty_like(t_) for t_ in outs]
+        o = dict(zip(["y", "gx", "gw"] + (["gvec"] if want_gvec else []) + (["gW"] if uvw else []) +
+                     (["g_gy", "g_x", "g_w", "g_vec"] if with_dbwd else []), ob))
+        cpb = torch.empty(N + 1, dtype=torch.int32, device=dev)
+        pmb = torch.empty(E, dtype=torch.int32, device=dev)
+        Wd = P(dv["W"]) if uvw else None
+        fa = (h, N, E, P(dv["rowptr"]), P(dv["src"]), P(dv["x"]), P(dv["vec"]), P(dv[wkey]), Wd, P(o["y"]), P(ws),
+              ws_bytes, sh)
+        ta = (N, E, P(dv["rowptr"]), P(dv["src"]), P(cpb), P(pmb), P(ws_t), ws_t_bytes, sh_side)
+        ba = (h, N, E, P(dv["rowptr"]), P(dv["src"]), P(cpb), P(pmb), P(dv["x"]), P(dv["vec"]), P(dv[wkey]), Wd,
+              P(dv["gy"]), P(o["gx"]), P(o["gw"]), P(o.get("gvec")), P(o.get("gW")), P(ws), ws_bytes, sh)
+        da = None
         if with_dbwd:
-            st |= dbwd_f(*e2e_dargs)
+            da = (h, N, E, P(dv["rowptr"]), P(dv["src"]), P(cpb), P(pmb), P(dv["x"]), P(dv["vec"]), P(dv[wkey]), None,
+                  P(dv["gy"]), P(dv["ggx"]), P(dv["ggw"]), P(dv["ggvec"]), P(o["g_gy"]), P(o["g_x"]), P(o["g_w"]),
+                  P(o["g_vec"]), P(ws), ws_bytes, sh)
+        sets.append((dv, ob, fa, ta, ba, da))
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    tr2_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step(k):
+        b = k % 2
+        dv, ob, fa, ta, ba, da = sets[b]
+        s_h2d.wait_event(comp_done[b])            # buffer set b is free once step k-2 has computed
+        with torch.cuda.stream(s_h2d):
+            for key in e2e_keys:
+                dv[key].copy_(host_in[key], non_blocking=True)
+        h2d_done[b].record(s_h2d)
+        side.wait_event(h2d_done[b])
+        st = tr_f(*ta)
+        tr2_done[b].record(side)
+        stream.wait_event(h2d_done[b])
+        stream.wait_event(d2h_done[b])            # step k-2's results are out of set b
+        st |= fwd_f(*fa)
+        stream.wait_event(tr2_done[b])
+        st |= bwd_f(*ba)
+        if with_dbwd:
+            st |= dbwd_f(*da)
+        comp_done[b].record(stream)
         if st:
             raise RuntimeError(lib.tp_last_error_message().decode())
-        for ho, dv in zip(host_out, outs):
-            ho.copy_(dv, non_blocking=True)
+        s_d2h.wait_event(comp_done[b])
+        with torch.cuda.stream(s_d2h):
+            for ho, t_ in zip(host_out, ob):
+                ho.copy_(t_, non_blocking=True)
+        d2h_done[b].record(s_d2h)
 
-    for _ in range(3):
-        e2e_step()
+    for k in range(3):
+        e2e_step(k)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
+    s_h2d.wait_stream(stream)
+    s_d2h.wait_stream(stream)
+    side.wait_stream(stream)
+    for k in range(args.e2e_steps):
+        e2e_step(k)
+    stream.wait_stream(s_d2h)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_s = e0.elapsed_time(e1) / 1e3
@@ -518,7 +554,9 @@ def run_ours(args, rank, world, local):
                              f"{l2 / 1e6:.0f} MB)", "parallelism": "replicas" if world > 1 else "single"},
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "edges/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": args.e2e_steps},
+                    "steps": args.e2e_steps,
+                    "pipeline": "two device buffer sets; the H2D copy of step k+1 and the D2H copy of step k-1 "
+                                "overlap step k on their own streams"},
             "gpu_launches": int(launches), "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
