@@ -336,7 +336,7 @@ def run_ours(args, rank, world, local):
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     ws_t_bytes = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD) if not uvw else 256 + 8 * (N + E) + 4096
     ws_t = torch.empty(ws_t_bytes, dtype=torch.uint8, device=dev)      # side-stream transpose scratch
-    stream = torch.cuda.current_stream(dev)
+    stream = torch.cuda.Stream(dev)    # a capturable stream for all of the bench's work
     side = torch.cuda.Stream(dev)
     sh = stream.cuda_stream
     sh_side = side.cuda_stream
@@ -421,6 +421,57 @@ def run_ours(args, rank, world, local):
     tr_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in evs)
     bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     dbwd_ms = statistics.mean(e[3].elapsed_time(e[6]) for e in evs) if with_dbwd else None
+    eager_ms_per_step = 1e3 * elapsed_max / args.steps
+
+    # The same steps replayed as CUDA graphs (one per input copy, captured from the same C ABI
+    # calls: transpose forked onto the side stream, joined before the backward), which removes
+    # the host launch path from between the kernels.  The per-call times above come from the
+    # eager loop; the step throughput from this one when the capture succeeds.
+    launch_mode, graph_note = "eager", None
+    graphs = []
+    try:
+        n_cap = lib.tp_launch_count()
+        for r in range(R):
+            g = torch.cuda.CUDAGraph()
+            fork, join = torch.cuda.Event(), torch.cuda.Event()
+            a_f, a_t, a_b = argsets[r]
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+                fork.record(stream)
+                side.wait_event(fork)
+                st = tr_f(*a_t)
+                join.record(side)
+                st |= fwd_f(*a_f)
+                stream.wait_event(join)
+                st |= bwd_f(*a_b)
+                if with_dbwd:
+                    st |= dbwd_f(*dargs[r])
+            if st:
+                raise RuntimeError(lib.tp_last_error_message().decode())
+            graphs.append(g)
+        per_step_launches = (lib.tp_launch_count() - n_cap) // R
+    except Exception as exc:  # noqa: BLE001
+        graphs, graph_note = [], f"capture failed: {exc}"[:200]
+    if graphs:
+        with torch.cuda.stream(stream):
+            for k in range(args.warmup):
+                graphs[k % R].replay()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        with ClockSampler(local) as clk:
+            start.record(stream)
+            with torch.cuda.stream(stream):
+                for k in range(args.steps):
+                    graphs[k % R].replay()
+            stop.record(stream)
+            torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        elapsed = start.elapsed_time(stop) / 1e3
+        elapsed_max = max_over_ranks(elapsed, world, dev)
+        launches = per_step_launches * args.steps
+        launch_mode = "cuda_graph"
 
     # End to end through the same calls: every step copies its inputs from pinned host memory
     # and its results back.  Two device buffer sets let the copies overlap: the inputs of step
@@ -550,6 +601,8 @@ def run_ours(args, rank, world, local):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOADS[args.workload], "name": args.workload, "N": N, "E": E,
                        "order": "cell-sorted" if args.order == "cell" else "generation order (random)",
+                       "launch": launch_mode, "eager_ms_per_step": eager_ms_per_step,
+                       **({"graph_note": graph_note} if graph_note else {}),
                        "l2": f"{R} rotating input copies of {copy_bytes / 1e6:.1f} MB (> 2x L2 of "
                              f"{l2 / 1e6:.0f} MB)", "parallelism": "replicas" if world > 1 else "single"},
             "roofline": roof, "cpu_baseline": cpu,
@@ -560,6 +613,7 @@ def run_ours(args, rank, world, local):
             "gpu_launches": int(launches), "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
+    graphs.clear()   # no graph outlives the process group
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
