@@ -105,6 +105,7 @@ template <class S, int NSL>
 __global__ void __launch_bounds__(kMaxThreads) k_uvw_edge_staged(const __grid_constant__ LaunchArgs a) {
   extern __shared__ __align__(128) unsigned char esm[];
   __shared__ __align__(8) uint64_t full_bar[kEdgeSlots];
+  __shared__ float sbat[32 * S::P];
   __shared__ uint32_t read_cnt[kEdgeSlots];
   __shared__ int last_fill[kEdgeSlots];
   __shared__ volatile int gather_failed;
@@ -153,6 +154,9 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_edge_staged(const __grid_co
         if (lane == 0) fill(first + k, j);
       }
     }
+    // the batch's path scalars (contiguous rows in receiver order), once for all warps
+    for (int t = threadIdx.x; t < ne * S::P; t += blockDim.x) sbat[t] = __ldg(a.w + (int64_t)base * S::P + t);
+    __syncthreads();
 #pragma unroll 1
     for (int k = 0; k < ne; ++k) {
       const int f = first + k, s2 = f % kEdgeSlots;
@@ -180,11 +184,9 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_edge_staged(const __grid_co
         if (k + kEdgeSlots < ne) fill(f + kEdgeSlots, jnext);
       }
       if (!ok) continue;
-      const int e = base + k;
       float sp[S::P];
-      const float* srow = a.w + (int64_t)e * S::P;
 #pragma unroll
-      for (int p = 0; p < S::P; ++p) sp[p] = __ldg(srow + p) * (a.has_coeff ? a.coeff[p] : 1.f);
+      for (int p = 0; p < S::P; ++p) sp[p] = sbat[k * S::P + p] * (a.has_coeff ? a.coeff[p] : 1.f);
       const float ux = __shfl_sync(kFull, vx, k), uy = __shfl_sync(kFull, vy, k), uz = __shfl_sync(kFull, vz, k);
       float rx, ry, rz, ir;
       edge_geometry(ux, uy, uz, rx, ry, rz, ir);
@@ -434,6 +436,7 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
   __shared__ int last_fill[kSendSlots];
   __shared__ volatile int gather_failed;
   __shared__ int32_t rtab[kRowTab];
+  __shared__ float sbat[STAGED ? 32 * S::P : 1];
   const int lane = threadIdx.x & 31;
   const int sl = threadIdx.x >> 5;
   const int node = blockIdx.x;
@@ -501,6 +504,12 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
           if (lane == 0) fill(first + k, i);
         }
       }
+      // the batch's path scalars, once for all slice warps
+      for (int t = threadIdx.x; t < ne * S::P; t += blockDim.x) {
+        const int kk = t / S::P;
+        sbat[t] = __ldg(a.w + (int64_t)__ldg(a.perm + base + kk) * S::P + (t - kk * S::P));
+      }
+      __syncthreads();
     }
 #pragma unroll 1
     for (int k = 0; k < ne; ++k) {
@@ -531,9 +540,14 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
       for (int p = 0; p < S::P; ++p) gs[p] = 0.f;
       if (e >= 0) {
         float s[S::P];
-        const float* srow = a.w + (int64_t)e * S::P;
+        if constexpr (STAGED) {
 #pragma unroll
-        for (int p = 0; p < S::P; ++p) s[p] = __ldg(srow + p) * (a.has_coeff ? a.coeff[p] : 1.f);
+          for (int p = 0; p < S::P; ++p) s[p] = sbat[k * S::P + p] * (a.has_coeff ? a.coeff[p] : 1.f);
+        } else {
+          const float* srow = a.w + (int64_t)e * S::P;
+#pragma unroll
+          for (int p = 0; p < S::P; ++p) s[p] = __ldg(srow + p) * (a.has_coeff ? a.coeff[p] : 1.f);
+        }
         if (act && grow) {
           float gyv[S::OUT_PC];
           if constexpr (STAGED) {
