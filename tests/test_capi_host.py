@@ -180,3 +180,23 @@ def test_bounded_wait_check_rejects_bad_arguments_before_the_device(lib):
     assert lib.tp_check_bounded_waits(0, None, C.byref(res)) == 1
     assert lib.tp_check_bounded_waits(2_000_000_000, None, C.byref(res)) == 1
     assert lib.tp_check_bounded_waits(1000, None, None) == 1
+
+
+def test_missing_library_fails_loudly_on_first_call(tmp_path):
+    """Without libtp.so the package still imports (so its build step can run), and the
+    first call raises instead of computing anything another way."""
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "import equivariant_tensor_product_b200._lib as L\n"
+        "L.LIB_PATH = %r\n"
+        "import equivariant_tensor_product_b200 as tp, synth\n"
+        "s = synth.CONFIGS['c1']\n"
+        "try:\n"
+        "    tp.Plan(s.irreps_in, s.irreps_sh, s.irreps_out, s.paths)\n"
+        "except ImportError as e:\n"
+        "    print('ImportError', e)\n"
+    ) % (ROOT, str(tmp_path / "libtp.so"))
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert "ImportError" in out.stdout and "libtp.so is missing" in out.stdout, (out.stdout, out.stderr)
