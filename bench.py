@@ -31,6 +31,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "edges/sec for fused TP conv fwd/fwd+bwd on 1 B200; % of HBM/FLOP roofline"
 WORKLOADS = {
+    "c1": "tiny correctness graph: 24 nodes x 8 incoming edges (192 edges), 4x0e+4x1o -> 4x0e+4x1o, SH lmax 1, "
+          "uvu, 4 paths; forward only (a latency: the graph is far too small to load the GPU)",
     "c2": "NequIP-like: 1,536 atoms, 46,080 directed edges, 32x0e+32x1o+32x2e -> "
           "32x0e+32x1e+32x1o+32x2e+32x2o, SH lmax 2, uvu, 15 paths; step = fwd + transpose + bwd(gx, gw)",
     "c3": "SevenNet/MACE-like l=3: 4,096 atoms, ~163k edges, 64x(0e,1o,2e,3o), SH lmax 3, uvu, 34 paths; "
@@ -644,11 +646,90 @@ def run_ours(args, rank, world, local):
     return 0
 
 
+def run_latency(args, rank, world, local):
+    """Forward-only workloads too small to load the GPU (c1): per-call latency through the C
+    ABI (CUDA events around each call, median), and the same call replayed as a CUDA graph."""
+    import torch
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from equivariant_tensor_product_b200 import build as tpbuild
+    tpbuild.build()
+    import equivariant_tensor_product_b200 as tp
+    import synth
+    lib = tp.load()
+    spec = synth.CONFIGS[args.workload]
+    d = synth.make_inputs(args.workload, args.n_atoms, seed=spec.seed + 7919 * rank)
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, spec.mode)
+    N, E = len(d["rowptr"]) - 1, len(d["src"])
+    g = {k: torch.as_tensor(np.ascontiguousarray(d[k])).to(dev) for k in ("rowptr", "src", "x", "vec", "w")}
+    y = torch.empty(N, plan.out_dim, device=dev)
+    stream = torch.cuda.Stream(dev)
+    P = lambda t: C.c_void_p(t.data_ptr())
+    a = (plan.handle, N, E, P(g["rowptr"]), P(g["src"]), P(g["x"]), P(g["vec"]), P(g["w"]), None, P(y), None, 0,
+         stream.cuda_stream)
+    for _ in range(args.warmup):
+        lib.tp_conv_fwd(*a)
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        for e0, e1 in evs:
+            e0.record(stream)
+            if lib.tp_conv_fwd(*a):
+                raise RuntimeError(lib.tp_last_error_message().decode())
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+    lat_ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=stream, capture_error_mode="thread_local"):
+        lib.tp_conv_fwd(*a)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            gr.replay()
+        start.record(stream)
+        for _ in range(args.steps):
+            gr.replay()
+        stop.record(stream)
+    torch.cuda.synchronize(dev)
+    graph_ms = start.elapsed_time(stop) / args.steps
+    # end to end: inputs up, forward, y down, each call
+    host = {k: torch.as_tensor(np.ascontiguousarray(d[k])).pin_memory() for k in ("rowptr", "src", "x", "vec", "w")}
+    hy = torch.empty(y.shape).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for k in host:
+                g[k].copy_(host[k], non_blocking=True)
+            lib.tp_conv_fwd(*a)
+            hy.copy_(y, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / max(args.e2e_steps, 1)
+    if rank == 0:
+        line = {"metric": METRIC, "value": E / (graph_ms * 1e-3), "unit": "edges/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": graph_ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOADS[args.workload], "name": args.workload, "N": N, "E": E,
+                           "launch": "cuda_graph", "eager_latency_us_median": 1e3 * lat_ms,
+                           "graph_latency_us": 1e3 * graph_ms, "parallelism": "single"},
+                "roofline": {"bound": "latency", "note": "192 edges: launch latency, no roofline applies"},
+                "cpu_baseline": None,
+                "e2e": {"value": E / (e2e_ms * 1e-3), "unit": "edges/s",
+                        "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host.values()),
+                        "d2h_bytes_per_step": hy.numel() * 4, "steps": args.e2e_steps},
+                "gpu_launches": args.steps, "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, rank)
+    if args.workload == "c1":
+        return run_latency(args, rank, world, local)
     return run_ours(args, rank, world, local)
 
 
