@@ -36,6 +36,19 @@ SIGNATURES = {
     "tp_version": (C.c_char_p, []),
     "tp_launch_count": (C.c_int64, []),
     "tp_check_bounded_waits": (C.c_int, [_i64, _p, C.POINTER(_i32)]),
+    # node-side operators (include/tp_block.h)
+    "tp_linear_create": (C.c_int, [C.POINTER(_p), C.c_char_p, C.c_char_p, _p]),
+    "tp_linear_destroy": (C.c_int, [_p]),
+    "tp_linear_query": (C.c_int, [_p, C.POINTER(_i64), C.POINTER(_i64), C.POINTER(_i64), C.POINTER(_i32)]),
+    "tp_linear_workspace_size": (C.c_int, [_p, _i64, _i32, C.POINTER(_sz)]),
+    "tp_linear_fwd": (C.c_int, [_p, _i64, _p, _p, _p, _i32, _p, _sz, _p]),
+    "tp_linear_bwd": (C.c_int, [_p, _i64, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "tp_gate_create": (C.c_int, [C.POINTER(_p), C.c_char_p, C.c_char_p, C.c_char_p]),
+    "tp_gate_destroy": (C.c_int, [_p]),
+    "tp_gate_query": (C.c_int, [_p, C.POINTER(_i64), C.POINTER(_i64)]),
+    "tp_gate_fwd": (C.c_int, [_p, _i64, _p, _p, _p]),
+    "tp_gate_bwd": (C.c_int, [_p, _i64, _p, _p, _p, _p]),
+    "tp_gate_dbwd": (C.c_int, [_p, _i64, _p, _p, _p, _p, _p, _p]),
 }
 
 _LIB = None

@@ -65,3 +65,98 @@ class TPConv(torch.autograd.Function):
 def tp_conv(plan: Plan, graph: Graph, x, vec, w):
     """y = conv(x, vec, w) with first and second derivatives through the CUDA kernels (uvu)."""
     return TPConv.apply(x, vec, w, plan, graph)
+
+
+# ---------------------------------------------------------------------------------------------
+# Node-side operators (include/tp_block.h).  The linear map's second-order terms are again
+# applications of the map and its adjoint: g_gy = fwd(ggx; W) + fwd(x; ggW),
+# g_x = bwd(gy; ggW).gx, g_W = bwd(ggx, gy).gW -- the same two entry points with other
+# arguments.  The gate's come from tp_gate_dbwd.
+# ---------------------------------------------------------------------------------------------
+
+from .block import Gate, Linear, tp_gate_bwd, tp_gate_dbwd, tp_gate_fwd, tp_linear_bwd, tp_linear_fwd  # noqa: E402
+
+
+class _LinearBwd(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, W, gy, lin, needs):
+        gx, gW = tp_linear_bwd(lin, x, W, gy, need_gx=needs[0], need_gW=needs[1])
+        ctx.save_for_backward(x, W, gy)
+        ctx.lin = lin
+        return gx, gW
+
+    @staticmethod
+    def backward(ctx, ggx, ggW):
+        x, W, gy = ctx.saved_tensors
+        lin = ctx.lin
+        c = lambda t: None if t is None else t.contiguous()
+        ggx, ggW = c(ggx), c(ggW)
+        g_x = g_W = g_gy = None
+        if ctx.needs_input_grad[2]:
+            if ggx is not None:
+                g_gy = tp_linear_fwd(lin, ggx, W)
+            if ggW is not None:
+                g_gy = tp_linear_fwd(lin, x, ggW, y=g_gy, accumulate=g_gy is not None)
+        if ctx.needs_input_grad[0] and ggW is not None:
+            g_x, _ = tp_linear_bwd(lin, None, ggW, gy, need_gx=True, need_gW=False)
+        if ctx.needs_input_grad[1] and ggx is not None:
+            _, g_W = tp_linear_bwd(lin, ggx, None, gy, need_gx=False, need_gW=True)
+        return g_x, g_W, g_gy, None, None
+
+
+class LinearFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, W, lin):
+        x, W = x.contiguous(), W.contiguous()
+        y = tp_linear_fwd(lin, x, W)
+        ctx.save_for_backward(x, W)
+        ctx.lin = lin
+        return y
+
+    @staticmethod
+    def backward(ctx, gy):
+        x, W = ctx.saved_tensors
+        needs = (ctx.needs_input_grad[0], ctx.needs_input_grad[1])
+        gx, gW = _LinearBwd.apply(x, W, gy.contiguous(), ctx.lin, needs)
+        return gx, gW, None
+
+
+def tp_linear(lin: Linear, x, W):
+    """y = linear(x; W) with first and second derivatives through the CUDA kernels."""
+    return LinearFn.apply(x, W, lin)
+
+
+class _GateBwd(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, gy, gate):
+        gx = tp_gate_bwd(gate, x, gy)
+        ctx.save_for_backward(x, gy)
+        ctx.gate = gate
+        return gx
+
+    @staticmethod
+    def backward(ctx, ggx):
+        x, gy = ctx.saved_tensors
+        g_gy, g_x = tp_gate_dbwd(ctx.gate, x, gy, ggx.contiguous(), need_g_gy=ctx.needs_input_grad[1],
+                                 need_g_x=ctx.needs_input_grad[0])
+        return g_x, g_gy, None
+
+
+class GateFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, gate):
+        x = x.contiguous()
+        y = tp_gate_fwd(gate, x)
+        ctx.save_for_backward(x)
+        ctx.gate = gate
+        return y
+
+    @staticmethod
+    def backward(ctx, gy):
+        (x,) = ctx.saved_tensors
+        return _GateBwd.apply(x, gy.contiguous(), ctx.gate), None
+
+
+def tp_gate(gate: Gate, x):
+    """y = gate(x) with first and second derivatives through the CUDA kernels."""
+    return GateFn.apply(x, gate)

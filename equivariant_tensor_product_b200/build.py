@@ -36,7 +36,7 @@ def _nvcc() -> str:
 def _sources():
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu"))) + sorted(glob.glob(os.path.join(GEN, "*.cu")))
     headers = (glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-               + glob.glob(os.path.join(GEN, "*.h")) + [os.path.join(ROOT, "include", "tp.h")])
+               + glob.glob(os.path.join(GEN, "*.h")) + glob.glob(os.path.join(ROOT, "include", "*.h")))
     return srcs, headers
 
 

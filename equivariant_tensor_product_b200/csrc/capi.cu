@@ -12,6 +12,7 @@
 
 #include "../../include/tp.h"
 #include "tp_common.h"
+#include "tp_host.h"
 
 using namespace tp;
 
@@ -233,6 +234,25 @@ tp_status_t debug_prologue(tp_plan_t plan, int64_t N, int64_t E, const int32_t* 
 }
 
 }  // namespace
+
+namespace tp {
+
+bool parse_irreps_terms(const char* s, std::vector<IrrepTerm>& out, std::string& why) {
+  std::vector<IrrepBlock> blocks;
+  out.clear();
+  if (!parse_irreps(s, blocks, why)) return false;
+  for (const IrrepBlock& b : blocks) out.push_back(IrrepTerm{b.mul, b.l, b.parity});
+  return true;
+}
+
+tp_status_t set_failure(tp_status_t st, const std::string& msg) {
+  g_msg = msg;
+  return st;
+}
+
+int* device_error_ptr() { return device_error_word(); }
+
+}  // namespace tp
 
 extern "C" {
 
