@@ -41,7 +41,13 @@ WORKLOADS = {
           "step = fwd + transpose + bwd(gx, gw, gvec) + dbwd(g_gy, g_x, g_w, g_vec)",
     "c4": "large streaming uvw: 100,000 atoms, ~3.0M edges, 128x(0e,1o,2e) -> 128x(0e,1e,1o,2e,2o), SH lmax 2, "
           "per-path 128x128 mixing, 15 paths; step = fwd + transpose + bwd(gx, gs, gW)",
+    "c2-layer": "interaction layer on the c2 graph (1,536 atoms, 46,080 edges): linear 32x(0e,1o,2e) -> same, "
+                "convolution (c2 paths, coefficient 1/average degree), linear -> 32x0e+64x0e+32x1o+32x2e, gate "
+                "-> 32x(0e,1o,2e); step = that forward + transpose + the backward to x, both linear weights and "
+                "the edge weights",
 }
+LAYER_MID = "32x0e+64x0e+32x1o+32x2e"
+LAYER_GATE = ("32x0e", "64x0e", "32x1o+32x2e")
 
 
 def parse():
@@ -230,6 +236,8 @@ def run_reference(args, rank):
     import synth
     from oracle.conv import set_threads
     cores = set_threads()
+    if args.workload == "c2-layer":
+        return run_reference_layer(args, cores)
     d = synth.make_inputs(args.workload)
     oracle_sample(d, 4, seed=0)                      # CG tables cached outside the timing
     ef, tf, eb, tb = oracle_sample(d, 16, seed=1)
@@ -646,6 +654,327 @@ def run_ours(args, rank, world, local):
     return 0
 
 
+def layer_node_bytes(lin, N, bwd):
+    """Algorithmic bytes of one linear call: fwd reads x and W, writes y; bwd reads x, W and gy,
+    writes gx and gW."""
+    if bwd:
+        return 4 * N * (2 * lin.in_dim + lin.out_dim) + 8 * lin.n_weights
+    return 4 * N * (lin.in_dim + lin.out_dim) + 4 * lin.n_weights
+
+
+def oracle_layer_sample(d, n_rows, seed, W1, W2, g_out):
+    """The interaction layer in float64 on the host: the node-side operators on every node and
+    the convolution on the edges into / out of n_rows sampled rows (as oracle_sample)."""
+    from oracle.block import GateSpec, gate, gate_backward, linear, linear_backward
+    spec = d["spec"]
+    ir = spec.irreps_in
+    gs = GateSpec(*LAYER_GATE)
+    N = len(d["rowptr"]) - 1
+    E = len(d["src"])
+    t0 = time.perf_counter()
+    h1 = linear(ir, ir, d["x"], W1).numpy()
+    t1 = time.perf_counter()
+    dd = dict(d)
+    dd["x"] = h1.astype(np.float32)
+    ef, tf, eb, tb = oracle_sample(dd, n_rows, seed)
+    t2 = time.perf_counter()
+    y = d["gy"]        # a node array of the convolution's output width (the sampled conv gives no full y)
+    h2 = linear(spec.irreps_out, LAYER_MID, y, W2)
+    gate(gs, h2)
+    g_h2 = gate_backward(gs, h2, g_out)
+    linear_backward(spec.irreps_out, LAYER_MID, y, W2, g_h2)
+    linear_backward(ir, ir, d["x"], W1, np.asarray(d["x"]))
+    t3 = time.perf_counter()
+    node_t = (t1 - t0) + (t3 - t2)
+    return 1.0 / (tf / ef + tb / eb + node_t / E), ef, eb, tf + tb + node_t
+
+
+def layer_weights(spec, N, rank=0):
+    rng = np.random.default_rng(spec.seed + 17 + 7919 * rank)
+    from oracle.block import linear_weight_count
+    W1 = (rng.standard_normal(linear_weight_count(spec.irreps_in, spec.irreps_in)) / math.sqrt(32)).astype(np.float32)
+    W2 = (rng.standard_normal(linear_weight_count(spec.irreps_out, LAYER_MID)) / math.sqrt(32)).astype(np.float32)
+    g_out = rng.standard_normal((N, 288), dtype=np.float32)
+    return W1, W2, g_out
+
+
+def run_reference_layer(args, cores):
+    import synth
+    spec = synth.CONFIGS["c2"]
+    d = synth.make_inputs("c2")
+    N = len(d["rowptr"]) - 1
+    W1, W2, g_out = layer_weights(spec, N)
+    oracle_sample(d, 4, seed=0)
+    v, ef, eb, t = oracle_layer_sample(d, 16, 1, W1, W2, g_out)
+    rows = int(max(2, min(256, 16 * 60.0 / max(1, args.steps + args.warmup) / t)))
+    for k in range(args.warmup):
+        oracle_layer_sample(d, rows, k, W1, W2, g_out)
+    vals, tot = [], 0.0
+    for k in range(args.steps):
+        v, ef, eb, t = oracle_layer_sample(d, rows, 1000 + k, W1, W2, g_out)
+        vals.append(v)
+        tot += t
+    value = statistics.median(vals)
+    sample = (f"per step: linears and gate (fwd + bwd) on all {N} nodes, conv fwd into and bwd out of {rows} "
+              f"sampled rows, float64")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload], "name": args.workload},
+            "cpu_baseline": {"value": value, "unit": "edges/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_layer(args, rank, world, local):
+    """One interaction layer per step: linear -> convolution -> linear -> gate, then the
+    backward of all four to x, both linear weights and the edge weights, every call through
+    the C ABI on one capturable stream (the transpose on a side stream)."""
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from equivariant_tensor_product_b200 import build as tpbuild
+    tpbuild.build()
+    import equivariant_tensor_product_b200 as tp
+    import synth
+    lib = tp.load()
+
+    spec = synth.CONFIGS["c2"]
+    d = synth.make_inputs("c2", args.n_atoms, seed=spec.seed + 7919 * rank)
+    if args.order == "cell":
+        d = synth.cell_sorted(d)
+    N, E = len(d["rowptr"]) - 1, len(d["src"])
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvu",
+                   path_coeff=[N / max(E, 1)] * len(spec.paths))
+    lin1, lin2 = tp.Linear(spec.irreps_in, spec.irreps_in), tp.Linear(spec.irreps_out, LAYER_MID)
+    gate = tp.Gate(*LAYER_GATE)
+    W1, W2, d["g_out"] = layer_weights(spec, N, rank)
+    in_dim, out_dim, nw = plan.in_dim, plan.out_dim, plan.n_edge_weights
+
+    keys = ["rowptr", "src", "x", "vec", "w", "g_out"]
+    copy_bytes = sum(d[k].nbytes for k in keys)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(2, math.ceil(2.5 * l2 / copy_bytes))
+    copies = []
+    for r in range(R):
+        src_d = d
+        if r:
+            rr = np.random.default_rng(spec.seed + 31 * r + 7919 * rank)
+            src_d = dict(d)
+            src_d["x"] = rr.standard_normal(d["x"].shape, dtype=np.float32)
+            src_d["g_out"] = rr.standard_normal(d["g_out"].shape, dtype=np.float32)
+            src_d["w"] = (d["w"] * rr.uniform(0.5, 1.5, size=(1, nw))).astype(np.float32)
+        copies.append({k: torch.as_tensor(np.ascontiguousarray(src_d[k])).to(dev) for k in keys})
+    W1d, W2d = torch.as_tensor(W1).to(dev), torch.as_tensor(W2).to(dev)
+    f32 = lambda *shape: torch.empty(*shape, device=dev)
+    h1, y, h2, out = f32(N, in_dim), f32(N, out_dim), f32(N, lin2.out_dim), f32(N, gate.out_dim)
+    g_h2, g_y, g_h1, gx, gw = f32(N, lin2.out_dim), f32(N, out_dim), f32(N, in_dim), f32(N, in_dim), f32(E, nw)
+    gW1, gW2 = f32(lin1.n_weights), f32(lin2.n_weights)
+    colptrs = [torch.empty(N + 1, dtype=torch.int32, device=dev) for _ in range(R)]
+    perms = [torch.empty(E, dtype=torch.int32, device=dev) for _ in range(R)]
+    ws_bytes = max(tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD), tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    wl_bytes = max(tp.tp_linear_workspace_size(lin, N, op) for lin in (lin1, lin2) for op in (0, 1))
+    wl = torch.empty(wl_bytes, dtype=torch.uint8, device=dev)
+    wt_bytes = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD)
+    wt = torch.empty(wt_bytes, dtype=torch.uint8, device=dev)
+    stream, side = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    sh, sh_side = stream.cuda_stream, side.cuda_stream
+    P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None
+    lf, lb, gf, gb = lib.tp_linear_fwd, lib.tp_linear_bwd, lib.tp_gate_fwd, lib.tp_gate_bwd
+    cf, cb, tr_f = lib.tp_conv_fwd, lib.tp_conv_bwd, lib.tp_csr_transpose
+
+    def op_list(cp, colptr, perm):
+        return [
+            ("linear_in fwd", lf, (lin1.handle, N, P(cp["x"]), P(W1d), P(h1), 0, P(wl), wl_bytes, sh)),
+            ("conv fwd", cf, (plan.handle, N, E, P(cp["rowptr"]), P(cp["src"]), P(h1), P(cp["vec"]), P(cp["w"]),
+                              None, P(y), P(ws), ws_bytes, sh)),
+            ("linear_out fwd", lf, (lin2.handle, N, P(y), P(W2d), P(h2), 0, P(wl), wl_bytes, sh)),
+            ("gate fwd", gf, (gate.handle, N, P(h2), P(out), sh)),
+            ("gate bwd", gb, (gate.handle, N, P(h2), P(cp["g_out"]), P(g_h2), sh)),
+            ("linear_out bwd", lb, (lin2.handle, N, P(y), P(W2d), P(g_h2), P(g_y), P(gW2), P(wl), wl_bytes, sh)),
+            ("conv bwd", cb, (plan.handle, N, E, P(cp["rowptr"]), P(cp["src"]), P(colptr), P(perm), P(h1),
+                              P(cp["vec"]), P(cp["w"]), None, P(g_y), P(g_h1), P(gw), None, None, P(ws), ws_bytes, sh)),
+            ("linear_in bwd", lb, (lin1.handle, N, P(cp["x"]), P(W1d), P(g_h1), P(gx), P(gW1), P(wl), wl_bytes, sh)),
+        ]
+
+    ops = [op_list(cp, colptrs[r], perms[r]) for r, cp in enumerate(copies)]
+    targs = [(N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(wt), wt_bytes, sh_side)
+             for r, cp in enumerate(copies)]
+    names = [o[0] for o in ops[0]]
+    conv_bwd_at = names.index("conv bwd")
+    tr_done = [torch.cuda.Event() for _ in range(R)]
+    step_done = [torch.cuda.Event() for _ in range(R)]
+
+    def step(k, ev=None):
+        r = k % R
+        side.wait_event(step_done[r])
+        st = tr_f(*targs[r])
+        tr_done[r].record(side)
+        for i, (_, fn, a) in enumerate(ops[r]):
+            if i == conv_bwd_at:
+                stream.wait_event(tr_done[r])
+            if ev is not None:
+                ev[i].record(stream)
+            st |= fn(*a)
+        if ev is not None:
+            ev[len(names)].record(stream)
+        step_done[r].record(stream)
+        if st:
+            raise RuntimeError(lib.tp_last_error_message().decode())
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    n0 = lib.tp_launch_count()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for k in range(args.steps):
+        step(k, evs[k])
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    per_step_launches = (lib.tp_launch_count() - n0) // max(args.steps, 1)
+    eager_ms = start.elapsed_time(stop) / args.steps
+    op_ms = {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, nm in enumerate(names)}
+
+    # the same steps as CUDA graphs (one per input copy) for the step throughput
+    graphs, launch_mode, graph_note = [], "eager", None
+    try:
+        for r in range(R):
+            g = torch.cuda.CUDAGraph()
+            fork, join = torch.cuda.Event(), torch.cuda.Event()
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+                fork.record(stream)
+                side.wait_event(fork)
+                st = tr_f(*targs[r])
+                join.record(side)
+                for i, (_, fn, a) in enumerate(ops[r]):
+                    if i == conv_bwd_at:
+                        stream.wait_event(join)
+                    st |= fn(*a)
+            if st:
+                raise RuntimeError(lib.tp_last_error_message().decode())
+            graphs.append(g)
+    except Exception as exc:  # noqa: BLE001
+        graphs, graph_note = [], f"capture failed: {exc}"[:200]
+    if world > 1:
+        dist.barrier()
+    with ClockSampler(local) as clk:
+        if graphs:
+            with torch.cuda.stream(stream):
+                for k in range(args.warmup):
+                    graphs[k % R].replay()
+            torch.cuda.synchronize(dev)
+            start.record(stream)
+            with torch.cuda.stream(stream):
+                for k in range(args.steps):
+                    graphs[k % R].replay()
+            stop.record(stream)
+            launch_mode = "cuda_graph"
+        else:
+            start.record(stream)
+            for k in range(args.steps):
+                step(k)
+            stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed_max = max_over_ranks(start.elapsed_time(stop) / 1e3, world, dev)
+
+    # end to end through the same calls from pinned host memory, one step after the other:
+    # inputs up, the layer forward and backward, the gradients and the output down
+    host_in = {k: torch.as_tensor(np.ascontiguousarray(d[k])).pin_memory() for k in keys}
+    dv = {k: torch.empty_like(host_in[k], device=dev) for k in keys}
+    outs = (out, gx, gw, gW1, gW2)
+    host_out = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in outs]
+    e_ops = op_list(dv, colptrs[0], perms[0])
+    e_tr = (N, E, P(dv["rowptr"]), P(dv["src"]), P(colptrs[0]), P(perms[0]), P(wt), wt_bytes, sh)
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for k_ in keys:
+                dv[k_].copy_(host_in[k_], non_blocking=True)
+        st = tr_f(*e_tr)
+        for _, fn, a in e_ops:
+            st |= fn(*a)
+        if st:
+            raise RuntimeError(lib.tp_last_error_message().decode())
+        with torch.cuda.stream(stream):
+            for ho, t_ in zip(host_out, outs):
+                ho.copy_(t_, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_value = replica_throughput(E, args.e2e_steps, world, max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev))
+    h2d = sum(t_.numel() * t_.element_size() for t_ in host_in.values())
+    d2h = sum(t_.numel() * t_.element_size() for t_ in host_out)
+
+    if rank == 0:
+        hbm, _, peak_note = measured_peaks()
+        alg = {"linear_in fwd": layer_node_bytes(lin1, N, False), "conv fwd": fwd_bytes(N, E, in_dim, out_dim, nw),
+               "linear_out fwd": layer_node_bytes(lin2, N, False),
+               "gate fwd": 4 * N * (gate.in_dim + gate.out_dim),
+               "gate bwd": 4 * N * (2 * gate.in_dim + gate.out_dim),
+               "linear_out bwd": layer_node_bytes(lin2, N, True),
+               "conv bwd": bwd_bytes(N, E, in_dim, out_dim, nw, False),
+               "linear_in bwd": layer_node_bytes(lin1, N, True)}
+        kname = max(op_ms, key=op_ms.get)
+        achieved = alg[kname] / (op_ms[kname] * 1e-3) / 1e9
+        step_s = elapsed_max / args.steps
+        roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "peak_note": peak_note, "traffic": traffic_from_profile(kname, "c2-layer"),
+                "algorithmic_bytes_per_launch": alg[kname],
+                "ops": {nm: {"ms": op_ms[nm], "algorithmic_bytes": alg[nm],
+                             "hbm_frac": alg[nm] / (op_ms[nm] * 1e-3) / 1e9 / hbm} for nm in names},
+                "step_roofline_frac": (sum(alg.values()) / (hbm * 1e9)) / step_s}
+        cpu = None
+        if not args.no_cpu_baseline:
+            from oracle.conv import set_threads
+            cores = set_threads()
+            oracle_sample(d, 4, seed=0)
+            v, ef, eb, t = oracle_layer_sample(d, min(N, 1536), 3, W1, W2, d["g_out"])
+            cpu = {"value": v, "unit": "edges/s", "cores": cores, "kind": "oracle",
+                   "sample": f"linears and gate (fwd + bwd) on all {N} nodes; conv fwd on the {ef} edges into and "
+                             f"bwd on the {eb} edges out of {min(N, 1536)} sampled rows; float64, {t:.1f} s"}
+        line = {
+            "metric": METRIC, "value": replica_throughput(E, args.steps, world, elapsed_max), "unit": "edges/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * step_s,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload], "name": args.workload, "N": N, "E": E,
+                       "order": "cell-sorted" if args.order == "cell" else "generation order (random)",
+                       "launch": launch_mode, "eager_ms_per_step": eager_ms,
+                       **({"graph_note": graph_note} if graph_note else {}),
+                       "l2": f"{R} rotating input copies of {copy_bytes / 1e6:.1f} MB (> 2x L2 of {l2 / 1e6:.0f} MB)",
+                       "parallelism": "replicas" if world > 1 else "single"},
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "edges/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": args.e2e_steps, "pipeline": "sequential on one stream"},
+            "gpu_launches": int(per_step_launches * args.steps), "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    graphs.clear()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def run_latency(args, rank, world, local):
     """Forward-only workloads too small to load the GPU (c1): per-call latency through the C
     ABI (CUDA events around each call, median), and the same call replayed as a CUDA graph."""
@@ -730,6 +1059,8 @@ def main():
         return run_reference(args, rank)
     if args.workload == "c1":
         return run_latency(args, rank, world, local)
+    if args.workload == "c2-layer":
+        return run_layer(args, rank, world, local)
     return run_ours(args, rank, world, local)
 
 

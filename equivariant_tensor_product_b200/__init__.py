@@ -6,7 +6,7 @@ the first call (plan creation, any op, load()) raises ImportError when the libra
 been built.  Importing the package itself does not need the library, so that its build
 module (`python -m equivariant_tensor_product_b200.build`) runs in a fresh checkout.
 """
-from ._lib import (TP_FLAG_CHECK_INDICES, TP_MODE_UVU, TP_MODE_UVW, TP_OP_BWD, TP_OP_DBWD, TP_OP_FWD,  # noqa: F401
+from ._lib import (TP_FLAG_CHECK_INDICES, TP_LINEAR_CUDA_CORES, TP_LINEAR_TENSOR_CORES, TP_MODE_UVU, TP_MODE_UVW, TP_OP_BWD, TP_OP_DBWD, TP_OP_FWD,  # noqa: F401
                    TPError, load)
 from .ops import (Plan, tp_conv_bwd, tp_conv_dbwd, tp_conv_fwd, tp_csr_transpose, tp_get_device_error,  # noqa: F401
                   tp_plan_create, tp_plan_query, tp_version, tp_workspace_size)

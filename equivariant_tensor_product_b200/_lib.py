@@ -12,6 +12,7 @@ TP_OK, TP_ERR_INVALID_ARG, TP_ERR_UNSUPPORTED, TP_ERR_BAD_GRAPH, TP_ERR_WORKSPAC
 TP_MODE_UVU, TP_MODE_UVW = 0, 1
 TP_FLAG_CHECK_INDICES = 1
 TP_OP_FWD, TP_OP_BWD, TP_OP_DBWD = 0, 1, 2
+TP_LINEAR_TENSOR_CORES, TP_LINEAR_CUDA_CORES = 1, 2
 
 _p = C.c_void_p
 _i64 = C.c_int64
@@ -37,7 +38,7 @@ SIGNATURES = {
     "tp_launch_count": (C.c_int64, []),
     "tp_check_bounded_waits": (C.c_int, [_i64, _p, C.POINTER(_i32)]),
     # node-side operators (include/tp_block.h)
-    "tp_linear_create": (C.c_int, [C.POINTER(_p), C.c_char_p, C.c_char_p, _p]),
+    "tp_linear_create": (C.c_int, [C.POINTER(_p), C.c_char_p, C.c_char_p, _p, C.c_uint32]),
     "tp_linear_destroy": (C.c_int, [_p]),
     "tp_linear_query": (C.c_int, [_p, C.POINTER(_i64), C.POINTER(_i64), C.POINTER(_i64), C.POINTER(_i32)]),
     "tp_linear_workspace_size": (C.c_int, [_p, _i64, _i32, C.POINTER(_sz)]),

@@ -17,16 +17,18 @@ __all__ = ["Linear", "Gate", "tp_linear_fwd", "tp_linear_bwd", "tp_linear_worksp
 
 class Linear:
     """Owns a tp_linear_t: y[n, o, w, m] = sum_k c_k sum_u W_k[u, w] x[n, in(k), u, m] over all
-    same-(l, parity) block pairs k = (i_in, i_out), lexicographic."""
+    same-(l, parity) block pairs k = (i_in, i_out), lexicographic.  flags: 0 (form chosen per
+    call by size), TP_LINEAR_TENSOR_CORES or TP_LINEAR_CUDA_CORES."""
 
-    def __init__(self, irreps_in: str, irreps_out: str, coeff: Optional[Sequence[float]] = None):
+    def __init__(self, irreps_in: str, irreps_out: str, coeff: Optional[Sequence[float]] = None, flags: int = 0):
         lib = load()
         self._lib = lib
         self.handle = C.c_void_p()
         self.irreps_in, self.irreps_out = irreps_in, irreps_out
         carr = (C.c_double * len(coeff))(*coeff) if coeff is not None else None
         check(lib.tp_linear_create(C.byref(self.handle), irreps_in.encode(), irreps_out.encode(),
-                                   C.cast(carr, C.c_void_p) if carr is not None else None), "tp_linear_create")
+                                   C.cast(carr, C.c_void_p) if carr is not None else None, int(flags)),
+              "tp_linear_create")
         vals = [C.c_int64() for _ in range(3)]
         n_instr = C.c_int32()
         check(lib.tp_linear_query(self.handle, *[C.byref(v) for v in vals], C.byref(n_instr)), "tp_linear_query")

@@ -32,6 +32,7 @@ constexpr int kLinMaxTypes = 8;     // (l <= 3) x (e, o)
 constexpr int kLinMaxBlocks = 16;
 constexpr int kLinSplits = 64;      // most split-K partials of a gW GEMM
 constexpr int kLinPromote = 16;     // K blocks summed in TMEM before the fp32 promotion
+constexpr int kLinGwChunks = 256;   // most node chunks (partials) of a CUDA-core gW
 
 // ---------------------------------------------------------------------------------------
 // Device side
@@ -113,16 +114,36 @@ __global__ void k_lin_prep(const __grid_constant__ InstrArgs a, const float* __r
   }
 }
 
-// gW[t] = c_k sum_z part[z][base_k + u * ld + w] in split order.
-__global__ void k_lin_reduce(const __grid_constant__ InstrArgs a, const float* __restrict__ part, float* gW) {
-  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < a.total; t += (int64_t)gridDim.x * blockDim.x) {
-    const int k = find_instr(a, t);
-    const int64_t r = t - a.woff[k];
-    const int u = (int)(r / a.mul_out[k]), w = (int)(r - (int64_t)u * a.mul_out[k]);
-    const int64_t idx = a.base[k] + (int64_t)u * a.ld[k] + w;
+// gW[t] = c_k sum_z part[z][base_k + u * ld + w]: a CTA takes 32 consecutive weights (one
+// per lane); warp i of 8 sums the partials z = i, i + 8, ... in order and the 8 warp sums
+// are added in warp order, so the result is deterministic.
+__global__ void __launch_bounds__(256) k_lin_reduce(const __grid_constant__ InstrArgs a, const float* __restrict__ part,
+                                                    float* gW) {
+  __shared__ float red[8][33];
+  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+  for (int64_t t0 = (int64_t)blockIdx.x * 32; t0 < a.total; t0 += (int64_t)gridDim.x * 32) {
+    const int64_t t = t0 + lane;
+    int k = 0, splits = 0;
+    int64_t idx = 0;
+    if (t < a.total) {
+      k = find_instr(a, t);
+      const int64_t r = t - a.woff[k];
+      const int u = (int)(r / a.mul_out[k]), w = (int)(r - (int64_t)u * a.mul_out[k]);
+      idx = a.base[k] + (int64_t)u * a.ld[k] + w;
+      splits = a.splits[k];
+    }
     float s = 0.f;
-    for (int z = 0; z < a.splits[k]; ++z) s += part[(int64_t)z * a.total + idx];
-    gW[t] = a.coeff[k] * s;
+#pragma unroll 4
+    for (int z = wp; z < splits; z += 8) s += __ldg(part + (int64_t)z * a.total + idx);
+    red[wp][lane] = s;
+    __syncthreads();
+    if (wp == 0 && t < a.total) {
+      float r = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) r += red[i][lane];
+      gW[t] = a.coeff[k] * r;
+    }
+    __syncthreads();
   }
 }
 
@@ -300,6 +321,209 @@ __global__ void k_gate(const __grid_constant__ GateArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Linear on the CUDA cores, straight from the node rows: the form for small channel counts,
+// where the map is bound by HBM or by launch latency and the regrouping of the tensor-core
+// form would only add traffic and launches.  One CTA takes a tile of NB consecutive nodes,
+// stages their rows in shared memory and produces every output block of them; each thread
+// computes one (channel, m) output for all NB nodes, so a weight read from L1 serves NB FMAs.
+//   out[n, off_j + c d + m] = sum_{terms t of j} c_t sum_v W[t](v, c) in[n, soff_t + v d + m]
+// with W[t](v, c) = W[woff_t + v * sv + c * sc]: (sv, sc) = (mul_out, 1) in the forward
+// (v = u, c = w) and (1, mul_out) for gx (v = w, c = u).
+// ---------------------------------------------------------------------------------------
+constexpr int kDirectThreads = 256;
+constexpr int kDirectNB = 8;                    // nodes per tile
+constexpr int kDirectSmemFloats = 56 * 1024;    // 224 KB: staged weights + rows
+
+struct DirectArgs {
+  int64_t N;
+  const float* in;
+  int64_t in_stride;
+  float* out;
+  int64_t out_stride;
+  const float* W;
+  int64_t n_weights, w_stage;                  // weights staged in shared memory (0: read from L2)
+  int acc, n_groups, sc_is_ld, vec, vec_w, n_instr, out_cols;
+  int o_off[kLinMaxBlocks], o_d[kLinMaxBlocks], t_begin[kLinMaxBlocks], t_count[kLinMaxBlocks];
+  int s_off[kLinMaxInstr], s_mul[kLinMaxInstr], w_ld[kLinMaxInstr], g_ld[kLinMaxInstr];
+  int i_mul_in[kLinMaxInstr], i_mul_out[kLinMaxInstr];
+  int64_t w_off[kLinMaxInstr];
+  float coeff[kLinMaxInstr];
+  int64_t i_woff[kLinMaxInstr];                // per instruction, in W order (for the staging)
+  float i_coeff[kLinMaxInstr];
+};
+
+// Copies count floats (a multiple of 4 when vec, with 16-byte aligned ends) into shared memory.
+__device__ __forceinline__ void stage(float* dst, const float* src, int64_t count, int vec) {
+  if (vec) {
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll 4
+    for (int64_t t = threadIdx.x; t < (count >> 2); t += blockDim.x) d4[t] = __ldg(s4 + t);
+  } else {
+#pragma unroll 4
+    for (int64_t t = threadIdx.x; t < count; t += blockDim.x) dst[t] = __ldg(src + t);
+  }
+}
+
+template <bool WS>
+__global__ void __launch_bounds__(kDirectThreads) k_lin_direct(const __grid_constant__ DirectArgs a) {
+  extern __shared__ __align__(16) float dsm[];
+  float* wsm = dsm;
+  float* xs = dsm + a.w_stage;
+  if constexpr (WS) {
+    // c_k W_k once per CTA: in the global [u][w] layout for the map, as [w][u] for the
+    // adjoint, so that a warp's consecutive output channels read consecutive words.  Every
+    // W_k spans a multiple of 16 floats (channel counts are multiples of 4), so a float4
+    // never straddles two of them.
+    if (a.vec_w && !a.sc_is_ld) {
+      const float4* w4 = reinterpret_cast<const float4*>(a.W);
+#pragma unroll 4
+      for (int64_t t = threadIdx.x; t < (a.n_weights >> 2); t += blockDim.x) {
+        int k = 0;
+        while (k + 1 < a.n_instr && 4 * t >= a.i_woff[k + 1]) ++k;
+        float4 v = __ldg(w4 + t);
+        const float ck = a.i_coeff[k];
+        v.x *= ck;
+        v.y *= ck;
+        v.z *= ck;
+        v.w *= ck;
+        reinterpret_cast<float4*>(wsm)[t] = v;
+      }
+    } else {
+      for (int64_t t = threadIdx.x; t < a.n_weights; t += blockDim.x) {
+        int k = 0;
+        while (k + 1 < a.n_instr && t >= a.i_woff[k + 1]) ++k;
+        int64_t dst = t;
+        if (a.sc_is_ld) {
+          const int64_t r = t - a.i_woff[k];
+          const int u = (int)(r / a.i_mul_out[k]), w = (int)(r - (int64_t)u * a.i_mul_out[k]);
+          dst = a.i_woff[k] + (int64_t)w * a.i_mul_in[k] + u;
+        }
+        wsm[dst] = a.i_coeff[k] * __ldg(a.W + t);
+      }
+    }
+  }
+  for (int64_t n0 = (int64_t)blockIdx.x * kDirectNB; n0 < a.N; n0 += (int64_t)gridDim.x * kDirectNB) {
+    const int nb_here = (int)min((int64_t)kDirectNB, a.N - n0);
+    __syncthreads();
+    stage(xs, a.in + n0 * a.in_stride, (int64_t)nb_here * a.in_stride, a.vec);
+    __syncthreads();
+    // all output blocks of the row in one pass: thread t takes row positions t, t + 256, ...
+    for (int t = threadIdx.x; t < a.out_cols; t += blockDim.x) {
+      int j = 0;
+      while (j + 1 < a.n_groups && t >= a.o_off[j + 1]) ++j;
+      const int d = a.o_d[j];
+      const int r = t - a.o_off[j];
+      const int c = r / d, m = r - c * d;
+      if (a.acc && a.t_count[j] == 0) continue;      // accumulate leaves blocks without terms
+      float acc[kDirectNB];
+#pragma unroll
+      for (int q = 0; q < kDirectNB; ++q) acc[q] = 0.f;
+      for (int k = a.t_begin[j]; k < a.t_begin[j] + a.t_count[j]; ++k) {
+        // staged: element (v, c) at w_off + v * ld + c for both the map and the adjoint
+        const int ld = a.w_ld[k];
+        const int64_t sv = (WS || !a.sc_is_ld) ? ld : 1, sc = (WS || !a.sc_is_ld) ? 1 : a.g_ld[k];
+        const float ck = WS ? 1.f : a.coeff[k];
+        const float* wp = (WS ? wsm : a.W) + a.w_off[k] + c * sc;
+        const float* xp = xs + a.s_off[k] + m;
+        for (int v = 0; v < a.s_mul[k]; v += 4) {      // channel counts are multiples of 4
+          float wv[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) wv[i] = ck * (WS ? wp[(v + i) * sv] : __ldg(wp + (v + i) * sv));
+#pragma unroll
+          for (int q = 0; q < kDirectNB; ++q) {        // rows past nb_here hold stale data, never stored
+            const float* xq = xp + q * a.in_stride + v * d;
+            acc[q] = fmaf(wv[0], xq[0], acc[q]);
+            acc[q] = fmaf(wv[1], xq[d], acc[q]);
+            acc[q] = fmaf(wv[2], xq[2 * d], acc[q]);
+            acc[q] = fmaf(wv[3], xq[3 * d], acc[q]);
+          }
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < kDirectNB; ++q)
+        if (q < nb_here) {
+          float* o = a.out + (n0 + q) * a.out_stride + t;
+          *o = a.acc ? *o + acc[q] : acc[q];
+        }
+    }
+  }
+}
+
+// Per-CTA partial weight gradients on the CUDA cores: CTA (z, r) sums over the nodes of
+// chunk z; each thread owns one 4 x 4 tile (u0..u0+3, w0..w0+3) of one W_k (channel counts
+// are multiples of 4) and adds the outer products of x[n, in(k), u, m] and gy[n, out(k), w, m]
+// over the chunk's (n, m): 8 shared-memory loads per 16 FMAs.
+//   part[z][woff_k + u mul_out + w] = sum_{n in chunk z, m} x[n, in(k), u, m] gy[n, out(k), w, m]
+// (coefficients are applied by the reduction, k_lin_reduce).
+struct DirectGwArgs {
+  int64_t N, chunk;
+  const float* x;
+  const float* gy;
+  int64_t x_stride, gy_stride;
+  float* part;
+  int64_t n_weights;
+  int n_instr, vec, n_tiles;
+  int tile0[kLinMaxInstr + 1];      // first 4 x 4 tile of each instruction; tile0[n_instr] = n_tiles
+  int64_t woff[kLinMaxInstr];
+  int xoff[kLinMaxInstr], goff[kLinMaxInstr], mul_out[kLinMaxInstr], d[kLinMaxInstr];
+};
+
+__global__ void __launch_bounds__(kDirectThreads) k_lin_direct_gw(const __grid_constant__ DirectGwArgs a) {
+  extern __shared__ __align__(16) float gsm[];
+  float* xs = gsm;
+  float* gs = gsm + kDirectNB * a.x_stride;
+  const int64_t nb0 = (int64_t)blockIdx.x * a.chunk, nb1 = min(a.N, nb0 + a.chunk);
+  const int T = blockIdx.y * kDirectThreads + threadIdx.x;
+  const bool own = T < a.n_tiles;
+  int k = 0, xo = 0, go = 0, d = 0, u0 = 0, w0 = 0;
+  if (own) {
+    while (k + 1 < a.n_instr && T >= a.tile0[k + 1]) ++k;
+    const int tw_n = a.mul_out[k] / 4, r = T - a.tile0[k];
+    u0 = 4 * (r / tw_n);
+    w0 = 4 * (r - (r / tw_n) * tw_n);
+    d = a.d[k];
+    xo = a.xoff[k] + u0 * d;
+    go = a.goff[k] + w0 * d;
+  }
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int64_t n0 = nb0; n0 < nb1; n0 += kDirectNB) {
+    const int nb_here = (int)min((int64_t)kDirectNB, nb1 - n0);
+    __syncthreads();
+    stage(xs, a.x + n0 * a.x_stride, (int64_t)nb_here * a.x_stride, a.vec);
+    stage(gs, a.gy + n0 * a.gy_stride, (int64_t)nb_here * a.gy_stride, a.vec);
+    __syncthreads();
+    for (int q = 0; q < nb_here; ++q) {
+      const float* xq = xs + q * a.x_stride + xo;
+      const float* gq = gs + q * a.gy_stride + go;
+      for (int m = 0; m < d; ++m) {
+        float xv[4], gv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          xv[i] = xq[i * d + m];
+          gv[i] = gq[i * d + m];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xv[i], gv[j], acc[i][j]);
+      }
+    }
+  }
+  if (own) {
+    float* dst = a.part + (int64_t)blockIdx.x * a.n_weights + a.woff[k] + w0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4*>(dst + (int64_t)(u0 + i) * a.mul_out[k]) =
+          make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+  }
+}
+
 size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
@@ -344,6 +568,7 @@ struct tp_linear_s {
   int64_t wt_base[kLinMaxBlocks];   // per output block: its rows of Wt
   int64_t wg_base[kLinMaxBlocks];   // per input block: its rows of Wg
   int type_of_in[kLinMaxBlocks], type_of_out[kLinMaxBlocks];
+  uint32_t flags = 0;
 };
 
 namespace {
@@ -362,13 +587,13 @@ LinWs lin_ws(const tp_linear_s* L, int64_t N, bool bwd) {
   w.wsplit = off;
   off += al256(sizeof(float) * 2 * (size_t)std::max<int64_t>(1, L->n_weights));
   w.part = off;
-  if (bwd) off += al256(sizeof(float) * (size_t)kLinSplits * (size_t)std::max<int64_t>(1, L->n_weights));
+  if (bwd) off += al256(sizeof(float) * (size_t)std::max(kLinSplits, kLinGwChunks) * (size_t)std::max<int64_t>(1, L->n_weights));
   w.total = off;
   return w;
 }
 
 int lin_splits(int64_t rows) {
-  const int64_t per = (int64_t)TC_BK * kLinPromote;
+  const int64_t per = (int64_t)TC_BK * 4;   // short splits: many CTAs, little serial latency
   return (int)std::max<int64_t>(1, std::min<int64_t>(kLinSplits, (rows + per - 1) / per));
 }
 
@@ -470,13 +695,143 @@ cudaError_t launch_prep(const tp_linear_s* L, const float* W, float* dst, int tr
   return cudaGetLastError();
 }
 
+// The tensor-core form pays a regrouping pass and several launches; it wins when the
+// channel counts make the map compute heavy and the node count fills the GPU.
+bool use_tensor_cores(const tp_linear_s* L, int64_t N) {
+  if (L->flags & TP_LINEAR_TENSOR_CORES) return true;
+  if (L->flags & TP_LINEAR_CUDA_CORES) return false;
+  if ((int64_t)kDirectNB * (L->in_dim + L->out_dim) > kDirectSmemFloats) return true;   // rows too wide to stage
+  if (N < 4096 || L->n_types == 0) return false;
+  for (int q = 0; q < L->n_types; ++q)
+    if (std::min(L->types[q].K, L->types[q].Nn) < 64) return false;
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaError_t set_smem(const void* fn, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  if (bytes > 227 * 1024) return cudaErrorInvalidValue;
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+// out rows = the map (forward: in = x) or its adjoint (gx: in = gy) on the CUDA cores.
+cudaError_t launch_direct(const tp_linear_s* L, int64_t N, const float* in, const float* W, float* out, int acc,
+                          bool adjoint, cudaStream_t s) {
+  DirectArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.N = N;
+  a.in = in;
+  a.in_stride = adjoint ? L->out_dim : L->in_dim;
+  a.out = out;
+  a.out_stride = adjoint ? L->in_dim : L->out_dim;
+  a.W = W;
+  a.acc = acc;
+  a.sc_is_ld = adjoint ? 1 : 0;
+  const auto& dst = adjoint ? L->in : L->out;
+  const auto& dst_off = adjoint ? L->in_off : L->out_off;
+  int nt = 0;
+  for (int j = 0; j < (int)dst.size(); ++j) {
+    a.o_off[j] = (int)dst_off[j];
+    a.o_d[j] = 2 * dst[j].l + 1;
+    a.t_begin[j] = nt;
+    for (int k = 0; k < L->n_instr; ++k) {
+      if ((adjoint ? L->ins_in[k] : L->ins_out[k]) != j) continue;
+      const int src_blk = adjoint ? L->ins_out[k] : L->ins_in[k];
+      a.s_off[nt] = (int)(adjoint ? L->out_off[src_blk] : L->in_off[src_blk]);
+      a.s_mul[nt] = adjoint ? L->out[src_blk].mul : L->in[src_blk].mul;
+      a.w_off[nt] = L->ins_woff[k];
+      // row length of the staged layout ([u][w] for the map, [w][u] for the adjoint) and of
+      // the global one ([u][w])
+      a.w_ld[nt] = adjoint ? L->in[L->ins_in[k]].mul : L->out[L->ins_out[k]].mul;
+      a.g_ld[nt] = L->out[L->ins_out[k]].mul;
+      a.coeff[nt] = L->coeff[k];
+      ++nt;
+    }
+    a.t_count[j] = nt - a.t_begin[j];
+  }
+  a.n_groups = (int)dst.size();
+  a.out_cols = (int)a.out_stride;
+  a.n_instr = L->n_instr;
+  for (int k = 0; k < L->n_instr; ++k) {
+    a.i_woff[k] = L->ins_woff[k];
+    a.i_coeff[k] = L->coeff[k];
+    a.i_mul_in[k] = L->in[L->ins_in[k]].mul;
+    a.i_mul_out[k] = L->out[L->ins_out[k]].mul;
+  }
+  a.n_weights = L->n_weights;
+  a.vec = aligned16(in) && a.in_stride % 4 == 0;
+  a.vec_w = aligned16(W) && L->n_weights % 4 == 0;
+  const int64_t rows = (int64_t)kDirectNB * a.in_stride;
+  if (rows > kDirectSmemFloats) return cudaErrorInvalidValue;
+  const bool ws = L->n_weights + rows + 4 <= kDirectSmemFloats;
+  a.w_stage = ws ? (L->n_weights + 3) / 4 * 4 : 0;
+  const size_t smem = sizeof(float) * (size_t)(a.w_stage + rows);
+  const void* fn = ws ? reinterpret_cast<const void*>(k_lin_direct<true>) : reinterpret_cast<const void*>(k_lin_direct<false>);
+  cudaError_t e = set_smem(fn, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = (N + kDirectNB - 1) / kDirectNB;
+  const unsigned grid = (unsigned)std::min<int64_t>(tiles, (int64_t)sm_count() * 4);
+  if (ws) k_lin_direct<true><<<grid, kDirectThreads, smem, s>>>(a);
+  else k_lin_direct<false><<<grid, kDirectThreads, smem, s>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+// gW on the CUDA cores: per-CTA partials over node chunks, then the fixed-order reduction.
+cudaError_t launch_direct_gw(const tp_linear_s* L, int64_t N, const float* x, const float* gy, float* part,
+                             float* gW, cudaStream_t s) {
+  DirectGwArgs a;
+  std::memset(&a, 0, sizeof(a));
+  const int64_t Z = std::max<int64_t>(1, std::min<int64_t>(kLinGwChunks, (N + kDirectNB - 1) / kDirectNB));
+  a.N = N;
+  a.chunk = (N + Z - 1) / Z;
+  a.x = x;
+  a.gy = gy;
+  a.x_stride = L->in_dim;
+  a.gy_stride = L->out_dim;
+  a.part = part;
+  a.n_weights = L->n_weights;
+  a.n_instr = L->n_instr;
+  a.vec = aligned16(x) && aligned16(gy) && L->in_dim % 4 == 0 && L->out_dim % 4 == 0;
+  if ((int64_t)kDirectNB * (L->in_dim + L->out_dim) > kDirectSmemFloats) return cudaErrorInvalidValue;
+  for (int k = 0; k < L->n_instr; ++k) {
+    a.tile0[k] = a.n_tiles;
+    a.n_tiles += (L->in[L->ins_in[k]].mul / 4) * (L->out[L->ins_out[k]].mul / 4);
+    a.woff[k] = L->ins_woff[k];
+    a.xoff[k] = (int)L->in_off[L->ins_in[k]];
+    a.goff[k] = (int)L->out_off[L->ins_out[k]];
+    a.mul_out[k] = L->out[L->ins_out[k]].mul;
+    a.d[k] = 2 * L->in[L->ins_in[k]].l + 1;
+  }
+  const size_t smem = sizeof(float) * (size_t)kDirectNB * (size_t)(L->in_dim + L->out_dim);
+  cudaError_t e = set_smem(reinterpret_cast<const void*>(k_lin_direct_gw), smem);
+  if (e != cudaSuccess) return e;
+  a.tile0[L->n_instr] = a.n_tiles;
+  const int64_t tranges = (a.n_tiles + kDirectThreads - 1) / kDirectThreads;
+  k_lin_direct_gw<<<dim3((unsigned)Z, (unsigned)tranges), kDirectThreads, smem, s>>>(a);
+  count_launches(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  InstrArgs r = instr_args(L);
+  for (int k = 0; k < L->n_instr; ++k) {
+    r.base[k] = L->ins_woff[k];
+    r.ld[k] = L->out[L->ins_out[k]].mul;
+    r.splits[k] = (int)Z;
+  }
+  k_lin_reduce<<<grid_for(L->n_weights, 32), 256, 0, s>>>(r, part, gW);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 extern "C" {
 
-tp_status_t tp_linear_create(tp_linear_t* lin, const char* irreps_in, const char* irreps_out, const double* coeff) {
+tp_status_t tp_linear_create(tp_linear_t* lin, const char* irreps_in, const char* irreps_out, const double* coeff,
+                             uint32_t flags) {
   if (!lin) return fail(TP_ERR_INVALID_ARG, "lin is NULL");
   *lin = nullptr;
+  if ((flags & ~3u) || flags == 3u) return fail(TP_ERR_INVALID_ARG, "flags: TP_LINEAR_TENSOR_CORES or TP_LINEAR_CUDA_CORES");
   std::vector<IrrepTerm> in, out;
   std::string why;
   if (!parse_irreps_terms(irreps_in, in, why)) return fail(TP_ERR_INVALID_ARG, "irreps_in: " + why);
@@ -492,6 +847,7 @@ tp_status_t tp_linear_create(tp_linear_t* lin, const char* irreps_in, const char
   if (!L) return fail(TP_ERR_INVALID_ARG, "out of host memory");
   L->in = in;
   L->out = out;
+  L->flags = flags;
   for (const IrrepTerm& t : in) {
     L->in_off.push_back(L->in_dim);
     L->in_dim += (int64_t)t.mul * (2 * t.l + 1);
@@ -610,6 +966,10 @@ tp_status_t tp_linear_fwd(tp_linear_t lin, int64_t N, const float* x, const floa
   if (!x || !y || (lin->n_weights && !W)) return fail(TP_ERR_INVALID_ARG, "x, W and y must not be NULL");
   if (!aligned4(x) || !aligned4(y) || !aligned4(W)) return fail(TP_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!use_tensor_cores(lin, N)) {
+    cudaError_t e = launch_direct(lin, N, x, W, y, accumulate ? 1 : 0, false, s);
+    return e == cudaSuccess ? TP_OK : cuda_failed(e, "linear (CUDA cores)");
+  }
   const LinWs L = lin_ws(lin, N, false);
   char* base = static_cast<char*>(ws);
   float* XA = reinterpret_cast<float*>(base + L.xa);
@@ -662,6 +1022,13 @@ tp_status_t tp_linear_bwd(tp_linear_t lin, int64_t N, const float* x, const floa
   if (!gx && !gW) return TP_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const LinWs L = lin_ws(lin, N, true);
+  if (!use_tensor_cores(lin, N)) {
+    cudaError_t e = cudaSuccess;
+    if (gx) e = launch_direct(lin, N, gy, W, gx, 0, true, s);
+    if (e == cudaSuccess && gW && lin->n_weights)
+      e = launch_direct_gw(lin, N, x, gy, reinterpret_cast<float*>(static_cast<char*>(ws) + L.part), gW, s);
+    return e == cudaSuccess ? TP_OK : cuda_failed(e, "linear backward (CUDA cores)");
+  }
   char* base = static_cast<char*>(ws);
   float* XA = reinterpret_cast<float*>(base + L.xa);
   float* GA = reinterpret_cast<float*>(base + L.ga);
@@ -724,7 +1091,7 @@ tp_status_t tp_linear_bwd(tp_linear_t lin, int64_t N, const float* x, const floa
           r.splits[k] = op.splits;
         }
     }
-    k_lin_reduce<<<grid_for(lin->n_weights, 256), 256, 0, s>>>(r, part, gW);
+    k_lin_reduce<<<grid_for(lin->n_weights, 32), 256, 0, s>>>(r, part, gW);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_failed(e, "linear gW reduction");
   }

@@ -19,10 +19,11 @@
  *
  *   y[n, o, w, m] = sum_{k: out(k) = o} c_k sum_u W_k[u, w] x[n, in(k), u, m]
  *
- * Output blocks that no instruction reaches are zero.  The map runs on the tcgen05 tensor
- * cores in 3xTF32 (fp32-accurate, see tp.h) as one GEMM per output block over the
- * concatenated input channels of its irrep; the inputs are first regrouped into
- * [(node, m)][channel] rows in the workspace.  Backward: gx = the adjoint map applied to gy,
+ * Output blocks that no instruction reaches are zero.  Wide maps on many nodes run on the
+ * tcgen05 tensor cores in 3xTF32 (fp32-accurate, see tp.h) as one GEMM per output block over
+ * the concatenated input channels of its irrep, after the inputs are regrouped into
+ * [(node, m)][channel] rows in the workspace; narrow maps run on the CUDA cores straight from
+ * the node rows (see tp_linear_create).  Backward: gx = the adjoint map applied to gy,
  * gW_k[u, w] = c_k sum_{n, m} x[n, in(k), u, m] gy[n, out(k), w, m] (split-K GEMM, fixed
  * split order: deterministic).  Second order needs no entry point of its own: with
  * cotangents (ggx, ggW) of (gx, gW),
@@ -55,10 +56,17 @@ extern "C" {
 typedef struct tp_linear_s* tp_linear_t;
 typedef struct tp_gate_s* tp_gate_t;
 
+enum { TP_LINEAR_TENSOR_CORES = 1, TP_LINEAR_CUDA_CORES = 2 };
+
 /* Builds a linear map.  irreps strings as in tp.h ("32x0e+32x1o"); l <= 3; every
  * multiplicity a multiple of 4 (TMA row pitch), else TP_ERR_UNSUPPORTED.  coeff: one double
- * per instruction, or NULL for 1.0.  At most 64 instructions and 16 blocks per string. */
-tp_status_t tp_linear_create(tp_linear_t* lin, const char* irreps_in, const char* irreps_out, const double* coeff);
+ * per instruction, or NULL for 1.0.  At most 64 instructions and 16 blocks per string.
+ * flags: 0 picks the form per call -- the tcgen05 GEMMs when N >= 4096 and every irrep has
+ * at least 64 input and 64 output channels, otherwise the CUDA-core form, which reads the
+ * node rows in place (one launch for y or gx, two for gW); TP_LINEAR_TENSOR_CORES or
+ * TP_LINEAR_CUDA_CORES forces one.  Both give the same sums to fp32 rounding. */
+tp_status_t tp_linear_create(tp_linear_t* lin, const char* irreps_in, const char* irreps_out, const double* coeff,
+                             uint32_t flags);
 tp_status_t tp_linear_destroy(tp_linear_t lin);
 
 /* Feature widths, weight count (sum of mul_in * mul_out over instructions), instructions. */
@@ -66,7 +74,8 @@ tp_status_t tp_linear_query(tp_linear_t lin, int64_t* in_dim, int64_t* out_dim, 
                             int32_t* n_instructions);
 
 /* Device workspace bytes for N nodes: op TP_OP_FWD (regrouped inputs + split weights) or
- * TP_OP_BWD (regrouped inputs and output gradients, split weights, split-K partials). */
+ * TP_OP_BWD (regrouped inputs and output gradients, split weights, split-K partials), enough
+ * for either form; 256-byte aligned (any torch allocation is). */
 tp_status_t tp_linear_workspace_size(tp_linear_t lin, int64_t N, int32_t op, size_t* bytes);
 
 /* y[N, out_dim] = linear(x[N, in_dim]; W[n_weights]); accumulate = 1 adds into y instead of

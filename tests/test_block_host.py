@@ -37,7 +37,7 @@ def test_linear_sizes_match_the_oracle(tp, ir_in, ir_out):
     fwd = tp.tp_linear_workspace_size(lin, N, tp.TP_OP_FWD)
     bwd = tp.tp_linear_workspace_size(lin, N, tp.TP_OP_BWD)
     assert fwd <= 4 * N * lin.in_dim + 8 * lin.n_weights + 4096
-    assert bwd <= 4 * N * (lin.in_dim + lin.out_dim) + (8 + 4 * 64) * lin.n_weights + 4096
+    assert bwd <= 4 * N * (lin.in_dim + lin.out_dim) + (8 + 4 * 256) * lin.n_weights + 4096
 
 
 @pytest.mark.parametrize("ir_in,ir_out,status", [
@@ -52,9 +52,12 @@ def test_linear_validation(tp, ir_in, ir_out, status):
     assert e.value.status == status
 
 
-def test_linear_rejects_nonfinite_coefficients(tp):
+def test_linear_rejects_nonfinite_coefficients_and_bad_flags(tp):
     with pytest.raises(tp.TPError):
         tp.Linear("4x0e", "4x0e", coeff=[float("nan")])
+    for flags in (3, 4):
+        with pytest.raises(tp.TPError):
+            tp.Linear("4x0e", "4x0e", flags=flags)
 
 
 @pytest.mark.parametrize("args,status", [
@@ -115,5 +118,6 @@ def test_no_cpu_fallback_without_device(tp):
     g = tp.Gate("4x0e", "4x0e", "4x1o")
     fake = C.c_void_p(0x10000)
     assert lib.tp_gate_fwd(g.handle, 4, fake, fake, None) == 5
-    lin = tp.Linear("32x0e", "32x0e")
-    assert lib.tp_linear_fwd(lin.handle, 4, fake, fake, fake, 0, fake, 1 << 24, None) == 5
+    for form in (tp.TP_LINEAR_TENSOR_CORES, tp.TP_LINEAR_CUDA_CORES):
+        lin = tp.Linear("32x0e", "32x0e", flags=form)
+        assert lib.tp_linear_fwd(lin.handle, 4, fake, fake, fake, 0, fake, 1 << 24, None) == 5

@@ -40,12 +40,16 @@ LINEARS = [
 ]
 
 
+FORMS = [0, 1, 2]     # chosen by size, tcgen05 GEMMs, CUDA cores
+
+
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("ir_in,ir_out,N", LINEARS)
-def test_linear_forward_and_backward(tp, ir_in, ir_out, N):
+def test_linear_forward_and_backward(tp, ir_in, ir_out, N, form):
     rng = np.random.default_rng(N)
     n_ins = len(linear_instructions(ir_in, ir_out))
     coeff = rng.uniform(0.5, 1.5, n_ins)
-    lin = tp.Linear(ir_in, ir_out, coeff=list(coeff))
+    lin = tp.Linear(ir_in, ir_out, coeff=list(coeff), flags=form)
     x = rng.standard_normal((N, Irreps(ir_in).dim)).astype(np.float32)
     W = rng.standard_normal(linear_weight_count(ir_in, ir_out)).astype(np.float32)
     gy = rng.standard_normal((N, Irreps(ir_out).dim)).astype(np.float32)
@@ -62,10 +66,11 @@ def test_linear_forward_and_backward(tp, ir_in, ir_out, N):
     assert torch.equal(gW2, gW)
 
 
-def test_linear_accumulate_and_empty(tp):
+@pytest.mark.parametrize("form", [1, 2])
+def test_linear_accumulate_and_empty(tp, form):
     ir_in, ir_out = "32x0e+32x1e+32x1o+32x2e+32x2o", "32x0e+64x0e+32x1o+32x2e+32x3o"
     rng = np.random.default_rng(5)
-    lin = tp.Linear(ir_in, ir_out)
+    lin = tp.Linear(ir_in, ir_out, flags=form)
     N = 200
     x = rng.standard_normal((N, lin.in_dim)).astype(np.float32)
     W = rng.standard_normal(lin.n_weights).astype(np.float32)
@@ -86,10 +91,11 @@ def test_linear_accumulate_and_empty(tp):
     assert gx.shape == (0, lin.in_dim) and bool((gW == 0).all())
 
 
-def test_linear_second_order_through_autograd(tp):
+@pytest.mark.parametrize("form", [1, 2])
+def test_linear_second_order_through_autograd(tp, form):
     ir_in, ir_out = "32x0e+32x1o+32x2e+32x1e", "64x0e+32x1o+32x2e+32x2o"
     rng = np.random.default_rng(6)
-    lin = tp.Linear(ir_in, ir_out)
+    lin = tp.Linear(ir_in, ir_out, flags=form)
     N = 333
     x = rng.standard_normal((N, lin.in_dim)).astype(np.float32)
     W = rng.standard_normal(lin.n_weights).astype(np.float32)
