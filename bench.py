@@ -42,7 +42,7 @@ WORKLOADS = {
     "c4": "large streaming uvw: 100,000 atoms, ~3.0M edges, 128x(0e,1o,2e) -> 128x(0e,1e,1o,2e,2o), SH lmax 2, "
           "per-path 128x128 mixing, 15 paths; step = fwd + transpose + bwd(gx, gs, gW)",
     "c2-layer": "interaction layer on the c2 graph (1,536 atoms, 46,080 edges): linear 32x(0e,1o,2e) -> same, "
-                "convolution (c2 paths, coefficient 1/average degree), linear -> 32x0e+64x0e+32x1o+32x2e, gate "
+                "convolution (c2 paths), linear with coefficient 1/average degree -> 32x0e+64x0e+32x1o+32x2e, gate "
                 "-> 32x(0e,1o,2e); step = that forward + transpose + the backward to x, both linear weights and "
                 "the edge weights",
 }
@@ -689,11 +689,11 @@ def oracle_layer_sample(d, n_rows, seed, W1, W2, g_out):
     return 1.0 / (tf / ef + tb / eb + node_t / E), ef, eb, tf + tb + node_t
 
 
-def layer_weights(spec, N, rank=0):
+def layer_weights(spec, N, n_w1, n_w2, rank=0):
+    """Seeded weights of the two linear maps (N(0, 1/32): fan-in 32) and the upstream gradient."""
     rng = np.random.default_rng(spec.seed + 17 + 7919 * rank)
-    from oracle.block import linear_weight_count
-    W1 = (rng.standard_normal(linear_weight_count(spec.irreps_in, spec.irreps_in)) / math.sqrt(32)).astype(np.float32)
-    W2 = (rng.standard_normal(linear_weight_count(spec.irreps_out, LAYER_MID)) / math.sqrt(32)).astype(np.float32)
+    W1 = (rng.standard_normal(n_w1) / math.sqrt(32)).astype(np.float32)
+    W2 = (rng.standard_normal(n_w2) / math.sqrt(32)).astype(np.float32)
     g_out = rng.standard_normal((N, 288), dtype=np.float32)
     return W1, W2, g_out
 
@@ -703,7 +703,9 @@ def run_reference_layer(args, cores):
     spec = synth.CONFIGS["c2"]
     d = synth.make_inputs("c2")
     N = len(d["rowptr"]) - 1
-    W1, W2, g_out = layer_weights(spec, N)
+    from oracle.block import linear_weight_count
+    W1, W2, g_out = layer_weights(spec, N, linear_weight_count(spec.irreps_in, spec.irreps_in),
+                                  linear_weight_count(spec.irreps_out, LAYER_MID))
     oracle_sample(d, 4, seed=0)
     v, ef, eb, t = oracle_layer_sample(d, 16, 1, W1, W2, g_out)
     rows = int(max(2, min(256, 16 * 60.0 / max(1, args.steps + args.warmup) / t)))
@@ -749,11 +751,15 @@ def run_layer(args, rank, world, local):
     if args.order == "cell":
         d = synth.cell_sorted(d)
     N, E = len(d["rowptr"]) - 1, len(d["src"])
-    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvu",
-                   path_coeff=[N / max(E, 1)] * len(spec.paths))
-    lin1, lin2 = tp.Linear(spec.irreps_in, spec.irreps_in), tp.Linear(spec.irreps_out, LAYER_MID)
+    # the 1/average-degree scale of the aggregated messages rides on the next linear map's
+    # coefficients (it commutes with the map), which keeps the convolution on its
+    # unit-coefficient compiled instances
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvu")
+    n2 = tp.Linear(spec.irreps_out, LAYER_MID).n_instructions
+    lin1 = tp.Linear(spec.irreps_in, spec.irreps_in)
+    lin2 = tp.Linear(spec.irreps_out, LAYER_MID, coeff=[N / max(E, 1)] * n2)
     gate = tp.Gate(*LAYER_GATE)
-    W1, W2, d["g_out"] = layer_weights(spec, N, rank)
+    W1, W2, d["g_out"] = layer_weights(spec, N, lin1.n_weights, lin2.n_weights, rank)
     in_dim, out_dim, nw = plan.in_dim, plan.out_dim, plan.n_edge_weights
 
     keys = ["rowptr", "src", "x", "vec", "w", "g_out"]

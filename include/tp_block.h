@@ -3,7 +3,9 @@
  * sit around the tensor-product convolution of tp.h: the irreps-wise linear map
  * (self-interaction before the convolution, mixing of its path-concatenated outputs after
  * it) and the gate nonlinearity.  The 1/(average degree) scale of the aggregated messages
- * is the convolution plan's path coefficient (tp_plan_create, path_coeff).
+ * is either the convolution plan's path coefficient (tp_plan_create, path_coeff) or, since
+ * it commutes with the linear map, that map's instruction coefficients -- the cheaper form:
+ * the convolution's compiled fast instances take unit path coefficients.
  *
  * The pages name these layers without defining them ("Accelerating Tensor Products in
  * E(3)-Equivariant Graph Neural Networks", abstract: NequIP's equivariant interaction layers,
