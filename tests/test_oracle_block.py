@@ -217,3 +217,95 @@ def test_gate_double_backward_gradgradcheck():
     xd = x.detach().numpy()
     jv = (gate(s, xd + h * ggx).numpy() - gate(s, xd - h * ggx).numpy()) / (2 * h)
     np.testing.assert_allclose(r["g_gy"].numpy(), jv, rtol=1e-6, atol=1e-8)
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def _permute_blocks(irreps: str, x, to_mu: bool):
+    """[u][m] <-> [m][u] inside every block of a feature row."""
+    ir = Irreps(irreps)
+    out = x.clone()
+    for (mul, l, _), off in zip(ir.blocks, ir.offsets):
+        d = 2 * l + 1
+        blk = x[:, off:off + mul * d]
+        out[:, off:off + mul * d] = (blk.reshape(-1, mul, d).transpose(1, 2) if to_mu
+                                     else blk.reshape(-1, d, mul).transpose(1, 2)).reshape(-1, mul * d)
+    return out
+
+
+@pytest.mark.parametrize("mutation", ["w_transposed", "m_u_swapped", "dropped_instruction", "coeff_ignored"])
+def test_planted_linear_mistakes_are_caught(mutation, monkeypatch):
+    """Plant a plausible mistake in the oracle's linear map (CPU only); a pin must fail."""
+    import oracle.block as ob
+    good = ob._linear_t
+
+    def bad(ir_in, ir_out, x, W, coeff):
+        ins = linear_instructions(ir_in, ir_out)
+        a, b = Irreps(ir_in), Irreps(ir_out)
+        if mutation == "w_transposed":          # W_k read as [mul_out][mul_in]
+            parts, off = [], 0
+            for i, o in ins:
+                mi, mo = a.blocks[i][0], b.blocks[o][0]
+                parts.append(W[off:off + mi * mo].reshape(mo, mi).T.reshape(-1))
+                off += mi * mo
+            return good(ir_in, ir_out, x, torch.cat(parts), coeff)
+        if mutation == "m_u_swapped":           # blocks read as [m][u]
+            return good(ir_in, ir_out, _permute_blocks(ir_in, x, True), W, coeff)
+        if mutation == "dropped_instruction":   # the last instruction left out
+            mi, mo = a.blocks[ins[-1][0]][0], b.blocks[ins[-1][1]][0]
+            W2 = W.clone()
+            W2[len(W) - mi * mo:] = 0
+            return good(ir_in, ir_out, x, W2, coeff)
+        return good(ir_in, ir_out, x, W, None)   # coefficients ignored
+
+    monkeypatch.setattr(ob, "_linear_t", bad)
+    pins = [test_scalar_linear_is_a_matrix_product, test_inputs_of_one_irrep_sum_into_the_output_with_their_coefficients,
+            test_vector_block_mixes_channels_and_keeps_m,
+            lambda: test_linear_commutes_with_rotations_and_inversion(False)]
+    caught = 0
+    for pin in pins:
+        try:
+            pin()
+        except AssertionError:
+            caught += 1
+    assert caught, mutation
+
+
+@pytest.mark.parametrize("mutation", ["sigmoid_on_scalars", "tanh_on_even", "gate_shifted", "gate_unsquashed"])
+def test_planted_gate_mistakes_are_caught(mutation, monkeypatch):
+    """Plant a plausible mistake in the oracle's gate (CPU only); a pin must fail."""
+    import oracle.block as ob
+
+    def bad(spec, x):
+        N = x.shape[0]
+        cols, off = [], 0
+        for m, _, p in spec.scalar_blocks:
+            s = x[:, off:off + m]
+            if mutation == "sigmoid_on_scalars":
+                cols.append(torch.sigmoid(s))
+            elif mutation == "tanh_on_even":
+                cols.append(torch.tanh(s))
+            else:
+                cols.append(torch.nn.functional.silu(s) if p == 1 else torch.tanh(s))
+            off += m
+        g = x[:, off:off + spec.n_gate]
+        if mutation == "gate_shifted":
+            g = torch.roll(g, 1, dims=1)
+        gates = g if mutation == "gate_unsquashed" else torch.sigmoid(g)
+        off += spec.n_gate
+        c = 0
+        for m, l, _ in spec.gated_blocks:
+            d = 2 * l + 1
+            v = x[:, off:off + m * d].reshape(N, m, d)
+            cols.append((v * gates[:, c:c + m, None]).reshape(N, m * d))
+            off += m * d
+            c += m
+        return torch.cat(cols, dim=1)
+
+    monkeypatch.setattr(ob, "_gate_t", bad)
+    caught = False
+    try:
+        test_gate_matches_the_logistic_function()
+    except AssertionError:
+        caught = True
+    assert caught, mutation
