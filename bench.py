@@ -45,9 +45,16 @@ WORKLOADS = {
                 "convolution (c2 paths), linear with coefficient 1/average degree -> 32x0e+64x0e+32x1o+32x2e, gate "
                 "-> 32x(0e,1o,2e); step = that forward + transpose + the backward to x, both linear weights and "
                 "the edge weights",
+    "c4-layer": "interaction layer on the c4 graph (100,000 atoms, ~3.0M edges): linear 128x(0e,1o,2e) -> same, uvw "
+                "convolution (c4 paths, 128x128 mixing), linear with coefficient 1/average degree -> "
+                "128x0e+256x0e+128x1o+128x2e, gate -> 128x(0e,1o,2e); step = that forward + transpose + the backward "
+                "to x, both linear weights, the edge scalars and the mixing weights",
 }
-LAYER_MID = "32x0e+64x0e+32x1o+32x2e"
-LAYER_GATE = ("32x0e", "64x0e", "32x1o+32x2e")
+
+
+def layer_shapes(mul):
+    """Gate input of the layer (scalars, gates for the two gated blocks, gated) and the gate's split."""
+    return (f"{mul}x0e+{2 * mul}x0e+{mul}x1o+{mul}x2e", (f"{mul}x0e", f"{2 * mul}x0e", f"{mul}x1o+{mul}x2e"))
 
 
 def parse():
@@ -218,10 +225,13 @@ def oracle_sample(d, n_rows, seed):
     mask = np.isin(d["src"], rows)
     eb = np.nonzero(mask)[0]
     rpb = np.concatenate([[0], np.cumsum(np.bincount(d["dst"][eb], minlength=N))])
+    uvw = spec.mode == "uvw"
+    wf = dict(s=d["s"][eids], W=d["W"]) if uvw else dict(w=d["w"][eids])
+    wb = dict(s=d["s"][eb], W=d["W"]) if uvw else dict(w=d["w"][eb])
     t0 = time.perf_counter()
-    forward(op, rpf, d["src"][eids], d["x"], d["vec"][eids], w=d["w"][eids])
+    forward(op, rpf, d["src"][eids], d["x"], d["vec"][eids], **wf)
     t1 = time.perf_counter()
-    backward(op, rpb, d["src"][eb], d["x"], d["vec"][eb], d["gy"], w=d["w"][eb])
+    backward(op, rpb, d["src"][eb], d["x"], d["vec"][eb], d["gy"], **wb)
     t2 = time.perf_counter()
     return len(eids), t1 - t0, len(eb), t2 - t1
 
@@ -236,7 +246,7 @@ def run_reference(args, rank):
     import synth
     from oracle.conv import set_threads
     cores = set_threads()
-    if args.workload == "c2-layer":
+    if args.workload.endswith("-layer"):
         return run_reference_layer(args, cores)
     d = synth.make_inputs(args.workload)
     oracle_sample(d, 4, seed=0)                      # CG tables cached outside the timing
@@ -654,6 +664,14 @@ def run_ours(args, rank, world, local):
     return 0
 
 
+def linear_flops(ir_in, ir_out, N):
+    """2 N sum_k (2l+1) mul_in mul_out over the linear map's instructions (same (l, parity) pairs)."""
+    def terms(s):
+        return [(int(t.split("x")[0]), int(t.split("x")[1][:-1]), t[-1]) for t in s.split("+")]
+    return 2 * N * sum((2 * li + 1) * mi * mo for mi, li, pi in terms(ir_in) for mo, lo, po in terms(ir_out)
+                       if (li, pi) == (lo, po))
+
+
 def layer_node_bytes(lin, N, bwd):
     """Algorithmic bytes of one linear call: fwd reads x and W, writes y; bwd reads x, W and gy,
     writes gx and gW."""
@@ -668,7 +686,8 @@ def oracle_layer_sample(d, n_rows, seed, W1, W2, g_out):
     from oracle.block import GateSpec, gate, gate_backward, linear, linear_backward
     spec = d["spec"]
     ir = spec.irreps_in
-    gs = GateSpec(*LAYER_GATE)
+    mid, gate_args = layer_shapes(int(ir.split("x")[0]))
+    gs = GateSpec(*gate_args)
     N = len(d["rowptr"]) - 1
     E = len(d["src"])
     t0 = time.perf_counter()
@@ -679,33 +698,36 @@ def oracle_layer_sample(d, n_rows, seed, W1, W2, g_out):
     ef, tf, eb, tb = oracle_sample(dd, n_rows, seed)
     t2 = time.perf_counter()
     y = d["gy"]        # a node array of the convolution's output width (the sampled conv gives no full y)
-    h2 = linear(spec.irreps_out, LAYER_MID, y, W2)
+    h2 = linear(spec.irreps_out, mid, y, W2)
     gate(gs, h2)
     g_h2 = gate_backward(gs, h2, g_out)
-    linear_backward(spec.irreps_out, LAYER_MID, y, W2, g_h2)
+    linear_backward(spec.irreps_out, mid, y, W2, g_h2)
     linear_backward(ir, ir, d["x"], W1, np.asarray(d["x"]))
     t3 = time.perf_counter()
     node_t = (t1 - t0) + (t3 - t2)
     return 1.0 / (tf / ef + tb / eb + node_t / E), ef, eb, tf + tb + node_t
 
 
-def layer_weights(spec, N, n_w1, n_w2, rank=0):
-    """Seeded weights of the two linear maps (N(0, 1/32): fan-in 32) and the upstream gradient."""
+def layer_weights(spec, N, n_w1, n_w2, out_dim, rank=0):
+    """Seeded weights of the two linear maps (N(0, 1/fan-in)) and the upstream gradient."""
+    mul = int(spec.irreps_in.split("x")[0])
     rng = np.random.default_rng(spec.seed + 17 + 7919 * rank)
-    W1 = (rng.standard_normal(n_w1) / math.sqrt(32)).astype(np.float32)
-    W2 = (rng.standard_normal(n_w2) / math.sqrt(32)).astype(np.float32)
-    g_out = rng.standard_normal((N, 288), dtype=np.float32)
+    W1 = (rng.standard_normal(n_w1) / math.sqrt(mul)).astype(np.float32)
+    W2 = (rng.standard_normal(n_w2) / math.sqrt(mul)).astype(np.float32)
+    g_out = rng.standard_normal((N, out_dim), dtype=np.float32)
     return W1, W2, g_out
 
 
 def run_reference_layer(args, cores):
     import synth
-    spec = synth.CONFIGS["c2"]
-    d = synth.make_inputs("c2")
+    from oracle.block import GateSpec, linear_weight_count
+    base = args.workload.split("-")[0]
+    spec = synth.CONFIGS[base]
+    d = synth.make_inputs(base)
     N = len(d["rowptr"]) - 1
-    from oracle.block import linear_weight_count
+    mid, gate_args = layer_shapes(int(spec.irreps_in.split("x")[0]))
     W1, W2, g_out = layer_weights(spec, N, linear_weight_count(spec.irreps_in, spec.irreps_in),
-                                  linear_weight_count(spec.irreps_out, LAYER_MID))
+                                  linear_weight_count(spec.irreps_out, mid), GateSpec(*gate_args).out_dim)
     oracle_sample(d, 4, seed=0)
     v, ef, eb, t = oracle_layer_sample(d, 16, 1, W1, W2, g_out)
     rows = int(max(2, min(256, 16 * 60.0 / max(1, args.steps + args.warmup) / t)))
@@ -746,23 +768,27 @@ def run_layer(args, rank, world, local):
     import synth
     lib = tp.load()
 
-    spec = synth.CONFIGS["c2"]
-    d = synth.make_inputs("c2", args.n_atoms, seed=spec.seed + 7919 * rank)
+    base = args.workload.split("-")[0]
+    spec = synth.CONFIGS[base]
+    d = synth.make_inputs(base, args.n_atoms, seed=spec.seed + 7919 * rank)
     if args.order == "cell":
         d = synth.cell_sorted(d)
     N, E = len(d["rowptr"]) - 1, len(d["src"])
+    uvw = spec.mode == "uvw"
+    wkey = "s" if uvw else "w"
+    mid, gate_args = layer_shapes(int(spec.irreps_in.split("x")[0]))
     # the 1/average-degree scale of the aggregated messages rides on the next linear map's
     # coefficients (it commutes with the map), which keeps the convolution on its
     # unit-coefficient compiled instances
-    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvu")
-    n2 = tp.Linear(spec.irreps_out, LAYER_MID).n_instructions
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, spec.mode)
+    n2 = tp.Linear(spec.irreps_out, mid).n_instructions
     lin1 = tp.Linear(spec.irreps_in, spec.irreps_in)
-    lin2 = tp.Linear(spec.irreps_out, LAYER_MID, coeff=[N / max(E, 1)] * n2)
-    gate = tp.Gate(*LAYER_GATE)
-    W1, W2, d["g_out"] = layer_weights(spec, N, lin1.n_weights, lin2.n_weights, rank)
+    lin2 = tp.Linear(spec.irreps_out, mid, coeff=[N / max(E, 1)] * n2)
+    gate = tp.Gate(*gate_args)
+    W1, W2, d["g_out"] = layer_weights(spec, N, lin1.n_weights, lin2.n_weights, gate.out_dim, rank)
     in_dim, out_dim, nw = plan.in_dim, plan.out_dim, plan.n_edge_weights
 
-    keys = ["rowptr", "src", "x", "vec", "w", "g_out"]
+    keys = ["rowptr", "src", "x", "vec", wkey, "g_out"] + (["W"] if uvw else [])
     copy_bytes = sum(d[k].nbytes for k in keys)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     R = max(2, math.ceil(2.5 * l2 / copy_bytes))
@@ -774,21 +800,22 @@ def run_layer(args, rank, world, local):
             src_d = dict(d)
             src_d["x"] = rr.standard_normal(d["x"].shape, dtype=np.float32)
             src_d["g_out"] = rr.standard_normal(d["g_out"].shape, dtype=np.float32)
-            src_d["w"] = (d["w"] * rr.uniform(0.5, 1.5, size=(1, nw))).astype(np.float32)
+            src_d[wkey] = (d[wkey] * rr.uniform(0.5, 1.5, size=(1, nw))).astype(np.float32)
         copies.append({k: torch.as_tensor(np.ascontiguousarray(src_d[k])).to(dev) for k in keys})
     W1d, W2d = torch.as_tensor(W1).to(dev), torch.as_tensor(W2).to(dev)
     f32 = lambda *shape: torch.empty(*shape, device=dev)
     h1, y, h2, out = f32(N, in_dim), f32(N, out_dim), f32(N, lin2.out_dim), f32(N, gate.out_dim)
     g_h2, g_y, g_h1, gx, gw = f32(N, lin2.out_dim), f32(N, out_dim), f32(N, in_dim), f32(N, in_dim), f32(E, nw)
     gW1, gW2 = f32(lin1.n_weights), f32(lin2.n_weights)
+    gWc = f32(plan.n_shared_weights) if uvw else None
     colptrs = [torch.empty(N + 1, dtype=torch.int32, device=dev) for _ in range(R)]
     perms = [torch.empty(E, dtype=torch.int32, device=dev) for _ in range(R)]
     ws_bytes = max(tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD), tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     wl_bytes = max(tp.tp_linear_workspace_size(lin, N, op) for lin in (lin1, lin2) for op in (0, 1))
     wl = torch.empty(wl_bytes, dtype=torch.uint8, device=dev)
-    wt_bytes = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD)
-    wt = torch.empty(wt_bytes, dtype=torch.uint8, device=dev)
+    wt_bytes = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD) if not uvw else 256 + 8 * (N + E) + 4096
+    wt = torch.empty(wt_bytes, dtype=torch.uint8, device=dev)      # side-stream transpose scratch
     stream, side = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     sh, sh_side = stream.cuda_stream, side.cuda_stream
     P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None
@@ -798,14 +825,15 @@ def run_layer(args, rank, world, local):
     def op_list(cp, colptr, perm):
         return [
             ("linear_in fwd", lf, (lin1.handle, N, P(cp["x"]), P(W1d), P(h1), 0, P(wl), wl_bytes, sh)),
-            ("conv fwd", cf, (plan.handle, N, E, P(cp["rowptr"]), P(cp["src"]), P(h1), P(cp["vec"]), P(cp["w"]),
-                              None, P(y), P(ws), ws_bytes, sh)),
+            ("conv fwd", cf, (plan.handle, N, E, P(cp["rowptr"]), P(cp["src"]), P(h1), P(cp["vec"]), P(cp[wkey]),
+                              P(cp.get("W")), P(y), P(ws), ws_bytes, sh)),
             ("linear_out fwd", lf, (lin2.handle, N, P(y), P(W2d), P(h2), 0, P(wl), wl_bytes, sh)),
             ("gate fwd", gf, (gate.handle, N, P(h2), P(out), sh)),
             ("gate bwd", gb, (gate.handle, N, P(h2), P(cp["g_out"]), P(g_h2), sh)),
             ("linear_out bwd", lb, (lin2.handle, N, P(y), P(W2d), P(g_h2), P(g_y), P(gW2), P(wl), wl_bytes, sh)),
             ("conv bwd", cb, (plan.handle, N, E, P(cp["rowptr"]), P(cp["src"]), P(colptr), P(perm), P(h1),
-                              P(cp["vec"]), P(cp["w"]), None, P(g_y), P(g_h1), P(gw), None, None, P(ws), ws_bytes, sh)),
+                              P(cp["vec"]), P(cp[wkey]), P(cp.get("W")), P(g_y), P(g_h1), P(gw), None, P(gWc),
+                              P(ws), ws_bytes, sh)),
             ("linear_in bwd", lb, (lin1.handle, N, P(cp["x"]), P(W1d), P(g_h1), P(gx), P(gW1), P(wl), wl_bytes, sh)),
         ]
 
@@ -900,7 +928,7 @@ def run_layer(args, rank, world, local):
     # inputs up, the layer forward and backward, the gradients and the output down
     host_in = {k: torch.as_tensor(np.ascontiguousarray(d[k])).pin_memory() for k in keys}
     dv = {k: torch.empty_like(host_in[k], device=dev) for k in keys}
-    outs = (out, gx, gw, gW1, gW2)
+    outs = (out, gx, gw, gW1, gW2) + ((gWc,) if uvw else ())
     host_out = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in outs]
     e_ops = op_list(dv, colptrs[0], perms[0])
     e_tr = (N, E, P(dv["rowptr"]), P(dv["src"]), P(colptrs[0]), P(perms[0]), P(wt), wt_bytes, sh)
@@ -940,24 +968,40 @@ def run_layer(args, rank, world, local):
                "linear_out bwd": layer_node_bytes(lin2, N, True),
                "conv bwd": bwd_bytes(N, E, in_dim, out_dim, nw, False),
                "linear_in bwd": layer_node_bytes(lin1, N, True)}
+        fl1, fl2 = linear_flops(spec.irreps_in, spec.irreps_in, N), linear_flops(spec.irreps_out, mid, N)
+        flops = {"linear_in fwd": fl1, "linear_out fwd": fl2, "linear_out bwd": 2 * fl2, "linear_in bwd": 2 * fl1}
         kname = max(op_ms, key=op_ms.get)
-        achieved = alg[kname] / (op_ms[kname] * 1e-3) / 1e9
         step_s = elapsed_max / args.steps
-        roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "peak_note": peak_note, "traffic": traffic_from_profile(kname, "c2-layer"),
-                "algorithmic_bytes_per_launch": alg[kname],
-                "ops": {nm: {"ms": op_ms[nm], "algorithmic_bytes": alg[nm],
-                             "hbm_frac": alg[nm] / (op_ms[nm] * 1e-3) / 1e9 / hbm} for nm in names},
-                "step_roofline_frac": (sum(alg.values()) / (hbm * 1e9)) / step_s}
+        ops = {nm: {"ms": op_ms[nm], "algorithmic_bytes": alg[nm],
+                    "hbm_frac": alg[nm] / (op_ms[nm] * 1e-3) / 1e9 / hbm,
+                    **({"flops": flops[nm], "tflops": flops[nm] / (op_ms[nm] * 1e-3) / 1e12} if nm in flops else {})}
+               for nm in names}
+        if uvw and kname.startswith("conv"):
+            # the uvw convolution is bound by the fp32 pipe (its per-edge CG work), as in the c4 line
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            peak = 2 * 128 * sms * clk.max_mhz_or(1965.0) * 1e6 / 1e12
+            fl = uvw_bwd_flops(spec, E) * (1.0 if kname == "conv bwd" else 0.5)
+            achieved = fl / (op_ms[kname] * 1e-3) / 1e12
+            roof = {"bound": "alu", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "peak_note": "fp32 FMA peak from the unit counts and max clock",
+                    "traffic": None, "algorithmic_flops_per_call": fl, "ops": ops,
+                    "step_roofline_frac": (sum(alg.values()) / (hbm * 1e9)) / step_s}
+        else:
+            achieved = alg[kname] / (op_ms[kname] * 1e-3) / 1e9
+            roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "peak_note": peak_note, "traffic": traffic_from_profile(kname, args.workload),
+                    "algorithmic_bytes_per_launch": alg[kname], "ops": ops,
+                    "step_roofline_frac": (sum(alg.values()) / (hbm * 1e9)) / step_s}
         cpu = None
         if not args.no_cpu_baseline:
             from oracle.conv import set_threads
             cores = set_threads()
             oracle_sample(d, 4, seed=0)
-            v, ef, eb, t = oracle_layer_sample(d, min(N, 1536), 3, W1, W2, d["g_out"])
+            n_rows = min(N, 64 if uvw else 1536)
+            v, ef, eb, t = oracle_layer_sample(d, n_rows, 3, W1, W2, d["g_out"])
             cpu = {"value": v, "unit": "edges/s", "cores": cores, "kind": "oracle",
                    "sample": f"linears and gate (fwd + bwd) on all {N} nodes; conv fwd on the {ef} edges into and "
-                             f"bwd on the {eb} edges out of {min(N, 1536)} sampled rows; float64, {t:.1f} s"}
+                             f"bwd on the {eb} edges out of {n_rows} sampled rows; float64, {t:.1f} s"}
         line = {
             "metric": METRIC, "value": replica_throughput(E, args.steps, world, elapsed_max), "unit": "edges/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * step_s,
@@ -1065,7 +1109,7 @@ def main():
         return run_reference(args, rank)
     if args.workload == "c1":
         return run_latency(args, rank, world, local)
-    if args.workload == "c2-layer":
+    if args.workload.endswith("-layer"):
         return run_layer(args, rank, world, local)
     return run_ours(args, rank, world, local)
 
