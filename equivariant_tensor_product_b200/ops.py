@@ -174,7 +174,9 @@ def tp_conv_dbwd(plan: Plan, rowptr, src, x, vec, w, gy, ggx=None, ggw=None, ggv
     return g_gy, g_x, g_w, g_vec
 
 
-def tp_get_device_error(plan: Plan, ws: torch.Tensor, stream=None) -> int:
+def tp_get_device_error(plan: Optional[Plan], ws: Optional[torch.Tensor], stream=None) -> int:
+    """Reads and clears the device error word (plan None: the per-device word)."""
     code = C.c_int32()
-    check(load().tp_get_device_error(plan.handle, _ptr(ws), _stream(stream), C.byref(code)), "tp_get_device_error")
+    check(load().tp_get_device_error(plan.handle if plan is not None else None, _ptr(ws), _stream(stream),
+                                     C.byref(code)), "tp_get_device_error")
     return code.value

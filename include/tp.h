@@ -158,8 +158,9 @@ tp_status_t tp_conv_dbwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* ro
                          size_t ws_bytes, tp_stream_t stream);
 
 /* Reads (and clears) the device error word after the work on `stream` finished;
- * synchronises the stream.  Check-mode plans read the word of workspace `ws`; other plans
- * read the per-device word (ws unused).  *code: 0 = none, 1 = bad rowptr, 2 = bad src,
+ * synchronises the stream.  Check-mode plans read the word of workspace `ws`; other plans,
+ * and plan == NULL, read the per-device word (ws unused) -- the word the linear maps of
+ * tp_block.h report their bounded-wait timeouts to as well.  *code: 0 = none, 1 = bad rowptr, 2 = bad src,
  * 3 = bad perm / transpose entry, 6 = a bounded device wait gave up. */
 tp_status_t tp_get_device_error(tp_plan_t plan, void* ws, tp_stream_t stream, int32_t* code);
 

@@ -44,7 +44,7 @@
  * `stream` and returns.  Errors: host checks return a status before anything is enqueued
  * (NULL arguments, sizes, 4-byte alignment, irreps rules); TP_ERR_CUDA for a failed launch.
  * The GEMMs' device waits are bounded (4 s) and a wait that gives up records code 6 in the
- * per-device error word that tp_get_device_error reads for plans without index checks.
+ * per-device error word, which tp_get_device_error(NULL, NULL, stream, &code) reads.
  */
 #ifndef TP_BLOCK_H_
 #define TP_BLOCK_H_

@@ -176,6 +176,16 @@ def test_no_cpu_fallback_without_device(lib, tp):
     assert b"cuda" in lib.tp_last_error_message().lower() or lib.tp_last_error_message()
 
 
+def test_device_error_word_without_a_plan(lib):
+    """plan NULL reads the per-device word (used by the linear maps); code NULL is rejected
+    first; without a device the read fails loudly instead of reporting 0."""
+    import torch
+    code = C.c_int32(-1)
+    assert lib.tp_get_device_error(None, None, None, None) == 1
+    if not torch.cuda.is_available():
+        assert lib.tp_get_device_error(None, None, None, C.byref(code)) == 5
+
+
 def test_bounded_wait_check_rejects_bad_arguments_before_the_device(lib):
     res = C.c_int32(-1)
     assert lib.tp_check_bounded_waits(0, None, C.byref(res)) == 1

@@ -7,7 +7,8 @@
 * Memory contract: with outputs and workspace supplied by the caller, a call allocates no
   device memory at all (the library never allocates; the workspace is node sized plus int
   edge indices).
-* The per-device error word of plans without index checks reads 0 after normal calls.
+* The per-device error word of plans without index checks (and of the linear maps, read
+  without a plan) reads 0 after normal calls.
 """
 import ctypes as C
 import time
@@ -89,3 +90,9 @@ def test_device_error_word_reads_zero_after_normal_calls(tp):
     tp.tp_conv_fwd(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["w"])
     tp.tp_conv_bwd(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["w"], g["gy"])
     assert tp.tp_get_device_error(plan, None) == 0
+    # the linear maps' tensor-core GEMMs report to the same per-device word, read without a plan
+    lin = tp.Linear("32x0e+32x1o", "32x0e+32x1o", flags=tp.TP_LINEAR_TENSOR_CORES)
+    xl = torch.randn(300, lin.in_dim, device="cuda")
+    Wl = torch.randn(lin.n_weights, device="cuda")
+    tp.tp_linear_bwd(lin, xl, Wl, tp.tp_linear_fwd(lin, xl, Wl))
+    assert tp.tp_get_device_error(None, None) == 0
