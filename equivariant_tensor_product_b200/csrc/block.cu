@@ -1,9 +1,11 @@
 // Node-side operators of the interaction layer (include/tp_block.h): the irreps-wise
-// linear map on the tcgen05 tensor cores (3xTF32, the persistent GEMM of tp_mma.cuh with
-// its own operand regrouping and epilogues) and the gate nonlinearity (elementwise).
+// linear map, in two forms -- on the CUDA cores straight from the node rows (narrow maps or
+// few nodes: k_lin_direct, k_lin_direct_gw) or on the tcgen05 tensor cores (3xTF32, the
+// persistent GEMM of tp_mma.cuh with its own operand regrouping and epilogues) -- and the
+// gate nonlinearity (elementwise, k_gate).
 //
-// Linear, per irrep type t = (l, parity) that has instructions (every input block of type t
-// is connected to every output block of type t):
+// Tensor-core linear, per irrep type t = (l, parity) that has instructions (every input
+// block of type t is connected to every output block of type t):
 //   XA_t[(n, m)][kc]  = x[n, b, u, m]          kc = (input block b of type t, channel u)
 //   GA_t[(n, m)][oc]  = gy[n, o, w, m]         oc = (output block o of type t, channel w)
 //   y_o   = XA_t . Wt_o^T     Wt_o[w][kc] = c_k W_k[u, w]      one GEMM per output block
@@ -49,7 +51,6 @@ struct GatherArgs {
   int d[kLinMaxTypes], K[kLinMaxTypes], nblk[kLinMaxTypes];
   int64_t cum[kLinMaxTypes];                       // group g starts at dst + N * cum[g]
   int boff[kLinMaxTypes][kLinMaxBlocks];           // block offset in the source row
-  int bmul[kLinMaxTypes][kLinMaxBlocks];
   int bcat[kLinMaxTypes][kLinMaxBlocks];           // first concatenated channel of the block
   float* zdst;
   int64_t zstride;
@@ -622,7 +623,6 @@ GatherArgs gather_args(const tp_linear_s* L, int64_t N, const float* src, float*
     for (int b = 0; b < g.nblk[q]; ++b) {
       const int blk = out_side ? T.out_blk[b] : T.in_blk[b];
       g.boff[q][b] = (int)(out_side ? L->out_off[blk] : L->in_off[blk]);
-      g.bmul[q][b] = out_side ? L->out[blk].mul : L->in[blk].mul;
       g.bcat[q][b] = out_side ? T.out_cat[b] : T.in_cat[b];
     }
   }
