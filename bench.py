@@ -65,6 +65,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="c2", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the records of the other configurations measured after the headline")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--n-atoms", type=int, default=None,
                     help="same-density replica with fewer atoms (profiling small cases)")
@@ -129,16 +131,89 @@ def uvw_bwd_flops(spec, E):
     return E * mul * per
 
 
-def dbwd_flops_estimate(spec, E):
-    """Double-backward fp32 flops by the published-count estimate u * sum_p (20 nnz_p + 10 d3_p)
-    per edge (three couplings per path and their SH-derivative terms); an estimate, not a count
-    of the generated code."""
+def _ls(irreps):
+    return [int(b.split("x")[1][:-1]) for b in irreps.split("+")]
+
+
+def _cg_terms(spec):
+    """Per path (l1, l2, l3, nnz) and, for the outer products the generated bodies share, the
+    number of distinct index pairs used per block pair: (in, sh) -> (m1, m2) for the couplings
+    C(x, Y); (sh, out) -> (m2, m3) for the transposed ones; (in, out) -> (m1, m3) for the
+    direction gradient.  Pairs of an l2 = 0 block cost nothing (Y_0 = 1)."""
     from equivariant_tensor_product_b200.csrc.codegen import cg_nonzeros
+    li, lsh, lo = _ls(spec.irreps_in), _ls(spec.irreps_sh), _ls(spec.irreps_out)
+    paths, u_xy, u_yg, u_xg = [], {}, {}, {}
+    for a, b, o in spec.paths:
+        nz = cg_nonzeros(li[a], lsh[b], lo[o])
+        paths.append((li[a], lsh[b], lo[o], len(nz)))
+        if lsh[b] > 0:
+            u_xy.setdefault((a, b), set()).update((i, j) for i, j, k, c in nz)
+            u_yg.setdefault((b, o), set()).update((j, k) for i, j, k, c in nz)
+            u_xg.setdefault((a, o), set()).update((i, k) for i, j, k, c in nz)
+    n = lambda u: sum(len(v) for v in u.values())
+    return paths, n(u_xy), n(u_yg), n(u_xg)
+
+
+def fwd_flops(spec, E):
+    """Useful fp32 flops of the uvu forward, per edge and channel: one product per shared
+    (m1, m2) pair, then per path and m3 a chain over its CG non-zeros (2 flops each) and the
+    weighted accumulation (2 per m3; the first product of a chain saves one, counted as 2 nnz
+    + d3 in total)."""
+    paths, uxy, _, _ = _cg_terms(spec)
     mul = int(spec.irreps_in.split("x")[0])
-    ls = lambda irr: [int(b.split("x")[1][0]) for b in irr.split("+")]
-    li, lsh, lo = ls(spec.irreps_in), ls(spec.irreps_sh), ls(spec.irreps_out)
-    per = sum(20 * len(cg_nonzeros(li[a], lsh[b], lo[o])) + 10 * (2 * lo[o] + 1) for a, b, o in spec.paths)
+    return E * mul * (uxy + sum(2 * nnz + (2 * l3 + 1) for _, _, l3, nnz in paths))
+
+
+def bwd_flops(spec, E, gvec):
+    """uvu backward (gx, gw[, gvec]) per edge and channel: products per shared (m2, m3) pair;
+    per path the chains z_m1 = sum C Y gy (2 nnz - d1), gx += w z (2 d1) and gw = <x, z>
+    (2 d1 - 1); with gvec, products per shared (m1, m3) pair and per path with l2 > 0 the
+    chains q_m2 = sum C x gy (2 nnz - d2) and gY += w q (2 d2).  The per-edge (not per-channel)
+    direction-gradient epilogue is not counted."""
+    paths, _, uyg, uxg = _cg_terms(spec)
+    mul = int(spec.irreps_in.split("x")[0])
+    per = uyg + sum(2 * nnz + 3 * (2 * l1 + 1) - 1 for l1, _, _, nnz in paths)
+    if gvec:
+        per += uxg + sum(2 * nnz + (2 * l2 + 1) for _, l2, _, nnz in paths if l2 > 0)
     return E * mul * per
+
+
+def dbwd_flops(spec, E):
+    """uvu double backward per edge and channel, term by term:
+      g_gy: per shared (m1, m2) pair q = x Y (1) and h = ggx Y + x Y' (3); per path two chains
+            over the non-zeros (t = C q, u = C h: 4 nnz - 2 d3) and acc += ggw t + w u (4 d3);
+      g_x, g_w: per shared (m2, m3) pair r = Y gy and r' = Y' gy (2); per path z = C r and
+            z' = C r' (4 nnz - 2 d1), g_x += ggw z + w z' (4 d1), g_w = <ggx, z> + <x, z'> (4 d1);
+      g_vec: per shared (m1, m3) pair s = x gy and s' = ggx gy (2); per path with l2 > 0 the
+            chains qa = C s and qb = C s' (4 nnz - 2 d2), G1 += ggw qa + w qb (4 d2), G2 += w qa
+            (2 d2).
+    Y' = dY[ggvec] and the per-edge SH derivative terms are per edge, not per channel, and are
+    not counted."""
+    paths, uxy, uyg, uxg = _cg_terms(spec)
+    mul = int(spec.irreps_in.split("x")[0])
+    per = 4 * uxy + 2 * uyg + 2 * uxg
+    for l1, l2, l3, nnz in paths:
+        per += 4 * nnz + 2 * (2 * l3 + 1)
+        per += 4 * nnz + 6 * (2 * l1 + 1)
+        if l2 > 0:
+            per += 4 * nnz + 4 * (2 * l2 + 1)
+    return E * mul * per
+
+
+def uvw_fwd_cg_flops(spec, E):
+    """CUDA-core flops of the uvw edge pass per edge and channel: as the uvu forward with the
+    per-path scalar s[e, p] in place of w (the mixing runs on the tensor cores)."""
+    return fwd_flops(spec, E)
+
+
+def uvw_gemm_flops(spec, N, bwd):
+    """Mixing contractions: forward 2 N sum_p d3 mul_in mul_out; backward three of the same
+    size (x W, B W^T and x^T B, the last two with d1 in place of d3)."""
+    li, lo = _ls(spec.irreps_in), _ls(spec.irreps_out)
+    mi, mo = int(spec.irreps_in.split("x")[0]), int(spec.irreps_out.split("x")[0])
+    if bwd:
+        return 3 * 2 * N * sum((2 * li[a] + 1) * mi * mo for a, b, o in spec.paths)
+    return 2 * N * sum((2 * lo[o] + 1) * mi * mo for a, b, o in spec.paths)
 
 
 def bwd_bytes(N, E, in_dim, out_dim, nw, gvec):
@@ -269,7 +344,8 @@ def run_reference(args, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOADS[args.workload], "name": args.workload},
+            "config": {"workload": WORKLOADS[args.workload], "name": args.workload, "N": len(d["rowptr"]) - 1,
+                       "E": len(d["src"]), "order": "generation order (random)", "parallelism": "single"},
             "cpu_baseline": {"value": value, "unit": "edges/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -311,31 +387,44 @@ def measured_peaks():
     return 6650.0, 1590.0, "of fallback"
 
 
-def run_ours(args, rank, world, local):
-    import torch
-    import torch.distributed as dist
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+def tc_peak_3xtf32(bf16_tflops):
+    """fp32 work through 3xTF32 on tcgen05: the TF32 rate (the measured bf16 peak times the
+    nominal TF32 / bf16 ratio, 1.1 / 2.25 PFLOP/s) divided by the three MMAs per product."""
+    return bf16_tflops * (1.1 / 2.25) / 3.0
 
-    from equivariant_tensor_product_b200 import build as tpbuild
-    tpbuild.build()
-    import equivariant_tensor_product_b200 as tp
+
+def pass_roofline(ms, nbytes, flops, hbm_gbs, fp32_tflops, gemm_flops=0.0, tc_tflops=None):
+    """Roofline of one call: the slowest of its algorithmic bytes at the HBM peak, its CUDA-core
+    flops at the fp32 FMA peak and its tensor-core flops at the 3xTF32 peak; frac = that time
+    over the measured time."""
+    t = {"hbm": nbytes / (hbm_gbs * 1e9), "alu": flops / (fp32_tflops * 1e12)}
+    if gemm_flops and tc_tflops:
+        t["tensor"] = gemm_flops / (tc_tflops * 1e12)
+    bound = max(t, key=t.get)
+    sec = ms * 1e-3
+    out = {"ms": ms, "bound": bound, "roofline_ms": 1e3 * t[bound], "frac": t[bound] / sec,
+           "algorithmic_bytes": nbytes, "cuda_core_flops": flops, "achieved_GBps": nbytes / sec / 1e9,
+           "achieved_fp32_TFLOPs": flops / sec / 1e12, "hbm_frac": t["hbm"] / sec, "alu_frac": t["alu"] / sec}
+    if "tensor" in t:
+        out.update({"tensor_flops": gemm_flops, "tensor_frac": t["tensor"] / sec})
+    return out
+
+
+def prepare_workload(tp, lib, torch, dev, name, n_atoms=None, order="random", rank=0):
+    """Inputs of one convolution workload resident in HBM (R rotating seeded copies, together
+    more than 2.5 x L2), its output buffers and workspaces, and the C-ABI argument tuples of
+    one step: forward, the transpose on a side stream, backward (and double backward)."""
+    import types
     import synth
-    lib = tp.load()
-
-    spec = synth.CONFIGS[args.workload]
+    spec = synth.CONFIGS[name]
     with_dbwd = "dbwd" in spec.passes
-    d = synth.make_inputs(args.workload, args.n_atoms, with_gg=with_dbwd, seed=spec.seed + 7919 * rank)
-    if args.order == "cell":
+    d = synth.make_inputs(name, n_atoms, with_gg=with_dbwd, seed=spec.seed + 7919 * rank)
+    if order == "cell":
         d = synth.cell_sorted(d)
     plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, spec.mode)
     N, E = len(d["rowptr"]) - 1, len(d["src"])
     in_dim, out_dim, nw = plan.in_dim, plan.out_dim, plan.n_edge_weights
-    want_gvec = "dbwd" in spec.passes or args.workload == "c5"
-
+    want_gvec = with_dbwd or name == "c5"
     uvw = spec.mode == "uvw"
     wkey = "s" if uvw else "w"
     keys = ["rowptr", "src", "x", "vec", wkey, "gy"] + (["W"] if uvw else [])
@@ -344,9 +433,8 @@ def run_ours(args, rank, world, local):
     R = max(2, math.ceil(2.5 * l2 / copy_bytes))
     copies = []
     for r in range(R):
-        if r == 0:
-            src_d = d
-        else:
+        src_d = d
+        if r:
             rng = np.random.default_rng(spec.seed + 31 * r + 7919 * rank)
             src_d = dict(d)
             src_d["x"] = rng.standard_normal(d["x"].shape, dtype=np.float32)
@@ -361,20 +449,18 @@ def run_ours(args, rank, world, local):
     # forward of step k runs on the main stream (they are independent); the backward waits
     colptrs = [torch.empty(N + 1, dtype=torch.int32, device=dev) for _ in range(R)]
     perms = [torch.empty(E, dtype=torch.int32, device=dev) for _ in range(R)]
-    colptr, perm = colptrs[0], perms[0]
     gW = torch.empty(plan.n_shared_weights, device=dev) if uvw else None
     ws_bytes = max(tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD), tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD),
                    tp.tp_workspace_size(plan, N, E, tp.TP_OP_DBWD) if with_dbwd else 0)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    ws_t_bytes = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD) if not uvw else 256 + 8 * (N + E) + 4096
+    ws_t_bytes = max(256, tp.tp_csr_transpose_workspace_size(N, E))
     ws_t = torch.empty(ws_t_bytes, dtype=torch.uint8, device=dev)      # side-stream transpose scratch
-    stream = torch.cuda.Stream(dev)    # a capturable stream for all of the bench's work
-    side = torch.cuda.Stream(dev)
-    sh = stream.cuda_stream
-    sh_side = side.cuda_stream
+    # the transpose's side stream runs at a higher priority, so that its few small kernels get
+    # SM slots as the forward's CTAs retire instead of queueing behind all of them
+    stream, side = torch.cuda.Stream(dev), torch.cuda.Stream(dev, priority=-1)
+    sh, sh_side = stream.cuda_stream, side.cuda_stream
     h = plan.handle
     P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None
-
     argsets = []
     for r, cp in enumerate(copies):
         Wp = P(cp["W"]) if uvw else None
@@ -385,155 +471,333 @@ def run_ours(args, rank, world, local):
             (h, N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(cp["x"]), P(cp["vec"]),
              P(cp[wkey]), Wp, P(cp["gy"]), P(gx), P(gw), P(gvec), P(gW), P(ws), ws_bytes, sh),
         ))
+    dargs, dbuf = None, {}
     if with_dbwd:   # second-order upstream gradients, one set shared by the copies (each > L2)
-        gg = {k: torch.as_tensor(np.ascontiguousarray(d[k])).to(dev) for k in ("ggx", "ggw", "ggvec")}
-        g_gy = torch.empty(N, out_dim, device=dev)
-        g_x = torch.empty(N, in_dim, device=dev)
-        g_w = torch.empty(E, nw, device=dev)
-        g_vec = torch.empty(E, 3, device=dev)
+        dbuf = {k: torch.as_tensor(np.ascontiguousarray(d[k])).to(dev) for k in ("ggx", "ggw", "ggvec")}
+        dbuf.update(g_gy=torch.empty(N, out_dim, device=dev), g_x=torch.empty(N, in_dim, device=dev),
+                    g_w=torch.empty(E, nw, device=dev), g_vec=torch.empty(E, 3, device=dev))
         dargs = [(h, N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(cp["x"]), P(cp["vec"]),
-                  P(cp[wkey]), None, P(cp["gy"]), P(gg["ggx"]), P(gg["ggw"]), P(gg["ggvec"]), P(g_gy), P(g_x),
-                  P(g_w), P(g_vec), P(ws), ws_bytes, sh) for r, cp in enumerate(copies)]
-    dbwd_f = lib.tp_conv_dbwd
-    tr_done = [torch.cuda.Event() for _ in range(R)]
-    bwd_done = [torch.cuda.Event() for _ in range(R)]
-    fwd_f, tr_f, bwd_f = lib.tp_conv_fwd, lib.tp_csr_transpose, lib.tp_conv_bwd
+                  P(cp[wkey]), None, P(cp["gy"]), P(dbuf["ggx"]), P(dbuf["ggw"]), P(dbuf["ggvec"]),
+                  P(dbuf["g_gy"]), P(dbuf["g_x"]), P(dbuf["g_w"]), P(dbuf["g_vec"]), P(ws), ws_bytes, sh)
+                 for r, cp in enumerate(copies)]
+    return types.SimpleNamespace(
+        name=name, spec=spec, d=d, plan=plan, N=N, E=E, in_dim=in_dim, out_dim=out_dim, nw=nw, uvw=uvw, wkey=wkey,
+        keys=keys, with_dbwd=with_dbwd, want_gvec=want_gvec, copy_bytes=copy_bytes, l2=l2, R=R, copies=copies,
+        y=y, gx=gx, gw=gw, gvec=gvec, gW=gW, colptrs=colptrs, perms=perms, ws=ws, ws_bytes=ws_bytes, ws_t=ws_t,
+        ws_t_bytes=ws_t_bytes, stream=stream, side=side, argsets=argsets, dargs=dargs, dbuf=dbuf, P=P,
+        tr_done=[torch.cuda.Event() for _ in range(R)], bwd_done=[torch.cuda.Event() for _ in range(R)],
+        order=order, dev=dev)
 
-    def step(k, ev=None):
-        r = k % R
-        a_f, a_t, a_b = argsets[r]
-        # side stream: this step's transpose, once the backward that last read this copy is done
-        side.wait_event(bwd_done[r])
-        if ev is not None:
-            ev[4].record(side)
-        st = tr_f(*a_t)
-        if ev is not None:
-            ev[5].record(side)
-        tr_done[r].record(side)
-        if ev is not None:
-            ev[0].record(stream)
-        st |= fwd_f(*a_f)
-        if ev is not None:
-            ev[1].record(stream)
-        stream.wait_event(tr_done[r])
-        if ev is not None:
-            ev[2].record(stream)
-        st |= bwd_f(*a_b)
-        if ev is not None:
-            ev[3].record(stream)
-        if with_dbwd:
-            st |= dbwd_f(*dargs[r])
-            if ev is not None:
-                ev[6].record(stream)
-        bwd_done[r].record(stream)
-        if st:
-            raise RuntimeError(lib.tp_last_error_message().decode())
 
-    for k in range(args.warmup):
-        step(k)
-    torch.cuda.synchronize(dev)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+def eager_step(w, lib, k, ev=None):
+    """One step through the C ABI: transpose (side stream), forward, backward (+ dbwd)."""
+    r = k % w.R
+    a_f, a_t, a_b = w.argsets[r]
+    w.side.wait_event(w.bwd_done[r])          # the backward that last read this copy is done
+    if ev is not None:
+        ev[4].record(w.side)
+    st = lib.tp_csr_transpose(*a_t)
+    if ev is not None:
+        ev[5].record(w.side)
+    w.tr_done[r].record(w.side)
+    if ev is not None:
+        ev[0].record(w.stream)
+    st |= lib.tp_conv_fwd(*a_f)
+    if ev is not None:
+        ev[1].record(w.stream)
+    w.stream.wait_event(w.tr_done[r])
+    if ev is not None:
+        ev[2].record(w.stream)
+    st |= lib.tp_conv_bwd(*a_b)
+    if ev is not None:
+        ev[3].record(w.stream)
+    if w.with_dbwd:
+        st |= lib.tp_conv_dbwd(*w.dargs[r])
+        if ev is not None:
+            ev[6].record(w.stream)
+    w.bwd_done[r].record(w.stream)
+    if st:
+        raise RuntimeError(lib.tp_last_error_message().decode())
+
+
+def time_eager(w, lib, torch, steps, warmup, local, world):
+    """Eager steps with an event pair around every call: per-call mean times and the step time."""
+    import torch.distributed as dist
+    for k in range(warmup):
+        eager_step(w, lib, k)
+    torch.cuda.synchronize(w.dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(w.dev)
+    free0 = torch.cuda.mem_get_info(w.dev)[0]
     n0 = lib.tp_launch_count()
     with ClockSampler(local) as clk:
-        start.record(stream)
-        for k in range(args.steps):
-            step(k, evs[k])
-        stop.record(stream)
-        torch.cuda.synchronize(dev)
+        start.record(w.stream)
+        for k in range(steps):
+            eager_step(w, lib, k, evs[k])
+        stop.record(w.stream)
+        torch.cuda.synchronize(w.dev)
     launches = lib.tp_launch_count() - n0
+    free1 = torch.cuda.mem_get_info(w.dev)[0]
     if world > 1:
         dist.barrier()
-    elapsed = start.elapsed_time(stop) / 1e3
-    elapsed_max = max_over_ranks(elapsed, world, dev)
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    tr_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in evs)
-    bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    dbwd_ms = statistics.mean(e[3].elapsed_time(e[6]) for e in evs) if with_dbwd else None
-    eager_ms_per_step = 1e3 * elapsed_max / args.steps
+    km = {"fwd": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
+          "transpose": statistics.mean(e[4].elapsed_time(e[5]) for e in evs),
+          "bwd": statistics.mean(e[2].elapsed_time(e[3]) for e in evs)}
+    if w.with_dbwd:
+        km["dbwd"] = statistics.mean(e[3].elapsed_time(e[6]) for e in evs)
+    return start.elapsed_time(stop) / 1e3, km, launches, clk, free0 - free1
 
-    # The same steps replayed as CUDA graphs (one per input copy, captured from the same C ABI
-    # calls: transpose forked onto the side stream, joined before the backward), which removes
-    # the host launch path from between the kernels.  The per-call times above come from the
-    # eager loop; the step throughput from this one when the capture succeeds.
-    launch_mode, graph_note = "eager", None
+
+def time_graphs(w, lib, torch, steps, warmup, local, world):
+    """The same steps captured as one CUDA graph per input copy (transpose forked onto the side
+    stream and joined before the backward) and replayed: removes the host launch path from
+    between the kernels.  Returns (elapsed_s, launches, clk, note); elapsed None if capture
+    failed."""
+    import torch.distributed as dist
     graphs = []
     try:
         n_cap = lib.tp_launch_count()
-        for r in range(R):
+        for r in range(w.R):
             g = torch.cuda.CUDAGraph()
             fork, join = torch.cuda.Event(), torch.cuda.Event()
-            a_f, a_t, a_b = argsets[r]
-            with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
-                fork.record(stream)
-                side.wait_event(fork)
-                st = tr_f(*a_t)
-                join.record(side)
-                st |= fwd_f(*a_f)
-                stream.wait_event(join)
-                st |= bwd_f(*a_b)
-                if with_dbwd:
-                    st |= dbwd_f(*dargs[r])
+            a_f, a_t, a_b = w.argsets[r]
+            with torch.cuda.graph(g, stream=w.stream, capture_error_mode="thread_local"):
+                fork.record(w.stream)
+                w.side.wait_event(fork)
+                st = lib.tp_csr_transpose(*a_t)
+                join.record(w.side)
+                st |= lib.tp_conv_fwd(*a_f)
+                w.stream.wait_event(join)
+                st |= lib.tp_conv_bwd(*a_b)
+                if w.with_dbwd:
+                    st |= lib.tp_conv_dbwd(*w.dargs[r])
             if st:
                 raise RuntimeError(lib.tp_last_error_message().decode())
             graphs.append(g)
-        per_step_launches = (lib.tp_launch_count() - n_cap) // R
+        per_step = (lib.tp_launch_count() - n_cap) // w.R
     except Exception as exc:  # noqa: BLE001
-        graphs, graph_note = [], f"capture failed: {exc}"[:200]
-    if graphs:
-        with torch.cuda.stream(stream):
-            for k in range(args.warmup):
-                graphs[k % R].replay()
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-        with ClockSampler(local) as clk:
-            start.record(stream)
-            with torch.cuda.stream(stream):
-                for k in range(args.steps):
-                    graphs[k % R].replay()
-            stop.record(stream)
-            torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        elapsed = start.elapsed_time(stop) / 1e3
-        elapsed_max = max_over_ranks(elapsed, world, dev)
-        launches = per_step_launches * args.steps
-        launch_mode = "cuda_graph"
+        return None, 0, None, f"capture failed: {exc}"[:200]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(w.stream):
+        for k in range(warmup):
+            graphs[k % w.R].replay()
+    torch.cuda.synchronize(w.dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(w.dev)
+    with ClockSampler(local) as clk:
+        start.record(w.stream)
+        with torch.cuda.stream(w.stream):
+            for k in range(steps):
+                graphs[k % w.R].replay()
+        stop.record(w.stream)
+        torch.cuda.synchronize(w.dev)
+    if world > 1:
+        dist.barrier()
+    elapsed = start.elapsed_time(stop) / 1e3
+    graphs.clear()   # no graph outlives the process group
+    return elapsed, per_step * steps, clk, None
+
+
+def pass_rooflines(w, km, hbm, fp32_peak, tc_peak):
+    """Per-call rooflines of a workload: bytes and CUDA-core flops from the algorithmic counts
+    above (and the mixing GEMMs for uvw)."""
+    N, E, spec = w.N, w.E, w.spec
+    out = {}
+    if w.uvw:
+        fb = fwd_bytes(N, E, w.in_dim, w.out_dim, w.nw) + 4 * w.plan.n_shared_weights
+        bb = bwd_bytes(N, E, w.in_dim, w.out_dim, w.nw, w.want_gvec) + 8 * w.plan.n_shared_weights
+        out["fwd"] = pass_roofline(km["fwd"], fb, uvw_fwd_cg_flops(spec, E), hbm, fp32_peak,
+                                   uvw_gemm_flops(spec, N, False), tc_peak)
+        out["bwd"] = pass_roofline(km["bwd"], bb, uvw_bwd_flops(spec, E), hbm, fp32_peak,
+                                   uvw_gemm_flops(spec, N, True), tc_peak)
+    else:
+        out["fwd"] = pass_roofline(km["fwd"], fwd_bytes(N, E, w.in_dim, w.out_dim, w.nw), fwd_flops(spec, E), hbm,
+                                   fp32_peak)
+        out["bwd"] = pass_roofline(km["bwd"], bwd_bytes(N, E, w.in_dim, w.out_dim, w.nw, w.want_gvec),
+                                   bwd_flops(spec, E, w.want_gvec), hbm, fp32_peak)
+        if w.with_dbwd:
+            out["dbwd"] = pass_roofline(km["dbwd"], dbwd_bytes(N, E, w.in_dim, w.out_dim, w.nw), dbwd_flops(spec, E),
+                                        hbm, fp32_peak)
+    return out
+
+
+KERNEL_OF_PASS = {("uvu", "fwd"): "k_fwd_uvu", ("uvu", "bwd"): "k_bwd_uvu",
+                  ("uvu", "dbwd"): "k_dbwd_recv + k_dbwd_send",
+                  ("uvw", "fwd"): "tp_conv_fwd (uvw: k_uvw_edge_staged, mixing GEMMs)",
+                  ("uvw", "bwd"): "tp_conv_bwd (uvw: k_uvw_send, x W / B W^T / x^T B GEMMs)"}
+
+
+def config_record(tp, lib, torch, dev, name, steps, warmup, local, hbm, fp32_peak, tc_peak, order="random"):
+    """A compact measured record of one workload in the same run: per-call times and rooflines
+    (eager loop) and the step time (CUDA-graph replay)."""
+    w = prepare_workload(tp, lib, torch, dev, name, order=order)
+    el, km, _, clk_e, _ = time_eager(w, lib, torch, steps, warmup, local, 1)
+    eg, _, clk_g, note = time_graphs(w, lib, torch, steps, warmup, local, 1)
+    ms = 1e3 * (eg if eg is not None else el) / steps
+    rec = {"workload": WORKLOADS[name], "N": w.N, "E": w.E, "order": "cell-sorted" if order == "cell" else
+           "generation order (random)", "steps": steps, "ms_per_step": ms, "edges_per_s": w.E / (ms * 1e-3),
+           "launch": "cuda_graph" if eg is not None else "eager", "eager_ms_per_step": 1e3 * el / steps,
+           "kernel_ms": km, "passes": pass_rooflines(w, km, hbm, fp32_peak, tc_peak),
+           "clocks": (clk_g or clk_e).summary()}
+    if note:
+        rec["graph_note"] = note
+    del w
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from equivariant_tensor_product_b200 import build as tpbuild
+    tpbuild.build()
+    import equivariant_tensor_product_b200 as tp
+    lib = tp.load()
+
+    w = prepare_workload(tp, lib, torch, dev, args.workload, args.n_atoms, args.order, rank)
+    N, E, spec, uvw = w.N, w.E, w.spec, w.uvw
+    elapsed, km, launches, clk, free_drop = time_eager(w, lib, torch, args.steps, args.warmup, local, world)
+    elapsed_max = max_over_ranks(elapsed, world, dev)
+    eager_ms_per_step = 1e3 * elapsed_max / args.steps
+    launch_mode, graph_note = "eager", None
+    eg, lg, clk_g, graph_note = time_graphs(w, lib, torch, args.steps, args.warmup, local, world)
+    if eg is not None:
+        elapsed = eg
+        elapsed_max = max_over_ranks(eg, world, dev)
+        launches, clk, launch_mode = lg, clk_g, "cuda_graph"
 
     # End to end through the same calls: every step copies its inputs from pinned host memory
     # and its results back.  Two device buffer sets let the copies overlap: the inputs of step
     # k+1 go up and the results of step k-1 come down (each on its own copy stream) while step
     # k computes; nothing is skipped or cached between steps.
-    e2e_keys = keys + (["ggx", "ggw", "ggvec"] if with_dbwd else [])
-    host_in = {k: torch.as_tensor(np.ascontiguousarray(d[k])).pin_memory() for k in e2e_keys}
-    outs = (y, gx, gw) + ((gvec,) if want_gvec else ()) + ((gW,) if uvw else ()) + \
-        ((g_gy, g_x, g_w, g_vec) if with_dbwd else ())
+    e2e_value, h2d, d2h = run_e2e(w, lib, torch, args.e2e_steps, world)
+
+    if rank == 0:
+        hbm, bf16, peak_note = measured_peaks()
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        fp32_peak = 2 * 128 * sms * clk.max_mhz_or(1965.0) * 1e6 / 1e12
+        tc_peak = tc_peak_3xtf32(bf16)
+        passes = pass_rooflines(w, km, hbm, fp32_peak, tc_peak)
+        dom = max(passes, key=lambda k: passes[k]["ms"])
+        dp = passes[dom]
+        kname = KERNEL_OF_PASS[(spec.mode, dom)]
+        if dp["bound"] == "hbm":
+            roof = {"bound": "hbm", "kernel": kname, "achieved": dp["achieved_GBps"], "peak": hbm, "unit": "GB/s",
+                    "frac": dp["achieved_GBps"] / hbm, "peak_note": peak_note,
+                    "traffic": traffic_from_profile(kname, args.workload),
+                    "algorithmic_bytes_per_launch": dp["algorithmic_bytes"]}
+        elif dp["bound"] == "alu":
+            roof = {"bound": "alu", "kernel": kname, "achieved": dp["achieved_fp32_TFLOPs"], "peak": fp32_peak,
+                    "unit": "TFLOP/s", "frac": dp["achieved_fp32_TFLOPs"] / fp32_peak,
+                    "peak_note": "fp32 FMA peak: 2 flop x 128 lanes x SMs x max SM clock; flops counted from the "
+                                 "term lists of bench.py (fwd_flops, bwd_flops, dbwd_flops, uvw_bwd_flops)",
+                    "traffic": traffic_from_profile(kname, args.workload),
+                    "algorithmic_flops_per_call": dp["cuda_core_flops"], "hbm_frac": dp["hbm_frac"]}
+        else:
+            roof = {"bound": "tensor", "kernel": kname, "achieved": dp["tensor_flops"] / (dp["ms"] * 1e-3) / 1e12,
+                    "peak": tc_peak, "unit": "TFLOP/s", "frac": dp["tensor_frac"],
+                    "peak_note": f"3xTF32 from the measured bf16 peak ({peak_note})", "traffic": None}
+        roof.update({"kernel_ms": km, "passes": passes,
+                     "step_roofline_frac": sum(p["roofline_ms"] for p in passes.values()) /
+                     (1e3 * elapsed / args.steps)})
+        cpu = None
+        if not args.no_cpu_baseline and not uvw:
+            from oracle.conv import set_threads
+            cores = set_threads()
+            oracle_sample(w.d, 4, seed=0)            # CG tables cached outside the timing
+            n_rows = min(N, 1536)
+            ef, tf, eb, tb = oracle_sample(w.d, n_rows, seed=3)
+            cpu = {"value": cpu_edges_per_s(ef, tf, eb, tb), "unit": "edges/s", "cores": cores, "kind": "oracle",
+                   "sample": f"fwd on the {ef} edges into {n_rows} receivers + bwd on the {eb} edges leaving "
+                             f"{n_rows} senders of the same workload (rank 0's copy), float64 torch CPU, "
+                             f"{tf + tb:.1f} s"}
+        value = replica_throughput(E, args.steps, world, elapsed_max)
+        line = {
+            "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * elapsed_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload], "name": args.workload, "N": N, "E": E,
+                       "order": "cell-sorted" if args.order == "cell" else "generation order (random)",
+                       "launch": launch_mode, "eager_ms_per_step": eager_ms_per_step,
+                       **({"graph_note": graph_note} if graph_note else {}),
+                       "l2": f"{w.R} rotating input copies of {w.copy_bytes / 1e6:.1f} MB (> 2x L2 of "
+                             f"{w.l2 / 1e6:.0f} MB)", "parallelism": "replicas" if world > 1 else "single"},
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "edges/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": args.e2e_steps,
+                    "pipeline": "two device buffer sets; the H2D copy of step k+1 and the D2H copy of step k-1 "
+                                "overlap step k on their own streams"},
+            "gpu_launches": int(launches), "clocks": clk.summary(),
+            "memory": {"workspace_bytes": w.ws_bytes, "transpose_workspace_bytes": w.ws_t_bytes,
+                       "edge_sized_float_scratch_bytes": 0,
+                       "device_free_bytes_lost_during_timed_steps": int(free_drop),
+                       "note": "the library allocates nothing: every buffer, workspaces included, is the caller's; "
+                               "the workspaces hold int32 graph indices (and, for uvw, node- and weight-sized "
+                               "state), never an edge x feature float tensor"},
+            "library": tp.tp_version(),
+        }
+        if world == 1 and not args.no_per_config and args.workload == "c2" and args.n_atoms is None:
+            # the other configurations measured in the same run (compact records)
+            del w
+            torch.cuda.empty_cache()
+            per = {}
+            for name, st, wu in (("c3", 100, 5), ("c5", 30, 3), ("c4", 10, 3)):
+                per[name] = config_record(tp, lib, torch, dev, name, st, wu, local, hbm, fp32_peak, tc_peak)
+            for name, st, wu in (("c3", 100, 5), ("c4", 10, 3)):
+                per[name + "-cell"] = config_record(tp, lib, torch, dev, name, st, wu, local, hbm, fp32_peak,
+                                                    tc_peak, order="cell")
+            line["per_config"] = per
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(w, lib, torch, e2e_steps, world):
+    """End-to-end leg: the same calls with the inputs copied up from pinned host memory and every
+    output copied back inside the timed region, pipelined over two device buffer sets."""
+    dev, P, N, E = w.dev, w.P, w.N, w.E
+    stream, side = w.stream, w.side
+    sh, sh_side = stream.cuda_stream, side.cuda_stream
+    h = w.plan.handle
+    wkey, uvw = w.wkey, w.uvw
+    e2e_keys = w.keys + (["ggx", "ggw", "ggvec"] if w.with_dbwd else [])
+    host_in = {k: torch.as_tensor(np.ascontiguousarray(w.d[k])).pin_memory() for k in e2e_keys}
+    outs = (w.y, w.gx, w.gw) + ((w.gvec,) if w.want_gvec else ()) + ((w.gW,) if uvw else ()) + \
+        (tuple(w.dbuf[k] for k in ("g_gy", "g_x", "g_w", "g_vec")) if w.with_dbwd else ())
     host_out = [torch.empty(t_.shape, dtype=t_.dtype).pin_memory() for t_ in outs]
     s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     sets = []
     for b in range(2):
         dv = {k: torch.empty_like(host_in[k], device=dev) for k in e2e_keys}
         ob = [torch.empty_like(t_) for t_ in outs]
-        o = dict(zip(["y", "gx", "gw"] + (["gvec"] if want_gvec else []) + (["gW"] if uvw else []) +
-                     (["g_gy", "g_x", "g_w", "g_vec"] if with_dbwd else []), ob))
+        o = dict(zip(["y", "gx", "gw"] + (["gvec"] if w.want_gvec else []) + (["gW"] if uvw else []) +
+                     (["g_gy", "g_x", "g_w", "g_vec"] if w.with_dbwd else []), ob))
         cpb = torch.empty(N + 1, dtype=torch.int32, device=dev)
         pmb = torch.empty(E, dtype=torch.int32, device=dev)
         Wd = P(dv["W"]) if uvw else None
-        fa = (h, N, E, P(dv["rowptr"]), P(dv["src"]), P(dv["x"]), P(dv["vec"]), P(dv[wkey]), Wd, P(o["y"]), P(ws),
-              ws_bytes, sh)
-        ta = (N, E, P(dv["rowptr"]), P(dv["src"]), P(cpb), P(pmb), P(ws_t), ws_t_bytes, sh_side)
+        fa = (h, N, E, P(dv["rowptr"]), P(dv["src"]), P(dv["x"]), P(dv["vec"]), P(dv[wkey]), Wd, P(o["y"]), P(w.ws),
+              w.ws_bytes, sh)
+        ta = (N, E, P(dv["rowptr"]), P(dv["src"]), P(cpb), P(pmb), P(w.ws_t), w.ws_t_bytes, sh_side)
         ba = (h, N, E, P(dv["rowptr"]), P(dv["src"]), P(cpb), P(pmb), P(dv["x"]), P(dv["vec"]), P(dv[wkey]), Wd,
-              P(dv["gy"]), P(o["gx"]), P(o["gw"]), P(o.get("gvec")), P(o.get("gW")), P(ws), ws_bytes, sh)
+              P(dv["gy"]), P(o["gx"]), P(o["gw"]), P(o.get("gvec")), P(o.get("gW")), P(w.ws), w.ws_bytes, sh)
         da = None
-        if with_dbwd:
+        if w.with_dbwd:
             da = (h, N, E, P(dv["rowptr"]), P(dv["src"]), P(cpb), P(pmb), P(dv["x"]), P(dv["vec"]), P(dv[wkey]), None,
                   P(dv["gy"]), P(dv["ggx"]), P(dv["ggw"]), P(dv["ggvec"]), P(o["g_gy"]), P(o["g_x"]), P(o["g_w"]),
-                  P(o["g_vec"]), P(ws), ws_bytes, sh)
+                  P(o["g_vec"]), P(w.ws), w.ws_bytes, sh)
         sets.append((dv, ob, fa, ta, ba, da))
     h2d_done = [torch.cuda.Event() for _ in range(2)]
     tr2_done = [torch.cuda.Event() for _ in range(2)]
@@ -549,15 +813,15 @@ def run_ours(args, rank, world, local):
                 dv[key].copy_(host_in[key], non_blocking=True)
         h2d_done[b].record(s_h2d)
         side.wait_event(h2d_done[b])
-        st = tr_f(*ta)
+        st = lib.tp_csr_transpose(*ta)
         tr2_done[b].record(side)
         stream.wait_event(h2d_done[b])
         stream.wait_event(d2h_done[b])            # step k-2's results are out of set b
-        st |= fwd_f(*fa)
+        st |= lib.tp_conv_fwd(*fa)
         stream.wait_event(tr2_done[b])
-        st |= bwd_f(*ba)
-        if with_dbwd:
-            st |= dbwd_f(*da)
+        st |= lib.tp_conv_bwd(*ba)
+        if w.with_dbwd:
+            st |= lib.tp_conv_dbwd(*da)
         comp_done[b].record(stream)
         if st:
             raise RuntimeError(lib.tp_last_error_message().decode())
@@ -575,93 +839,16 @@ def run_ours(args, rank, world, local):
     s_h2d.wait_stream(stream)
     s_d2h.wait_stream(stream)
     side.wait_stream(stream)
-    for k in range(args.e2e_steps):
+    for k in range(e2e_steps):
         e2e_step(k)
     stream.wait_stream(s_d2h)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_s = e0.elapsed_time(e1) / 1e3
-    e2e_value = replica_throughput(E, args.e2e_steps, world, max_over_ranks(e2e_s, world, dev))
+    value = replica_throughput(E, e2e_steps, world, max_over_ranks(e2e_s, world, dev))
     h2d = sum(host_in[k].numel() * host_in[k].element_size() for k in e2e_keys)
     d2h = sum(t_.numel() * t_.element_size() for t_ in host_out)
-
-    if rank == 0:
-        hbm, _, peak_note = measured_peaks()
-        fb = fwd_bytes(N, E, in_dim, out_dim, nw)
-        bb = bwd_bytes(N, E, in_dim, out_dim, nw, want_gvec)
-        db = dbwd_bytes(N, E, in_dim, out_dim, nw) if with_dbwd else 0
-        kernel_ms = {"fwd": fwd_ms, "transpose": tr_ms, "bwd": bwd_ms}
-        if with_dbwd:
-            kernel_ms["dbwd"] = dbwd_ms
-        if uvw:
-            # CUDA-core bound: the per-edge CG work of the backward call (sender pass) against
-            # 2 flop x 128 fp32 lanes x SMs x max SM clock; the mixing GEMMs are not counted
-            sms = torch.cuda.get_device_properties(dev).multi_processor_count
-            peak = 2 * 128 * sms * clk.max_mhz_or(1965.0) * 1e6 / 1e12
-            flops = uvw_bwd_flops(spec, E)
-            achieved = flops / (bwd_ms * 1e-3) / 1e12
-            roof = {"bound": "alu", "kernel": "tp_conv_bwd (uvw: k_uvw_send, x W / B W^T / x^T B GEMMs)",
-                    "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                    "peak_note": "fp32 FMA peak from the unit counts and max clock", "traffic": None,
-                    "algorithmic_flops_per_call": flops, "kernel_ms": kernel_ms}
-        else:
-            cands = [("k_fwd_uvu", fb, fwd_ms), ("k_bwd_uvu", bb, bwd_ms)]
-            if with_dbwd:
-                cands.append(("k_dbwd_recv + k_dbwd_send", db, dbwd_ms))
-            kname, kbytes, kms = max(cands, key=lambda t: t[2])
-            if kname.startswith("k_dbwd"):
-                # the double backward is bound by the fp32 pipe, not by its bytes
-                sms = torch.cuda.get_device_properties(dev).multi_processor_count
-                peak = 2 * 128 * sms * clk.max_mhz_or(1965.0) * 1e6 / 1e12
-                flops = dbwd_flops_estimate(spec, E)
-                achieved = flops / (kms * 1e-3) / 1e12
-                roof = {"bound": "alu", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                        "frac": achieved / peak, "peak_note": "fp32 FMA peak from the unit counts and max clock; "
-                        "flops by the estimate u * sum_p (20 nnz_p + 10 d3_p) per edge", "traffic": None,
-                        "algorithmic_flops_per_call": flops, "algorithmic_bytes_per_call": kbytes,
-                        "hbm_frac": kbytes / (kms * 1e-3) / 1e9 / hbm, "kernel_ms": kernel_ms}
-            else:
-                achieved = kbytes / (kms * 1e-3) / 1e9
-                roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                        "frac": achieved / hbm, "peak_note": peak_note,
-                        "traffic": traffic_from_profile(kname, args.workload),
-                        "algorithmic_bytes_per_launch": kbytes, "kernel_ms": kernel_ms,
-                        "step_roofline_frac": ((fb + bb + db) / (hbm * 1e9)) / (elapsed / args.steps)}
-        cpu = None
-        if not args.no_cpu_baseline and not uvw:
-            from oracle.conv import set_threads
-            cores = set_threads()
-            oracle_sample(d, 4, seed=0)              # CG tables cached outside the timing
-            n_rows = min(N, 1536)
-            ef, tf, eb, tb = oracle_sample(d, n_rows, seed=3)
-            cpu = {"value": cpu_edges_per_s(ef, tf, eb, tb), "unit": "edges/s", "cores": cores, "kind": "oracle",
-                   "sample": f"fwd on the {ef} edges into {n_rows} receivers + bwd on the {eb} edges leaving "
-                             f"{n_rows} senders of the same workload (rank 0's copy), float64 torch CPU, "
-                             f"{tf + tb:.1f} s"}
-        value = replica_throughput(E, args.steps, world, elapsed_max)
-        line = {
-            "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1e3 * elapsed_max / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOADS[args.workload], "name": args.workload, "N": N, "E": E,
-                       "order": "cell-sorted" if args.order == "cell" else "generation order (random)",
-                       "launch": launch_mode, "eager_ms_per_step": eager_ms_per_step,
-                       **({"graph_note": graph_note} if graph_note else {}),
-                       "l2": f"{R} rotating input copies of {copy_bytes / 1e6:.1f} MB (> 2x L2 of "
-                             f"{l2 / 1e6:.0f} MB)", "parallelism": "replicas" if world > 1 else "single"},
-            "roofline": roof, "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "edges/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": args.e2e_steps,
-                    "pipeline": "two device buffer sets; the H2D copy of step k+1 and the D2H copy of step k-1 "
-                                "overlap step k on their own streams"},
-            "gpu_launches": int(launches), "clocks": clk.summary(),
-        }
-        print(json.dumps(line), flush=True)
-    graphs.clear()   # no graph outlives the process group
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    return 0
+    return value, h2d, d2h
 
 
 def linear_flops(ir_in, ir_out, N):
@@ -814,9 +1001,9 @@ def run_layer(args, rank, world, local):
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     wl_bytes = max(tp.tp_linear_workspace_size(lin, N, op) for lin in (lin1, lin2) for op in (0, 1))
     wl = torch.empty(wl_bytes, dtype=torch.uint8, device=dev)
-    wt_bytes = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD) if not uvw else 256 + 8 * (N + E) + 4096
+    wt_bytes = max(256, tp.tp_csr_transpose_workspace_size(N, E))
     wt = torch.empty(wt_bytes, dtype=torch.uint8, device=dev)      # side-stream transpose scratch
-    stream, side = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    stream, side = torch.cuda.Stream(dev), torch.cuda.Stream(dev, priority=-1)   # transpose: high priority
     sh, sh_side = stream.cuda_stream, side.cuda_stream
     P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None
     lf, lb, gf, gb = lib.tp_linear_fwd, lib.tp_linear_bwd, lib.tp_gate_fwd, lib.tp_gate_bwd

@@ -25,6 +25,7 @@ SIGNATURES = {
     "tp_plan_destroy": (C.c_int, [_p]),
     "tp_plan_query": (C.c_int, [_p, C.POINTER(_i64), C.POINTER(_i64), C.POINTER(_i64), C.POINTER(_i64)]),
     "tp_workspace_size": (C.c_int, [_p, _i64, _i64, _i32, C.POINTER(_sz)]),
+    "tp_csr_transpose_workspace_size": (C.c_int, [_i64, _i64, C.POINTER(_sz)]),
     "tp_csr_transpose": (C.c_int, [_i64, _i64, _p, _p, _p, _p, _p, _sz, _p]),
     "tp_conv_fwd": (C.c_int, [_p, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "tp_conv_bwd": (C.c_int, [_p, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz,

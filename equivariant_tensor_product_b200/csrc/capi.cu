@@ -111,10 +111,10 @@ bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t header, colptr, counts, perm, tmp, total;
+  size_t header, colptr, perm, scratch, total;
 };
 
-// header (error word) | colptr[N+1] | counts[N] | perm[E] | tmp[E]
+// header (error word) | colptr[N+1] | perm[E] | transpose scratch (int32, see csr.cu)
 WsLayout ws_layout(int64_t N, int64_t E) {
   WsLayout L{};
   size_t off = 0;
@@ -122,19 +122,21 @@ WsLayout ws_layout(int64_t N, int64_t E) {
   off += 256;
   L.colptr = off;
   off += align256(sizeof(int32_t) * (size_t)(N + 1));
-  L.counts = off;
-  off += align256(sizeof(int32_t) * (size_t)(N > 0 ? N : 1));
   L.perm = off;
   off += align256(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
-  L.tmp = off;
-  off += align256(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+  L.scratch = off;
+  off += align256(sizeof(int32_t) * (size_t)transpose_scratch_ints(N, E));
   L.total = off;
   return L;
 }
 
 // uvw regions (floats, 256-byte aligned).  Forward: A | Wt (hi, lo).  Backward, after the
 // transpose region: A (x W) | G (B) | xT | Wt (Wg hi, lo, Wx hi, lo) | part.
-constexpr int kUvwSplits = 64;
+// Split-K partials of the gW GEMM: one per 1,536 nodes, at most 64.  Every split then
+// reduces at least ~768 * d1 rows (24 or more K blocks), so the fp32 promotion of the
+// accumulator (every 16 K blocks) runs at every size beyond a few hundred nodes, and a large
+// graph keeps 64 splits of parallel work.
+int uvw_splits(int64_t N) { return (int)std::min<int64_t>(64, std::max<int64_t>(1, (N + 1535) / 1536)); }
 struct UvwLayout {
   size_t A, G, xT, Wt, part, total;
 };
@@ -154,7 +156,7 @@ UvwLayout uvw_layout(tp_plan_t plan, int64_t N, int64_t E, bool bwd) {
   U.Wt = off;
   off += align256(w_bytes * (bwd ? 4 : 2));
   U.part = off;
-  if (bwd) off += align256(w_bytes * kUvwSplits);
+  if (bwd) off += align256(w_bytes * uvw_splits(N));
   U.total = off;
   return U;
 }
@@ -404,6 +406,14 @@ tp_status_t tp_workspace_size(tp_plan_t plan, int64_t N, int64_t E, int32_t op, 
   return TP_OK;
 }
 
+tp_status_t tp_csr_transpose_workspace_size(int64_t N, int64_t E, size_t* bytes) {
+  if (!bytes) return fail(TP_ERR_INVALID_ARG, "bytes is NULL");
+  if (N < 0 || E < 0 || N >= (int64_t)1 << 31 || E >= (int64_t)1 << 31)
+    return fail(TP_ERR_INVALID_ARG, "N and E must be in [0, 2^31)");
+  *bytes = sizeof(int32_t) * (size_t)transpose_scratch_ints(N, E);
+  return TP_OK;
+}
+
 tp_status_t tp_csr_transpose(int64_t N, int64_t E, const int32_t* rowptr, const int32_t* src,
                              int32_t* colptr, int32_t* perm, void* ws, size_t ws_bytes,
                              tp_stream_t stream) {
@@ -412,14 +422,11 @@ tp_status_t tp_csr_transpose(int64_t N, int64_t E, const int32_t* rowptr, const 
     return fail(TP_ERR_INVALID_ARG, "N and E must be in [0, 2^31)");
   if (!colptr || (E > 0 && (!src || !perm))) return fail(TP_ERR_INVALID_ARG, "null pointer");
   if (!aligned4(src) || !aligned4(colptr) || !aligned4(perm)) return fail(TP_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
-  const WsLayout L = ws_layout(N, E);
-  const size_t need = L.tmp + align256(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+  const size_t need = sizeof(int32_t) * (size_t)transpose_scratch_ints(N, E);
   if (!ws || ws_bytes < need) return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes", need);
-  char* w = static_cast<char*>(ws);
+  if (reinterpret_cast<uintptr_t>(ws) & 3u) return fail(TP_ERR_INVALID_ARG, "workspace must be 4-byte aligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_csr_transpose((int)N, (int)E, src, colptr, perm,
-                                       reinterpret_cast<int32_t*>(w + L.counts),
-                                       reinterpret_cast<int32_t*>(w + L.tmp), s);
+  cudaError_t e = launch_csr_transpose((int)N, (int)E, src, colptr, perm, static_cast<int32_t*>(ws), s);
   if (e != cudaSuccess) return cuda_fail(e, "csr_transpose");
   return TP_OK;
 }
@@ -478,8 +485,7 @@ tp_status_t sender_order(int64_t N, int64_t E, const int32_t* src, const int32_t
   char* w = static_cast<char*>(ws);
   int32_t* cp = reinterpret_cast<int32_t*>(w + L.colptr);
   int32_t* pm = reinterpret_cast<int32_t*>(w + L.perm);
-  cudaError_t e = launch_csr_transpose((int)N, (int)E, src, cp, pm, reinterpret_cast<int32_t*>(w + L.counts),
-                                       reinterpret_cast<int32_t*>(w + L.tmp), s);
+  cudaError_t e = launch_csr_transpose((int)N, (int)E, src, cp, pm, reinterpret_cast<int32_t*>(w + L.scratch), s);
   if (e != cudaSuccess) return cuda_fail(e, "csr_transpose");
   colptr = cp;
   perm = pm;
@@ -534,7 +540,7 @@ tp_status_t tp_conv_bwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* row
     a.Wt = reinterpret_cast<float*>(wsb + U.Wt);
     a.xT = reinterpret_cast<float*>(wsb + U.xT);
     a.part = reinterpret_cast<float*>(wsb + U.part);
-    a.splits = kUvwSplits;
+    a.splits = uvw_splits(N);
     a.gW = gW;
     a.nw = plan->n_paths;
     cudaError_t e = plan->ops->uvw_bwd(a, s);

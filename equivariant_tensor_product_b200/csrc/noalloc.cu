@@ -5,23 +5,25 @@
 // memory belongs to a pool it does not control, a framework that has reserved (almost) all
 // of the GPU up front so a fresh cudaMalloc would fail, or a loop that must not call
 // cudaMalloc/cudaFree because those calls synchronise the device.  This entry point needs
-// nothing from them beyond the inputs and outputs: the per-sender counters and the
-// unordered scatter buffer that tp_csr_transpose takes from the caller's workspace live in
-// one file-scope __device__ array instead.
+// nothing from them beyond the inputs and outputs: the scratch that tp_csr_transpose takes
+// from the caller's workspace (the radix sort's second id buffer and its per-tile digit
+// counts) lives in one file-scope __device__ array instead.
 //
 // Costs and rules of that choice:
-//   * every GPU that loads the library holds the array (kScratchInts int32, about 4.5 MB)
+//   * every GPU that loads the library holds the array (kScratchInts int32, about 5.3 MB)
 //     until the process exits;
 //   * N <= kNoAllocMaxN and E <= kNoAllocMaxE, larger graphs are rejected
 //     (TP_ERR_UNSUPPORTED) before any work is enqueued;
 //   * all calls share the array: two calls whose work overlaps on the GPU (different
 //     streams, or different host threads, without ordering between them) race and produce
 //     wrong results; order them on one stream or synchronise between them;
-//   * the array keeps whatever the last call left in it; the counters are cleared at the
-//     start of every call, the scatter buffer is fully written before it is read.
+//   * the array keeps whatever the last call left in it; every kernel of a call writes the
+//     part it later reads (digit counts, scans, ids) before reading it, so nothing needs
+//     clearing;
 //   * the first call on each device looks up the array's device address
 //     (cudaGetSymbolAddress) with that device current; make that first call before any
-//     stream capture.
+//     stream capture.  The address is kept until exit: a cudaDeviceReset between calls is
+//     not supported.
 #include <mutex>
 
 #include "../../include/tp.h"
@@ -31,10 +33,21 @@ namespace {
 
 constexpr int64_t kNoAllocMaxN = 1 << 17;   // 131,072 nodes
 constexpr int64_t kNoAllocMaxE = 1 << 20;   // 1,048,576 edges
-constexpr int64_t kScratchInts = kNoAllocMaxN + kNoAllocMaxE;
+
+// The largest transpose scratch over every N <= kNoAllocMaxN at E = kNoAllocMaxE (the digit
+// width, and so the count table, depends on the number of key bits of N).
+constexpr int64_t max_scratch_ints() {
+  int64_t best = tp::transpose_scratch_ints(kNoAllocMaxN, kNoAllocMaxE);
+  for (int64_t n = 1; n < kNoAllocMaxN; n = 2 * n + 1) {
+    const int64_t v = tp::transpose_scratch_ints(n, kNoAllocMaxE);
+    if (v > best) best = v;
+  }
+  return best;
+}
+constexpr int64_t kScratchInts = max_scratch_ints();
 constexpr int kMaxDevices = 64;
 
-// counts[kNoAllocMaxN] followed by the scatter buffer tmp[kNoAllocMaxE].
+// The radix sort's scratch (see csr.cu): an id buffer and per-tile digit counts.
 static __device__ __align__(256) int32_t g_transpose_scratch[kScratchInts];
 
 std::mutex g_mu;
@@ -73,8 +86,9 @@ extern "C" tp_status_t tp_csr_transpose_noalloc(int64_t N, int64_t E, const int3
     return TP_ERR_INVALID_ARG;
   int32_t* scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) return TP_ERR_CUDA;
-  if (tp::launch_csr_transpose((int)N, (int)E, src, colptr, perm, scratch, scratch + kNoAllocMaxN,
-                               reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (tp::transpose_scratch_ints(N, E) > kScratchInts) return TP_ERR_UNSUPPORTED;
+  if (tp::launch_csr_transpose((int)N, (int)E, src, colptr, perm, scratch, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
     return TP_ERR_CUDA;
   return TP_OK;
 }

@@ -83,7 +83,37 @@ extern const int kRegistrySize;
 // CSR helpers (csr.cu)
 cudaError_t launch_csr_validate(int N, int E, const int32_t* rowptr, const int32_t* src, int* err,
                                 cudaStream_t s);
+
+// The transpose is a radix sort of edge ids keyed by sender (keys 0..N, N = invalid sender):
+// tiles of kRadixTile edges, passes of at most kRadixMaxBits-bit digits.
+constexpr int kRadixItems = 8;                         // items per thread of a tile
+constexpr int kRadixTile = 256 * kRadixItems;          // 2,048 edges per CTA
+constexpr int kRadixMaxBits = 11;
+constexpr int kRadixMaxDigits = 1 << kRadixMaxBits;
+
+struct RadixPlan {
+  int passes, bits, radix;   // passes of `bits`-bit digits, radix = 2^bits buckets
+  int64_t tiles;
+};
+
+constexpr RadixPlan radix_plan(int64_t N, int64_t E) {
+  int key_bits = 1;                                    // keys lie in [0, N]
+  while (key_bits < 32 && ((int64_t)1 << key_bits) <= N) ++key_bits;
+  const int passes = (key_bits + kRadixMaxBits - 1) / kRadixMaxBits;
+  const int bits = (key_bits + passes - 1) / passes;
+  return RadixPlan{passes, bits, 1 << bits, (E + kRadixTile - 1) / kRadixTile};
+}
+
+// int32 scratch of one transpose: a second id buffer when there is more than one pass, and
+// the per-digit, per-tile counts followed by the digit totals.
+constexpr int64_t transpose_scratch_ints(int64_t N, int64_t E) {
+  const RadixPlan p = radix_plan(N, E);
+  return (p.passes > 1 ? E : 0) + (int64_t)p.radix * (p.tiles + 1);
+}
+
+// colptr[N+1] and perm[E] of the stable receiver->sender transpose; scratch holds
+// transpose_scratch_ints(N, E) int32.
 cudaError_t launch_csr_transpose(int N, int E, const int32_t* src, int32_t* colptr, int32_t* perm,
-                                 int32_t* counts, int32_t* tmp, cudaStream_t s);
+                                 int32_t* scratch, cudaStream_t s);
 
 }  // namespace tp

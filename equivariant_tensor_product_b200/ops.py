@@ -15,7 +15,7 @@ import torch
 from . import _lib
 from ._lib import TP_MODE_UVU, TP_MODE_UVW, TP_OP_BWD, TP_OP_DBWD, TP_OP_FWD, check, load
 
-__all__ = ["Plan", "tp_plan_create", "tp_plan_query", "tp_workspace_size", "tp_csr_transpose",
+__all__ = ["Plan", "tp_plan_create", "tp_plan_query", "tp_workspace_size", "tp_csr_transpose_workspace_size", "tp_csr_transpose",
            "tp_conv_fwd", "tp_conv_bwd", "tp_conv_dbwd", "tp_get_device_error", "tp_version"]
 
 
@@ -95,15 +95,21 @@ def _workspace(plan, N, E, op, ws, device):
     return ws
 
 
+def tp_csr_transpose_workspace_size(N: int, E: int) -> int:
+    out = C.c_size_t()
+    check(load().tp_csr_transpose_workspace_size(int(N), int(E), C.byref(out)), "tp_csr_transpose_workspace_size")
+    return out.value
+
+
 def tp_csr_transpose(rowptr: Optional[torch.Tensor], src: torch.Tensor, N: int, colptr=None, perm=None,
                      ws=None, stream=None):
     E = src.numel()
     dev = src.device
     colptr = torch.empty(N + 1, dtype=torch.int32, device=dev) if colptr is None else colptr
     perm = torch.empty(E, dtype=torch.int32, device=dev) if perm is None else perm
-    need = 256 + 4 * (N + 1) + 4 * max(N, 1) + 8 * max(E, 1) + 4 * 256
+    need = tp_csr_transpose_workspace_size(N, E)
     if ws is None:
-        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     st = load().tp_csr_transpose(N, E, _ptr(rowptr, torch.int32, "rowptr"), _ptr(src, torch.int32, "src"),
                                  _ptr(colptr, torch.int32, "colptr"), _ptr(perm, torch.int32, "perm"),
                                  _ptr(ws), ws.numel(), _stream(stream))

@@ -105,14 +105,25 @@ tp_status_t tp_plan_query(tp_plan_t plan, int64_t* in_dim, int64_t* out_dim,
 
 /* Bytes of device workspace a call of kind op (TP_OP_*) needs for N nodes and E edges:
  * forward 0 (256 with TP_FLAG_CHECK_INDICES, for the error word); backward and double
- * backward 256 + int32 colptr[N+1], counts[N], perm[E], tmp[E] (room to build the
- * transpose in place; only the 256-byte header is used when colptr/perm are given).
- * The workspace never holds an edge x feature float tensor. */
+ * backward 256 + int32 colptr[N+1] + perm[E] + the transpose's scratch
+ * (tp_csr_transpose_workspace_size), room to build the transpose in place; only the
+ * 256-byte header is used when colptr/perm are given.  uvw adds node- and weight-sized
+ * float regions.  The workspace never holds an edge x feature float tensor. */
 tp_status_t tp_workspace_size(tp_plan_t plan, int64_t N, int64_t E, int32_t op, size_t* bytes);
 
-/* Stable receiver->sender transpose: colptr[N+1] = exclusive scan of bincount(src),
- * perm[E] = stable argsort of src (bit exact).  rowptr may be NULL.  Workspace: at least
- * tp_workspace_size(., N, E, TP_OP_BWD) bytes or 4*(N+E)+256. */
+/* Bytes of scratch tp_csr_transpose needs for N nodes and E edges. */
+tp_status_t tp_csr_transpose_workspace_size(int64_t N, int64_t E, size_t* bytes);
+
+/* Stable receiver->sender transpose (the sender order of the backward passes):
+ * colptr[N+1] = exclusive scan of bincount(src), perm[E] = stable argsort of src (bit
+ * exact), computed as a radix sort of the edge ids keyed by sender: O(E) work per pass and
+ * ceil(log2(N+1) / 11) passes, whatever the degree distribution.  rowptr may be NULL.
+ * Senders should lie in [0, N); an edge whose sender does not is placed after all valid
+ * edges (perm[colptr[N]..E) lists those edges in increasing order) and colptr[N] counts the
+ * valid edges.  Workspace: ws 4-byte aligned, ws_bytes >= tp_csr_transpose_workspace_size
+ * (int32 scratch: an id buffer of E when more than one pass is needed, plus per-tile digit
+ * counts, about 4 bytes per edge at most).  TP_ERR_INVALID_ARG for null or misaligned
+ * pointers or sizes outside [0, 2^31), TP_ERR_WORKSPACE for a short workspace. */
 tp_status_t tp_csr_transpose(int64_t N, int64_t E, const int32_t* rowptr, const int32_t* src,
                              int32_t* colptr, int32_t* perm, void* ws, size_t ws_bytes,
                              tp_stream_t stream);
@@ -121,15 +132,18 @@ tp_status_t tp_csr_transpose(int64_t N, int64_t E, const int32_t* rowptr, const 
  * memory -- e.g. an MD engine whose device memory is owned by a pool it does not control,
  * a framework that has reserved nearly all of the GPU up front, or a loop that must avoid
  * cudaMalloc/cudaFree because they synchronise the device.  It takes no workspace: its
- * scratch (per-sender counters and the scatter buffer) is a fixed int32 array inside the
- * library (about 4.5 MB, held on every GPU that loads the library until exit).  The source
- * pages have no counterpart; this is an interface convenience.
+ * scratch (the radix sort's second id buffer and digit counts) is a fixed int32 array
+ * inside the library (about 5.3 MB, held on every GPU that loads the library until exit).
+ * The source pages have no counterpart; this is an interface convenience.
  *   Limits: N <= 131072 and E <= 1048576, else TP_ERR_UNSUPPORTED with nothing enqueued.
+ *   Senders outside [0, N) are handled as by tp_csr_transpose (placed last, not counted).
  *   Calls share the array: calls whose work overlaps on the GPU race; order them on one
- *   stream.  Counters are cleared at the start of every call.  The first call on a device
- *   looks up the array's device address with that device current: make it before any
- *   stream capture.  Other errors: TP_ERR_INVALID_ARG (null, misaligned, negative sizes),
- *   TP_ERR_CUDA.  No message is set for tp_last_error_message. */
+ *   stream.  Every call writes the parts of the array it reads before reading them.  The
+ *   first call on a device looks up the array's device address with that device current:
+ *   make it before any stream capture.  The address is kept for the life of the process, so
+ *   a cudaDeviceReset between calls is not supported.  Other errors: TP_ERR_INVALID_ARG
+ *   (null, misaligned, negative sizes), TP_ERR_CUDA.  No message is set for
+ *   tp_last_error_message. */
 tp_status_t tp_csr_transpose_noalloc(int64_t N, int64_t E, const int32_t* rowptr,
                                      const int32_t* src, int32_t* colptr, int32_t* perm,
                                      tp_stream_t stream);

@@ -97,8 +97,20 @@ def test_workspace_contract(tp):
     assert tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD) == 0
     for op in (tp.TP_OP_BWD, tp.TP_OP_DBWD):
         b = tp.tp_workspace_size(plan, N, E, op)
-        # int32 graph indices only: at most 8 bytes per edge + O(N) + alignment
-        assert 8 * E <= b <= 8 * E + 8 * (N + 1) + 6 * 256
+        # int32 graph indices only: perm, the radix sort's id buffer and its digit counts
+        # (at most 4 bytes per edge plus one 2,048-entry row), colptr, alignment
+        assert 8 * E <= b <= 12 * E + 4 * (N + 1) + 4 * 2 * 2048 + 6 * 256
+
+
+def test_transpose_workspace_is_int_sized(tp):
+    # one 11-bit pass up to 2,047 nodes (no second id buffer), then two passes
+    assert tp.tp_csr_transpose_workspace_size(1536, 46080) == 4 * 2048 * (23 + 1)
+    assert tp.tp_csr_transpose_workspace_size(100_000, 3_001_138) == 4 * (3_001_138 + 512 * (1466 + 1))
+    assert tp.tp_csr_transpose_workspace_size(0, 0) == 4 * 2
+    for N, E in ((24, 192), (4096, 162_892), (8192, 294_643), (2**31 - 1, 2**31 - 1)):
+        assert tp.tp_csr_transpose_workspace_size(N, E) <= 8 * E + 4 * 2 * 2048
+    with pytest.raises(tp.TPError):
+        tp.tp_csr_transpose_workspace_size(-1, 4)
 
 
 def test_uvw_rejects_multiplicities_off_the_tma_pitch(tp):
@@ -121,10 +133,10 @@ def test_uvw_workspace_is_node_sized(tp):
     b = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD)
     # fwd: A and W regrouped for the GEMM (TF32 hi and lo)
     assert a_bytes <= f <= a_bytes + 2 * 4 * plan.n_shared_weights + 4096
-    # bwd: transpose ints (8 bytes/edge + O(N)), A, G, x as K-contiguous rows, W regrouped
-    # twice (hi and lo each), 64 split-K partials of gW
+    # bwd: transpose ints (at most 12 bytes/edge + O(N)), A, G, x as K-contiguous rows, W
+    # regrouped twice (hi and lo each), at most 64 split-K partials of gW
     x_bytes = 4 * N * plan.in_dim
-    assert b <= 8 * E + 12 * (N + 1) + 2 * a_bytes + x_bytes + 68 * 4 * plan.n_shared_weights + 16 * 256
+    assert b <= 12 * E + 12 * (N + 1) + 2 * a_bytes + x_bytes + 68 * 4 * plan.n_shared_weights + 16 * 2048
     with pytest.raises(tp.TPError):
         tp.tp_workspace_size(plan, N, E, tp.TP_OP_DBWD)
 

@@ -192,6 +192,64 @@ def test_transpose_adversarial(tp):
     _check_transpose(tp, rowptr, src, N)
     # no edges at all
     _check_transpose(tp, np.zeros(6, np.int32), np.zeros(0, np.int32), 5)
+    # no nodes, no edges
+    _check_transpose(tp, np.zeros(1, np.int32), np.zeros(0, np.int32), 0)
+    # a ragged last tile, node counts at the one-pass / two-pass boundary of the digit width
+    for N in (2047, 2048, 4095):
+        E = 2048 * 3 + 17
+        src = rng.integers(0, N, E).astype(np.int32)
+        rowptr = np.concatenate([[0], np.cumsum(np.bincount(rng.integers(0, N, E), minlength=N))]).astype(np.int32)
+        _check_transpose(tp, rowptr, src, N)
+    # many nodes and few edges: long runs of senders without edges in colptr
+    N, E = 300_000, 64
+    src = rng.integers(0, N, E).astype(np.int32)
+    src[:8] = N - 1
+    rowptr = np.concatenate([[0], np.cumsum(np.bincount(rng.integers(0, N, E), minlength=N))]).astype(np.int32)
+    _check_transpose(tp, rowptr, src, N)
+
+
+def test_transpose_hub_sender_is_linear_time(tp):
+    """One sender with 1.2M out-edges among 1.25M: a radix sort does O(E) work whatever the
+    degree distribution; the call takes well under 1 ms on a B200."""
+    rng = np.random.default_rng(11)
+    N, E = 2000, 1_250_000
+    src = rng.integers(0, N, E).astype(np.int32)
+    src[rng.random(E) < 0.96] = 1234
+    assert (src == 1234).sum() >= 1_000_000
+    rowptr = np.concatenate([[0], np.cumsum(np.bincount(rng.integers(0, N, E), minlength=N))]).astype(np.int32)
+    _check_transpose(tp, rowptr, src, N)
+    r, s_ = dev(rowptr), dev(src)
+    colptr = torch.empty(N + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(E, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tp.tp_csr_transpose_workspace_size(N, E), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        tp.tp_csr_transpose(r, s_, N, colptr=colptr, perm=perm, ws=ws)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(10):
+        tp.tp_csr_transpose(r, s_, N, colptr=colptr, perm=perm, ws=ws)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / 10
+    assert ms < 1.0, f"transpose of a 1.2M-edge hub took {ms:.3f} ms"
+
+
+def test_transpose_senders_out_of_range_go_last(tp):
+    """Edges whose sender lies outside [0, N) are not counted in colptr and follow every valid
+    edge in perm, in increasing edge order."""
+    rng = np.random.default_rng(5)
+    N, E = 700, 9000
+    src = rng.integers(0, N, E).astype(np.int32)
+    bad = rng.random(E) < 0.05
+    src[bad] = rng.choice(np.array([-1, -5, N, N + 3, 2**31 - 1], np.int32), bad.sum())
+    rowptr = np.concatenate([[0], np.cumsum(np.bincount(rng.integers(0, N, E), minlength=N))]).astype(np.int32)
+    colptr, perm = tp.tp_csr_transpose(dev(rowptr), dev(src), N)
+    valid = ~bad
+    key = np.where(valid, src, N)
+    np.testing.assert_array_equal(perm.cpu().numpy(), np.argsort(key, kind="stable"))
+    ref_col = np.concatenate([[0], np.cumsum(np.bincount(src[valid], minlength=N))])
+    np.testing.assert_array_equal(colptr.cpu().numpy(), ref_col)
+    assert colptr[-1].item() == int(valid.sum())
 
 
 # ------------------------------------------------------------------------------------------

@@ -45,6 +45,24 @@ def test_c4_replica_forward_backward_complete(tp):
     assert_close(gW.view(r["gW"].shape), r["gW"], "c4 replica gW")
 
 
+def test_c4_replica_gW_through_promoted_accumulation(tp):
+    """gW element by element against the float64 oracle at a size where every split-K partial
+    of the gW GEMM reduces more than 16 K blocks of 32 rows for every input irrep, so the
+    fp32 promotion of the tensor-core accumulator runs inside each split, as it does at full
+    size (3,000 atoms: 2 splits of 1,500 * d1 rows, i.e. 47 to 235 K blocks each)."""
+    d = inputs("c4", 3000)
+    N = len(d["rowptr"]) - 1
+    splits = min(64, max(1, (N + 1535) // 1536))
+    assert splits >= 2 and (N // splits) // 32 > 16
+    plan, op = plans(d["spec"], tp)
+    g = device_inputs(d)
+    gx, gs, _, gW = _bwd(tp, plan, g, gvec=False)
+    r = backward(op, d["rowptr"], d["src"], d["x"], d["vec"], d["gy"], s=d["s"], W=d["W"])
+    assert_close(gW.view(r["gW"].shape), r["gW"], "c4 3,000-atom gW")
+    assert_close(gx, r["gx"], "c4 3,000-atom gx")
+    assert_close(gs, r["gs"], "c4 3,000-atom gs")
+
+
 def test_c4_full_size_sampled_and_adjoint(tp):
     d = inputs("c4")
     plan, op = plans(d["spec"], tp)

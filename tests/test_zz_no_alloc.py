@@ -69,6 +69,29 @@ def test_noalloc_matches_workspace_transpose_twice_in_a_row(lib):
     torch.cuda.synchronize()
 
 
+def test_noalloc_at_its_limits_and_when_empty(lib):
+    """The largest accepted graph (N = 131,072, E = 1,048,576: the last sender's counter and
+    the last slot of every scratch region in use), then graphs without edges or nodes, then a
+    small graph again, each against tp_csr_transpose and a stable numpy argsort."""
+    rng = np.random.default_rng(9)
+    N, E = 1 << 17, 1 << 20
+    src = rng.integers(0, N, E).astype(np.int32)
+    src[-4096:] = N - 1
+    rowptr = np.concatenate([[0], np.cumsum(np.bincount(rng.integers(0, N, E), minlength=N))]).astype(np.int32)
+    cases = [(rowptr, src, N),
+             (np.zeros(11, np.int32), np.zeros(0, np.int32), 10),
+             (np.zeros(1, np.int32), np.zeros(0, np.int32), 0),
+             _graph(4, 500, 12, 499) + (500,)]
+    for rowptr, src, n in cases:
+        got = _noalloc(lib, rowptr, src, n)
+        want = _existing(rowptr, src, n)
+        np.testing.assert_array_equal(got[0], want[0])
+        np.testing.assert_array_equal(got[1], want[1])
+        np.testing.assert_array_equal(got[1], np.argsort(src, kind="stable"))
+        np.testing.assert_array_equal(got[0], np.concatenate([[0], np.cumsum(np.bincount(src, minlength=n))]))
+    torch.cuda.synchronize()
+
+
 def test_noalloc_rejects_graphs_beyond_its_array(lib):
     fake = C.c_void_p(0x10000)   # never touched: the size check comes first
     assert lib.tp_csr_transpose_noalloc(1 << 17 | 1, 10, fake, fake, fake, fake, None) == 2
