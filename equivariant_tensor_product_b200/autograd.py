@@ -1,10 +1,13 @@
 """torch.autograd wrapper: forward -> tp_conv_fwd, backward -> tp_conv_bwd, and the backward's
 own backward -> tp_conv_dbwd, so force training (a loss on d(energy)/d(positions)) can
-differentiate twice through the convolution.  Marshalling only (see ops.py)."""
+differentiate twice through the convolution (uvu; uvw mode differentiates once, to x, the
+edge vectors, the per-edge scalars and the shared mixing weights W).  Marshalling only (see
+ops.py)."""
 from __future__ import annotations
 
 import torch
 
+from ._lib import TP_MODE_UVW
 from .ops import Plan, tp_conv_bwd, tp_conv_dbwd, tp_conv_fwd, tp_csr_transpose
 
 
@@ -26,45 +29,53 @@ class Graph:
 
 class _Bwd(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, x, vec, w, gy, plan, graph, needs):
+    def forward(ctx, x, vec, w, W, gy, plan, graph, needs):
         colptr, perm = graph.transpose()
-        gx, gw, gvec, _ = tp_conv_bwd(plan, graph.rowptr, graph.src, x, vec, w, gy, colptr=colptr, perm=perm,
-                                      need_gx=needs[0], need_gvec=needs[1], need_gw=needs[2])
+        gx, gw, gvec, gW = tp_conv_bwd(plan, graph.rowptr, graph.src, x, vec, w, gy, W=W, colptr=colptr, perm=perm,
+                                       need_gx=needs[0], need_gvec=needs[1], need_gw=needs[2],
+                                       need_gW=W is not None and needs[3])
         ctx.save_for_backward(x, vec, w, gy)
         ctx.plan, ctx.graph = plan, graph
-        return gx, gvec, gw
+        return gx, gvec, gw, gW
 
     @staticmethod
-    def backward(ctx, ggx, ggvec, ggw):
+    def backward(ctx, ggx, ggvec, ggw, ggW):
+        if ctx.plan.mode == TP_MODE_UVW:
+            raise RuntimeError("second derivatives of the uvw convolution are not implemented (tp_conv_dbwd is uvu)")
         x, vec, w, gy = ctx.saved_tensors
         colptr, perm = ctx.graph.transpose()
         c = lambda t: None if t is None else t.contiguous()
-        need = tuple(n for n, k in zip(("g_x", "g_vec", "g_w", "g_gy"), range(4)) if ctx.needs_input_grad[k])
+        need = tuple(n for n, k in zip(("g_x", "g_vec", "g_w", "g_gy"), (0, 1, 2, 4)) if ctx.needs_input_grad[k])
         g_gy, g_x, g_w, g_vec = tp_conv_dbwd(ctx.plan, ctx.graph.rowptr, ctx.graph.src, x, vec, w, gy,
                                              ggx=c(ggx), ggw=c(ggw), ggvec=c(ggvec), colptr=colptr, perm=perm,
                                              need=need)
-        return g_x, g_vec, g_w, g_gy, None, None, None
+        return g_x, g_vec, g_w, None, g_gy, None, None, None
 
 
 class TPConv(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, x, vec, w, plan, graph):
-        y = tp_conv_fwd(plan, graph.rowptr, graph.src, x.contiguous(), vec.contiguous(), w.contiguous())
-        ctx.save_for_backward(x, vec, w)
+    def forward(ctx, x, vec, w, W, plan, graph):
+        W = None if W is None else W.contiguous()
+        y = tp_conv_fwd(plan, graph.rowptr, graph.src, x.contiguous(), vec.contiguous(), w.contiguous(), W=W)
+        ctx.save_for_backward(x, vec, w, W)
         ctx.plan, ctx.graph = plan, graph
         return y
 
     @staticmethod
     def backward(ctx, gy):
-        x, vec, w = ctx.saved_tensors
-        needs = (ctx.needs_input_grad[0], ctx.needs_input_grad[1], ctx.needs_input_grad[2])
-        gx, gvec, gw = _Bwd.apply(x, vec, w, gy.contiguous(), ctx.plan, ctx.graph, needs)
-        return gx, gvec, gw, None, None
+        x, vec, w, W = ctx.saved_tensors
+        n = ctx.needs_input_grad
+        gx, gvec, gw, gW = _Bwd.apply(x, vec, w, W, gy.contiguous(), ctx.plan, ctx.graph, (n[0], n[1], n[2], n[3]))
+        return gx, gvec, gw, gW, None, None
 
 
-def tp_conv(plan: Plan, graph: Graph, x, vec, w):
-    """y = conv(x, vec, w) with first and second derivatives through the CUDA kernels (uvu)."""
-    return TPConv.apply(x, vec, w, plan, graph)
+def tp_conv(plan: Plan, graph: Graph, x, vec, w, W=None):
+    """y = conv(x, vec, w) with derivatives through the CUDA kernels: first and second order in
+    uvu mode (w = per-edge weights [E, n_edge_weights]); first order in uvw mode (w = per-edge
+    path scalars s [E, P], W = shared mixing weights [P, mul_in, mul_out], gradients to both)."""
+    if (plan.mode == TP_MODE_UVW) != (W is not None):
+        raise ValueError("W is required in uvw mode and must be None in uvu mode")
+    return TPConv.apply(x, vec, w, W, plan, graph)
 
 
 # ---------------------------------------------------------------------------------------------

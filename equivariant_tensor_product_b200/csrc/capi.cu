@@ -21,7 +21,8 @@ struct IrrepBlock {
 };
 
 struct tp_plan_s {
-  const SpecOps* ops;
+  const SpecOps* ops;   // compiled specialisation, or NULL: runtime path table `gen`
+  GenTable* gen;
   int mode;
   int mul_in, mul_out;
   int64_t in_dim, out_dim, nw, n_shared;
@@ -235,6 +236,83 @@ tp_status_t debug_prologue(tp_plan_t plan, int64_t N, int64_t E, const int32_t* 
   return TP_OK;
 }
 
+// The runtime path table of a plan without a compiled specialisation: block offsets, paths
+// per block and the (block, 32-channel slice) tasks of the receiver and sender passes.
+bool build_gen_table(const std::vector<IrrepBlock>& bi, const std::vector<IrrepBlock>& bs,
+                     const std::vector<IrrepBlock>& bo, const int32_t* paths, int n_paths, const double* coeff,
+                     GenTable& T, std::string& why) {
+  std::memset(&T, 0, sizeof(T));
+  T.n_paths = n_paths;
+  T.n_in = (int)bi.size();
+  T.n_out = (int)bo.size();
+  int off = 0;
+  for (int k = 0; k < T.n_in; ++k) {
+    T.in_off[k] = off;
+    T.in_mul[k] = bi[k].mul;
+    T.in_l[k] = bi[k].l;
+    off += bi[k].mul * (2 * bi[k].l + 1);
+  }
+  off = 0;
+  for (int k = 0; k < T.n_out; ++k) {
+    T.out_off[k] = off;
+    T.out_mul[k] = bo[k].mul;
+    T.out_l[k] = bo[k].l;
+    off += bo[k].mul * (2 * bo[k].l + 1);
+  }
+  int w_off = 0;
+  for (int p = 0; p < n_paths; ++p) {
+    const int a = paths[3 * p], b = paths[3 * p + 1], o = paths[3 * p + 2];
+    GenPath& P = T.path[p];
+    P.l1 = (int16_t)bi[a].l;
+    P.l2 = (int16_t)bs[b].l;
+    P.l3 = (int16_t)bo[o].l;
+    P.tid = (int16_t)gen_triple_id(bi[a].l, bs[b].l, bo[o].l);
+    if (P.tid < 0) {
+      why = "path outside the generated triples";
+      return false;
+    }
+    P.in_off = T.in_off[a];
+    P.out_off = T.out_off[o];
+    P.mul = bi[a].mul;
+    P.w_off = w_off;
+    P.in_block = a;
+    P.out_block = o;
+    P.coeff = coeff ? (float)coeff[p] : 1.0f;
+    w_off += bi[a].mul;
+    T.lmax_sh = std::max(T.lmax_sh, bs[b].l);
+  }
+  int q = 0;
+  for (int o = 0; o < T.n_out; ++o) {
+    T.out_first[o] = q;
+    for (int p = 0; p < n_paths; ++p)
+      if (paths[3 * p + 2] == o) T.out_paths[q++] = p;
+  }
+  T.out_first[T.n_out] = q;
+  q = 0;
+  for (int a = 0; a < T.n_in; ++a) {
+    T.in_first[a] = q;
+    for (int p = 0; p < n_paths; ++p)
+      if (paths[3 * p] == a) T.in_paths[q++] = p;
+  }
+  T.in_first[T.n_in] = q;
+  for (int pass = 0; pass < 2; ++pass) {
+    const auto& blocks = pass == 0 ? bo : bi;
+    int n = 0;
+    for (int k = 0; k < (int)blocks.size(); ++k)
+      for (int sl = 0; sl < (blocks[k].mul + 31) / 32; ++sl) {
+        if (n >= kGenMaxTasks || sl > 255) {
+          why = "too many 32-channel slices for the runtime path table (at most 256 over all blocks)";
+          return false;
+        }
+        (pass == 0 ? T.rtask_block : T.stask_block)[n] = (uint8_t)k;
+        (pass == 0 ? T.rtask_slice : T.stask_slice)[n] = (uint8_t)sl;
+        ++n;
+      }
+    (pass == 0 ? T.n_rtask : T.n_stask) = n;
+  }
+  return true;
+}
+
 }  // namespace
 
 namespace tp {
@@ -310,14 +388,19 @@ tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* i
     if (mode == TP_MODE_UVU && bi[a].mul != bo[o].mul)
       return fail(TP_ERR_INVALID_ARG, "path %d: uvu needs equal input and output multiplicity", p);
   }
-  const int mul_in = bi[0].mul, mul_out = bo[0].mul;
-  for (auto& b : bi)
-    if (b.mul != mul_in) return fail(TP_ERR_UNSUPPORTED, "input blocks must share one multiplicity");
-  for (auto& b : bo)
-    if (b.mul != mul_out) return fail(TP_ERR_UNSUPPORTED, "output blocks must share one multiplicity");
-  // find the compiled specialisation
+  int mul_in = 0, mul_out = 0;
+  bool uniform = true;
+  for (auto& b : bi) {
+    uniform = uniform && b.mul == bi[0].mul;
+    mul_in = std::max(mul_in, b.mul);
+  }
+  for (auto& b : bo) {
+    uniform = uniform && b.mul == bo[0].mul;
+    mul_out = std::max(mul_out, b.mul);
+  }
+  // the compiled specialisation of this irreps / path list, if the build ships one
   const SpecOps* found = nullptr;
-  for (int r = 0; r < kRegistrySize && !found; ++r) {
+  for (int r = 0; r < kRegistrySize && !found && uniform; ++r) {
     const SpecOps* s = kRegistry[r];
     if (s->n_in != (int)bi.size() || s->n_sh != (int)bs.size() || s->n_out != (int)bo.size() ||
         s->n_paths != n_paths)
@@ -331,20 +414,31 @@ tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* i
            s->paths[p][2] == paths[3 * p + 2];
     if (ok) found = s;
   }
-  if (!found)
+  if (mode == TP_MODE_UVW && !found)
     return fail(TP_ERR_UNSUPPORTED,
-                "no compiled specialisation for this irreps/path list (shipped: all-paths lmax 1/2/3 "
-                "and the 4-path lmax-1 list)");
+                "uvw runs on the compiled path lists (all paths of lmax 1, 2 or 3, uniform multiplicity); "
+                "uvu takes any path list");
   if (mode == TP_MODE_UVW && (!found->uvw_fwd || !found->uvw_bwd))
     return fail(TP_ERR_UNSUPPORTED, "spec '%s' has no uvw kernels", found->name);
   // the uvw GEMMs load their operands by TMA, whose row pitches are multiples of 16 bytes
   if (mode == TP_MODE_UVW && (mul_in % 4 != 0 || mul_out % 4 != 0))
     return fail(TP_ERR_UNSUPPORTED, "uvw needs multiplicities that are multiples of 4 (got %d, %d)", mul_in,
                 mul_out);
+  GenTable* gen = nullptr;
+  if (!found) {
+    gen = new (std::nothrow) GenTable;
+    if (!gen) return fail(TP_ERR_INVALID_ARG, "out of host memory");
+    std::string why2;
+    if (!build_gen_table(bi, bs, bo, paths, n_paths, path_coeff, *gen, why2)) {
+      delete gen;
+      return fail(TP_ERR_UNSUPPORTED, "%s", why2.c_str());
+    }
+  }
   tp_plan_s* pl = new (std::nothrow) tp_plan_s;
   if (!pl) return fail(TP_ERR_INVALID_ARG, "out of host memory");
   std::memset(pl, 0, sizeof(*pl));
   pl->ops = found;
+  pl->gen = gen;
   pl->mode = mode;
   pl->mul_in = mul_in;
   pl->mul_out = mul_out;
@@ -354,13 +448,16 @@ tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* i
   pl->in_dim = in_dim;
   pl->out_dim = out_dim;
   pl->n_paths = n_paths;
-  pl->nw = mode == TP_MODE_UVU ? (int64_t)n_paths * mul_in : n_paths;
+  int64_t nw = 0;
+  for (int p = 0; p < n_paths; ++p) nw += bi[paths[3 * p]].mul;
+  pl->nw = mode == TP_MODE_UVU ? nw : n_paths;
   pl->n_shared = mode == TP_MODE_UVW ? (int64_t)n_paths * mul_in * mul_out : 0;
   pl->has_coeff = 0;
   for (int p = 0; p < kMaxPaths; ++p) pl->coeff[p] = 1.0f;
   if (path_coeff) {
     for (int p = 0; p < n_paths; ++p) {
       if (!std::isfinite(path_coeff[p])) {
+        delete pl->gen;
         delete pl;
         return fail(TP_ERR_INVALID_ARG, "path_coeff[%d] is not finite", p);
       }
@@ -374,6 +471,7 @@ tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* i
 }
 
 tp_status_t tp_plan_destroy(tp_plan_t plan) {
+  if (plan) delete plan->gen;
   delete plan;
   return TP_OK;
 }
@@ -465,6 +563,8 @@ tp_status_t tp_conv_fwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* row
     a.Wt = reinterpret_cast<float*>(wsb + U.Wt);
     a.nw = plan->n_paths;
     e = plan->ops->uvw_fwd(a, s);
+  } else if (plan->gen) {
+    e = launch_gen_fwd(a, *plan->gen, s);
   } else {
     e = plan->ops->fwd_uvu(a, s);
   }
@@ -547,6 +647,11 @@ tp_status_t tp_conv_bwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* row
     if (e != cudaSuccess) return cuda_fail(e, "tp_conv_bwd (uvw) launch");
     return TP_OK;
   }
+  if (plan->gen) {
+    cudaError_t e = launch_gen_bwd(a, *plan->gen, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tp_conv_bwd launch");
+    return TP_OK;
+  }
   if (gvec) {
     const int nsl = a.n_slices <= 1 ? 1 : (a.n_slices == 2 ? 2 : 4);
     while (a.split * nsl > 4) a.split >>= 1;
@@ -588,7 +693,7 @@ tp_status_t tp_conv_dbwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* ro
   a.ggvec = ggvec;
   if (g_gy) {
     a.y = g_gy;
-    cudaError_t e = plan->ops->dbwd_recv(a, s);
+    cudaError_t e = plan->gen ? launch_gen_dbwd(a, *plan->gen, true, false, s) : plan->ops->dbwd_recv(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "tp_conv_dbwd receiver pass");
   }
   if (!g_x && !g_w && !g_vec) return TP_OK;
@@ -599,6 +704,11 @@ tp_status_t tp_conv_dbwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* ro
   a.gx = g_x;
   a.gw = g_w;
   a.gvec = g_vec;
+  if (plan->gen) {
+    cudaError_t e = launch_gen_dbwd(a, *plan->gen, false, true, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tp_conv_dbwd sender pass");
+    return TP_OK;
+  }
   if (g_vec) {
     const int nsl = a.n_slices <= 1 ? 1 : (a.n_slices == 2 ? 2 : 4);
     while (a.split * nsl > 4) a.split >>= 1;

@@ -838,6 +838,113 @@ def gen_spec_header(spec: Spec) -> str:
 
 
 # ---------------------------------------------------------------------------
+# Runtime path table: one set of contractions per (l1, l2, l3) triple
+# ---------------------------------------------------------------------------
+
+def all_triples():
+    """Every (l1, l2, l3) with l <= 3 that satisfies the triangle rule, lexicographic (34)."""
+    return [(a, b, c) for a in range(4) for b in range(4) for c in range(4) if abs(a - b) <= c <= a + b]
+
+
+def _gen_triple(l1, l2, l3) -> List[str]:
+    """fwd: t[m3] = sum C x[m1] Y[m2];  tx: z[m1] = sum C Y[m2] g[m3];  ty: q[m2] = sum C x[m1] g[m3]."""
+    nz = cg_nonzeros(l1, l2, l3)
+    d1, d2, d3 = 2 * l1 + 1, 2 * l2 + 1, 2 * l3 + 1
+    L = [f"template <> struct Cg<{l1}, {l2}, {l3}> {{",
+         f"  static constexpr int L1 = {l1}, L2 = {l2}, L3 = {l3}, D1 = {d1}, D2 = {d2}, D3 = {d3}, NNZ = {len(nz)};"]
+
+    def body(name, a, an, b, bn, out, on, key_pair, key_out):
+        L.append(f"  __device__ __forceinline__ static void {name}(const float (&{a})[{an}], const float (&{b})[{bn}], "
+                 f"float (&{out})[{on}]) {{")
+        used = sorted({key_pair(i, j, k) for i, j, k, c in nz})
+        for (u, v) in used:
+            # products with Y_0 (= 1) need no multiply
+            if name == "fwd":
+                e = f"{a}[{u}]" if l2 == 0 else f"{a}[{u}] * {b}[{v}]"
+            elif name == "tx":
+                e = f"{b}[{v}]" if l2 == 0 else f"{a}[{u}] * {b}[{v}]"
+            else:
+                e = f"{a}[{u}] * {b}[{v}]"
+            L.append(f"    const float p{u}_{v} = {e};")
+        for m in range(on):
+            terms = [(c, "p%d_%d" % key_pair(i, j, k)) for (i, j, k, c) in nz if key_out(i, j, k) == m]
+            L.extend(line.replace("      ", "    ", 1) for line in _chain(terms, f"{out}[{m}]", decl=False))
+        L.append("  }")
+
+    body("fwd", "x", d1, "Y", d2, "t", d3, lambda i, j, k: (i, j), lambda i, j, k: k)
+    body("tx", "Y", d2, "g", d3, "z", d1, lambda i, j, k: (j, k), lambda i, j, k: i)
+    body("ty", "x", d1, "g", d3, "q", d2, lambda i, j, k: (i, k), lambda i, j, k: j)
+    L.append("};")
+    return L
+
+
+def _gen_sh_block(l) -> List[str]:
+    """Real SH of one degree l as Cartesian polynomials of r_hat, their gradient and the Hessian
+    applied to a direction d (for the double backward)."""
+    polys = sh_polys()[l]
+    d = 2 * l + 1
+    L = [f"template <> struct ShBlock<{l}> {{", f"  static constexpr int L = {l}, D = {d};",
+         f"  __device__ __forceinline__ static void sh(float rx, float ry, float rz, float (&Y)[{d}]) {{"]
+    L += _monomials_code(max(l, 1))
+    L.append("    (void)rx; (void)ry; (void)rz;")
+    for m in range(d):
+        L.append(f"    Y[{m}] = {_poly_expr(polys[m])};")
+    L.append("  }")
+    L.append(f"  __device__ __forceinline__ static void grad(float rx, float ry, float rz, float (&G)[{d}][3]) {{")
+    L += _monomials_code(max(l - 1, 1))
+    L.append("    (void)rx; (void)ry; (void)rz;")
+    for m in range(d):
+        for ax in range(3):
+            L.append(f"    G[{m}][{ax}] = {_poly_expr(dpoly(polys[m], ax))};")
+    L.append("  }")
+    L.append("};")
+    return L
+
+
+def gen_generic_header() -> str:
+    tr = all_triples()
+    L = ["// Generated by codegen.py.  Do not edit.",
+         "// Contractions of the real Clebsch-Gordan tensor of every (l1, l2, l3) triple with l <= 3 (non-zero",
+         "// entries only, unrolled), for the runtime path table of plans without a compiled specialisation,",
+         "// and the real spherical harmonics of each degree, all degrees at once (ShAll) with gradients and",
+         "// Hessian-direction products.",
+         "#pragma once",
+         "namespace tp {",
+         "namespace gen {",
+         f"constexpr int kNumTriples = {len(tr)};",
+         "template <int L1, int L2, int L3> struct Cg;"]
+    for t in tr:
+        L += _gen_triple(*t)
+    ids = [-1] * 64
+    for k, (a, b, c) in enumerate(tr):
+        ids[a * 16 + b * 4 + c] = k
+    L.append("__host__ __device__ inline int triple_id(int l1, int l2, int l3) {")
+    L.append(f"  constexpr int v[64] = {{{', '.join(map(str, ids))}}};")
+    L.append("  return (l1 | l2 | l3) >= 0 && l1 < 4 && l2 < 4 && l3 < 4 ? v[l1 * 16 + l2 * 4 + l3] : -1;")
+    L.append("}")
+    L.append("// Calls f(Cg<l1, l2, l3>{}) for the triple with id `id` (warp-uniform in every caller).")
+    L.append("template <class F>")
+    L.append("__device__ __forceinline__ void with_triple(int id, F&& f) {")
+    L.append("  switch (id) {")
+    for k, (a, b, c) in enumerate(tr):
+        L.append(f"    case {k}: f(Cg<{a}, {b}, {c}>{{}}); break;")
+    L.append("    default: break;")
+    L.append("  }")
+    L.append("}")
+    L.append("template <int L> struct ShBlock;")
+    for l in range(4):
+        L += _gen_sh_block(l)
+    allsh = Spec("all", [0], [0, 1, 2, 3], [0], [(0, 0, 0)])
+    L.append("struct ShAll {")
+    L.append("  static constexpr int NSH = 16;")
+    L += _gen_sh(allsh)
+    L.append("};")
+    L.append("}  // namespace gen")
+    L.append("}  // namespace tp")
+    return "\n".join(L) + "\n"
+
+
+# ---------------------------------------------------------------------------
 # The compiled specialisations
 # ---------------------------------------------------------------------------
 
@@ -935,6 +1042,7 @@ def main(outdir: str):
     reg.append(f"const int kRegistrySize = {len(specs)};")
     reg.append("}  // namespace tp")
     write("registry.cu", "\n".join(reg) + "\n")
+    write("generic_cg.h", gen_generic_header())
     # CG table dump (text) for the host-side table tests
     lines = []
     for l1, l2, l3 in product(range(4), repeat=3):

@@ -56,6 +56,39 @@ struct LaunchArgs {
   float coeff[kMaxPaths];
 };
 
+// Runtime path table: plans whose path list has no compiled specialisation run kernels that
+// take this table by value and dispatch every path to the unrolled contractions of its
+// (l1, l2, l3) triple (generic.cu).
+constexpr int kGenMaxTasks = 256;
+
+struct GenPath {
+  int16_t l1, l2, l3, tid;   // degrees and the triple id of the generated contractions
+  int32_t in_off;            // offset of the path's input block in a row of x (uvw: of x W)
+  int32_t out_off;           // offset of its output block in a row of y
+  int32_t mul;               // channels (uvu: of the path; uvw: output channels)
+  int32_t w_off;             // uvu: first weight of the path in an edge's w row; uvw: path index
+  int32_t in_block, out_block;
+  float coeff;
+};
+
+struct GenTable {
+  int n_paths, n_in, n_out, lmax_sh;
+  int in_off[kMaxBlocks], in_mul[kMaxBlocks], in_l[kMaxBlocks];
+  int out_off[kMaxBlocks], out_mul[kMaxBlocks], out_l[kMaxBlocks];
+  int out_first[kMaxBlocks + 1], out_paths[kMaxPaths];   // paths into each output block, path order
+  int in_first[kMaxBlocks + 1], in_paths[kMaxPaths];     // paths reading each input block
+  int n_rtask, n_stask;                                  // receiver / sender tasks: (block, 32-channel slice)
+  uint8_t rtask_block[kGenMaxTasks], rtask_slice[kGenMaxTasks];
+  uint8_t stask_block[kGenMaxTasks], stask_slice[kGenMaxTasks];
+  GenPath path[kMaxPaths];
+};
+
+// Id of the (l1, l2, l3) triple in the generated contractions, or -1.
+int gen_triple_id(int l1, int l2, int l3);
+cudaError_t launch_gen_fwd(const LaunchArgs& a, const GenTable& T, cudaStream_t s);
+cudaError_t launch_gen_bwd(const LaunchArgs& a, const GenTable& T, cudaStream_t s);
+cudaError_t launch_gen_dbwd(const LaunchArgs& a, const GenTable& T, bool recv, bool send, cudaStream_t s);
+
 // Number of kernels the library has launched in this process (diagnostics).
 void count_launches(int n);
 

@@ -12,16 +12,49 @@ from oracle import OraclePlan, backward, double_backward, forward
 
 TOL = 1e-4
 
+# (tensor name, irreps block, max|err| / max|ref| of the tensor, max|err| / max|ref| of the block)
+BLOCK_RECORDS = []
 
-def assert_close(gpu, ref, name, tol=TOL):
+
+def irreps_blocks(irreps):
+    """Column ranges of the blocks of an irreps string: [(label, start, stop)]."""
+    out, start = [], 0
+    for term in irreps.split("+"):
+        mul, ir = term.split("x")
+        width = int(mul) * (2 * int(ir[:-1]) + 1)
+        out.append((term, start, start + width))
+        start += width
+    return out
+
+
+def block_error_ratios(g, r, irreps):
+    """Per irreps block of the last axis: max|err| over the tensor's max|ref| and over the
+    block's own max|ref|."""
+    scale = float(r.abs().max()) if r.numel() else 0.0
+    rows = []
+    for label, a, b in irreps_blocks(irreps):
+        err = float((g[..., a:b] - r[..., a:b]).abs().max()) if g.numel() else 0.0
+        bscale = float(r[..., a:b].abs().max()) if r.numel() else 0.0
+        rows.append((label, err / scale if scale else 0.0, err / bscale if bscale else 0.0))
+    return rows
+
+
+def assert_close(gpu, ref, name, tol=TOL, irreps=None):
+    """Per tensor max|gpu - ref| <= tol * max|ref|.  With `irreps` (the layout of the last axis)
+    the error of every irreps block is recorded too (reported in the pytest summary)."""
     g = gpu.detach().double().cpu() if isinstance(gpu, torch.Tensor) else torch.as_tensor(gpu, dtype=torch.float64)
     r = ref.detach().double().cpu() if isinstance(ref, torch.Tensor) else torch.as_tensor(ref, dtype=torch.float64)
     assert g.shape == r.shape, (name, g.shape, r.shape)
     assert torch.isfinite(g).all(), f"{name}: non-finite values"
     err = float((g - r).abs().max()) if g.numel() else 0.0
     scale = float(r.abs().max()) if r.numel() else 0.0
+    blocks = ""
+    if irreps is not None:
+        rows = block_error_ratios(g, r, irreps)
+        BLOCK_RECORDS.extend((name, lab, a, b) for lab, a, b in rows)
+        blocks = "; per block " + ", ".join(f"{lab}: {a:.1e}" for lab, a, _ in rows)
     assert err <= tol * scale or (scale == 0.0 and err == 0.0), \
-        f"{name}: max|err| = {err:.3e} > {tol} * max|ref| = {tol * scale:.3e}"
+        f"{name}: max|err| = {err:.3e} > {tol} * max|ref| = {tol * scale:.3e}{blocks}"
     return err / scale if scale else 0.0
 
 

@@ -71,16 +71,33 @@ def test_plan_matches_config_sizes(tp, name):
     (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 1, 0)]), 1),          # triangle
     (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(1, 1, 1)]), 1),          # parity 1o x 1o -> 1o
     (("4x0e+4x1o", "1x0e+1x1o", "8x0e+8x1o", [(0, 0, 0)]), 1),          # uvu multiplicity
-    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 0, 0)]), 2),          # valid, not compiled
+    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 0, 0)]), 0),          # valid, runtime path table
+    (("8x1o+4x0e", "1x0e+1x1o+1x2e", "4x1o+8x2e+8x1o", [(1, 1, 0), (0, 0, 1)]), 1),   # 1o x 0e -> 2e
+    (("8x1o+4x0e", "1x0e+1x1o+1x2e", "4x1o+8x2e+8x1o", [(1, 1, 0), (0, 1, 2)]), 1),   # 1o x 1o -> 1o
+    (("8x1o+4x0e", "1x0e+1x1o+1x2e", "4x1o+8x2e+8x1o", [(1, 1, 0), (0, 1, 1), (0, 2, 2), (0, 0, 2)]), 0),
+    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 0, 0)] * 65), 2),    # more than 64 paths
+    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(1, 1, 0), (0, 0, 0)]), "uvw"),   # uvw: compiled lists only
     (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 0, 2)]), 1),          # index out of range
 ])
 def test_plan_validation(tp, args, status):
+    mode = "uvu"
+    if status == "uvw":
+        mode, status = "uvw", 2
     if status == 0:
-        tp.Plan(*args)
+        tp.Plan(*args, mode)
         return
     with pytest.raises(tp.TPError) as ei:
-        tp.Plan(*args)
+        tp.Plan(*args, mode)
     assert ei.value.status == status, str(ei.value)
+
+
+def test_path_table_plan_sizes(tp):
+    """Blocks of different multiplicities: widths and the per-edge weight count follow the
+    blocks of each path (uvu: the path's input multiplicity)."""
+    plan = tp.Plan("8x1o+4x0e", "1x0e+1x1o+1x2e", "4x1o+8x2e+8x1o", [(1, 1, 0), (0, 1, 1), (0, 2, 2), (0, 0, 2)])
+    assert plan.in_dim == 8 * 3 + 4
+    assert plan.out_dim == 4 * 3 + 8 * 5 + 8 * 3
+    assert plan.n_edge_weights == 4 + 8 + 8 + 8
 
 
 def test_path_coeff_rejects_nan(tp):

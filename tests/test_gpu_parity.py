@@ -48,7 +48,7 @@ def test_c1_forward_complete(tp):
     g = device_inputs(d)
     y = _fwd(tp, plan, g)
     ref = forward(op, d["rowptr"], d["src"], d["x"], d["vec"], w=d["w"])
-    assert_close(y, ref, "c1 y")
+    assert_close(y, ref, "c1 y", irreps=d["spec"].irreps_out)
 
 
 def test_c1_backward_and_double_backward_complete(tp):
@@ -57,7 +57,7 @@ def test_c1_backward_and_double_backward_complete(tp):
     g = device_inputs(d)
     gx, gw, gvec = _bwd(tp, plan, g)
     ref = backward(op, d["rowptr"], d["src"], d["x"], d["vec"], d["gy"], w=d["w"])
-    assert_close(gx, ref["gx"], "c1 gx")
+    assert_close(gx, ref["gx"], "c1 gx", irreps=d["spec"].irreps_in)
     assert_close(gw, ref["gw"], "c1 gw")
     assert_close(gvec, ref["gvec"], "c1 gvec")
     h = tp.tp_conv_dbwd(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["w"], g["gy"], g["ggx"], g["ggw"],
@@ -74,10 +74,11 @@ def test_c2_full_size_forward_backward_complete(tp):
     plan, op = plans(d["spec"], tp)
     g = device_inputs(d)
     y = _fwd(tp, plan, g)
-    assert_close(y, forward(op, d["rowptr"], d["src"], d["x"], d["vec"], w=d["w"]), "c2 y")
+    assert_close(y, forward(op, d["rowptr"], d["src"], d["x"], d["vec"], w=d["w"]), "c2 y",
+                 irreps=d["spec"].irreps_out)
     gx, gw, gvec = _bwd(tp, plan, g)
     ref = backward(op, d["rowptr"], d["src"], d["x"], d["vec"], d["gy"], w=d["w"])
-    assert_close(gx, ref["gx"], "c2 gx")
+    assert_close(gx, ref["gx"], "c2 gx", irreps=d["spec"].irreps_in)
     assert_close(gw, ref["gw"], "c2 gw")
     assert_close(gvec, ref["gvec"], "c2 gvec")
 
@@ -88,10 +89,11 @@ def test_replica_forward_backward_complete(tp, name, n_atoms):
     plan, op = plans(d["spec"], tp)
     g = device_inputs(d)
     y = _fwd(tp, plan, g)
-    assert_close(y, forward(op, d["rowptr"], d["src"], d["x"], d["vec"], w=d["w"]), f"{name} y")
+    assert_close(y, forward(op, d["rowptr"], d["src"], d["x"], d["vec"], w=d["w"]), f"{name} y",
+                 irreps=d["spec"].irreps_out)
     gx, gw, gvec = _bwd(tp, plan, g)
     ref = backward(op, d["rowptr"], d["src"], d["x"], d["vec"], d["gy"], w=d["w"])
-    assert_close(gx, ref["gx"], f"{name} gx")
+    assert_close(gx, ref["gx"], f"{name} gx", irreps=d["spec"].irreps_in)
     assert_close(gw, ref["gw"], f"{name} gw")
     assert_close(gvec, ref["gvec"], f"{name} gvec")
 
@@ -104,8 +106,9 @@ def test_c5_replica_double_backward_complete(tp):
                         g["ggvec"])
     ref = double_backward(op, d["rowptr"], d["src"], d["x"], d["vec"], d["gy"], d["ggx"], d["ggw"], d["ggvec"],
                           w=d["w"])
+    lay = {"g_gy": d["spec"].irreps_out, "g_x": d["spec"].irreps_in}
     for k, name in enumerate(("g_gy", "g_x", "g_w", "g_vec")):
-        assert_close(h[k], ref[name], f"c5 replica {name}")
+        assert_close(h[k], ref[name], f"c5 replica {name}", irreps=lay.get(name))
 
 
 def test_force_training_special_case(tp):

@@ -36,10 +36,10 @@ def test_c4_replica_forward_backward_complete(tp):
     g = device_inputs(d)
     y = _fwd(tp, plan, g)
     ref = forward(op, d["rowptr"], d["src"], d["x"], d["vec"], s=d["s"], W=d["W"])
-    assert_close(y, ref, "c4 replica y")
+    assert_close(y, ref, "c4 replica y", irreps=d["spec"].irreps_out)
     gx, gs, gvec, gW = _bwd(tp, plan, g)
     r = backward(op, d["rowptr"], d["src"], d["x"], d["vec"], d["gy"], s=d["s"], W=d["W"])
-    assert_close(gx, r["gx"], "c4 replica gx")
+    assert_close(gx, r["gx"], "c4 replica gx", irreps=d["spec"].irreps_in)
     assert_close(gs, r["gs"], "c4 replica gs")
     assert_close(gvec, r["gvec"], "c4 replica gvec")
     assert_close(gW.view(r["gW"].shape), r["gW"], "c4 replica gW")
@@ -94,3 +94,21 @@ def test_uvw_deterministic(tp):
     a, b = _bwd(tp, plan, g), _bwd(tp, plan, g)
     for u, v in zip(a, b):
         assert torch.equal(u, v)
+
+
+def test_uvw_through_autograd(tp):
+    """tp_conv in uvw mode: gradients to x, the edge vectors, the per-edge path scalars and the
+    shared mixing weights W through torch autograd, against the float64 oracle."""
+    d = inputs("c4", 240)
+    plan, op = plans(d["spec"], tp)
+    graph = tp.autograd.Graph(dev(d["rowptr"]), dev(d["src"]))
+    x, vec, s, W = (dev(d[k]).requires_grad_() for k in ("x", "vec", "s", "W"))
+    y = tp.tp_conv(plan, graph, x, vec, s, W)
+    (y * dev(d["gy"])).sum().backward()
+    r = backward(op, d["rowptr"], d["src"], d["x"], d["vec"], d["gy"], s=d["s"], W=d["W"])
+    assert_close(x.grad, r["gx"], "autograd uvw gx")
+    assert_close(vec.grad, r["gvec"], "autograd uvw gvec")
+    assert_close(s.grad, r["gs"], "autograd uvw gs")
+    assert_close(W.grad, r["gW"], "autograd uvw gW")
+    with pytest.raises(ValueError):
+        tp.tp_conv(plan, graph, x, vec, s)
