@@ -33,6 +33,8 @@ SIGNATURES = {
     "tp_conv_dbwd": (C.c_int, [_p, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                _p, _p, _sz, _p]),
     "tp_get_device_error": (C.c_int, [_p, _p, _p, C.POINTER(_i32)]),
+    "tp_gather_rows": (C.c_int, [_p, _i64, _p, _i64, _p, _p]),
+    "tp_add_rows": (C.c_int, [_p, _i64, _p, _i64, _p, _p]),
     "tp_status_string": (C.c_char_p, [C.c_int]),
     "tp_last_error_message": (C.c_char_p, []),
     "tp_version": (C.c_char_p, []),

@@ -36,7 +36,7 @@ class _Bwd(torch.autograd.Function):
                                        need_gW=W is not None and needs[3])
         ctx.save_for_backward(x, vec, w, gy)
         ctx.plan, ctx.graph = plan, graph
-        return gx, gvec, gw, gW
+        return gx, gvec, gw, None if gW is None else gW.view(W.shape)
 
     @staticmethod
     def backward(ctx, ggx, ggvec, ggw, ggW):

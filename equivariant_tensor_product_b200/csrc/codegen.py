@@ -858,14 +858,8 @@ def _gen_triple(l1, l2, l3) -> List[str]:
                  f"float (&{out})[{on}]) {{")
         used = sorted({key_pair(i, j, k) for i, j, k, c in nz})
         for (u, v) in used:
-            # products with Y_0 (= 1) need no multiply
-            if name == "fwd":
-                e = f"{a}[{u}]" if l2 == 0 else f"{a}[{u}] * {b}[{v}]"
-            elif name == "tx":
-                e = f"{b}[{v}]" if l2 == 0 else f"{a}[{u}] * {b}[{v}]"
-            else:
-                e = f"{a}[{u}] * {b}[{v}]"
-            L.append(f"    const float p{u}_{v} = {e};")
+            # no shortcut for l2 = 0: the double backward passes dY (zero for l = 0) in place of Y
+            L.append(f"    const float p{u}_{v} = {a}[{u}] * {b}[{v}];")
         for m in range(on):
             terms = [(c, "p%d_%d" % key_pair(i, j, k)) for (i, j, k, c) in nz if key_out(i, j, k) == m]
             L.extend(line.replace("      ", "    ", 1) for line in _chain(terms, f"{out}[{m}]", decl=False))

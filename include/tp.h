@@ -171,6 +171,21 @@ tp_status_t tp_conv_dbwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* ro
                          float* g_gy, float* g_x, float* g_w, float* g_vec, void* ws,
                          size_t ws_bytes, tp_stream_t stream);
 
+/* Row movement of receiver-range sharding over several GPUs (one process per GPU): a rank
+ * owning a contiguous range of receivers gathers the x rows its peers need before the halo
+ * exchange, and adds the gradient partials its peers send back for the senders it owns
+ * ("Sobek: Streaming Equivariant Tensor Product Convolutions", abstract: graphs far beyond
+ * one device's memory; the exchange itself is the caller's collective).
+ *   tp_gather_rows: dst[k, :] = src[idx[k], :] for k < n (rows of row_len floats).
+ *   tp_add_rows:    dst[idx[k], :] += src[k, :] for k < n; the n indices of one call must be
+ *                   distinct, which makes the result independent of the schedule.
+ * idx holds valid row indices of the respective arrays (not checked on the device).
+ * TP_ERR_INVALID_ARG for n < 0, row_len <= 0, NULL or non-4-byte-aligned pointers with n > 0. */
+tp_status_t tp_gather_rows(const float* src, int64_t row_len, const int32_t* idx, int64_t n, float* dst,
+                           tp_stream_t stream);
+tp_status_t tp_add_rows(float* dst, int64_t row_len, const int32_t* idx, int64_t n, const float* src,
+                        tp_stream_t stream);
+
 /* Reads (and clears) the device error word after the work on `stream` finished;
  * synchronises the stream.  Check-mode plans read the word of workspace `ws`; other plans,
  * and plan == NULL, read the per-device word (ws unused) -- the word the linear maps of
