@@ -162,6 +162,22 @@ UvwLayout uvw_layout(tp_plan_t plan, int64_t N, int64_t E, bool bwd) {
   return U;
 }
 
+// uvw through the path table: x W per path (fwd and bwd), its gradient B and the gW node-chunk
+// partials (bwd), after the transpose region in the backward.
+UvwLayout gen_uvw_layout(tp_plan_t plan, int64_t N, int64_t E, bool bwd) {
+  UvwLayout U{};
+  size_t off = bwd ? ws_layout(N, E).total : 256;
+  const size_t xt_bytes = sizeof(float) * (size_t)(N > 0 ? N : 1) * plan->gen->xt_dim;
+  U.A = off;
+  off += align256(xt_bytes);
+  U.G = off;
+  if (bwd) off += align256(xt_bytes);
+  U.xT = U.Wt = U.part = off;
+  if (bwd) off += align256(sizeof(float) * (size_t)plan->n_shared * uvw_splits(N));
+  U.total = off;
+  return U;
+}
+
 int pick_split(int64_t N, int64_t E) {
   if (N <= 0) return 1;
   const double avg = (double)E / (double)N;
@@ -240,8 +256,11 @@ tp_status_t debug_prologue(tp_plan_t plan, int64_t N, int64_t E, const int32_t* 
 // per block and the (block, 32-channel slice) tasks of the receiver and sender passes.
 bool build_gen_table(const std::vector<IrrepBlock>& bi, const std::vector<IrrepBlock>& bs,
                      const std::vector<IrrepBlock>& bo, const int32_t* paths, int n_paths, const double* coeff,
-                     GenTable& T, std::string& why) {
+                     bool uvw, GenTable& T, std::string& why) {
   std::memset(&T, 0, sizeof(T));
+  T.uvw = uvw ? 1 : 0;
+  T.mul_in = bi[0].mul;
+  T.mul_out = bo[0].mul;
   T.n_paths = n_paths;
   T.n_in = (int)bi.size();
   T.n_out = (int)bo.size();
@@ -271,10 +290,11 @@ bool build_gen_table(const std::vector<IrrepBlock>& bi, const std::vector<IrrepB
       why = "path outside the generated triples";
       return false;
     }
-    P.in_off = T.in_off[a];
+    P.in_off = uvw ? T.xt_dim : T.in_off[a];     // uvw: the path's block in a row of x W
     P.out_off = T.out_off[o];
-    P.mul = bi[a].mul;
-    P.w_off = w_off;
+    P.mul = uvw ? bo[o].mul : bi[a].mul;
+    P.w_off = uvw ? p : w_off;
+    if (uvw) T.xt_dim += bo[o].mul * (2 * bi[a].l + 1);
     P.in_block = a;
     P.out_block = o;
     P.coeff = coeff ? (float)coeff[p] : 1.0f;
@@ -414,22 +434,19 @@ tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* i
            s->paths[p][2] == paths[3 * p + 2];
     if (ok) found = s;
   }
-  if (mode == TP_MODE_UVW && !found)
-    return fail(TP_ERR_UNSUPPORTED,
-                "uvw runs on the compiled path lists (all paths of lmax 1, 2 or 3, uniform multiplicity); "
-                "uvu takes any path list");
-  if (mode == TP_MODE_UVW && (!found->uvw_fwd || !found->uvw_bwd))
-    return fail(TP_ERR_UNSUPPORTED, "spec '%s' has no uvw kernels", found->name);
-  // the uvw GEMMs load their operands by TMA, whose row pitches are multiples of 16 bytes
-  if (mode == TP_MODE_UVW && (mul_in % 4 != 0 || mul_out % 4 != 0))
-    return fail(TP_ERR_UNSUPPORTED, "uvw needs multiplicities that are multiples of 4 (got %d, %d)", mul_in,
-                mul_out);
+  // uvw shares one W_p [mul_in, mul_out] per path: one multiplicity per side
+  if (mode == TP_MODE_UVW && !uniform)
+    return fail(TP_ERR_UNSUPPORTED, "uvw needs one multiplicity for all input blocks and one for all output blocks");
+  if (found && mode == TP_MODE_UVW && (!found->uvw_fwd || !found->uvw_bwd)) found = nullptr;
+  // the compiled uvw GEMMs load their operands by TMA, whose row pitches are multiples of 16
+  // bytes; other multiplicities take the path table
+  if (found && mode == TP_MODE_UVW && (mul_in % 4 != 0 || mul_out % 4 != 0)) found = nullptr;
   GenTable* gen = nullptr;
   if (!found) {
     gen = new (std::nothrow) GenTable;
     if (!gen) return fail(TP_ERR_INVALID_ARG, "out of host memory");
     std::string why2;
-    if (!build_gen_table(bi, bs, bo, paths, n_paths, path_coeff, *gen, why2)) {
+    if (!build_gen_table(bi, bs, bo, paths, n_paths, path_coeff, mode == TP_MODE_UVW, *gen, why2)) {
       delete gen;
       return fail(TP_ERR_UNSUPPORTED, "%s", why2.c_str());
     }
@@ -494,7 +511,7 @@ tp_status_t tp_workspace_size(tp_plan_t plan, int64_t N, int64_t E, int32_t op, 
   size_t need = 0;
   if (plan->mode == TP_MODE_UVW) {
     if (op == TP_OP_DBWD) return fail(TP_ERR_UNSUPPORTED, "double backward is implemented for uvu");
-    need = uvw_layout(plan, N, E, op == TP_OP_BWD).total;
+    need = plan->gen ? gen_uvw_layout(plan, N, E, op == TP_OP_BWD).total : uvw_layout(plan, N, E, op == TP_OP_BWD).total;
   } else if (op == TP_OP_FWD) {
     need = (plan->flags & TP_FLAG_CHECK_INDICES) ? 256 : 0;
   } else {
@@ -555,7 +572,13 @@ tp_status_t tp_conv_fwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* row
   a.w = w;
   a.y = y;
   cudaError_t e;
-  if (plan->mode == TP_MODE_UVW) {
+  if (plan->mode == TP_MODE_UVW && plan->gen) {
+    const UvwLayout U = gen_uvw_layout(plan, N, E, false);
+    a.W = W;
+    a.A = reinterpret_cast<float*>(static_cast<char*>(ws) + U.A);
+    a.nw = plan->n_paths;
+    e = launch_gen_uvw_fwd(a, *plan->gen, s);
+  } else if (plan->mode == TP_MODE_UVW) {
     const UvwLayout U = uvw_layout(plan, N, E, false);
     char* wsb = static_cast<char*>(ws);
     a.W = W;
@@ -631,6 +654,20 @@ tp_status_t tp_conv_bwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* row
   a.gx = gx;
   a.gw = gw;
   a.gvec = gvec;
+  if (plan->mode == TP_MODE_UVW && plan->gen) {
+    const UvwLayout U = gen_uvw_layout(plan, N, E, true);
+    char* wsb = static_cast<char*>(ws);
+    a.W = W;
+    a.A = reinterpret_cast<float*>(wsb + U.A);
+    a.G = reinterpret_cast<float*>(wsb + U.G);
+    a.part = reinterpret_cast<float*>(wsb + U.part);
+    a.splits = uvw_splits(N);
+    a.gW = gW;
+    a.nw = plan->n_paths;
+    cudaError_t e = launch_gen_uvw_bwd(a, *plan->gen, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tp_conv_bwd (uvw) launch");
+    return TP_OK;
+  }
   if (plan->mode == TP_MODE_UVW) {
     const UvwLayout U = uvw_layout(plan, N, E, true);
     char* wsb = static_cast<char*>(ws);

@@ -17,6 +17,8 @@
 //                channels reduced across the warp.
 // Every output element is written by exactly one warp, in a fixed order: deterministic, no
 // float atomics, no edge-sized intermediate.
+#include <algorithm>
+
 #include "generic_cg.h"
 #include "tp_common.h"
 #include "tp_kernels.cuh"
@@ -247,12 +249,13 @@ __global__ void __launch_bounds__(32 * kGenWarps) k_gen_send(const __grid_consta
 }
 
 // ---------------------------------------------------------------------------------------
-// Direction gradient per edge (uvu).  MODE 0: gvec[e] = sum_m gY_m dY_m/dv with
+// Direction gradient per edge.  MODE 0: gvec[e] = sum_m gY_m dY_m/dv with
 // gY = sum_{p, u} c_p w_p Q_p(x[src], gy[dst]), Q(x, g)[m2] = sum C x[m1] g[m3].
 // MODE 1: g_vec[e] = sum_m G1_m dY_m/dv + G2_m (d^2 Y_m / dv^2) ggvec with
 // G1 = sum c_p (ggw_p Q_p(x, gy) + w_p Q_p(ggx, gy)), G2 = sum c_p w_p Q_p(x, gy).
+// UVW (MODE 0): x is x W per path and w the per-edge path scalar s[e, p].
 // ---------------------------------------------------------------------------------------
-template <int MODE>
+template <int MODE, bool UVW = false>
 __global__ void __launch_bounds__(32 * kGenWarps) k_gen_edge(const __grid_constant__ LaunchArgs a,
                                                              const __grid_constant__ GenTable T) {
   const int lane = threadIdx.x & 31;
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(32 * kGenWarps) k_gen_edge(const __grid_consta
         float xv[Cg::D1], gyv[Cg::D3], qa[Cg::D2];
         load_row(a.x + (int64_t)j * a.in_dim + P.in_off + (int64_t)c * Cg::D1, xv);
         load_row(a.gy + (int64_t)i * a.out_dim + P.out_off + (int64_t)c * Cg::D3, gyv);
-        const int64_t widx = (int64_t)e * a.nw + P.w_off + c;
+        const int64_t widx = (int64_t)e * a.nw + (UVW ? p : P.w_off + c);
         const float w = P.coeff * __ldg(a.w + widx);
         Cg::ty(xv, gyv, qa);
         if constexpr (MODE == 0) {
@@ -359,6 +362,189 @@ __global__ void __launch_bounds__(32 * kGenWarps) k_gen_edge(const __grid_consta
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// uvw through the path table ("Sobek", abstract: the shared multiplicity mixing W_p kept,
+// applied on node state instead of per edge).  Forward: xt_p[j] = W_p^T x_a[j] per path and
+// node, then the receiver pass with xt_p as the path's input rows and s[e, p] as its weight.
+// Backward: B_p[j] = sum_{e: src=j} c_p s_p C_p^T(Y, gy[dst]) (sender pass, which also gives
+// gs[e, p] = c_p <xt_p[j], C_p^T(Y, gy[dst])>), gx_a[j] = sum_{p: in=a} W_p B_p[j],
+// gW_p = sum_j x_a[j] B_p[j]^T (node chunks, summed in chunk order).  Layout of a row of xt
+// and of B: path after path, [w][m1] inside a path.
+// ---------------------------------------------------------------------------------------
+
+// xt[j, off_p + w d1 + m1] = sum_u W[p, u, w] x[j, in_a + u d1 + m1]: one thread per (j, p, w)
+__global__ void __launch_bounds__(256) k_gen_xw(const __grid_constant__ LaunchArgs a,
+                                                const __grid_constant__ GenTable T) {
+  const int64_t per_node = (int64_t)T.n_paths * T.mul_out;
+  const int64_t total = (int64_t)a.N * per_node;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t j = t / per_node;
+    const int r = (int)(t - j * per_node);
+    const int p = r / T.mul_out, w = r - p * T.mul_out;
+    const GenPath P = T.path[p];
+    const int d1 = 2 * P.l1 + 1;
+    const float* xr = a.x + j * a.in_dim + T.in_off[P.in_block];
+    const float* Wp = a.W + (int64_t)p * T.mul_in * T.mul_out + w;
+    float acc[7];
+    zero(acc);
+    for (int u = 0; u < T.mul_in; ++u) {
+      const float wv = __ldg(Wp + (int64_t)u * T.mul_out);
+#pragma unroll
+      for (int m = 0; m < 7; ++m)
+        if (m < d1) acc[m] = fmaf(wv, __ldg(xr + u * d1 + m), acc[m]);
+    }
+    float* o = a.A + j * T.xt_dim + P.in_off + (int64_t)w * d1;
+#pragma unroll
+    for (int m = 0; m < 7; ++m)
+      if (m < d1) o[m] = acc[m];
+  }
+}
+
+// One warp per (sender, path): B_p[j] (all output channels, in groups of four 32-channel
+// slices kept in registers) and gs[e, p] (a warp sum per edge; later groups add to it).
+__global__ void __launch_bounds__(32 * kGenWarps) k_gen_send_uvw(const __grid_constant__ LaunchArgs a,
+                                                                 const __grid_constant__ GenTable T) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (int64_t)blockIdx.x * kGenWarps + (threadIdx.x >> 5);
+  if (wid >= (int64_t)a.N * T.n_paths) return;
+  const int node = (int)(wid / T.n_paths), p = (int)(wid - (int64_t)node * T.n_paths);
+  const GenPath P = T.path[p];
+  const int q0 = __ldg(a.colptr + node), q1 = __ldg(a.colptr + node + 1);
+  const int n_sl = (T.mul_out + 31) / 32;
+  gen::with_triple(P.tid, [&](auto cg) {
+    using Cg = decltype(cg);
+    for (int g0 = 0; g0 < n_sl; g0 += 4) {
+      float B[4][Cg::D1], xt[4][Cg::D1];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        zero(B[k]);
+        zero(xt[k]);
+        const int c = (g0 + k) * 32 + lane;
+        if (g0 + k < n_sl && c < T.mul_out) load_row(a.A + (int64_t)node * T.xt_dim + P.in_off + (int64_t)c * Cg::D1, xt[k]);
+      }
+      for (int base = q0; base < q1; base += 32) {
+        const int my_q = base + lane;
+        int my_e = -1, my_i = 0;
+        float vx = 0.f, vy = 0.f, vz = 0.f;
+        if (my_q < q1) {
+          my_e = __ldg(a.perm + my_q);
+          my_i = find_row(a.rowptr, a.N, my_e);
+          vx = __ldg(a.vec + 3 * (int64_t)my_e);
+          vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
+          vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
+        }
+        const int ne = min(32, q1 - base);
+        for (int k = 0; k < ne; ++k) {
+          const int e = __shfl_sync(kFull, my_e, k), i = __shfl_sync(kFull, my_i, k);
+          const float ux = __shfl_sync(kFull, vx, k), uy = __shfl_sync(kFull, vy, k), uz = __shfl_sync(kFull, vz, k);
+          float rx, ry, rz, ir;
+          edge_geometry(ux, uy, uz, rx, ry, rz, ir);
+          float Y[Cg::D2];
+          gen::ShBlock<Cg::L2>::sh(rx, ry, rz, Y);
+          const float sc = P.coeff * __ldg(a.w + (int64_t)e * a.nw + p);
+          float part = 0.f;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int c = (g0 + kk) * 32 + lane;
+            if (g0 + kk < n_sl && c < T.mul_out) {
+              float gyv[Cg::D3], z[Cg::D1];
+              load_row(a.gy + (int64_t)i * a.out_dim + P.out_off + (int64_t)c * Cg::D3, gyv);
+              Cg::tx(Y, gyv, z);
+#pragma unroll
+              for (int m = 0; m < Cg::D1; ++m) {
+                B[kk][m] = fmaf(sc, z[m], B[kk][m]);
+                part = fmaf(xt[kk][m], z[m], part);
+              }
+            }
+          }
+          part = warp_sum(part);
+          if (lane == 0 && a.gw) {
+            float* gs = a.gw + (int64_t)e * a.nw + p;
+            *gs = g0 == 0 ? P.coeff * part : *gs + P.coeff * part;
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = (g0 + k) * 32 + lane;
+        if (g0 + k < n_sl && c < T.mul_out) {
+          float* o = a.G + (int64_t)node * T.xt_dim + P.in_off + (int64_t)c * Cg::D1;
+#pragma unroll
+          for (int m = 0; m < Cg::D1; ++m) o[m] = B[k][m];
+        }
+      }
+    }
+  });
+}
+
+// gx[j, in_a + u d1 + m1] = sum_{p: in(p) = a} sum_w W[p, u, w] B[j, off_p + w d1 + m1]:
+// one thread per (j, input block, u)
+__global__ void __launch_bounds__(256) k_gen_bw(const __grid_constant__ LaunchArgs a,
+                                                const __grid_constant__ GenTable T) {
+  const int64_t per_node = (int64_t)T.n_in * T.mul_in;
+  const int64_t total = (int64_t)a.N * per_node;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t j = t / per_node;
+    const int r = (int)(t - j * per_node);
+    const int ib = r / T.mul_in, u = r - ib * T.mul_in;
+    const int d1 = 2 * T.in_l[ib] + 1;
+    float acc[7];
+    zero(acc);
+    for (int pi = T.in_first[ib]; pi < T.in_first[ib + 1]; ++pi) {
+      const int p = T.in_paths[pi];
+      const float* Wr = a.W + ((int64_t)p * T.mul_in + u) * T.mul_out;
+      const float* Br = a.G + j * T.xt_dim + T.path[p].in_off;
+      for (int w = 0; w < T.mul_out; ++w) {
+        const float wv = __ldg(Wr + w);
+#pragma unroll
+        for (int m = 0; m < 7; ++m)
+          if (m < d1) acc[m] = fmaf(wv, Br[w * d1 + m], acc[m]);
+      }
+    }
+    float* o = a.gx + j * a.in_dim + T.in_off[ib] + (int64_t)u * d1;
+#pragma unroll
+    for (int m = 0; m < 7; ++m)
+      if (m < d1) o[m] = acc[m];
+  }
+}
+
+// part[z, p, u, w] = sum over the nodes j of chunk z and m1 of x[j, in_a + u d1 + m1] B[j, off_p + w d1 + m1]
+__global__ void __launch_bounds__(256) k_gen_gw_part(const __grid_constant__ LaunchArgs a,
+                                                     const __grid_constant__ GenTable T) {
+  const int64_t n_sh = (int64_t)T.n_paths * T.mul_in * T.mul_out;
+  const int z = blockIdx.y;
+  const int64_t chunk = ((int64_t)a.N + a.splits - 1) / a.splits;
+  const int64_t j0 = z * chunk, j1 = min((int64_t)a.N, j0 + chunk);
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < n_sh; t += (int64_t)gridDim.x * blockDim.x) {
+    const int p = (int)(t / ((int64_t)T.mul_in * T.mul_out));
+    const int r = (int)(t - (int64_t)p * T.mul_in * T.mul_out);
+    const int u = r / T.mul_out, w = r - u * T.mul_out;
+    const GenPath P = T.path[p];
+    const int d1 = 2 * P.l1 + 1;
+    float acc = 0.f;
+    for (int64_t j = j0; j < j1; ++j) {
+      const float* xr = a.x + j * a.in_dim + T.in_off[P.in_block] + (int64_t)u * d1;
+      const float* Br = a.G + j * T.xt_dim + P.in_off + (int64_t)w * d1;
+      for (int m = 0; m < d1; ++m) acc = fmaf(__ldg(xr + m), Br[m], acc);
+    }
+    a.part[(int64_t)z * n_sh + t] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(256) k_gen_gw_reduce(const __grid_constant__ LaunchArgs a, int64_t n_sh) {
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < n_sh; t += (int64_t)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int z = 0; z < a.splits; ++z) s += a.part[(int64_t)z * n_sh + t];
+    a.gW[t] = s;
+  }
+}
+
+unsigned flat_grid(int64_t n) {
+  int64_t g = (n + 255) / 256;
+  if (g > 148 * 32) g = 148 * 32;
+  return (unsigned)(g < 1 ? 1 : g);
+}
+
 unsigned warps_grid(int64_t warps) { return (unsigned)((warps + kGenWarps - 1) / kGenWarps); }
 
 }  // namespace
@@ -405,6 +591,58 @@ cudaError_t launch_gen_dbwd(const LaunchArgs& a, const GenTable& T, bool recv, b
   if (send && a.gvec && a.E > 0) {
     k_gen_edge<1><<<warps_grid(a.E), 32 * kGenWarps, 0, s>>>(a, T);
     count_launches(1);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gen_uvw_fwd(const LaunchArgs& a, const GenTable& T, cudaStream_t s) {
+  if (a.N == 0) return cudaSuccess;
+  k_gen_xw<<<flat_grid((int64_t)a.N * T.n_paths * T.mul_out), 256, 0, s>>>(a, T);
+  count_launches(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || T.n_rtask == 0) return e;
+  LaunchArgs b = a;                 // the receiver pass reads x W per path
+  b.x = a.A;
+  b.in_dim = T.xt_dim;
+  b.nw = T.n_paths;
+  k_gen_recv<0, true><<<warps_grid((int64_t)a.N * T.n_rtask), 32 * kGenWarps, 0, s>>>(b, T);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gen_uvw_bwd(const LaunchArgs& a, const GenTable& T, cudaStream_t s) {
+  if (a.N == 0) return cudaSuccess;
+  k_gen_xw<<<flat_grid((int64_t)a.N * T.n_paths * T.mul_out), 256, 0, s>>>(a, T);
+  count_launches(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (a.gw || a.gx || a.gW) {
+    LaunchArgs b = a;
+    b.nw = T.n_paths;
+    k_gen_send_uvw<<<warps_grid((int64_t)a.N * T.n_paths), 32 * kGenWarps, 0, s>>>(b, T);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (a.gvec && a.E > 0) {
+    LaunchArgs b = a;
+    b.x = a.A;
+    b.in_dim = T.xt_dim;
+    b.nw = T.n_paths;
+    k_gen_edge<0, true><<<warps_grid(a.E), 32 * kGenWarps, 0, s>>>(b, T);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (a.gx) {
+    k_gen_bw<<<flat_grid((int64_t)a.N * T.n_in * T.mul_in), 256, 0, s>>>(a, T);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (a.gW) {
+    const int64_t n_sh = (int64_t)T.n_paths * T.mul_in * T.mul_out;
+    const dim3 grid((unsigned)std::min<int64_t>((n_sh + 255) / 256, 1024), (unsigned)a.splits);
+    k_gen_gw_part<<<grid, 256, 0, s>>>(a, T);
+    k_gen_gw_reduce<<<flat_grid(n_sh), 256, 0, s>>>(a, n_sh);
+    count_launches(2);
   }
   return cudaGetLastError();
 }

@@ -73,6 +73,9 @@ struct GenPath {
 
 struct GenTable {
   int n_paths, n_in, n_out, lmax_sh;
+  int uvw;                   // uvw: path p reads the rows of x W_p (offset path[p].in_off in a row of
+  int xt_dim;                // xt_dim floats), mul_in / mul_out uniform; W is [P][mul_in][mul_out]
+  int mul_in, mul_out;
   int in_off[kMaxBlocks], in_mul[kMaxBlocks], in_l[kMaxBlocks];
   int out_off[kMaxBlocks], out_mul[kMaxBlocks], out_l[kMaxBlocks];
   int out_first[kMaxBlocks + 1], out_paths[kMaxPaths];   // paths into each output block, path order
@@ -88,6 +91,10 @@ int gen_triple_id(int l1, int l2, int l3);
 cudaError_t launch_gen_fwd(const LaunchArgs& a, const GenTable& T, cudaStream_t s);
 cudaError_t launch_gen_bwd(const LaunchArgs& a, const GenTable& T, cudaStream_t s);
 cudaError_t launch_gen_dbwd(const LaunchArgs& a, const GenTable& T, bool recv, bool send, cudaStream_t s);
+// uvw through the path table.  fwd: a.A = x W per path [N, xt_dim] (workspace).  bwd: a.A as
+// in fwd, a.G = its gradient B [N, xt_dim], a.part = a.splits node-chunk partials of gW.
+cudaError_t launch_gen_uvw_fwd(const LaunchArgs& a, const GenTable& T, cudaStream_t s);
+cudaError_t launch_gen_uvw_bwd(const LaunchArgs& a, const GenTable& T, cudaStream_t s);
 
 // Number of kernels the library has launched in this process (diagnostics).
 void count_launches(int n);

@@ -83,17 +83,27 @@ enum { TP_MODE_UVU = 0, TP_MODE_UVW = 1 };
 enum { TP_FLAG_CHECK_INDICES = 1 };
 enum { TP_OP_FWD = 0, TP_OP_BWD = 1, TP_OP_DBWD = 2 };
 
-/* Builds a plan from irreps strings and a path list.
+/* Builds a plan from irreps strings and a path list ("FlashTP: Fused, Sparsity-Aware Tensor
+ * Product for Machine Learning Interatomic Potentials", abstract: the tensor product over the
+ * model's paths; "Sobek: Streaming Equivariant Tensor Product Convolutions", abstract: uvu and
+ * uvw operator families).
  *   irreps_in/out: "32x0e+32x1o+32x2e" (mul x l parity); irreps_sh: "1x0e+1x1o+1x2e"
  *   (multiplicity 1, parity (-1)^l).  paths: [n_paths][3] = (i_in, i_sh, i_out) block
- *   indices; their order fixes the weight layout.  Rules: triangle |l1-l2| <= l3 <= l1+l2,
- *   parity p3 = p1 * p2, uvu needs mul_in == mul_out.  path_coeff: NULL = all 1.0.
- *   All blocks of irreps_in share one multiplicity, and of irreps_out too.  uvw needs
- *   multiplicities that are multiples of 4 (its GEMM operands are loaded by TMA, whose row
- *   pitch must be a multiple of 16 bytes); others return TP_ERR_UNSUPPORTED.
- * Errors: TP_ERR_INVALID_ARG (syntax, rule violations), TP_ERR_UNSUPPORTED (no compiled
- * specialisation for this path list: the build ships lmax 1/2/3 "all paths" lists and the
- * 4-path lmax-1 list; or l > 3; or uvw on a list without a uvw kernel). */
+ *   indices, any subset, order or repetition of allowed triples (at most 64 paths); their
+ *   order fixes the weight layout: uvu w[e] holds the paths in list order, each path's
+ *   mul_in(path) channels contiguous; uvw s[e, p] and W[p][mul_in][mul_out].  Rules:
+ *   triangle |l1-l2| <= l3 <= l1+l2, parity p3 = p1 * p2, uvu needs mul_in == mul_out per
+ *   path (blocks may differ from each other), uvw needs one multiplicity for all input
+ *   blocks and one for all output blocks.  Output blocks no path reaches are zero.
+ *   path_coeff: NULL = all 1.0.
+ * The lists the build compiles whole (all paths of lmax 1, 2 and 3, and the 4-path lmax-1
+ * list, with uniform multiplicities; uvw with multiplicities that are multiples of 4, the
+ * TMA row-pitch rule of its tensor-core GEMMs) run their specialised kernels; every other
+ * valid list runs the runtime path table (per-triple unrolled contractions chosen at run
+ * time).
+ * Errors: TP_ERR_INVALID_ARG (syntax, rule violations), TP_ERR_UNSUPPORTED (l > 3, more than
+ * 64 paths or 16 blocks, more than 256 32-channel slices, uvw with blocks of different
+ * multiplicities). */
 tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* irreps_sh,
                            const char* irreps_out, const int32_t* paths, int32_t n_paths,
                            int32_t mode, const double* path_coeff, uint32_t flags);

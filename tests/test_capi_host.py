@@ -76,13 +76,14 @@ def test_plan_matches_config_sizes(tp, name):
     (("8x1o+4x0e", "1x0e+1x1o+1x2e", "4x1o+8x2e+8x1o", [(1, 1, 0), (0, 1, 2)]), 1),   # 1o x 1o -> 1o
     (("8x1o+4x0e", "1x0e+1x1o+1x2e", "4x1o+8x2e+8x1o", [(1, 1, 0), (0, 1, 1), (0, 2, 2), (0, 0, 2)]), 0),
     (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 0, 0)] * 65), 2),    # more than 64 paths
-    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(1, 1, 0), (0, 0, 0)]), "uvw"),   # uvw: compiled lists only
+    (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(1, 1, 0), (0, 0, 0)]), "uvw"),   # uvw, runtime path table
+    (("4x0e+8x1o", "1x0e+1x1o", "4x0e+4x1o", [(1, 1, 0), (0, 0, 0)]), "uvw-2"),  # uvw: one mul per side
     (("4x0e+4x1o", "1x0e+1x1o", "4x0e+4x1o", [(0, 0, 2)]), 1),          # index out of range
 ])
 def test_plan_validation(tp, args, status):
     mode = "uvu"
-    if status == "uvw":
-        mode, status = "uvw", 2
+    if isinstance(status, str):
+        mode, status = "uvw", int(status[4:] or 0)
     if status == 0:
         tp.Plan(*args, mode)
         return
@@ -130,13 +131,16 @@ def test_transpose_workspace_is_int_sized(tp):
         tp.tp_csr_transpose_workspace_size(-1, 4)
 
 
-def test_uvw_rejects_multiplicities_off_the_tma_pitch(tp):
-    # the mixing GEMMs load rows by TMA, whose row pitch must be a multiple of 16 bytes
+def test_uvw_multiplicities_off_the_tma_pitch_take_the_path_table(tp):
+    # the compiled mixing GEMMs load rows by TMA, whose row pitch must be a multiple of 16
+    # bytes; other multiplicities run through the path table (node-sized x W, no TMA)
     spec = synth.CONFIGS["c4"]
-    bad_in = "+".join(f"30x{b.split('x')[1]}" for b in spec.irreps_in.split("+"))
-    with pytest.raises(tp.TPError) as e:
-        tp.Plan(bad_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvw")
-    assert e.value.status == 2
+    odd_in = "+".join(f"30x{b.split('x')[1]}" for b in spec.irreps_in.split("+"))
+    plan = tp.Plan(odd_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvw")
+    assert plan.n_shared_weights == len(spec.paths) * 30 * 128
+    N, E = 1000, 30000
+    # forward workspace: x W per path (N x sum_p d1_p x mul_out floats), node sized
+    assert tp.tp_workspace_size(plan, N, E, tp.TP_OP_FWD) <= 4 * N * 51 * 128 + 1024
     ok_in = "+".join(f"36x{b.split('x')[1]}" for b in spec.irreps_in.split("+"))
     tp.Plan(ok_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvw")
 

@@ -160,3 +160,47 @@ def test_path_table_deterministic_and_index_check(tp):
     ws = torch.zeros(tp.tp_workspace_size(chk, 300, len(src), tp.TP_OP_FWD), dtype=torch.uint8, device="cuda")
     tp.tp_conv_fwd(chk, g["rowptr"], dev(bad), g["x"], g["vec"], g["w"], ws=ws)
     assert tp.tp_get_device_error(chk, ws) == 2
+
+
+def _check_uvw(tp, spec, N=120, max_deg=16, seed=0, coeff=None, tag=""):
+    ir_in, ir_sh, ir_out, paths = spec
+    plan = tp.Plan(ir_in, ir_sh, ir_out, paths, "uvw", path_coeff=coeff)
+    op = OraclePlan(ir_in, ir_sh, ir_out, paths, "uvw", path_coeff=coeff)
+    rowptr, src, vec, rng = random_graph(seed, N, max_deg)
+    E = len(src)
+    mi, mo = int(ir_in.split("x")[0]), int(ir_out.split("x")[0])
+    x = rng.standard_normal((N, plan.in_dim)).astype(np.float32)
+    s_ = rng.standard_normal((E, len(paths))).astype(np.float32)
+    W = (rng.standard_normal((len(paths), mi, mo)) / np.sqrt(mi)).astype(np.float32)
+    gy = rng.standard_normal((N, plan.out_dim)).astype(np.float32)
+    g = {k: dev(v) for k, v in dict(rowptr=rowptr, src=src, vec=vec, x=x, s=s_, W=W, gy=gy).items()}
+    y = tp.tp_conv_fwd(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["s"], W=g["W"])
+    assert_close(y, forward(op, rowptr, src, x, vec, s=s_, W=W), f"{tag} y", irreps=ir_out)
+    gx, gs, gvec, gW = tp.tp_conv_bwd(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["s"], g["gy"], W=g["W"],
+                                      need_gvec=True, need_gW=True)
+    r = backward(op, rowptr, src, x, vec, gy, s=s_, W=W)
+    assert_close(gx, r["gx"], f"{tag} gx", irreps=ir_in)
+    assert_close(gs, r["gs"], f"{tag} gs")
+    assert_close(gvec, r["gvec"], f"{tag} gvec")
+    assert_close(gW.view(r["gW"].shape), r["gW"], f"{tag} gW")
+
+
+def _uniform(spec, mi, mo):
+    ir_in, ir_sh, ir_out, paths = spec
+    relabel = lambda irr, m: "+".join(f"{m}x{b.split('x')[1]}" for b in irr.split("+"))
+    return relabel(ir_in, mi), ir_sh, relabel(ir_out, mo), paths
+
+
+@pytest.mark.parametrize("lmax,mi,mo,n_keep,seed", [(2, 16, 24, 8, 21), (3, 8, 40, 14, 22), (1, 5, 7, 4, 23)])
+def test_uvw_random_path_subsets(tp, lmax, mi, mo, n_keep, seed):
+    spec = _uniform(random_spec(seed, lmax, (8,), n_keep), mi, mo)
+    coeff = list(np.random.default_rng(seed).uniform(0.5, 1.5, len(spec[3])))
+    _check_uvw(tp, spec, seed=seed, coeff=coeff, tag=f"uvw lmax {lmax} {mi}->{mo}")
+
+
+def test_uvw_config_list_off_the_tma_pitch(tp):
+    """The c4 path list with 30 input channels (not a multiple of 4): the path table."""
+    import synth
+    c4 = synth.CONFIGS["c4"]
+    spec = _uniform((c4.irreps_in, c4.irreps_sh, c4.irreps_out, c4.paths), 30, 20)
+    _check_uvw(tp, spec, N=60, seed=24, tag="uvw c4 list 30->20")
