@@ -356,10 +356,32 @@ def run_reference(args, rank):
 # GPU side
 # ------------------------------------------------------------------------------------------
 
-def kernel_source_hash():
+SPEC_OF_WORKLOAD = {"c1": "l1_c1", "c2": "full_l2", "c3": "full_l3", "c4": "full_l2", "c5": "full_l3",
+                    "c2-layer": "full_l2", "c4-layer": "full_l2"}
+
+
+def kernel_source_hash(kernel="", workload="c2"):
+    """Hash of the sources a kernel is built from: the edge-kernel templates and the generated
+    body of the workload's path list (uvw: also its GEMM), or the transpose's own file."""
+    csrc = os.path.join(ROOT, "equivariant_tensor_product_b200", "csrc")
+    if kernel.startswith("k_radix") or kernel.startswith("k_colptr"):
+        files = [os.path.join(csrc, "csr.cu")]
+    else:
+        files = [os.path.join(csrc, "tp_kernels.cuh")]
+        if "uvw" in kernel or "gemm" in kernel:
+            files += [os.path.join(csrc, "tp_uvw.cuh"), os.path.join(csrc, "tp_mma.cuh")]
+        spec = SPEC_OF_WORKLOAD.get(workload)
+        gen = os.path.join(csrc, "gen", f"spec_{spec}.h")
+        if spec and not os.path.exists(gen):
+            sys.path.insert(0, csrc)
+            import codegen
+            sys.path.pop(0)
+            codegen.main(os.path.join(csrc, "gen"))
+        if spec:
+            files.append(gen)
     h = hashlib.sha256()
-    for f in ("tp_kernels.cuh", "tp_common.h", "csr.cu", "codegen.py"):
-        with open(os.path.join(ROOT, "equivariant_tensor_product_b200", "csrc", f), "rb") as fh:
+    for f in files:
+        with open(f, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
@@ -372,7 +394,7 @@ def traffic_from_profile(kernel, workload):
     try:
         rec = json.load(open(path))
         e = rec.get(workload, {}).get(kernel)
-        if e and e.get("source_hash") == kernel_source_hash():
+        if e and e.get("source_hash") == kernel_source_hash(kernel, workload):
             return e["dram_bytes_per_launch"]
     except Exception:  # noqa: BLE001
         return None
