@@ -21,6 +21,11 @@ coupling, graph aggregation) and "The GPU Workload That Rewrites Molecular Physi
 products).  Backward and double backward are the vector-Jacobian products of this map
 ("Sobek", abstract: forward, backward and double backward), taken by torch autograd.
 
+``oracle.gaunt`` holds the second operator, the spherical-grid (Gaunt) tensor-product
+convolution ("The Price of Freedom: Exploring Expressivity and Runtime Tradeoffs in
+Equivariant Tensor Products", abstract), with its Gaunt coefficients integrated on an exact
+quadrature grid and pinned against sympy's closed form.
+
 Pins (tests/test_oracle_*.py): SH against scipy's complex spherical harmonics and the
 addition theorem; Wigner-D group law; CG against sympy's Clebsch-Gordan coefficients,
 orthogonality and equivariance; operator equivariance, parity, the l=0 case against
