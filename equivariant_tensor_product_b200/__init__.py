@@ -14,3 +14,4 @@ from .ops import (Plan, tp_conv_bwd, tp_conv_dbwd, tp_conv_fwd, tp_csr_transpose
 from .autograd import GateFn, LinearFn, TPConv, tp_conv, tp_gate, tp_linear  # noqa: F401
 from .block import (Gate, Linear, tp_gate_bwd, tp_gate_dbwd, tp_gate_fwd, tp_linear_bwd, tp_linear_fwd,  # noqa: F401
                     tp_linear_workspace_size)
+from .gaunt import Gaunt, tp_gaunt_bwd, tp_gaunt_fwd, tp_gaunt_workspace_size  # noqa: F401

@@ -40,6 +40,13 @@ SIGNATURES = {
     "tp_version": (C.c_char_p, []),
     "tp_launch_count": (C.c_int64, []),
     "tp_check_bounded_waits": (C.c_int, [_i64, _p, C.POINTER(_i32)]),
+    # the spherical-grid (Gaunt) convolution (include/tp_gaunt.h)
+    "tp_gaunt_create": (C.c_int, [C.POINTER(_p), C.c_char_p, _i32, C.c_char_p]),
+    "tp_gaunt_destroy": (C.c_int, [_p]),
+    "tp_gaunt_query": (C.c_int, [_p, C.POINTER(_i64), C.POINTER(_i64), C.POINTER(_i64), C.POINTER(_i32)]),
+    "tp_gaunt_workspace_size": (C.c_int, [_p, _i64, _i64, _i32, C.POINTER(_sz)]),
+    "tp_gaunt_fwd": (C.c_int, [_p, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "tp_gaunt_bwd": (C.c_int, [_p, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     # node-side operators (include/tp_block.h)
     "tp_linear_create": (C.c_int, [C.POINTER(_p), C.c_char_p, C.c_char_p, _p, C.c_uint32]),
     "tp_linear_destroy": (C.c_int, [_p]),

@@ -939,6 +939,84 @@ def gen_generic_header() -> str:
 
 
 # ---------------------------------------------------------------------------
+# Spherical grid of the Gaunt (grid) convolution
+# ---------------------------------------------------------------------------
+
+def _gauss_legendre(n: int):
+    """Nodes and weights of n-point Gauss-Legendre on [-1, 1], by Newton's iteration on P_n
+    from the Chebyshev guesses (the textbook recurrence; float64)."""
+    nodes, weights = [], []
+    for k in range(n):
+        t = math.cos(math.pi * (k + 0.75) / (n + 0.5))
+        for _ in range(100):
+            p0, p1 = 1.0, t
+            for j in range(2, n + 1):
+                p0, p1 = p1, ((2 * j - 1) * t * p1 - (j - 1) * p0) / j
+            dp = n * (t * p1 - p0) / (t * t - 1.0) if n > 1 else 1.0
+            step = p1 / dp
+            t -= step
+            if abs(step) < 1e-16:
+                break
+        p0, p1 = 1.0, t
+        for j in range(2, n + 1):
+            p0, p1 = p1, ((2 * j - 1) * t * p1 - (j - 1) * p0) / j
+        dp = n * (t * p1 - p0) / (t * t - 1.0) if n > 1 else 1.0
+        nodes.append(t)
+        weights.append(2.0 / ((1.0 - t * t) * dp * dp))
+    return nodes, weights
+
+
+def _poly_value(p: Poly, x: float, y: float, z: float) -> float:
+    return sum(c * x ** i * y ** j * z ** k for (i, j, k), c in p.items())
+
+
+def gaunt_grid(L: int):
+    """Points (x, y, z), weights summing to 1 and the harmonics of degrees 0..L at every point,
+    for a grid that integrates polynomials of degree <= 3 L exactly on the sphere (products
+    of three degree-L functions): ceil((3L+1)/2) Gauss-Legendre nodes in cos(theta) times
+    3L+1 equispaced azimuths."""
+    D = 3 * L
+    n_t, n_p = D // 2 + 1, D + 1
+    nodes, wts = _gauss_legendre(n_t)
+    polys = sh_polys()
+    pts, q, Y = [], [], []
+    for t, a in zip(nodes, wts):
+        st = math.sqrt(max(0.0, 1.0 - t * t))
+        for j in range(n_p):
+            ph = 2.0 * math.pi * j / n_p
+            x, y, z = st * math.cos(ph), st * math.sin(ph), t
+            pts.append((x, y, z))
+            q.append(a / (2.0 * n_p))
+            Y.append([_poly_value(polys[l][m], x, y, z) for l in range(L + 1) for m in range(2 * l + 1)])
+    return pts, q, Y
+
+
+def gen_gaunt_header() -> str:
+    L_ = ["// Generated by codegen.py.  Do not edit.",
+          "// Spherical grids of the Gaunt (grid) convolution: for L = 1, 2, 3 the points, quadrature weights",
+          "// (summing to 1) and the real spherical harmonics of degrees 0..L at the points, exact for",
+          "// polynomials of degree 3L on the sphere.",
+          "#pragma once",
+          "namespace tp {",
+          "namespace gaunt {",
+          "template <int L> struct Grid;"]
+    for Lg in (1, 2, 3):
+        pts, q, Y = gaunt_grid(Lg)
+        ng, nsh = len(pts), (Lg + 1) ** 2
+        L_.append(f"template <> struct Grid<{Lg}> {{")
+        L_.append(f"  static constexpr int NG = {ng}, NSH = {nsh};")
+        for name, vals in (("px", [p[0] for p in pts]), ("py", [p[1] for p in pts]), ("pz", [p[2] for p in pts]), ("q", q)):
+            L_.append(f"  __device__ __forceinline__ static float {name}(int g) {{ constexpr float v[{ng}] = {{"
+                      + ", ".join(_flt(v) for v in vals) + "}; return v[g]; }")
+        flat = [Y[g][k] for g in range(ng) for k in range(nsh)]
+        L_.append(f"  __device__ __forceinline__ static float Y(int g, int k) {{ constexpr float v[{ng * nsh}] = {{"
+                  + ", ".join(_flt(v) for v in flat) + f"}}; return v[g * {nsh} + k]; }}")
+        L_.append("};")
+    L_ += ["}  // namespace gaunt", "}  // namespace tp"]
+    return "\n".join(L_) + "\n"
+
+
+# ---------------------------------------------------------------------------
 # The compiled specialisations
 # ---------------------------------------------------------------------------
 
@@ -1037,6 +1115,7 @@ def main(outdir: str):
     reg.append("}  // namespace tp")
     write("registry.cu", "\n".join(reg) + "\n")
     write("generic_cg.h", gen_generic_header())
+    write("gaunt_grid.h", gen_gaunt_header())
     # CG table dump (text) for the host-side table tests
     lines = []
     for l1, l2, l3 in product(range(4), repeat=3):

@@ -244,3 +244,21 @@ def test_missing_library_fails_loudly_on_first_call(tmp_path):
     ) % (ROOT, str(tmp_path / "libtp.so"))
     out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
     assert "ImportError" in out.stdout and "libtp.so is missing" in out.stdout, (out.stdout, out.stderr)
+
+
+def test_gaunt_plan_contract(tp):
+    g = tp.Gaunt("32x0e+32x1o+32x2e", 2, "32x0e+32x1o+32x2e")
+    assert (g.in_dim, g.out_dim, g.n_edge_weights, g.grid_points) == (288, 288, 96, 28)
+    assert tp.Gaunt("4x1o", 1, "4x0e").grid_points == 8
+    assert tp.Gaunt("4x3o", 0, "4x3o").grid_points == 50
+    N, E = 1000, 30000
+    f = tp.tp_gaunt_workspace_size(g, N, E, tp.TP_OP_FWD)
+    b = tp.tp_gaunt_workspace_size(g, N, E, tp.TP_OP_BWD)
+    assert 4 * N * 28 * 32 <= f <= 4 * N * 28 * 32 + 256            # node sized
+    assert b <= 2 * f + 12 * E + 8 * (N + 1) + 4 * 2 * 2048 + 1024
+    for args, status in ((("4x1e", 1, "4x0e"), 1), (("4x0e+8x1o", 1, "4x0e"), 1), (("4x0e", 1, "8x0e"), 1),
+                         (("4x4e", 1, "4x0e"), 2), (("4x0e", 4, "4x0e"), 2), (("256x0e", 1, "256x0e"), 2),
+                         (("4x1o+4x0e", 1, "4x0e"), 1)):
+        with pytest.raises(tp.TPError) as e:
+            tp.Gaunt(*args)
+        assert e.value.status == status, args
