@@ -45,6 +45,9 @@ WORKLOADS = {
                 "convolution (c2 paths), linear with coefficient 1/average degree -> 32x0e+64x0e+32x1o+32x2e, gate "
                 "-> 32x(0e,1o,2e); step = that forward + transpose + the backward to x, both linear weights and "
                 "the edge weights",
+    "c2-gaunt": "spherical-grid (Gaunt) convolution on the c2 graph (1,536 atoms, 46,080 edges): 32x0e+32x1o+32x2e "
+                "-> same, edge filter degrees 0..2 with per-degree radial weights, 28-point grid; step = fwd + "
+                "transpose + bwd(gx, gw)",
     "c4-layer": "interaction layer on the c4 graph (100,000 atoms, ~3.0M edges): linear 128x(0e,1o,2e) -> same, uvw "
                 "convolution (c4 paths, 128x128 mixing), linear with coefficient 1/average degree -> "
                 "128x0e+256x0e+128x1o+128x2e, gate -> 128x(0e,1o,2e); step = that forward + transpose + the backward "
@@ -323,6 +326,8 @@ def run_reference(args, rank):
     cores = set_threads()
     if args.workload.endswith("-layer"):
         return run_reference_layer(args, cores)
+    if args.workload == "c2-gaunt":
+        return run_reference_gaunt(args, cores)
     d = synth.make_inputs(args.workload)
     oracle_sample(d, 4, seed=0)                      # CG tables cached outside the timing
     ef, tf, eb, tb = oracle_sample(d, 16, seed=1)
@@ -927,6 +932,51 @@ def layer_weights(spec, N, n_w1, n_w2, out_dim, rank=0):
     return W1, W2, g_out
 
 
+def run_reference_gaunt(args, cores):
+    """The float64 oracle of the Gaunt convolution on sampled receivers of the c2 graph."""
+    import synth
+    from oracle.gaunt import GauntPlan, gaunt_backward, gaunt_forward
+    d = synth.make_inputs("c2")
+    N = len(d["rowptr"]) - 1
+    op = GauntPlan(*GAUNT_SPEC)
+    rng = np.random.default_rng(1029)
+    x = rng.standard_normal((N, op.in_dim))
+    rp = np.asarray(d["rowptr"], dtype=np.int64)
+
+    def sample(n_rows, seed):
+        rows = np.sort(np.random.default_rng(seed).choice(N, size=n_rows, replace=False))
+        eids = np.concatenate([np.arange(rp[i], rp[i + 1]) for i in rows])
+        rpf = np.concatenate([[0], np.cumsum(rp[rows + 1] - rp[rows])])
+        w = rng.standard_normal((len(eids), op.nw))
+        gy = rng.standard_normal((n_rows, op.out_dim))
+        t0 = time.perf_counter()
+        gaunt_forward(op, rpf, d["src"][eids], x, d["vec"][eids], w)
+        gaunt_backward(op, rpf, d["src"][eids], x, d["vec"][eids], w, gy)
+        return len(eids), time.perf_counter() - t0
+
+    sample(4, 0)
+    e, t = sample(16, 1)
+    rows = int(max(2, min(512, 16 * 60.0 / max(1, args.steps + args.warmup) / max(t, 1e-3))))
+    for k in range(args.warmup):
+        sample(rows, 100 + k)
+    tot_e = tot_t = 0.0
+    for k in range(args.steps):
+        e, t = sample(rows, 1000 + k)
+        tot_e += e
+        tot_t += t
+    value = tot_e / tot_t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOADS["c2-gaunt"], "name": "c2-gaunt", "N": N, "E": len(d["src"]),
+                       "parallelism": "single"},
+            "cpu_baseline": {"value": value, "unit": "edges/s", "cores": cores, "kind": "oracle",
+                             "sample": f"fwd + bwd on the edges into {rows} random receivers per step, float64"},
+            "e2e": {"value": value, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference_layer(args, cores):
     import synth
     from oracle.block import GateSpec, linear_weight_count
@@ -1311,6 +1361,200 @@ def run_latency(args, rank, world, local):
     return 0
 
 
+GAUNT_SPEC = ("32x0e+32x1o+32x2e", 2, "32x0e+32x1o+32x2e")
+
+
+def gaunt_counts(N, E, mul, ng, d_in, d_out, lmax_sh):
+    """Algorithmic bytes and flops of the Gaunt convolution (fwd, bwd).  Bytes: the operator's
+    inputs and outputs (as fwd_bytes / bwd_bytes, w being (lmax_sh + 1) x mul per edge; the
+    node grids are workspace, not counted).  Flops of the grid method, per edge and channel:
+    the filter on the grid (2 (lmax_sh + 1) per point) and the product-accumulate (2 per point),
+    plus per edge the dot products r_hat . r_g and the Legendre values (2 (3 + lmax_sh) per point,
+    shared by the channels); per node and channel the transforms to and from the grid (2 ng d_in
+    and 2 ng d_out).  The backward counts the grid transforms of x and gy, the filter, the
+    accumulation of gF, the weight gradient (2 (lmax_sh + 1) per point) and the direction terms
+    (10 per point)."""
+    nw = (lmax_sh + 1) * mul
+    fb = E * (4 + 12 + 4 * nw) + 4 * N * (d_in + d_out) + 4 * (N + 1)
+    bb = E * (4 + 12 + 8 * nw) + 4 * N * (2 * d_in + d_out) + 8 * (N + 1)
+    per_edge_geo = ng * 2 * (3 + lmax_sh)
+    ff = E * (mul * ng * (2 * (lmax_sh + 1) + 2) + per_edge_geo) + N * mul * 2 * ng * (d_in + d_out)
+    bf = E * (mul * ng * (2 * (lmax_sh + 1) + 2 + 2 * (lmax_sh + 1) + 2 + 10) + per_edge_geo) + \
+        N * mul * 2 * ng * (2 * d_in + d_out)
+    return fb, bb, ff, bf
+
+
+def run_gaunt(args, rank, world, local):
+    """The spherical-grid (Gaunt) convolution on the c2 graph: forward, the transpose on a
+    side stream, backward (gx, gw), through include/tp_gaunt.h, timed as the convolution
+    workloads are (rotating inputs > 2 x L2, CUDA graphs, end to end with host copies)."""
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from equivariant_tensor_product_b200 import build as tpbuild
+    tpbuild.build()
+    import equivariant_tensor_product_b200 as tp
+    import synth
+    lib = tp.load()
+    spec = synth.CONFIGS["c2"]
+    d = synth.make_inputs("c2", args.n_atoms, seed=spec.seed + 7919 * rank)
+    N, E = len(d["rowptr"]) - 1, len(d["src"])
+    g = tp.Gaunt(*GAUNT_SPEC)
+    rng = np.random.default_rng(spec.seed + 29 + 7919 * rank)
+    mul = int(GAUNT_SPEC[0].split("x")[0])
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copy_bytes = 4 * (N * (g.in_dim + g.out_dim) + E * (g.n_edge_weights + 4)) + 4 * (N + 1)
+    R = max(2, math.ceil(2.5 * l2 / copy_bytes))
+    copies = []
+    for r in range(R):
+        cp = {"rowptr": d["rowptr"], "src": d["src"], "vec": d["vec"],
+              "x": rng.standard_normal((N, g.in_dim), dtype=np.float32),
+              "w": rng.standard_normal((E, g.n_edge_weights), dtype=np.float32),
+              "gy": rng.standard_normal((N, g.out_dim), dtype=np.float32)}
+        copies.append({k: torch.as_tensor(np.ascontiguousarray(v)).to(dev) for k, v in cp.items()})
+    y = torch.empty(N, g.out_dim, device=dev)
+    gx = torch.empty(N, g.in_dim, device=dev)
+    gw = torch.empty(E, g.n_edge_weights, device=dev)
+    wsf = torch.empty(tp.tp_gaunt_workspace_size(g, N, E, tp.TP_OP_FWD), dtype=torch.uint8, device=dev)
+    wsb = torch.empty(tp.tp_gaunt_workspace_size(g, N, E, tp.TP_OP_BWD), dtype=torch.uint8, device=dev)
+    wst_bytes = max(256, tp.tp_csr_transpose_workspace_size(N, E))
+    wst = torch.empty(wst_bytes, dtype=torch.uint8, device=dev)
+    colptrs = [torch.empty(N + 1, dtype=torch.int32, device=dev) for _ in range(R)]
+    perms = [torch.empty(E, dtype=torch.int32, device=dev) for _ in range(R)]
+    stream, side = torch.cuda.Stream(dev), torch.cuda.Stream(dev, priority=-1)
+    sh, sh_side = stream.cuda_stream, side.cuda_stream
+    P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None
+    ff_, tf_, bf_ = lib.tp_gaunt_fwd, lib.tp_csr_transpose, lib.tp_gaunt_bwd
+    args_r = []
+    for r, cp in enumerate(copies):
+        args_r.append(((g.handle, N, E, P(cp["rowptr"]), P(cp["src"]), P(cp["x"]), P(cp["vec"]), P(cp["w"]), P(y),
+                        P(wsf), wsf.numel(), sh),
+                       (N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(wst), wst_bytes, sh_side),
+                       (g.handle, N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(cp["x"]),
+                        P(cp["vec"]), P(cp["w"]), P(cp["gy"]), P(gx), P(gw), None, P(wsb), wsb.numel(), sh)))
+    tr_done = [torch.cuda.Event() for _ in range(R)]
+    bwd_done = [torch.cuda.Event() for _ in range(R)]
+
+    def step(k, ev=None):
+        r = k % R
+        a_f, a_t, a_b = args_r[r]
+        side.wait_event(bwd_done[r])
+        st = tf_(*a_t)
+        tr_done[r].record(side)
+        if ev is not None:
+            ev[0].record(stream)
+        st |= ff_(*a_f)
+        if ev is not None:
+            ev[1].record(stream)
+        stream.wait_event(tr_done[r])
+        if ev is not None:
+            ev[2].record(stream)
+        st |= bf_(*a_b)
+        if ev is not None:
+            ev[3].record(stream)
+        bwd_done[r].record(stream)
+        if st:
+            raise RuntimeError(lib.tp_last_error_message().decode())
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    n0 = lib.tp_launch_count()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            step(k, evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    launches = lib.tp_launch_count() - n0
+    elapsed_max = max_over_ranks(start.elapsed_time(stop) / 1e3, world, dev)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    # end to end: inputs up from pinned memory, outputs down, every step (sequential copies)
+    host = {k: torch.as_tensor(np.ascontiguousarray(v.cpu().numpy())).pin_memory() for k, v in copies[0].items()}
+    hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (y, gx, gw)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for k in range(args.e2e_steps):
+            for key in host:
+                copies[0][key].copy_(host[key], non_blocking=True)
+            side.wait_stream(stream)
+            step(0)
+            stream.wait_stream(side)
+            for ho, t in zip(hout, (y, gx, gw)):
+                ho.copy_(t, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+    if rank == 0:
+        hbm, _, peak_note = measured_peaks()
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        fp32_peak = 2 * 128 * sms * clk.max_mhz_or(1965.0) * 1e6 / 1e12
+        d_in = sum(2 * int(t.split("x")[1][:-1]) + 1 for t in GAUNT_SPEC[0].split("+"))
+        d_out = sum(2 * int(t.split("x")[1][:-1]) + 1 for t in GAUNT_SPEC[2].split("+"))
+        fb, bb, fl_f, fl_b = gaunt_counts(N, E, mul, g.grid_points, d_in, d_out, GAUNT_SPEC[1])
+        passes = {"fwd": pass_roofline(fwd_ms, fb, fl_f, hbm, fp32_peak),
+                  "bwd": pass_roofline(bwd_ms, bb, fl_b, hbm, fp32_peak)}
+        dom = max(passes, key=lambda k: passes[k]["ms"])
+        dp = passes[dom]
+        kname = {"fwd": "k_gaunt_fwd", "bwd": "k_gaunt_bwd"}[dom]
+        if dp["bound"] == "hbm":
+            roof = {"bound": "hbm", "kernel": kname, "achieved": dp["achieved_GBps"], "peak": hbm, "unit": "GB/s",
+                    "frac": dp["achieved_GBps"] / hbm, "peak_note": peak_note}
+        else:
+            roof = {"bound": "alu", "kernel": kname, "achieved": dp["achieved_fp32_TFLOPs"], "peak": fp32_peak,
+                    "unit": "TFLOP/s", "frac": dp["achieved_fp32_TFLOPs"] / fp32_peak,
+                    "peak_note": "fp32 FMA peak; flops of the grid method by bench.gaunt_counts"}
+        roof.update({"traffic": traffic_from_profile(kname, "c2-gaunt"), "passes": passes,
+                     "kernel_ms": {"fwd": fwd_ms, "bwd": bwd_ms}})
+        cpu = None
+        if not args.no_cpu_baseline:
+            from oracle.conv import set_threads
+            from oracle.gaunt import GauntPlan, gaunt_backward, gaunt_forward
+            cores = set_threads()
+            op = GauntPlan(*GAUNT_SPEC)
+            rows = np.sort(np.random.default_rng(3).choice(N, size=min(N, 256), replace=False))
+            rp = np.asarray(d["rowptr"], dtype=np.int64)
+            eids = np.concatenate([np.arange(rp[i], rp[i + 1]) for i in rows])
+            rpf = np.concatenate([[0], np.cumsum(rp[rows + 1] - rp[rows])])
+            xs, ws_, gys = (copies[0][k].cpu().numpy() for k in ("x", "w", "gy"))
+            t0 = time.perf_counter()
+            gaunt_forward(op, rpf, d["src"][eids], xs, d["vec"][eids], ws_[eids])
+            gaunt_backward(op, rpf, d["src"][eids], xs, d["vec"][eids], ws_[eids], gys[rows])
+            t1 = time.perf_counter()
+            cpu = {"value": len(eids) / (t1 - t0), "unit": "edges/s", "cores": cores, "kind": "oracle",
+                   "sample": f"fwd + bwd on the {len(eids)} edges into 256 random receivers, float64, {t1 - t0:.1f} s"}
+        line = {"metric": METRIC, "value": replica_throughput(E, args.steps, world, elapsed_max), "unit": "edges/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * elapsed_max / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOADS["c2-gaunt"], "name": "c2-gaunt", "N": N, "E": E, "launch": "eager",
+                           "grid_points": g.grid_points,
+                           "l2": f"{R} rotating input copies of {copy_bytes / 1e6:.1f} MB (> 2x L2 of {l2 / 1e6:.0f} MB)",
+                           "parallelism": "replicas" if world > 1 else "single"},
+                "roofline": roof, "cpu_baseline": cpu,
+                "e2e": {"value": E * args.e2e_steps / e2e_s, "unit": "edges/s",
+                        "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host.values()),
+                        "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout),
+                        "steps": args.e2e_steps},
+                "gpu_launches": int(launches), "clocks": clk.summary(), "library": tp.tp_version()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
@@ -1318,6 +1562,8 @@ def main():
         return run_reference(args, rank)
     if args.workload == "c1":
         return run_latency(args, rank, world, local)
+    if args.workload == "c2-gaunt":
+        return run_gaunt(args, rank, world, local)
     if args.workload.endswith("-layer"):
         return run_layer(args, rank, world, local)
     return run_ours(args, rank, world, local)

@@ -1008,6 +1008,16 @@ def gen_gaunt_header() -> str:
         for name, vals in (("px", [p[0] for p in pts]), ("py", [p[1] for p in pts]), ("pz", [p[2] for p in pts]), ("q", q)):
             L_.append(f"  __device__ __forceinline__ static float {name}(int g) {{ constexpr float v[{ng}] = {{"
                       + ", ".join(_flt(v) for v in vals) + "}; return v[g]; }")
+        # the grid is a product: point g = k * NP + j has cos(theta) = ct(k), azimuth phi_j
+        D = 3 * Lg
+        n_t, n_p = D // 2 + 1, D + 1
+        nodes, _ = _gauss_legendre(n_t)
+        L_.append(f"  static constexpr int NT = {n_t}, NP = {n_p};")
+        for name, vals in (("ct", nodes), ("st", [math.sqrt(max(0.0, 1.0 - t * t)) for t in nodes]),
+                           ("cp", [math.cos(2.0 * math.pi * j / n_p) for j in range(n_p)]),
+                           ("sp", [math.sin(2.0 * math.pi * j / n_p) for j in range(n_p)])):
+            L_.append(f"  __device__ __forceinline__ static float {name}(int i) {{ constexpr float v[{len(vals)}] = {{"
+                      + ", ".join(_flt(v) for v in vals) + "}; return v[i]; }")
         flat = [Y[g][k] for g in range(ng) for k in range(nsh)]
         L_.append(f"  __device__ __forceinline__ static float Y(int g, int k) {{ constexpr float v[{ng * nsh}] = {{"
                   + ", ".join(_flt(v) for v in flat) + f"}}; return v[g * {nsh} + k]; }}")

@@ -34,6 +34,7 @@ namespace {
 
 struct GauntArgs {
   int N, E, mul, lmax_sh, nw, in_dim, out_dim, nsl;
+  int split;                   // warps that split a node's edges (nsl * split <= 4)
   int in_off[4], out_off[4];   // offset of the block of degree l in a row, -1 when absent
   const int32_t *rowptr, *src, *colptr, *perm;
   const float *x, *vec, *w, *gy;
@@ -41,17 +42,28 @@ struct GauntArgs {
   float *y, *gx, *gw, *gvec;
 };
 
-// (2l+1) P_l(t) and its derivative for l = 0..3
-__device__ __forceinline__ void legendre_weighted(float t, float (&E)[4], float (&dE)[4]) {
-  const float t2 = t * t;
-  E[0] = 1.f;
-  E[1] = 3.f * t;
-  E[2] = 5.f * fmaf(1.5f, t2, -0.5f);
-  E[3] = 7.f * t * fmaf(2.5f, t2, -1.5f);
-  dE[0] = 0.f;
-  dE[1] = 3.f;
-  dE[2] = 15.f * t;
-  dE[3] = 7.f * fmaf(7.5f, t2, -1.5f);
+// The filter sum_l w_l (2l+1) P_l(t) as a cubic in t: a0 + a1 t + a2 t^2 + a3 t^3
+// (3 P_1 = 3t, 5 P_2 = 7.5 t^2 - 2.5, 7 P_3 = 17.5 t^3 - 10.5 t).
+__device__ __forceinline__ void filter_cubic(const float (&wl)[4], float (&c)[4]) {
+  c[0] = fmaf(-2.5f, wl[2], wl[0]);
+  c[1] = fmaf(-10.5f, wl[3], 3.f * wl[1]);
+  c[2] = 7.5f * wl[2];
+  c[3] = 17.5f * wl[3];
+}
+
+// t_g = r_hat . r_g for every grid point, from the grid's product structure: r_g has
+// cos(theta) = ct(k), sin(theta) = st(k) and azimuth phi_j, so t = rz ct(k) + st(k) (rx cos phi_j + ry sin phi_j).
+template <class Gr>
+__device__ __forceinline__ void grid_dots(float rx, float ry, float rz, float (&t)[Gr::NG]) {
+  float c[Gr::NP];
+#pragma unroll
+  for (int j = 0; j < Gr::NP; ++j) c[j] = fmaf(rx, Gr::cp(j), ry * Gr::sp(j));
+#pragma unroll
+  for (int k = 0; k < Gr::NT; ++k) {
+    const float z = rz * Gr::ct(k);
+#pragma unroll
+    for (int j = 0; j < Gr::NP; ++j) t[k * Gr::NP + j] = fmaf(Gr::st(k), c[j], z);
+  }
 }
 
 // MODE 0: F from x (input blocks); MODE 1: Gq from gy (output blocks, times q_g).  One thread
@@ -91,10 +103,16 @@ __device__ __forceinline__ void edge_weights(const GauntArgs& a, int e, int u, b
     wl[l] = (act && l <= a.lmax_sh && (l == 0 || ir > 0.f)) ? __ldg(a.w + (int64_t)e * a.nw + l * a.mul + u) : 0.f;
 }
 
+// Forward: CTA = one receiver; warp w = (slice w / split, phase w % split); the phases take
+// interleaved edges of the row and their grid accumulators are added through shared memory in
+// phase order.  Each edge's grid row F[src][.][u] is loaded in one batch before the pointwise
+// math.
 template <int L>
 __global__ void __launch_bounds__(128) k_gaunt_fwd(const __grid_constant__ GauntArgs a) {
   using Gr = gaunt::Grid<L>;
-  const int lane = threadIdx.x & 31, sl = threadIdx.x >> 5;
+  extern __shared__ float red[];             // [(split-1) * nsl][NG][32]
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int st = a.split, sl = wid / st, phase = wid - sl * st;
   const int i = blockIdx.x;
   const int u = sl * 32 + lane;
   const bool act = u < a.mul;
@@ -102,8 +120,8 @@ __global__ void __launch_bounds__(128) k_gaunt_fwd(const __grid_constant__ Gaunt
   float acc[Gr::NG];
 #pragma unroll
   for (int g = 0; g < Gr::NG; ++g) acc[g] = 0.f;
-  for (int base = e0; base < e1; base += 32) {
-    const int my_e = base + lane;
+  for (int base = e0 + phase; base < e1; base += 32 * st) {
+    const int my_e = base + lane * st;
     int my_j = 0;
     float vx = 0.f, vy = 0.f, vz = 0.f;
     if (my_e < e1) {
@@ -112,26 +130,76 @@ __global__ void __launch_bounds__(128) k_gaunt_fwd(const __grid_constant__ Gaunt
       vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
       vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
     }
-    const int ne = min(32, e1 - base);
-    for (int k = 0; k < ne; ++k) {
-      const int j = __shfl_sync(kFull, my_j, k);
-      float rx, ry, rz, ir;
-      edge_geometry(__shfl_sync(kFull, vx, k), __shfl_sync(kFull, vy, k), __shfl_sync(kFull, vz, k), rx, ry, rz, ir);
-      if (!act) continue;
-      float wl[4];
-      edge_weights(a, base + k, u, act, ir, wl);
-      const float* Fr = a.F + (int64_t)j * Gr::NG * a.mul + u;
+    const int ne = min(32, (e1 - base + st - 1) / st);
+    if constexpr (Gr::NG <= 32) {
+      // small grids: the row of edge k + 1 is loaded while edge k is computed (a larger grid
+      // would not fit two rows in registers)
+      float fn[Gr::NG];
+      {
+        const int j0 = __shfl_sync(kFull, my_j, 0);
 #pragma unroll
-      for (int g = 0; g < Gr::NG; ++g) {
-        const float t = fmaf(rx, Gr::px(g), fmaf(ry, Gr::py(g), rz * Gr::pz(g)));
-        float E[4], dE[4];
-        legendre_weighted(t, E, dE);
-        const float s = fmaf(wl[3], E[3], fmaf(wl[2], E[2], fmaf(wl[1], E[1], wl[0])));
-        acc[g] = fmaf(__ldg(Fr + (int64_t)g * a.mul), s, acc[g]);
+        for (int g = 0; g < Gr::NG; ++g) fn[g] = act ? __ldg(a.F + ((int64_t)j0 * Gr::NG + g) * a.mul + u) : 0.f;
+      }
+      for (int k = 0; k < ne; ++k) {
+        float f[Gr::NG];
+#pragma unroll
+        for (int g = 0; g < Gr::NG; ++g) f[g] = fn[g];
+        const int jn = __shfl_sync(kFull, my_j, min(k + 1, 31));
+        if (act && k + 1 < ne) {
+#pragma unroll
+          for (int g = 0; g < Gr::NG; ++g) fn[g] = __ldg(a.F + ((int64_t)jn * Gr::NG + g) * a.mul + u);
+        }
+        float rx, ry, rz, ir;
+        edge_geometry(__shfl_sync(kFull, vx, k), __shfl_sync(kFull, vy, k), __shfl_sync(kFull, vz, k), rx, ry, rz, ir);
+        if (!act) continue;
+        float wl[4], cf[4], tg[Gr::NG];
+        edge_weights(a, base + k * st, u, act, ir, wl);
+        filter_cubic(wl, cf);
+        grid_dots<Gr>(rx, ry, rz, tg);
+#pragma unroll
+        for (int g = 0; g < Gr::NG; ++g) {
+          const float s = fmaf(fmaf(fmaf(cf[3], tg[g], cf[2]), tg[g], cf[1]), tg[g], cf[0]);
+          acc[g] = fmaf(f[g], s, acc[g]);
+        }
+      }
+    } else {
+      for (int k = 0; k < ne; ++k) {
+        const int j = __shfl_sync(kFull, my_j, k);
+        float rx, ry, rz, ir;
+        edge_geometry(__shfl_sync(kFull, vx, k), __shfl_sync(kFull, vy, k), __shfl_sync(kFull, vz, k), rx, ry, rz, ir);
+        if (!act) continue;
+        float wl[4], cf[4], tg[Gr::NG];
+        edge_weights(a, base + k * st, u, act, ir, wl);
+        filter_cubic(wl, cf);
+        const float* Fr = a.F + (int64_t)j * Gr::NG * a.mul + u;
+        float f[Gr::NG];
+#pragma unroll
+        for (int g = 0; g < Gr::NG; ++g) f[g] = __ldg(Fr + (int64_t)g * a.mul);
+        grid_dots<Gr>(rx, ry, rz, tg);
+#pragma unroll
+        for (int g = 0; g < Gr::NG; ++g) {
+          const float s = fmaf(fmaf(fmaf(cf[3], tg[g], cf[2]), tg[g], cf[1]), tg[g], cf[0]);
+          acc[g] = fmaf(f[g], s, acc[g]);
+        }
       }
     }
   }
-  if (!act) return;
+  if (st > 1) {
+    if (phase > 0) {
+      float* dst = red + (((size_t)(phase - 1) * a.nsl + sl) * Gr::NG) * 32 + lane;
+#pragma unroll
+      for (int g = 0; g < Gr::NG; ++g) dst[g * 32] = acc[g];
+    }
+    __syncthreads();
+    if (phase == 0) {
+      for (int ph = 1; ph < st; ++ph) {
+        const float* srcp = red + (((size_t)(ph - 1) * a.nsl + sl) * Gr::NG) * 32 + lane;
+#pragma unroll
+        for (int g = 0; g < Gr::NG; ++g) acc[g] += srcp[g * 32];
+      }
+    }
+  }
+  if (!act || phase != 0) return;
   float* yr = a.y + (int64_t)i * a.out_dim;
 #pragma unroll
   for (int l = 0; l <= L; ++l) {
@@ -146,11 +214,14 @@ __global__ void __launch_bounds__(128) k_gaunt_fwd(const __grid_constant__ Gaunt
   }
 }
 
+// Backward: CTA = one sender, warps as in the forward, out-edges in the stable transpose order.
 template <int L>
 __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ GauntArgs a) {
   using Gr = gaunt::Grid<L>;
-  __shared__ float part[32][4][4];   // per edge of a batch and slice: the gvec partial sums
-  const int lane = threadIdx.x & 31, sl = threadIdx.x >> 5;
+  extern __shared__ float red[];             // [(split-1) * nsl][NG][32]
+  __shared__ float part[4][32][4][4];        // [phase][edge of the batch][slice][4]: gvec partials
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int st = a.split, sl = wid / st, phase = wid - sl * st;
   const int j = blockIdx.x;
   const int u = sl * 32 + lane;
   const bool act = u < a.mul;
@@ -162,8 +233,8 @@ __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ Gaunt
     Fj[g] = act ? __ldg(Fr + (int64_t)g * a.mul) : 0.f;
     gF[g] = 0.f;
   }
-  for (int base = q0; base < q1; base += 32) {
-    const int my_q = base + lane;
+  for (int base = q0 + phase; base < q1; base += 32 * st) {
+    const int my_q = base + lane * st;
     int my_e = 0, my_i = 0;
     float vx = 0.f, vy = 0.f, vz = 0.f;
     if (my_q < q1) {
@@ -173,7 +244,7 @@ __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ Gaunt
       vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
       vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
     }
-    const int ne = min(32, q1 - base);
+    const int ne = min(32, (q1 - base + st - 1) / st);
     for (int k = 0; k < ne; ++k) {
       const int e = __shfl_sync(kFull, my_e, k), i = __shfl_sync(kFull, my_i, k);
       float rx, ry, rz, ir;
@@ -183,24 +254,35 @@ __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ Gaunt
       float gw[4] = {0.f, 0.f, 0.f, 0.f};
       float hx = 0.f, hy = 0.f, hz = 0.f, hs = 0.f;
       if (act) {
-        const float* Gr_ = a.Gq + (int64_t)i * Gr::NG * a.mul + u;
+        const float* Gp = a.Gq + (int64_t)i * Gr::NG * a.mul + u;
+        float gq[Gr::NG], tg[Gr::NG], cf[4];
+#pragma unroll
+        for (int g = 0; g < Gr::NG; ++g) gq[g] = __ldg(Gp + (int64_t)g * a.mul);
+        filter_cubic(wl, cf);
+        grid_dots<Gr>(rx, ry, rz, tg);
+        // moments sum_g h t^n give the weight gradient: (2l+1) P_l(t) is a cubic in t
+        float M0 = 0.f, M1 = 0.f, M2 = 0.f, M3 = 0.f;
 #pragma unroll
         for (int g = 0; g < Gr::NG; ++g) {
-          const float t = fmaf(rx, Gr::px(g), fmaf(ry, Gr::py(g), rz * Gr::pz(g)));
-          float E[4], dE[4];
-          legendre_weighted(t, E, dE);
-          const float gq = __ldg(Gr_ + (int64_t)g * a.mul);
-          const float s = fmaf(wl[3], E[3], fmaf(wl[2], E[2], fmaf(wl[1], E[1], wl[0])));
-          gF[g] = fmaf(s, gq, gF[g]);
-          const float h = Fj[g] * gq;
-#pragma unroll
-          for (int l = 0; l < 4; ++l) gw[l] = fmaf(E[l], h, gw[l]);
-          const float c = h * fmaf(wl[3], dE[3], fmaf(wl[2], dE[2], wl[1] * dE[1]));
-          hx = fmaf(c, Gr::px(g), hx);
-          hy = fmaf(c, Gr::py(g), hy);
-          hz = fmaf(c, Gr::pz(g), hz);
+          const float t = tg[g];
+          const float s = fmaf(fmaf(fmaf(cf[3], t, cf[2]), t, cf[1]), t, cf[0]);
+          gF[g] = fmaf(s, gq[g], gF[g]);
+          const float h = Fj[g] * gq[g];
+          const float ht = h * t, ht2 = ht * t;
+          M0 += h;
+          M1 += ht;
+          M2 += ht2;
+          M3 = fmaf(ht2, t, M3);
+          const float c = h * fmaf(fmaf(3.f * cf[3], t, 2.f * cf[2]), t, cf[1]);   // h s'(t)
+          hx = fmaf(c, Gr::st(g / Gr::NP) * Gr::cp(g % Gr::NP), hx);
+          hy = fmaf(c, Gr::st(g / Gr::NP) * Gr::sp(g % Gr::NP), hy);
+          hz = fmaf(c, Gr::ct(g / Gr::NP), hz);
           hs = fmaf(c, t, hs);
         }
+        gw[0] = M0;
+        gw[1] = 3.f * M1;
+        gw[2] = fmaf(7.5f, M2, -2.5f * M0);
+        gw[3] = fmaf(17.5f, M3, -10.5f * M1);
         if (a.gw) {
           for (int l = 0; l <= a.lmax_sh; ++l)
             a.gw[(int64_t)e * a.nw + l * a.mul + u] = (l == 0 || ir > 0.f) ? gw[l] : 0.f;
@@ -211,23 +293,31 @@ __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ Gaunt
         hy = warp_sum(hy);
         hz = warp_sum(hz);
         hs = warp_sum(hs);
-        if (lane == 0) {
-          part[k][sl][0] = hx;
-          part[k][sl][1] = hy;
-          part[k][sl][2] = hz;
-          part[k][sl][3] = hs;
+        if (a.nsl == 1) {
+          if (lane == 0) {
+            float* gv = a.gvec + 3 * (int64_t)e;
+            gv[0] = ir * (hx - rx * hs);
+            gv[1] = ir * (hy - ry * hs);
+            gv[2] = ir * (hz - rz * hs);
+          }
+        } else if (lane == 0) {
+          part[phase][k][sl][0] = hx;
+          part[phase][k][sl][1] = hy;
+          part[phase][k][sl][2] = hz;
+          part[phase][k][sl][3] = hs;
         }
       }
     }
-    if (a.gvec) {
-      __syncthreads();
+    if (a.gvec && a.nsl > 1) {
+      // the slices of this phase have written their partials of the batch's edges
+      named_barrier(1 + phase, 32 * a.nsl);
       if (sl == 0 && lane < ne) {
         float h0 = 0.f, h1 = 0.f, h2 = 0.f, h3 = 0.f;
         for (int s2 = 0; s2 < a.nsl; ++s2) {
-          h0 += part[lane][s2][0];
-          h1 += part[lane][s2][1];
-          h2 += part[lane][s2][2];
-          h3 += part[lane][s2][3];
+          h0 += part[phase][lane][s2][0];
+          h1 += part[phase][lane][s2][1];
+          h2 += part[phase][lane][s2][2];
+          h3 += part[phase][lane][s2][3];
         }
         float rx, ry, rz, ir;
         edge_geometry(vx, vy, vz, rx, ry, rz, ir);
@@ -236,10 +326,25 @@ __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ Gaunt
         gv[1] = ir * (h1 - ry * h3);
         gv[2] = ir * (h2 - rz * h3);
       }
-      __syncthreads();
+      named_barrier(1 + phase, 32 * a.nsl);
     }
   }
-  if (!act || !a.gx) return;
+  if (st > 1) {
+    if (phase > 0) {
+      float* dst = red + (((size_t)(phase - 1) * a.nsl + sl) * Gr::NG) * 32 + lane;
+#pragma unroll
+      for (int g = 0; g < Gr::NG; ++g) dst[g * 32] = gF[g];
+    }
+    __syncthreads();
+    if (phase == 0) {
+      for (int ph = 1; ph < st; ++ph) {
+        const float* srcp = red + (((size_t)(ph - 1) * a.nsl + sl) * Gr::NG) * 32 + lane;
+#pragma unroll
+        for (int g = 0; g < Gr::NG; ++g) gF[g] += srcp[g * 32];
+      }
+    }
+  }
+  if (!act || !a.gx || phase != 0) return;
   float* gr = a.gx + (int64_t)j * a.in_dim;
 #pragma unroll
   for (int l = 0; l <= L; ++l) {
@@ -261,9 +366,14 @@ unsigned node_grid(int64_t n) {
 }
 
 template <int L>
+size_t red_bytes(const GauntArgs& a) {
+  return sizeof(float) * (size_t)(a.split - 1) * a.nsl * gaunt::Grid<L>::NG * 32;
+}
+
+template <int L>
 cudaError_t gaunt_fwd_seq(const GauntArgs& a, cudaStream_t s) {
   k_gaunt_to_grid<L, 0><<<node_grid((int64_t)a.N * a.mul), 256, 0, s>>>(a);
-  k_gaunt_fwd<L><<<(unsigned)a.N, 32 * a.nsl, 0, s>>>(a);
+  k_gaunt_fwd<L><<<(unsigned)a.N, 32 * a.nsl * a.split, red_bytes<L>(a), s>>>(a);
   count_launches(2);
   return cudaGetLastError();
 }
@@ -272,7 +382,7 @@ template <int L>
 cudaError_t gaunt_bwd_seq(const GauntArgs& a, cudaStream_t s) {
   k_gaunt_to_grid<L, 0><<<node_grid((int64_t)a.N * a.mul), 256, 0, s>>>(a);
   k_gaunt_to_grid<L, 1><<<node_grid((int64_t)a.N * a.mul), 256, 0, s>>>(a);
-  k_gaunt_bwd<L><<<(unsigned)a.N, 32 * a.nsl, 0, s>>>(a);
+  k_gaunt_bwd<L><<<(unsigned)a.N, 32 * a.nsl * a.split, red_bytes<L>(a), s>>>(a);
   count_launches(3);
   return cudaGetLastError();
 }
@@ -339,6 +449,9 @@ tp::GauntArgs base(const tp_gaunt_s* p, int64_t N, int64_t E) {
   a.in_dim = (int)p->in_dim;
   a.out_dim = (int)p->out_dim;
   a.nsl = (p->mul + 31) / 32;
+  // warps per node: up to 4 over the slices and the phases that split the node's edges
+  const double avg = N > 0 ? (double)E / (double)N : 0.0;
+  a.split = std::max(1, std::min(4 / a.nsl, avg >= 24.0 ? 4 : avg >= 8.0 ? 2 : 1));
   std::memcpy(a.in_off, p->in_off, sizeof(a.in_off));
   std::memcpy(a.out_off, p->out_off, sizeof(a.out_off));
   return a;
