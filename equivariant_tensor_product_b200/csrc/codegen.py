@@ -797,6 +797,276 @@ def _gen_fwd2(spec: Spec) -> List[str]:
     return L
 
 
+def _km_blocks(spec: Spec):
+    """Per input block a of the uvw receiver pass: the rows r = (p, m3) of the paths reading a
+    (path order), their count n, the padded width W (a multiple of 4), the offset of the block's
+    d1 x W matrix in an edge's K row and the index of its first accumulator pair."""
+    blocks, off, pb = [], 0, 0
+    for a, l1 in enumerate(spec.in_ls):
+        rows = [(p, m3) for p in range(spec.P) if spec.paths[p][0] == a for m3 in range(spec.a_d[p])]
+        if not rows:
+            continue
+        n, d1 = len(rows), 2 * l1 + 1
+        W = (n + 3) // 4 * 4
+        blocks.append(dict(a=a, d1=d1, rows=rows, n=n, W=W, off=off, pb=pb))
+        off += d1 * W
+        pb += (n + 1) // 2
+    return blocks, off, pb
+
+
+def _gen_km(spec: Spec) -> List[str]:
+    """uvw receiver pass with the per-edge coupling matrix
+         K_e[(a, m1), (p, m3)] = c_p s[e, p] sum_m2 C_p[m1, m2, m3] Y(v_e)[m2]      (in(p) = a)
+       so that, per channel, A[(p, m3)] += sum_m1 x[a, m1] K_e[(a, m1), (p, m3)]: the edge's
+       harmonics, path scalars and CG entries are folded once per edge (shared by all channels)
+       and the per-channel work is a dense d1 x n product per input block, evaluated two
+       accumulator rows at a time (FFMA2).  K rows: [block][m1][W] floats, zero padded."""
+    blocks, krow, pairs = _km_blocks(spec)
+    L = [f"  static constexpr int KM_ROW = {krow};",
+         f"  static constexpr int KM_PAIRS = {pairs};"]
+    # entries of the K row, in order, as (cost, expression); pads are 0
+    entries = []
+    for B in blocks:
+        for m1 in range(B["d1"]):
+            for r in range(B["W"]):
+                if r >= B["n"]:
+                    entries.append((0, "0.0f"))
+                    continue
+                p, m3 = B["rows"][r]
+                b = spec.paths[p][1]
+                lb = spec.sh_ls[b]
+                nz = [(j, c) for (i, j, k, c) in cg_nonzeros(*spec.triples[p]) if i == m1 and k == m3]
+                if not nz:
+                    entries.append((0, "0.0f"))
+                    continue
+                if lb == 0:
+                    expr = f"{_flt(nz[0][1])} * cs[{p}]"
+                else:
+                    t = " + ".join(f"{_flt(c)} * Y[{spec.sh_cum[b] + j}]" for j, c in nz)
+                    expr = f"cs[{p}] * ({t})"
+                entries.append((len(nz) + 1, expr))
+    groups = [entries[4 * g:4 * g + 4] for g in range(krow // 4)]
+    gcost = [1 + sum(c for c, _ in grp) for grp in groups]
+    # K row of one edge, built by H threads: thread h writes a contiguous run of float4 groups
+    L.append("  template <int H>")
+    L.append(f"  __device__ __forceinline__ static void km_build(int h, const float (&Y)[{spec.NSH}], "
+             f"const float (&cs)[{spec.P}], float4* __restrict__ k) {{")
+    L.append("    (void)Y;")
+    for H in (1, 2, 4):
+        total = sum(gcost)
+        cuts, acc, part = [0], 0, 1
+        for g, c in enumerate(gcost):
+            acc += c
+            if part < H and acc >= total * part / H:
+                cuts.append(g + 1)
+                part += 1
+        while len(cuts) < H:
+            cuts.append(len(groups))
+        cuts.append(len(groups))
+        L.append(f"    if constexpr (H == {H}) {{")
+        for h in range(H):
+            L.append(f"      if (h == {h}) {{")
+            for g in range(cuts[h], cuts[h + 1]):
+                ex = [e for _, e in groups[g]]
+                L.append(f"        k[{g}] = make_float4({ex[0]}, {ex[1]}, {ex[2]}, {ex[3]});")
+            L.append("      }")
+        L.append("    }")
+    L.append("  }")
+    # per-channel products, one and two channels sharing the K loads
+    for nch in (1, 2):
+        if nch == 1:
+            L.append(f"  __device__ __forceinline__ static void km_apply1(const float (&x0)[{spec.IN_PC}], "
+                     f"const float4* __restrict__ k, float2 (&a0)[{pairs}]) {{")
+        else:
+            L.append(f"  __device__ __forceinline__ static void km_apply2(const float (&x0)[{spec.IN_PC}], "
+                     f"const float (&x1)[{spec.IN_PC}], const float4* __restrict__ k, float2 (&a0)[{pairs}], "
+                     f"float2 (&a1)[{pairs}]) {{")
+        for B in blocks:
+            npair = (B["n"] + 1) // 2
+            for m1 in range(B["d1"]):
+                xi = spec.in_cum[B["a"]] + m1
+                L.append("    {")
+                for ch in range(nch):
+                    L.append(f"      const float2 u{ch} = make_float2(x{ch}[{xi}], x{ch}[{xi}]);")
+                for q in range(B["W"] // 4):
+                    g = (B["off"] + m1 * B["W"]) // 4 + q
+                    L.append(f"      {{ const float4 v = k[{g}];")
+                    for half, (lo, hi) in enumerate((("x", "y"), ("z", "w"))):
+                        pi = 2 * q + half
+                        if pi >= npair:
+                            continue
+                        for ch in range(nch):
+                            L.append(f"        a{ch}[{B['pb'] + pi}] = __ffma2_rn(u{ch}, make_float2(v.{lo}, v.{hi}), a{ch}[{B['pb'] + pi}]);")
+                    L.append("      }")
+                L.append("    }")
+        L.append("  }")
+    # store into the node state A (the store_uvw layout)
+    outs = _uvw_tables(spec)
+    L.append(f"  __device__ __forceinline__ static void km_store(float* __restrict__ base, int64_t N, int mul, "
+             f"int64_t i, int c, const float2 (&acc)[{pairs}]) {{")
+    for B in blocks:
+        for r, (p, m3) in enumerate(B["rows"]):
+            o = spec.paths[p][2]
+            t = outs[o]
+            pl = t["paths"].index(p)
+            idx = f"N * mul * {t['cumA']} + ((i * {t['d3']} + {m3}) * {t['cnt']} + {pl}) * (int64_t)mul + c"
+            L.append(f"    base[{idx}] = acc[{B['pb'] + r // 2}].{'x' if r % 2 == 0 else 'y'};")
+    L.append("  }")
+    return L
+
+
+def _kmt_blocks(spec: Spec):
+    """Per output block o of the uvw sender pass: the rows r = (p, m1) of the paths into o (path
+    order), their count n, padded width W, the offset of the block's d3 x W matrix in an edge's
+    K row and the index of its first row pair."""
+    blocks, off, pb = [], 0, 0
+    for o, l3 in enumerate(spec.out_ls):
+        rows = [(p, m1) for p in range(spec.P) if spec.paths[p][2] == o
+                for m1 in range(2 * spec.triples[p][0] + 1)]
+        if not rows:
+            continue
+        n, d3 = len(rows), 2 * l3 + 1
+        W = (n + 3) // 4 * 4
+        blocks.append(dict(o=o, d3=d3, rows=rows, n=n, W=W, off=off, pb=pb))
+        off += d3 * W
+        pb += (n + 1) // 2
+    return blocks, off, pb
+
+
+def _gen_kmt(spec: Spec) -> List[str]:
+    """uvw sender pass with the transposed per-edge coupling matrix
+         K_e[(o, m3), (p, m1)] = c_p sum_m2 C_p[m1, m2, m3] Y(v_e)[m2]      (out(p) = o)
+       per channel w:  z[(p, m1)] = sum_m3 K_e[(o, m3), (p, m1)] gy[o, m3]   (two rows per FFMA2)
+                       bt[(p, m1)] += s[e, p] z[(p, m1)],   gs[p] += sum_m1 xt[(p, m1)] z[(p, m1)].
+       The sender state xt / bt is held in the same row-pair order.  An edge's row in shared
+       memory: the K entries ([block][m3][W], zero padded), then s[e, p] per row pair."""
+    blocks, krow, pairs = _kmt_blocks(spec)
+    srow = (2 * pairs + 3) // 4 * 4
+    L = [f"  static constexpr int KMT_ROW = {krow + srow};",
+         f"  static constexpr int KMT_PAIRS = {pairs};"]
+    rows_flat = []                       # (pair index, half) -> (p, m1) or None
+    for B in blocks:
+        for q in range((B["n"] + 1) // 2):
+            for h in range(2):
+                r = 2 * q + h
+                rows_flat.append(B["rows"][r] if r < B["n"] else None)
+    entries = []
+    for B in blocks:
+        for m3 in range(B["d3"]):
+            for r in range(B["W"]):
+                if r >= B["n"]:
+                    entries.append((0, "0.0f"))
+                    continue
+                p, m1 = B["rows"][r]
+                b = spec.paths[p][1]
+                lb = spec.sh_ls[b]
+                nz = [(j, c) for (i, j, k, c) in cg_nonzeros(*spec.triples[p]) if i == m1 and k == m3]
+                if not nz:
+                    entries.append((0, "0.0f"))
+                elif lb == 0:
+                    entries.append((2, f"{_flt(nz[0][1])} * cf[{p}]"))
+                else:
+                    t = " + ".join(f"{_flt(c)} * Y[{spec.sh_cum[b] + j}]" for j, c in nz)
+                    entries.append((len(nz) + 1, f"cf[{p}] * ({t})"))
+    for rf in rows_flat:
+        entries.append((1, "0.0f" if rf is None else f"s[{rf[0]}]"))
+    while len(entries) % 4:
+        entries.append((0, "0.0f"))
+    assert len(entries) == krow + srow
+    groups = [entries[4 * g:4 * g + 4] for g in range(len(entries) // 4)]
+    gcost = [1 + sum(c for c, _ in grp) for grp in groups]
+    L.append("  template <int H>")
+    L.append(f"  __device__ __forceinline__ static void kmt_build(int h, const float (&Y)[{spec.NSH}], "
+             f"const float (&cf)[{spec.P}], const float (&s)[{spec.P}], float4* __restrict__ k) {{")
+    L.append("    (void)Y;")
+    for H in (1, 2, 4):
+        total = sum(gcost)
+        cuts, acc, part = [0], 0, 1
+        for g, c in enumerate(gcost):
+            acc += c
+            if part < H and acc >= total * part / H:
+                cuts.append(g + 1)
+                part += 1
+        while len(cuts) < H:
+            cuts.append(len(groups))
+        cuts.append(len(groups))
+        L.append(f"    if constexpr (H == {H}) {{")
+        for h in range(H):
+            L.append(f"      if (h == {h}) {{")
+            for g in range(cuts[h], cuts[h + 1]):
+                ex = [e for _, e in groups[g]]
+                L.append(f"        k[{g}] = make_float4({ex[0]}, {ex[1]}, {ex[2]}, {ex[3]});")
+            L.append("      }")
+        L.append("    }")
+    L.append("  }")
+    # per channel: z, bt, gs
+    L.append(f"  __device__ __forceinline__ static void kmt_apply(const float (&gy)[{spec.OUT_PC}], "
+             f"const float4* __restrict__ k, const float2 (&xt)[{pairs}], float2 (&bt)[{pairs}], "
+             f"float (&gs)[{spec.P}]) {{")
+    L.append(f"    float2 z[{pairs}];")
+    for B in blocks:
+        npair = (B["n"] + 1) // 2
+        for m3 in range(B["d3"]):
+            gi = spec.out_cum[B["o"]] + m3
+            L.append("    {")
+            L.append(f"      const float2 g = make_float2(gy[{gi}], gy[{gi}]);")
+            for q in range(B["W"] // 4):
+                g = (B["off"] + m3 * B["W"]) // 4 + q
+                L.append(f"      {{ const float4 v = k[{g}];")
+                for half, (lo, hi) in enumerate((("x", "y"), ("z", "w"))):
+                    pi = 2 * q + half
+                    if pi >= npair:
+                        continue
+                    zi = B["pb"] + pi
+                    if m3 == 0:
+                        L.append(f"        z[{zi}] = __fmul2_rn(g, make_float2(v.{lo}, v.{hi}));")
+                    else:
+                        L.append(f"        z[{zi}] = __ffma2_rn(g, make_float2(v.{lo}, v.{hi}), z[{zi}]);")
+                L.append("      }")
+            L.append("    }")
+    sg = krow // 4
+    for q4 in range((pairs + 1) // 2):
+        L.append(f"    {{ const float4 v = k[{sg + q4}];")
+        for half, (lo, hi) in enumerate((("x", "y"), ("z", "w"))):
+            q = 2 * q4 + half
+            if q >= pairs:
+                continue
+            L.append(f"      bt[{q}] = __ffma2_rn(make_float2(v.{lo}, v.{hi}), z[{q}], bt[{q}]);")
+        L.append("    }")
+    # gs: products in pairs, then the halves summed per path
+    terms = {p: [] for p in range(spec.P)}
+    for q in range(pairs):
+        L.append(f"    const float2 h{q} = __fmul2_rn(xt[{q}], z[{q}]);")
+        for half in range(2):
+            rf = rows_flat[2 * q + half]
+            if rf is not None:
+                terms[rf[0]].append(f"h{q}.{'x' if half == 0 else 'y'}")
+    for p in range(spec.P):
+        t = terms[p]
+        L.append(f"    gs[{p}] = {' + '.join(t) if t else '0.0f'};")
+    L.append("  }")
+    # sender state in row-pair order (the load_xt / store_xt layout in memory)
+    ins, _ = _uvw_in_tables(spec)
+    for name, const in (("kmt_load_xt", True), ("kmt_store_bt", False)):
+        L.append(f"  __device__ __forceinline__ static void {name}({'const ' if const else ''}float* __restrict__ base, "
+                 f"int64_t N, int mul, int64_t j, int c, {'float2' if const else 'const float2'} (&v)[{pairs}]) {{")
+        for q in range(pairs):
+            for half in range(2):
+                rf = rows_flat[2 * q + half]
+                comp = f"v[{q}].{'x' if half == 0 else 'y'}"
+                if rf is None:
+                    if const:
+                        L.append(f"    {comp} = 0.0f;")
+                    continue
+                p, m1 = rf
+                t = ins[spec.paths[p][0]]
+                pl = t["paths"].index(p)
+                idx = f"N * mul * {t['cumX']} + ((j * {t['d1']} + {m1}) * {t['cnt']} + {pl}) * (int64_t)mul + c"
+                L.append(f"    {comp} = __ldg(base + {idx});" if const else f"    base[{idx}] = {comp};")
+        L.append("  }")
+    return L
+
+
 def gen_spec_header(spec: Spec) -> str:
     L = [f"// Generated by codegen.py for spec '{spec.name}'.  Do not edit.",
          f"// inputs l={spec.in_ls}  SH l={spec.sh_ls}  outputs l={spec.out_ls}",
@@ -833,6 +1103,8 @@ def gen_spec_header(spec: Spec) -> str:
     lay, xt_cum, xt_pc = _gen_uvw_send_layout(spec)
     L += lay
     L += _gen_uvw_send(spec, xt_cum, xt_pc)
+    L += _gen_km(spec)
+    L += _gen_kmt(spec)
     L.append("};")
     return "\n".join(L) + "\n"
 

@@ -211,6 +211,169 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_edge_staged(const __grid_co
   if (act) S::store_uvw(a.A, a.N, a.mul, row, c, acc);
 }
 
+// Receiver pass with the per-edge coupling matrix K_e (S::km_build): one CTA per receiver,
+// NW warps, every lane CH channels (c, and c + 32 when CH = 2, of its warp's 32 CH).  The
+// row's edges are taken in batches of KB.  The K rows of a batch (the edge's harmonics, path
+// scalars and CG entries folded once for all channels; 32 NW / KB threads per edge, each a
+// part of the row) are written into one of two shared-memory buffers while the warps still
+// walk the previous batch: its inputs (edge vectors and path scalars) are copied by
+// cp.async at the start of that batch.  Every warp reads each sender's x row from a ring of
+// copy-engine slots that runs ahead across batch boundaries, and accumulates
+// A[(p, m3)] += x[a, m1] K_e two rows at a time.  Same sums as k_uvw_edge, in another
+// association (per edge, C Y s first).  Needs no index checks and 16-byte aligned rows (the
+// launcher checks).
+template <class S, int NW, int KB, int CH, int MINB>
+__global__ void __launch_bounds__(32 * NW, MINB) k_uvw_recv_km(const __grid_constant__ LaunchArgs a) {
+  static_assert((32 * NW) % KB == 0, "threads per edge");
+  constexpr int H = 32 * NW / KB;
+  static_assert(H == 1 || H == 2 || H == 4, "parts of a K row");
+  constexpr int NIN = S::P + 3;   // per edge: path scalars, edge vector
+  extern __shared__ __align__(128) unsigned char esm[];
+  __shared__ __align__(8) uint64_t full_bar[kEdgeSlots];
+  __shared__ uint32_t read_cnt[kEdgeSlots];
+  __shared__ int last_fill[kEdgeSlots];
+  __shared__ volatile int gather_failed;
+  __shared__ float stage[2][KB * NIN];
+  __shared__ int stage_src[2][KB + kEdgeSlots];
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  const int row = blockIdx.x;
+  const int c0 = wid * 32 * CH + lane, c1 = c0 + 32;
+  const bool act0 = c0 < a.mul, act1 = CH == 2 && c1 < a.mul;
+  const int e0 = __ldg(a.rowptr + row), e1 = __ldg(a.rowptr + row + 1);
+  const uint32_t row_bytes = (uint32_t)a.in_dim * 4u;
+  float4* kbuf = reinterpret_cast<float4*>(esm + (size_t)kEdgeSlots * row_bytes);   // [2][KB][KM_ROW]
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < kEdgeSlots; ++s2) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sm_addr(&full_bar[s2])) : "memory");
+      read_cnt[s2] = 0;
+      last_fill[s2] = -1;
+    }
+    gather_failed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  // ring fill f carries the x row of edge e0 + f, sender j
+  auto fill = [&](int f, int j) {
+    const int s2 = f % kEdgeSlots;
+    const uint32_t mb = sm_addr(&full_bar[s2]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(row_bytes) : "memory");
+    bulk_g2s(sm_addr(esm + (size_t)s2 * row_bytes), a.x + (int64_t)j * a.in_dim, row_bytes, mb);
+    last_fill[s2] = f;
+  };
+  // the inputs of the batch at edge b0 into stage buffer sb (cp.async, one group per thread):
+  // path scalars and edge vectors of its edges, senders of its edges and the ring's lookahead
+  auto stage_inputs = [&](int b0, int sb) {
+    const int nb = min(KB, e1 - b0);
+    for (int t = threadIdx.x; t < nb * NIN; t += 32 * NW) {
+      const int k = t / NIN, v = t - k * NIN;
+      const float* src = v < S::P ? a.w + (int64_t)(b0 + k) * S::P + v : a.vec + 3 * (int64_t)(b0 + k) + (v - S::P);
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sm_addr(&stage[sb][t])), "l"(src) : "memory");
+    }
+    const int ns = min(KB + kEdgeSlots, e1 - b0);
+    for (int t = threadIdx.x; t < ns; t += 32 * NW)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sm_addr(&stage_src[sb][t])), "l"(a.src + b0 + t) : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  // K rows of the batch at edge b0 (stage buffer sb) into buffer kb
+  auto build = [&](int b0, int sb, float4* kb) {
+    const int k = threadIdx.x % KB, h = threadIdx.x / KB;
+    if (b0 + k < e1) {
+      const float* in = stage[sb] + k * NIN;
+      float rx, ry, rz, ir;
+      edge_geometry(in[S::P], in[S::P + 1], in[S::P + 2], rx, ry, rz, ir);
+      float Y[S::NSH], cs[S::P];
+      S::sh(rx, ry, rz, Y);
+#pragma unroll
+      for (int p = 0; p < S::P; ++p) cs[p] = in[p] * (a.has_coeff ? a.coeff[p] : 1.f);
+      S::template km_build<H>(h, Y, cs, kb + (size_t)k * (S::KM_ROW / 4));
+    }
+  };
+  float2 acc0[S::KM_PAIRS], acc1[CH == 2 ? S::KM_PAIRS : 1];
+#pragma unroll
+  for (int k = 0; k < S::KM_PAIRS; ++k) acc0[k] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < (CH == 2 ? S::KM_PAIRS : 1); ++k) acc1[k] = make_float2(0.f, 0.f);
+  const int ntot = e1 - e0;
+  if (ntot > 0) {
+    stage_inputs(e0, 0);
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int f = 0; f < min(ntot, kEdgeSlots); ++f) fill(f, stage_src[0][f]);
+    build(e0, 0, kbuf);
+    __syncthreads();
+  }
+  int buf = 0;
+  for (int base = e0; base < e1; base += KB) {
+    const int ne = min(KB, e1 - base);
+    const bool more = base + KB < e1;
+    if (more) stage_inputs(base + KB, buf ^ 1);
+    const float4* kcur = kbuf + (size_t)buf * KB * (S::KM_ROW / 4);
+#pragma unroll 1
+    for (int k = 0; k < ne; ++k) {
+      const int f = base - e0 + k, s2 = f % kEdgeSlots;
+      bool ok = !gather_failed;
+      if (ok) ok = slot_wait(sm_addr(&full_bar[s2]), (uint32_t)((f / kEdgeSlots) & 1));
+      ok = __all_sync(kFull, ok);
+      if (!ok) gather_failed = 1;
+      const float* xrow = reinterpret_cast<const float*>(esm + (size_t)s2 * row_bytes);
+      float x0[S::IN_PC], x1[CH == 2 ? S::IN_PC : 1];
+      if (ok) {
+        if (act0) S::load_in_shared(xrow, a.mul, c0, x0);
+        if constexpr (CH == 2) {
+          if (act1) S::load_in_shared(xrow, a.mul, c1, x1);
+        }
+      }
+      // this warp is done with the slot; the last of the NW warps refills it
+      __syncwarp();
+      int last = 0;
+      if (lane == 0 && ok) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        uint32_t old;
+        asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(old) : "r"(sm_addr(&read_cnt[s2])) : "memory");
+        last = old == NW - 1;
+      }
+      last = __shfl_sync(kFull, last, 0);
+      if (last && lane == 0) {
+        read_cnt[s2] = 0;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (f + kEdgeSlots < ntot) fill(f + kEdgeSlots, stage_src[buf][k + kEdgeSlots]);
+      }
+      if (!ok) continue;
+      const float4* kr = kcur + (size_t)k * (S::KM_ROW / 4);
+      if constexpr (CH == 2) {
+        if (act1) S::km_apply2(x0, x1, kr, acc0, acc1);
+        else if (act0) S::km_apply1(x0, kr, acc0);
+      } else if (act0) {
+        S::km_apply1(x0, kr, acc0);
+      }
+    }
+    if (more) {   // the next batch's K rows into the other buffer (last read two batches ago)
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      __syncthreads();
+      build(base + KB, buf ^ 1, kbuf + (size_t)(buf ^ 1) * KB * (S::KM_ROW / 4));
+    }
+    __syncthreads();
+    buf ^= 1;
+  }
+  if (gather_failed && threadIdx.x == 0) {   // let the issued copies land, then report
+    for (int s2 = 0; s2 < kEdgeSlots; ++s2) {
+      const int f = last_fill[s2];
+      if (f < 0) continue;
+      const uint32_t mb = sm_addr(&full_bar[s2]);
+      const unsigned long long t0 = now_ns();
+      while (!slot_ready(mb, (uint32_t)((f / kEdgeSlots) & 1)) && now_ns() - t0 < kGatherWaitNs) {
+      }
+    }
+    report(a, kDevGatherTimeout);
+  }
+  if (act0) S::km_store(a.A, a.N, a.mul, row, c0, acc0);
+  if constexpr (CH == 2) {
+    if (act1) S::km_store(a.A, a.N, a.mul, row, c1, acc1);
+  }
+}
+
 // Wt[o][w][pl * mul + u] = W[path_of(o, pl)][u][w]: B operand of the forward mixing GEMM
 // (hi at Wt, lo at Wt + P * mul * mul_out).
 template <class S>
@@ -659,6 +822,155 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
   if (act) S::store_xt(a.G, a.N, a.mul_out, node, c, bt);
 }
 
+// Sender pass with the transposed per-edge coupling matrix (S::kmt_build), without gvec: as
+// the STAGED k_uvw_send (one CTA per sender, NSL slice warps, lane = output channel, the
+// receivers' gy rows staged by the copy engine), but per batch of 32 out-edges the CTA first
+// writes each edge's K row and path scalars into shared memory (warp h builds part h of every
+// edge's row), so that per channel z = K gy, bt += s z and gs += xt . z are dense products
+// evaluated two rows at a time.
+template <class S, int NSL, int MINB>
+__global__ void __launch_bounds__(32 * NSL, MINB) k_uvw_send_km(const __grid_constant__ LaunchArgs a) {
+  extern __shared__ float smem[];
+  constexpr int NV = S::P;
+  __shared__ __align__(8) uint64_t full_bar[kSendSlots];
+  __shared__ uint32_t read_cnt[kSendSlots];
+  __shared__ int last_fill[kSendSlots];
+  __shared__ volatile int gather_failed;
+  __shared__ int32_t rtab[kRowTab];
+  const int lane = threadIdx.x & 31;
+  const int sl = threadIdx.x >> 5;
+  const int node = blockIdx.x;
+  const int c = sl * 32 + lane;
+  const bool act = c < a.mul_out;
+  const int q0 = __ldg(a.colptr + node), q1 = __ldg(a.colptr + node + 1);
+  // shared memory: [32 edges][NSL][NV] partials | K rows [32][KMT_ROW] | gy ring
+  float4* krows = reinterpret_cast<float4*>(smem + (32 * NSL * NV + 3) / 4 * 4);
+  unsigned char* ring = reinterpret_cast<unsigned char*>(krows + 32 * (S::KMT_ROW / 4));
+  const uint32_t row_bytes = (uint32_t)a.out_dim * 4u;
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < kSendSlots; ++s2) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sm_addr(&full_bar[s2])) : "memory");
+      read_cnt[s2] = 0;
+      last_fill[s2] = -1;
+    }
+    gather_failed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  const RowTab rt = load_row_tab(a.rowptr, a.N, rtab);
+  __syncthreads();
+  auto fill = [&](int f, int i) {
+    const int s2 = f % kSendSlots;
+    const uint32_t mb = sm_addr(&full_bar[s2]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(row_bytes) : "memory");
+    bulk_g2s(sm_addr(ring + (size_t)s2 * row_bytes), a.gy + (int64_t)i * a.out_dim, row_bytes, mb);
+    last_fill[s2] = f;
+  };
+  float2 xt[S::KMT_PAIRS], bt[S::KMT_PAIRS];
+#pragma unroll
+  for (int k = 0; k < S::KMT_PAIRS; ++k) xt[k] = bt[k] = make_float2(0.f, 0.f);
+  if (act) S::kmt_load_xt(a.A, a.N, a.mul_out, node, c, xt);
+  float* slot = smem;   // [32 edges][NSL][NV]
+  int first = 0;
+  for (int base = q0; base < q1; base += 32) {
+    const int my_q = base + lane;
+    int my_e = -1, my_i = 0;
+    float vx = 0.f, vy = 0.f, vz = 0.f;
+    if (my_q < q1) {
+      my_e = __ldg(a.perm + my_q);
+      my_i = find_row_tab(a.rowptr, a.N, rtab, rt, my_e);
+      vx = __ldg(a.vec + 3 * (int64_t)my_e);
+      vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
+      vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
+    }
+    const int ne = min(32, q1 - base);
+    if (sl == 0) {
+      for (int k = 0; k < min(ne, kSendSlots); ++k) {
+        const int i = __shfl_sync(kFull, my_i, k);
+        if (lane == 0) fill(first + k, i);
+      }
+    }
+    if (my_e >= 0) {   // part sl of the K row of edge base + lane
+      float rx, ry, rz, ir;
+      edge_geometry(vx, vy, vz, rx, ry, rz, ir);
+      float Y[S::NSH], cf[S::P], sv[S::P];
+      S::sh(rx, ry, rz, Y);
+#pragma unroll
+      for (int p = 0; p < S::P; ++p) {
+        cf[p] = a.has_coeff ? a.coeff[p] : 1.f;
+        sv[p] = __ldg(a.w + (int64_t)my_e * S::P + p);
+      }
+      S::template kmt_build<NSL>(sl, Y, cf, sv, krows + (size_t)lane * (S::KMT_ROW / 4));
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int k = 0; k < ne; ++k) {
+      const int f = first + k, s2 = f % kSendSlots;
+      bool ok = !gather_failed;
+      if (ok) ok = slot_wait(sm_addr(&full_bar[s2]), (uint32_t)((f / kSendSlots) & 1));
+      ok = __all_sync(kFull, ok);
+      if (!ok) gather_failed = 1;
+      float gs[S::P];
+#pragma unroll
+      for (int p = 0; p < S::P; ++p) gs[p] = 0.f;
+      if (ok && act) {
+        float gyv[S::OUT_PC];
+        S::load_out_shared(reinterpret_cast<const float*>(ring + (size_t)s2 * row_bytes), a.mul_out, c, gyv);
+        S::kmt_apply(gyv, krows + (size_t)k * (S::KMT_ROW / 4), xt, bt, gs);
+      }
+      // this warp is done with the slot; the last of the NSL warps refills it
+      __syncwarp();
+      int last = 0;
+      if (lane == 0 && ok) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        uint32_t old;
+        asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(old) : "r"(sm_addr(&read_cnt[s2])) : "memory");
+        last = old == NSL - 1;
+      }
+      last = __shfl_sync(kFull, last, 0);
+      const int inext = __shfl_sync(kFull, my_i, min(k + kSendSlots, 31));
+      if (last && lane == 0) {
+        read_cnt[s2] = 0;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (k + kSendSlots < ne) fill(f + kSendSlots, inext);
+      }
+      float r[(NV + 15) / 16 * 16];
+#pragma unroll
+      for (int v = 0; v < (NV + 15) / 16 * 16; ++v) r[v] = v < NV ? gs[v < NV ? v : 0] : 0.f;
+      float* sp = slot + ((size_t)k * NSL + sl) * NV;
+#pragma unroll
+      for (int g = 0; g < (NV + 15) / 16; ++g) {
+        const float tot = warp_reduce_scatter16(&r[16 * g], lane);
+        const int v = 16 * g + ((lane >> 1) & 15);
+        if (!(lane & 1) && v < NV) sp[v] = tot;
+      }
+    }
+    __syncthreads();
+    if (sl == 0 && lane < ne && a.gw) {
+      float* gsr = a.gw + (int64_t)my_e * S::P;
+#pragma unroll
+      for (int p = 0; p < S::P; ++p) {
+        float t = 0.f;
+        for (int s2 = 0; s2 < NSL; ++s2) t += slot[((size_t)lane * NSL + s2) * NV + p];
+        gsr[p] = t;
+      }
+    }
+    __syncthreads();
+    first += ne;
+  }
+  if (gather_failed && threadIdx.x == 0) {   // let the issued copies land, then report
+    for (int s2 = 0; s2 < kSendSlots; ++s2) {
+      const int f = last_fill[s2];
+      if (f < 0) continue;
+      const uint32_t mb = sm_addr(&full_bar[s2]);
+      const unsigned long long t0 = now_ns();
+      while (!slot_ready(mb, (uint32_t)((f / kSendSlots) & 1)) && now_ns() - t0 < kGatherWaitNs) {
+      }
+    }
+    report(a, kDevGatherTimeout);
+  }
+  if (act) S::kmt_store_bt(a.G, a.N, a.mul_out, node, c, bt);
+}
+
 // ---------------------------------------------------------------------------------------
 // Host sequences
 // ---------------------------------------------------------------------------------------
@@ -675,6 +987,22 @@ cudaError_t with_d(int d, F&& f) {
 template <class S>
 cudaError_t launch_uvw_edge(const LaunchArgs& a, cudaStream_t s) {
   const int nsl = (a.mul + 31) / 32;
+  if constexpr (S::KM_PAIRS <= 32) {
+    if (!a.check && a.mul >= 64 && a.mul <= 128 && a.in_dim % 4 == 0 && (reinterpret_cast<uintptr_t>(a.x) & 15u) == 0) {
+      // per-edge coupling matrices in shared memory, two channels per lane
+      constexpr int KB = 16;
+      auto go = [&](auto kern, int threads, int kb) -> cudaError_t {
+        const size_t sm = (size_t)kEdgeSlots * a.in_dim * sizeof(float) + (size_t)2 * kb * S::KM_ROW * sizeof(float);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        kern<<<(unsigned)a.N, threads, sm, s>>>(a);
+        count_launches(1);
+        return cudaGetLastError();
+      };
+      if (a.mul > 64) return go(k_uvw_recv_km<S, 2, KB, 2, 1>, 64, KB);
+      return go(k_uvw_recv_km<S, 1, KB, 2, 1>, 32, KB);
+    }
+  }
   if (!a.check && nsl == 4 && a.in_dim % 4 == 0 && (reinterpret_cast<uintptr_t>(a.x) & 15u) == 0) {
     // every slice of a receiver in one CTA, the x rows staged by the copy engine
     const size_t sm = (size_t)kEdgeSlots * a.in_dim * sizeof(float);
@@ -774,7 +1102,22 @@ cudaError_t launch_uvw_bwd(const LaunchArgs& a, cudaStream_t s) {
   using T1 = std::integral_constant<int, 1>;
   using T2 = std::integral_constant<int, 2>;
   using T4 = std::integral_constant<int, 4>;
-  if (nsl == 1) e = gv ? send(std::true_type{}, T1{}) : send(std::false_type{}, T1{});
+  auto send_km = [&](auto nsl_tag) -> cudaError_t {
+    constexpr int NS = decltype(nsl_tag)::value;
+    const size_t sm = sizeof(float) * ((size_t)(32 * NS * S::P + 3) / 4 * 4 + (size_t)32 * S::KMT_ROW) +
+                      (size_t)kSendSlots * a.out_dim * sizeof(float);
+    auto kern = k_uvw_send_km<S, NS, 12 / NS>;   // three CTAs of four warps per SM
+    cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (r != cudaSuccess) return r;
+    kern<<<(unsigned)a.N, 32 * NS, sm, s>>>(a);
+    return cudaSuccess;
+  };
+  if (staged && !gv && S::KMT_PAIRS <= 32) {
+    // per-edge coupling matrices in shared memory (the direction gradient takes the CG form)
+    if constexpr (S::KMT_PAIRS <= 32) {
+      e = nsl == 1 ? send_km(T1{}) : nsl == 2 ? send_km(T2{}) : send_km(T4{});
+    }
+  } else if (nsl == 1) e = gv ? send(std::true_type{}, T1{}) : send(std::false_type{}, T1{});
   else if (nsl == 2) e = gv ? send(std::true_type{}, T2{}) : send(std::false_type{}, T2{});
   else e = gv ? send(std::true_type{}, T4{}) : send(std::false_type{}, T4{});
   if (e != cudaSuccess) return e;

@@ -79,9 +79,12 @@ def test_uvu_channel_counts_and_long_rows(tp, mul):
         assert_close(out[k], ref[k], f"mul {mul} {k}")
 
 
-@pytest.mark.parametrize("mul_in,mul_out", [(128, 128), (64, 32), (32, 96)])
-def test_uvw_channel_counts_and_long_rows(tp, mul_in, mul_out):
-    spec = synth.CONFIGS["c4"]
+# (128, 128): the receiver pass with per-edge coupling matrices, two warps; (64, 32): one warp;
+# (96, 64): the second warp's upper 32 channels idle; (32, 96): the general receiver pass
+@pytest.mark.parametrize("mul_in,mul_out,cfg", [(128, 128, "c4"), (64, 32, "c4"), (96, 64, "c4"), (32, 96, "c4"),
+                                                (64, 64, "c1"), (128, 32, "c1")])
+def test_uvw_channel_counts_and_long_rows(tp, mul_in, mul_out, cfg):
+    spec = synth.CONFIGS[cfg]
     ins, outs = _irreps(spec.irreps_in, mul_in), _irreps(spec.irreps_out, mul_out)
     plan = tp.Plan(ins, spec.irreps_sh, outs, spec.paths, "uvw")
     op = OraclePlan(ins, spec.irreps_sh, outs, spec.paths, "uvw")
@@ -104,6 +107,12 @@ def test_uvw_channel_counts_and_long_rows(tp, mul_in, mul_out):
     assert_close(gs, ref["gs"], f"uvw {mul_in}/{mul_out} gs")
     assert_close(gvec, ref["gvec"], f"uvw {mul_in}/{mul_out} gvec")
     assert_close(gW.view(ref["gW"].shape), ref["gW"], f"uvw {mul_in}/{mul_out} gW")
+    # without the direction gradient the sender pass takes its coupling-matrix form
+    gx2, gs2, _, gW2 = tp.tp_conv_bwd(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["s"], g["gy"], W=g["W"],
+                                      need_gvec=False, need_gW=True)
+    assert_close(gx2, ref["gx"], f"uvw {mul_in}/{mul_out} gx (no gvec)")
+    assert_close(gs2, ref["gs"], f"uvw {mul_in}/{mul_out} gs (no gvec)")
+    assert_close(gW2.view(ref["gW"].shape), ref["gW"], f"uvw {mul_in}/{mul_out} gW (no gvec)")
 
 
 def test_rows_off_16_byte_boundaries_take_the_general_path(tp):
