@@ -136,6 +136,7 @@ __device__ __forceinline__ unsigned long long global_ns() {
 // On its own timeout it raises the abort flag.  Returns false when the caller must stop.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, volatile int* abort_flag,
                                           unsigned long long limit_ns = kWaitNs) {
+  if (mbar_try_wait(mbar, parity)) return true;   // the common case reads no clock
   const unsigned long long t0 = global_ns();
   for (;;) {
     if (mbar_try_wait(mbar, parity)) return true;
@@ -279,7 +280,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ volatile int abort_flag;
-  char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned by an offset from the shared array itself, so that the compiler keeps the accesses
+  // in the shared window (a round trip through an integer would make them generic)
+  char* smem = tc_smem_raw + ((1024u - (smem_u32(tc_smem_raw) & 1023u)) & 1023u);
   float* T = reinterpret_cast<float*>(smem + ST * SH::STAGE_BYTES);
   const uint32_t smem_s = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
