@@ -852,7 +852,7 @@ def _gen_km(spec: Spec) -> List[str]:
     L.append(f"  __device__ __forceinline__ static void km_build(int h, const float (&Y)[{spec.NSH}], "
              f"const float (&cs)[{spec.P}], float4* __restrict__ k) {{")
     L.append("    (void)Y;")
-    for H in (1, 2, 4):
+    for H in (1, 2, 4, 8):
         total = sum(gcost)
         cuts, acc, part = [0], 0, 1
         for g, c in enumerate(gcost):

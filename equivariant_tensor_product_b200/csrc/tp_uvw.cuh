@@ -222,19 +222,19 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_edge_staged(const __grid_co
 // A[(p, m3)] += x[a, m1] K_e two rows at a time.  Same sums as k_uvw_edge, in another
 // association (per edge, C Y s first).  Needs no index checks and 16-byte aligned rows (the
 // launcher checks).
-template <class S, int NW, int KB, int CH, int MINB>
+template <class S, int NW, int KB, int CH, int MINB, int R = kEdgeSlots>
 __global__ void __launch_bounds__(32 * NW, MINB) k_uvw_recv_km(const __grid_constant__ LaunchArgs a) {
   static_assert((32 * NW) % KB == 0, "threads per edge");
   constexpr int H = 32 * NW / KB;
-  static_assert(H == 1 || H == 2 || H == 4, "parts of a K row");
+  static_assert(H == 1 || H == 2 || H == 4 || H == 8, "parts of a K row");
   constexpr int NIN = S::P + 3;   // per edge: path scalars, edge vector
   extern __shared__ __align__(128) unsigned char esm[];
-  __shared__ __align__(8) uint64_t full_bar[kEdgeSlots];
-  __shared__ uint32_t read_cnt[kEdgeSlots];
-  __shared__ int last_fill[kEdgeSlots];
+  __shared__ __align__(8) uint64_t full_bar[R];
+  __shared__ uint32_t read_cnt[R];
+  __shared__ int last_fill[R];
   __shared__ volatile int gather_failed;
   __shared__ float stage[2][KB * NIN];
-  __shared__ int stage_src[2][KB + kEdgeSlots];
+  __shared__ int stage_src[2][KB + R];
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
   const int row = blockIdx.x;
@@ -242,9 +242,9 @@ __global__ void __launch_bounds__(32 * NW, MINB) k_uvw_recv_km(const __grid_cons
   const bool act0 = c0 < a.mul, act1 = CH == 2 && c1 < a.mul;
   const int e0 = __ldg(a.rowptr + row), e1 = __ldg(a.rowptr + row + 1);
   const uint32_t row_bytes = (uint32_t)a.in_dim * 4u;
-  float4* kbuf = reinterpret_cast<float4*>(esm + (size_t)kEdgeSlots * row_bytes);   // [2][KB][KM_ROW]
+  float4* kbuf = reinterpret_cast<float4*>(esm + (size_t)R * row_bytes);   // [2][KB][KM_ROW]
   if (threadIdx.x == 0) {
-    for (int s2 = 0; s2 < kEdgeSlots; ++s2) {
+    for (int s2 = 0; s2 < R; ++s2) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sm_addr(&full_bar[s2])) : "memory");
       read_cnt[s2] = 0;
       last_fill[s2] = -1;
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(32 * NW, MINB) k_uvw_recv_km(const __grid_cons
   __syncthreads();
   // ring fill f carries the x row of edge e0 + f, sender j
   auto fill = [&](int f, int j) {
-    const int s2 = f % kEdgeSlots;
+    const int s2 = f % R;
     const uint32_t mb = sm_addr(&full_bar[s2]);
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mb), "r"(row_bytes) : "memory");
     bulk_g2s(sm_addr(esm + (size_t)s2 * row_bytes), a.x + (int64_t)j * a.in_dim, row_bytes, mb);
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(32 * NW, MINB) k_uvw_recv_km(const __grid_cons
       const float* src = v < S::P ? a.w + (int64_t)(b0 + k) * S::P + v : a.vec + 3 * (int64_t)(b0 + k) + (v - S::P);
       asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sm_addr(&stage[sb][t])), "l"(src) : "memory");
     }
-    const int ns = min(KB + kEdgeSlots, e1 - b0);
+    const int ns = min(KB + R, e1 - b0);
     for (int t = threadIdx.x; t < ns; t += 32 * NW)
       asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sm_addr(&stage_src[sb][t])), "l"(a.src + b0 + t) : "memory");
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(32 * NW, MINB) k_uvw_recv_km(const __grid_cons
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
     if (threadIdx.x == 0)
-      for (int f = 0; f < min(ntot, kEdgeSlots); ++f) fill(f, stage_src[0][f]);
+      for (int f = 0; f < min(ntot, R); ++f) fill(f, stage_src[0][f]);
     build(e0, 0, kbuf);
     __syncthreads();
   }
@@ -312,9 +312,9 @@ __global__ void __launch_bounds__(32 * NW, MINB) k_uvw_recv_km(const __grid_cons
     const float4* kcur = kbuf + (size_t)buf * KB * (S::KM_ROW / 4);
 #pragma unroll 1
     for (int k = 0; k < ne; ++k) {
-      const int f = base - e0 + k, s2 = f % kEdgeSlots;
+      const int f = base - e0 + k, s2 = f % R;
       bool ok = !gather_failed;
-      if (ok) ok = slot_wait(sm_addr(&full_bar[s2]), (uint32_t)((f / kEdgeSlots) & 1));
+      if (ok) ok = slot_wait(sm_addr(&full_bar[s2]), (uint32_t)((f / R) & 1));
       ok = __all_sync(kFull, ok);
       if (!ok) gather_failed = 1;
       const float* xrow = reinterpret_cast<const float*>(esm + (size_t)s2 * row_bytes);
@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(32 * NW, MINB) k_uvw_recv_km(const __grid_cons
       if (last && lane == 0) {
         read_cnt[s2] = 0;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        if (f + kEdgeSlots < ntot) fill(f + kEdgeSlots, stage_src[buf][k + kEdgeSlots]);
+        if (f + R < ntot) fill(f + R, stage_src[buf][k + R]);
       }
       if (!ok) continue;
       const float4* kr = kcur + (size_t)k * (S::KM_ROW / 4);
@@ -358,12 +358,12 @@ __global__ void __launch_bounds__(32 * NW, MINB) k_uvw_recv_km(const __grid_cons
     buf ^= 1;
   }
   if (gather_failed && threadIdx.x == 0) {   // let the issued copies land, then report
-    for (int s2 = 0; s2 < kEdgeSlots; ++s2) {
+    for (int s2 = 0; s2 < R; ++s2) {
       const int f = last_fill[s2];
       if (f < 0) continue;
       const uint32_t mb = sm_addr(&full_bar[s2]);
       const unsigned long long t0 = now_ns();
-      while (!slot_ready(mb, (uint32_t)((f / kEdgeSlots) & 1)) && now_ns() - t0 < kGatherWaitNs) {
+      while (!slot_ready(mb, (uint32_t)((f / R) & 1)) && now_ns() - t0 < kGatherWaitNs) {
       }
     }
     report(a, kDevGatherTimeout);
@@ -828,8 +828,9 @@ __global__ void __launch_bounds__(kMaxThreads) k_uvw_send(const __grid_constant_
 // writes each edge's K row and path scalars into shared memory (warp h builds part h of every
 // edge's row), so that per channel z = K gy, bt += s z and gs += xt . z are dense products
 // evaluated two rows at a time.
-template <class S, int NSL, int MINB>
+template <class S, int NSL, int MINB, int KB>
 __global__ void __launch_bounds__(32 * NSL, MINB) k_uvw_send_km(const __grid_constant__ LaunchArgs a) {
+  static_assert(KB == 16 || KB == 32, "edges per batch");
   extern __shared__ float smem[];
   constexpr int NV = S::P;
   __shared__ __align__(8) uint64_t full_bar[kSendSlots];
@@ -843,9 +844,9 @@ __global__ void __launch_bounds__(32 * NSL, MINB) k_uvw_send_km(const __grid_con
   const int c = sl * 32 + lane;
   const bool act = c < a.mul_out;
   const int q0 = __ldg(a.colptr + node), q1 = __ldg(a.colptr + node + 1);
-  // shared memory: [32 edges][NSL][NV] partials | K rows [32][KMT_ROW] | gy ring
-  float4* krows = reinterpret_cast<float4*>(smem + (32 * NSL * NV + 3) / 4 * 4);
-  unsigned char* ring = reinterpret_cast<unsigned char*>(krows + 32 * (S::KMT_ROW / 4));
+  // shared memory: [KB edges][NSL][NV] partials | K rows [KB][KMT_ROW] | gy ring
+  float4* krows = reinterpret_cast<float4*>(smem + (KB * NSL * NV + 3) / 4 * 4);
+  unsigned char* ring = reinterpret_cast<unsigned char*>(krows + KB * (S::KMT_ROW / 4));
   const uint32_t row_bytes = (uint32_t)a.out_dim * 4u;
   if (threadIdx.x == 0) {
     for (int s2 = 0; s2 < kSendSlots; ++s2) {
@@ -869,20 +870,20 @@ __global__ void __launch_bounds__(32 * NSL, MINB) k_uvw_send_km(const __grid_con
 #pragma unroll
   for (int k = 0; k < S::KMT_PAIRS; ++k) xt[k] = bt[k] = make_float2(0.f, 0.f);
   if (act) S::kmt_load_xt(a.A, a.N, a.mul_out, node, c, xt);
-  float* slot = smem;   // [32 edges][NSL][NV]
+  float* slot = smem;   // [KB edges][NSL][NV]
   int first = 0;
-  for (int base = q0; base < q1; base += 32) {
+  for (int base = q0; base < q1; base += KB) {
     const int my_q = base + lane;
     int my_e = -1, my_i = 0;
     float vx = 0.f, vy = 0.f, vz = 0.f;
-    if (my_q < q1) {
+    if (lane < KB && my_q < q1) {
       my_e = __ldg(a.perm + my_q);
       my_i = find_row_tab(a.rowptr, a.N, rtab, rt, my_e);
       vx = __ldg(a.vec + 3 * (int64_t)my_e);
       vy = __ldg(a.vec + 3 * (int64_t)my_e + 1);
       vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
     }
-    const int ne = min(32, q1 - base);
+    const int ne = min(KB, q1 - base);
     if (sl == 0) {
       for (int k = 0; k < min(ne, kSendSlots); ++k) {
         const int i = __shfl_sync(kFull, my_i, k);
@@ -927,7 +928,7 @@ __global__ void __launch_bounds__(32 * NSL, MINB) k_uvw_send_km(const __grid_con
         last = old == NSL - 1;
       }
       last = __shfl_sync(kFull, last, 0);
-      const int inext = __shfl_sync(kFull, my_i, min(k + kSendSlots, 31));
+      const int inext = __shfl_sync(kFull, my_i, min(k + kSendSlots, KB - 1));
       if (last && lane == 0) {
         read_cnt[s2] = 0;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -999,7 +1000,8 @@ cudaError_t launch_uvw_edge(const LaunchArgs& a, cudaStream_t s) {
         count_launches(1);
         return cudaGetLastError();
       };
-      if (a.mul > 64) return go(k_uvw_recv_km<S, 2, KB, 2, 1>, 64, KB);
+      // two warps, eight edges per K batch, six CTAs per SM (168 registers)
+      if (a.mul > 64) return go(k_uvw_recv_km<S, 2, 8, 2, 6>, 64, 8);
       return go(k_uvw_recv_km<S, 1, KB, 2, 1>, 32, KB);
     }
   }
@@ -1104,9 +1106,10 @@ cudaError_t launch_uvw_bwd(const LaunchArgs& a, cudaStream_t s) {
   using T4 = std::integral_constant<int, 4>;
   auto send_km = [&](auto nsl_tag) -> cudaError_t {
     constexpr int NS = decltype(nsl_tag)::value;
-    const size_t sm = sizeof(float) * ((size_t)(32 * NS * S::P + 3) / 4 * 4 + (size_t)32 * S::KMT_ROW) +
+    constexpr int KB = 32;
+    const size_t sm = sizeof(float) * ((size_t)(KB * NS * S::P + 3) / 4 * 4 + (size_t)KB * S::KMT_ROW) +
                       (size_t)kSendSlots * a.out_dim * sizeof(float);
-    auto kern = k_uvw_send_km<S, NS, 12 / NS>;   // three CTAs of four warps per SM
+    auto kern = k_uvw_send_km<S, NS, 12 / NS, KB>;   // three CTAs of four warps per SM
     cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (r != cudaSuccess) return r;
     kern<<<(unsigned)a.N, 32 * NS, sm, s>>>(a);
