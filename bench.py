@@ -1364,23 +1364,24 @@ def run_latency(args, rank, world, local):
 GAUNT_SPEC = ("32x0e+32x1o+32x2e", 2, "32x0e+32x1o+32x2e")
 
 
-def gaunt_counts(N, E, mul, ng, d_in, d_out, lmax_sh):
+def gaunt_counts(N, E, mul, ng, d_in, d_out, lmax_sh, need_gvec=False):
     """Algorithmic bytes and flops of the Gaunt convolution (fwd, bwd).  Bytes: the operator's
     inputs and outputs (as fwd_bytes / bwd_bytes, w being (lmax_sh + 1) x mul per edge; the
-    node grids are workspace, not counted).  Flops of the grid method, per edge and channel:
-    the filter on the grid (2 (lmax_sh + 1) per point) and the product-accumulate (2 per point),
-    plus per edge the dot products r_hat . r_g and the Legendre values (2 (3 + lmax_sh) per point,
-    shared by the channels); per node and channel the transforms to and from the grid (2 ng d_in
-    and 2 ng d_out).  The backward counts the grid transforms of x and gy, the filter, the
-    accumulation of gF, the weight gradient (2 (lmax_sh + 1) per point) and the direction terms
-    (10 per point)."""
+    node grids are workspace, not counted).  Flops of the grid method (an FMA is 2), per edge,
+    channel and grid point: the filter sum_l w_l (2l+1) P_l(t) as a polynomial of degree
+    lmax_sh in t = r_hat . r_g by Horner's rule (2 lmax_sh) and the product-accumulate (2);
+    per edge the dot products t (2 per point, shared by the channels); per node and channel
+    the transforms to and from the grid (2 ng d_in and 2 ng d_out).  The backward (gx, gw):
+    the grid transforms of x and gy, the filter, the accumulation of gF (2), h = F Gq (1) and
+    the weight moments sum h t^n, n <= lmax_sh (2 lmax_sh + 1); with need_gvec also the
+    direction terms (the derivative of the filter, 2 lmax_sh - 1, and four accumulations, 8)."""
     nw = (lmax_sh + 1) * mul
     fb = E * (4 + 12 + 4 * nw) + 4 * N * (d_in + d_out) + 4 * (N + 1)
-    bb = E * (4 + 12 + 8 * nw) + 4 * N * (2 * d_in + d_out) + 8 * (N + 1)
-    per_edge_geo = ng * 2 * (3 + lmax_sh)
-    ff = E * (mul * ng * (2 * (lmax_sh + 1) + 2) + per_edge_geo) + N * mul * 2 * ng * (d_in + d_out)
-    bf = E * (mul * ng * (2 * (lmax_sh + 1) + 2 + 2 * (lmax_sh + 1) + 2 + 10) + per_edge_geo) + \
-        N * mul * 2 * ng * (2 * d_in + d_out)
+    bb = E * (4 + 12 + 8 * nw + (12 if need_gvec else 0)) + 4 * N * (2 * d_in + d_out) + 8 * (N + 1)
+    per_edge_geo = 2 * ng
+    ff = E * (mul * ng * (2 * lmax_sh + 2) + per_edge_geo) + N * mul * 2 * ng * (d_in + d_out)
+    per_point_b = (2 * lmax_sh + 2) + 1 + (2 * lmax_sh + 1) + ((2 * lmax_sh - 1 + 8) if need_gvec and lmax_sh else 0)
+    bf = E * (mul * ng * per_point_b + per_edge_geo) + N * mul * 2 * ng * (2 * d_in + d_out)
     return fb, bb, ff, bf
 
 

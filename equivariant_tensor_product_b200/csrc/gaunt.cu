@@ -15,8 +15,11 @@
 //                          gF[g] += S_e(g) Gq[dst][g][u];  gw[e, l2, u] = sum_g (2l2+1) P_l2(t_g) F_j(g) Gq(g);
 //                          gvec[e] = |v|^-1 sum_{g,u} F_j Gq S_e'(t_g) (r_g - t_g v_hat);
 //                          gx[j, u, lm] = sum_g Y_lm(r_g) gF[g]
-// Grid rows are node sized; nothing per edge is stored.  One warp per 32-channel slice of a
-// node, every warp of a CTA walking the node's edges in order; sums in fixed order.
+// Grid rows are node sized ([node][32-channel slice][pairs of grid points][lane]), nothing per
+// edge is stored; the pointwise work runs on two grid points per FFMA2, the filter by Horner's
+// rule of the plan's filter degree, and the backward computes the weight moments and the
+// direction terms only when their outputs are requested.  Warps per node: (slice, phase), the
+// phases splitting the node's edges; sums in fixed order.
 #include <algorithm>
 #include <cstring>
 #include <new>
@@ -38,7 +41,7 @@ struct GauntArgs {
   int in_off[4], out_off[4];   // offset of the block of degree l in a row, -1 when absent
   const int32_t *rowptr, *src, *colptr, *perm;
   const float *x, *vec, *w, *gy;
-  float *F, *Gq;               // [N][NG][mul]
+  float2 *F, *Gq;              // [N][nsl][NG / 2][32 lanes] pairs of grid points
   float *y, *gx, *gw, *gvec;
 };
 
@@ -51,30 +54,47 @@ __device__ __forceinline__ void filter_cubic(const float (&wl)[4], float (&c)[4]
   c[3] = 17.5f * wl[3];
 }
 
-// t_g = r_hat . r_g for every grid point, from the grid's product structure: r_g has
-// cos(theta) = ct(k), sin(theta) = st(k) and azimuth phi_j, so t = rz ct(k) + st(k) (rx cos phi_j + ry sin phi_j).
+__device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
+
+// t_g = r_hat . r_g for every grid point, in pairs of points, from the grid's product structure:
+// r_g has cos(theta) = ct(k), sin(theta) = st(k) and azimuth phi_j, so
+// t = rz ct(k) + st(k) (rx cos phi_j + ry sin phi_j).
 template <class Gr>
-__device__ __forceinline__ void grid_dots(float rx, float ry, float rz, float (&t)[Gr::NG]) {
-  float c[Gr::NP];
+__device__ __forceinline__ void grid_dots2(float rx, float ry, float rz, float2 (&t)[Gr::NG / 2]) {
+  float c[Gr::NP], z[Gr::NT];
 #pragma unroll
   for (int j = 0; j < Gr::NP; ++j) c[j] = fmaf(rx, Gr::cp(j), ry * Gr::sp(j));
 #pragma unroll
-  for (int k = 0; k < Gr::NT; ++k) {
-    const float z = rz * Gr::ct(k);
+  for (int k = 0; k < Gr::NT; ++k) z[k] = rz * Gr::ct(k);
 #pragma unroll
-    for (int j = 0; j < Gr::NP; ++j) t[k * Gr::NP + j] = fmaf(Gr::st(k), c[j], z);
+  for (int g2 = 0; g2 < Gr::NG / 2; ++g2) {
+    const int g0 = 2 * g2, g1 = 2 * g2 + 1;
+    t[g2] = make_float2(fmaf(Gr::st(g0 / Gr::NP), c[g0 % Gr::NP], z[g0 / Gr::NP]),
+                        fmaf(Gr::st(g1 / Gr::NP), c[g1 % Gr::NP], z[g1 / Gr::NP]));
   }
 }
 
+// Horner of degree D in pairs: sum_{d <= D} c_d t^d
+template <int D>
+__device__ __forceinline__ float2 horner2(const float (&c)[4], float2 t) {
+  float2 s = dup2(c[D]);
+#pragma unroll
+  for (int d = D - 1; d >= 0; --d) s = __ffma2_rn(s, t, dup2(c[d]));
+  return s;
+}
+
 // MODE 0: F from x (input blocks); MODE 1: Gq from gy (output blocks, times q_g).  One thread
-// per (node, channel).
+// per (node, slice, lane); lanes past the channel count write zeros.
 template <int L, int MODE>
 __global__ void __launch_bounds__(256) k_gaunt_to_grid(const __grid_constant__ GauntArgs a) {
   using Gr = gaunt::Grid<L>;
-  const int64_t total = (int64_t)a.N * a.mul;
+  const int64_t total = (int64_t)a.N * a.nsl * 32;
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t j = t / a.mul;
-    const int u = (int)(t - j * a.mul);
+    const int64_t js = t >> 5;            // node * nsl + slice
+    const int lane = (int)(t & 31);
+    const int64_t j = js / a.nsl;
+    const int u = (int)(js - j * a.nsl) * 32 + lane;
+    const bool act = u < a.mul;
     const float* row = MODE == 0 ? a.x + j * a.in_dim : a.gy + j * a.out_dim;
     const int* off = MODE == 0 ? a.in_off : a.out_off;
     float c[Gr::NSH];
@@ -82,44 +102,63 @@ __global__ void __launch_bounds__(256) k_gaunt_to_grid(const __grid_constant__ G
     for (int l = 0; l <= L; ++l) {
 #pragma unroll
       for (int m = 0; m < 2 * l + 1; ++m)
-        c[l * l + m] = off[l] >= 0 ? __ldg(row + off[l] + u * (2 * l + 1) + m) : 0.f;
+        c[l * l + m] = (act && off[l] >= 0) ? __ldg(row + off[l] + u * (2 * l + 1) + m) : 0.f;
     }
-    float* out = (MODE == 0 ? a.F : a.Gq) + j * (int64_t)Gr::NG * a.mul + u;
+    float2* out = (MODE == 0 ? a.F : a.Gq) + js * (Gr::NG / 2) * 32 + lane;
 #pragma unroll
-    for (int g = 0; g < Gr::NG; ++g) {
-      float v = 0.f;
+    for (int g2 = 0; g2 < Gr::NG / 2; ++g2) {
+      float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-      for (int k = 0; k < Gr::NSH; ++k) v = fmaf(c[k], Gr::Y(g, k), v);
-      out[(int64_t)g * a.mul] = MODE == 1 ? Gr::q(g) * v : v;
+      for (int k = 0; k < Gr::NSH; ++k) {
+        v0 = fmaf(c[k], Gr::Y(2 * g2, k), v0);
+        v1 = fmaf(c[k], Gr::Y(2 * g2 + 1, k), v1);
+      }
+      out[g2 * 32] = MODE == 1 ? make_float2(Gr::q(2 * g2) * v0, Gr::q(2 * g2 + 1) * v1) : make_float2(v0, v1);
     }
   }
 }
 
-// w_l2 (2l2+1 folded into E) of edge e for channel u; filter degrees above lmax_sh read as 0,
-// degrees above 0 of a zero-length edge too (its harmonics are Y_0 = 1, Y_l>0 = 0)
+// w_l2 (2l2+1 folded into the cubic) of edge e for channel u; filter degrees above LSH read as
+// 0, degrees above 0 of a zero-length edge too (its harmonics are Y_0 = 1, Y_l>0 = 0)
+template <int LSH>
 __device__ __forceinline__ void edge_weights(const GauntArgs& a, int e, int u, bool act, float ir, float (&wl)[4]) {
 #pragma unroll
   for (int l = 0; l < 4; ++l)
-    wl[l] = (act && l <= a.lmax_sh && (l == 0 || ir > 0.f)) ? __ldg(a.w + (int64_t)e * a.nw + l * a.mul + u) : 0.f;
+    wl[l] = (act && l <= LSH && (l == 0 || ir > 0.f)) ? __ldg(a.w + (int64_t)e * a.nw + l * a.mul + u) : 0.f;
 }
 
 // Forward: CTA = one receiver; warp w = (slice w / split, phase w % split); the phases take
 // interleaved edges of the row and their grid accumulators are added through shared memory in
-// phase order.  Each edge's grid row F[src][.][u] is loaded in one batch before the pointwise
-// math.
-template <int L>
+// phase order.  Per edge and lane (channel): the sender's grid row (pairs of points), the
+// filter by Horner's rule, acc += F S, all two points per FFMA2.  On grids of <= 32 points
+// the next edge's row is loaded while the current one is computed.
+template <int L, int LSH>
 __global__ void __launch_bounds__(128) k_gaunt_fwd(const __grid_constant__ GauntArgs a) {
   using Gr = gaunt::Grid<L>;
-  extern __shared__ float red[];             // [(split-1) * nsl][NG][32]
+  constexpr int NGP = Gr::NG / 2;
+  constexpr bool PF = Gr::NG <= 32;
+  extern __shared__ float2 red2[];            // [(split-1) * nsl][NGP][32]
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int st = a.split, sl = wid / st, phase = wid - sl * st;
   const int i = blockIdx.x;
   const int u = sl * 32 + lane;
   const bool act = u < a.mul;
   const int e0 = __ldg(a.rowptr + i), e1 = __ldg(a.rowptr + i + 1);
-  float acc[Gr::NG];
+  float2 acc[NGP];
 #pragma unroll
-  for (int g = 0; g < Gr::NG; ++g) acc[g] = 0.f;
+  for (int g = 0; g < NGP; ++g) acc[g] = make_float2(0.f, 0.f);
+  auto row_of = [&](int j) { return a.F + ((int64_t)j * a.nsl + sl) * NGP * 32 + lane; };
+  auto edge = [&](int e, float vx, float vy, float vz, const float2 (&f)[NGP]) {
+    float rx, ry, rz, ir;
+    edge_geometry(vx, vy, vz, rx, ry, rz, ir);
+    float wl[4], cf[4];
+    edge_weights<LSH>(a, e, u, act, ir, wl);
+    filter_cubic(wl, cf);
+    float2 t[NGP];
+    grid_dots2<Gr>(rx, ry, rz, t);
+#pragma unroll
+    for (int g = 0; g < NGP; ++g) acc[g] = __ffma2_rn(f[g], horner2<LSH>(cf, t[g]), acc[g]);
+  };
   for (int base = e0 + phase; base < e1; base += 32 * st) {
     const int my_e = base + lane * st;
     int my_j = 0;
@@ -131,71 +170,57 @@ __global__ void __launch_bounds__(128) k_gaunt_fwd(const __grid_constant__ Gaunt
       vz = __ldg(a.vec + 3 * (int64_t)my_e + 2);
     }
     const int ne = min(32, (e1 - base + st - 1) / st);
-    if constexpr (Gr::NG <= 32) {
-      // small grids: the row of edge k + 1 is loaded while edge k is computed (a larger grid
-      // would not fit two rows in registers)
-      float fn[Gr::NG];
+    if constexpr (PF) {
+      // two row buffers: the row of edge k + 1 is loaded while edge k is computed
+      float2 fa[NGP], fb[NGP];
       {
-        const int j0 = __shfl_sync(kFull, my_j, 0);
+        const float2* r = row_of(__shfl_sync(kFull, my_j, 0));
 #pragma unroll
-        for (int g = 0; g < Gr::NG; ++g) fn[g] = act ? __ldg(a.F + ((int64_t)j0 * Gr::NG + g) * a.mul + u) : 0.f;
+        for (int g = 0; g < NGP; ++g) fa[g] = r[g * 32];
       }
-      for (int k = 0; k < ne; ++k) {
-        float f[Gr::NG];
+      for (int k = 0; k < ne; k += 2) {
+        const bool two = k + 1 < ne;
+        {
+          const float2* r = row_of(__shfl_sync(kFull, my_j, min(k + 1, 31)));
+          if (two) {
 #pragma unroll
-        for (int g = 0; g < Gr::NG; ++g) f[g] = fn[g];
-        const int jn = __shfl_sync(kFull, my_j, min(k + 1, 31));
-        if (act && k + 1 < ne) {
-#pragma unroll
-          for (int g = 0; g < Gr::NG; ++g) fn[g] = __ldg(a.F + ((int64_t)jn * Gr::NG + g) * a.mul + u);
+            for (int g = 0; g < NGP; ++g) fb[g] = r[g * 32];
+          }
         }
-        float rx, ry, rz, ir;
-        edge_geometry(__shfl_sync(kFull, vx, k), __shfl_sync(kFull, vy, k), __shfl_sync(kFull, vz, k), rx, ry, rz, ir);
-        if (!act) continue;
-        float wl[4], cf[4], tg[Gr::NG];
-        edge_weights(a, base + k * st, u, act, ir, wl);
-        filter_cubic(wl, cf);
-        grid_dots<Gr>(rx, ry, rz, tg);
+        edge(base + k * st, __shfl_sync(kFull, vx, k), __shfl_sync(kFull, vy, k), __shfl_sync(kFull, vz, k), fa);
+        if (!two) break;
+        {
+          const float2* r = row_of(__shfl_sync(kFull, my_j, min(k + 2, 31)));
+          if (k + 2 < ne) {
 #pragma unroll
-        for (int g = 0; g < Gr::NG; ++g) {
-          const float s = fmaf(fmaf(fmaf(cf[3], tg[g], cf[2]), tg[g], cf[1]), tg[g], cf[0]);
-          acc[g] = fmaf(f[g], s, acc[g]);
+            for (int g = 0; g < NGP; ++g) fa[g] = r[g * 32];
+          }
         }
+        edge(base + (k + 1) * st, __shfl_sync(kFull, vx, k + 1), __shfl_sync(kFull, vy, k + 1),
+             __shfl_sync(kFull, vz, k + 1), fb);
       }
     } else {
       for (int k = 0; k < ne; ++k) {
-        const int j = __shfl_sync(kFull, my_j, k);
-        float rx, ry, rz, ir;
-        edge_geometry(__shfl_sync(kFull, vx, k), __shfl_sync(kFull, vy, k), __shfl_sync(kFull, vz, k), rx, ry, rz, ir);
-        if (!act) continue;
-        float wl[4], cf[4], tg[Gr::NG];
-        edge_weights(a, base + k * st, u, act, ir, wl);
-        filter_cubic(wl, cf);
-        const float* Fr = a.F + (int64_t)j * Gr::NG * a.mul + u;
-        float f[Gr::NG];
+        const float2* r = row_of(__shfl_sync(kFull, my_j, k));
+        float2 f[NGP];
 #pragma unroll
-        for (int g = 0; g < Gr::NG; ++g) f[g] = __ldg(Fr + (int64_t)g * a.mul);
-        grid_dots<Gr>(rx, ry, rz, tg);
-#pragma unroll
-        for (int g = 0; g < Gr::NG; ++g) {
-          const float s = fmaf(fmaf(fmaf(cf[3], tg[g], cf[2]), tg[g], cf[1]), tg[g], cf[0]);
-          acc[g] = fmaf(f[g], s, acc[g]);
-        }
+        for (int g = 0; g < NGP; ++g) f[g] = r[g * 32];
+        edge(base + k * st, __shfl_sync(kFull, vx, k), __shfl_sync(kFull, vy, k), __shfl_sync(kFull, vz, k), f);
       }
     }
   }
   if (st > 1) {
     if (phase > 0) {
-      float* dst = red + (((size_t)(phase - 1) * a.nsl + sl) * Gr::NG) * 32 + lane;
+      float2* dst = red2 + (((size_t)(phase - 1) * a.nsl + sl) * NGP) * 32 + lane;
 #pragma unroll
-      for (int g = 0; g < Gr::NG; ++g) dst[g * 32] = acc[g];
+      for (int g = 0; g < NGP; ++g) dst[g * 32] = acc[g];
     }
     __syncthreads();
     if (phase == 0) {
       for (int ph = 1; ph < st; ++ph) {
-        const float* srcp = red + (((size_t)(ph - 1) * a.nsl + sl) * Gr::NG) * 32 + lane;
+        const float2* srcp = red2 + (((size_t)(ph - 1) * a.nsl + sl) * NGP) * 32 + lane;
 #pragma unroll
-        for (int g = 0; g < Gr::NG; ++g) acc[g] += srcp[g * 32];
+        for (int g = 0; g < NGP; ++g) acc[g] = __fadd2_rn(acc[g], srcp[g * 32]);
       }
     }
   }
@@ -208,30 +233,39 @@ __global__ void __launch_bounds__(128) k_gaunt_fwd(const __grid_constant__ Gaunt
     for (int m = 0; m < 2 * l + 1; ++m) {
       float v = 0.f;
 #pragma unroll
-      for (int g = 0; g < Gr::NG; ++g) v = fmaf(Gr::q(g) * Gr::Y(g, l * l + m), acc[g], v);
+      for (int g = 0; g < NGP; ++g) {
+        v = fmaf(Gr::q(2 * g) * Gr::Y(2 * g, l * l + m), acc[g].x, v);
+        v = fmaf(Gr::q(2 * g + 1) * Gr::Y(2 * g + 1, l * l + m), acc[g].y, v);
+      }
       yr[a.out_off[l] + u * (2 * l + 1) + m] = v;
     }
   }
 }
 
 // Backward: CTA = one sender, warps as in the forward, out-edges in the stable transpose order.
-template <int L>
+// Per edge and lane: the receiver's grid row Gq (pairs), the filter S, gF += S Gq; with GW the
+// moments sum_g h t^n (n <= LSH) of h = F Gq give the weight gradient, (2l+1) P_l being a
+// polynomial in t; with GVEC the direction terms h S'(t) (r_g - t r_hat).
+template <int L, int LSH, bool GW, bool GVEC>
 __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ GauntArgs a) {
   using Gr = gaunt::Grid<L>;
-  extern __shared__ float red[];             // [(split-1) * nsl][NG][32]
-  __shared__ float part[4][32][4][4];        // [phase][edge of the batch][slice][4]: gvec partials
+  constexpr int NGP = Gr::NG / 2;
+  extern __shared__ float2 red2[];            // [(split-1) * nsl][NGP][32]
+  __shared__ float part[4][32][4][4];         // [phase][edge of the batch][slice][4]: gvec partials
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int st = a.split, sl = wid / st, phase = wid - sl * st;
   const int j = blockIdx.x;
   const int u = sl * 32 + lane;
   const bool act = u < a.mul;
   const int q0 = __ldg(a.colptr + j), q1 = __ldg(a.colptr + j + 1);
-  float Fj[Gr::NG], gF[Gr::NG];
-  const float* Fr = a.F + (int64_t)j * Gr::NG * a.mul + u;
+  float2 Fj[NGP], gF[NGP];
+  {
+    const float2* Fr = a.F + ((int64_t)j * a.nsl + sl) * NGP * 32 + lane;
 #pragma unroll
-  for (int g = 0; g < Gr::NG; ++g) {
-    Fj[g] = act ? __ldg(Fr + (int64_t)g * a.mul) : 0.f;
-    gF[g] = 0.f;
+    for (int g = 0; g < NGP; ++g) {
+      Fj[g] = Fr[g * 32];
+      gF[g] = make_float2(0.f, 0.f);
+    }
   }
   for (int base = q0 + phase; base < q1; base += 32 * st) {
     const int my_q = base + lane * st;
@@ -250,45 +284,62 @@ __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ Gaunt
       float rx, ry, rz, ir;
       edge_geometry(__shfl_sync(kFull, vx, k), __shfl_sync(kFull, vy, k), __shfl_sync(kFull, vz, k), rx, ry, rz, ir);
       float wl[4];
-      edge_weights(a, e, u, act, ir, wl);
-      float gw[4] = {0.f, 0.f, 0.f, 0.f};
+      edge_weights<LSH>(a, e, u, act, ir, wl);
       float hx = 0.f, hy = 0.f, hz = 0.f, hs = 0.f;
-      if (act) {
-        const float* Gp = a.Gq + (int64_t)i * Gr::NG * a.mul + u;
-        float gq[Gr::NG], tg[Gr::NG], cf[4];
+      {
+        const float2* Gp = a.Gq + ((int64_t)i * a.nsl + sl) * NGP * 32 + lane;
+        float2 gq[NGP], t[NGP];
+        float cf[4];
 #pragma unroll
-        for (int g = 0; g < Gr::NG; ++g) gq[g] = __ldg(Gp + (int64_t)g * a.mul);
+        for (int g = 0; g < NGP; ++g) gq[g] = Gp[g * 32];
         filter_cubic(wl, cf);
-        grid_dots<Gr>(rx, ry, rz, tg);
-        // moments sum_g h t^n give the weight gradient: (2l+1) P_l(t) is a cubic in t
-        float M0 = 0.f, M1 = 0.f, M2 = 0.f, M3 = 0.f;
+        grid_dots2<Gr>(rx, ry, rz, t);
+        float2 M[LSH + 1];
 #pragma unroll
-        for (int g = 0; g < Gr::NG; ++g) {
-          const float t = tg[g];
-          const float s = fmaf(fmaf(fmaf(cf[3], t, cf[2]), t, cf[1]), t, cf[0]);
-          gF[g] = fmaf(s, gq[g], gF[g]);
-          const float h = Fj[g] * gq[g];
-          const float ht = h * t, ht2 = ht * t;
-          M0 += h;
-          M1 += ht;
-          M2 += ht2;
-          M3 = fmaf(ht2, t, M3);
-          const float c = h * fmaf(fmaf(3.f * cf[3], t, 2.f * cf[2]), t, cf[1]);   // h s'(t)
-          hx = fmaf(c, Gr::st(g / Gr::NP) * Gr::cp(g % Gr::NP), hx);
-          hy = fmaf(c, Gr::st(g / Gr::NP) * Gr::sp(g % Gr::NP), hy);
-          hz = fmaf(c, Gr::ct(g / Gr::NP), hz);
-          hs = fmaf(c, t, hs);
+        for (int n = 0; n <= LSH; ++n) M[n] = make_float2(0.f, 0.f);
+        const float dc[4] = {cf[1], 2.f * cf[2], 3.f * cf[3], 0.f};   // S'(t)
+#pragma unroll
+        for (int g = 0; g < NGP; ++g) {
+          gF[g] = __ffma2_rn(horner2<LSH>(cf, t[g]), gq[g], gF[g]);
+          if constexpr (GW || GVEC) {
+            const float2 h = __fmul2_rn(Fj[g], gq[g]);
+            if constexpr (GW) {
+              float2 ht = h;
+              M[0] = __fadd2_rn(M[0], ht);
+#pragma unroll
+              for (int n = 1; n <= LSH; ++n) {
+                ht = __fmul2_rn(ht, t[g]);
+                M[n] = __fadd2_rn(M[n], ht);
+              }
+            }
+            if constexpr (GVEC && LSH > 0) {
+              const float2 c2 = __fmul2_rn(h, horner2<LSH - 1>(dc, t[g]));   // h S'(t)
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const int gg = 2 * g + hh;
+                const float c = hh ? c2.y : c2.x;
+                hx = fmaf(c, Gr::st(gg / Gr::NP) * Gr::cp(gg % Gr::NP), hx);
+                hy = fmaf(c, Gr::st(gg / Gr::NP) * Gr::sp(gg % Gr::NP), hy);
+                hz = fmaf(c, Gr::ct(gg / Gr::NP), hz);
+                hs = fmaf(c, hh ? t[g].y : t[g].x, hs);
+              }
+            }
+          }
         }
-        gw[0] = M0;
-        gw[1] = 3.f * M1;
-        gw[2] = fmaf(7.5f, M2, -2.5f * M0);
-        gw[3] = fmaf(17.5f, M3, -10.5f * M1);
-        if (a.gw) {
-          for (int l = 0; l <= a.lmax_sh; ++l)
-            a.gw[(int64_t)e * a.nw + l * a.mul + u] = (l == 0 || ir > 0.f) ? gw[l] : 0.f;
+        if constexpr (GW) {
+          float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int n = 0; n <= LSH; ++n) m[n] = M[n].x + M[n].y;
+          // (2l+1) P_l(t) = 1, 3t, 7.5t^2 - 2.5, 17.5t^3 - 10.5t
+          const float gw[4] = {m[0], 3.f * m[1], fmaf(7.5f, m[2], -2.5f * m[0]), fmaf(17.5f, m[3], -10.5f * m[1])};
+          if (act) {
+#pragma unroll
+            for (int l = 0; l <= LSH; ++l)
+              a.gw[(int64_t)e * a.nw + l * a.mul + u] = (l == 0 || ir > 0.f) ? gw[l] : 0.f;
+          }
         }
       }
-      if (a.gvec) {
+      if constexpr (GVEC) {
         hx = warp_sum(hx);
         hy = warp_sum(hy);
         hz = warp_sum(hz);
@@ -308,7 +359,7 @@ __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ Gaunt
         }
       }
     }
-    if (a.gvec && a.nsl > 1) {
+    if (GVEC && a.nsl > 1) {
       // the slices of this phase have written their partials of the batch's edges
       named_barrier(1 + phase, 32 * a.nsl);
       if (sl == 0 && lane < ne) {
@@ -331,16 +382,16 @@ __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ Gaunt
   }
   if (st > 1) {
     if (phase > 0) {
-      float* dst = red + (((size_t)(phase - 1) * a.nsl + sl) * Gr::NG) * 32 + lane;
+      float2* dst = red2 + (((size_t)(phase - 1) * a.nsl + sl) * NGP) * 32 + lane;
 #pragma unroll
-      for (int g = 0; g < Gr::NG; ++g) dst[g * 32] = gF[g];
+      for (int g = 0; g < NGP; ++g) dst[g * 32] = gF[g];
     }
     __syncthreads();
     if (phase == 0) {
       for (int ph = 1; ph < st; ++ph) {
-        const float* srcp = red + (((size_t)(ph - 1) * a.nsl + sl) * Gr::NG) * 32 + lane;
+        const float2* srcp = red2 + (((size_t)(ph - 1) * a.nsl + sl) * NGP) * 32 + lane;
 #pragma unroll
-        for (int g = 0; g < Gr::NG; ++g) gF[g] += srcp[g * 32];
+        for (int g = 0; g < NGP; ++g) gF[g] = __fadd2_rn(gF[g], srcp[g * 32]);
       }
     }
   }
@@ -353,7 +404,10 @@ __global__ void __launch_bounds__(128) k_gaunt_bwd(const __grid_constant__ Gaunt
     for (int m = 0; m < 2 * l + 1; ++m) {
       float v = 0.f;
 #pragma unroll
-      for (int g = 0; g < Gr::NG; ++g) v = fmaf(Gr::Y(g, l * l + m), gF[g], v);
+      for (int g = 0; g < NGP; ++g) {
+        v = fmaf(Gr::Y(2 * g, l * l + m), gF[g].x, v);
+        v = fmaf(Gr::Y(2 * g + 1, l * l + m), gF[g].y, v);
+      }
       gr[a.in_off[l] + u * (2 * l + 1) + m] = v;
     }
   }
@@ -367,24 +421,50 @@ unsigned node_grid(int64_t n) {
 
 template <int L>
 size_t red_bytes(const GauntArgs& a) {
-  return sizeof(float) * (size_t)(a.split - 1) * a.nsl * gaunt::Grid<L>::NG * 32;
+  return sizeof(float2) * (size_t)(a.split - 1) * a.nsl * (gaunt::Grid<L>::NG / 2) * 32;
 }
 
-template <int L>
+template <int L, int LSH>
 cudaError_t gaunt_fwd_seq(const GauntArgs& a, cudaStream_t s) {
-  k_gaunt_to_grid<L, 0><<<node_grid((int64_t)a.N * a.mul), 256, 0, s>>>(a);
-  k_gaunt_fwd<L><<<(unsigned)a.N, 32 * a.nsl * a.split, red_bytes<L>(a), s>>>(a);
+  k_gaunt_to_grid<L, 0><<<node_grid((int64_t)a.N * a.nsl * 32), 256, 0, s>>>(a);
+  k_gaunt_fwd<L, LSH><<<(unsigned)a.N, 32 * a.nsl * a.split, red_bytes<L>(a), s>>>(a);
   count_launches(2);
   return cudaGetLastError();
 }
 
-template <int L>
+template <int L, int LSH>
 cudaError_t gaunt_bwd_seq(const GauntArgs& a, cudaStream_t s) {
-  k_gaunt_to_grid<L, 0><<<node_grid((int64_t)a.N * a.mul), 256, 0, s>>>(a);
-  k_gaunt_to_grid<L, 1><<<node_grid((int64_t)a.N * a.mul), 256, 0, s>>>(a);
-  k_gaunt_bwd<L><<<(unsigned)a.N, 32 * a.nsl * a.split, red_bytes<L>(a), s>>>(a);
+  k_gaunt_to_grid<L, 0><<<node_grid((int64_t)a.N * a.nsl * 32), 256, 0, s>>>(a);
+  k_gaunt_to_grid<L, 1><<<node_grid((int64_t)a.N * a.nsl * 32), 256, 0, s>>>(a);
+  const unsigned grid = (unsigned)a.N, threads = 32 * a.nsl * a.split;
+  const size_t rb = red_bytes<L>(a);
+  if (a.gvec) {
+    if (a.gw) k_gaunt_bwd<L, LSH, true, true><<<grid, threads, rb, s>>>(a);
+    else k_gaunt_bwd<L, LSH, false, true><<<grid, threads, rb, s>>>(a);
+  } else {
+    if (a.gw) k_gaunt_bwd<L, LSH, true, false><<<grid, threads, rb, s>>>(a);
+    else k_gaunt_bwd<L, LSH, false, false><<<grid, threads, rb, s>>>(a);
+  }
   count_launches(3);
   return cudaGetLastError();
+}
+
+// dispatch over (grid degree L, filter degree LSH <= L)
+template <bool FWD>
+cudaError_t gaunt_seq(int L, int LSH, const GauntArgs& a, cudaStream_t s) {
+#define TP_GAUNT_CASE(LL, SS) \
+  if (L == LL && LSH == SS) return FWD ? gaunt_fwd_seq<LL, SS>(a, s) : gaunt_bwd_seq<LL, SS>(a, s);
+  TP_GAUNT_CASE(1, 0)
+  TP_GAUNT_CASE(1, 1)
+  TP_GAUNT_CASE(2, 0)
+  TP_GAUNT_CASE(2, 1)
+  TP_GAUNT_CASE(2, 2)
+  TP_GAUNT_CASE(3, 0)
+  TP_GAUNT_CASE(3, 1)
+  TP_GAUNT_CASE(3, 2)
+  TP_GAUNT_CASE(3, 3)
+#undef TP_GAUNT_CASE
+  return cudaErrorInvalidValue;
 }
 
 size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -430,7 +510,9 @@ bool gaunt_irreps(const char* s, int& mul, int (&off)[4], int64_t& dim, std::str
 
 int grid_points(int L) { return L == 1 ? tp::gaunt::Grid<1>::NG : L == 2 ? tp::gaunt::Grid<2>::NG : tp::gaunt::Grid<3>::NG; }
 
-size_t grid_bytes(const tp_gaunt_s* p, int64_t N) { return tp::al256(sizeof(float) * (size_t)(N > 0 ? N : 1) * p->ng * p->mul); }
+size_t grid_bytes(const tp_gaunt_s* p, int64_t N) {
+  return tp::al256(sizeof(float) * (size_t)(N > 0 ? N : 1) * p->ng * 32 * (size_t)((p->mul + 31) / 32));
+}
 
 // header 256 | colptr[N+1] | perm[E] | transpose scratch  (the transpose region of the backward)
 size_t transpose_bytes(int64_t N, int64_t E) {
@@ -539,10 +621,9 @@ tp_status_t tp_gaunt_fwd(tp_gaunt_t plan, int64_t N, int64_t E, const int32_t* r
   a.vec = vec;
   a.w = w;
   a.y = y;
-  a.F = static_cast<float*>(ws);
+  a.F = static_cast<float2*>(ws);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = plan->L == 1 ? tp::gaunt_fwd_seq<1>(a, s) : plan->L == 2 ? tp::gaunt_fwd_seq<2>(a, s)
-                                                                            : tp::gaunt_fwd_seq<3>(a, s);
+  cudaError_t e = tp::gaunt_seq<true>(plan->L, plan->lmax_sh, a, s);
   if (e != cudaSuccess) return tp::set_failure(TP_ERR_CUDA, std::string("tp_gaunt_fwd: ") + cudaGetErrorString(e));
   return TP_OK;
 }
@@ -591,10 +672,9 @@ tp_status_t tp_gaunt_bwd(tp_gaunt_t plan, int64_t N, int64_t E, const int32_t* r
   a.gx = gx;
   a.gw = gw;
   a.gvec = gvec;
-  a.F = reinterpret_cast<float*>(wsb);
-  a.Gq = reinterpret_cast<float*>(wsb + gb);
-  cudaError_t e = plan->L == 1 ? tp::gaunt_bwd_seq<1>(a, s) : plan->L == 2 ? tp::gaunt_bwd_seq<2>(a, s)
-                                                                            : tp::gaunt_bwd_seq<3>(a, s);
+  a.F = reinterpret_cast<float2*>(wsb);
+  a.Gq = reinterpret_cast<float2*>(wsb + gb);
+  cudaError_t e = tp::gaunt_seq<false>(plan->L, plan->lmax_sh, a, s);
   if (e != cudaSuccess) return tp::set_failure(TP_ERR_CUDA, std::string("tp_gaunt_bwd: ") + cudaGetErrorString(e));
   return TP_OK;
 }

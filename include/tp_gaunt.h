@@ -40,9 +40,9 @@ tp_status_t tp_gaunt_destroy(tp_gaunt_t plan);
 tp_status_t tp_gaunt_query(tp_gaunt_t plan, int64_t* in_dim, int64_t* out_dim, int64_t* n_edge_weights,
                            int32_t* grid_points);
 
-/* Workspace bytes: forward N x grid x u floats (the node features on the grid); backward
- * twice that (also the receivers' adjoint on the grid) plus room to build the transpose
- * (int32) when colptr / perm are not given. */
+/* Workspace bytes: forward N x grid x 32 ceil(u / 32) floats (the node features on the grid, in
+ * 32-channel slices); backward twice that (also the receivers' adjoint on the grid) plus room
+ * to build the transpose (int32) when colptr / perm are not given. */
 tp_status_t tp_gaunt_workspace_size(tp_gaunt_t plan, int64_t N, int64_t E, int32_t op, size_t* bytes);
 
 /* Forward: y[N, out_dim]. */
