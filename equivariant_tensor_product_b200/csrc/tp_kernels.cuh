@@ -311,7 +311,7 @@ struct GatherFwd {
 };
 
 template <class S>
-__global__ void __launch_bounds__(kMaxThreads, 4) k_fwd_uvu_gather(const __grid_constant__ LaunchArgs a) {
+__global__ void __launch_bounds__(kMaxThreads, S::IN_PC + S::P + S::OUT_PC <= 48 ? 4 : 2) k_fwd_uvu_gather(const __grid_constant__ LaunchArgs a) {
   using G = GatherFwd<S>;
   constexpr int MUL = 32;
   constexpr int in_dim = S::IN_PC * MUL, nw = S::P * MUL;
@@ -930,7 +930,7 @@ struct FwdLaunch {
   cudaStream_t s;
   template <int MUL, bool FAST>
   cudaError_t run() const {
-    if constexpr (kPrefetch<S> && MUL == 32 && FAST) {
+    if constexpr (MUL == 32 && FAST) {
       // rows start on 16-byte boundaries: stage them with the copy engine
       if (((reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.w)) & 15u) == 0) {
         const size_t sm = GatherFwd<S>::smem_bytes(a.split);
