@@ -115,6 +115,37 @@ def test_uvw_channel_counts_and_long_rows(tp, mul_in, mul_out, cfg):
     assert_close(gW2.view(ref["gW"].shape), ref["gW"], f"uvw {mul_in}/{mul_out} gW (no gvec)")
 
 
+def test_uvw_path_coefficients(tp):
+    """Non-unit path coefficients through the uvw edge passes (the coupling matrices fold c_p
+    in with s[e, p] in the receiver pass and into K_e in the sender pass)."""
+    spec = synth.CONFIGS["c4"]
+    ins, outs = _irreps(spec.irreps_in, 128), _irreps(spec.irreps_out, 64)
+    coeff = np.linspace(-1.5, 2.0, len(spec.paths))
+    plan = tp.Plan(ins, spec.irreps_sh, outs, spec.paths, "uvw", path_coeff=coeff)
+    op = OraclePlan(ins, spec.irreps_sh, outs, spec.paths, "uvw", path_coeff=coeff)
+    rng = np.random.default_rng(11)
+    N = 40
+    rowptr, src, vec = _graph(rng, N, DEGREES[:10])
+    E = len(src)
+    P = len(spec.paths)
+    x = rng.standard_normal((N, plan.in_dim)).astype(np.float32)
+    s = rng.standard_normal((E, P)).astype(np.float32)
+    W = (rng.standard_normal((P, 128, 64)) / np.sqrt(128)).astype(np.float32)
+    gy = rng.standard_normal((N, plan.out_dim)).astype(np.float32)
+    g = dict(rowptr=dev(rowptr), src=dev(src), x=dev(x), vec=dev(vec), s=dev(s), W=dev(W), gy=dev(gy))
+    y = tp.tp_conv_fwd(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["s"], W=g["W"])
+    assert_close(y, forward(op, rowptr, src, x, vec, s=s, W=W), "uvw coeff y")
+    ref = backward(op, rowptr, src, x, vec, gy, s=s, W=W)
+    for need_gvec in (False, True):
+        gx, gs, gvec, gW = tp.tp_conv_bwd(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["s"], g["gy"], W=g["W"],
+                                          need_gvec=need_gvec, need_gW=True)
+        assert_close(gx, ref["gx"], f"uvw coeff gx ({need_gvec})")
+        assert_close(gs, ref["gs"], f"uvw coeff gs ({need_gvec})")
+        assert_close(gW.view(ref["gW"].shape), ref["gW"], f"uvw coeff gW ({need_gvec})")
+        if need_gvec:
+            assert_close(gvec, ref["gvec"], "uvw coeff gvec")
+
+
 def test_rows_off_16_byte_boundaries_take_the_general_path(tp):
     spec = synth.CONFIGS["c2"]
     d = synth.make_inputs("c2", 192)
