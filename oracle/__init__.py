@@ -21,6 +21,11 @@ coupling, graph aggregation) and "The GPU Workload That Rewrites Molecular Physi
 products).  Backward and double backward are the vector-Jacobian products of this map
 ("Sobek", abstract: forward, backward and double backward), taken by torch autograd.
 
+``oracle.radial`` composes the same map with the radial projection fused in: the uvu
+weights formed as w = h @ W_r from the radial network's last hidden layer ("Sobek",
+abstract: the radial projection reordered so that edge-specific weights are never
+materialised), with its backward to (x, vec, h, W_r) by autograd.
+
 ``oracle.gaunt`` holds the second operator, the spherical-grid (Gaunt) tensor-product
 convolution ("The Price of Freedom: Exploring Expressivity and Runtime Tradeoffs in
 Equivariant Tensor Products", abstract), with its Gaunt coefficients integrated on an exact
@@ -34,3 +39,4 @@ scipy.sparse SpMV, finite differences, gradgradcheck and a pure-Python brute-for
 from .irreps import Irreps, OraclePlan  # noqa: F401
 from .so3 import real_sh, wigner_D, cg_real, random_rotation  # noqa: F401
 from .conv import forward, backward, double_backward, forward_uvw_reassociated  # noqa: F401
+from .radial import forward_radial, backward_radial  # noqa: F401

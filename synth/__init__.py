@@ -255,6 +255,30 @@ def _radial_weights(rng, r: np.ndarray, cutoff: float, hidden, n_out: int,
     return out
 
 
+def radial_hidden(d: dict, seed: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Inputs of the convolution with the radial projection fused in, for workload ``d``:
+    the radial network's last hidden layer h[E, H] (the Bessel basis of |vec| through the
+    workload's bias-free hidden layers with SiLU, N(0, 1/fan_in) weights) and its output
+    layer W_r[H, nw] (N(0, 1/H)), both float64 -> float32.  Its own seed, so the workload's
+    other arrays are unchanged."""
+    spec = d["spec"]
+    rng = np.random.default_rng(spec.seed + 7919 if seed is None else seed)
+    sizes = [8] + list(spec.mlp_hidden)
+    mats = [rng.normal(0.0, 1.0 / math.sqrt(a), size=(a, b)) for a, b in zip(sizes[:-1], sizes[1:])]
+    H, nw = sizes[-1], n_edge_weights(spec)
+    Wr = rng.normal(0.0, 1.0 / math.sqrt(H), size=(H, nw)).astype(np.float32)
+    r = np.linalg.norm(np.asarray(d["vec"], dtype=np.float64), axis=1)
+    h = np.empty((len(r), H), dtype=np.float32)
+    nb = np.arange(1, 9, dtype=np.float64)
+    for s in range(0, len(r), 65536):
+        rr = np.maximum(r[s:s + 65536], 1e-9)[:, None]
+        z = math.sqrt(2.0 / spec.cutoff) * np.sin(nb * math.pi * rr / spec.cutoff) / rr
+        for m in mats:
+            z = _silu(z @ m)
+        h[s:s + 65536] = z
+    return h, Wr
+
+
 # ---------------------------------------------------------------------------
 # Public generator
 # ---------------------------------------------------------------------------

@@ -36,3 +36,14 @@ def test_cell_sorted_is_a_relabelling_of_the_same_workload():
     # spatial labels: senders sit closer to their receivers in label space
     gap = lambda g: np.abs(g["src"].astype(np.int64) - g["dst"]).mean()
     assert gap(e) < gap(d)
+
+
+def test_radial_hidden_inputs_are_seeded_and_shaped():
+    d = synth.make_inputs("c1")
+    h, Wr = synth.radial_hidden(d)
+    h2, Wr2 = synth.radial_hidden(synth.make_inputs("c1"))
+    H = d["spec"].mlp_hidden[-1]
+    assert h.shape == (len(d["src"]), H) and Wr.shape == (H, d["w"].shape[1])
+    assert h.dtype == np.float32 and Wr.dtype == np.float32
+    assert np.array_equal(h, h2) and np.array_equal(Wr, Wr2)
+    assert np.all(np.isfinite(h)) and np.abs(h).max() > 0
