@@ -32,6 +32,10 @@ SIGNATURES = {
                               _p]),
     "tp_conv_dbwd": (C.c_int, [_p, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                _p, _p, _sz, _p]),
+    "tp_radial_workspace_size": (C.c_int, [_p, _i64, _i64, _i32, _i32, C.POINTER(_sz)]),
+    "tp_conv_fwd_radial": (C.c_int, [_p, _i64, _i64, _i32, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "tp_conv_bwd_radial": (C.c_int, [_p, _i64, _i64, _i32, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
+                                     _p, _p, _sz, _p]),
     "tp_get_device_error": (C.c_int, [_p, _p, _p, C.POINTER(_i32)]),
     "tp_gather_rows": (C.c_int, [_p, _i64, _p, _i64, _p, _p]),
     "tp_add_rows": (C.c_int, [_p, _i64, _p, _i64, _p, _p]),

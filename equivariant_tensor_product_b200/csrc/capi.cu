@@ -23,6 +23,7 @@ struct IrrepBlock {
 struct tp_plan_s {
   const SpecOps* ops;   // compiled specialisation, or NULL: runtime path table `gen`
   GenTable* gen;
+  GenTable* rad;        // uvu: the path table of the fused radial projection (== gen when set)
   int mode;
   int mul_in, mul_out;
   int64_t in_dim, out_dim, nw, n_shared;
@@ -354,6 +355,52 @@ int* device_error_ptr() { return device_error_word(); }
 
 }  // namespace tp
 
+namespace {
+
+// Host checks shared by the radial entry points; fills the sizes of `a`.
+tp_status_t radial_args(tp_plan_t plan, int64_t N, int64_t E, int32_t H, RadArgs& a) {
+  tp_status_t st = check_sizes(plan, N, E);
+  if (st != TP_OK) return st;
+  if (plan->mode != TP_MODE_UVU || !plan->rad)
+    return fail(TP_ERR_UNSUPPORTED, "the fused radial projection is implemented for uvu plans");
+  if (H < 4 || H > kRadMaxHidden || H % 4 != 0)
+    return fail(TP_ERR_UNSUPPORTED, "hidden width must be a multiple of 4 in [4, %d]", kRadMaxHidden);
+  std::memset(&a, 0, sizeof(a));
+  a.N = (int)N;
+  a.E = (int)E;
+  a.H = H;
+  a.nw = (int)plan->nw;
+  a.nwp = (a.nw + 3) & ~3;
+  a.in_dim = (int)plan->in_dim;
+  a.out_dim = (int)plan->out_dim;
+  a.check = (plan->flags & TP_FLAG_CHECK_INDICES) ? 1 : 0;
+  a.splits = rad_splits(*plan->rad, E);
+  a.mul = plan->mul_in;
+  a.spec = 0;
+  if (plan->ops && std::strcmp(plan->ops->name, "full_l2") == 0) a.spec = 2;
+  if (plan->ops && std::strcmp(plan->ops->name, "full_l3") == 0) a.spec = 3;
+  if (rad_chunk(a, false, nullptr) == 0 || rad_chunk(a, true, nullptr) == 0)
+    return fail(TP_ERR_UNSUPPORTED, "%d weights per edge do not fit the shared-memory chunk of four edges", a.nw);
+  return TP_OK;
+}
+
+struct RadLayout {
+  size_t WrT, part, total;
+};
+// backward: the transpose region, then W_r^T [nw, H] and the gW_r partials [splits, H, nw]
+RadLayout rad_layout(const RadArgs& a) {
+  RadLayout L{};
+  size_t off = ws_layout(a.N, a.E).total;
+  L.WrT = off;
+  off += align256(sizeof(float) * (size_t)a.H * a.nw);
+  L.part = off;
+  off += align256(sizeof(float) * (size_t)a.H * a.nw * a.splits);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* tp_version(void) { return "tp-b200 0.1 (sm_100a)"; }
@@ -451,11 +498,26 @@ tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* i
       return fail(TP_ERR_UNSUPPORTED, "%s", why2.c_str());
     }
   }
+  // the fused radial projection runs through the path table for every uvu plan
+  GenTable* rad = gen;
+  if (mode == TP_MODE_UVU && !rad) {
+    rad = new (std::nothrow) GenTable;
+    std::string why3;
+    if (rad && !build_gen_table(bi, bs, bo, paths, n_paths, path_coeff, false, *rad, why3)) {
+      delete rad;
+      rad = nullptr;
+    }
+  }
   tp_plan_s* pl = new (std::nothrow) tp_plan_s;
-  if (!pl) return fail(TP_ERR_INVALID_ARG, "out of host memory");
+  if (!pl) {
+    if (rad != gen) delete rad;
+    delete gen;
+    return fail(TP_ERR_INVALID_ARG, "out of host memory");
+  }
   std::memset(pl, 0, sizeof(*pl));
   pl->ops = found;
   pl->gen = gen;
+  pl->rad = mode == TP_MODE_UVU ? rad : nullptr;
   pl->mode = mode;
   pl->mul_in = mul_in;
   pl->mul_out = mul_out;
@@ -474,6 +536,7 @@ tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* i
   if (path_coeff) {
     for (int p = 0; p < n_paths; ++p) {
       if (!std::isfinite(path_coeff[p])) {
+        if (pl->rad != pl->gen) delete pl->rad;
         delete pl->gen;
         delete pl;
         return fail(TP_ERR_INVALID_ARG, "path_coeff[%d] is not finite", p);
@@ -488,6 +551,7 @@ tp_status_t tp_plan_create(tp_plan_t* plan, const char* irreps_in, const char* i
 }
 
 tp_status_t tp_plan_destroy(tp_plan_t plan) {
+  if (plan && plan->rad != plan->gen) delete plan->rad;
   if (plan) delete plan->gen;
   delete plan;
   return TP_OK;
@@ -752,6 +816,97 @@ tp_status_t tp_conv_dbwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* ro
   }
   cudaError_t e = plan->ops->dbwd_send(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "tp_conv_dbwd sender pass");
+  return TP_OK;
+}
+
+tp_status_t tp_radial_workspace_size(tp_plan_t plan, int64_t N, int64_t E, int32_t H, int32_t op, size_t* bytes) {
+  RadArgs a;
+  tp_status_t st = radial_args(plan, N, E, H, a);
+  if (st != TP_OK) return st;
+  if (!bytes) return fail(TP_ERR_INVALID_ARG, "bytes is NULL");
+  if (op == TP_OP_FWD) *bytes = (plan->flags & TP_FLAG_CHECK_INDICES) ? 256 : 0;
+  else if (op == TP_OP_BWD) *bytes = rad_layout(a).total;
+  else return fail(TP_ERR_UNSUPPORTED, "the fused radial projection has a forward and a backward");
+  return TP_OK;
+}
+
+tp_status_t tp_conv_fwd_radial(tp_plan_t plan, int64_t N, int64_t E, int32_t H, const int32_t* rowptr,
+                               const int32_t* src, const float* x, const float* vec, const float* h,
+                               const float* Wr, float* y, void* ws, size_t ws_bytes, tp_stream_t stream) {
+  RadArgs a;
+  tp_status_t st = radial_args(plan, N, E, H, a);
+  if (st != TP_OK) return st;
+  if (N == 0) return TP_OK;
+  if (!rowptr || !x || !y || !Wr) return fail(TP_ERR_INVALID_ARG, "rowptr, x, Wr and y must not be NULL");
+  if (E > 0 && (!src || !vec || !h)) return fail(TP_ERR_INVALID_ARG, "src, vec and h must not be NULL");
+  for (const void* p : {(const void*)rowptr, (const void*)src, (const void*)x, (const void*)vec, (const void*)h,
+                        (const void*)Wr, (const void*)y})
+    if (!aligned4(p)) return fail(TP_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(h) & 15u) != 0) return fail(TP_ERR_INVALID_ARG, "h must be 16-byte aligned");
+  if ((plan->flags & TP_FLAG_CHECK_INDICES) && (!ws || ws_bytes < 256))
+    return fail(TP_ERR_WORKSPACE, "TP_FLAG_CHECK_INDICES needs a 256-byte workspace");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = debug_prologue(plan, N, E, rowptr, src, ws, s, &a.err);
+  if (st != TP_OK) return st;
+  a.rowptr = rowptr;
+  a.src = src;
+  a.x = x;
+  a.vec = vec;
+  a.h = h;
+  a.Wr = Wr;
+  a.y = y;
+  cudaError_t e = launch_rad_fwd(a, *plan->rad, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tp_conv_fwd_radial launch");
+  return TP_OK;
+}
+
+tp_status_t tp_conv_bwd_radial(tp_plan_t plan, int64_t N, int64_t E, int32_t H, const int32_t* rowptr,
+                               const int32_t* src, const int32_t* colptr, const int32_t* perm, const float* x,
+                               const float* vec, const float* h, const float* Wr, const float* gy, float* gx,
+                               float* gh, float* gWr, float* gvec, void* ws, size_t ws_bytes, tp_stream_t stream) {
+  RadArgs a;
+  tp_status_t st = radial_args(plan, N, E, H, a);
+  if (st != TP_OK) return st;
+  if (N == 0) {
+    if (gWr && H > 0) {
+      cudaError_t e = cudaMemsetAsync(gWr, 0, sizeof(float) * (size_t)H * plan->nw, reinterpret_cast<cudaStream_t>(stream));
+      if (e != cudaSuccess) return cuda_fail(e, "tp_conv_bwd_radial");
+    }
+    return TP_OK;
+  }
+  if (!rowptr || !x || !gy || !Wr) return fail(TP_ERR_INVALID_ARG, "rowptr, x, Wr and gy must not be NULL");
+  if (E > 0 && (!src || !vec || !h)) return fail(TP_ERR_INVALID_ARG, "src, vec and h must not be NULL");
+  for (const void* p : {(const void*)rowptr, (const void*)src, (const void*)colptr, (const void*)perm,
+                        (const void*)x, (const void*)vec, (const void*)h, (const void*)Wr, (const void*)gy,
+                        (const void*)gx, (const void*)gh, (const void*)gWr, (const void*)gvec})
+    if (!aligned4(p)) return fail(TP_ERR_INVALID_ARG, "pointers must be 4-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(h) & 15u) != 0) return fail(TP_ERR_INVALID_ARG, "h must be 16-byte aligned");
+  if (!gx && !gh && !gWr && !gvec) return TP_OK;
+  const RadLayout L = rad_layout(a);
+  if (!ws || ws_bytes < L.total) return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes", L.total);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = debug_prologue(plan, N, E, rowptr, src, ws, s, &a.err);
+  if (st != TP_OK) return st;
+  st = sender_order(N, E, src, colptr, perm, ws, ws_bytes, s);
+  if (st != TP_OK) return st;
+  char* wsb = static_cast<char*>(ws);
+  a.rowptr = rowptr;
+  a.src = src;
+  a.colptr = colptr;
+  a.perm = perm;
+  a.x = x;
+  a.vec = vec;
+  a.h = h;
+  a.Wr = Wr;
+  a.gy = gy;
+  a.gx = gx;
+  a.gh = gh;
+  a.gvec = gvec;
+  a.gWr = gWr;
+  a.WrT = reinterpret_cast<float*>(wsb + L.WrT);
+  a.part = reinterpret_cast<float*>(wsb + L.part);
+  cudaError_t e = launch_rad_bwd(a, *plan->rad, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tp_conv_bwd_radial launch");
   return TP_OK;
 }
 

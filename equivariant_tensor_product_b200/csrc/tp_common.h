@@ -96,6 +96,42 @@ cudaError_t launch_gen_dbwd(const LaunchArgs& a, const GenTable& T, bool recv, b
 cudaError_t launch_gen_uvw_fwd(const LaunchArgs& a, const GenTable& T, cudaStream_t s);
 cudaError_t launch_gen_uvw_bwd(const LaunchArgs& a, const GenTable& T, cudaStream_t s);
 
+// Convolution with the radial projection fused in (radial.cu): the uvu weights are formed on
+// chip as w[e, c] = sum_k h[e, k] W_r[k, c] from the radial network's last hidden layer h[E, H]
+// and its output layer W_r[H, nw]; the table is the plan's path table (built for every uvu plan).
+struct RadArgs {
+  int N, E, H;               // H: hidden width, a multiple of 4, at most kRadMaxHidden
+  int nw, nwp;               // weights per edge; row pitch of the shared-memory weight tiles
+  int in_dim, out_dim;
+  int check, splits;         // index checks; edge chunks of the gW_r partials
+  int spec;                  // compiled whole path list of the plan: 2 = all paths of lmax 2, 3 = of lmax 3, 0 = none
+  int mul;                   // its (uniform) multiplicity
+  const int32_t* rowptr;
+  const int32_t* src;
+  const int32_t* colptr;
+  const int32_t* perm;
+  const float* x;
+  const float* vec;
+  const float* h;            // [E, H]
+  const float* Wr;           // [H, nw]
+  const float* gy;
+  float* y;
+  float* gx;
+  float* gh;                 // [E, H]
+  float* gvec;
+  float* gWr;                // [H, nw]
+  float* WrT;                // workspace: W_r transposed, [nw, H]
+  float* part;               // workspace: gW_r partials, [splits, H, nw]
+  int* err;
+};
+constexpr int kRadMaxHidden = 64;
+// Edges per shared-memory chunk (4, 8, 16 or 32) and the bytes of dynamic shared memory of
+// the forward (bwd = false) or sender pass (bwd = true); 0 edges when even 4 do not fit.
+int rad_chunk(const RadArgs& a, bool bwd, size_t* smem_bytes);
+int rad_splits(const GenTable& T, int64_t E);
+cudaError_t launch_rad_fwd(const RadArgs& a, const GenTable& T, cudaStream_t s);
+cudaError_t launch_rad_bwd(const RadArgs& a, const GenTable& T, cudaStream_t s);
+
 // Number of kernels the library has launched in this process (diagnostics).
 void count_launches(int n);
 

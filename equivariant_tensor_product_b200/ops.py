@@ -16,7 +16,8 @@ from . import _lib
 from ._lib import TP_MODE_UVU, TP_MODE_UVW, TP_OP_BWD, TP_OP_DBWD, TP_OP_FWD, check, load
 
 __all__ = ["Plan", "tp_plan_create", "tp_plan_query", "tp_workspace_size", "tp_csr_transpose_workspace_size", "tp_csr_transpose",
-           "tp_conv_fwd", "tp_conv_bwd", "tp_conv_dbwd", "tp_get_device_error", "tp_version"]
+           "tp_conv_fwd", "tp_conv_bwd", "tp_conv_dbwd", "tp_radial_workspace_size", "tp_conv_fwd_radial",
+           "tp_conv_bwd_radial", "tp_get_device_error", "tp_version"]
 
 
 class Plan:
@@ -155,6 +156,68 @@ def tp_conv_bwd(plan: Plan, rowptr, src, x, vec, w, gy, W=None, colptr=None, per
                             _stream(stream))
     check(st, "tp_conv_bwd")
     return gx, gw, gvec, gW
+
+
+def tp_radial_workspace_size(plan: Plan, N: int, E: int, H: int, op: int) -> int:
+    out = C.c_size_t()
+    check(load().tp_radial_workspace_size(plan.handle, int(N), int(E), int(H), int(op), C.byref(out)),
+          "tp_radial_workspace_size")
+    return out.value
+
+
+def _radial_workspace(plan, N, E, H, op, ws, device):
+    need = tp_radial_workspace_size(plan, N, E, H, op)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    elif ws.numel() < need:
+        raise ValueError(f"workspace needs {need} bytes, got {ws.numel()}")
+    return ws
+
+
+def tp_conv_fwd_radial(plan: Plan, rowptr, src, x, vec, h, Wr, y=None, ws=None, stream=None):
+    """uvu forward with the weights formed in the kernels as h[E, H] @ Wr[H, nw]."""
+    N = rowptr.numel() - 1
+    E = src.numel()
+    H = Wr.shape[0]
+    if y is None:
+        y = torch.empty(N, plan.out_dim, dtype=torch.float32, device=x.device)
+    ws = _radial_workspace(plan, N, E, H, TP_OP_FWD, ws, x.device)
+    st = load().tp_conv_fwd_radial(plan.handle, N, E, H, _ptr(rowptr, torch.int32, "rowptr"),
+                                   _ptr(src, torch.int32, "src"), _ptr(x, torch.float32, "x"),
+                                   _ptr(vec, torch.float32, "vec"), _ptr(h, torch.float32, "h"),
+                                   _ptr(Wr, torch.float32, "Wr"), _ptr(y, torch.float32, "y"), _ptr(ws), ws.numel(),
+                                   _stream(stream))
+    check(st, "tp_conv_fwd_radial")
+    return y
+
+
+def tp_conv_bwd_radial(plan: Plan, rowptr, src, x, vec, h, Wr, gy, colptr=None, perm=None, need_gx=True,
+                       need_gh=True, need_gWr=True, need_gvec=False, gx=None, gh=None, gWr=None, gvec=None,
+                       ws=None, stream=None):
+    """VJP of tp_conv_fwd_radial: (gx, gh, gWr, gvec), each None when not requested."""
+    N = rowptr.numel() - 1
+    E = src.numel()
+    H = Wr.shape[0]
+    dev = x.device
+    if need_gx and gx is None:
+        gx = torch.empty(N, plan.in_dim, dtype=torch.float32, device=dev)
+    if need_gh and gh is None:
+        gh = torch.empty(E, H, dtype=torch.float32, device=dev)
+    if need_gWr and gWr is None:
+        gWr = torch.empty(H, plan.n_edge_weights, dtype=torch.float32, device=dev)
+    if need_gvec and gvec is None:
+        gvec = torch.empty(E, 3, dtype=torch.float32, device=dev)
+    ws = _radial_workspace(plan, N, E, H, TP_OP_BWD, ws, dev)
+    st = load().tp_conv_bwd_radial(plan.handle, N, E, H, _ptr(rowptr, torch.int32, "rowptr"),
+                                   _ptr(src, torch.int32, "src"), _ptr(colptr, torch.int32, "colptr"),
+                                   _ptr(perm, torch.int32, "perm"), _ptr(x, torch.float32, "x"),
+                                   _ptr(vec, torch.float32, "vec"), _ptr(h, torch.float32, "h"),
+                                   _ptr(Wr, torch.float32, "Wr"), _ptr(gy, torch.float32, "gy"),
+                                   _ptr(gx, torch.float32, "gx"), _ptr(gh, torch.float32, "gh"),
+                                   _ptr(gWr, torch.float32, "gWr"), _ptr(gvec, torch.float32, "gvec"), _ptr(ws),
+                                   ws.numel(), _stream(stream))
+    check(st, "tp_conv_bwd_radial")
+    return gx, gh, gWr, gvec
 
 
 def tp_conv_dbwd(plan: Plan, rowptr, src, x, vec, w, gy, ggx=None, ggw=None, ggvec=None, W=None, colptr=None,

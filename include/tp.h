@@ -181,6 +181,37 @@ tp_status_t tp_conv_dbwd(tp_plan_t plan, int64_t N, int64_t E, const int32_t* ro
                          float* g_gy, float* g_x, float* g_w, float* g_vec, void* ws,
                          size_t ws_bytes, tp_stream_t stream);
 
+/* The uvu convolution with the radial projection fused in ("Sobek: Streaming Equivariant
+ * Tensor Product Convolutions", abstract: the radial projection reordered so that
+ * edge-specific weights are never materialised).  Instead of w[E, nw] the caller passes the
+ * radial network's last hidden layer and its bias-free output layer,
+ *   h   [E, H]   fp32, row e belongs to edge e (receiver-sorted order, like vec); 16-byte aligned
+ *   Wr  [H, nw]  fp32, nw = n_edge_weights of the plan, columns in the w layout above
+ * and the library forms w[e, c] = sum_k h[e, k] Wr[k, c] in on-chip memory, chunk by chunk,
+ * and uses it there (fp32, k ascending): y equals tp_conv_fwd with that w, and no edge x nw
+ * tensor exists at any point.  H is a multiple of 4 in [4, 64]; any uvu plan (the path table
+ * runs the coupling); uvw plans give TP_ERR_UNSUPPORTED, as do plans whose weight rows do not
+ * fit four edges' on-chip tiles (nw above about 6,000).  Errors and ownership as tp_conv_fwd.
+ *
+ * tp_radial_workspace_size: bytes for op TP_OP_FWD (0, or 256 with TP_FLAG_CHECK_INDICES) or
+ * TP_OP_BWD (the transpose region of tp_workspace_size, Wr transposed and per-split partials
+ * of gWr: H x nw floats per split, at most 256 splits; nothing edge-sized).
+ *
+ * tp_conv_bwd_radial: the VJP against gy[N, out_dim] with respect to x, vec, h and Wr:
+ * gx[N, in_dim], gh[E, H], gWr[H, nw], gvec[E, 3]; each NULL output is skipped; colptr/perm
+ * as in tp_conv_bwd (NULL: built in the workspace).  gW_r is a deterministic sum of fixed
+ * edge-range partials. */
+tp_status_t tp_radial_workspace_size(tp_plan_t plan, int64_t N, int64_t E, int32_t H, int32_t op,
+                                     size_t* bytes);
+tp_status_t tp_conv_fwd_radial(tp_plan_t plan, int64_t N, int64_t E, int32_t H, const int32_t* rowptr,
+                               const int32_t* src, const float* x, const float* vec, const float* h,
+                               const float* Wr, float* y, void* ws, size_t ws_bytes, tp_stream_t stream);
+tp_status_t tp_conv_bwd_radial(tp_plan_t plan, int64_t N, int64_t E, int32_t H, const int32_t* rowptr,
+                               const int32_t* src, const int32_t* colptr, const int32_t* perm,
+                               const float* x, const float* vec, const float* h, const float* Wr,
+                               const float* gy, float* gx, float* gh, float* gWr, float* gvec,
+                               void* ws, size_t ws_bytes, tp_stream_t stream);
+
 /* Row movement of receiver-range sharding over several GPUs (one process per GPU): a rank
  * owning a contiguous range of receivers gathers the x rows its peers need before the halo
  * exchange, and adds the gradient partials its peers send back for the senders it owns

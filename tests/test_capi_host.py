@@ -262,3 +262,43 @@ def test_gaunt_plan_contract(tp):
         with pytest.raises(tp.TPError) as e:
             tp.Gaunt(*args)
         assert e.value.status == status, args
+
+
+def test_radial_contract_on_the_host(lib, tp):
+    """The fused radial projection: hidden widths, plan modes and arguments are checked before
+    the device; the backward workspace is the transpose region plus W_r-sized regions (W_r
+    transposed and at most 256 gW_r partials), nothing edge x feature sized."""
+    spec = synth.CONFIGS["c2"]
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths)
+    N, E, H, nw = 1536, 46080, 64, plan.n_edge_weights
+    assert tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_FWD) == 0
+    b = tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_BWD)
+    base = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD)
+    extra = b - base
+    assert 4 * H * nw * 2 <= extra <= 4 * H * nw * 257 + 512
+    assert tp.tp_radial_workspace_size(plan, 10 * N, 10 * E, H, tp.TP_OP_BWD) - tp.tp_workspace_size(
+        plan, 10 * N, 10 * E, tp.TP_OP_BWD) <= 4 * H * nw * 257 + 512
+    for bad_h in (0, 3, 68):
+        with pytest.raises(tp.TPError):
+            tp.tp_radial_workspace_size(plan, N, E, bad_h, tp.TP_OP_FWD)
+    with pytest.raises(tp.TPError):
+        tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_DBWD)
+    c4 = synth.CONFIGS["c4"]
+    uvw = tp.Plan(c4.irreps_in, c4.irreps_sh, c4.irreps_out, c4.paths, "uvw")
+    with pytest.raises(tp.TPError):
+        tp.tp_radial_workspace_size(uvw, N, E, H, tp.TP_OP_FWD)
+    h = plan.handle
+    fake, odd, off8 = C.c_void_p(0x10000), C.c_void_p(0x10002), C.c_void_p(0x10008)
+    # hidden width not a multiple of 4: unsupported
+    assert lib.tp_conv_fwd_radial(h, 4, 8, 6, fake, fake, fake, fake, fake, fake, fake, None, 0, None) == 2
+    # null output, null edge inputs with E > 0, misaligned pointers, h not on 16 bytes
+    assert lib.tp_conv_fwd_radial(h, 4, 8, 8, fake, fake, fake, fake, fake, fake, None, None, 0, None) == 1
+    assert lib.tp_conv_fwd_radial(h, 4, 8, 8, fake, None, fake, fake, fake, fake, fake, None, 0, None) == 1
+    assert lib.tp_conv_fwd_radial(h, 4, 8, 8, fake, fake, odd, fake, fake, fake, fake, None, 0, None) == 1
+    assert lib.tp_conv_fwd_radial(h, 4, 8, 8, fake, fake, fake, fake, off8, fake, fake, None, 0, None) == 1
+    # N = 0 is a no-op
+    assert lib.tp_conv_fwd_radial(h, 0, 0, 8, None, None, None, None, None, None, None, None, 0, None) == 0
+    # backward: workspace too small
+    st = lib.tp_conv_bwd_radial(h, 4, 8, 8, fake, fake, None, None, fake, fake, fake, fake, fake, fake, fake,
+                                fake, None, fake, 16, None)
+    assert st == 4
