@@ -48,6 +48,11 @@ WORKLOADS = {
     "c2-gaunt": "spherical-grid (Gaunt) convolution on the c2 graph (1,536 atoms, 46,080 edges): 32x0e+32x1o+32x2e "
                 "-> same, edge filter degrees 0..2 with per-degree radial weights, 28-point grid; step = fwd + "
                 "transpose + bwd(gx, gw)",
+    "c2-radial": "c2 with the radial projection fused in (1,536 atoms, 46,080 edges, c2 irreps and paths): the "
+                 "edge weights formed in the kernels from the radial network's last hidden layer h[E, 64] and its "
+                 "output layer W_r[64, 480]; step = fwd + transpose + bwd(gx, gh, gW_r)",
+    "c3-radial": "c3 with the radial projection fused in (4,096 atoms, ~163k edges, c3 irreps and paths): h[E, 64], "
+                 "W_r[64, 2176]; step = fwd + transpose + bwd(gx, gh, gW_r)",
     "c4-layer": "interaction layer on the c4 graph (100,000 atoms, ~3.0M edges): linear 128x(0e,1o,2e) -> same, uvw "
                 "convolution (c4 paths, 128x128 mixing), linear with coefficient 1/average degree -> "
                 "128x0e+256x0e+128x1o+128x2e, gate -> 128x(0e,1o,2e); step = that forward + transpose + the backward "
@@ -328,6 +333,8 @@ def run_reference(args, rank):
         return run_reference_layer(args, cores)
     if args.workload == "c2-gaunt":
         return run_reference_gaunt(args, cores)
+    if args.workload.endswith("-radial"):
+        return run_reference_radial(args, cores)
     d = synth.make_inputs(args.workload)
     oracle_sample(d, 4, seed=0)                      # CG tables cached outside the timing
     ef, tf, eb, tb = oracle_sample(d, 16, seed=1)
@@ -1385,6 +1392,246 @@ def gaunt_counts(N, E, mul, ng, d_in, d_out, lmax_sh, need_gvec=False):
     return fb, bb, ff, bf
 
 
+def radial_counts(spec, N, E, H):
+    """Algorithmic bytes and CUDA-core flops of the fused-radial forward and backward.
+    Forward: per edge src + vec + the hidden row (4 H), node rows x and y, rowptr, W_r once;
+    flops = the uvu forward's (fwd_flops) + the projection 2 H nw per edge.  Backward (gx, gh,
+    gW_r): per edge perm + vec + h read + gh write (8 H), x read, gy read, gx write, colptr +
+    rowptr, W_r read and gW_r write; flops = the uvu backward's (bwd_flops, no gvec) + three
+    H x nw products per edge (the projection, gh = gw W_r^T, gW_r += h^T gw)."""
+    import synth
+    nw = sum(int(spec.irreps_in.split("+")[a].split("x")[0]) for a, b, o in spec.paths)
+    in_dim, out_dim = synth.irreps_dim(spec.irreps_in), synth.irreps_dim(spec.irreps_out)
+    fb = E * (4 + 12 + 4 * H) + 4 * N * (in_dim + out_dim) + 4 * (N + 1) + 4 * H * nw
+    bb = E * (4 + 12 + 8 * H) + 4 * N * (2 * in_dim + out_dim) + 8 * (N + 1) + 8 * H * nw
+    ff = fwd_flops(spec, E) + 2 * E * H * nw
+    bf = bwd_flops(spec, E, False) + 3 * 2 * E * H * nw
+    return fb, bb, ff, bf, nw
+
+
+def run_radial(args, rank, world, local):
+    """The convolution with the radial projection fused in (tp_conv_fwd_radial / bwd_radial):
+    forward, the transpose on a side stream, backward (gx, gh, gW_r), timed as the other
+    workloads are (rotating inputs > 2 x L2, CUDA events, end to end with host copies)."""
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from equivariant_tensor_product_b200 import build as tpbuild
+    tpbuild.build()
+    import equivariant_tensor_product_b200 as tp
+    import synth
+    base = args.workload.split("-")[0]
+    spec = synth.CONFIGS[base]
+    lib = tp.load()
+    d = synth.make_inputs(base, args.n_atoms, seed=spec.seed + 7919 * rank)
+    h0, Wr0 = synth.radial_hidden(d)
+    N, E, H = len(d["rowptr"]) - 1, len(d["src"]), h0.shape[1]
+    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths)
+    rng = np.random.default_rng(spec.seed + 31 + 7919 * rank)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copy_bytes = 4 * (N * (plan.in_dim + plan.out_dim) + E * (H + 4)) + 4 * (N + 1)
+    R = max(2, math.ceil(2.5 * l2 / copy_bytes))
+    copies = []
+    for r in range(R):
+        cp = {"rowptr": d["rowptr"], "src": d["src"], "vec": d["vec"],
+              "x": d["x"] if r == 0 else rng.standard_normal((N, plan.in_dim), dtype=np.float32),
+              "h": h0 if r == 0 else np.ascontiguousarray(h0[rng.permutation(E)]),
+              "gy": rng.standard_normal((N, plan.out_dim), dtype=np.float32)}
+        copies.append({k: torch.as_tensor(np.ascontiguousarray(v)).to(dev) for k, v in cp.items()})
+    Wr = torch.as_tensor(Wr0).to(dev)
+    y = torch.empty(N, plan.out_dim, device=dev)
+    gx = torch.empty(N, plan.in_dim, device=dev)
+    gh = torch.empty(E, H, device=dev)
+    gWr = torch.empty_like(Wr)
+    wsf = torch.empty(max(256, tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_FWD)), dtype=torch.uint8,
+                      device=dev)
+    wsb = torch.empty(tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_BWD), dtype=torch.uint8, device=dev)
+    wst_bytes = max(256, tp.tp_csr_transpose_workspace_size(N, E))
+    wst = torch.empty(wst_bytes, dtype=torch.uint8, device=dev)
+    colptrs = [torch.empty(N + 1, dtype=torch.int32, device=dev) for _ in range(R)]
+    perms = [torch.empty(E, dtype=torch.int32, device=dev) for _ in range(R)]
+    stream, side = torch.cuda.Stream(dev), torch.cuda.Stream(dev, priority=-1)
+    sh, sh_side = stream.cuda_stream, side.cuda_stream
+    P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None
+    ff_, tf_, bf_ = lib.tp_conv_fwd_radial, lib.tp_csr_transpose, lib.tp_conv_bwd_radial
+    args_r = []
+    for r, cp in enumerate(copies):
+        args_r.append(((plan.handle, N, E, H, P(cp["rowptr"]), P(cp["src"]), P(cp["x"]), P(cp["vec"]), P(cp["h"]),
+                        P(Wr), P(y), P(wsf), wsf.numel(), sh),
+                       (N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(wst), wst_bytes, sh_side),
+                       (plan.handle, N, E, H, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(cp["x"]),
+                        P(cp["vec"]), P(cp["h"]), P(Wr), P(cp["gy"]), P(gx), P(gh), P(gWr), None, P(wsb),
+                        wsb.numel(), sh)))
+    tr_done = [torch.cuda.Event() for _ in range(R)]
+    bwd_done = [torch.cuda.Event() for _ in range(R)]
+
+    def step(k, ev=None):
+        r = k % R
+        a_f, a_t, a_b = args_r[r]
+        side.wait_event(bwd_done[r])
+        st = tf_(*a_t)
+        tr_done[r].record(side)
+        if ev is not None:
+            ev[0].record(stream)
+        st |= ff_(*a_f)
+        if ev is not None:
+            ev[1].record(stream)
+        stream.wait_event(tr_done[r])
+        if ev is not None:
+            ev[2].record(stream)
+        st |= bf_(*a_b)
+        if ev is not None:
+            ev[3].record(stream)
+        bwd_done[r].record(stream)
+        if st:
+            raise RuntimeError(lib.tp_last_error_message().decode())
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    n0 = lib.tp_launch_count()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            step(k, evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    launches = lib.tp_launch_count() - n0
+    elapsed_max = max_over_ranks(start.elapsed_time(stop) / 1e3, world, dev)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    # end to end: inputs up from pinned memory, outputs down, every step (sequential copies)
+    host = {k: torch.as_tensor(np.ascontiguousarray(v.cpu().numpy())).pin_memory() for k, v in copies[0].items()}
+    hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (y, gx, gh, gWr)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for k in range(args.e2e_steps):
+            for key in host:
+                copies[0][key].copy_(host[key], non_blocking=True)
+            side.wait_stream(stream)
+            step(0)
+            stream.wait_stream(side)
+            for ho, t in zip(hout, (y, gx, gh, gWr)):
+                ho.copy_(t, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+    if rank == 0:
+        hbm, _, peak_note = measured_peaks()
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        fp32_peak = 2 * 128 * sms * clk.max_mhz_or(1965.0) * 1e6 / 1e12
+        fb, bb, fl_f, fl_b, nw = radial_counts(spec, N, E, H)
+        passes = {"fwd": pass_roofline(fwd_ms, fb, fl_f, hbm, fp32_peak),
+                  "bwd": pass_roofline(bwd_ms, bb, fl_b, hbm, fp32_peak)}
+        dom = max(passes, key=lambda k: passes[k]["ms"])
+        dp = passes[dom]
+        kname = {"fwd": "k_rad_fwd", "bwd": "k_rad_send"}[dom]
+        if dp["bound"] == "hbm":
+            roof = {"bound": "hbm", "kernel": kname, "achieved": dp["achieved_GBps"], "peak": hbm, "unit": "GB/s",
+                    "frac": dp["achieved_GBps"] / hbm, "peak_note": peak_note}
+        else:
+            roof = {"bound": "alu", "kernel": kname, "achieved": dp["achieved_fp32_TFLOPs"], "peak": fp32_peak,
+                    "unit": "TFLOP/s", "frac": dp["achieved_fp32_TFLOPs"] / fp32_peak,
+                    "peak_note": "fp32 FMA peak; flops by bench.radial_counts"}
+        roof.update({"traffic": traffic_from_profile(kname, args.workload), "passes": passes,
+                     "kernel_ms": {"fwd": fwd_ms, "bwd": bwd_ms}})
+        cpu = None
+        if not args.no_cpu_baseline:
+            from oracle import OraclePlan
+            from oracle.conv import set_threads
+            from oracle.radial import backward_radial, forward_radial
+            cores = set_threads()
+            op = OraclePlan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvu")
+            n_rows = 64 if base == "c2" else 16
+            rows = np.sort(np.random.default_rng(3).choice(N, size=min(N, n_rows), replace=False))
+            rp = np.asarray(d["rowptr"], dtype=np.int64)
+            eids = np.concatenate([np.arange(rp[i], rp[i + 1]) for i in rows])
+            rpf = np.concatenate([[0], np.cumsum(rp[rows + 1] - rp[rows])])
+            gys = copies[0]["gy"].cpu().numpy()
+            t0 = time.perf_counter()
+            forward_radial(op, rpf, d["src"][eids], d["x"], d["vec"][eids], h0[eids], Wr0)
+            backward_radial(op, rpf, d["src"][eids], d["x"], d["vec"][eids], h0[eids], Wr0, gys[rows])
+            t1 = time.perf_counter()
+            cpu = {"value": len(eids) / (t1 - t0), "unit": "edges/s", "cores": cores, "kind": "oracle",
+                   "sample": f"fwd + bwd on the {len(eids)} edges into {len(rows)} random receivers, float64, "
+                             f"{t1 - t0:.1f} s"}
+        line = {"metric": METRIC, "value": replica_throughput(E, args.steps, world, elapsed_max), "unit": "edges/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * elapsed_max / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOADS[args.workload], "name": args.workload, "N": N, "E": E, "H": H,
+                           "n_edge_weights": nw, "launch": "eager",
+                           "l2": f"{R} rotating input copies of {copy_bytes / 1e6:.1f} MB (> 2x L2 of {l2 / 1e6:.0f} MB)",
+                           "parallelism": "replicas" if world > 1 else "single"},
+                "roofline": roof, "cpu_baseline": cpu,
+                "e2e": {"value": E * args.e2e_steps / e2e_s, "unit": "edges/s",
+                        "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host.values()),
+                        "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout),
+                        "steps": args.e2e_steps},
+                "memory": {"workspace_bytes": wsb.numel(), "edge_weight_bytes_not_materialised": 4 * E * nw},
+                "gpu_launches": int(launches), "clocks": clk.summary(), "library": tp.tp_version()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference_radial(args, cores):
+    """The float64 oracle of the fused-radial convolution on sampled receivers of the graph."""
+    import synth
+    from oracle import OraclePlan
+    from oracle.radial import backward_radial, forward_radial
+    base = args.workload.split("-")[0]
+    spec = synth.CONFIGS[base]
+    d = synth.make_inputs(base)
+    h, Wr = synth.radial_hidden(d)
+    N = len(d["rowptr"]) - 1
+    op = OraclePlan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths, "uvu")
+    rp = np.asarray(d["rowptr"], dtype=np.int64)
+
+    def sample(n_rows, seed):
+        rows = np.sort(np.random.default_rng(seed).choice(N, size=n_rows, replace=False))
+        eids = np.concatenate([np.arange(rp[i], rp[i + 1]) for i in rows])
+        rpf = np.concatenate([[0], np.cumsum(rp[rows + 1] - rp[rows])])
+        t0 = time.perf_counter()
+        forward_radial(op, rpf, d["src"][eids], d["x"], d["vec"][eids], h[eids], Wr)
+        backward_radial(op, rpf, d["src"][eids], d["x"], d["vec"][eids], h[eids], Wr, d["gy"][rows])
+        return len(eids), time.perf_counter() - t0
+
+    sample(4, 0)
+    e, t = sample(8, 1)
+    rows = int(max(2, min(512, 8 * 60.0 / max(1, args.steps + args.warmup) / max(t, 1e-3))))
+    for k in range(args.warmup):
+        sample(rows, 100 + k)
+    tot_e = tot_t = 0.0
+    for k in range(args.steps):
+        e, t = sample(rows, 1000 + k)
+        tot_e += e
+        tot_t += t
+    value = tot_e / tot_t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "edges/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload], "name": args.workload, "N": N, "E": len(d["src"]),
+                       "parallelism": "single"},
+            "cpu_baseline": {"value": value, "unit": "edges/s", "cores": cores, "kind": "oracle",
+                             "sample": f"fwd + bwd on the edges into {rows} random receivers per step, float64"},
+            "e2e": {"value": value, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_gaunt(args, rank, world, local):
     """The spherical-grid (Gaunt) convolution on the c2 graph: forward, the transpose on a
     side stream, backward (gx, gw), through include/tp_gaunt.h, timed as the convolution
@@ -1565,6 +1812,8 @@ def main():
         return run_latency(args, rank, world, local)
     if args.workload == "c2-gaunt":
         return run_gaunt(args, rank, world, local)
+    if args.workload.endswith("-radial"):
+        return run_radial(args, rank, world, local)
     if args.workload.endswith("-layer"):
         return run_layer(args, rank, world, local)
     return run_ours(args, rank, world, local)

@@ -43,3 +43,18 @@ def test_layer_node_bytes_count_each_array_once():
     assert bench.layer_node_bytes(lin, N, False) == 4 * N * (Irreps(ir_in).dim + Irreps(ir_out).dim) + 4 * nw
     # backward: x and gy read, gx written, W read and gW written
     assert bench.layer_node_bytes(lin, N, True) == 4 * N * (2 * Irreps(ir_in).dim + Irreps(ir_out).dim) + 8 * nw
+
+
+@pytest.mark.parametrize("base", ["c2", "c3"])
+def test_radial_counts_match_the_plan(base):
+    """The fused-radial workload counts W_r's width as the plan's weights per edge, and its
+    flops are the plain convolution's plus 2 H nw per edge (forward) and three such products
+    (backward: projection, gh, gW_r); the edge stream is the hidden row, not the weights."""
+    spec = synth.CONFIGS[base]
+    N, E, H = 100, 1000, 64
+    fb, bb, ff, bf, nw = bench.radial_counts(spec, N, E, H)
+    assert nw == synth.n_edge_weights(spec)
+    assert ff == bench.fwd_flops(spec, E) + 2 * E * H * nw
+    assert bf == bench.bwd_flops(spec, E, False) + 6 * E * H * nw
+    in_dim, out_dim = synth.irreps_dim(spec.irreps_in), synth.irreps_dim(spec.irreps_out)
+    assert fb == bench.fwd_bytes(N, E, in_dim, out_dim, nw) - E * 4 * nw + E * 4 * H + 4 * H * nw
