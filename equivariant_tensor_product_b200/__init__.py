@@ -11,7 +11,7 @@ from ._lib import (TP_FLAG_CHECK_INDICES, TP_LINEAR_CUDA_CORES, TP_LINEAR_TENSOR
 from .ops import (Plan, tp_conv_bwd, tp_conv_dbwd, tp_conv_fwd, tp_csr_transpose, tp_csr_transpose_workspace_size,  # noqa: F401
                   tp_conv_bwd_radial, tp_conv_fwd_radial, tp_get_device_error, tp_radial_workspace_size,
                   tp_plan_create, tp_plan_query, tp_version, tp_workspace_size)
-from .autograd import GateFn, LinearFn, TPConv, tp_conv, tp_gate, tp_linear  # noqa: F401
+from .autograd import GateFn, LinearFn, TPConv, TPConvRadial, tp_conv, tp_conv_radial, tp_gate, tp_linear  # noqa: F401
 from .block import (Gate, Linear, tp_gate_bwd, tp_gate_dbwd, tp_gate_fwd, tp_linear_bwd, tp_linear_fwd,  # noqa: F401
                     tp_linear_workspace_size)
 from .gaunt import Gaunt, tp_gaunt_bwd, tp_gaunt_fwd, tp_gaunt_workspace_size  # noqa: F401

@@ -1,14 +1,16 @@
 """torch.autograd wrapper: forward -> tp_conv_fwd, backward -> tp_conv_bwd, and the backward's
 own backward -> tp_conv_dbwd, so force training (a loss on d(energy)/d(positions)) can
 differentiate twice through the convolution (uvu; uvw mode differentiates once, to x, the
-edge vectors, the per-edge scalars and the shared mixing weights W).  Marshalling only (see
-ops.py)."""
+edge vectors, the per-edge scalars and the shared mixing weights W; the radial-projection form
+differentiates once, to x, the edge vectors, the hidden layer h and the output matrix W_r).
+Marshalling only (see ops.py)."""
 from __future__ import annotations
 
 import torch
 
 from ._lib import TP_MODE_UVW
-from .ops import Plan, tp_conv_bwd, tp_conv_dbwd, tp_conv_fwd, tp_csr_transpose
+from .ops import (Plan, tp_conv_bwd, tp_conv_bwd_radial, tp_conv_dbwd, tp_conv_fwd, tp_conv_fwd_radial,
+                  tp_csr_transpose)
 
 
 class Graph:
@@ -171,3 +173,33 @@ class GateFn(torch.autograd.Function):
 def tp_gate(gate: Gate, x):
     """y = gate(x) with first and second derivatives through the CUDA kernels."""
     return GateFn.apply(x, gate)
+
+
+class TPConvRadial(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, vec, h, Wr, plan, graph):
+        x, vec, h, Wr = x.contiguous(), vec.contiguous(), h.contiguous(), Wr.contiguous()
+        y = tp_conv_fwd_radial(plan, graph.rowptr, graph.src, x, vec, h, Wr)
+        ctx.save_for_backward(x, vec, h, Wr)
+        ctx.plan, ctx.graph = plan, graph
+        return y
+
+    @staticmethod
+    @torch.autograd.function.once_differentiable
+    def backward(ctx, gy):
+        x, vec, h, Wr = ctx.saved_tensors
+        n = ctx.needs_input_grad
+        colptr, perm = ctx.graph.transpose()
+        gx, gh, gWr, gvec = tp_conv_bwd_radial(ctx.plan, ctx.graph.rowptr, ctx.graph.src, x, vec, h, Wr,
+                                               gy.contiguous(), colptr=colptr, perm=perm, need_gx=n[0],
+                                               need_gvec=n[1], need_gh=n[2], need_gWr=n[3])
+        return gx, gvec, gh, gWr, None, None
+
+
+def tp_conv_radial(plan: Plan, graph: Graph, x, vec, h, Wr):
+    """y = conv(x, vec, w) with w = h @ Wr formed inside the kernels (uvu plans; h [E, H] the
+    radial network's last hidden layer, Wr [H, n_edge_weights] its output layer); first-order
+    derivatives to x, vec, h and Wr through the CUDA kernels."""
+    if plan.mode == TP_MODE_UVW:
+        raise ValueError("the fused radial projection is implemented for uvu plans")
+    return TPConvRadial.apply(x, vec, h, Wr, plan, graph)

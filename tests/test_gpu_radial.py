@@ -124,3 +124,43 @@ def test_no_edges_and_empty_rows(tp):
     h_np = rng.standard_normal((8, H)).astype(np.float32)
     _check_complete(tp, ir_in, ir_sh, ir_out, paths, rowptr_np, src_np, vec_np, x.cpu().numpy(), h_np,
                     Wr.cpu().numpy(), gy.cpu().numpy(), "empty rows")
+
+
+def test_autograd_first_derivatives(tp):
+    """tp_conv_radial through torch autograd: gradients to x, vec, h and W_r against the oracle."""
+    from equivariant_tensor_product_b200.autograd import Graph, tp_conv_radial
+    d = synth.make_inputs("c2", 128, with_gy=True)
+    h, Wr = synth.radial_hidden(d)
+    s = d["spec"]
+    plan = tp.Plan(s.irreps_in, s.irreps_sh, s.irreps_out, s.paths)
+    op = OraclePlan(s.irreps_in, s.irreps_sh, s.irreps_out, s.paths, "uvu")
+    graph = Graph(dev(d["rowptr"]), dev(d["src"]))
+    leaves = [dev(a).requires_grad_(True) for a in (d["x"], d["vec"], h, Wr)]
+    y = tp_conv_radial(plan, graph, *leaves)
+    (y * dev(d["gy"])).sum().backward()
+    r = backward_radial(op, d["rowptr"], d["src"], d["x"], d["vec"], h, Wr, d["gy"])
+    assert_close(y, forward_radial(op, d["rowptr"], d["src"], d["x"], d["vec"], h, Wr), "autograd y")
+    for t, name in zip(leaves, ("gx", "gvec", "gh", "gWr")):
+        assert_close(t.grad, r[name], f"autograd {name}")
+
+
+def test_index_check_reports_bad_sender(tp):
+    d = synth.make_inputs("c1", with_gy=True)
+    h, Wr = synth.radial_hidden(d)
+    s = d["spec"]
+    plan = tp.Plan(s.irreps_in, s.irreps_sh, s.irreps_out, s.paths, flags=tp.TP_FLAG_CHECK_INDICES)
+    g = {k: dev(v) for k, v in dict(rowptr=d["rowptr"], src=d["src"], vec=d["vec"], x=d["x"], h=h, Wr=Wr,
+                                    gy=d["gy"]).items()}
+    bad = g["src"].clone()
+    bad[5] = 10_000
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    y = tp.tp_conv_fwd_radial(plan, g["rowptr"], bad, g["x"], g["vec"], g["h"], g["Wr"], ws=ws)
+    assert tp.tp_get_device_error(plan, ws) == 2
+    assert torch.isfinite(y).all()
+    tp.tp_conv_fwd_radial(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["h"], g["Wr"], ws=ws)
+    assert tp.tp_get_device_error(plan, ws) == 0
+    N, E, H = len(d["rowptr"]) - 1, len(d["src"]), h.shape[1]
+    wsb = torch.zeros(tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_BWD), dtype=torch.uint8, device="cuda")
+    tp.tp_conv_bwd_radial(plan, g["rowptr"], bad, g["x"], g["vec"], g["h"], g["Wr"], g["gy"], ws=wsb)
+    assert tp.tp_get_device_error(plan, wsb) == 2
+    torch.cuda.synchronize()
