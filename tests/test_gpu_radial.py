@@ -164,3 +164,20 @@ def test_index_check_reports_bad_sender(tp):
     tp.tp_conv_bwd_radial(plan, g["rowptr"], bad, g["x"], g["vec"], g["h"], g["Wr"], g["gy"], ws=wsb)
     assert tp.tp_get_device_error(plan, wsb) == 2
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("lmax,mul", [(2, 64), (2, 128), (3, 32), (3, 48)])
+def test_compiled_lists_at_other_channel_counts(tp, lmax, mul):
+    """All paths of lmax 2 or 3 at other multiplicities: wider weight rows change the chunk size
+    (and with it the kernel: the compiled-list instances or the path-table ones), ragged slices."""
+    ls = range(lmax + 1)
+    ir_in = "+".join(f"{mul}x{l}{'e' if l % 2 == 0 else 'o'}" for l in ls)
+    ir_sh = "+".join(f"1x{l}{'e' if l % 2 == 0 else 'o'}" for l in ls)
+    spec = synth.CONFIGS["c2" if lmax == 2 else "c3"]
+    ir_out = "+".join(f"{mul}x{b.split('x')[1]}" for b in spec.irreps_out.split("+"))
+    paths = synth.L2_PATHS if lmax == 2 else synth.L3_PATHS
+    rowptr, src, vec, rng = random_graph(20 + mul, 40, 12)
+    op = OraclePlan(ir_in, ir_sh, ir_out, paths, "uvu")
+    f = lambda *shape: rng.standard_normal(shape).astype(np.float32)
+    _check_complete(tp, ir_in, ir_sh, ir_out, paths, rowptr, src, vec, f(40, op.irr_in.dim), f(len(src), 64),
+                    (f(64, op.n_weights) / 8).astype(np.float32), f(40, op.irr_out.dim), f"lmax {lmax} mul {mul}")
