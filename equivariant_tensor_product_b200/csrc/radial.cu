@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kRadThreads) k_rad_send(const __grid_constant_
 // warps of a CTA run the same triple's code), load the x and gy slices of a batch before using
 // them, and are summed in warp order at the end.
 // ---------------------------------------------------------------------------------------
-constexpr int kGwrChunk = 32;
+constexpr int kGwrChunk = 64;
 constexpr int kGwrBatch = 4;
 
 __global__ void __launch_bounds__(kGwrThreads) k_rad_gwr(const __grid_constant__ RadArgs a,
