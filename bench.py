@@ -791,6 +791,7 @@ def run_ours(args, rank, world, local):
             for name, st, wu in (("c3", 100, 5), ("c4", 10, 3)):
                 per[name + "-cell"] = config_record(tp, lib, torch, dev, name, st, wu, local, hbm, fp32_peak,
                                                     tc_peak, order="cell")
+            per["c2-radial"] = radial_record(tp, lib, torch, dev, local, "c2", 30, 3, hbm, fp32_peak)
             line["per_config"] = per
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -1409,6 +1410,114 @@ def radial_counts(spec, N, E, H):
     return fb, bb, ff, bf, nw
 
 
+class RadialRun:
+    """Inputs, buffers and one eager step of the fused-radial workload: forward, the transpose
+    on a higher-priority side stream, backward (gx, gh, gW_r), R rotating input copies (together
+    > 2.5 x L2) so that no step starts with its inputs in L2."""
+
+    def __init__(self, tp, lib, torch, dev, base, n_atoms=None, rank=0):
+        import synth
+        spec = synth.CONFIGS[base]
+        d = synth.make_inputs(base, n_atoms, seed=spec.seed + 7919 * rank)
+        h0, Wr0 = synth.radial_hidden(d)
+        N, E, H = len(d["rowptr"]) - 1, len(d["src"]), h0.shape[1]
+        plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths)
+        rng = np.random.default_rng(spec.seed + 31 + 7919 * rank)
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        copy_bytes = 4 * (N * (plan.in_dim + plan.out_dim) + E * (H + 4)) + 4 * (N + 1)
+        R = max(2, math.ceil(2.5 * l2 / copy_bytes))
+        copies = []
+        for r in range(R):
+            cp = {"rowptr": d["rowptr"], "src": d["src"], "vec": d["vec"],
+                  "x": d["x"] if r == 0 else rng.standard_normal((N, plan.in_dim), dtype=np.float32),
+                  "h": h0 if r == 0 else np.ascontiguousarray(h0[rng.permutation(E)]),
+                  "gy": rng.standard_normal((N, plan.out_dim), dtype=np.float32)}
+            copies.append({k: torch.as_tensor(np.ascontiguousarray(v)).to(dev) for k, v in cp.items()})
+        Wr = torch.as_tensor(Wr0).to(dev)
+        self.y = torch.empty(N, plan.out_dim, device=dev)
+        self.gx = torch.empty(N, plan.in_dim, device=dev)
+        self.gh = torch.empty(E, H, device=dev)
+        self.gWr = torch.empty_like(Wr)
+        wsf = torch.empty(max(256, tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_FWD)), dtype=torch.uint8,
+                          device=dev)
+        wsb = torch.empty(tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_BWD), dtype=torch.uint8, device=dev)
+        wst_bytes = max(256, tp.tp_csr_transpose_workspace_size(N, E))
+        wst = torch.empty(wst_bytes, dtype=torch.uint8, device=dev)
+        colptrs = [torch.empty(N + 1, dtype=torch.int32, device=dev) for _ in range(R)]
+        perms = [torch.empty(E, dtype=torch.int32, device=dev) for _ in range(R)]
+        self.stream, self.side = torch.cuda.Stream(dev), torch.cuda.Stream(dev, priority=-1)
+        sh, sh_side = self.stream.cuda_stream, self.side.cuda_stream
+        P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None
+        self.lib = lib
+        self.fns = (lib.tp_conv_fwd_radial, lib.tp_csr_transpose, lib.tp_conv_bwd_radial)
+        self.args_r = []
+        for r, cp in enumerate(copies):
+            self.args_r.append(((plan.handle, N, E, H, P(cp["rowptr"]), P(cp["src"]), P(cp["x"]), P(cp["vec"]),
+                                 P(cp["h"]), P(Wr), P(self.y), P(wsf), wsf.numel(), sh),
+                                (N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(wst), wst_bytes,
+                                 sh_side),
+                                (plan.handle, N, E, H, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]),
+                                 P(cp["x"]), P(cp["vec"]), P(cp["h"]), P(Wr), P(cp["gy"]), P(self.gx), P(self.gh),
+                                 P(self.gWr), None, P(wsb), wsb.numel(), sh)))
+        self.tr_done = [torch.cuda.Event() for _ in range(R)]
+        self.bwd_done = [torch.cuda.Event() for _ in range(R)]
+        self.spec, self.d, self.h0, self.Wr0, self.plan = spec, d, h0, Wr0, plan
+        self.N, self.E, self.H, self.R, self.copies = N, E, H, R, copies
+        self.copy_bytes, self.l2, self.ws_bytes = copy_bytes, l2, wsb.numel()
+
+    def step(self, k, ev=None):
+        r = k % self.R
+        a_f, a_t, a_b = self.args_r[r]
+        ff_, tf_, bf_ = self.fns
+        self.side.wait_event(self.bwd_done[r])
+        st = tf_(*a_t)
+        self.tr_done[r].record(self.side)
+        if ev is not None:
+            ev[0].record(self.stream)
+        st |= ff_(*a_f)
+        if ev is not None:
+            ev[1].record(self.stream)
+        self.stream.wait_event(self.tr_done[r])
+        if ev is not None:
+            ev[2].record(self.stream)
+        st |= bf_(*a_b)
+        if ev is not None:
+            ev[3].record(self.stream)
+        self.bwd_done[r].record(self.stream)
+        if st:
+            raise RuntimeError(self.lib.tp_last_error_message().decode())
+
+
+def radial_record(tp, lib, torch, dev, local, base, steps, warmup, hbm, fp32_peak):
+    """Compact measured record of the fused-radial workload in the same run as the headline."""
+    rr = RadialRun(tp, lib, torch, dev, base)
+    for k in range(warmup):
+        rr.step(k)
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        start.record(rr.stream)
+        for k in range(steps):
+            rr.step(k, evs[k])
+        stop.record(rr.stream)
+        torch.cuda.synchronize(dev)
+    ms = start.elapsed_time(stop) / steps
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    fb, bb, fl_f, fl_b, nw = radial_counts(rr.spec, rr.N, rr.E, rr.H)
+    rec = {"workload": WORKLOADS[base + "-radial"], "N": rr.N, "E": rr.E, "H": rr.H, "steps": steps,
+           "ms_per_step": ms, "edges_per_s": rr.E / (ms * 1e-3), "launch": "eager",
+           "kernel_ms": {"fwd": fwd_ms, "bwd": bwd_ms},
+           "passes": {"fwd": pass_roofline(fwd_ms, fb, fl_f, hbm, fp32_peak),
+                      "bwd": pass_roofline(bwd_ms, bb, fl_b, hbm, fp32_peak)},
+           "edge_weight_bytes_not_materialised": 4 * rr.E * nw, "clocks": clk.summary()}
+    del rr
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_radial(args, rank, world, local):
     """The convolution with the radial projection fused in (tp_conv_fwd_radial / bwd_radial):
     forward, the transpose on a side stream, backward (gx, gh, gW_r), timed as the other
@@ -1423,72 +1532,15 @@ def run_radial(args, rank, world, local):
     from equivariant_tensor_product_b200 import build as tpbuild
     tpbuild.build()
     import equivariant_tensor_product_b200 as tp
-    import synth
     base = args.workload.split("-")[0]
-    spec = synth.CONFIGS[base]
     lib = tp.load()
-    d = synth.make_inputs(base, args.n_atoms, seed=spec.seed + 7919 * rank)
-    h0, Wr0 = synth.radial_hidden(d)
-    N, E, H = len(d["rowptr"]) - 1, len(d["src"]), h0.shape[1]
-    plan = tp.Plan(spec.irreps_in, spec.irreps_sh, spec.irreps_out, spec.paths)
-    rng = np.random.default_rng(spec.seed + 31 + 7919 * rank)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    copy_bytes = 4 * (N * (plan.in_dim + plan.out_dim) + E * (H + 4)) + 4 * (N + 1)
-    R = max(2, math.ceil(2.5 * l2 / copy_bytes))
-    copies = []
-    for r in range(R):
-        cp = {"rowptr": d["rowptr"], "src": d["src"], "vec": d["vec"],
-              "x": d["x"] if r == 0 else rng.standard_normal((N, plan.in_dim), dtype=np.float32),
-              "h": h0 if r == 0 else np.ascontiguousarray(h0[rng.permutation(E)]),
-              "gy": rng.standard_normal((N, plan.out_dim), dtype=np.float32)}
-        copies.append({k: torch.as_tensor(np.ascontiguousarray(v)).to(dev) for k, v in cp.items()})
-    Wr = torch.as_tensor(Wr0).to(dev)
-    y = torch.empty(N, plan.out_dim, device=dev)
-    gx = torch.empty(N, plan.in_dim, device=dev)
-    gh = torch.empty(E, H, device=dev)
-    gWr = torch.empty_like(Wr)
-    wsf = torch.empty(max(256, tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_FWD)), dtype=torch.uint8,
-                      device=dev)
-    wsb = torch.empty(tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_BWD), dtype=torch.uint8, device=dev)
-    wst_bytes = max(256, tp.tp_csr_transpose_workspace_size(N, E))
-    wst = torch.empty(wst_bytes, dtype=torch.uint8, device=dev)
-    colptrs = [torch.empty(N + 1, dtype=torch.int32, device=dev) for _ in range(R)]
-    perms = [torch.empty(E, dtype=torch.int32, device=dev) for _ in range(R)]
-    stream, side = torch.cuda.Stream(dev), torch.cuda.Stream(dev, priority=-1)
-    sh, sh_side = stream.cuda_stream, side.cuda_stream
-    P = lambda t: C.c_void_p(t.data_ptr()) if t is not None else None
-    ff_, tf_, bf_ = lib.tp_conv_fwd_radial, lib.tp_csr_transpose, lib.tp_conv_bwd_radial
-    args_r = []
-    for r, cp in enumerate(copies):
-        args_r.append(((plan.handle, N, E, H, P(cp["rowptr"]), P(cp["src"]), P(cp["x"]), P(cp["vec"]), P(cp["h"]),
-                        P(Wr), P(y), P(wsf), wsf.numel(), sh),
-                       (N, E, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(wst), wst_bytes, sh_side),
-                       (plan.handle, N, E, H, P(cp["rowptr"]), P(cp["src"]), P(colptrs[r]), P(perms[r]), P(cp["x"]),
-                        P(cp["vec"]), P(cp["h"]), P(Wr), P(cp["gy"]), P(gx), P(gh), P(gWr), None, P(wsb),
-                        wsb.numel(), sh)))
-    tr_done = [torch.cuda.Event() for _ in range(R)]
-    bwd_done = [torch.cuda.Event() for _ in range(R)]
-
-    def step(k, ev=None):
-        r = k % R
-        a_f, a_t, a_b = args_r[r]
-        side.wait_event(bwd_done[r])
-        st = tf_(*a_t)
-        tr_done[r].record(side)
-        if ev is not None:
-            ev[0].record(stream)
-        st |= ff_(*a_f)
-        if ev is not None:
-            ev[1].record(stream)
-        stream.wait_event(tr_done[r])
-        if ev is not None:
-            ev[2].record(stream)
-        st |= bf_(*a_b)
-        if ev is not None:
-            ev[3].record(stream)
-        bwd_done[r].record(stream)
-        if st:
-            raise RuntimeError(lib.tp_last_error_message().decode())
+    rr = RadialRun(tp, lib, torch, dev, base, args.n_atoms, rank)
+    spec, d, h0, Wr0, plan = rr.spec, rr.d, rr.h0, rr.Wr0, rr.plan
+    N, E, H, R, copies = rr.N, rr.E, rr.H, rr.R, rr.copies
+    copy_bytes, l2 = rr.copy_bytes, rr.l2
+    y, gx, gh, gWr = rr.y, rr.gx, rr.gh, rr.gWr
+    stream, side = rr.stream, rr.side
+    step = rr.step
 
     for k in range(args.warmup):
         step(k)
@@ -1578,7 +1630,7 @@ def run_radial(args, rank, world, local):
                         "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host.values()),
                         "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout),
                         "steps": args.e2e_steps},
-                "memory": {"workspace_bytes": wsb.numel(), "edge_weight_bytes_not_materialised": 4 * E * nw},
+                "memory": {"workspace_bytes": rr.ws_bytes, "edge_weight_bytes_not_materialised": 4 * E * nw},
                 "gpu_launches": int(launches), "clocks": clk.summary(), "library": tp.tp_version()}
         print(json.dumps(line), flush=True)
     if world > 1:
