@@ -283,8 +283,10 @@ __global__ void __launch_bounds__(kRadThreads) k_rad_send(const __grid_constant_
 constexpr int kGwrChunk = 64;
 constexpr int kGwrBatch = 4;
 
+template <int HC>
 __global__ void __launch_bounds__(kGwrThreads) k_rad_gwr(const __grid_constant__ RadArgs a,
                                                          const __grid_constant__ GenTable T) {
+  const int H = HC ? HC : a.H;          // hidden width (a compile-time 64 in the common case)
   __shared__ __align__(16) float hs[kGwrChunk * kRadMaxHidden];
   __shared__ float Ys[kGwrChunk * 16];
   __shared__ int js[kGwrChunk], is[kGwrChunk];
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(kGwrThreads) k_rad_gwr(const __grid_constant__
   for (int64_t c0 = lo; c0 < hi; c0 += kGwrChunk) {
     const int ne = (int)(hi - c0 < kGwrChunk ? hi - c0 : kGwrChunk);
     __syncthreads();
-    for (int t = threadIdx.x; t < ne * a.H; t += blockDim.x) hs[t] = __ldg(a.h + c0 * a.H + t);
+    for (int t = threadIdx.x; t < ne * H; t += blockDim.x) hs[t] = __ldg(a.h + c0 * H + t);
     if (threadIdx.x < ne) {
       const int r = threadIdx.x, e = (int)c0 + r;
       int j = __ldg(a.src + e);
@@ -364,11 +366,11 @@ __global__ void __launch_bounds__(kGwrThreads) k_rad_gwr(const __grid_constant__
       for (int b = 0; b < kGwrBatch; ++b) {
         if (b >= nb) break;
         // k pairs: one FFMA2 per two hidden units
-        const float4* hr = reinterpret_cast<const float4*>(hs + (r0 + b) * a.H);
+        const float4* hr = reinterpret_cast<const float4*>(hs + (r0 + b) * H);
         const float2 gb = make_float2(g[b], g[b]);
 #pragma unroll
         for (int k4 = 0; k4 < kRadMaxHidden / 4; ++k4) {
-          if (4 * k4 < a.H) {
+          if (4 * k4 < H) {
             const float4 hv = hr[k4];
             acc[2 * k4] = __ffma2_rn(make_float2(hv.x, hv.y), gb, acc[2 * k4]);
             acc[2 * k4 + 1] = __ffma2_rn(make_float2(hv.z, hv.w), gb, acc[2 * k4 + 1]);
@@ -381,23 +383,23 @@ __global__ void __launch_bounds__(kGwrThreads) k_rad_gwr(const __grid_constant__
   if (act && warp > 0) {
 #pragma unroll
     for (int k = 0; k < kRadMaxHidden / 2; ++k)
-      if (2 * k < a.H) red[((warp - 1) * (kRadMaxHidden / 2) + k) * 32 + lane] = acc[k];
+      if (2 * k < H) red[((warp - 1) * (kRadMaxHidden / 2) + k) * 32 + lane] = acc[k];
   }
   __syncthreads();
   if (!act || warp > 0) return;
   for (int w = 1; w < kGwrWarps; ++w) {
 #pragma unroll
     for (int k = 0; k < kRadMaxHidden / 2; ++k)
-      if (2 * k < a.H) {
+      if (2 * k < H) {
         const float2 v = red[((w - 1) * (kRadMaxHidden / 2) + k) * 32 + lane];
         acc[k].x += v.x;
         acc[k].y += v.y;
       }
   }
-  float* out = a.part + (int64_t)blockIdx.y * a.H * a.nw + P.w_off + c;
+  float* out = a.part + (int64_t)blockIdx.y * H * a.nw + P.w_off + c;
 #pragma unroll
   for (int k = 0; k < kRadMaxHidden / 2; ++k)
-    if (2 * k < a.H) {
+    if (2 * k < H) {
       out[(int64_t)(2 * k) * a.nw] = acc[k].x;
       out[(int64_t)(2 * k + 1) * a.nw] = acc[k].y;
     }
@@ -507,7 +509,8 @@ cudaError_t launch_rad_bwd(const RadArgs& a, const GenTable& T, cudaStream_t s) 
   if (a.gWr) {
     if (a.E == 0) return cudaMemsetAsync(a.gWr, 0, sizeof(float) * (size_t)a.H * a.nw, s);
     const dim3 grid((unsigned)rad_units(T), (unsigned)a.splits);
-    k_rad_gwr<<<grid, kGwrThreads, 0, s>>>(a, T);
+    if (a.H == kRadMaxHidden) k_rad_gwr<kRadMaxHidden><<<grid, kGwrThreads, 0, s>>>(a, T);
+    else k_rad_gwr<0><<<grid, kGwrThreads, 0, s>>>(a, T);
     k_rad_gwr_reduce<<<rad_flat_grid((int64_t)a.H * a.nw), 256, 0, s>>>(a);
     count_launches(2);
     e = cudaGetLastError();
