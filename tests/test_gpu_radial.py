@@ -181,3 +181,40 @@ def test_compiled_lists_at_other_channel_counts(tp, lmax, mul):
     f = lambda *shape: rng.standard_normal(shape).astype(np.float32)
     _check_complete(tp, ir_in, ir_sh, ir_out, paths, rowptr, src, vec, f(40, op.irr_in.dim), f(len(src), 64),
                     (f(64, op.n_weights) / 8).astype(np.float32), f(40, op.irr_out.dim), f"lmax {lmax} mul {mul}")
+
+
+def test_calls_allocate_no_device_memory(tp):
+    """With caller-supplied outputs and workspace, the fused-radial calls allocate nothing: no
+    torch allocation and no change of the device's free memory; the backward workspace holds
+    W_r-sized regions beyond the transpose's, nothing edge x feature sized."""
+    d = synth.make_inputs("c2", 512, with_gy=True)
+    h, Wr = synth.radial_hidden(d)
+    s = d["spec"]
+    plan = tp.Plan(s.irreps_in, s.irreps_sh, s.irreps_out, s.paths)
+    g = {k: dev(v) for k, v in dict(rowptr=d["rowptr"], src=d["src"], vec=d["vec"], x=d["x"], h=h, Wr=Wr,
+                                    gy=d["gy"]).items()}
+    N, E, H = len(d["rowptr"]) - 1, len(d["src"]), h.shape[1]
+    ws = torch.empty(tp.tp_radial_workspace_size(plan, N, E, H, tp.TP_OP_BWD), dtype=torch.uint8, device="cuda")
+    y = torch.empty(N, plan.out_dim, device="cuda")
+    gx = torch.empty(N, plan.in_dim, device="cuda")
+    gh = torch.empty(E, H, device="cuda")
+    gWr = torch.empty(H, plan.n_edge_weights, device="cuda")
+    gvec = torch.empty(E, 3, device="cuda")
+    colptr, perm = tp.tp_csr_transpose(g["rowptr"], g["src"], N)
+    # first calls outside the measurement (kernel attributes, module load)
+    tp.tp_conv_fwd_radial(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["h"], g["Wr"], y=y, ws=ws)
+    tp.tp_conv_bwd_radial(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["h"], g["Wr"], g["gy"], colptr=colptr,
+                          perm=perm, need_gvec=True, gx=gx, gh=gh, gWr=gWr, gvec=gvec, ws=ws)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    before = torch.cuda.memory_allocated()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        tp.tp_conv_fwd_radial(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["h"], g["Wr"], y=y, ws=ws)
+        tp.tp_conv_bwd_radial(plan, g["rowptr"], g["src"], g["x"], g["vec"], g["h"], g["Wr"], g["gy"],
+                              colptr=colptr, perm=perm, need_gvec=True, gx=gx, gh=gh, gWr=gWr, gvec=gvec, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.cuda.max_memory_allocated() == before
+    assert torch.cuda.mem_get_info()[0] == free0
+    base = tp.tp_workspace_size(plan, N, E, tp.TP_OP_BWD)
+    assert ws.numel() - base <= 4 * H * plan.n_edge_weights * 257 + 512
