@@ -369,7 +369,7 @@ def run_reference(args, rank):
 # ------------------------------------------------------------------------------------------
 
 SPEC_OF_WORKLOAD = {"c1": "l1_c1", "c2": "full_l2", "c3": "full_l3", "c4": "full_l2", "c5": "full_l3",
-                    "c2-layer": "full_l2", "c4-layer": "full_l2"}
+                    "c2-layer": "full_l2", "c4-layer": "full_l2", "c2-radial": "full_l2", "c3-radial": "full_l3"}
 
 
 def kernel_source_hash(kernel="", workload="c2"):
@@ -380,6 +380,8 @@ def kernel_source_hash(kernel="", workload="c2"):
         files = [os.path.join(csrc, "csr.cu")]
     else:
         files = [os.path.join(csrc, "tp_kernels.cuh")]
+        if kernel.startswith("k_rad_"):
+            files += [os.path.join(csrc, f) for f in ("radial.cuh", "radial.cu", "radial_spec.cu")]
         if "uvw" in kernel or "gemm" in kernel:
             files += [os.path.join(csrc, "tp_uvw.cuh"), os.path.join(csrc, "tp_mma.cuh")]
         spec = SPEC_OF_WORKLOAD.get(workload)
@@ -1587,7 +1589,7 @@ def run_radial(args, rank, world, local):
                   "bwd": pass_roofline(bwd_ms, bb, fl_b, hbm, fp32_peak)}
         dom = max(passes, key=lambda k: passes[k]["ms"])
         dp = passes[dom]
-        kname = {"fwd": "k_rad_fwd", "bwd": "k_rad_send"}[dom]
+        kname = {"fwd": "k_rad_fwd", "bwd": "k_rad_send + k_rad_gwr"}[dom]
         if dp["bound"] == "hbm":
             roof = {"bound": "hbm", "kernel": kname, "achieved": dp["achieved_GBps"], "peak": hbm, "unit": "GB/s",
                     "frac": dp["achieved_GBps"] / hbm, "peak_note": peak_note}
