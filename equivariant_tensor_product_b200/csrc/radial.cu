@@ -461,8 +461,10 @@ int rad_chunk(const RadArgs& a, bool bwd, size_t* smem_bytes) {
 }
 
 int rad_splits(const GenTable& T, int64_t E) {
+  // one wave: the gW_r pass keeps three CTAs per SM resident (its registers), so
+  // units x splits <= 3 x 148 avoids a partly filled second wave
   const int ctas = rad_units(T);
-  int64_t sp = (4 * 148 + ctas - 1) / ctas;     // about four CTAs per SM
+  int64_t sp = (3 * 148) / ctas;
   sp = std::min<int64_t>(sp, std::max<int64_t>(1, (E + kGwrChunk - 1) / kGwrChunk));
   return (int)std::max<int64_t>(1, std::min<int64_t>(sp, 256));
 }
