@@ -276,15 +276,15 @@ __global__ void __launch_bounds__(kRadThreads) k_rad_send(const __grid_constant_
 // ---------------------------------------------------------------------------------------
 // gW_r partials: part[s][k][w_off(p) + u] = sum over split s's edges of h[e, k] gw[e, p, u],
 // gw recomputed as c_p <x[src e], C_p^T(Y, gy[dst e])>.  A CTA per ((path, 32-channel slice)
-// unit, edge split): its warps take interleaved batches of four edges of each staged chunk (all
+// unit, edge split): its warps take interleaved batches of two edges of each staged chunk (all
 // warps of a CTA run the same triple's code), load the x and gy slices of a batch before using
-// them, and are summed in warp order at the end.
+// them, and are summed in warp order at the end; 128 registers, four CTAs per SM.
 // ---------------------------------------------------------------------------------------
 constexpr int kGwrChunk = 64;
-constexpr int kGwrBatch = 4;
+constexpr int kGwrBatch = 2;
 
 template <int HC>
-__global__ void __launch_bounds__(kGwrThreads) k_rad_gwr(const __grid_constant__ RadArgs a,
+__global__ void __launch_bounds__(kGwrThreads, 4) k_rad_gwr(const __grid_constant__ RadArgs a,
                                                          const __grid_constant__ GenTable T) {
   const int H = HC ? HC : a.H;          // hidden width (a compile-time 64 in the common case)
   __shared__ __align__(16) float hs[kGwrChunk * kRadMaxHidden];
@@ -461,10 +461,10 @@ int rad_chunk(const RadArgs& a, bool bwd, size_t* smem_bytes) {
 }
 
 int rad_splits(const GenTable& T, int64_t E) {
-  // one wave: the gW_r pass keeps three CTAs per SM resident (its registers), so
-  // units x splits <= 3 x 148 avoids a partly filled second wave
+  // one wave: the gW_r pass keeps four CTAs per SM resident (128 registers), so
+  // units x splits <= 4 x 148 avoids a partly filled second wave
   const int ctas = rad_units(T);
-  int64_t sp = (3 * 148) / ctas;
+  int64_t sp = (4 * 148) / ctas;
   sp = std::min<int64_t>(sp, std::max<int64_t>(1, (E + kGwrChunk - 1) / kGwrChunk));
   return (int)std::max<int64_t>(1, std::min<int64_t>(sp, 256));
 }
