@@ -7,9 +7,10 @@
 //   k_rad_fwd_spec   one CTA per receiver: warp = (32-channel slice, edge phase); each warp
 //                    keeps its row sums in registers across chunks; phases are summed through
 //                    shared memory in phase order at the end.
-//   k_rad_send_spec  one CTA per sender: the same warps; gx in registers, gw of the chunk into
-//                    shared memory (then gh as in radial.cu), gvec per edge from the generated
-//                    SH-gradient sums, reduced over lanes and then over slices in slice order.
+//   k_rad_send_spec  one CTA per sender: the same warps; gx in registers, the receivers' gy
+//                    rows read from L2, the chunk's gw written over its w in shared memory (then
+//                    gh as in radial.cu), gvec per edge from the generated SH-gradient sums,
+//                    reduced over lanes and then over slices in slice order.
 #include "radial.cuh"
 #include "spec_full_l2.h"
 #include "spec_full_l3.h"
@@ -104,11 +105,33 @@ __global__ void __launch_bounds__(kRadThreads, 2) k_rad_fwd_spec(const __grid_co
   }
 }
 
+// Shared memory of the compiled-list sender pass: hs [H][CE + 4] | ws [CE][nwp] (the chunk's w,
+// overwritten in place by its gw) | gvec partials [CE][8][4] | Ys [CE][16] | es, ns [CE].  The
+// receivers' gy rows are read from L2 by the coupling, so one weight tile of 32 edges fits
+// two CTAs per SM.
+__host__ __device__ inline size_t send_smem_floats(int H, int CE, int nwp) {
+  return (size_t)H * (CE + 4) + (size_t)CE * nwp + 32 * (size_t)CE + 16 * (size_t)CE + 2 * round4(CE);
+}
+
+template <int CE>
+__device__ __forceinline__ RadSmem send_smem(float* base, const RadArgs& a) {
+  RadSmem s;
+  s.hs = base;
+  s.ws = s.hs + a.H * (CE + 4);
+  s.gs = s.ws;
+  s.vs = s.xn = nullptr;
+  s.rs = s.ws + CE * a.nwp;
+  s.Ys = s.rs + 32 * CE;
+  s.es = reinterpret_cast<int*>(s.Ys + CE * 16);
+  s.ns = s.es + round4(CE);
+  return s;
+}
+
 template <class S, int CE, bool GVEC>
 __global__ void __launch_bounds__(kRadThreads, 2) k_rad_send_spec(const __grid_constant__ RadArgs a,
                                                                   const __grid_constant__ GenTable T) {
   extern __shared__ float4 rad_smem_raw[];
-  const RadSmem s = rad_smem<CE>(reinterpret_cast<float*>(rad_smem_raw), a, true);
+  const RadSmem s = send_smem<CE>(reinterpret_cast<float*>(rad_smem_raw), a);
   const int node = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nsl = (a.mul + 31) >> 5, phases = kRadWarps / nsl;
   const int sl = warp % nsl, ph = warp / nsl;
@@ -125,7 +148,6 @@ __global__ void __launch_bounds__(kRadThreads, 2) k_rad_send_spec(const __grid_c
   for (int k = 0; k < S::IN_PC; ++k) gx[k] = xr[k] = 0.f;
   if (act) S::load_in(a.x + (int64_t)node * a.in_dim, a.mul, c, xr);
   float* gvp = s.rs;                       // gvec partials [CE][nsl][4] (gx lives in registers)
-  const int gp = round4(a.out_dim);
   for (int c0 = q0; c0 < q1; c0 += CE) {
     const int ne = min(CE, q1 - c0);
     __syncthreads();
@@ -154,7 +176,7 @@ __global__ void __launch_bounds__(kRadThreads, 2) k_rad_send_spec(const __grid_c
       for (int m = 0; m < S::NSH; ++m) s.Ys[r * 16 + m] = Y[m];
     }
     __syncthreads();
-    stage_chunk<CE>(a, s, ne, a.gy, a.out_dim);
+    stage_chunk<CE>(a, s, ne, a.gy, 0);    // the hidden rows only; gy rows are read from L2
     __syncthreads();
     project<CE>(a, s);
     __syncthreads();
@@ -170,11 +192,12 @@ __global__ void __launch_bounds__(kRadThreads, 2) k_rad_send_spec(const __grid_c
         }
         if (act) {
           float gya[S::OUT_PC], wa[S::P], gw[S::P];
-          S::load_out_shared(s.vs + r * gp, a.mul, c, gya);
+          S::load_out(a.gy + (int64_t)s.ns[r] * a.out_dim, a.mul, c, gya);
           const float* wr = s.ws + r * a.nwp + c;
 #pragma unroll
           for (int p = 0; p < S::P; ++p) wa[p] = T.path[p].coeff * wr[p * a.mul];
           S::template bwd<GVEC>(xr, Y, wa, gya, gx, gw, gY);
+          // gw overwrites w in place: this lane's entries of edge r are read above and by nobody else
           float* gr = s.gs + r * a.nwp + c;
 #pragma unroll
           for (int p = 0; p < S::P; ++p) gr[p * a.mul] = T.path[p].coeff * gw[p];
@@ -290,19 +313,34 @@ cudaError_t launch_rad_fwd_spec(const RadArgs& a, const GenTable& T, int ce, siz
 
 cudaError_t launch_rad_send_spec(const RadArgs& a, const GenTable& T, int ce, size_t smem, cudaStream_t s,
                                  bool* handled) {
-  *handled = true;
-  if (a.spec == 2 && spec_fits<Spec_full_l2>(a, ce, true)) {
-    if (ce == 16) return a.gvec ? spec_launch(k_rad_send_spec<Spec_full_l2, 16, true>, smem, s, a, T)
-                                : spec_launch(k_rad_send_spec<Spec_full_l2, 16, false>, smem, s, a, T);
-    if (ce == 8) return a.gvec ? spec_launch(k_rad_send_spec<Spec_full_l2, 8, true>, smem, s, a, T)
-                               : spec_launch(k_rad_send_spec<Spec_full_l2, 8, false>, smem, s, a, T);
-  }
-  if (a.spec == 3 && spec_fits<Spec_full_l3>(a, ce, true)) {
-    if (ce == 4) return a.gvec ? spec_launch(k_rad_send_spec<Spec_full_l3, 4, true>, smem, s, a, T)
-                               : spec_launch(k_rad_send_spec<Spec_full_l3, 4, false>, smem, s, a, T);
-  }
+  (void)ce;
+  (void)smem;
   *handled = false;
-  return cudaSuccess;
+  if (a.spec != 2 && a.spec != 3) return cudaSuccess;
+  // this pass's own chunk: the largest instantiated size whose weight tile fits the tile budget
+  const int sizes[2][2] = {{32, 16}, {8, 4}};
+  int c2 = 0;
+  for (int q = 0; q < 2 && !c2; ++q) {
+    const int v = sizes[a.spec - 2][q];
+    if ((size_t)v * a.nwp * 4 <= (size_t)kRadTileBudget || q == 1) c2 = v;
+  }
+  const size_t sm = sizeof(float) * send_smem_floats(a.H, c2, a.nwp);
+  const int nsl = (a.mul + 31) / 32;
+  if (sm > (size_t)kRadSmemBudget || nsl < 1 || nsl > kRadWarps) return cudaSuccess;
+  const int phases = kRadWarps / nsl;
+  const size_t red = (size_t)(phases - 1) * nsl * (a.spec == 2 ? Spec_full_l2::IN_PC : Spec_full_l3::IN_PC) * 32;
+  if (red > (size_t)c2 * a.nwp) return cudaSuccess;
+  *handled = true;
+  if (a.spec == 2) {
+    if (c2 == 32) return a.gvec ? spec_launch(k_rad_send_spec<Spec_full_l2, 32, true>, sm, s, a, T)
+                                : spec_launch(k_rad_send_spec<Spec_full_l2, 32, false>, sm, s, a, T);
+    return a.gvec ? spec_launch(k_rad_send_spec<Spec_full_l2, 16, true>, sm, s, a, T)
+                  : spec_launch(k_rad_send_spec<Spec_full_l2, 16, false>, sm, s, a, T);
+  }
+  if (c2 == 8) return a.gvec ? spec_launch(k_rad_send_spec<Spec_full_l3, 8, true>, sm, s, a, T)
+                             : spec_launch(k_rad_send_spec<Spec_full_l3, 8, false>, sm, s, a, T);
+  return a.gvec ? spec_launch(k_rad_send_spec<Spec_full_l3, 4, true>, sm, s, a, T)
+                : spec_launch(k_rad_send_spec<Spec_full_l3, 4, false>, sm, s, a, T);
 }
 
 }  // namespace tp
