@@ -4,9 +4,9 @@
 // kernels -- every path of an edge in one generated chain over the non-zero Clebsch-Gordan
 // entries, the x (x) Y products shared by the paths of each (l1, l2) pair ("FlashTP", abstract:
 // path-aggregated execution) -- instead of the path table's chain per path.
-//   k_rad_fwd_spec   one CTA per receiver: warp = (32-channel slice, edge phase); each warp
-//                    keeps its row sums in registers across chunks; phases are summed through
-//                    shared memory in phase order at the end.
+//   k_rad_fwd_spec   one CTA per receiver: warp = (32-channel slice, edge phase); the senders'
+//                    x rows read from L2; each warp keeps its row sums in registers across
+//                    chunks; phases are summed through shared memory in phase order at the end.
 //   k_rad_send_spec  one CTA per sender: the same warps; gx in registers, the receivers' gy
 //                    rows read from L2, the chunk's gw written over its w in shared memory (then
 //                    gh as in radial.cu), gvec per edge from the generated SH-gradient sums,
@@ -20,11 +20,29 @@ namespace {
 
 using namespace rad;
 
+// Shared memory of the compiled-list forward: hs [H][CE + 4] | ws [CE][nwp] | Ys [CE][16] |
+// es, ns [CE]; the senders' x rows are read from L2 by the coupling.
+__host__ __device__ inline size_t fwd_smem_floats(int H, int CE, int nwp) {
+  return (size_t)H * (CE + 4) + (size_t)CE * nwp + 16 * (size_t)CE + 2 * round4(CE);
+}
+
+template <int CE>
+__device__ __forceinline__ RadSmem fwd_smem(float* base, const RadArgs& a) {
+  RadSmem s;
+  s.hs = base;
+  s.ws = s.hs + a.H * (CE + 4);
+  s.gs = s.vs = s.xn = s.rs = nullptr;
+  s.Ys = s.ws + CE * a.nwp;
+  s.es = reinterpret_cast<int*>(s.Ys + CE * 16);
+  s.ns = s.es + round4(CE);
+  return s;
+}
+
 template <class S, int CE>
 __global__ void __launch_bounds__(kRadThreads, 2) k_rad_fwd_spec(const __grid_constant__ RadArgs a,
                                                                  const __grid_constant__ GenTable T) {
   extern __shared__ float4 rad_smem_raw[];
-  const RadSmem s = rad_smem<CE>(reinterpret_cast<float*>(rad_smem_raw), a, false);
+  const RadSmem s = fwd_smem<CE>(reinterpret_cast<float*>(rad_smem_raw), a);
   const int row = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nsl = (a.mul + 31) >> 5, phases = kRadWarps / nsl;
   const int sl = warp % nsl, ph = warp / nsl;
@@ -39,7 +57,6 @@ __global__ void __launch_bounds__(kRadThreads, 2) k_rad_fwd_spec(const __grid_co
   float acc[S::OUT_PC];
 #pragma unroll
   for (int k = 0; k < S::OUT_PC; ++k) acc[k] = 0.f;
-  const int xp = round4(a.in_dim);
   for (int c0 = e0; c0 < e1; c0 += CE) {
     const int ne = min(CE, e1 - c0);
     __syncthreads();
@@ -68,7 +85,7 @@ __global__ void __launch_bounds__(kRadThreads, 2) k_rad_fwd_spec(const __grid_co
       for (int m = 0; m < S::NSH; ++m) s.Ys[r * 16 + m] = Y[m];
     }
     __syncthreads();
-    stage_chunk<CE>(a, s, ne, a.x, a.in_dim);
+    stage_chunk<CE>(a, s, ne, a.x, 0);     // the hidden rows only; x rows are read from L2
     __syncthreads();
     project<CE>(a, s);
     __syncthreads();
@@ -76,7 +93,7 @@ __global__ void __launch_bounds__(kRadThreads, 2) k_rad_fwd_spec(const __grid_co
       for (int r = ph; r < ne; r += phases) {
         if (s.es[r] < 0) continue;
         float xa[S::IN_PC], wa[S::P], Y[S::NSH];
-        S::load_in_shared(s.vs + r * xp, a.mul, c, xa);
+        S::load_in(a.x + (int64_t)s.ns[r] * a.in_dim, a.mul, c, xa);
         const float* wr = s.ws + r * a.nwp + c;
 #pragma unroll
         for (int p = 0; p < S::P; ++p) wa[p] = T.path[p].coeff * wr[p * a.mul];
@@ -281,34 +298,35 @@ cudaError_t spec_launch(K kern, size_t smem, cudaStream_t s, const RadArgs& a, c
   return cudaGetLastError();
 }
 
-// The phase reductions reuse the weight tile and the gvec partials the output-row region:
-// true when both fit (and the slices fit the warps).
-template <class S>
-bool spec_fits(const RadArgs& a, int ce, bool bwd) {
-  const int nsl = (a.mul + 31) / 32;
-  if (nsl < 1 || nsl > kRadWarps) return false;
-  const int phases = kRadWarps / nsl;
-  const size_t red = (size_t)(phases - 1) * nsl * (bwd ? S::IN_PC : S::OUT_PC) * 32;
-  if (red > (size_t)ce * a.nwp) return false;
-  if (bwd && (size_t)ce * nsl * 4 > (size_t)round4(a.in_dim)) return false;
-  return true;
-}
-
 }  // namespace
 
 cudaError_t launch_rad_fwd_spec(const RadArgs& a, const GenTable& T, int ce, size_t smem, cudaStream_t s,
                                 bool* handled) {
-  *handled = true;
-  if (a.spec == 2 && spec_fits<Spec_full_l2>(a, ce, false)) {
-    if (ce == 32) return spec_launch(k_rad_fwd_spec<Spec_full_l2, 32>, smem, s, a, T);
-    if (ce == 16) return spec_launch(k_rad_fwd_spec<Spec_full_l2, 16>, smem, s, a, T);
-  }
-  if (a.spec == 3 && spec_fits<Spec_full_l3>(a, ce, false)) {
-    if (ce == 8) return spec_launch(k_rad_fwd_spec<Spec_full_l3, 8>, smem, s, a, T);
-    if (ce == 4) return spec_launch(k_rad_fwd_spec<Spec_full_l3, 4>, smem, s, a, T);
-  }
+  (void)ce;
+  (void)smem;
   *handled = false;
-  return cudaSuccess;
+  if (a.spec != 2 && a.spec != 3) return cudaSuccess;
+  // this pass's own chunk: the largest instantiated size whose weight tile fits the tile budget
+  const int sizes[2][3] = {{32, 16, 16}, {16, 8, 4}};
+  int c2 = 0;
+  for (int q = 0; q < 3 && !c2; ++q) {
+    const int v = sizes[a.spec - 2][q];
+    if ((size_t)v * a.nwp * 4 <= (size_t)kRadTileBudget || q == 2) c2 = v;
+  }
+  const size_t sm = sizeof(float) * fwd_smem_floats(a.H, c2, a.nwp);
+  const int nsl = (a.mul + 31) / 32;
+  if (sm > (size_t)kRadSmemBudget || nsl < 1 || nsl > kRadWarps) return cudaSuccess;
+  const int phases = kRadWarps / nsl;
+  const size_t red = (size_t)(phases - 1) * nsl * (a.spec == 2 ? Spec_full_l2::OUT_PC : Spec_full_l3::OUT_PC) * 32;
+  if (red > (size_t)c2 * a.nwp) return cudaSuccess;
+  *handled = true;
+  if (a.spec == 2) {
+    if (c2 == 32) return spec_launch(k_rad_fwd_spec<Spec_full_l2, 32>, sm, s, a, T);
+    return spec_launch(k_rad_fwd_spec<Spec_full_l2, 16>, sm, s, a, T);
+  }
+  if (c2 == 16) return spec_launch(k_rad_fwd_spec<Spec_full_l3, 16>, sm, s, a, T);
+  if (c2 == 8) return spec_launch(k_rad_fwd_spec<Spec_full_l3, 8>, sm, s, a, T);
+  return spec_launch(k_rad_fwd_spec<Spec_full_l3, 4>, sm, s, a, T);
 }
 
 cudaError_t launch_rad_send_spec(const RadArgs& a, const GenTable& T, int ce, size_t smem, cudaStream_t s,
