@@ -156,7 +156,17 @@ __device__ __forceinline__ void project(const RadArgs& a, const RadSmem& s) {
 // over every fourth edge of the chunk, W_r read transposed (WrT) so that a warp's loads of one
 // column are contiguous.  Call after the chunk's gs is complete (a barrier after its writes).
 template <int CE>
+__device__ __forceinline__ void gh_chunk_pairs(const RadArgs& a, const RadSmem& s, int ne);
+
+template <int CE>
 __device__ __forceinline__ void gh_chunk(const RadArgs& a, const RadSmem& s, int ne) {
+  if constexpr (CE == 4 * kRadWarps) {
+    // the pair form uses 8-byte accesses to W_r^T and gh (the ABI promises 4-byte alignment)
+    if (((reinterpret_cast<uintptr_t>(a.WrT) | reinterpret_cast<uintptr_t>(a.gh)) & 7u) == 0) {
+      gh_chunk_pairs<CE>(a, s, ne);
+      return;
+    }
+  }
   constexpr int NQ = kRadThreads / 64, RQ = CE / NQ > 0 ? CE / NQ : 1;
   const int k = threadIdx.x & 63, quarter = threadIdx.x >> 6;
   if (k < a.H && quarter < CE) {
@@ -183,6 +193,48 @@ __device__ __forceinline__ void gh_chunk(const RadArgs& a, const RadSmem& s, int
       const int r = quarter + NQ * q;
       if (r < ne && s.es[r] >= 0) a.gh[(int64_t)s.es[r] * a.H + k] = acc[q];
     }
+  }
+}
+
+// gh for chunks of 4 edges per warp: lane = pair of hidden units (k, k + 1), warp = four edges
+// of the chunk.  A lane's W_r^T loads of one column are one 8-byte load (contiguous across the
+// warp), each gw value is a broadcast shared-memory read, and one FFMA2 updates both hidden
+// units of an edge.
+template <int CE>
+__device__ __forceinline__ void gh_chunk_pairs(const RadArgs& a, const RadSmem& s, int ne) {
+  const int kp = threadIdx.x & 31, r0 = 4 * (threadIdx.x >> 5);
+  if (2 * kp >= a.H) return;
+  float2 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+  const int nw4 = a.nw & ~3;
+  const float2* wt = reinterpret_cast<const float2*>(a.WrT) + kp;   // WrT[c][2 kp .. 2 kp + 1]
+  const int hp = a.H >> 1;
+  for (int c = 0; c < nw4; c += 4) {
+    float2 w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) w[u] = __ldg(wt + (int64_t)(c + u) * hp);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 g = *reinterpret_cast<const float4*>(s.gs + (r0 + q) * a.nwp + c);
+      acc[q] = __ffma2_rn(make_float2(g.x, g.x), w[0], acc[q]);
+      acc[q] = __ffma2_rn(make_float2(g.y, g.y), w[1], acc[q]);
+      acc[q] = __ffma2_rn(make_float2(g.z, g.z), w[2], acc[q]);
+      acc[q] = __ffma2_rn(make_float2(g.w, g.w), w[3], acc[q]);
+    }
+  }
+  for (int c = nw4; c < a.nw; ++c) {
+    const float2 wv = __ldg(wt + (int64_t)c * hp);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float g = s.gs[(r0 + q) * a.nwp + c];
+      acc[q] = __ffma2_rn(make_float2(g, g), wv, acc[q]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int r = r0 + q;
+    if (r < ne && s.es[r] >= 0) *reinterpret_cast<float2*>(a.gh + (int64_t)s.es[r] * a.H + 2 * kp) = acc[q];
   }
 }
 
