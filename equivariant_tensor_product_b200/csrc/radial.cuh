@@ -238,6 +238,61 @@ __device__ __forceinline__ void gh_chunk_pairs(const RadArgs& a, const RadSmem& 
   }
 }
 
+// gh for chunks of fewer than 32 edges, pair form: warp = (group of four edges, part of the
+// columns), lane = pair of hidden units; the column parts' sums go through `red` (32 H floats)
+// and are added in part order.  Every thread of the CTA must call it (it has barriers).
+template <int CE>
+__device__ __forceinline__ void gh_chunk_split(const RadArgs& a, const RadSmem& s, int ne, float* red) {
+  constexpr int G = CE / 4, NP = kRadWarps / G;
+  const int kp = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = warp % G, part = warp / G, r0 = 4 * g;
+  const int hp = a.H >> 1, nw4 = a.nw & ~3;
+  const int c_lo = ((nw4 >> 2) * part / NP) << 2, c_hi = ((nw4 >> 2) * (part + 1) / NP) << 2;
+  if (kp < hp) {
+    float2 acc[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+    const float2* wt = reinterpret_cast<const float2*>(a.WrT) + kp;
+    for (int c = c_lo; c < c_hi; c += 4) {
+      float2 w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) w[u] = __ldg(wt + (int64_t)(c + u) * hp);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(s.gs + (r0 + q) * a.nwp + c);
+        acc[q] = __ffma2_rn(make_float2(v.x, v.x), w[0], acc[q]);
+        acc[q] = __ffma2_rn(make_float2(v.y, v.y), w[1], acc[q]);
+        acc[q] = __ffma2_rn(make_float2(v.z, v.z), w[2], acc[q]);
+        acc[q] = __ffma2_rn(make_float2(v.w, v.w), w[3], acc[q]);
+      }
+    }
+    if (part == NP - 1) {
+      for (int c = nw4; c < a.nw; ++c) {
+        const float2 wv = __ldg(wt + (int64_t)c * hp);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float v = s.gs[(r0 + q) * a.nwp + c];
+          acc[q] = __ffma2_rn(make_float2(v, v), wv, acc[q]);
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      reinterpret_cast<float2*>(red)[(part * CE + r0 + q) * hp + kp] = acc[q];
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < CE * hp; t += blockDim.x) {
+    const int r = t / hp, k2 = t - r * hp;
+    float2 v = reinterpret_cast<const float2*>(red)[r * hp + k2];
+    for (int q = 1; q < NP; ++q) {
+      const float2 u = reinterpret_cast<const float2*>(red)[(q * CE + r) * hp + k2];
+      v.x += u.x;
+      v.y += u.y;
+    }
+    if (r < ne && s.es[r] >= 0) *reinterpret_cast<float2*>(a.gh + (int64_t)s.es[r] * a.H + 2 * k2) = v;
+  }
+}
+
 __device__ __forceinline__ void sh16(const float* __restrict__ vec, int e, float (&Y)[16], float& rx, float& ry,
                                      float& rz, float& ir) {
   edge_geometry(__ldg(vec + 3 * (int64_t)e), __ldg(vec + 3 * (int64_t)e + 1), __ldg(vec + 3 * (int64_t)e + 2), rx,

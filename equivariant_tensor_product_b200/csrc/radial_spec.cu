@@ -127,7 +127,8 @@ __global__ void __launch_bounds__(kRadThreads, 2) k_rad_fwd_spec(const __grid_co
 // receivers' gy rows are read from L2 by the coupling, so one weight tile of 32 edges fits
 // two CTAs per SM.
 __host__ __device__ inline size_t send_smem_floats(int H, int CE, int nwp) {
-  return (size_t)H * (CE + 4) + (size_t)CE * nwp + 32 * (size_t)CE + 16 * (size_t)CE + 2 * round4(CE);
+  return (size_t)H * (CE + 4) + (size_t)CE * nwp + 32 * (size_t)CE + 16 * (size_t)CE + 2 * round4(CE) +
+         32 * (size_t)H;
 }
 
 template <int CE>
@@ -141,6 +142,7 @@ __device__ __forceinline__ RadSmem send_smem(float* base, const RadArgs& a) {
   s.Ys = s.rs + 32 * CE;
   s.es = reinterpret_cast<int*>(s.Ys + CE * 16);
   s.ns = s.es + round4(CE);
+  s.xn = reinterpret_cast<float*>(s.ns + round4(CE));   // gh column-part sums [32 H]
   return s;
 }
 
@@ -268,7 +270,12 @@ __global__ void __launch_bounds__(kRadThreads, 2) k_rad_send_spec(const __grid_c
         g[2] = ir * (h2 - rz * sdeg);
       }
     }
-    if (a.gh) gh_chunk<CE>(a, s, ne);
+    if (a.gh) {
+      if (CE < 4 * kRadWarps && ((reinterpret_cast<uintptr_t>(a.WrT) | reinterpret_cast<uintptr_t>(a.gh)) & 7u) == 0)
+        gh_chunk_split<CE>(a, s, ne, s.xn);
+      else
+        gh_chunk<CE>(a, s, ne);
+    }
   }
   // phase sums of gx through the weight tile, added in phase order
   __syncthreads();
